@@ -1,0 +1,276 @@
+"""CPU oracle for the DeltaQuant W4A4 linear layer.
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the bench's CPU
+baseline may import this package; the library under video_diffusion_w4a4_b200
+never does, and this package never imports it.
+
+The arithmetic lives in dq_oracle.c (plain C, OpenMP over independent rows
+and cubes).  This module compiles it, marshals numpy arrays, and adds the one
+step that uses a library primitive: the truncated SVD of W from which the
+low-rank factors L1, L2 are taken (DeltaQuant page, key design 4, Eq. 3,
+following SVDQuant).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so in place.  -ffp-contract=off keeps every fp32
+    operation a single IEEE rounding, as the oracle's readings require."""
+    src = os.path.join(_HERE, "dq_oracle.c")
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(src):
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
+                               "-fno-fast-math", "-o", _SO, src, "-lm"])
+    return _SO
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_SO)
+        P, I, F, LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
+        lib.or_bf16_value.argtypes = [ctypes.c_uint16]
+        lib.or_bf16_value.restype = F
+        lib.or_bf16_round.argtypes = [ctypes.c_double]
+        lib.or_bf16_round.restype = ctypes.c_uint16
+        lib.or_e2m1_value.argtypes = [I]
+        lib.or_e2m1_value.restype = ctypes.c_double
+        lib.or_e4m3_value.argtypes = [I]
+        lib.or_e4m3_value.restype = ctypes.c_double
+        lib.or_e2m1_encode.argtypes = [F]
+        lib.or_e4m3_encode.argtypes = [F]
+        lib.or_e2m1_encode_array.argtypes = [P, LL, P]
+        lib.or_e4m3_encode_array.argtypes = [P, LL, P]
+        lib.or_num_cubes.argtypes = [I] * 6
+        lib.or_num_cubes.restype = LL
+        lib.or_cube_order.argtypes = [I] * 6 + [P] * 5
+        lib.or_cube_means.argtypes = [P] + [I] * 7 + [P]
+        lib.or_cube_split_f64.argtypes = [P] + [I] * 7 + [P, P]
+        lib.or_tensor_scale.argtypes = [F]
+        lib.or_tensor_scale.restype = F
+        lib.or_fp4_quantize.argtypes = [P, LL, I, F, P, P, P]
+        lib.or_quantize_activations.argtypes = [P] + [I] * 7 + [P] * 7
+        lib.or_residual.argtypes = [P, P, P, I, I, I, P]
+        lib.or_output_rows.argtypes = [P, P, F, P, P, P, P, P, P, F, I, I, P, P, P, I, P, LL, P]
+        _lib = lib
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data
+
+
+# --------------------------------------------------------------------------- formats
+
+def e2m1_value(codes) -> np.ndarray:
+    tab = np.array([_L().or_e2m1_value(c) for c in range(16)])
+    return tab[np.asarray(codes, dtype=np.int64) & 15]
+
+
+def e4m3_value(codes) -> np.ndarray:
+    tab = np.array([_L().or_e4m3_value(c) for c in range(256)])
+    return tab[np.asarray(codes, dtype=np.int64) & 255]
+
+
+def e2m1_encode(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    _L().or_e2m1_encode_array(_p(v), v.size, _p(out))
+    return out
+
+
+def e4m3_encode(v) -> np.ndarray:
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    _L().or_e4m3_encode_array(_p(v), v.size, _p(out))
+    return out
+
+
+def bf16_value(b) -> np.ndarray:
+    """BF16 bits -> float32 values, through the oracle's own decoder."""
+    b = np.asarray(b, dtype=np.uint16)
+    tab = np.array([_L().or_bf16_value(i) for i in range(65536)], dtype=np.float32)
+    return tab[b]
+
+
+def bf16_round(v) -> np.ndarray:
+    v = np.asarray(v, dtype=np.float64)
+    f = np.vectorize(lambda x: _L().or_bf16_round(float(x)), otypes=[np.uint16])
+    return f(v) if v.size else v.astype(np.uint16)
+
+
+def tensor_scale(amax: float) -> float:
+    return float(_L().or_tensor_scale(amax))
+
+
+# --------------------------------------------------------------------------- cubes
+
+def num_cubes(T, H, W, t, h, w) -> int:
+    return int(_L().or_num_cubes(T, H, W, t, h, w))
+
+
+def cube_order(T, H, W, t, h, w) -> dict:
+    N = T * H * W
+    K = num_cubes(T, H, W, t, h, w)
+    out = {k: np.empty(s, dtype=np.int32) for k, s in
+           (("row_of_n", N), ("cube_of_n", N), ("n_of_row", N), ("count", K), ("first", K))}
+    _L().or_cube_order(T, H, W, t, h, w, _p(out["row_of_n"]), _p(out["cube_of_n"]), _p(out["n_of_row"]),
+                       _p(out["count"]), _p(out["first"]))
+    return out
+
+
+def cube_means(X, T, H, W, cube) -> np.ndarray:
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    Ci = X.shape[1]
+    K = num_cubes(T, H, W, *cube)
+    m = np.empty((K, Ci), dtype=np.float32)
+    if _L().or_cube_means(_p(X), T, H, W, Ci, *cube, _p(m)):
+        raise RuntimeError("or_cube_means failed")
+    return m
+
+
+def cube_split_f64(X, T, H, W, cube):
+    """Eq. 1 in fp64 without quantisation: (mean K x Ci, delta N x Ci natural order)."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    Ci = X.shape[1]
+    K = num_cubes(T, H, W, *cube)
+    mean = np.empty((K, Ci), dtype=np.float64)
+    delta = np.empty((X.shape[0], Ci), dtype=np.float64)
+    if _L().or_cube_split_f64(_p(X), T, H, W, Ci, *cube, _p(mean), _p(delta)):
+        raise RuntimeError("or_cube_split_f64 failed")
+    return mean, delta
+
+
+# --------------------------------------------------------------------------- quantisers
+
+def fp4_quantize(Z, S: float | None = None):
+    """FP4 rows with E4M3 group-16 scales; returns (codes, scales, S)."""
+    Z = np.ascontiguousarray(Z, dtype=np.float32)
+    rows, cols = Z.shape
+    codes = np.empty((rows, cols // 2), dtype=np.uint8)
+    scales = np.empty((rows, cols // 16), dtype=np.uint8)
+    S_out = ctypes.c_float(0)
+    if _L().or_fp4_quantize(_p(Z), rows, cols, -1.0 if S is None else float(S), _p(codes), _p(scales),
+                            ctypes.byref(S_out)):
+        raise RuntimeError("or_fp4_quantize failed")
+    return codes, scales, float(S_out.value)
+
+
+def quantize_activations(X, T, H, W, cube) -> dict:
+    """Activation side of Eq. 2/3 over the whole X (natural (t,h,w) row order)."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    N, Ci = X.shape
+    assert N == T * H * W
+    K = num_cubes(T, H, W, *cube)
+    out = dict(dcodes=np.empty((N, Ci // 2), np.uint8), dscales=np.empty((N, Ci // 16), np.uint8),
+               q8=np.empty((K, Ci), np.uint8), s8=np.empty(K, np.float32),
+               means=np.empty((K, Ci), np.float32))
+    S = ctypes.c_float(0)
+    amax = ctypes.c_float(0)
+    rc = _L().or_quantize_activations(_p(X), T, H, W, Ci, *cube, _p(out["dcodes"]), _p(out["dscales"]),
+                                      ctypes.byref(S), _p(out["q8"]), _p(out["s8"]), _p(out["means"]),
+                                      ctypes.byref(amax))
+    if rc:
+        raise RuntimeError("or_quantize_activations failed")
+    out["S_delta"] = float(S.value)
+    out["amax_delta"] = float(amax.value)
+    out.update(cube_order(T, H, W, *cube))
+    return out
+
+
+def quantize_plain(X) -> dict:
+    """Plain per-token FP4 of X itself (no kernel/delta split), natural row order."""
+    xf = bf16_value(X)
+    codes, scales, S = fp4_quantize(xf)
+    return dict(dcodes=codes, dscales=scales, S_delta=S)
+
+
+# --------------------------------------------------------------------------- weight side
+
+def lowrank_factors(Wbits, r: int, seed: int = 0):
+    """Truncated SVD W^T ~ V_r S_r U_r^T split evenly: L1 = V_r S_r^1/2 (Ci x r),
+    L2 = S_r^1/2 U_r^T (r x Co), each rounded to BF16.  Also returns all
+    computed singular values (descending)."""
+    Wf = bf16_value(Wbits).astype(np.float64)
+    Co, Ci = Wf.shape
+    if min(Co, Ci) <= 2048:
+        U, s, Vt = np.linalg.svd(Wf, full_matrices=False)
+        Ur, sr, Vr = U[:, :r], s[:r], Vt[:r].T
+        sig = s
+    else:
+        from scipy.sparse.linalg import svds
+        v0 = np.random.default_rng(seed).standard_normal(min(Co, Ci))
+        U, s, Vt = svds(Wf, k=r, tol=0, v0=v0, which="LM")
+        order = np.argsort(s)[::-1]
+        Ur, sr, Vr = U[:, order], s[order], Vt[order].T
+        sig = sr
+    L1 = Vr * np.sqrt(sr)[None, :]
+    L2 = (Ur * np.sqrt(sr)[None, :]).T
+    return bf16_round_fast(L1), bf16_round_fast(L2), sig
+
+
+def bf16_round_fast(v) -> np.ndarray:
+    """Vectorised BF16 rounding, checked against the oracle's search-based
+    bf16_round in the tests."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    f = v.astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    lo = (u >> 16).astype(np.uint16)
+    cand = np.stack([lo - 1, lo, lo + 1]).astype(np.uint16)
+    vals = (cand.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    dist = np.abs(vals - v[None])
+    dist[np.isnan(dist)] = np.inf
+    best = dist.min(axis=0)
+    tie_even = (dist == best[None]) & ((cand & 1) == 0)
+    pick = np.where(tie_even.any(axis=0), np.argmax(tie_even, axis=0), np.argmin(dist, axis=0))
+    return np.take_along_axis(cand, pick[None], axis=0)[0]
+
+
+def residual(Wbits, L1, L2) -> np.ndarray:
+    Wbits = np.ascontiguousarray(Wbits, dtype=np.uint16)
+    L1 = np.ascontiguousarray(L1, dtype=np.uint16)
+    L2 = np.ascontiguousarray(L2, dtype=np.uint16)
+    Co, Ci = Wbits.shape
+    r = L1.shape[1]
+    R = np.empty((Co, Ci), dtype=np.float32)
+    _L().or_residual(_p(Wbits), _p(L1), _p(L2), Co, Ci, r, _p(R))
+    return R
+
+
+def quantize_weight(Wbits, L1, L2) -> dict:
+    R = residual(Wbits, L1, L2)
+    codes, scales, S = fp4_quantize(R)
+    return dict(R=R, wcodes=codes, wscales=scales, S_w=S)
+
+
+# --------------------------------------------------------------------------- output
+
+def output_rows(act: dict, wq: dict, X, L1, L2, rows, kernel: bool = True, lowrank: bool = True,
+                cube_major: bool = True) -> np.ndarray:
+    """fp64 Y rows (Eq. 3) for natural token indices `rows`."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    Co, Ci = wq["wcodes"].shape[0], wq["wcodes"].shape[1] * 2
+    r = L1.shape[1] if (lowrank and L1 is not None) else 0
+    Y = np.empty((rows.size, Co), dtype=np.float64)
+    arow = np.ascontiguousarray(act["row_of_n"], np.int32) if cube_major else None
+    cube = np.ascontiguousarray(act["cube_of_n"], np.int32) if kernel else None
+    rc = _L().or_output_rows(_p(act["dcodes"]), _p(act["dscales"]), act["S_delta"], _p(arow),
+                             _p(act["q8"]) if kernel else None, _p(act["s8"]) if kernel else None, _p(cube),
+                             _p(wq["wcodes"]), _p(wq["wscales"]), wq["S_w"], Co, Ci, _p(X),
+                             _p(np.ascontiguousarray(L1, np.uint16)) if r else None,
+                             _p(np.ascontiguousarray(L2, np.uint16)) if r else None, r,
+                             _p(rows), rows.size, _p(Y))
+    if rc:
+        raise RuntimeError("or_output_rows failed")
+    return Y

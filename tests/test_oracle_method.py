@@ -1,0 +1,339 @@
+"""Pins for the oracle's statement of the DeltaQuant layer.
+
+Source: papernotes.org, "DeltaQuant: 4-bit Video Diffusion Models with
+Spatiotemporal Delta Smoothing", key designs 2-4 (cube partition, Eq. 1
+kernel/delta split, Eq. 2-3 split product with the SVD low-rank branch,
+Eq. 4 quantiser).  Every check here compares the oracle with an independent
+statement: closed forms, exact fp64 invariants, brute-force assembly with a
+library matmul, hand-derived worked examples, or the Eckart-Young bound.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+
+def _x_f64(X):
+    return oracle.bf16_value(X).astype(np.float64)
+
+
+# ------------------------------------------------------------------ cube partition (design 2)
+
+@pytest.mark.parametrize("shape,cube", [((4, 8, 8), (1, 2, 2)), ((5, 7, 9), (2, 2, 2)), ((21, 45, 80), (2, 2, 2)),
+                                        ((3, 5, 6), (1, 1, 1)), ((4, 6, 10), (4, 6, 10)), ((7, 3, 5), (2, 4, 4))])
+def test_cube_order_closed_form(shape, cube):
+    T, H, W = shape
+    t, h, w = cube
+    o = oracle.cube_order(T, H, W, t, h, w)
+    N = T * H * W
+    assert np.array_equal(np.sort(o["row_of_n"]), np.arange(N))
+    assert np.array_equal(o["n_of_row"][o["row_of_n"]], np.arange(N))
+    KT, KH, KW = -(-T // t), -(-H // h), -(-W // w)
+    assert o["count"].size == KT * KH * KW == oracle.num_cubes(T, H, W, t, h, w)
+    # closed form for the first row of each cube and the row of each token
+    for n in range(0, N, max(1, N // 997)):
+        tt, hh, ww = n // (H * W), (n // W) % H, n % W
+        kt, kh, kw = tt // t, hh // h, ww // w
+        st, sh, sw = min(t, T - kt * t), min(h, H - kh * h), min(w, W - kw * w)
+        k = (kt * KH + kh) * KW + kw
+        base = kt * t * H * W + st * (kh * h * W + sh * kw * w)
+        rho = base + ((tt - kt * t) * sh + (hh - kh * h)) * sw + (ww - kw * w)
+        assert o["cube_of_n"][n] == k
+        assert o["first"][k] == base
+        assert o["row_of_n"][n] == rho
+        assert o["count"][k] == st * sh * sw
+
+
+# ------------------------------------------------------------------ Eq. 1
+
+@pytest.mark.parametrize("cube", [(1, 2, 2), (2, 2, 2), (2, 4, 4)])
+def test_eq1_fp64_split_is_exact_for_power_of_two_cubes(cube):
+    wl = synth.WORKLOADS["tiny"]
+    X = synth.activations(wl)
+    mean, delta = oracle.cube_split_f64(X, wl.T, wl.H, wl.W, cube)
+    o = oracle.cube_order(wl.T, wl.H, wl.W, *cube)
+    x = _x_f64(X)
+    # kernel + delta reconstructs X exactly
+    assert np.array_equal(mean[o["cube_of_n"]] + delta, x)
+    # deltas sum to zero per cube, exactly (power-of-two counts)
+    sums = np.zeros_like(mean)
+    np.add.at(sums, o["cube_of_n"], delta)
+    assert np.all(o["count"] & (o["count"] - 1) == 0)
+    assert np.array_equal(sums, np.zeros_like(sums))
+
+
+def test_eq1_ragged_cubes_mean_over_present_tokens():
+    T, H, W = 3, 5, 7
+    X = synth.normal_bf16((T * H * W, 32), sd=3.0, seed=11)
+    mean, delta = oracle.cube_split_f64(X, T, H, W, (2, 2, 2))
+    o = oracle.cube_order(T, H, W, 2, 2, 2)
+    x = _x_f64(X)
+    for k in range(o["count"].size):
+        rows = o["n_of_row"][o["first"][k]:o["first"][k] + o["count"][k]]
+        np.testing.assert_allclose(mean[k], x[rows].mean(axis=0), rtol=0, atol=1e-12)
+        assert np.abs(delta[rows].sum(axis=0)).max() < 1e-12
+    assert sorted(set(o["count"].tolist())) == [1, 2, 4, 8]
+
+
+def test_fp32_means_within_rounding_of_exact():
+    wl = synth.WORKLOADS["tiny"]
+    X = synth.activations(wl)
+    m32 = oracle.cube_means(X, wl.T, wl.H, wl.W, wl.cube).astype(np.float64)
+    m64, _ = oracle.cube_split_f64(X, wl.T, wl.H, wl.W, wl.cube)
+    # 3 sequential adds + 1 division, each within half an ulp of its result
+    bound = 4 * np.spacing(np.abs(m64).astype(np.float32).astype(np.float64) * 4 + 1e-30)
+    assert np.all(np.abs(m32 - m64) <= bound)
+
+
+def test_mean_is_sequential_fp32_sum_in_thw_order():
+    # hand-derived: a cube whose tokens, in (t,h,w) order, carry 2^30, 1, -2^30, 1
+    # in channel 0.  Summed one at a time in fp32: (0+2^30)+1 = 2^30 (the 1 is
+    # below half an ulp of 2^30), then 0, then 1; mean = 1/4.  Any other order
+    # or an fp64 sum would give 1/2.
+    T, H, W, Ci = 1, 2, 2, 16
+    vals = np.array([2.0 ** 30, 1.0, -(2.0 ** 30), 1.0])
+    Xf = np.zeros((4, Ci))
+    Xf[:, 0] = vals
+    X = oracle.bf16_round_fast(Xf)
+    m = oracle.cube_means(X, T, H, W, (1, 2, 2))
+    assert m[0, 0] == np.float32(0.25)
+    # the same tokens stored in another (t,h,w) arrangement change the order
+    Y = X[[0, 2, 1, 3]]          # tokens now visited as 2^30, -2^30, 1, 1
+    assert oracle.cube_means(Y, T, H, W, (1, 2, 2))[0, 0] == np.float32(0.5)
+
+
+# ------------------------------------------------------------------ Eq. 4 quantiser
+
+def test_fp4_reproduces_exact_grid_values():
+    rng = np.random.default_rng(2)
+    rows, cols = 64, 256
+    S = 2.0 ** -7
+    mags = oracle.e2m1_value(np.arange(8))
+    e4 = oracle.e4m3_value(np.arange(1, 127))
+    # each block: scale s_b on the E4M3 grid, codes anywhere, one element = +-6
+    sb = rng.choice(e4[(e4 >= 2.0 ** -6) & (e4 <= 448)], size=(rows, cols // 16))
+    q = rng.choice(np.concatenate([mags, -mags[1:]]), size=(rows, cols))
+    q[:, ::16] = 6.0 * rng.choice([-1, 1], size=(rows, cols // 16))
+    sb[0, 0] = 448.0
+    Z = (q * np.repeat(sb, 16, axis=1) * S)
+    assert np.array_equal(Z.astype(np.float32).astype(np.float64), Z)
+    codes, scales, S_out = oracle.fp4_quantize(Z.astype(np.float32))
+    # S = amax / (6*448) = (6*448*S)/(6*448)
+    assert S_out == S
+    assert np.array_equal(oracle.e4m3_value(scales), sb)
+    lo, hi = codes & 15, codes >> 4
+    dq = np.empty((rows, cols))
+    dq[:, 0::2], dq[:, 1::2] = oracle.e2m1_value(lo), oracle.e2m1_value(hi)
+    assert np.array_equal(dq, q)
+
+
+def test_fp4_amax_maps_to_qmax():
+    # Eq. 4: s = max|X| / q_max, so the largest element lands on q_max = 6
+    Z = synth.normal_bf16((32, 128), sd=2.0, seed=4)
+    Zf = oracle.bf16_value(Z)
+    codes, scales, S = oracle.fp4_quantize(Zf)
+    i = np.unravel_index(np.argmax(np.abs(Zf)), Zf.shape)
+    code = (codes[i[0], i[1] // 2] >> (4 * (i[1] % 2))) & 15
+    assert abs(oracle.e2m1_value([code])[0]) == 6.0
+    assert oracle.e4m3_value([scales[i[0], i[1] // 16]])[0] == 448.0
+    assert S == np.float32(np.abs(Zf).max()) / np.float32(2688.0)
+
+
+def test_fp4_monotone_and_bounded_error():
+    rng = np.random.default_rng(9)
+    base = rng.standard_normal((1, 16)).astype(np.float32)
+    sweep = np.linspace(-3, 3, 4001).astype(np.float32)
+    Z = np.repeat(base, sweep.size, axis=0)
+    Z[:, 5] = sweep
+    codes, scales, S = oracle.fp4_quantize(Z, S=2.0 ** -6)
+    c5 = (codes[:, 2] >> 4) & 15
+    dq = oracle.e2m1_value(c5) * oracle.e4m3_value(scales[:, 0]) * S
+    # blocks whose scale did not change must be monotone in the swept element
+    for s in np.unique(scales[:, 0]):
+        sel = scales[:, 0] == s
+        assert np.all(np.diff(dq[sel]) >= 0)
+    # element error at most half the coarsest step (2 * s_b * S) of its block
+    err = np.abs(dq - sweep)
+    assert np.all(err <= oracle.e4m3_value(scales[:, 0]) * S * 1.0 + 1e-12)
+
+
+def test_worked_example_eq1_eq4():
+    """Hand-derived example: one 1x2x2 cube of 16 channels.
+
+    Tokens in (t,h,w) order carry d = (3, -1, 1, -3);  x[n][c] = m_c + d_n g_c with
+      c = 0..7:   m_c = c/2, g_c = 1/16
+      c = 8..14:  m_c = 1,   g_c = 7/64
+      c = 15:     m_c = 14,  g_c = 0
+    Every x is exact in BF16 and every partial sum exact in fp32, so:
+      kernel token = m; max|m| = 14 -> s8 = 14/448 = 2^-5; q8 = E4M3(32 m) exactly
+        (0,16,32,48,64,80,96,112 | 32 | 448);
+      deltas d g; global amax = 3 * 7/64 = 21/64 -> S = (21/64)/2688 = 2^-13;
+      tokens 0, 3 (|d| = 3): block amax 21/64, (21/64)/(6 * 2^-13) = 448 -> s_b = 448,
+        eff = 448 * 2^-13 = 7/128; c < 8: (3/16)/(7/128) = 24/7 = 3.43 -> 3;
+        c = 8..14: exactly 6; c = 15: +0;
+      tokens 1, 2 (|d| = 1): block amax 7/64, (7/64)/(6 * 2^-13) = 448/3 = 149.3
+        -> E4M3 144 (160 is farther), eff = 144 * 2^-13 = 9/512;
+        c < 8: (1/16)/(9/512) = 3.56 -> 4 (past the 3.5 midpoint);
+        c = 8..14: 7/64 / (9/512) = 6.22 -> 6 (saturated); c = 15: +0.
+    """
+    Ci = 16
+    m = np.array([c / 2 for c in range(8)] + [1.0] * 7 + [14.0])
+    g = np.array([1 / 16] * 8 + [7 / 64] * 7 + [0.0])
+    d = np.array([3.0, -1.0, 1.0, -3.0])
+    Xf = m[None, :] + d[:, None] * g[None, :]
+    X = oracle.bf16_round_fast(Xf)
+    assert np.array_equal(oracle.bf16_value(X).astype(np.float64), Xf)
+    act = oracle.quantize_activations(X, 1, 2, 2, (1, 2, 2))
+    assert np.array_equal(act["means"][0].astype(np.float64), m)
+    assert act["s8"][0] == np.float32(2.0 ** -5)
+    assert np.array_equal(oracle.e4m3_value(act["q8"][0]), 32 * m)
+    assert act["amax_delta"] == np.float32(21 / 64)
+    assert act["S_delta"] == np.float32(2.0 ** -13)
+    assert list(oracle.e4m3_value(act["dscales"][:, 0])) == [448.0, 144.0, 144.0, 448.0]
+    codes = act["dcodes"]
+    got = np.empty((4, Ci), dtype=np.int64)
+    got[:, 0::2], got[:, 1::2] = codes & 15, codes >> 4
+    want = np.zeros((4, Ci), dtype=np.int64)
+    for n, (lo, mid) in enumerate([(5, 7), (8 | 6, 8 | 7), (6, 7), (8 | 5, 8 | 7)]):
+        want[n, :8], want[n, 8:15], want[n, 15] = lo, mid, 0
+    assert np.array_equal(got, want)
+
+
+# ------------------------------------------------------------------ Eq. 2 / Eq. 3 assembly
+
+def _dequant_rows(codes, scales, S):
+    rows, half = codes.shape
+    v = np.empty((rows, half * 2))
+    v[:, 0::2] = oracle.e2m1_value(codes & 15)
+    v[:, 1::2] = oracle.e2m1_value(codes >> 4)
+    return v * np.repeat(oracle.e4m3_value(scales), 16, axis=1) * S
+
+
+@pytest.fixture(scope="module")
+def tiny_case():
+    wl = synth.WORKLOADS["tiny"]
+    X = synth.activations(wl)
+    Wb = synth.weight(wl)
+    L1, L2, sig = oracle.lowrank_factors(Wb, wl.rank)
+    act = oracle.quantize_activations(X, wl.T, wl.H, wl.W, wl.cube)
+    wq = oracle.quantize_weight(Wb, L1, L2)
+    return wl, X, Wb, L1, L2, sig, act, wq
+
+
+def test_split_product_matches_brute_force(tiny_case):
+    wl, X, Wb, L1, L2, sig, act, wq = tiny_case
+    # A' = dq(delta) in natural order + broadcast of the dequantised kernel token
+    dqd = _dequant_rows(act["dcodes"], act["dscales"], act["S_delta"])[act["row_of_n"]]
+    dqk = oracle.e4m3_value(act["q8"]) * act["s8"][:, None].astype(np.float64)
+    A = dqd + dqk[act["cube_of_n"]]
+    dqW = _dequant_rows(wq["wcodes"], wq["wscales"], wq["S_w"])
+    l1, l2 = oracle.bf16_value(L1).astype(np.float64), oracle.bf16_value(L2).astype(np.float64)
+    Y_bf = A @ dqW.T + (_x_f64(X) @ l1) @ l2
+    Y = oracle.output_rows(act, wq, X, L1, L2, np.arange(wl.N))
+    np.testing.assert_allclose(Y, Y_bf, rtol=1e-12, atol=1e-12 * np.abs(Y_bf).max())
+
+
+def test_unit_cube_has_zero_deltas_and_reduces_to_w4a8(tiny_case):
+    wl, X, Wb, L1, L2, sig, _, wq = tiny_case
+    act = oracle.quantize_activations(X, wl.T, wl.H, wl.W, (1, 1, 1))
+    assert act["amax_delta"] == 0.0 and act["S_delta"] == 1.0
+    assert not act["dcodes"].any() and not act["dscales"].any()
+    assert np.array_equal(act["row_of_n"], np.arange(wl.N))
+    # per-token W4A8: q8 s8 dq(R)^T, plus the low-rank term
+    x = _x_f64(X)
+    s8 = np.abs(oracle.bf16_value(X)).max(axis=1) / np.float32(448.0)
+    assert np.array_equal(act["s8"], s8.astype(np.float32))
+    dqW = _dequant_rows(wq["wcodes"], wq["wscales"], wq["S_w"])
+    q = oracle.e4m3_value(act["q8"]) * act["s8"][:, None].astype(np.float64)
+    l1, l2 = oracle.bf16_value(L1).astype(np.float64), oracle.bf16_value(L2).astype(np.float64)
+    Y_ref = q @ dqW.T + (x @ l1) @ l2
+    Y = oracle.output_rows(act, wq, X, L1, L2, np.arange(wl.N))
+    np.testing.assert_allclose(Y, Y_ref, rtol=1e-12, atol=1e-12 * np.abs(Y_ref).max())
+
+
+def test_residual_against_library_matmul(tiny_case):
+    wl, X, Wb, L1, L2, *_ = tiny_case
+    R = oracle.residual(Wb, L1, L2)
+    l1, l2 = oracle.bf16_value(L1).astype(np.float64), oracle.bf16_value(L2).astype(np.float64)
+    ref = oracle.bf16_value(Wb).astype(np.float64) - (l1 @ l2).T
+    # different fp64 summation order: at most one fp32 rounding step apart
+    assert np.all(np.abs(R - ref) <= np.spacing(np.abs(ref).astype(np.float32)))
+
+
+def test_lowrank_eckart_young(tiny_case):
+    wl, X, Wb, L1, L2, sig, *_ = tiny_case
+    w = oracle.bf16_value(Wb).astype(np.float64)
+    l1, l2 = oracle.bf16_value(L1).astype(np.float64), oracle.bf16_value(L2).astype(np.float64)
+    err2 = np.linalg.norm(w - (l1 @ l2).T) ** 2
+    tail = np.sum(sig[wl.rank:] ** 2)
+    # BF16 rounding of the factors adds at most about 2^-8 relative on L1 L2
+    rnd = (2.0 ** -8 * np.linalg.norm(l1 @ l2)) ** 2
+    assert err2 <= (1 + 1e-3) * tail + 4 * rnd
+
+
+def test_full_rank_factors_reconstruct_w():
+    Wb = synth.normal_bf16((64, 48), sd=0.1, seed=21)
+    L1, L2, sig = oracle.lowrank_factors(Wb, 48)
+    w = oracle.bf16_value(Wb).astype(np.float64)
+    rec = (oracle.bf16_value(L1).astype(np.float64) @ oracle.bf16_value(L2).astype(np.float64)).T
+    assert np.linalg.norm(w - rec) <= 2.0 ** -7 * np.linalg.norm(w)
+
+
+# ------------------------------------------------------------------ the method's claim
+
+@pytest.mark.parametrize("name,shape", [("tiny", None), ("mid", (4, 16, 16, 512, 384))])
+def test_delta_split_beats_plain_fp4(name, shape):
+    """Design 1/3 and the cube-size ablation: on spatially and temporally
+    correlated activations, quantising deltas against a local FP8 kernel token
+    gives a lower Frobenius error than per-token-group FP4 of X itself."""
+    wl = synth.WORKLOADS["tiny"]
+    if shape:
+        T, H, W, Ci, Co = shape
+        wl = synth.Workload("mid", T, H, W, Ci, Co, 16, (1, 2, 2), (T, math.ceil(H / 4), math.ceil(W / 4)),
+                            (0.01, 50.0), (0.01, 20.0))
+    X = synth.activations(wl, seed=77)
+    Wb = synth.weight(wl, seed=78)
+    L1, L2, _ = oracle.lowrank_factors(Wb, wl.rank)
+    wq = oracle.quantize_weight(Wb, L1, L2)
+    rows = np.arange(0, wl.N, max(1, wl.N // 256))
+    ref = _x_f64(X)[rows] @ oracle.bf16_value(Wb).astype(np.float64).T
+    act = oracle.quantize_activations(X, wl.T, wl.H, wl.W, wl.cube)
+    y_dq = oracle.output_rows(act, wq, X, L1, L2, rows)
+    plain = oracle.quantize_plain(X)
+    plain.update(row_of_n=None, cube_of_n=None, q8=None, s8=None)
+    y_pl = oracle.output_rows(plain, wq, X, L1, L2, rows, kernel=False, cube_major=False)
+    e_dq = np.linalg.norm(y_dq - ref) / np.linalg.norm(ref)
+    e_pl = np.linalg.norm(y_pl - ref) / np.linalg.norm(ref)
+    assert e_dq < e_pl, (e_dq, e_pl)
+    assert e_dq < 0.2
+
+
+def test_delta_magnitudes_smaller_than_x():
+    """Design 1: residuals against the cube mean are smaller and have fewer outliers."""
+    wl = synth.WORKLOADS["tiny"]
+    X = synth.activations(wl)
+    _, delta = oracle.cube_split_f64(X, wl.T, wl.H, wl.W, wl.cube)
+    x = _x_f64(X)
+    assert np.abs(delta).max() < 0.5 * np.abs(x).max()
+    assert np.sqrt((delta ** 2).mean()) < 0.2 * np.sqrt((x ** 2).mean())
+
+
+def test_worked_example_fixture():
+    """The hand-derived worked example stored under tests/golden (closed-form
+    values written by make_worked_example.py, no oracle involved)."""
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "worked_cube_1x2x2.json")
+    g = json.load(open(path))
+    X = np.array(g["X_bf16"], dtype=np.uint16)
+    act = oracle.quantize_activations(X, g["T"], g["H"], g["W"], tuple(g["cube"]))
+    assert np.array_equal(act["means"][0], np.array(g["means"], np.float32))
+    assert act["s8"][0] == np.float32(g["s8"])
+    assert np.array_equal(act["q8"][0], np.array(g["q8"], np.uint8))
+    assert act["amax_delta"] == np.float32(g["amax_delta"])
+    assert act["S_delta"] == np.float32(g["S_delta"])
+    assert np.array_equal(act["dscales"][:, 0], np.array(g["dscales"], np.uint8))
+    assert np.array_equal(act["dcodes"], np.array(g["dcodes"], np.uint8))
