@@ -1,0 +1,368 @@
+"""Throughput of the DeltaQuant W4A4 linear layer on B200.
+
+One step = one forward of the whole layer (cube statistics, cube encode,
+kernel-token product, main FP4 product with the low-rank slab and the
+scatter epilogue) over one synthetic activation tensor X resident in HBM.
+Default workload: the Wan-like 480p attention projection (T=21, H=30, W=52,
+N=32760 tokens, Ci=Co=5120, rank 32, cube 1x2x2).
+
+Prints one JSON line (rank 0).  `value` is whole-job TFLOP/s with
+F = 2 N Ci Co + 2 K Ci Co + 2 N r (Ci + Co) (main + kernel-token + low-rank
+products, real rows only) per step; tokens/s and the per-stage breakdown are
+extra keys.  --impl reference times the CPU oracle on a bounded sample of
+the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "W4A4 DeltaQuant linear TFLOPS & tokens/s; % of dense FP4 / HBM roofline"
+FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+
+
+def layer_flops(wl, K):
+    return 2.0 * wl.N * wl.Ci * wl.Co + 2.0 * K * wl.Ci * wl.Co + 2.0 * wl.N * wl.rank * (wl.Ci + wl.Co)
+
+
+def stage_model(wl, K, slab):
+    """Algorithmic work per launch of each stage (bytes that must cross HBM,
+    tensor FLOPs).  Stage 1 reads X twice (statistics, then encode: the
+    per-tensor delta scale needs every delta first)."""
+    N, Ci, Co, r = wl.N, wl.Ci, wl.Co, wl.rank
+    quant_bytes = (4.0 * N * Ci                      # X read by a1 and a2
+                   + N * Ci / 2 + N * Ci / 16        # delta codes + scales
+                   + K * Ci * 3                      # q8 (E4M3) + its BF16 copy
+                   + N * r * 4 * 2                   # X L1 partials (write + read)
+                   + N * slab * 2 + 2 * r * Ci)      # U hi/lo, L1
+    kernel_flops = 2.0 * K * Ci * Co
+    kernel_bytes = K * Ci * 2 + Co * Ci * 2 + K * Co * 4
+    main_flops = 2.0 * N * Ci * Co + 2.0 * N * slab * Co
+    main_bytes = N * Ci * 9 / 16 + Co * Ci * 9 / 16 + N * slab * 2 + Co * slab * 2 + K * Co * 4 + N * Co * 2
+    return dict(quantize=dict(bytes=quant_bytes, flops=2.0 * N * Ci * r),
+                kernel_gemm=dict(bytes=kernel_bytes, flops=kernel_flops),
+                main_gemm=dict(bytes=main_bytes, flops=main_flops))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]), source="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", str(self.index)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return dict(sm_mhz=statistics.median(sm), sm_max_mhz=mx, reasons=sorted(reasons), samples=len(sm))
+
+
+def parse_cube(s):
+    return tuple(int(v) for v in s.split(",")) if s else None
+
+
+# --------------------------------------------------------------------------- reference arm (CPU oracle)
+
+def oracle_sample(wl, cube, X, Wb, L1, L2, wq, ntok):
+    """Oracle over a bounded sample: the first `ntok`-token prefix of whole
+    cube rows (a slab of frames cut at cube boundaries), quantised as its own
+    tensor, then its Y rows.  Returns (seconds, flops of the sample)."""
+    import oracle
+    t, h, w = cube
+    # rows of whole cube-rows: take frames [0, t) and cube rows until ntok tokens
+    per_cube_row = t * h * wl.W
+    n_rows = max(1, ntok // per_cube_row)
+    Hs = min(wl.H, n_rows * h)
+    Ts = min(wl.T, t)
+    idx = (np.arange(Ts)[:, None, None] * wl.H * wl.W + np.arange(Hs)[None, :, None] * wl.W
+           + np.arange(wl.W)[None, None, :]).reshape(-1)
+    Xs = np.ascontiguousarray(X[idx])
+    t0 = time.perf_counter()
+    act = oracle.quantize_activations(Xs, Ts, Hs, wl.W, cube)
+    rows = np.arange(Xs.shape[0])
+    oracle.output_rows(act, wq, Xs, L1, L2, rows)
+    dt = time.perf_counter() - t0
+    K = oracle.num_cubes(Ts, Hs, wl.W, *cube)
+    sub = synth.Workload("sample", Ts, Hs, wl.W, wl.Ci, wl.Co, wl.rank, cube, wl.grid, wl.x_outliers, wl.w_outliers)
+    return dt, layer_flops(sub, K), Xs.shape[0]
+
+
+def run_reference(args, wl, cube):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    X = synth.activations(wl)
+    Wb = synth.weight(wl)
+    L1, L2, _ = oracle.lowrank_factors(Wb, wl.rank)
+    wq = oracle.quantize_weight(Wb, L1, L2)
+    ntok = args.sample_tokens
+    for _ in range(args.warmup):
+        oracle_sample(wl, cube, X, Wb, L1, L2, wq, ntok)
+    times, flops, toks = [], 0.0, 0
+    for _ in range(args.steps):
+        dt, f, n = oracle_sample(wl, cube, X, Wb, L1, L2, wq, ntok)
+        times.append(dt)
+        flops, toks = f, n
+    t = sum(times) / len(times)
+    value = flops / t / 1e12
+    cores = os.cpu_count()
+    sample = (f"{toks} tokens ({cube[0]}x{cube[1]}x{cube[2]} cubes, whole cube rows of frame slab 0) of "
+              f"{wl.name}, full Ci={wl.Ci}, Co={wl.Co}, r={wl.rank}; fp64 Y rows; per step")
+    line = dict(metric=METRIC, value=value, unit="TFLOP/s", impl="reference", n_gpus=args.gpus, steps=args.steps,
+                warmup=args.warmup, ms_per_step=t * 1e3, higher_is_better=True, scaling="weak", vs_baseline=None,
+                dtype="f64", data="synthetic",
+                config=dict(workload=wl.name, T=wl.T, H=wl.H, W=wl.W, Ci=wl.Ci, Co=wl.Co, rank=wl.rank,
+                            cube=list(cube), sample_tokens=toks),
+                tokens_per_s=toks / t,
+                cpu_baseline=dict(value=value, unit="TFLOP/s", cores=cores, kind="oracle", sample=sample),
+                e2e=dict(value=value, unit="TFLOP/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="dq", choices=["dq", "reference"])
+    ap.add_argument("--workload", default="wan480p_proj", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--cube", default=None, help="override the cube, e.g. 2,2,2")
+    ap.add_argument("--sample-tokens", type=int, default=256, help="oracle sample size (tokens)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = synth.WORKLOADS[args.workload]
+    cube = parse_cube(args.cube) or wl.cube
+    wl = wl.with_cube(cube)
+    if args.impl == "reference":
+        return run_reference(args, wl, cube)
+
+    import torch
+    import video_diffusion_w4a4_b200 as dq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    t, h, w = cube
+    K = dq.dq_cube_count(wl.T, wl.H, wl.W, t, h, w)
+    # inputs: each rank its own activation tensor (a different denoising step), one shared weight
+    X = synth.activations(wl, tau=rank)
+    Wb = synth.weight(wl)
+    t0 = time.perf_counter()
+    packed, L1m, L2s = dq.dq_pack_weight(Wb, wl.rank)
+    pack_s = time.perf_counter() - t0
+    Xd = torch.from_numpy(X.view(np.int16)).to(dev)
+    Pd = torch.from_numpy(packed).to(dev)
+    L1d = torch.from_numpy(L1m.view(np.int16)).to(dev)
+    L2d = torch.from_numpy(L2s.view(np.int16)).to(dev)
+    Yd = torch.empty((wl.N, wl.Co), dtype=torch.int16, device=dev)
+    lay = dq.dq_workspace_layout_get(wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank)
+    ws = torch.zeros(lay.total_bytes, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream(dev)
+
+    def step(events=None):
+        dq.dq_linear_forward_ex(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd, ws,
+                                lay.total_bytes, dq.DQ_STAGE_ALL, events, st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    status = dq.dq_read_device_status(ws, st, clear=True)
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {dq.dq_status_string(status)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(st)
+        for i in range(args.steps):
+            step(evs[i])
+        end.record(st)
+        torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    ms = start.elapsed_time(end) / args.steps
+    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+                for j, n in enumerate(("quantize", "kernel_gemm", "main_gemm"))}
+    status = dq.dq_read_device_status(ws, st, clear=True)
+    if status != 0:
+        raise RuntimeError(f"device status after timing: {dq.dq_status_string(status)}")
+    if dist:
+        tm = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        ms = float(tm.item())
+
+    # end to end through the host-buffer entry point: pinned X in, Y out, copies inside the timed region
+    Xh = torch.from_numpy(X.view(np.int16)).pin_memory()
+    Yh = torch.empty((wl.N, wl.Co), dtype=torch.int16).pin_memory()
+    Xd2, Yd2 = torch.empty_like(Xd), torch.empty_like(Yd)
+
+    def e2e_step():
+        dq.dq_linear_forward_host(Xh, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yh, Xd2, Yd2,
+                                  ws, lay.total_bytes, st)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if dist:
+        tm = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tm.item())
+        dist.barrier()
+
+    F = layer_flops(wl, K)
+    value = F * world / (ms * 1e-3) / 1e12
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16"] * FP4_PER_BF16
+    model = stage_model(wl, K, lay.slab)
+    # dominant kernel = the stage with the largest share of the step
+    dom = max(stage_ms, key=stage_ms.get)
+    if dom == "quantize":
+        ach = model[dom]["bytes"] / (stage_ms[dom] * 1e-3) / 1e9
+        roof = dict(kernel="k_cube_stats+k_cube_encode", bound="hbm", achieved=ach, peak=peaks["hbm"], unit="GB/s")
+    else:
+        pk = fp4_peak if dom == "main_gemm" else peaks["bf16"]
+        ach = model[dom]["flops"] / (stage_ms[dom] * 1e-3) / 1e12
+        roof = dict(kernel="k_main_gemm" if dom == "main_gemm" else "k_kernel_gemm", bound="tensor", achieved=ach,
+                    peak=pk, unit="TFLOP/s")
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["peak_source"] = ("measured" if peaks["source"] == "measured" else "fallback") + (
+        " bf16 x 4 (nominal FP4:BF16)" if roof["unit"] == "TFLOP/s" and dom == "main_gemm" else "")
+    stages = {}
+    for n, tms in stage_ms.items():
+        m = model[n]
+        stages[n] = dict(ms=tms, tflops=m["flops"] / (tms * 1e-3) / 1e12, gbs=m["bytes"] / (tms * 1e-3) / 1e9)
+    stages["quantize"]["frac_hbm"] = stages["quantize"]["gbs"] / peaks["hbm"]
+    stages["kernel_gemm"]["frac_bf16"] = stages["kernel_gemm"]["tflops"] / peaks["bf16"]
+    stages["main_gemm"]["frac_fp4"] = stages["main_gemm"]["tflops"] / fp4_peak
+    layer_bytes = sum(m["bytes"] for m in model.values())
+    layer_roof_ms = max(F / (fp4_peak * 1e12), layer_bytes / (peaks["hbm"] * 1e9)) * 1e3
+    line = dict(metric=METRIC, value=value, unit="TFLOP/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+                ms_per_step=ms, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="e2m1/e4m3->f32",
+                data="synthetic",
+                config=dict(workload=wl.name, T=wl.T, H=wl.H, W=wl.W, N=wl.N, Ci=wl.Ci, Co=wl.Co, rank=wl.rank,
+                            cube=list(cube), K=K, parallelism=f"dp{world} (independent layer per GPU)",
+                            l2="inputs larger than L2 (X %.0f MB, Y %.0f MB)" % (wl.N * wl.Ci * 2 / 1e6,
+                                                                                 wl.N * wl.Co * 2 / 1e6)),
+                tokens_per_s=wl.N * world / (ms * 1e-3),
+                layer_roofline_frac=layer_roof_ms / ms,
+                roofline=roof, stages=stages,
+                e2e=dict(value=F * world / (e2e_ms * 1e-3) / 1e12, unit="TFLOP/s",
+                         h2d_bytes_per_step=wl.N * wl.Ci * 2, d2h_bytes_per_step=wl.N * wl.Co * 2, ms_per_step=e2e_ms),
+                gpu_launches=4 * args.steps, pack_seconds=pack_s)
+    clk_sum = clk.summary()
+    if clk_sum:
+        line["clocks"] = clk_sum
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        L1, L2 = dq.dq_lowrank_factors(Wb, wl.rank)
+        wq = oracle.quantize_weight(Wb, L1, L2)
+        dt, f, n = oracle_sample(wl, cube, X, Wb, L1, L2, wq, args.sample_tokens)
+        line["cpu_baseline"] = dict(value=f / dt / 1e12, unit="TFLOP/s", cores=os.cpu_count(), kind="oracle",
+                                    sample=f"{n} tokens of {wl.name} (whole cube rows, frame slab 0), "
+                                           f"Ci={wl.Ci}, Co={wl.Co}, r={wl.rank}, {dt:.1f} s")
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

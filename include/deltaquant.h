@@ -1,0 +1,255 @@
+/*
+ * deltaquant.h -- C ABI of the DeltaQuant W4A4 linear layer for B200 (sm_100a).
+ *
+ * The layer (papernotes.org, "DeltaQuant: 4-bit Video Diffusion Models with
+ * Spatiotemporal Delta Smoothing", key designs 2-4):
+ *   X (N = T*H*W tokens x Ci channels, BF16, rows in (t,h,w) row-major order)
+ *   is viewed as T x H x W x Ci and cut into t x h x w cubes (design 2).  Each
+ *   cube's fp32 mean is its kernel token, each token minus its cube's mean a
+ *   delta token (Eq. 1).  Kernel tokens are quantised to FP8 E4M3 with one fp32
+ *   scale per token; delta tokens to FP4 E2M1 with one E4M3 scale per 16
+ *   channels and one fp32 per-tensor scale (Eq. 4 with the NVFP4 reading).
+ *   W (Co x Ci) is split offline into rank-r BF16 factors L1, L2 from its SVD
+ *   and a residual R = W - L1 L2 quantised to the same FP4 format (Eq. 3):
+ *     Y = dq(delta) dq(R)^T + broadcast_cube(dq(kernel) dq(R)^T) + (X L1) L2
+ *   Y is N x Co BF16 in (t,h,w) order.
+ *
+ * Conventions for every entry point:
+ *   - The return value is a dq_status code; nothing aborts or exits.
+ *   - Arguments are checked before anything is launched or written.
+ *   - "host" pointers are ordinary CPU memory; "device" pointers are global
+ *     memory of the current CUDA device.  The caller owns every buffer.
+ *   - Online entry points are asynchronous on the given stream (a
+ *     cudaStream_t passed as void*; NULL = legacy default stream).  Errors
+ *     found by the device (bad packed-weight header, a bounded wait that ran
+ *     out) are written to a status word inside the workspace; read it with
+ *     dq_read_device_status after the stream has been synchronised.
+ *   - Inputs are never modified; outputs are fully overwritten.
+ *   - Shapes: Ci and Co multiples of 256; rank a multiple of 16 in [16, 128];
+ *     1 <= t <= T, 1 <= h <= H, 1 <= w <= W; t*h*w <= 128.  Anything else returns
+ *     DQ_ERR_UNSUPPORTED_SHAPE.  Device pointers must be 256-byte aligned
+ *     (DQ_ERR_ALIGNMENT otherwise).
+ */
+#ifndef DELTAQUANT_H
+#define DELTAQUANT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DQ_ABI_VERSION 1
+#define DQ_PACK_FORMAT_VERSION 1
+#define DQ_PACK_MAGIC 0x31575144u /* "DQW1" little-endian */
+
+typedef enum dq_status {
+    DQ_OK = 0,
+    DQ_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad flag */
+    DQ_ERR_UNSUPPORTED_SHAPE = 2,  /* shape outside the conventions above */
+    DQ_ERR_ALIGNMENT = 3,          /* a device pointer is not 256-byte aligned */
+    DQ_ERR_WORKSPACE_TOO_SMALL = 4,
+    DQ_ERR_CUDA = 5,               /* a CUDA runtime call failed */
+    DQ_ERR_DEVICE_TIMEOUT = 6,     /* a bounded device-side wait ran out */
+    DQ_ERR_BAD_PACKED_WEIGHT = 7,  /* packed-weight header does not match */
+    DQ_ERR_NO_DEVICE = 8,          /* no usable sm_100 device */
+    DQ_ERR_ALLOC = 9               /* host or device allocation failed */
+} dq_status;
+
+/* Text for a status code (static storage). */
+const char* dq_status_string(int status);
+
+/* DQ_ABI_VERSION of the loaded library. */
+int dq_abi_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Layout maps                                                               */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Cube partition (key design 2): KT = ceil(T/t), KH = ceil(H/h), KW = ceil(W/w),
+ * K = KT*KH*KW cubes, cube k = (kt*KH + kh)*KW + kw.  Edge cubes that the
+ * lattice cuts short hold fewer tokens (their mean is over those tokens).
+ * Cube-major order lists the cubes in k order and, inside a cube, its tokens
+ * in (t,h,w) order.  dq_cube_major_row maps natural token n to its cube-major
+ * row and cube.
+ */
+int dq_cube_count(int T, int H, int W, int t, int h, int w, long long* K);
+int dq_cube_major_row(int T, int H, int W, int t, int h, int w, long long n, long long* row,
+                      long long* cube);
+
+/*
+ * Scale-factor layout of an FP4 matrix with `rows` rows and `cols` columns
+ * (one E4M3 scale per 16 consecutive columns of a row).  Rows are grouped by
+ * 128 and columns by 64; each (row group, column group) owns 512 contiguous
+ * bytes in which scale (row, block) sits at
+ *   (row % 32) * 16 + ((row % 128) / 32) * 4 + (block % 4),
+ * groups ordered row-group-major:
+ *   offset = ((row/128) * (cols/64) + block/4) * 512 + (the above).
+ * This is the order in which the tensor cores' block-scaled MMA reads scale
+ * factors from tensor memory after a 32x128-bit copy, so tiles move with bulk
+ * copies and no reshuffle.  Total size: ceil(rows/128) * (cols/64) * 512.
+ */
+int dq_sf_offset(long long row, int block, int cols, size_t* offset);
+int dq_sf_bytes(long long rows, int cols, size_t* bytes);
+
+/* ------------------------------------------------------------------------ */
+/* Offline weight packing (host only, synchronous)                           */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Packed weight blob (device copy of what dq_pack_weight writes), all
+ * sections 256-byte aligned:
+ *   header  256 bytes: uint32 magic, uint32 version, int32 Co, Ci, rank,
+ *           slab, float S_W, then uint64 byte offsets of the sections below.
+ *   codes   Co x Ci/2 bytes, E2M1 codes of R, row o = output channel,
+ *           channel 2i in the low nibble of byte i.
+ *   scales  E4M3 group-16 scales of R in the scale-factor layout above.
+ *   dqw     Co x Ci BF16 values q * s_b of R (exact: at most 6 significant
+ *           bits), the operand of the kernel-token product.
+ * S_W is R's per-tensor scale.  dq_packed_weight_bytes gives the size.
+ */
+typedef struct dq_packed_layout {
+    size_t total_bytes;
+    size_t off_codes, off_scales, off_dqw;
+    int Co, Ci, rank, slab;
+} dq_packed_layout;
+
+int dq_packed_weight_layout(int Co, int Ci, int rank, dq_packed_layout* out);
+int dq_packed_weight_bytes(int Co, int Ci, int rank, size_t* bytes);
+
+/*
+ * Width of the low-rank slab: 2*rank rounded up to a multiple of 64.  The
+ * up-projection runs as extra K-steps of the main product with A = [U_hi | U_lo]
+ * and B = [L2^T | L2^T], zero-padded to this width.
+ */
+int dq_lowrank_slab_width(int rank);
+
+/*
+ * Rank-r factors from a truncated SVD of W (SVDQuant low-rank branch, Eq. 3):
+ * W^T ~ V_r S_r U_r^T, L1 = V_r S_r^(1/2) (Ci x r), L2 = S_r^(1/2) U_r^T (r x Co),
+ * both rounded to BF16 (nearest even).  Randomised subspace iteration in fp64
+ * with the given seed.  W: host Co x Ci BF16 (y = x W^T).  Outputs: host, caller-owned.
+ */
+int dq_lowrank_factors(const uint16_t* W, int Co, int Ci, int rank, uint64_t seed, uint16_t* L1,
+                       uint16_t* L2);
+
+/*
+ * Pack W with given BF16 factors L1 (Ci x r, host) and L2 (r x Co, host):
+ *   R[o][i] = fl32(W[o][i] - sum_j L1[i][j] L2[j][o]) (fp64 sum, ascending j),
+ *   S_W = amax(R)/2688 (1 if 0), s_b = E4M3(amax_b / (6 S_W)),
+ *   q = E2M1(R / (s_b S_W))   (Eq. 4 per 16-channel group, nearest even, saturating).
+ * Writes the packed blob (host, packed_bytes >= dq_packed_weight_bytes), the
+ * tensor-core copies of the factors: L1_mma = L1^T (r x Ci BF16, host) and
+ * L2_slab (Co x slab BF16, host, [L2^T | L2^T | 0]), and optionally S_W.
+ */
+int dq_pack_weight_factors(const uint16_t* W, const uint16_t* L1, const uint16_t* L2, int Co, int Ci,
+                           int rank, void* packed, size_t packed_bytes, uint16_t* L1_mma,
+                           uint16_t* L2_slab, float* S_W);
+
+/* dq_lowrank_factors (seed 0) followed by dq_pack_weight_factors. */
+int dq_pack_weight(const uint16_t* W, int Co, int Ci, int rank, void* packed, size_t packed_bytes,
+                   uint16_t* L1_mma, uint16_t* L2_slab);
+
+/* ------------------------------------------------------------------------ */
+/* Online forward (device, asynchronous)                                      */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Workspace carve-up (all offsets 256-byte aligned).  Tensors a test or a
+ * profiler may read after a forward:
+ *   status     int32 device status word (0 = ok, else a dq_status)
+ *   scalars    uint32[4]: [0] bits of max|delta| (fp32), [1] S_delta (fp32)
+ *   kamax      K uint32: bits of max_c |mean_k[c]| per cube (fp32)
+ *   s8         K fp32 kernel-token scales
+ *   q8         K x Ci E4M3 kernel tokens
+ *   q8_bf16    K_pad x Ci BF16 copy of q8 (the kernel-token product's A operand)
+ *   dcodes     N x Ci/2 E2M1 delta codes, cube-major rows
+ *   dscales    delta group scales, scale-factor layout over N rows
+ *   u_part     splits x N x rank fp32 partial sums of X L1 (cube-major rows)
+ *   u_hilo     N x slab BF16: U' = (X L1)/(S_delta S_W) split as hi + lo
+ *   p          K x Co fp32: s8 S_W q8 dqw^T (the per-cube kernel term)
+ */
+typedef struct dq_workspace_layout {
+    size_t total_bytes;
+    size_t off_status, off_scalars, off_kamax, off_s8, off_q8, off_q8_bf16, off_dcodes, off_dscales,
+        off_u_part, off_u_hilo, off_p;
+    long long N, K, N_pad, K_pad;
+    int splits, slab;
+} dq_workspace_layout;
+
+int dq_workspace_layout_get(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                            dq_workspace_layout* out);
+int dq_workspace_bytes(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                       size_t* bytes);
+
+/* Stage selection for dq_linear_forward_ex. */
+#define DQ_STAGE_QUANTIZE 1    /* cube statistics + cube encode (kernels a1, a2) */
+#define DQ_STAGE_KERNEL_GEMM 2 /* kernel-token product P (kernel c) */
+#define DQ_STAGE_MAIN_GEMM 4   /* block-scaled FP4 product + low-rank slab + epilogue (kernel b) */
+#define DQ_STAGE_ALL 7
+
+/*
+ * Y = DeltaQuant linear layer of X (see top of file), on `stream`.
+ *   X        device, N x Ci BF16, (t,h,w) row-major
+ *   packed_W device, the blob written by dq_pack_weight (copied to device)
+ *   L1_mma   device, rank x Ci BF16;  L2_slab device, Co x slab BF16
+ *   Y        device, N x Co BF16, (t,h,w) row-major
+ * Uses a library-owned workspace on the current device, allocated on the
+ * first call for the largest shape seen so far (a blocking cudaMalloc; make
+ * that first call before any stream capture).  Calls that share the library
+ * workspace must be ordered (same stream); use _ex for concurrent calls.
+ */
+int dq_linear_forward(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                      const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y, void* stream);
+
+/*
+ * As dq_linear_forward with a caller-owned device workspace of at least
+ * dq_workspace_bytes bytes, a stage mask (DQ_STAGE_*; stages read what
+ * earlier stages left in the same workspace), and optional timing events:
+ * stage_events NULL or an array of 4 cudaEvent_t (as void*) recorded before
+ * the first stage and after each of the three stages.
+ */
+int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                         const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y,
+                         void* workspace, size_t workspace_bytes, int stage_mask, void* const* stage_events,
+                         void* stream);
+
+/*
+ * As dq_linear_forward_ex with HOST X and Y (pinned for asynchronous copies):
+ * copies X to X_dev, runs the layer, copies Y_dev to Y, all on `stream`.
+ * X_dev (N x Ci BF16) and Y_dev (N x Co BF16) are caller-owned device buffers.
+ */
+int dq_linear_forward_host(const void* X_host, int T, int H, int W, int t, int h, int w, int Ci, int Co,
+                           int rank, const void* packed_W, const void* L1_mma, const void* L2_slab,
+                           void* Y_host, void* X_dev, void* Y_dev, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/*
+ * Synchronises `stream`, reads the workspace status word into *status, and
+ * clears it when `clear` is nonzero.  workspace NULL = the library workspace.
+ */
+int dq_read_device_status(const void* workspace, void* stream, int* status, int clear);
+
+/*
+ * Failure-detection self test: launches one kernel that waits on an mbarrier
+ * nothing arrives at, with a wait budget of budget_us microseconds.  It must
+ * come back with DQ_ERR_DEVICE_TIMEOUT in *status (and the context usable).
+ */
+int dq_selftest_bounded_wait(int budget_us, void* stream, int* status);
+
+/*
+ * Format self test: for each of the n fp32 values in `in` (device), writes the
+ * E2M1 code (low nibble, round to nearest even, saturating), the E4M3 code
+ * (same rules) and that E4M3 code's value, using the very conversions the
+ * quantisers use.  All buffers are device memory of n elements; asynchronous.
+ */
+int dq_selftest_convert(const float* in, long long n, uint8_t* e2m1, uint8_t* e4m3, float* e4m3_value,
+                        void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DELTAQUANT_H */

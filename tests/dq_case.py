@@ -1,0 +1,112 @@
+"""Shared helpers for the GPU parity tests: run one layer through the C ABI on
+the GPU, run the oracle on the same seeded inputs, and compare.
+
+Tolerance (bit-exact for every quantised tensor; Y per element within
+max(1 BF16 ulp of the reference, 1e-3 * RMS of the reference rows)) follows
+the parity bar stated for this layer: fp32 tensor-core accumulation and a
+BF16 output against an fp64 product of the same dequantised operands.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+import synth
+
+
+def sf_unpermute(buf: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """Scale-factor layout (include/deltaquant.h) -> plain rows x cols/16."""
+    r = np.arange(rows, dtype=np.int64)[:, None]
+    b = np.arange(cols // 16, dtype=np.int64)[None, :]
+    off = ((r // 128) * (cols // 64) + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + b % 4
+    return buf[off]
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def y_tolerance(y_ref: np.ndarray) -> np.ndarray:
+    rms = np.sqrt(np.mean(y_ref ** 2))
+    a = np.abs(y_ref)
+    ulp = np.where(a > 0, np.exp2(np.floor(np.log2(np.where(a > 0, a, 1.0))) - 7), 0.0)
+    return np.maximum(ulp, 1e-3 * rms)
+
+
+def assert_y_close(y_bits: np.ndarray, y_ref: np.ndarray, what: str = "Y") -> dict:
+    y = bf16_bits_to_f64(y_bits)
+    tol = y_tolerance(y_ref)
+    err = np.abs(y - y_ref)
+    bad = err > tol
+    info = dict(max_err_over_tol=float((err / tol).max()), n_bad=int(bad.sum()), n=int(err.size))
+    assert not bad.any(), f"{what}: {info}, first bad at {np.argwhere(bad)[:5].tolist()}"
+    return info
+
+
+class Case:
+    """One layer instance: workload, inputs, oracle factors."""
+
+    def __init__(self, wl: synth.Workload, cube=None, seed=None, tau: int = 0, X=None, Wb=None):
+        self.wl = wl
+        self.cube = tuple(cube or wl.cube)
+        self.X = synth.activations(wl, seed=seed, tau=tau) if X is None else X
+        self.Wb = synth.weight(wl, seed=seed) if Wb is None else Wb
+        self.L1, self.L2, _ = oracle.lowrank_factors(self.Wb, wl.rank)
+
+    # ---------------------------------------------------------------- GPU
+    def run_gpu(self, dq, torch, stage_mask=7, packed_override=None):
+        wl, (t, h, w) = self.wl, self.cube
+        packed, L1m, L2s, S_W = dq.dq_pack_weight_factors(self.Wb, self.L1, self.L2)
+        if packed_override is not None:
+            packed = packed_override(packed)
+        dev = torch.device("cuda")
+        Xd = torch.from_numpy(self.X.view(np.int16)).to(dev)
+        Pd = torch.from_numpy(packed).to(dev)
+        L1d = torch.from_numpy(L1m.view(np.int16)).to(dev)
+        L2d = torch.from_numpy(L2s.view(np.int16)).to(dev)
+        Yd = torch.empty((wl.N, wl.Co), dtype=torch.int16, device=dev)
+        lay = dq.dq_workspace_layout_get(wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank)
+        ws = torch.zeros(lay.total_bytes, dtype=torch.uint8, device=dev)
+        dq.dq_linear_forward_ex(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd, ws,
+                                lay.total_bytes, stage_mask, None, torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        status = dq.dq_read_device_status(ws, torch.cuda.current_stream(), clear=True)
+        wsh = ws.cpu().numpy()
+        N, K, Ci = lay.N, lay.K, wl.Ci
+        out = dict(status=status, layout=lay, S_W=S_W, packed=packed,
+                   Y=Yd.cpu().numpy().view(np.uint16),
+                   amax_delta=wsh[lay.off_scalars:lay.off_scalars + 4].view(np.float32)[0],
+                   S_delta=wsh[lay.off_scalars + 4:lay.off_scalars + 8].view(np.float32)[0],
+                   s8=wsh[lay.off_s8:lay.off_s8 + 4 * K].view(np.float32),
+                   q8=wsh[lay.off_q8:lay.off_q8 + K * Ci].reshape(K, Ci),
+                   q8_bf16=wsh[lay.off_q8_bf16:lay.off_q8_bf16 + 2 * K * Ci].view(np.uint16).reshape(K, Ci),
+                   dcodes=wsh[lay.off_dcodes:lay.off_dcodes + N * Ci // 2].reshape(N, Ci // 2),
+                   dscales=sf_unpermute(wsh[lay.off_dscales:], N, Ci),
+                   p=wsh[lay.off_p:lay.off_p + 4 * K * wl.Co].view(np.float32).reshape(K, wl.Co))
+        return out
+
+    # ---------------------------------------------------------------- oracle
+    def run_oracle(self):
+        wl = self.wl
+        act = oracle.quantize_activations(self.X, wl.T, wl.H, wl.W, self.cube)
+        wq = oracle.quantize_weight(self.Wb, self.L1, self.L2)
+        return act, wq
+
+    def oracle_rows(self, act, wq, rows):
+        return oracle.output_rows(act, wq, self.X, self.L1, self.L2, rows)
+
+
+def compare_quantised(g: dict, act: dict, wq: dict) -> None:
+    """Every quantised tensor bit-exact against the oracle."""
+    assert g["status"] == 0, g["status"]
+    assert np.float32(g["amax_delta"]) == np.float32(act["amax_delta"])
+    assert np.float32(g["S_delta"]) == np.float32(act["S_delta"])
+    assert np.float32(g["S_W"]) == np.float32(wq["S_w"])
+    assert np.array_equal(g["s8"], act["s8"]), "s8"
+    bad = np.argwhere(g["q8"] != act["q8"])
+    assert bad.size == 0, ("q8", bad[:5].tolist(), g["q8"][tuple(bad[0])], act["q8"][tuple(bad[0])])
+    assert np.array_equal(bf16_bits_to_f64(g["q8_bf16"]), oracle.e4m3_value(act["q8"])), "q8 as BF16"
+    bad = np.argwhere(g["dscales"] != act["dscales"])
+    assert bad.size == 0, ("delta scales", bad[:5].tolist())
+    bad = np.argwhere(g["dcodes"] != act["dcodes"])
+    assert bad.size == 0, ("delta codes", bad[:5].tolist(), g["dcodes"][tuple(bad[0])], act["dcodes"][tuple(bad[0])])

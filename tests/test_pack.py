@@ -1,0 +1,76 @@
+"""The library's offline weight packer (host C++) against the oracle.
+
+Given the same BF16 factors L1, L2 (taken from the oracle's own SVD), the
+residual codes, the group scales (through the scale-factor layout) and the
+per-tensor scale must be bit-exact; the BF16 dequantised weight must equal
+code * scale exactly.  The library's own randomised SVD is pinned by the
+Eckart-Young bound with singular values from the oracle."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+
+@pytest.fixture(scope="module")
+def dq():
+    from video_diffusion_w4a4_b200 import build
+    build.build()
+    import video_diffusion_w4a4_b200 as m
+    return m
+
+
+def _unpack_scales(dq, blob, off, rows, cols):
+    idx = np.array([[dq.dq_sf_offset(r, b, cols) for b in range(cols // 16)] for r in range(rows)])
+    return blob[off + idx]
+
+
+@pytest.mark.parametrize("shape", [(256, 256, 16), (512, 1024, 32), (1024, 512, 48)])
+def test_pack_bit_exact(dq, shape):
+    Co, Ci, r = shape
+    wl = synth.Workload("pack", 1, 1, 1, Ci, Co, r, (1, 1, 1), (1, 1, 1), (0.0, 1.0), (0.01, 20.0))
+    Wb = synth.weight(wl, seed=Co * 7 + Ci)
+    L1, L2, _ = oracle.lowrank_factors(Wb, r)
+    wq = oracle.quantize_weight(Wb, L1, L2)
+    packed, L1m, L2s, S_W = dq.dq_pack_weight_factors(Wb, L1, L2)
+    lay = dq.dq_packed_weight_layout(Co, Ci, r)
+    hdr = packed[:256].view(np.uint32)
+    assert hdr[0] == 0x31575144 and hdr[1] == 1
+    assert list(packed[8:24].view(np.int32)) == [Co, Ci, r, lay.slab]
+    assert packed[24:28].view(np.float32)[0] == np.float32(wq["S_w"]) == np.float32(S_W)
+    codes = packed[lay.off_codes:lay.off_codes + Co * Ci // 2].reshape(Co, Ci // 2)
+    assert np.array_equal(codes, wq["wcodes"])
+    assert np.array_equal(_unpack_scales(dq, packed, lay.off_scales, Co, Ci), wq["wscales"])
+    dqw = packed[lay.off_dqw:lay.off_dqw + Co * Ci * 2].view(np.uint16).reshape(Co, Ci)
+    q = np.empty((Co, Ci))
+    q[:, 0::2] = oracle.e2m1_value(wq["wcodes"] & 15)
+    q[:, 1::2] = oracle.e2m1_value(wq["wcodes"] >> 4)
+    want = q * np.repeat(oracle.e4m3_value(wq["wscales"]), 16, axis=1)
+    assert np.array_equal(oracle.bf16_value(dqw).astype(np.float64), want)
+    assert np.array_equal(L1m, L1.T)
+    assert np.array_equal(L2s[:, :r], L2.T) and np.array_equal(L2s[:, r:2 * r], L2.T)
+    assert not L2s[:, 2 * r:].any()
+
+
+@pytest.mark.parametrize("shape", [(256, 256, 16), (768, 1024, 32)])
+def test_library_svd_eckart_young(dq, shape):
+    Co, Ci, r = shape
+    wl = synth.Workload("svd", 1, 1, 1, Ci, Co, r, (1, 1, 1), (1, 1, 1), (0.0, 1.0), (0.01, 20.0))
+    Wb = synth.weight(wl, seed=99)
+    L1, L2 = dq.dq_lowrank_factors(Wb, r)
+    w = oracle.bf16_value(Wb).astype(np.float64)
+    sig = np.linalg.svd(w, compute_uv=False)
+    l1, l2 = oracle.bf16_value(L1).astype(np.float64), oracle.bf16_value(L2).astype(np.float64)
+    err2 = np.linalg.norm(w - (l1 @ l2).T) ** 2
+    tail = np.sum(sig[r:] ** 2)
+    rnd = (2.0 ** -8 * np.linalg.norm(l1 @ l2)) ** 2
+    assert err2 <= (1 + 1e-3) * tail + 4 * rnd, (err2, tail, rnd)
+
+
+def test_pack_weight_end_to_end_matches_factor_path(dq):
+    wl = synth.WORKLOADS["tiny"]
+    Wb = synth.weight(wl)
+    packed, L1m, L2s = dq.dq_pack_weight(Wb, wl.rank)
+    L1, L2 = dq.dq_lowrank_factors(Wb, wl.rank, seed=0)
+    p2, L1m2, L2s2, _ = dq.dq_pack_weight_factors(Wb, L1, L2)
+    assert np.array_equal(packed, p2) and np.array_equal(L1m, L1m2) and np.array_equal(L2s, L2s2)

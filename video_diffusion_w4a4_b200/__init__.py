@@ -1,0 +1,264 @@
+"""Python binding of libdeltaquant (the C ABI in include/deltaquant.h).
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels (or, for the offline packer, its C++ host code).  Device
+buffers are passed as torch tensors (their data_ptr) or raw integer
+addresses; streams as torch.cuda.Stream or raw cudaStream_t integers.  The
+functions keep the C names.  If the shared library is missing this module
+raises ImportError: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdeltaquant.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python video_diffusion_w4a4_b200/build.py` "
+                      "(or __graft_entry__.build())")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+DQ_OK = 0
+DQ_ERR_INVALID_ARG = 1
+DQ_ERR_UNSUPPORTED_SHAPE = 2
+DQ_ERR_ALIGNMENT = 3
+DQ_ERR_WORKSPACE_TOO_SMALL = 4
+DQ_ERR_CUDA = 5
+DQ_ERR_DEVICE_TIMEOUT = 6
+DQ_ERR_BAD_PACKED_WEIGHT = 7
+DQ_ERR_NO_DEVICE = 8
+DQ_ERR_ALLOC = 9
+DQ_STAGE_QUANTIZE, DQ_STAGE_KERNEL_GEMM, DQ_STAGE_MAIN_GEMM, DQ_STAGE_ALL = 1, 2, 4, 7
+
+
+class dq_packed_layout(ctypes.Structure):
+    _fields_ = [("total_bytes", ctypes.c_size_t), ("off_codes", ctypes.c_size_t), ("off_scales", ctypes.c_size_t),
+                ("off_dqw", ctypes.c_size_t), ("Co", ctypes.c_int), ("Ci", ctypes.c_int), ("rank", ctypes.c_int),
+                ("slab", ctypes.c_int)]
+
+
+class dq_workspace_layout(ctypes.Structure):
+    _fields_ = [("total_bytes", ctypes.c_size_t)] + [
+        (n, ctypes.c_size_t) for n in ("off_status", "off_scalars", "off_kamax", "off_s8", "off_q8", "off_q8_bf16",
+                                       "off_dcodes", "off_dscales", "off_u_part", "off_u_hilo", "off_p")] + [
+        ("N", ctypes.c_longlong), ("K", ctypes.c_longlong), ("N_pad", ctypes.c_longlong), ("K_pad", ctypes.c_longlong),
+        ("splits", ctypes.c_int), ("slab", ctypes.c_int)]
+
+
+_P, _I, _SZ, _LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
+_SIGS = {
+    "dq_status_string": ([_I], ctypes.c_char_p),
+    "dq_abi_version": ([], _I),
+    "dq_cube_count": ([_I] * 6 + [ctypes.POINTER(_LL)], _I),
+    "dq_cube_major_row": ([_I] * 6 + [_LL, ctypes.POINTER(_LL), ctypes.POINTER(_LL)], _I),
+    "dq_sf_offset": ([_LL, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "dq_sf_bytes": ([_LL, _I, ctypes.POINTER(_SZ)], _I),
+    "dq_packed_weight_layout": ([_I, _I, _I, ctypes.POINTER(dq_packed_layout)], _I),
+    "dq_packed_weight_bytes": ([_I, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "dq_lowrank_slab_width": ([_I], _I),
+    "dq_lowrank_factors": ([_P, _I, _I, _I, ctypes.c_uint64, _P, _P], _I),
+    "dq_pack_weight_factors": ([_P, _P, _P, _I, _I, _I, _P, _SZ, _P, _P, ctypes.POINTER(ctypes.c_float)], _I),
+    "dq_pack_weight": ([_P, _I, _I, _I, _P, _SZ, _P, _P], _I),
+    "dq_workspace_layout_get": ([_I] * 9 + [ctypes.POINTER(dq_workspace_layout)], _I),
+    "dq_workspace_bytes": ([_I] * 9 + [ctypes.POINTER(_SZ)], _I),
+    "dq_linear_forward": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P], _I),
+    "dq_linear_forward_ex": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P, _SZ, _I, _P, _P], _I),
+    "dq_linear_forward_host": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
+    "dq_read_device_status": ([_P, _P, ctypes.POINTER(_I), _I], _I),
+    "dq_selftest_bounded_wait": ([_I, _P, ctypes.POINTER(_I)], _I),
+    "dq_selftest_convert": ([_P, _LL, _P, _P, _P, _P], _I),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+
+class DQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {dq_status_string(status)} ({status})")
+        self.status = status
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != DQ_OK:
+        raise DQError(fn, rc)
+
+
+def _ptr(x) -> int | None:
+    """Device/host address of a torch tensor, numpy array or raw int."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if isinstance(x, np.ndarray):
+        return x.ctypes.data
+    return x.data_ptr()
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+# ------------------------------------------------------------------ layout maps
+
+def dq_status_string(status: int) -> str:
+    return _lib.dq_status_string(status).decode()
+
+
+def dq_abi_version() -> int:
+    return _lib.dq_abi_version()
+
+
+def dq_cube_count(T, H, W, t, h, w) -> int:
+    K = ctypes.c_longlong()
+    _check("dq_cube_count", _lib.dq_cube_count(T, H, W, t, h, w, ctypes.byref(K)))
+    return K.value
+
+
+def dq_cube_major_row(T, H, W, t, h, w, n) -> tuple[int, int]:
+    row, cube = ctypes.c_longlong(), ctypes.c_longlong()
+    _check("dq_cube_major_row", _lib.dq_cube_major_row(T, H, W, t, h, w, n, ctypes.byref(row), ctypes.byref(cube)))
+    return row.value, cube.value
+
+
+def dq_sf_offset(row: int, block: int, cols: int) -> int:
+    off = ctypes.c_size_t()
+    _check("dq_sf_offset", _lib.dq_sf_offset(row, block, cols, ctypes.byref(off)))
+    return off.value
+
+
+def dq_sf_bytes(rows: int, cols: int) -> int:
+    b = ctypes.c_size_t()
+    _check("dq_sf_bytes", _lib.dq_sf_bytes(rows, cols, ctypes.byref(b)))
+    return b.value
+
+
+def dq_lowrank_slab_width(rank: int) -> int:
+    return _lib.dq_lowrank_slab_width(rank)
+
+
+def dq_packed_weight_layout(Co, Ci, rank) -> dq_packed_layout:
+    L = dq_packed_layout()
+    _check("dq_packed_weight_layout", _lib.dq_packed_weight_layout(Co, Ci, rank, ctypes.byref(L)))
+    return L
+
+
+def dq_packed_weight_bytes(Co, Ci, rank) -> int:
+    b = ctypes.c_size_t()
+    _check("dq_packed_weight_bytes", _lib.dq_packed_weight_bytes(Co, Ci, rank, ctypes.byref(b)))
+    return b.value
+
+
+# ------------------------------------------------------------------ offline packing (host arrays)
+
+def dq_lowrank_factors(W: np.ndarray, rank: int, seed: int = 0):
+    """W: uint16 BF16 bits (Co, Ci).  Returns (L1 (Ci, r), L2 (r, Co)) as BF16 bits."""
+    W = np.ascontiguousarray(W, dtype=np.uint16)
+    Co, Ci = W.shape
+    L1 = np.empty((Ci, rank), np.uint16)
+    L2 = np.empty((rank, Co), np.uint16)
+    _check("dq_lowrank_factors", _lib.dq_lowrank_factors(W.ctypes.data, Co, Ci, rank, seed, L1.ctypes.data,
+                                                         L2.ctypes.data))
+    return L1, L2
+
+
+def dq_pack_weight_factors(W: np.ndarray, L1: np.ndarray, L2: np.ndarray):
+    """Returns (packed blob uint8, L1_mma (r, Ci) BF16 bits, L2_slab (Co, slab) BF16 bits, S_W)."""
+    W = np.ascontiguousarray(W, dtype=np.uint16)
+    L1 = np.ascontiguousarray(L1, dtype=np.uint16)
+    L2 = np.ascontiguousarray(L2, dtype=np.uint16)
+    Co, Ci = W.shape
+    r = L1.shape[1]
+    lay = dq_packed_weight_layout(Co, Ci, r)
+    packed = np.empty(lay.total_bytes, np.uint8)
+    L1m = np.empty((r, Ci), np.uint16)
+    L2s = np.empty((Co, lay.slab), np.uint16)
+    S = ctypes.c_float()
+    _check("dq_pack_weight_factors",
+           _lib.dq_pack_weight_factors(W.ctypes.data, L1.ctypes.data, L2.ctypes.data, Co, Ci, r, packed.ctypes.data,
+                                       packed.size, L1m.ctypes.data, L2s.ctypes.data, ctypes.byref(S)))
+    return packed, L1m, L2s, S.value
+
+
+def dq_pack_weight(W: np.ndarray, rank: int):
+    """SVD factors (seed 0) + packing.  Returns (packed, L1_mma, L2_slab)."""
+    W = np.ascontiguousarray(W, dtype=np.uint16)
+    Co, Ci = W.shape
+    lay = dq_packed_weight_layout(Co, Ci, rank)
+    packed = np.empty(lay.total_bytes, np.uint8)
+    L1m = np.empty((rank, Ci), np.uint16)
+    L2s = np.empty((Co, lay.slab), np.uint16)
+    _check("dq_pack_weight", _lib.dq_pack_weight(W.ctypes.data, Co, Ci, rank, packed.ctypes.data, packed.size,
+                                                 L1m.ctypes.data, L2s.ctypes.data))
+    return packed, L1m, L2s
+
+
+# ------------------------------------------------------------------ online (device)
+
+def dq_workspace_layout_get(T, H, W, t, h, w, Ci, Co, rank) -> dq_workspace_layout:
+    L = dq_workspace_layout()
+    _check("dq_workspace_layout_get", _lib.dq_workspace_layout_get(T, H, W, t, h, w, Ci, Co, rank, ctypes.byref(L)))
+    return L
+
+
+def dq_workspace_bytes(T, H, W, t, h, w, Ci, Co, rank) -> int:
+    b = ctypes.c_size_t()
+    _check("dq_workspace_bytes", _lib.dq_workspace_bytes(T, H, W, t, h, w, Ci, Co, rank, ctypes.byref(b)))
+    return b.value
+
+
+def dq_linear_forward(X, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y, stream=None) -> None:
+    _check("dq_linear_forward", _lib.dq_linear_forward(_ptr(X), T, H, W, t, h, w, Ci, Co, rank, _ptr(packed_W),
+                                                       _ptr(L1_mma), _ptr(L2_slab), _ptr(Y), _stream(stream)))
+
+
+def dq_linear_forward_ex(X, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y, workspace,
+                         workspace_bytes, stage_mask=DQ_STAGE_ALL, stage_events=None, stream=None) -> None:
+    ev = None
+    if stage_events is not None:
+        arr = (ctypes.c_void_p * 4)(*[e.cuda_event if hasattr(e, "cuda_event") else e for e in stage_events])
+        ev = ctypes.cast(arr, ctypes.c_void_p)
+    _check("dq_linear_forward_ex",
+           _lib.dq_linear_forward_ex(_ptr(X), T, H, W, t, h, w, Ci, Co, rank, _ptr(packed_W), _ptr(L1_mma),
+                                     _ptr(L2_slab), _ptr(Y), _ptr(workspace), workspace_bytes, stage_mask, ev,
+                                     _stream(stream)))
+
+
+def dq_linear_forward_host(X_host, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y_host, X_dev, Y_dev,
+                           workspace, workspace_bytes, stream=None) -> None:
+    _check("dq_linear_forward_host",
+           _lib.dq_linear_forward_host(_ptr(X_host), T, H, W, t, h, w, Ci, Co, rank, _ptr(packed_W), _ptr(L1_mma),
+                                       _ptr(L2_slab), _ptr(Y_host), _ptr(X_dev), _ptr(Y_dev), _ptr(workspace),
+                                       workspace_bytes, _stream(stream)))
+
+
+def dq_read_device_status(workspace=None, stream=None, clear: bool = False) -> int:
+    s = ctypes.c_int()
+    _check("dq_read_device_status",
+           _lib.dq_read_device_status(_ptr(workspace), _stream(stream), ctypes.byref(s), int(clear)))
+    return s.value
+
+
+def dq_selftest_bounded_wait(budget_us: int, stream=None) -> int:
+    s = ctypes.c_int()
+    _check("dq_selftest_bounded_wait", _lib.dq_selftest_bounded_wait(budget_us, _stream(stream), ctypes.byref(s)))
+    return s.value
+
+
+def dq_selftest_convert(inp, n, e2m1, e4m3, e4m3_value, stream=None) -> None:
+    _check("dq_selftest_convert", _lib.dq_selftest_convert(_ptr(inp), n, _ptr(e2m1), _ptr(e4m3), _ptr(e4m3_value),
+                                                           _stream(stream)))
+
+
+def loaded_library_path() -> str:
+    return LIB_PATH

@@ -1,0 +1,332 @@
+// Online entry points of libdeltaquant: argument checks, workspace carve-up,
+// TMA tensor maps, and the launch sequence of the DeltaQuant layer
+//   a1 cube statistics -> a2 cube encode -> (c) kernel-token product ->
+//   (b) main FP4 product with low-rank slab and scatter epilogue.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <map>
+#include <mutex>
+
+#include "../../include/deltaquant.h"
+#include "dq_common.h"
+#include "dq_internal.h"
+
+namespace {
+
+using dq::Geom;
+
+constexpr uint64_t kWaitBudgetNs = 2000000000ull;  // 2 s per wait: far above any legitimate wait
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D map over a row-major matrix: inner = elements per row, outer = rows.
+bool map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t inner, uint64_t outer,
+            uint32_t box_inner, uint32_t box_outer) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * (uint64_t)esize};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return f(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 4-D map over X viewed as T x H x W x Ci (BF16), boxes of 64 channels x bw x bh x bt tokens.
+bool map_x(CUtensorMap* m, const void* X, const Geom& g, int Ci, int bw, int bh, int bt) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)Ci, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.T};
+    cuuint64_t strides[3] = {(cuuint64_t)Ci * 2, (cuuint64_t)g.W * Ci * 2, (cuuint64_t)g.H * g.W * Ci * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)bw, (cuuint32_t)bh, (cuuint32_t)bt};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(X), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p) { return ((uintptr_t)p & 255u) == 0; }
+
+int check_shape(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank) {
+    if (T <= 0 || H <= 0 || W <= 0 || t <= 0 || h <= 0 || w <= 0) return DQ_ERR_INVALID_ARG;
+    if (t > T || h > H || w > W) return DQ_ERR_UNSUPPORTED_SHAPE;
+    if (t * h * w > 128) return DQ_ERR_UNSUPPORTED_SHAPE;
+    if (Ci < 256 || Co < 256 || Ci % 256 || Co % 256) return DQ_ERR_UNSUPPORTED_SHAPE;
+    if (rank < 16 || rank > 128 || rank % 16 || rank > Ci || rank > Co) return DQ_ERR_UNSUPPORTED_SHAPE;
+    if ((long long)T * H * W >= (1ll << 31)) return DQ_ERR_UNSUPPORTED_SHAPE;
+    return DQ_OK;
+}
+
+struct LibWorkspace {
+    void* ptr = nullptr;
+    size_t bytes = 0;
+};
+std::mutex g_ws_mu;
+std::map<int, LibWorkspace> g_ws;
+
+int ensure_lib_workspace(size_t need, void** ws) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DQ_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    LibWorkspace& L = g_ws[dev];
+    if (L.bytes < need) {
+        if (L.ptr) {
+            cudaDeviceSynchronize();
+            cudaFree(L.ptr);
+            L.ptr = nullptr;
+            L.bytes = 0;
+        }
+        if (cudaMalloc(&L.ptr, need) != cudaSuccess) {
+            L.ptr = nullptr;
+            return DQ_ERR_ALLOC;
+        }
+        cudaMemset(L.ptr, 0, 256);
+        L.bytes = need;
+    }
+    *ws = L.ptr;
+    return DQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dq_workspace_layout_get(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                            dq_workspace_layout* out) {
+    if (!out) return DQ_ERR_INVALID_ARG;
+    int rc = check_shape(T, H, W, t, h, w, Ci, Co, rank);
+    if (rc) return rc;
+    dq::WsLayout L = dq::ws_layout(dq::make_geom(T, H, W, t, h, w), Ci, Co, rank);
+    out->total_bytes = L.total;
+    out->off_status = L.off_status;
+    out->off_scalars = L.off_scalars;
+    out->off_kamax = L.off_kamax;
+    out->off_s8 = L.off_s8;
+    out->off_q8 = L.off_q8;
+    out->off_q8_bf16 = L.off_q8_bf16;
+    out->off_dcodes = L.off_dcodes;
+    out->off_dscales = L.off_dscales;
+    out->off_u_part = L.off_u_part;
+    out->off_u_hilo = L.off_u_hilo;
+    out->off_p = L.off_p;
+    out->N = L.N;
+    out->K = L.K;
+    out->N_pad = L.N_pad;
+    out->K_pad = L.K_pad;
+    out->splits = L.splits;
+    out->slab = L.slab;
+    return DQ_OK;
+}
+
+int dq_workspace_bytes(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank, size_t* bytes) {
+    if (!bytes) return DQ_ERR_INVALID_ARG;
+    dq_workspace_layout L;
+    int rc = dq_workspace_layout_get(T, H, W, t, h, w, Ci, Co, rank, &L);
+    if (rc) return rc;
+    *bytes = L.total_bytes;
+    return DQ_OK;
+}
+
+int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                         const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y, void* workspace,
+                         size_t workspace_bytes, int stage_mask, void* const* stage_events, void* stream) {
+    int rc = check_shape(T, H, W, t, h, w, Ci, Co, rank);
+    if (rc) return rc;
+    if (!X || !packed_W || !L1_mma || !L2_slab || !Y || !workspace) return DQ_ERR_INVALID_ARG;
+    if (stage_mask <= 0 || stage_mask > DQ_STAGE_ALL) return DQ_ERR_INVALID_ARG;
+    if (!aligned(X) || !aligned(packed_W) || !aligned(L1_mma) || !aligned(L2_slab) || !aligned(Y) ||
+        !aligned(workspace))
+        return DQ_ERR_ALIGNMENT;
+    const Geom g = dq::make_geom(T, H, W, t, h, w);
+    const dq::WsLayout wl = dq::ws_layout(g, Ci, Co, rank);
+    if (workspace_bytes < wl.total) return DQ_ERR_WORKSPACE_TOO_SMALL;
+    if (!encode_fn()) return DQ_ERR_NO_DEVICE;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t* ws = (uint8_t*)workspace;
+    const dq::PackedLayout pl = dq::packed_layout(Co, Ci, rank);
+    const uint8_t* pw = (const uint8_t*)packed_W;
+
+    dq::QuantParams qp;
+    memset(&qp, 0, sizeof(qp));
+    qp.g = g;
+    qp.Ci = Ci;
+    qp.rank = rank;
+    qp.slab = wl.slab;
+    qp.splits = wl.splits;
+    qp.chunks_per_split = Ci / 64 / wl.splits;
+    qp.nw = dq::imin(128 / (t * h * w), g.KW);
+    qp.bt = t;
+    qp.bh = h;
+    qp.bw = qp.nw * w;
+    qp.nbw = (int)dq::cdiv(g.KW, qp.nw);
+    qp.n_boxes = g.KT * g.KH * qp.nbw;
+    qp.status = (int*)(ws + wl.off_status);
+    qp.scalars = (uint32_t*)(ws + wl.off_scalars);
+    qp.kamax = (uint32_t*)(ws + wl.off_kamax);
+    qp.s8 = (float*)(ws + wl.off_s8);
+    qp.q8 = ws + wl.off_q8;
+    qp.q8_bf16 = (uint16_t*)(ws + wl.off_q8_bf16);
+    qp.dcodes = ws + wl.off_dcodes;
+    qp.dscales = ws + wl.off_dscales;
+    qp.u_part = (float*)(ws + wl.off_u_part);
+    qp.u_hilo = (uint16_t*)(ws + wl.off_u_hilo);
+    qp.packed_w = pw;
+    qp.budget_ns = kWaitBudgetNs;
+
+    dq::GemmParams gp;
+    memset(&gp, 0, sizeof(gp));
+    gp.g = g;
+    gp.Nout = Co;
+    gp.Ci = Ci;
+    gp.scalars = qp.scalars;
+    gp.packed_w = pw;
+    gp.status = qp.status;
+    gp.budget_ns = kWaitBudgetNs;
+
+    auto rec = [&](int i) {
+        if (stage_events && stage_events[i]) cudaEventRecord((cudaEvent_t)stage_events[i], st);
+    };
+    rec(0);
+    if (stage_mask & DQ_STAGE_QUANTIZE) {
+        CUtensorMap tm_x, tm_l1;
+        if (!map_x(&tm_x, X, g, Ci, qp.bw, qp.bh, qp.bt)) return DQ_ERR_CUDA;
+        if (!map_2d(&tm_l1, L1_mma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, rank, 64, rank)) return DQ_ERR_CUDA;
+        if (cudaMemsetAsync(ws + wl.off_scalars, 0, 16, st) != cudaSuccess) return DQ_ERR_CUDA;
+        if (cudaMemsetAsync(ws + wl.off_kamax, 0, (size_t)g.K * 4, st) != cudaSuccess) return DQ_ERR_CUDA;
+        if (dq::launch_cube_stats(tm_x, tm_l1, qp, st) != cudaSuccess) return DQ_ERR_CUDA;
+        if (dq::launch_cube_encode(tm_x, qp, st) != cudaSuccess) return DQ_ERR_CUDA;
+    }
+    rec(1);
+    if (stage_mask & DQ_STAGE_KERNEL_GEMM) {
+        CUtensorMap tm_a, tm_b;
+        if (!map_2d(&tm_a, ws + wl.off_q8_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, g.K, 64, 128))
+            return DQ_ERR_CUDA;
+        if (!map_2d(&tm_b, pw + pl.off_dqw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, Co, 64, 256)) return DQ_ERR_CUDA;
+        dq::GemmParams p = gp;
+        p.M = (int)g.K;
+        p.k_stages = Ci / 64;
+        p.s8 = qp.s8;
+        p.pout = (float*)(ws + wl.off_p);
+        if (dq::launch_kernel_gemm(tm_a, tm_b, p, st) != cudaSuccess) return DQ_ERR_CUDA;
+    }
+    rec(2);
+    if (stage_mask & DQ_STAGE_MAIN_GEMM) {
+        CUtensorMap tm_a, tm_b, tm_sa, tm_sb;
+        if (!map_2d(&tm_a, ws + wl.off_dcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Ci / 2, g.N, 128, 128))
+            return DQ_ERR_CUDA;
+        if (!map_2d(&tm_b, pw + pl.off_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Ci / 2, Co, 128, 256))
+            return DQ_ERR_CUDA;
+        if (!map_2d(&tm_sa, ws + wl.off_u_hilo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wl.slab, g.N, 64, 128))
+            return DQ_ERR_CUDA;
+        if (!map_2d(&tm_sb, L2_slab, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wl.slab, Co, 64, 256)) return DQ_ERR_CUDA;
+        dq::GemmParams p = gp;
+        p.M = (int)g.N;
+        p.k_stages = Ci / 256;
+        p.slab_stages = wl.slab / 64;
+        p.sfa = ws + wl.off_dscales;
+        p.sfb = pw + pl.off_scales;
+        p.p = (const float*)(ws + wl.off_p);
+        p.Y = (uint16_t*)Y;
+        if (dq::launch_main_gemm(tm_a, tm_b, tm_sa, tm_sb, p, st) != cudaSuccess) return DQ_ERR_CUDA;
+    }
+    rec(3);
+    return DQ_OK;
+}
+
+int dq_linear_forward(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                      const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y, void* stream) {
+    size_t need = 0;
+    int rc = dq_workspace_bytes(T, H, W, t, h, w, Ci, Co, rank, &need);
+    if (rc) return rc;
+    void* ws = nullptr;
+    rc = ensure_lib_workspace(need, &ws);
+    if (rc) return rc;
+    return dq_linear_forward_ex(X, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y, ws, need,
+                                DQ_STAGE_ALL, nullptr, stream);
+}
+
+int dq_linear_forward_host(const void* X_host, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                           const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y_host, void* X_dev,
+                           void* Y_dev, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_shape(T, H, W, t, h, w, Ci, Co, rank);
+    if (rc) return rc;
+    if (!X_host || !Y_host || !X_dev || !Y_dev) return DQ_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    size_t N = (size_t)T * H * W;
+    if (cudaMemcpyAsync(X_dev, X_host, N * Ci * 2, cudaMemcpyHostToDevice, st) != cudaSuccess) return DQ_ERR_CUDA;
+    rc = dq_linear_forward_ex(X_dev, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y_dev, workspace,
+                              workspace_bytes, DQ_STAGE_ALL, nullptr, stream);
+    if (rc) return rc;
+    if (cudaMemcpyAsync(Y_host, Y_dev, N * Co * 2, cudaMemcpyDeviceToHost, st) != cudaSuccess) return DQ_ERR_CUDA;
+    return DQ_OK;
+}
+
+int dq_read_device_status(const void* workspace, void* stream, int* status, int clear) {
+    if (!status) return DQ_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    const void* ws = workspace;
+    if (!ws) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return DQ_ERR_NO_DEVICE;
+        std::lock_guard<std::mutex> lk(g_ws_mu);
+        auto it = g_ws.find(dev);
+        if (it == g_ws.end() || !it->second.ptr) {
+            *status = DQ_OK;
+            return DQ_OK;
+        }
+        ws = it->second.ptr;
+    }
+    int h = 0;
+    if (cudaMemcpyAsync(&h, ws, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return DQ_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DQ_ERR_CUDA;
+    if (clear) {
+        if (cudaMemsetAsync(const_cast<void*>(ws), 0, sizeof(int), st) != cudaSuccess) return DQ_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return DQ_ERR_CUDA;
+    }
+    *status = h;
+    return DQ_OK;
+}
+
+int dq_selftest_bounded_wait(int budget_us, void* stream, int* status) {
+    if (!status || budget_us <= 0) return DQ_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    int* d = nullptr;
+    if (cudaMalloc(&d, sizeof(int)) != cudaSuccess) return DQ_ERR_ALLOC;
+    int rc = DQ_OK;
+    if (cudaMemsetAsync(d, 0, sizeof(int), st) != cudaSuccess ||
+        dq::launch_selftest_wait(d, (uint64_t)budget_us * 1000ull, st) != cudaSuccess ||
+        cudaMemcpyAsync(status, d, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        rc = DQ_ERR_CUDA;
+    cudaFree(d);
+    return rc;
+}
+
+int dq_selftest_convert(const float* in, long long n, uint8_t* e2m1, uint8_t* e4m3, float* e4m3_value,
+                        void* stream) {
+    if (n < 0 || (n > 0 && (!in || !e2m1 || !e4m3 || !e4m3_value))) return DQ_ERR_INVALID_ARG;
+    if (dq::launch_selftest_convert(in, n, e2m1, e4m3, e4m3_value, (cudaStream_t)stream) != cudaSuccess)
+        return DQ_ERR_CUDA;
+    return DQ_OK;
+}
+
+}  // extern "C"

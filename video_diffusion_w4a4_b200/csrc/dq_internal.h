@@ -1,0 +1,67 @@
+// Kernel parameter blocks and launchers shared between the C-ABI layer
+// (dq_api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dq_common.h"
+
+namespace dq {
+
+struct QuantParams {
+    Geom g;
+    int Ci, rank, slab, splits, chunks_per_split;
+    int nw;             // whole cubes per box along w
+    int bt, bh, bw;     // box extent in tokens: t x h x (nw w)
+    int nbw;            // boxes along w
+    int n_boxes;
+    int* status;
+    uint32_t* scalars;  // [0] bits of max|delta|, [1] S_delta
+    uint32_t* kamax;
+    float* s8;
+    uint8_t* q8;
+    uint16_t* q8_bf16;
+    uint8_t* dcodes;
+    uint8_t* dscales;
+    float* u_part;
+    uint16_t* u_hilo;
+    const uint8_t* packed_w;
+    uint64_t budget_ns;
+};
+
+struct GemmParams {
+    Geom g;
+    int M;               // valid rows of A
+    int Nout;            // output columns (Co)
+    int Ci;
+    int k_stages;        // main-operand K stages
+    int slab_stages;     // extra BF16 K stages (low-rank slab), main product only
+    const uint8_t* sfa;  // delta scales (scale-factor layout, M rows)
+    const uint8_t* sfb;  // weight scales (scale-factor layout, Co rows)
+    const float* p;      // per-cube kernel term, K x Co fp32 (main product)
+    const uint32_t* scalars;
+    const uint8_t* packed_w;
+    const float* s8;     // kernel-token scales (kernel-token product)
+    float* pout;         // kernel-token product output, K x Co fp32
+    uint16_t* Y;         // main product output, N x Co BF16 (t,h,w) order
+    int* status;
+    uint64_t budget_ns;
+};
+
+size_t quant_smem_bytes(int nw, int rank, bool stats);
+cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
+                              cudaStream_t st);
+cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const QuantParams& p, cudaStream_t st);
+
+cudaError_t launch_kernel_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmParams& p,
+                               cudaStream_t st);
+cudaError_t launch_main_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_sa,
+                             const CUtensorMap& tm_sb, const GemmParams& p, cudaStream_t st);
+
+cudaError_t launch_selftest_wait(int* status, uint64_t budget_ns, cudaStream_t st);
+cudaError_t launch_selftest_convert(const float* in, long long n, uint8_t* e2m1, uint8_t* e4m3, float* back,
+                                    cudaStream_t st);
+
+}  // namespace dq
