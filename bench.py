@@ -198,7 +198,9 @@ def main():
     ap.add_argument("--impl", default="dq", choices=["dq", "reference"])
     ap.add_argument("--workload", default="wan480p_proj", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--cube", default=None, help="override the cube, e.g. 2,2,2")
-    ap.add_argument("--sample-tokens", type=int, default=256, help="oracle sample size (tokens)")
+    ap.add_argument("--frames", type=int, default=None, help="override T (smaller cases for profiling)")
+    ap.add_argument("--sample-tokens", type=int, default=256, help="oracle sample size per reference step (tokens)")
+    ap.add_argument("--baseline-tokens", type=int, default=2048, help="oracle sample size of the cpu_baseline leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     args = ap.parse_args()
@@ -207,6 +209,10 @@ def main():
     wl = synth.WORKLOADS[args.workload]
     cube = parse_cube(args.cube) or wl.cube
     wl = wl.with_cube(cube)
+    if args.frames:
+        wl = synth.Workload(wl.name if args.frames == wl.T else f"{wl.name}_T{args.frames}", args.frames, wl.H, wl.W,
+                            wl.Ci, wl.Co, wl.rank, cube, (args.frames,) + tuple(wl.grid[1:]), wl.x_outliers,
+                            wl.w_outliers, wl.gelu)
     if args.impl == "reference":
         return run_reference(args, wl, cube)
 
@@ -254,6 +260,9 @@ def main():
         raise RuntimeError(f"device status after warm-up: {dq.dq_status_string(status)}")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for row in evs:          # torch creates CUDA events lazily; create them before handing them to the library
+        for e in row:
+            e.record(st)
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -353,7 +362,7 @@ def main():
         oracle.build()
         L1, L2 = dq.dq_lowrank_factors(Wb, wl.rank)
         wq = oracle.quantize_weight(Wb, L1, L2)
-        dt, f, n = oracle_sample(wl, cube, X, Wb, L1, L2, wq, args.sample_tokens)
+        dt, f, n = oracle_sample(wl, cube, X, Wb, L1, L2, wq, args.baseline_tokens)
         line["cpu_baseline"] = dict(value=f / dt / 1e12, unit="TFLOP/s", cores=os.cpu_count(), kind="oracle",
                                     sample=f"{n} tokens of {wl.name} (whole cube rows, frame slab 0), "
                                            f"Ci={wl.Ci}, Co={wl.Co}, r={wl.rank}, {dt:.1f} s")

@@ -1,0 +1,93 @@
+"""GPU parity at the full Wan-like sizes, in the launch configuration the bench
+times.  Every quantised tensor (delta codes and scales, S_delta, kernel
+tokens and their scales, weight codes and scales, S_W) is compared in full
+and bit-exact; Y is compared on the rows of sampled cubes (random interior
+cubes plus the first, last and ragged-edge cubes), which the oracle computes
+one by one in fp64.
+
+The cube-size sweep on the 480p shape also records the relative Frobenius
+error of Y against the unquantised product X W^T, next to plain per-token
+NVFP4 (no kernel/delta split), and checks the method's claim that the split
+lowers it (DeltaQuant note, key design 2 and the cube-size ablation)."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from dq_case import Case, assert_y_close, bf16_bits_to_f64, compare_quantised
+
+pytestmark = pytest.mark.gpu
+
+OUT = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "gpurun_out")
+
+
+@pytest.fixture(scope="module")
+def env():
+    import torch
+    assert torch.cuda.is_available(), "the GPU tests need a CUDA device"
+    import video_diffusion_w4a4_b200 as dq
+    return dq, torch
+
+
+def sample_rows(wl, cube, n_cubes=48, seed=0):
+    o = oracle.cube_order(wl.T, wl.H, wl.W, *cube)
+    K = o["count"].size
+    rng = np.random.default_rng(seed)
+    ks = set(rng.choice(K, size=min(n_cubes, K), replace=False).tolist())
+    ks |= {0, K - 1}
+    ks |= set(np.flatnonzero(o["count"] < o["count"].max())[:8].tolist())   # ragged edge cubes
+    rows = np.concatenate([o["n_of_row"][o["first"][k]:o["first"][k] + o["count"][k]] for k in sorted(ks)])
+    return np.sort(rows)
+
+
+def _record(name, info):
+    os.makedirs(OUT, exist_ok=True)
+    with open(os.path.join(OUT, f"parity_{name}.json"), "w") as f:
+        json.dump(info, f, indent=1)
+
+
+@pytest.mark.parametrize("name", ["wan480p_proj", "wan720p_ffn_up", "wan720p_ffn_down"])
+def test_full_size(env, name):
+    dq, torch = env
+    wl = synth.WORKLOADS[name]
+    case = Case(wl)
+    g = case.run_gpu(dq, torch)
+    act, wq = case.run_oracle()
+    compare_quantised(g, act, wq)
+    lay = dq.dq_packed_weight_layout(wl.Co, wl.Ci, wl.rank)
+    codes = g["packed"][lay.off_codes:lay.off_codes + wl.Co * wl.Ci // 2].reshape(wl.Co, wl.Ci // 2)
+    assert np.array_equal(codes, wq["wcodes"])
+    rows = sample_rows(wl, case.cube)
+    info = assert_y_close(g["Y"][rows], case.oracle_rows(act, wq, rows))
+    info.update(rows=int(rows.size), N=wl.N, K=int(g["layout"].K))
+    _record(name, info)
+
+
+@pytest.mark.parametrize("cube", [(1, 1, 1), (1, 2, 2), (2, 2, 2), (2, 4, 4)])
+def test_cube_sweep(env, cube):
+    dq, torch = env
+    wl = synth.WORKLOADS["wan480p_cube_sweep"].with_cube(cube)
+    case = Case(wl)
+    g = case.run_gpu(dq, torch)
+    act, wq = case.run_oracle()
+    compare_quantised(g, act, wq)
+    rows = sample_rows(wl, cube, n_cubes=32)
+    y_ref = case.oracle_rows(act, wq, rows)
+    info = assert_y_close(g["Y"][rows], y_ref)
+    # error against the unquantised product, next to plain per-token NVFP4
+    x = oracle.bf16_value(case.X[rows]).astype(np.float64)
+    w = oracle.bf16_value(case.Wb).astype(np.float64)
+    exact = x @ w.T
+    plain = oracle.quantize_plain(case.X[rows])
+    plain.update(row_of_n=None, cube_of_n=None, q8=None, s8=None)
+    y_plain = oracle.output_rows(plain, wq, case.X[rows], case.L1, case.L2, np.arange(rows.size), kernel=False,
+                                 cube_major=False)
+    rel = lambda y: float(np.linalg.norm(y - exact) / np.linalg.norm(exact))
+    info.update(cube=list(cube), rel_err_gpu=rel(bf16_bits_to_f64(g["Y"][rows])), rel_err_oracle=rel(y_ref),
+                rel_err_plain_nvfp4=rel(y_plain))
+    _record("sweep_%d%d%d" % cube, info)
+    if cube != (1, 1, 1):
+        assert info["rel_err_gpu"] < info["rel_err_plain_nvfp4"], info

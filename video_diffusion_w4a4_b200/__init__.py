@@ -226,7 +226,10 @@ def dq_linear_forward_ex(X, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2
                          workspace_bytes, stage_mask=DQ_STAGE_ALL, stage_events=None, stream=None) -> None:
     ev = None
     if stage_events is not None:
-        arr = (ctypes.c_void_p * 4)(*[e.cuda_event if hasattr(e, "cuda_event") else e for e in stage_events])
+        handles = [e.cuda_event if hasattr(e, "cuda_event") else e for e in stage_events]
+        if len(handles) != 4 or not all(handles):
+            raise ValueError("stage_events needs 4 created CUDA events (record a torch.cuda.Event once first)")
+        arr = (ctypes.c_void_p * 4)(*handles)
         ev = ctypes.cast(arr, ctypes.c_void_p)
     _check("dq_linear_forward_ex",
            _lib.dq_linear_forward_ex(_ptr(X), T, H, W, t, h, w, Ci, Co, rank, _ptr(packed_W), _ptr(L1_mma),
