@@ -248,6 +248,16 @@ int dq_selftest_bounded_wait(int budget_us, void* stream, int* status);
 int dq_selftest_convert(const float* in, long long n, uint8_t* e2m1, uint8_t* e4m3, float* e4m3_value,
                         void* stream);
 
+/*
+ * Quotient self test: the quantisers compute fl32(a / b) (b > 0) from the
+ * correctly rounded reciprocal of b with one product and one FMA correction
+ * step.  This draws n operand pairs from a counter-based hash of `seed` on the
+ * device and counts, into *mismatches (host), the pairs where that quotient
+ * differs in any bit from IEEE division; first_ab (host, 2 floats) receives
+ * the first mismatching pair.  Synchronous.
+ */
+int dq_selftest_divide(long long n, uint64_t seed, unsigned long long* mismatches, float* first_ab, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -177,3 +177,11 @@ def test_bounded_wait_times_out_and_context_survives(env):
     assert dq.dq_selftest_bounded_wait(2000, st) == dq.DQ_ERR_DEVICE_TIMEOUT
     # the context is still usable: a normal layer runs and is correct
     test_parity_small(env, "tiny", None)
+
+
+def test_quotient_path_matches_ieee_division(env):
+    """The quantisers' reciprocal + FMA-correction quotient equals IEEE
+    division bit for bit (Markstein's correction theorem), on 2^28 pairs."""
+    dq, torch = env
+    bad, first = dq.dq_selftest_divide(1 << 28, seed=12345, stream=torch.cuda.current_stream())
+    assert bad == 0, (bad, first)

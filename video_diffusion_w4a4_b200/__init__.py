@@ -72,6 +72,7 @@ _SIGS = {
     "dq_read_device_status": ([_P, _P, ctypes.POINTER(_I), _I], _I),
     "dq_selftest_bounded_wait": ([_I, _P, ctypes.POINTER(_I)], _I),
     "dq_selftest_convert": ([_P, _LL, _P, _P, _P, _P], _I),
+    "dq_selftest_divide": ([_LL, ctypes.c_uint64, ctypes.POINTER(ctypes.c_ulonglong), _P, _P], _I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -261,6 +262,14 @@ def dq_selftest_bounded_wait(budget_us: int, stream=None) -> int:
 def dq_selftest_convert(inp, n, e2m1, e4m3, e4m3_value, stream=None) -> None:
     _check("dq_selftest_convert", _lib.dq_selftest_convert(_ptr(inp), n, _ptr(e2m1), _ptr(e4m3), _ptr(e4m3_value),
                                                            _stream(stream)))
+
+
+def dq_selftest_divide(n: int, seed: int = 1, stream=None):
+    """Returns (mismatch count, first mismatching (a, b) or None)."""
+    cnt = ctypes.c_ulonglong()
+    ab = np.zeros(2, np.float32)
+    _check("dq_selftest_divide", _lib.dq_selftest_divide(n, seed, ctypes.byref(cnt), ab.ctypes.data, _stream(stream)))
+    return cnt.value, (tuple(ab.tolist()) if cnt.value else None)
 
 
 def loaded_library_path() -> str:

@@ -329,4 +329,20 @@ int dq_selftest_convert(const float* in, long long n, uint8_t* e2m1, uint8_t* e4
     return DQ_OK;
 }
 
+int dq_selftest_divide(long long n, uint64_t seed, unsigned long long* mismatches, float* first_ab, void* stream) {
+    if (n < 0 || !mismatches || !first_ab) return DQ_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned long long* d = nullptr;
+    if (cudaMalloc(&d, 16) != cudaSuccess) return DQ_ERR_ALLOC;
+    int rc = DQ_OK;
+    if (cudaMemsetAsync(d, 0, 16, st) != cudaSuccess ||
+        dq::launch_selftest_divide(n, seed, d, (float*)(d + 1), st) != cudaSuccess ||
+        cudaMemcpyAsync(mismatches, d, 8, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemcpyAsync(first_ab, d + 1, 8, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+        rc = DQ_ERR_CUDA;
+    cudaFree(d);
+    return rc;
+}
+
 }  // extern "C"

@@ -31,6 +31,47 @@ __global__ void k_selftest_convert(const float* in, long long n, uint8_t* e2m1, 
     e4m3_back[i] = e4m3_to_f32(c);
 }
 
+__device__ __forceinline__ uint64_t mix64d(uint64_t x) {
+    x += 0x9E3779B97F4A7C15ull;
+    x = (x ^ (x >> 30)) * 0xBF58476D1CE4E5B9ull;
+    x = (x ^ (x >> 27)) * 0x94D049BB133111EBull;
+    return x ^ (x >> 31);
+}
+
+// Compares the quantisers' quotient path (correctly rounded reciprocal, one
+// product, one FMA correction) with IEEE division, bit for bit, on operand
+// pairs drawn from a counter-based hash: a with exponent in [-40, 12] (and
+// exact zeros of either sign), b > 0 with exponent in [-30, 12].
+__global__ void k_selftest_divide(long long n, uint64_t seed, unsigned long long* mismatches, float* first) {
+    long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    unsigned long long bad = 0;
+    for (; i < n; i += stride) {
+        uint64_t h1 = mix64d(seed ^ (uint64_t)(2 * i)), h2 = mix64d(seed ^ (uint64_t)(2 * i + 1));
+        uint32_t ma = (uint32_t)(h1 & 0x7FFFFFu), mb = (uint32_t)(h2 & 0x7FFFFFu);
+        int ea = (int)((h1 >> 23) % 53) - 40, eb = (int)((h2 >> 23) % 43) - 30;
+        uint32_t sa = (uint32_t)((h1 >> 40) & 1u) << 31;
+        float a = __uint_as_float(sa | ((uint32_t)(ea + 127) << 23) | ma);
+        if (((h1 >> 41) & 1023u) == 0) a = __uint_as_float(sa);          // signed zeros
+        float b = __uint_as_float(((uint32_t)(eb + 127) << 23) | mb);
+        float q0 = __fdiv_rn(a, b);
+        float q1 = div_pos(a, b, __frcp_rn(b));
+        if (__float_as_uint(q0) != __float_as_uint(q1)) {
+            if (atomicAdd(mismatches, 1ull) == 0ull) {
+                first[0] = a;
+                first[1] = b;
+            }
+            bad++;
+        }
+    }
+}
+
+cudaError_t launch_selftest_divide(long long n, uint64_t seed, unsigned long long* mismatches, float* first,
+                                   cudaStream_t st) {
+    k_selftest_divide<<<148 * 8, 256, 0, st>>>(n, seed, mismatches, first);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_selftest_wait(int* status, uint64_t budget_ns, cudaStream_t st) {
     k_selftest_wait<<<1, 32, 0, st>>>(status, budget_ns);
     return cudaGetLastError();

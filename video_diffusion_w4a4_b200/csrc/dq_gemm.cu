@@ -3,21 +3,27 @@
 // DeltaQuant note (papernotes.org), key design 4, Eq. 2/3:
 //   Y = Q4(delta) Q4(R)  +  broadcast_cube(Q8(kernel) Q4(R))  +  X L1 L2
 //
-//   (c) k_kernel_gemm: P'[k][o] = s8_k S_W sum_c q8[k][c] (q s_b)[o][c].  The
-//       operands are the E4M3 kernel tokens and the dequantised weight q*s_b,
-//       both exact in BF16, so the product runs as kind::f16 (BF16 x BF16 ->
-//       fp32).  (No FP8 tensor-core kind takes E4M3 group-16 weight scales.)
-//   (b) k_main_gemm: acc[rho][o] = sum_c (q s)_delta (q s)_R with
+//   (c) kernel-token product: P'[k][o] = s8_k S_W sum_c q8[k][c] (q s_b)[o][c].
+//       Both operands (the E4M3 kernel tokens and the dequantised weight
+//       q*s_b) are exact in BF16, so it runs as kind::f16 (BF16 x BF16 -> fp32).
+//       No FP8 tensor-core kind takes E4M3 group-16 weight scales.
+//   (b) main product: acc[rho][o] = sum_c (q s)_delta (q s)_R with
 //       kind::mxf4nvf4 block-16 scaled FP4 MMAs, then the low-rank
 //       up-projection as extra BF16 K-steps [U_hi | U_lo] x [L2^T | L2^T] into
 //       the same tensor-memory accumulator; the epilogue forms
 //       Y[n(rho)][o] = S_delta S_W acc + P'[k(rho)][o] and scatters each
 //       cube-major row back to its (t,h,w) position.
 //
-// Structure (both): one 128 x 256 output tile per CTA; warp 0 issues TMA
-// loads into a 4-stage shared-memory ring, warp 1 owns tensor memory and
-// issues the MMAs from one thread, warps 2-5 drain the fp32 accumulator from
-// tensor memory (each warp its 32-lane sub-partition).  All waits are bounded.
+// One persistent kernel template serves both: one CTA per SM walks the
+// 128 x 256 output tiles tile = blockIdx.x + i * gridDim.x.  Warp 0 streams
+// operand tiles with TMA into a 4-stage shared-memory ring that runs on across
+// tiles; warp 1 owns tensor memory and issues the MMAs from one thread; warps
+// 2-9 drain the fp32 accumulator, two warps per 32-lane sub-partition, each
+// half of the columns.  The kernel-token product double-buffers its
+// accumulator in tensor memory so the epilogue of one tile overlaps the MMAs
+// of the next; the main product needs tensor-memory columns for the block
+// scale factors, so it keeps one accumulator and instead has its epilogue load
+// the P' rows of a tile into registers while that tile's MMAs run.
 #include "dq_common.h"
 #include "dq_internal.h"
 #include "dq_ptx.cuh"
@@ -28,6 +34,8 @@ namespace {
 
 constexpr int kStages = 4;
 constexpr int kTileM = 128, kTileN = 256;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kABytes = kTileM * 128;  // 128 rows x 128 bytes
 constexpr uint32_t kBBytes = kTileN * 128;  // 256 rows x 128 bytes
 constexpr uint32_t kSFABytes = 4 * 512;     // 128 rows x 4 k-steps of 64
@@ -49,7 +57,7 @@ __host__ __device__ constexpr GSmem g_smem_layout(bool scaled) {
     L.sfb = off;
     if (scaled) off += kStages * kSFBBytes;
     L.bars = off;
-    off += (2 * kStages + 2) * 8;
+    off += (2 * kStages + 5) * 8;
     L.misc = off;
     off += 64;
     L.total = off;
@@ -60,133 +68,37 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) { return smem_desc(s
 
 }  // namespace
 
-// ------------------------------------------------------------------ (c) kernel-token product
-
-__global__ void __launch_bounds__(192, 1) k_kernel_gemm(const __grid_constant__ CUtensorMap tm_a,
-                                                         const __grid_constant__ CUtensorMap tm_b, GemmParams p) {
+template <bool kMain>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+           const __grid_constant__ CUtensorMap tm_sa, const __grid_constant__ CUtensorMap tm_sb, GemmParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    constexpr GSmem L = g_smem_layout(false);
+    constexpr GSmem L = g_smem_layout(kMain);
+    constexpr int kBufs = kMain ? 1 : 2;
     uint64_t* full = (uint64_t*)(sm + L.bars);
     uint64_t* empty = full + kStages;
-    uint64_t* accf = empty + kStages;
+    uint64_t* accf = empty + kStages;   // [2]
+    uint64_t* acce = accf + 2;          // [2]
+    uint64_t* drain = acce + 2;
     uint32_t* tmem_slot = (uint32_t*)(sm + L.misc);
     volatile int* abort_flag = (volatile int*)(sm + L.misc + 8);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n0 = blockIdx.x * kTileN, m0 = blockIdx.y * kTileM;
-    const int nk = p.k_stages;
-
-    if (tid == 0) {
-        for (int s = 0; s < kStages; s++) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        mbar_init(accf, 1);
-        *abort_flag = 0;
-        fence_barrier_init();
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, 256);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            prefetch_tmap(&tm_a);
-            prefetch_tmap(&tm_b);
-            int issued = 0;
-            for (int i = 0; i < nk; i++) {
-                int s = i % kStages;
-                if (i >= kStages && !mbar_wait(&empty[s], ((i / kStages) - 1) & 1, abort_flag, p.status, p.budget_ns))
-                    break;
-                mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
-                tma_load_2d(sm + L.a + s * kABytes, &tm_a, &full[s], i * 64, m0);
-                tma_load_2d(sm + L.b + s * kBBytes, &tm_b, &full[s], i * 64, n0);
-                issued = i + 1;
-            }
-            for (int i = (issued > kStages ? issued - kStages : 0); i < issued; i++)
-                mbar_wait(&full[i % kStages], (i / kStages) & 1, abort_flag, nullptr, p.budget_ns, false);
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(kTileM, kTileN);
-            for (int i = 0; i < nk; i++) {
-                int s = i % kStages;
-                if (!mbar_wait(&full[s], (i / kStages) & 1, abort_flag, p.status, p.budget_ns)) break;
-                tc_fence_after();
-                uint32_t aa = smem_u32(sm + L.a + s * kABytes), bb = smem_u32(sm + L.b + s * kBBytes);
-#pragma unroll
-                for (int k = 0; k < 4; k++)
-                    mma_bf16(tmem, desc_k_sw128(aa + 32 * k), desc_k_sw128(bb + 32 * k), idesc, (i | k) != 0);
-                tc_commit(&empty[s]);
-            }
-            tc_commit(accf);
-            mbar_wait(accf, 0, abort_flag, nullptr, p.budget_ns, false);
-        }
-        __syncwarp();
-    } else {
-        // epilogue: P'[m][n] = s8[m] S_W acc
-        const int quad = warp & 3;
-        const int row = m0 + quad * 32 + lane;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0, abort_flag, p.status, p.budget_ns));
-        tc_fence_after();
-        if (ok) {
-            const float sw = reinterpret_cast<const PackedHeader*>(p.packed_w)->S_W;
-            const float scale = (row < p.M) ? __fmul_rn(p.s8[row], sw) : 0.f;
-            float* dst = p.pout + (size_t)row * p.Nout + n0;
-            for (int c = 0; c < kTileN; c += 16) {
-                uint32_t r[16];
-                tmem_ld_x16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c, r);
-                tmem_ld_wait();
-                if (row < p.M) {
-#pragma unroll
-                    for (int v = 0; v < 16; v += 4)
-                        *reinterpret_cast<float4*>(dst + c + v) =
-                            make_float4(__uint_as_float(r[v]) * scale, __uint_as_float(r[v + 1]) * scale,
-                                        __uint_as_float(r[v + 2]) * scale, __uint_as_float(r[v + 3]) * scale);
-                }
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 256);
-    }
-}
-
-// ------------------------------------------------------------------ (b) main product
-
-__global__ void __launch_bounds__(192, 1) k_main_gemm(const __grid_constant__ CUtensorMap tm_a,
-                                                       const __grid_constant__ CUtensorMap tm_b,
-                                                       const __grid_constant__ CUtensorMap tm_sa,
-                                                       const __grid_constant__ CUtensorMap tm_sb, GemmParams p) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    constexpr GSmem L = g_smem_layout(true);
-    uint64_t* full = (uint64_t*)(sm + L.bars);
-    uint64_t* empty = full + kStages;
-    uint64_t* accf = empty + kStages;
-    uint32_t* tmem_slot = (uint32_t*)(sm + L.misc);
-    volatile int* abort_flag = (volatile int*)(sm + L.misc + 8);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n0 = blockIdx.x * kTileN, m0 = blockIdx.y * kTileM;
+    const int num_n = p.Nout / kTileN;
+    const int num_tiles = (int)cdiv(p.M, kTileM) * num_n;
     const int nk = p.k_stages, ntot = p.k_stages + p.slab_stages;
-    const int kgroups = p.Ci / 64;
 
     if (tid == 0) {
         for (int s = 0; s < kStages; s++) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accf, 1);
+        for (int b = 0; b < 2; b++) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acce[b], 32 * kEpiWarps);
+        }
+        mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -198,105 +110,188 @@ __global__ void __launch_bounds__(192, 1) k_main_gemm(const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_sfa = tmem + 256, t_sfb = tmem + 272;
 
     if (warp == 0) {
+        // ------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tm_a);
             prefetch_tmap(&tm_b);
-            prefetch_tmap(&tm_sa);
-            prefetch_tmap(&tm_sb);
-            int issued = 0;
-            for (int i = 0; i < ntot; i++) {
-                int s = i % kStages;
-                if (i >= kStages && !mbar_wait(&empty[s], ((i / kStages) - 1) & 1, abort_flag, p.status, p.budget_ns))
-                    break;
-                if (i < nk) {
-                    mbar_arrive_expect_tx(&full[s], kABytes + kBBytes + kSFABytes + kSFBBytes);
-                    tma_load_2d(sm + L.a + s * kABytes, &tm_a, &full[s], i * 128, m0);
-                    tma_load_2d(sm + L.b + s * kBBytes, &tm_b, &full[s], i * 128, n0);
-                    const uint8_t* sa = p.sfa + ((size_t)(m0 >> 7) * kgroups + 4 * i) * 512;
-                    bulk_load(sm + L.sfa + s * kSFABytes, sa, kSFABytes, &full[s]);
-#pragma unroll
-                    for (int g = 0; g < 2; g++) {
-                        const uint8_t* sb = p.sfb + ((size_t)((n0 >> 7) + g) * kgroups + 4 * i) * 512;
-                        bulk_load(sm + L.sfb + s * kSFBBytes + g * (kSFBBytes / 2), sb, kSFBBytes / 2, &full[s]);
-                    }
-                } else {
-                    mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
-                    tma_load_2d(sm + L.a + s * kABytes, &tm_sa, &full[s], (i - nk) * 64, m0);
-                    tma_load_2d(sm + L.b + s * kBBytes, &tm_sb, &full[s], (i - nk) * 64, n0);
-                }
-                issued = i + 1;
+            if (kMain) {
+                prefetch_tmap(&tm_sa);
+                prefetch_tmap(&tm_sb);
             }
-            for (int i = (issued > kStages ? issued - kStages : 0); i < issued; i++)
-                mbar_wait(&full[i % kStages], (i / kStages) & 1, abort_flag, nullptr, p.budget_ns, false);
+            const int kgroups = p.Ci / 64;
+            long long g = 0;
+            bool alive = true;
+            for (int tile = blockIdx.x; alive && tile < num_tiles; tile += gridDim.x) {
+                const int m0 = (tile / num_n) * kTileM, n0 = (tile % num_n) * kTileN;
+                for (int i = 0; i < ntot; i++, g++) {
+                    const int s = (int)(g % kStages);
+                    if (g >= kStages &&
+                        !mbar_wait(&empty[s], (uint32_t)((g / kStages) - 1) & 1, abort_flag, p.status, p.budget_ns)) {
+                        alive = false;
+                        break;
+                    }
+                    if (!kMain) {
+                        mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
+                        tma_load_2d(sm + L.a + s * kABytes, &tm_a, &full[s], i * 64, m0);
+                        tma_load_2d(sm + L.b + s * kBBytes, &tm_b, &full[s], i * 64, n0);
+                    } else if (i < nk) {
+                        mbar_arrive_expect_tx(&full[s], kABytes + kBBytes + kSFABytes + kSFBBytes);
+                        tma_load_2d(sm + L.a + s * kABytes, &tm_a, &full[s], i * 128, m0);
+                        tma_load_2d(sm + L.b + s * kBBytes, &tm_b, &full[s], i * 128, n0);
+                        bulk_load(sm + L.sfa + s * kSFABytes, p.sfa + ((size_t)(m0 >> 7) * kgroups + 4 * i) * 512,
+                                  kSFABytes, &full[s]);
+#pragma unroll
+                        for (int h = 0; h < 2; h++)
+                            bulk_load(sm + L.sfb + s * kSFBBytes + h * (kSFBBytes / 2),
+                                      p.sfb + ((size_t)((n0 >> 7) + h) * kgroups + 4 * i) * 512, kSFBBytes / 2,
+                                      &full[s]);
+                    } else {
+                        mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
+                        tma_load_2d(sm + L.a + s * kABytes, &tm_sa, &full[s], (i - nk) * 64, m0);
+                        tma_load_2d(sm + L.b + s * kBBytes, &tm_sb, &full[s], (i - nk) * 64, n0);
+                    }
+                }
+            }
+            // every issued load lands before shared memory is released
+            for (long long q = (g > kStages ? g - kStages : 0); q < g; q++)
+                mbar_wait(&full[q % kStages], (uint32_t)(q / kStages) & 1, abort_flag, nullptr, p.budget_ns, false);
         }
     } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t id4 = idesc_nvfp4(kTileM, kTileN), id16 = idesc_bf16(kTileM, kTileN);
-            for (int i = 0; i < ntot; i++) {
-                int s = i % kStages;
-                if (!mbar_wait(&full[s], (i / kStages) & 1, abort_flag, p.status, p.budget_ns)) break;
+            const uint32_t id_main = kMain ? idesc_nvfp4(kTileM, kTileN) : idesc_bf16(kTileM, kTileN);
+            const uint32_t id_slab = idesc_bf16(kTileM, kTileN);
+            const uint32_t t_sfa = tmem + 256, t_sfb = tmem + 272;
+            long long g = 0;
+            int it = 0;
+            bool alive = true;
+            for (int tile = blockIdx.x; alive && tile < num_tiles; tile += gridDim.x, it++) {
+                const int buf = it % kBufs, use = it / kBufs;
+                const uint32_t acc = tmem + (uint32_t)(buf * 256);
+                if (use > 0 && !mbar_wait(&acce[buf], (uint32_t)(use - 1) & 1, abort_flag, p.status, p.budget_ns))
+                    break;
                 tc_fence_after();
-                uint32_t aa = smem_u32(sm + L.a + s * kABytes), bb = smem_u32(sm + L.b + s * kBBytes);
-                if (i < nk) {
-                    uint32_t fa = smem_u32(sm + L.sfa + s * kSFABytes), fb = smem_u32(sm + L.sfb + s * kSFBBytes);
-#pragma unroll
-                    for (int k = 0; k < 4; k++) {
-                        tmem_cp_32x128b_x4(t_sfa + 4 * k, desc_sf(fa + 512 * k));
-                        tmem_cp_32x128b_x4(t_sfb + 8 * k, desc_sf(fb + 512 * k));
-                        tmem_cp_32x128b_x4(t_sfb + 8 * k + 4, desc_sf(fb + kSFBBytes / 2 + 512 * k));
+                for (int i = 0; i < ntot; i++, g++) {
+                    const int s = (int)(g % kStages);
+                    if (!mbar_wait(&full[s], (uint32_t)(g / kStages) & 1, abort_flag, p.status, p.budget_ns)) {
+                        alive = false;
+                        break;
                     }
+                    tc_fence_after();
+                    const uint32_t aa = smem_u32(sm + L.a + s * kABytes), bb = smem_u32(sm + L.b + s * kBBytes);
+                    if (kMain && i < nk) {
+                        const uint32_t fa = smem_u32(sm + L.sfa + s * kSFABytes);
+                        const uint32_t fb = smem_u32(sm + L.sfb + s * kSFBBytes);
 #pragma unroll
-                    for (int k = 0; k < 4; k++)
-                        mma_nvfp4(tmem, desc_k_sw128(aa + 32 * k), desc_k_sw128(bb + 32 * k), id4, t_sfa + 4 * k,
-                                  t_sfb + 8 * k, (i | k) != 0);
-                } else {
+                        for (int k = 0; k < 4; k++) {
+                            tmem_cp_32x128b_x4(t_sfa + 4 * k, desc_sf(fa + 512 * k));
+                            tmem_cp_32x128b_x4(t_sfb + 8 * k, desc_sf(fb + 512 * k));
+                            tmem_cp_32x128b_x4(t_sfb + 8 * k + 4, desc_sf(fb + kSFBBytes / 2 + 512 * k));
+                        }
 #pragma unroll
-                    for (int k = 0; k < 4; k++)
-                        mma_bf16(tmem, desc_k_sw128(aa + 32 * k), desc_k_sw128(bb + 32 * k), id16, 1u);
+                        for (int k = 0; k < 4; k++)
+                            mma_nvfp4(acc, desc_k_sw128(aa + 32 * k), desc_k_sw128(bb + 32 * k), id_main,
+                                      t_sfa + 4 * k, t_sfb + 8 * k, (i | k) != 0);
+                    } else {
+                        const uint32_t id = kMain ? id_slab : id_main;
+#pragma unroll
+                        for (int k = 0; k < 4; k++)
+                            mma_bf16(acc, desc_k_sw128(aa + 32 * k), desc_k_sw128(bb + 32 * k), id,
+                                     (kMain || (i | k) != 0) ? 1u : 0u);
+                    }
+                    tc_commit(&empty[s]);
                 }
-                tc_commit(&empty[s]);
+                if (alive) tc_commit(&accf[buf]);
             }
-            tc_commit(accf);
-            mbar_wait(accf, 0, abort_flag, nullptr, p.budget_ns, false);
+            // no MMA may still run when tensor memory is released
+            tc_commit(drain);
+            mbar_wait(drain, 0, abort_flag, nullptr, p.budget_ns, false);
         }
         __syncwarp();
     } else {
-        // epilogue: Y[n][o] = bf16(S_delta S_W acc + P'[k][o]), row scattered to (t,h,w) order
-        const int quad = warp & 3;
-        const long long rho = (long long)m0 + quad * 32 + lane;
-        const bool row_ok = rho < p.M;
-        long long n = 0, k = 0;
-        if (row_ok) row_to_token(p.g, rho, &n, &k);
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0, abort_flag, p.status, p.budget_ns));
-        tc_fence_after();
-        if (ok) {
-            const float SS =
-                __fmul_rn(__uint_as_float(p.scalars[1]), reinterpret_cast<const PackedHeader*>(p.packed_w)->S_W);
-            const float* prow = p.p + (size_t)k * p.Nout + n0;
-            uint16_t* yrow = p.Y + (size_t)n * p.Nout + n0;
-            for (int c = 0; c < kTileN; c += 16) {
-                uint32_t r[16];
-                tmem_ld_x16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c, r);
-                tmem_ld_wait();
-                if (row_ok) {
-                    uint32_t packed[8];
+        // ------------------------------------------------ epilogue warps
+        const int quad = warp & 3, half = (warp - 2) >> 2;
+        const float S_W = reinterpret_cast<const PackedHeader*>(p.packed_w)->S_W;
+        const float SS = kMain ? __fmul_rn(__uint_as_float(p.scalars[1]), S_W) : 0.f;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, it++) {
+            const int buf = it % kBufs, use = it / kBufs;
+            const int m0 = (tile / num_n) * kTileM, n0 = (tile % num_n) * kTileN;
+            const long long rho = (long long)m0 + quad * 32 + lane;
+            const bool row_ok = rho < p.M;
+            const int c_base = n0 + half * 128;
+            const uint32_t tacc = tmem + (uint32_t)(buf * 256) + ((uint32_t)(quad * 32) << 16) + (uint32_t)(half * 128);
+            if (kMain) {
+                // the P' row segment of this token's cube, fetched while the tile's MMAs run
+                long long n = 0, k = 0;
+                if (row_ok) row_to_token(p.g, rho, &n, &k);
+                float4 pf[32];
+                const float4* prow = reinterpret_cast<const float4*>(p.p + (size_t)k * p.Nout + c_base);
 #pragma unroll
-                    for (int v = 0; v < 16; v += 4) {
-                        float4 pv = *reinterpret_cast<const float4*>(prow + c + v);
-                        float y0 = fmaf(SS, __uint_as_float(r[v]), pv.x);
-                        float y1 = fmaf(SS, __uint_as_float(r[v + 1]), pv.y);
-                        float y2 = fmaf(SS, __uint_as_float(r[v + 2]), pv.z);
-                        float y3 = fmaf(SS, __uint_as_float(r[v + 3]), pv.w);
-                        packed[v / 2] = (uint32_t)f32_to_bf16_rn(y0) | ((uint32_t)f32_to_bf16_rn(y1) << 16);
-                        packed[v / 2 + 1] = (uint32_t)f32_to_bf16_rn(y2) | ((uint32_t)f32_to_bf16_rn(y3) << 16);
+                for (int v = 0; v < 32; v++) pf[v] = row_ok ? __ldg(prow + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+                const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], (uint32_t)use & 1, abort_flag,
+                                                                  p.status, p.budget_ns));
+                if (!ok) break;
+                tc_fence_after();
+                uint16_t* yrow = p.Y + (size_t)n * p.Nout + c_base;
+#pragma unroll
+                for (int c = 0; c < 128; c += 32) {
+                    uint32_t r0[16], r1[16];
+                    tmem_ld_x16(tacc + (uint32_t)c, r0);
+                    tmem_ld_x16(tacc + (uint32_t)c + 16, r1);
+                    tmem_ld_wait();
+                    if (row_ok) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int v = 0; v < 16; v += 2) {
+                            const float4 q = pf[(c + v) / 4];
+                            const float a0 = (v & 2) ? q.z : q.x, a1 = (v & 2) ? q.w : q.y;
+                            pk[v / 2] = (uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(r0[v]), a0)) |
+                                        ((uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(r0[v + 1]), a1)) << 16);
+                            const float4 q2 = pf[(c + 16 + v) / 4];
+                            const float b0 = (v & 2) ? q2.z : q2.x, b1 = (v & 2) ? q2.w : q2.y;
+                            pk[8 + v / 2] =
+                                (uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(r1[v]), b0)) |
+                                ((uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(r1[v + 1]), b1)) << 16);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(yrow + c);
+                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                        dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+                        dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
                     }
-                    reinterpret_cast<uint4*>(yrow + c)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                    reinterpret_cast<uint4*>(yrow + c)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                }
+            } else {
+                const float scale = row_ok ? __fmul_rn(p.s8[rho], S_W) : 0.f;
+                const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], (uint32_t)use & 1, abort_flag,
+                                                                  p.status, p.budget_ns));
+                if (!ok) break;
+                tc_fence_after();
+                float* dst = p.pout + (size_t)rho * p.Nout + c_base;
+#pragma unroll
+                for (int c = 0; c < 128; c += 32) {
+                    uint32_t r0[16], r1[16];
+                    tmem_ld_x16(tacc + (uint32_t)c, r0);
+                    tmem_ld_x16(tacc + (uint32_t)c + 16, r1);
+                    tmem_ld_wait();
+                    if (row_ok) {
+#pragma unroll
+                        for (int v = 0; v < 16; v += 4) {
+                            *reinterpret_cast<float4*>(dst + c + v) =
+                                make_float4(__uint_as_float(r0[v]) * scale, __uint_as_float(r0[v + 1]) * scale,
+                                            __uint_as_float(r0[v + 2]) * scale, __uint_as_float(r0[v + 3]) * scale);
+                            *reinterpret_cast<float4*>(dst + c + 16 + v) =
+                                make_float4(__uint_as_float(r1[v]) * scale, __uint_as_float(r1[v + 1]) * scale,
+                                            __uint_as_float(r1[v + 2]) * scale, __uint_as_float(r1[v + 3]) * scale);
+                        }
+                    }
                 }
             }
+            // tensor-memory buffer free for the next tile
+            tc_fence_before();
+            mbar_arrive(&acce[buf]);
         }
     }
     tc_fence_before();
@@ -309,23 +304,36 @@ __global__ void __launch_bounds__(192, 1) k_main_gemm(const __grid_constant__ CU
 
 // ------------------------------------------------------------------ launchers
 
+namespace {
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+}  // namespace
+
 cudaError_t launch_kernel_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmParams& p,
                                cudaStream_t st) {
     constexpr size_t smem = g_smem_layout(false).total + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_kernel_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.Nout / kTileN, (unsigned)cdiv(p.M, kTileM));
-    k_kernel_gemm<<<grid, 192, smem, st>>>(tm_a, tm_b, p);
+    const int tiles = (int)cdiv(p.M, kTileM) * (p.Nout / kTileN);
+    k_gemm<false><<<imin(tiles, sm_count()), kThreads, smem, st>>>(tm_a, tm_b, tm_a, tm_b, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_main_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_sa,
                              const CUtensorMap& tm_sb, const GemmParams& p, cudaStream_t st) {
     constexpr size_t smem = g_smem_layout(true).total + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_main_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.Nout / kTileN, (unsigned)cdiv(p.M, kTileM));
-    k_main_gemm<<<grid, 192, smem, st>>>(tm_a, tm_b, tm_sa, tm_sb, p);
+    const int tiles = (int)cdiv(p.M, kTileM) * (p.Nout / kTileN);
+    k_gemm<true><<<imin(tiles, sm_count()), kThreads, smem, st>>>(tm_a, tm_b, tm_sa, tm_sb, p);
     return cudaGetLastError();
 }
 

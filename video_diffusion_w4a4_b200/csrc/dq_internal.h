@@ -61,6 +61,8 @@ cudaError_t launch_main_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, c
                              const CUtensorMap& tm_sb, const GemmParams& p, cudaStream_t st);
 
 cudaError_t launch_selftest_wait(int* status, uint64_t budget_ns, cudaStream_t st);
+cudaError_t launch_selftest_divide(long long n, uint64_t seed, unsigned long long* mismatches, float* first,
+                                   cudaStream_t st);
 cudaError_t launch_selftest_convert(const float* in, long long n, uint8_t* e2m1, uint8_t* e4m3, float* back,
                                     cudaStream_t st);
 

@@ -263,6 +263,17 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
     return __half2float(__half(hr));
 }
 
+// fl32(a / b) for b > 0 from rb = fl32(1 / b): one product and one FMA
+// correction step (Markstein), which returns the correctly rounded quotient
+// when rb is the correctly rounded reciprocal; the result takes a's sign, as
+// IEEE division by a positive b does (also for a = -0 and for underflow).
+__device__ __forceinline__ float div_pos(float a, float b, float rb) {
+    float q = __fmul_rn(a, rb);
+    float r = __fmaf_rn(-q, b, a);
+    q = __fmaf_rn(r, rb, q);
+    return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(a) & 0x80000000u));
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 

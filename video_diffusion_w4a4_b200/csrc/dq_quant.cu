@@ -101,25 +101,45 @@ __device__ __forceinline__ bool box_row(const QuantParams& p, const BoxPos& B, i
     return true;
 }
 
-// Sequential fp32 sum of the cube's tokens in (t,h,w) order, divided by the
-// count (Eq. 1, kernel token).  No fused multiply-add is involved.
-__device__ __forceinline__ float cube_mean(const QuantParams& p, const BoxPos& B, const uint8_t* xs, int j, int c,
-                                           bool* valid) {
-    const Geom& g = p.g;
-    int kw = B.bkw * p.nw + j;
-    if (kw >= g.KW) {
-        *valid = false;
-        return 0.f;
-    }
-    *valid = true;
-    int st = imin(g.t, g.T - B.t0), sh = imin(g.h, g.H - B.h0), sw = imin(g.w, g.W - kw * g.w);
-    float acc = 0.f;
+// Kernel tokens (Eq. 1) of cube slot j for channels [8g, 8g+8) of the chunk:
+// an fp32 running sum over the cube's tokens in (t,h,w) order, then the
+// division by the token count (a product with the exact reciprocal when the
+// count is a power of two, which gives the identical rounding).  Returns
+// false for cube slots past the end of the lattice.
+__device__ __forceinline__ bool cube_mean8(const QuantParams& p, const BoxPos& B, const uint8_t* xs, int j, int g,
+                                           int st, int sh, float (&m)[8]) {
+    const Geom& g_ = p.g;
+    const int kw = B.bkw * p.nw + j;
+    if (kw >= g_.KW) return false;
+    const int sw = imin(g_.w, g_.W - kw * g_.w);
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; e++) acc[e] = 0.f;
     for (int dt = 0; dt < st; dt++)
         for (int dh = 0; dh < sh; dh++) {
-            int row0 = (dt * p.bh + dh) * p.bw + j * g.w;
-            for (int dw = 0; dw < sw; dw++) acc = __fadd_rn(acc, ld_x_swz(xs, row0 + dw, c));
+            const int row0 = (dt * p.bh + dh) * p.bw + j * g_.w;
+            for (int dw = 0; dw < sw; dw++) {
+                uint4 v = ld_x8_swz(xs, row0 + dw, g);
+                acc[0] = __fadd_rn(acc[0], bf16_lo(v.x));
+                acc[1] = __fadd_rn(acc[1], bf16_hi(v.x));
+                acc[2] = __fadd_rn(acc[2], bf16_lo(v.y));
+                acc[3] = __fadd_rn(acc[3], bf16_hi(v.y));
+                acc[4] = __fadd_rn(acc[4], bf16_lo(v.z));
+                acc[5] = __fadd_rn(acc[5], bf16_hi(v.z));
+                acc[6] = __fadd_rn(acc[6], bf16_lo(v.w));
+                acc[7] = __fadd_rn(acc[7], bf16_hi(v.w));
+            }
         }
-    return __fdiv_rn(acc, (float)(st * sh * sw));
+    const int cnt = st * sh * sw;
+    if ((cnt & (cnt - 1)) == 0) {
+        const float inv = __frcp_rn((float)cnt);
+#pragma unroll
+        for (int e = 0; e < 8; e++) m[e] = __fmul_rn(acc[e], inv);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; e++) m[e] = __fdiv_rn(acc[e], (float)cnt);
+    }
+    return true;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -221,6 +241,7 @@ __global__ void __launch_bounds__(192, 1) k_cube_stats(const __grid_constant__ C
         int myj = -1;
         long long myrho = 0, myk = 0;
         const bool row_ok = box_row(p, B, tid, &myj, &myrho, &myk);
+        const int st = imin(p.g.t, p.g.T - B.t0), sh = imin(p.g.h, p.g.H - B.h0);
         for (int i = 0; i < nchunks; i++) {
             int s = i % kQStages;
             // a failed wait skips the work but keeps the barrier protocol
@@ -228,13 +249,17 @@ __global__ void __launch_bounds__(192, 1) k_cube_stats(const __grid_constant__ C
                                                               p.budget_ns));
             const uint8_t* xs = sm + L.x + s * 16384;
             // kernel tokens of the box's cubes for these 64 channels
-            for (int q = tid; ok && q < p.nw * 64; q += 128) {
-                int j = q >> 6, c = q & 63;
-                bool v;
-                float m = cube_mean(p, B, xs, j, c, &v);
-                means[j * kMeanStride + c] = m;
-                float am = warp_max(fabsf(m));
-                if (lane == 0 && v) atomicMax(&kmax[j], __float_as_uint(am));
+            for (int q = tid; ok && q < p.nw * 8; q += 128) {
+                const int j = q >> 3, g8 = q & 7;
+                float m[8];
+                if (!cube_mean8(p, B, xs, j, g8, st, sh, m)) continue;
+                float* dst = means + j * kMeanStride + 8 * g8;
+                *reinterpret_cast<float4*>(dst) = make_float4(m[0], m[1], m[2], m[3]);
+                *reinterpret_cast<float4*>(dst + 4) = make_float4(m[4], m[5], m[6], m[7]);
+                float am = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; e++) am = fmaxf(am, fabsf(m[e]));
+                atomicMax(&kmax[j], __float_as_uint(am));
             }
             bar_sync(1, 128);
             // delta amax of this thread's token row
@@ -310,6 +335,7 @@ __global__ void __launch_bounds__(160, 1) k_cube_encode(const __grid_constant__ 
     volatile int* abort_flag = (volatile int*)(sm + L.misc + 8);
     float* means = (float*)(sm + L.means);
     float* s8s = (float*)(sm + L.s8);
+    float* rs8s = (float*)(sm + L.kmax);   // reciprocals of s8 (the kmax slot is unused in this kernel)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int box = blockIdx.x, split = blockIdx.y;
@@ -344,6 +370,7 @@ __global__ void __launch_bounds__(160, 1) k_cube_encode(const __grid_constant__ 
             if (split == 0) p.s8[k] = s;
         }
         s8s[j] = s;
+        rs8s[j] = (s != 0.f) ? __frcp_rn(s) : 0.f;
     }
     if (box == 0 && split == 0 && tid == 0) p.scalars[1] = __float_as_uint(S);
     __syncthreads();
@@ -367,6 +394,7 @@ __global__ void __launch_bounds__(160, 1) k_cube_encode(const __grid_constant__ 
         int myj = -1;
         long long myrho = 0, myk = 0;
         const bool row_ok = box_row(p, B, tid, &myj, &myrho, &myk);
+        const int st = imin(p.g.t, p.g.T - B.t0), sh = imin(p.g.h, p.g.H - B.h0);
         for (int i = 0; i < nchunks; i++) {
             int s = i % kQStages;
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (i / kQStages) & 1, abort_flag, p.status,
@@ -374,18 +402,30 @@ __global__ void __launch_bounds__(160, 1) k_cube_encode(const __grid_constant__ 
             const uint8_t* xs = sm + L.x + s * 16384;
             const int c0 = c_base + i * 64;
             // kernel tokens: means, FP8 E4M3 codes with the per-token scale s8 = max|mean| / 448
-            for (int q = tid; ok && q < p.nw * 64; q += 128) {
-                int j = q >> 6, c = q & 63;
-                bool v;
-                float m = cube_mean(p, B, xs, j, c, &v);
-                means[j * kMeanStride + c] = m;
-                if (v) {
-                    long long k = ((long long)B.bkt * p.g.KH + B.bkh) * p.g.KW + (B.bkw * p.nw + j);
-                    float s8 = s8s[j];
-                    uint32_t code = (s8 == 0.f) ? 0u : (cvt_e4m3x2(__fdiv_rn(m, s8), 0.f) & 0xFFu);
-                    p.q8[(size_t)k * Ci + c0 + c] = (uint8_t)code;
-                    p.q8_bf16[(size_t)k * Ci + c0 + c] = f32_to_bf16_rn(e4m3_to_f32(code));
+            for (int q = tid; ok && q < p.nw * 8; q += 128) {
+                const int j = q >> 3, g8 = q & 7;
+                float m[8];
+                if (!cube_mean8(p, B, xs, j, g8, st, sh, m)) continue;
+                float* dst = means + j * kMeanStride + 8 * g8;
+                *reinterpret_cast<float4*>(dst) = make_float4(m[0], m[1], m[2], m[3]);
+                *reinterpret_cast<float4*>(dst + 4) = make_float4(m[4], m[5], m[6], m[7]);
+                const long long k = ((long long)B.bkt * p.g.KH + B.bkh) * p.g.KW + (B.bkw * p.nw + j);
+                const float s8 = s8s[j], rs8 = rs8s[j];
+                uint32_t c[4] = {0u, 0u, 0u, 0u};
+                if (s8 != 0.f) {
+#pragma unroll
+                    for (int e = 0; e < 4; e++)
+                        c[e] = cvt_e4m3x2(div_pos(m[2 * e], s8, rs8), div_pos(m[2 * e + 1], s8, rs8));
                 }
+                *reinterpret_cast<uint2*>(p.q8 + (size_t)k * Ci + c0 + 8 * g8) =
+                    make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+                uint32_t bfw[4];
+#pragma unroll
+                for (int e = 0; e < 4; e++)
+                    bfw[e] = (uint32_t)f32_to_bf16_rn(e4m3_to_f32(c[e] & 0xFF)) |
+                             ((uint32_t)f32_to_bf16_rn(e4m3_to_f32(c[e] >> 8)) << 16);
+                *reinterpret_cast<uint4*>(p.q8_bf16 + (size_t)k * Ci + c0 + 8 * g8) =
+                    make_uint4(bfw[0], bfw[1], bfw[2], bfw[3]);
             }
             bar_sync(1, 128);
             // delta tokens: FP4 E2M1 with E4M3 group-16 scales under S
@@ -416,13 +456,15 @@ __global__ void __launch_bounds__(160, 1) k_cube_encode(const __grid_constant__ 
                     uint32_t sb = cvt_e4m3x2(__fdiv_rn(am, denom), 0.f) & 0xFFu;
                     float eff = __fmul_rn(e4m3_to_f32(sb), S);
                     sc |= sb << (8 * b);
+                    const float reff = (eff != 0.f) ? __frcp_rn(eff) : 0.f;
 #pragma unroll
                     for (int e = 0; e < 16; e += 8) {
                         uint32_t wv = 0;
                         if (eff != 0.f) {
 #pragma unroll
                             for (int u = 0; u < 8; u += 2)
-                                wv |= cvt_e2m1x2(__fdiv_rn(z[e + u], eff), __fdiv_rn(z[e + u + 1], eff)) << (4 * u);
+                                wv |= cvt_e2m1x2(div_pos(z[e + u], eff, reff), div_pos(z[e + u + 1], eff, reff))
+                                      << (4 * u);
                         }
                         codes[2 * b + e / 8] = wv;
                     }
