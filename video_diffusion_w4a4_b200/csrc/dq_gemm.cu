@@ -17,13 +17,16 @@
 // One persistent kernel template serves both: one CTA per SM walks the
 // 128 x 256 output tiles tile = blockIdx.x + i * gridDim.x.  Warp 0 streams
 // operand tiles with TMA into a 4-stage shared-memory ring that runs on across
-// tiles; warp 1 owns tensor memory and issues the MMAs from one thread; warps
-// 2-9 drain the fp32 accumulator, two warps per 32-lane sub-partition, each
+// tiles; warp 1 owns tensor memory and issues the MMAs from one thread; warp 2
+// copies the block scale factors into tensor memory (main product); warps
+// 3-10 drain the fp32 accumulator, two warps per 32-lane sub-partition, each
 // half of the columns.  The kernel-token product double-buffers its
 // accumulator in tensor memory so the epilogue of one tile overlaps the MMAs
 // of the next; the main product needs tensor-memory columns for the block
-// scale factors, so it keeps one accumulator and instead has its epilogue load
-// the P' rows of a tile into registers while that tile's MMAs run.
+// scale factors (a 48-column slot per ring stage), so it keeps one
+// accumulator: its epilogue warps copy their slice of it into registers,
+// release tensor memory, and then fetch P' and write Y while the next tile's
+// MMAs run.
 #include "dq_common.h"
 #include "dq_internal.h"
 #include "dq_ptx.cuh"
@@ -35,7 +38,7 @@ namespace {
 constexpr int kStages = 4;
 constexpr int kTileM = 128, kTileN = 256;
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kThreads = 96 + 32 * kEpiWarps;   // producer, MMA, scale-factor copies, epilogue
 constexpr uint32_t kABytes = kTileM * 128;  // 128 rows x 128 bytes
 constexpr uint32_t kBBytes = kTileN * 128;  // 256 rows x 128 bytes
 constexpr uint32_t kSFABytes = 4 * 512;     // 128 rows x 4 k-steps of 64
@@ -57,7 +60,7 @@ __host__ __device__ constexpr GSmem g_smem_layout(bool scaled) {
     L.sfb = off;
     if (scaled) off += kStages * kSFBBytes;
     L.bars = off;
-    off += (2 * kStages + 5) * 8;
+    off += (3 * kStages + 6) * 8;
     L.misc = off;
     off += 64;
     L.total = off;
@@ -81,6 +84,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* accf = empty + kStages;   // [2]
     uint64_t* acce = accf + 2;          // [2]
     uint64_t* drain = acce + 2;
+    uint64_t* drain_sf = drain + 1;
+    uint64_t* sfready = drain_sf + 1;   // [kStages]: block scales of a stage are in tensor memory
     uint32_t* tmem_slot = (uint32_t*)(sm + L.misc);
     volatile int* abort_flag = (volatile int*)(sm + L.misc + 8);
 
@@ -92,13 +97,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < kStages; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], kMain ? 2 : 1);   // main: MMA commit + scale-copy commit
+            mbar_init(&sfready[s], 1);
         }
         for (int b = 0; b < 2; b++) {
             mbar_init(&accf[b], 1);
             mbar_init(&acce[b], 32 * kEpiWarps);
         }
         mbar_init(drain, 1);
+        mbar_init(drain_sf, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -163,7 +170,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint32_t id_main = kMain ? idesc_nvfp4(kTileM, kTileN) : idesc_bf16(kTileM, kTileN);
             const uint32_t id_slab = idesc_bf16(kTileM, kTileN);
-            const uint32_t t_sfa = tmem + 256, t_sfb = tmem + 272;
+            // block scales: one 48-column slot per ring stage (16 SFA + 32 SFB columns),
+            // so the copies for one stage never wait on the MMAs still reading another
+            const uint32_t t_sf0 = tmem + 256;
             long long g = 0;
             int it = 0;
             bool alive = true;
@@ -182,14 +191,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint32_t aa = smem_u32(sm + L.a + s * kABytes), bb = smem_u32(sm + L.b + s * kBBytes);
                     if (kMain && i < nk) {
-                        const uint32_t fa = smem_u32(sm + L.sfa + s * kSFABytes);
-                        const uint32_t fb = smem_u32(sm + L.sfb + s * kSFBBytes);
-#pragma unroll
-                        for (int k = 0; k < 4; k++) {
-                            tmem_cp_32x128b_x4(t_sfa + 4 * k, desc_sf(fa + 512 * k));
-                            tmem_cp_32x128b_x4(t_sfb + 8 * k, desc_sf(fb + 512 * k));
-                            tmem_cp_32x128b_x4(t_sfb + 8 * k + 4, desc_sf(fb + kSFBBytes / 2 + 512 * k));
+                        const uint32_t t_sfa = t_sf0 + (uint32_t)(s * 48), t_sfb = t_sfa + 16;
+                        if (!mbar_wait(&sfready[s], (uint32_t)(g / kStages) & 1, abort_flag, p.status, p.budget_ns)) {
+                            alive = false;
+                            break;
                         }
+                        tc_fence_after();
 #pragma unroll
                         for (int k = 0; k < 4; k++)
                             mma_nvfp4(acc, desc_k_sw128(aa + 32 * k), desc_k_sw128(bb + 32 * k), id_main,
@@ -210,9 +217,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(drain, 0, abort_flag, nullptr, p.budget_ns, false);
         }
         __syncwarp();
+    } else if (warp == 2) {
+        // ------------------------------------------------ block-scale copies (main product)
+        // Copies each stage's scale factors from shared into tensor memory (its own
+        // 48-column slot) from a thread of its own, so the copies run ahead of the
+        // MMAs instead of sitting in the MMA thread's in-order stream.
+        if (kMain && lane == 0) {
+            const uint32_t t_sf0 = tmem + 256;
+            long long g = 0;
+            bool alive = true;
+            for (int tile = blockIdx.x; alive && tile < num_tiles; tile += gridDim.x) {
+                for (int i = 0; i < ntot; i++, g++) {
+                    const int s = (int)(g % kStages);
+                    if (!mbar_wait(&full[s], (uint32_t)(g / kStages) & 1, abort_flag, p.status, p.budget_ns)) {
+                        alive = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (i < nk) {
+                        const uint32_t t_sfa = t_sf0 + (uint32_t)(s * 48), t_sfb = t_sfa + 16;
+                        const uint32_t fa = smem_u32(sm + L.sfa + s * kSFABytes);
+                        const uint32_t fb = smem_u32(sm + L.sfb + s * kSFBBytes);
+#pragma unroll
+                        for (int k = 0; k < 4; k++) {
+                            tmem_cp_32x128b_x4(t_sfa + 4 * k, desc_sf(fa + 512 * k));
+                            tmem_cp_32x128b_x4(t_sfb + 8 * k, desc_sf(fb + 512 * k));
+                            tmem_cp_32x128b_x4(t_sfb + 8 * k + 4, desc_sf(fb + kSFBBytes / 2 + 512 * k));
+                        }
+                    }
+                    tc_commit(&sfready[s]);
+                    tc_commit(&empty[s]);
+                }
+            }
+            // no copy may still run when tensor memory is released
+            tc_commit(drain_sf);
+            mbar_wait(drain_sf, 0, abort_flag, nullptr, p.budget_ns, false);
+        }
+        __syncwarp();
     } else {
         // ------------------------------------------------ epilogue warps
-        const int quad = warp & 3, half = (warp - 2) >> 2;
+        const int quad = warp & 3, half = (warp - 3) >> 2;
         const float S_W = reinterpret_cast<const PackedHeader*>(p.packed_w)->S_W;
         const float SS = kMain ? __fmul_rn(__uint_as_float(p.scalars[1]), S_W) : 0.f;
         int it = 0;
@@ -224,45 +268,54 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c_base = n0 + half * 128;
             const uint32_t tacc = tmem + (uint32_t)(buf * 256) + ((uint32_t)(quad * 32) << 16) + (uint32_t)(half * 128);
             if (kMain) {
-                // the P' row segment of this token's cube, fetched while the tile's MMAs run
+                // Pull this warp's 128-column slice of the accumulator into registers and
+                // release tensor memory at once, so the next tile's MMAs start while this
+                // tile's P' rows are fetched and its Y rows are written.
                 long long n = 0, k = 0;
                 if (row_ok) row_to_token(p.g, rho, &n, &k);
-                float4 pf[32];
-                const float4* prow = reinterpret_cast<const float4*>(p.p + (size_t)k * p.Nout + c_base);
-#pragma unroll
-                for (int v = 0; v < 32; v++) pf[v] = row_ok ? __ldg(prow + v) : make_float4(0.f, 0.f, 0.f, 0.f);
                 const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], (uint32_t)use & 1, abort_flag,
                                                                   p.status, p.budget_ns));
                 if (!ok) break;
                 tc_fence_after();
-                uint16_t* yrow = p.Y + (size_t)n * p.Nout + c_base;
+                uint32_t acc[128];
 #pragma unroll
-                for (int c = 0; c < 128; c += 32) {
-                    uint32_t r0[16], r1[16];
-                    tmem_ld_x16(tacc + (uint32_t)c, r0);
-                    tmem_ld_x16(tacc + (uint32_t)c + 16, r1);
-                    tmem_ld_wait();
-                    if (row_ok) {
+                for (int c = 0; c < 128; c += 16)
+                    tmem_ld_x16(tacc + (uint32_t)c, *reinterpret_cast<uint32_t(*)[16]>(&acc[c]));
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&acce[buf]);
+                if (row_ok) {
+                    const float4* prow = reinterpret_cast<const float4*>(p.p + (size_t)k * p.Nout + c_base);
+                    uint16_t* yrow = p.Y + (size_t)n * p.Nout + c_base;
+                    float4 pa[8], pb[8];
+#pragma unroll
+                    for (int v = 0; v < 8; v++) pa[v] = __ldg(prow + v);
+#pragma unroll
+                    for (int c = 0; c < 128; c += 32) {
+                        // software pipeline: the next 32 columns of P' are in flight while these are used
+                        if (c + 32 < 128) {
+#pragma unroll
+                            for (int v = 0; v < 8; v++) pb[v] = __ldg(prow + (c + 32) / 4 + v);
+                        }
                         uint32_t pk[16];
 #pragma unroll
-                        for (int v = 0; v < 16; v += 2) {
-                            const float4 q = pf[(c + v) / 4];
+                        for (int v = 0; v < 32; v += 2) {
+                            const float4 q = pa[v / 4];
                             const float a0 = (v & 2) ? q.z : q.x, a1 = (v & 2) ? q.w : q.y;
-                            pk[v / 2] = (uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(r0[v]), a0)) |
-                                        ((uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(r0[v + 1]), a1)) << 16);
-                            const float4 q2 = pf[(c + 16 + v) / 4];
-                            const float b0 = (v & 2) ? q2.z : q2.x, b1 = (v & 2) ? q2.w : q2.y;
-                            pk[8 + v / 2] =
-                                (uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(r1[v]), b0)) |
-                                ((uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(r1[v + 1]), b1)) << 16);
+                            pk[v / 2] = (uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(acc[c + v]), a0)) |
+                                        ((uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(acc[c + v + 1]), a1))
+                                         << 16);
                         }
                         uint4* dst = reinterpret_cast<uint4*>(yrow + c);
                         dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                         dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
                         dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+#pragma unroll
+                        for (int v = 0; v < 8; v++) pa[v] = pb[v];
                     }
                 }
+                continue;   // tensor memory already released
             } else {
                 const float scale = row_ok ? __fmul_rn(p.s8[rho], S_W) : 0.f;
                 const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], (uint32_t)use & 1, abort_flag,

@@ -28,7 +28,7 @@ constexpr int kMeanStride = 68;  // floats per cube row of the means table (bank
 
 struct QSmem {
     // offsets in bytes from the 1024-aligned dynamic smem base
-    uint32_t x, l1, means, kmax, s8, bars, misc, total;
+    uint32_t x, l1, means, kmax, s8, bars, misc, total;  // means: 2 slots of nw x kMeanStride floats
 };
 
 __host__ __device__ inline QSmem q_smem_layout(int nw, int rank, bool with_l1) {
@@ -39,7 +39,7 @@ __host__ __device__ inline QSmem q_smem_layout(int nw, int rank, bool with_l1) {
     L.l1 = off;
     if (with_l1) off += kQStages * (uint32_t)align_up((size_t)rank * 128, 1024);
     L.means = off;
-    off += (uint32_t)nw * kMeanStride * 4;
+    off += 2u * (uint32_t)nw * kMeanStride * 4;   // two slots: chunk i uses slot i % 2
     L.kmax = off;
     off += (uint32_t)nw * 4;
     L.s8 = off;
@@ -151,9 +151,16 @@ __device__ __forceinline__ float warp_max(float v) {
 }  // namespace
 
 // ------------------------------------------------------------------ a1: statistics + X L1
+//
+// Warps 0-7 compute (thread t: token row t % 128, channel half t / 128 of each
+// 64-channel chunk), warp 8 loads, warp 9 owns tensor memory and issues the
+// X L1 MMAs.  One named barrier per chunk: the means table is double-buffered.
 
-__global__ void __launch_bounds__(192, 1) k_cube_stats(const __grid_constant__ CUtensorMap tm_x,
-                                                        const __grid_constant__ CUtensorMap tm_l1, QuantParams p) {
+constexpr int kQCompute = 256;
+
+__global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_constant__ CUtensorMap tm_x,
+                                                                  const __grid_constant__ CUtensorMap tm_l1,
+                                                                  QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const QSmem L = q_smem_layout(p.nw, p.rank, true);
@@ -162,8 +169,7 @@ __global__ void __launch_bounds__(192, 1) k_cube_stats(const __grid_constant__ C
     uint64_t* done = empty + kQStages;
     uint32_t* tmem_slot = (uint32_t*)(sm + L.misc);
     volatile int* abort_flag = (volatile int*)(sm + L.misc + 8);
-    float* red = (float*)(sm + L.misc + 16);  // 4 floats
-    float* means = (float*)(sm + L.means);
+    float* red = (float*)(sm + L.misc + 16);  // 8 floats
     uint32_t* kmax = (uint32_t*)(sm + L.kmax);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -180,14 +186,14 @@ __global__ void __launch_bounds__(192, 1) k_cube_stats(const __grid_constant__ C
     if (tid == 0) {
         for (int s = 0; s < kQStages; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 129);
+            mbar_init(&empty[s], kQCompute + 1);
         }
         mbar_init(done, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
     for (int j = tid; j < p.nw; j += blockDim.x) kmax[j] = 0u;
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(tmem_slot, tmem_cols);
         tmem_relinquish();
     }
@@ -196,7 +202,7 @@ __global__ void __launch_bounds__(192, 1) k_cube_stats(const __grid_constant__ C
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ---------------- producer
         if (lane == 0) {
             int issued = 0;
@@ -216,7 +222,7 @@ __global__ void __launch_bounds__(192, 1) k_cube_stats(const __grid_constant__ C
             for (int i = (issued > kQStages ? issued - kQStages : 0); i < issued; i++)
                 mbar_wait(&full[i % kQStages], (i / kQStages) & 1, abort_flag, nullptr, p.budget_ns, false);
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ---------------- MMA issuer: U += X_chunk L1_chunk^T (M = 128 rows, N = rank, K = 64)
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(128, p.rank);
@@ -236,20 +242,22 @@ __global__ void __launch_bounds__(192, 1) k_cube_stats(const __grid_constant__ C
         }
         __syncwarp();
     } else {
-        // ---------------- compute warps 0-3
+        // ---------------- compute warps 0-7
+        const int row = tid & 127, half = tid >> 7;
         float damax = 0.f;
         int myj = -1;
         long long myrho = 0, myk = 0;
-        const bool row_ok = box_row(p, B, tid, &myj, &myrho, &myk);
+        const bool row_ok = box_row(p, B, row, &myj, &myrho, &myk);
         const int st = imin(p.g.t, p.g.T - B.t0), sh = imin(p.g.h, p.g.H - B.h0);
         for (int i = 0; i < nchunks; i++) {
-            int s = i % kQStages;
+            const int s = i % kQStages;
+            float* means = (float*)(sm + L.means) + (i & 1) * p.nw * kMeanStride;
             // a failed wait skips the work but keeps the barrier protocol
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (i / kQStages) & 1, abort_flag, p.status,
                                                               p.budget_ns));
             const uint8_t* xs = sm + L.x + s * 16384;
             // kernel tokens of the box's cubes for these 64 channels
-            for (int q = tid; ok && q < p.nw * 8; q += 128) {
+            for (int q = tid; ok && q < p.nw * 8; q += kQCompute) {
                 const int j = q >> 3, g8 = q & 7;
                 float m[8];
                 if (!cube_mean8(p, B, xs, j, g8, st, sh, m)) continue;
@@ -261,13 +269,13 @@ __global__ void __launch_bounds__(192, 1) k_cube_stats(const __grid_constant__ C
                 for (int e = 0; e < 8; e++) am = fmaxf(am, fabsf(m[e]));
                 atomicMax(&kmax[j], __float_as_uint(am));
             }
-            bar_sync(1, 128);
-            // delta amax of this thread's token row
+            bar_sync(1, kQCompute);
+            // delta amax of this thread's half token row
             if (ok && row_ok) {
-                const float* mj = means + myj * kMeanStride;
+                const float* mj = means + myj * kMeanStride + 32 * half;
 #pragma unroll
-                for (int q8 = 0; q8 < 8; q8++) {
-                    uint4 xv = ld_x8_swz(xs, tid, q8);
+                for (int q8 = 0; q8 < 4; q8++) {
+                    uint4 xv = ld_x8_swz(xs, row, 4 * half + q8);
                     float4 m0 = *reinterpret_cast<const float4*>(mj + q8 * 8);
                     float4 m1 = *reinterpret_cast<const float4*>(mj + q8 * 8 + 4);
                     damax = fmaxf(damax, fabsf(__fsub_rn(bf16_lo(xv.x), m0.x)));
@@ -280,17 +288,16 @@ __global__ void __launch_bounds__(192, 1) k_cube_stats(const __grid_constant__ C
                     damax = fmaxf(damax, fabsf(__fsub_rn(bf16_hi(xv.w), m1.w)));
                 }
             }
-            bar_sync(1, 128);  // means table reused next chunk
             mbar_arrive(&empty[s]);
         }
-        // epilogue: U partial rows out of tensor memory
+        // epilogue: U partial rows out of tensor memory (sub-partition warp % 4; this warp's column half)
         const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, p.status, p.budget_ns));
         tc_fence_after();
         if (ok) {
             float* urow = p.u_part + ((size_t)split * p.g.N + (size_t)myrho) * p.rank;
-            for (int c = 0; c < p.rank; c += 16) {
+            for (int c = 16 * half; c < p.rank; c += 32) {
                 uint32_t r[16];
-                tmem_ld_x16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, r);
+                tmem_ld_x16(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)c, r);
                 tmem_ld_wait();
                 if (row_ok) {
 #pragma unroll
@@ -303,12 +310,13 @@ __global__ void __launch_bounds__(192, 1) k_cube_stats(const __grid_constant__ C
         }
         float wm = warp_max(damax);
         if (lane == 0) red[warp] = wm;
-        bar_sync(1, 128);
+        bar_sync(1, kQCompute);
         if (tid == 0) {
-            float bm = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+            float bm = 0.f;
+            for (int w = 0; w < 8; w++) bm = fmaxf(bm, red[w]);
             atomicMax(&p.scalars[0], __float_as_uint(bm));
         }
-        for (int j = tid; j < p.nw; j += 128) {
+        for (int j = tid; j < p.nw; j += kQCompute) {
             int kw = B.bkw * p.nw + j;
             if (kw < p.g.KW) {
                 long long k = ((long long)B.bkt * p.g.KH + B.bkh) * p.g.KW + kw;
@@ -318,22 +326,25 @@ __global__ void __launch_bounds__(192, 1) k_cube_stats(const __grid_constant__ C
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, tmem_cols);
     }
 }
 
 // ------------------------------------------------------------------ a2: encode
+//
+// Warps 0-7 compute (thread t: token row t % 128, channel half t / 128 of each
+// 64-channel chunk, i.e. two FP4 groups of 16), warp 8 loads.
 
-__global__ void __launch_bounds__(160, 1) k_cube_encode(const __grid_constant__ CUtensorMap tm_x, QuantParams p) {
+__global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_constant__ CUtensorMap tm_x,
+                                                                  QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const QSmem L = q_smem_layout(p.nw, p.rank, false);
     uint64_t* full = (uint64_t*)(sm + L.bars);
     uint64_t* empty = full + kQStages;
     volatile int* abort_flag = (volatile int*)(sm + L.misc + 8);
-    float* means = (float*)(sm + L.means);
     float* s8s = (float*)(sm + L.s8);
     float* rs8s = (float*)(sm + L.kmax);   // reciprocals of s8 (the kmax slot is unused in this kernel)
 
@@ -349,7 +360,7 @@ __global__ void __launch_bounds__(160, 1) k_cube_encode(const __grid_constant__ 
     if (tid == 0) {
         for (int s = 0; s < kQStages; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 128);
+            mbar_init(&empty[s], kQCompute);
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -375,7 +386,7 @@ __global__ void __launch_bounds__(160, 1) k_cube_encode(const __grid_constant__ 
     if (box == 0 && split == 0 && tid == 0) p.scalars[1] = __float_as_uint(S);
     __syncthreads();
 
-    if (warp == 4) {
+    if (warp == 8) {
         if (lane == 0) {
             int issued = 0;
             prefetch_tmap(&tm_x);
@@ -391,18 +402,20 @@ __global__ void __launch_bounds__(160, 1) k_cube_encode(const __grid_constant__ 
                 mbar_wait(&full[i % kQStages], (i / kQStages) & 1, abort_flag, nullptr, p.budget_ns, false);
         }
     } else {
+        const int row = tid & 127, half = tid >> 7;
         int myj = -1;
         long long myrho = 0, myk = 0;
-        const bool row_ok = box_row(p, B, tid, &myj, &myrho, &myk);
+        const bool row_ok = box_row(p, B, row, &myj, &myrho, &myk);
         const int st = imin(p.g.t, p.g.T - B.t0), sh = imin(p.g.h, p.g.H - B.h0);
         for (int i = 0; i < nchunks; i++) {
-            int s = i % kQStages;
+            const int s = i % kQStages;
+            float* means = (float*)(sm + L.means) + (i & 1) * p.nw * kMeanStride;
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (i / kQStages) & 1, abort_flag, p.status,
                                                               p.budget_ns));
             const uint8_t* xs = sm + L.x + s * 16384;
             const int c0 = c_base + i * 64;
             // kernel tokens: means, FP8 E4M3 codes with the per-token scale s8 = max|mean| / 448
-            for (int q = tid; ok && q < p.nw * 8; q += 128) {
+            for (int q = tid; ok && q < p.nw * 8; q += kQCompute) {
                 const int j = q >> 3, g8 = q & 7;
                 float m[8];
                 if (!cube_mean8(p, B, xs, j, g8, st, sh, m)) continue;
@@ -427,18 +440,18 @@ __global__ void __launch_bounds__(160, 1) k_cube_encode(const __grid_constant__ 
                 *reinterpret_cast<uint4*>(p.q8_bf16 + (size_t)k * Ci + c0 + 8 * g8) =
                     make_uint4(bfw[0], bfw[1], bfw[2], bfw[3]);
             }
-            bar_sync(1, 128);
-            // delta tokens: FP4 E2M1 with E4M3 group-16 scales under S
+            bar_sync(1, kQCompute);
+            // delta tokens: FP4 E2M1 with E4M3 group-16 scales under S (two groups per thread)
             if (ok && row_ok) {
-                const float* mj = means + myj * kMeanStride;
-                uint32_t codes[8];
+                const float* mj = means + myj * kMeanStride + 32 * half;
+                uint32_t codes[4];
                 uint32_t sc = 0;
 #pragma unroll
-                for (int b = 0; b < 4; b++) {
+                for (int b = 0; b < 2; b++) {
                     float z[16];
 #pragma unroll
                     for (int h = 0; h < 2; h++) {
-                        uint4 xv = ld_x8_swz(xs, tid, 2 * b + h);
+                        uint4 xv = ld_x8_swz(xs, row, 4 * half + 2 * b + h);
                         float4 m0 = *reinterpret_cast<const float4*>(mj + 16 * b + 8 * h);
                         float4 m1 = *reinterpret_cast<const float4*>(mj + 16 * b + 8 * h + 4);
                         z[8 * h + 0] = __fsub_rn(bf16_lo(xv.x), m0.x);
@@ -469,19 +482,18 @@ __global__ void __launch_bounds__(160, 1) k_cube_encode(const __grid_constant__ 
                         codes[2 * b + e / 8] = wv;
                     }
                 }
-                uint8_t* dst = p.dcodes + (size_t)myrho * (Ci / 2) + c0 / 2;
-                reinterpret_cast<uint4*>(dst)[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-                reinterpret_cast<uint4*>(dst)[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-                *reinterpret_cast<uint32_t*>(p.dscales + sf_offset(myrho, c0 / 16, Ci)) = sc;
+                uint8_t* dst = p.dcodes + (size_t)myrho * (Ci / 2) + c0 / 2 + 16 * half;
+                *reinterpret_cast<uint4*>(dst) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                *reinterpret_cast<uint16_t*>(p.dscales + sf_offset(myrho, c0 / 16 + 2 * half, Ci)) = (uint16_t)sc;
             }
-            bar_sync(1, 128);
             mbar_arrive(&empty[s]);
         }
-        // U' = (X L1) / (S_delta S_W) as BF16 hi + lo, slab zero-padded (split 0 only)
+        // U' = (X L1) / (S_delta S_W) as BF16 hi + lo, slab zero-padded (split 0 only; half the columns each)
         if (split == 0 && row_ok) {
             const float SS = __fmul_rn(S, hdr->S_W);
             uint16_t* dst = p.u_hilo + (size_t)myrho * p.slab;
-            for (int c = 0; c < p.rank; c += 2) {
+            const int cpb = p.rank / 2;
+            for (int c = half * cpb; c < (half + 1) * cpb; c += 2) {
                 float u0 = 0.f, u1 = 0.f;
                 for (int sp = 0; sp < p.splits; sp++) {
                     const float* src = p.u_part + ((size_t)sp * p.g.N + (size_t)myrho) * p.rank + c;
@@ -495,7 +507,8 @@ __global__ void __launch_bounds__(160, 1) k_cube_encode(const __grid_constant__ 
                 *reinterpret_cast<uint32_t*>(dst + c) = (uint32_t)h0 | ((uint32_t)h1 << 16);
                 *reinterpret_cast<uint32_t*>(dst + p.rank + c) = (uint32_t)l0 | ((uint32_t)l1 << 16);
             }
-            for (int c = 2 * p.rank; c < p.slab; c += 2) *reinterpret_cast<uint32_t*>(dst + c) = 0u;
+            const int zb = 2 * p.rank, zl = (p.slab - zb) / 2;
+            for (int c = zb + half * zl; c < zb + (half + 1) * zl; c += 2) *reinterpret_cast<uint32_t*>(dst + c) = 0u;
         }
     }
     __syncthreads();
@@ -513,7 +526,7 @@ cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1,
     cudaError_t e = cudaFuncSetAttribute(k_cube_stats, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(p.n_boxes, p.splits);
-    k_cube_stats<<<grid, 192, smem, st>>>(tm_x, tm_l1, p);
+    k_cube_stats<<<grid, kQCompute + 64, smem, st>>>(tm_x, tm_l1, p);
     return cudaGetLastError();
 }
 
@@ -522,7 +535,7 @@ cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const QuantParams& p, cu
     cudaError_t e = cudaFuncSetAttribute(k_cube_encode, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(p.n_boxes, p.splits);
-    k_cube_encode<<<grid, 160, smem, st>>>(tm_x, p);
+    k_cube_encode<<<grid, kQCompute + 32, smem, st>>>(tm_x, p);
     return cudaGetLastError();
 }
 
