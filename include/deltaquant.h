@@ -227,6 +227,29 @@ int dq_linear_forward_host(const void* X_host, int T, int H, int W, int t, int h
                            void* stream);
 
 /*
+ * Forward pass for callers that cannot allocate device memory (code running
+ * under a fixed memory plan such as CUDA-graph capture, processes whose
+ * allocator owns all device memory, embedded callers that may not grow their
+ * footprint).  The paper has no counterpart; this is a property of the library.
+ * Same layer and arguments as dq_linear_forward; the caller still provides X,
+ * the packed weight, the factors and Y.  The scratch workspace is a fixed
+ * 32 MiB array in device memory that the library declares: every GPU that
+ * loads the library holds it until the process exits.  Layers whose
+ * dq_workspace_bytes exceeds 32 MiB are refused with
+ * DQ_ERR_WORKSPACE_TOO_SMALL before anything is launched.  No cudaMalloc,
+ * cudaFree or other allocating call is made.
+ * The first call on a device looks up the array's device address and clears
+ * its status word (a short synchronous call): make that first call before any
+ * stream capture.  All calls share the one array and it keeps the previous
+ * call's contents; calls that may overlap on the GPU (different streams
+ * without ordering) race on it.  Device-side errors (bounded waits that ran
+ * out) are written to the array's status word, which this entry point cannot
+ * read back.
+ */
+int dq_linear_forward_noalloc(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                              const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y, void* stream);
+
+/*
  * Synchronises `stream`, reads the workspace status word into *status, and
  * clears it when `clear` is nonzero.  workspace NULL = the library workspace.
  */

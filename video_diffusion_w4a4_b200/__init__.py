@@ -69,6 +69,7 @@ _SIGS = {
     "dq_linear_forward": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P], _I),
     "dq_linear_forward_ex": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P, _SZ, _I, _P, _P], _I),
     "dq_linear_forward_host": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
+    "dq_linear_forward_noalloc": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P], _I),
     "dq_read_device_status": ([_P, _P, ctypes.POINTER(_I), _I], _I),
     "dq_selftest_bounded_wait": ([_I, _P, ctypes.POINTER(_I)], _I),
     "dq_selftest_convert": ([_P, _LL, _P, _P, _P, _P], _I),
@@ -244,6 +245,12 @@ def dq_linear_forward_host(X_host, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_
            _lib.dq_linear_forward_host(_ptr(X_host), T, H, W, t, h, w, Ci, Co, rank, _ptr(packed_W), _ptr(L1_mma),
                                        _ptr(L2_slab), _ptr(Y_host), _ptr(X_dev), _ptr(Y_dev), _ptr(workspace),
                                        workspace_bytes, _stream(stream)))
+
+
+def dq_linear_forward_noalloc(X, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y, stream=None) -> None:
+    _check("dq_linear_forward_noalloc",
+           _lib.dq_linear_forward_noalloc(_ptr(X), T, H, W, t, h, w, Ci, Co, rank, _ptr(packed_W), _ptr(L1_mma),
+                                          _ptr(L2_slab), _ptr(Y), _stream(stream)))
 
 
 def dq_read_device_status(workspace=None, stream=None, clear: bool = False) -> int:

@@ -21,7 +21,7 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fopenmp,-ffp-contract=off",
           "-I" + os.path.join(ROOT, "include")]
-SOURCES = ["dq_host.cpp", "dq_api.cu", "dq_quant.cu", "dq_gemm.cu", "dq_diag.cu"]
+SOURCES = ["dq_host.cpp", "dq_api.cu", "dq_quant.cu", "dq_gemm.cu", "dq_diag.cu", "dq_noalloc.cu"]
 HEADERS = ["dq_common.h", "dq_internal.h", "dq_ptx.cuh"]
 
 
