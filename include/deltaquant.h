@@ -26,7 +26,8 @@
  *     dq_read_device_status after the stream has been synchronised.
  *   - Inputs are never modified; outputs are fully overwritten.
  *   - Shapes: Ci and Co multiples of 256; rank a multiple of 16 in [16, 128];
- *     1 <= t <= T, 1 <= h <= H, 1 <= w <= W; t*h*w <= 128.  Anything else returns
+ *     1 <= t <= T, 1 <= h <= H, 1 <= w <= W (cubes of any size up to the whole
+ *     lattice, which gives one global kernel token).  Anything else returns
  *     DQ_ERR_UNSUPPORTED_SHAPE.  Device pointers must be 256-byte aligned
  *     (DQ_ERR_ALIGNMENT otherwise).
  */
@@ -59,6 +60,10 @@ typedef enum dq_status {
 
 /* Text for a status code (static storage). */
 const char* dq_status_string(int status);
+
+/* Text of the CUDA runtime error behind the last DQ_ERR_CUDA that an entry
+ * point returned on the calling thread ("" if none); static per-thread storage. */
+const char* dq_last_cuda_error(void);
 
 /* DQ_ABI_VERSION of the loaded library. */
 int dq_abi_version(void);
@@ -170,11 +175,13 @@ int dq_pack_weight(const uint16_t* W, int Co, int Ci, int rank, void* packed, si
  *   u_part     splits x N x rank fp32 partial sums of X L1 (cube-major rows)
  *   u_hilo     N x slab BF16: U' = (X L1)/(S_delta S_W) split as hi + lo
  *   p          K x Co fp32: s8 S_W q8 dqw^T (the per-cube kernel term)
+ *   means      K x Ci fp32 kernel tokens before quantisation, only for cubes
+ *              of more than 128 tokens (size 0 otherwise)
  */
 typedef struct dq_workspace_layout {
     size_t total_bytes;
     size_t off_status, off_scalars, off_kamax, off_s8, off_q8, off_q8_bf16, off_dcodes, off_dscales,
-        off_u_part, off_u_hilo, off_p;
+        off_u_part, off_u_hilo, off_p, off_means;
     long long N, K, N_pad, K_pad;
     int splits, slab;
 } dq_workspace_layout;

@@ -91,7 +91,7 @@ def test_argument_checks_before_any_launch(dq):
     assert call(r=24) == dq.DQ_ERR_UNSUPPORTED_SHAPE
     assert call(r=256, Ci=512, Co=512) == dq.DQ_ERR_UNSUPPORTED_SHAPE
     assert call(t=5) == dq.DQ_ERR_UNSUPPORTED_SHAPE
-    assert call(t=4, h=8, w=8) == dq.DQ_ERR_UNSUPPORTED_SHAPE       # 256 tokens per cube
+    assert call(t=4, h=9, w=8) == dq.DQ_ERR_UNSUPPORTED_SHAPE       # cube taller than the lattice
     assert call(T=0) == dq.DQ_ERR_INVALID_ARG
     assert call(X=0) == dq.DQ_ERR_INVALID_ARG
     assert call(Y=0x50008) == dq.DQ_ERR_ALIGNMENT

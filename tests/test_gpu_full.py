@@ -66,7 +66,7 @@ def test_full_size(env, name):
     _record(name, info)
 
 
-@pytest.mark.parametrize("cube", [(1, 1, 1), (1, 2, 2), (2, 2, 2), (2, 4, 4)])
+@pytest.mark.parametrize("cube", [(1, 1, 1), (1, 2, 2), (2, 2, 2), (2, 4, 4), (21, 30, 52)])
 def test_cube_sweep(env, cube):
     dq, torch = env
     wl = synth.WORKLOADS["wan480p_cube_sweep"].with_cube(cube)
@@ -89,5 +89,6 @@ def test_cube_sweep(env, cube):
     info.update(cube=list(cube), rel_err_gpu=rel(bf16_bits_to_f64(g["Y"][rows])), rel_err_oracle=rel(y_ref),
                 rel_err_plain_nvfp4=rel(y_plain))
     _record("sweep_%d%d%d" % cube, info)
-    if cube != (1, 1, 1):
+    if cube not in ((1, 1, 1), (21, 30, 52)):
+        # local cubes beat plain FP4 (the note's cube-size ablation: the global kernel loses the local structure)
         assert info["rel_err_gpu"] < info["rel_err_plain_nvfp4"], info

@@ -69,6 +69,10 @@ SMALL = [
     ("cube_244", _wl("cube_244", 4, 9, 18, 512, 256, 48, (2, 4, 4))),
     ("cube_418", _wl("cube_418", 6, 5, 20, 256, 256, 16, (4, 1, 8))),
     ("gelu_122", _wl("gelu_122", 2, 12, 40, 1024, 512, 64, (1, 2, 2), gelu=True)),
+    # cubes of more than 128 tokens: kernel tokens from the means kernel, boxes are row segments
+    ("global", _wl("global", 3, 10, 37, 512, 256, 16, (3, 10, 37))),
+    ("big_cube", _wl("big_cube", 5, 18, 21, 256, 256, 16, (2, 8, 16))),
+    ("wide_cube", _wl("wide_cube", 2, 3, 200, 256, 256, 16, (1, 2, 150))),
 ]
 
 

@@ -45,7 +45,7 @@ class dq_packed_layout(ctypes.Structure):
 class dq_workspace_layout(ctypes.Structure):
     _fields_ = [("total_bytes", ctypes.c_size_t)] + [
         (n, ctypes.c_size_t) for n in ("off_status", "off_scalars", "off_kamax", "off_s8", "off_q8", "off_q8_bf16",
-                                       "off_dcodes", "off_dscales", "off_u_part", "off_u_hilo", "off_p")] + [
+                                       "off_dcodes", "off_dscales", "off_u_part", "off_u_hilo", "off_p", "off_means")] + [
         ("N", ctypes.c_longlong), ("K", ctypes.c_longlong), ("N_pad", ctypes.c_longlong), ("K_pad", ctypes.c_longlong),
         ("splits", ctypes.c_int), ("slab", ctypes.c_int)]
 
@@ -53,6 +53,7 @@ class dq_workspace_layout(ctypes.Structure):
 _P, _I, _SZ, _LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
 _SIGS = {
     "dq_status_string": ([_I], ctypes.c_char_p),
+    "dq_last_cuda_error": ([], ctypes.c_char_p),
     "dq_abi_version": ([], _I),
     "dq_cube_count": ([_I] * 6 + [ctypes.POINTER(_LL)], _I),
     "dq_cube_major_row": ([_I] * 6 + [_LL, ctypes.POINTER(_LL), ctypes.POINTER(_LL)], _I),
@@ -83,7 +84,8 @@ for _name, (_args, _res) in _SIGS.items():
 
 class DQError(RuntimeError):
     def __init__(self, fn: str, status: int):
-        super().__init__(f"{fn}: {dq_status_string(status)} ({status})")
+        detail = f" [{_lib.dq_last_cuda_error().decode()}]" if status == DQ_ERR_CUDA else ""
+        super().__init__(f"{fn}: {dq_status_string(status)} ({status}){detail}")
         self.status = status
 
 

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdio.h>
 #include <string.h>
 
 #include <map>
@@ -66,10 +67,22 @@ bool map_x(CUtensorMap* m, const void* X, const Geom& g, int Ci, int bw, int bh,
 
 bool aligned(const void* p) { return ((uintptr_t)p & 255u) == 0; }
 
+// Text of the last CUDA runtime error an entry point of this thread returned DQ_ERR_CUDA for.
+thread_local char g_last_cuda_error[160] = "";
+
+int map_fail(const char* which) {
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed for %s", which);
+    return DQ_ERR_CUDA;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", where, cudaGetErrorString(e));
+    return DQ_ERR_CUDA;
+}
+
 int check_shape(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank) {
     if (T <= 0 || H <= 0 || W <= 0 || t <= 0 || h <= 0 || w <= 0) return DQ_ERR_INVALID_ARG;
     if (t > T || h > H || w > W) return DQ_ERR_UNSUPPORTED_SHAPE;
-    if (t * h * w > 128) return DQ_ERR_UNSUPPORTED_SHAPE;
     if (Ci < 256 || Co < 256 || Ci % 256 || Co % 256) return DQ_ERR_UNSUPPORTED_SHAPE;
     if (rank < 16 || rank > 128 || rank % 16 || rank > Ci || rank > Co) return DQ_ERR_UNSUPPORTED_SHAPE;
     if ((long long)T * H * W >= (1ll << 31)) return DQ_ERR_UNSUPPORTED_SHAPE;
@@ -128,6 +141,7 @@ int dq_workspace_layout_get(int T, int H, int W, int t, int h, int w, int Ci, in
     out->off_u_part = L.off_u_part;
     out->off_u_hilo = L.off_u_hilo;
     out->off_p = L.off_p;
+    out->off_means = L.off_means;
     out->N = L.N;
     out->K = L.K;
     out->N_pad = L.N_pad;
@@ -173,12 +187,26 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
     qp.slab = wl.slab;
     qp.splits = wl.splits;
     qp.chunks_per_split = Ci / 64 / wl.splits;
-    qp.nw = dq::imin(128 / (t * h * w), g.KW);
-    qp.bt = t;
-    qp.bh = h;
-    qp.bw = qp.nw * w;
-    qp.nbw = (int)dq::cdiv(g.KW, qp.nw);
-    qp.n_boxes = g.KT * g.KH * qp.nbw;
+    qp.big = (long long)t * h * w > 128;
+    if (!qp.big) {
+        // boxes of t x h x (nw w) tokens: nw whole cubes side by side along w
+        qp.nw = dq::imin(128 / (t * h * w), g.KW);
+        qp.bt = t;
+        qp.bh = h;
+        qp.bw = qp.nw * w;
+        qp.nbw = (int)dq::cdiv(g.KW, qp.nw);
+        qp.n_boxes = g.KT * g.KH * qp.nbw;
+    } else {
+        // boxes are segments of up to 128 tokens of one (t, h) row inside one cube
+        qp.nw = 1;
+        qp.bt = 1;
+        qp.bh = 1;
+        qp.bw = dq::imin(w, 128);
+        qp.nseg = (int)dq::cdiv(w, 128);
+        qp.nbw = g.KW * qp.nseg;
+        qp.n_boxes = g.T * g.H * qp.nbw;
+        qp.means = (float*)(ws + wl.off_means);
+    }
     qp.status = (int*)(ws + wl.off_status);
     qp.scalars = (uint32_t*)(ws + wl.off_scalars);
     qp.kamax = (uint32_t*)(ws + wl.off_kamax);
@@ -208,36 +236,40 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
     rec(0);
     if (stage_mask & DQ_STAGE_QUANTIZE) {
         CUtensorMap tm_x, tm_l1;
-        if (!map_x(&tm_x, X, g, Ci, qp.bw, qp.bh, qp.bt)) return DQ_ERR_CUDA;
-        if (!map_2d(&tm_l1, L1_mma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, rank, 64, rank)) return DQ_ERR_CUDA;
-        if (cudaMemsetAsync(ws + wl.off_scalars, 0, 16, st) != cudaSuccess) return DQ_ERR_CUDA;
-        if (cudaMemsetAsync(ws + wl.off_kamax, 0, (size_t)g.K * 4, st) != cudaSuccess) return DQ_ERR_CUDA;
-        if (dq::launch_cube_stats(tm_x, tm_l1, qp, st) != cudaSuccess) return DQ_ERR_CUDA;
-        if (dq::launch_cube_encode(tm_x, qp, st) != cudaSuccess) return DQ_ERR_CUDA;
+        cudaError_t e0;
+        if (!map_x(&tm_x, X, g, Ci, qp.bw, qp.bh, qp.bt)) return map_fail("X");
+        if (!map_2d(&tm_l1, L1_mma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, rank, 64, rank)) return map_fail("L1");
+        if ((e0 = cudaMemsetAsync(ws + wl.off_scalars, 0, 16, st)) != cudaSuccess) return cuda_fail(e0, "memset");
+        if ((e0 = cudaMemsetAsync(ws + wl.off_kamax, 0, (size_t)g.K * 4, st)) != cudaSuccess) return cuda_fail(e0, "memset");
+        cudaError_t e;
+        if (qp.big && (e = dq::launch_cube_means_big(tm_x, qp, st)) != cudaSuccess) return cuda_fail(e, "k_cube_means_big");
+        if ((e = dq::launch_cube_stats(tm_x, tm_l1, qp, st)) != cudaSuccess) return cuda_fail(e, "k_cube_stats");
+        if ((e = dq::launch_cube_encode(tm_x, qp, st)) != cudaSuccess) return cuda_fail(e, "k_cube_encode");
     }
     rec(1);
     if (stage_mask & DQ_STAGE_KERNEL_GEMM) {
         CUtensorMap tm_a, tm_b;
         if (!map_2d(&tm_a, ws + wl.off_q8_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, g.K, 64, 128))
-            return DQ_ERR_CUDA;
-        if (!map_2d(&tm_b, pw + pl.off_dqw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, Co, 64, 256)) return DQ_ERR_CUDA;
+            return map_fail("product A");
+        if (!map_2d(&tm_b, pw + pl.off_dqw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, Co, 64, 256)) return map_fail("product B");
         dq::GemmParams p = gp;
         p.M = (int)g.K;
         p.k_stages = Ci / 64;
         p.s8 = qp.s8;
         p.pout = (float*)(ws + wl.off_p);
-        if (dq::launch_kernel_gemm(tm_a, tm_b, p, st) != cudaSuccess) return DQ_ERR_CUDA;
+        cudaError_t e = dq::launch_kernel_gemm(tm_a, tm_b, p, st);
+        if (e != cudaSuccess) return cuda_fail(e, "kernel-token product");
     }
     rec(2);
     if (stage_mask & DQ_STAGE_MAIN_GEMM) {
         CUtensorMap tm_a, tm_b, tm_sa, tm_sb;
         if (!map_2d(&tm_a, ws + wl.off_dcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Ci / 2, g.N, 128, 128))
-            return DQ_ERR_CUDA;
+            return map_fail("product A");
         if (!map_2d(&tm_b, pw + pl.off_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Ci / 2, Co, 128, 256))
-            return DQ_ERR_CUDA;
+            return map_fail("product B");
         if (!map_2d(&tm_sa, ws + wl.off_u_hilo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wl.slab, g.N, 64, 128))
-            return DQ_ERR_CUDA;
-        if (!map_2d(&tm_sb, L2_slab, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wl.slab, Co, 64, 256)) return DQ_ERR_CUDA;
+            return map_fail("slab A");
+        if (!map_2d(&tm_sb, L2_slab, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wl.slab, Co, 64, 256)) return map_fail("slab B");
         dq::GemmParams p = gp;
         p.M = (int)g.N;
         p.k_stages = Ci / 256;
@@ -246,7 +278,8 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
         p.sfb = pw + pl.off_scales;
         p.p = (const float*)(ws + wl.off_p);
         p.Y = (uint16_t*)Y;
-        if (dq::launch_main_gemm(tm_a, tm_b, tm_sa, tm_sb, p, st) != cudaSuccess) return DQ_ERR_CUDA;
+        cudaError_t e = dq::launch_main_gemm(tm_a, tm_b, tm_sa, tm_sb, p, st);
+        if (e != cudaSuccess) return cuda_fail(e, "main product");
     }
     rec(3);
     return DQ_OK;
@@ -305,6 +338,8 @@ int dq_read_device_status(const void* workspace, void* stream, int* status, int 
     *status = h;
     return DQ_OK;
 }
+
+const char* dq_last_cuda_error(void) { return g_last_cuda_error; }
 
 int dq_selftest_bounded_wait(int budget_us, void* stream, int* status) {
     if (!status || budget_us <= 0) return DQ_ERR_INVALID_ARG;

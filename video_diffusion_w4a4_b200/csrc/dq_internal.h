@@ -17,6 +17,9 @@ struct QuantParams {
     int bt, bh, bw;     // box extent in tokens: t x h x (nw w)
     int nbw;            // boxes along w
     int n_boxes;
+    int big;            // cubes of more than 128 tokens: boxes are row segments of one cube,
+    int nseg;           //   nseg segments of up to 128 tokens per cube row; the kernel tokens
+    float* means;       //   come from `means` (K x Ci fp32), written by k_cube_means_big
     int* status;
     uint32_t* scalars;  // [0] bits of max|delta|, [1] S_delta
     uint32_t* kamax;
@@ -54,6 +57,7 @@ size_t quant_smem_bytes(int nw, int rank, bool stats);
 cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
                               cudaStream_t st);
 cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const QuantParams& p, cudaStream_t st);
+cudaError_t launch_cube_means_big(const CUtensorMap& tm_x, const QuantParams& p, cudaStream_t st);
 
 cudaError_t launch_kernel_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmParams& p,
                                cudaStream_t st);

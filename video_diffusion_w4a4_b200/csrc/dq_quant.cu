@@ -39,7 +39,7 @@ __host__ __device__ inline QSmem q_smem_layout(int nw, int rank, bool with_l1) {
     L.l1 = off;
     if (with_l1) off += kQStages * (uint32_t)align_up((size_t)rank * 128, 1024);
     L.means = off;
-    off += 2u * (uint32_t)nw * kMeanStride * 4;   // two slots: chunk i uses slot i % 2
+    off += 2u * (uint32_t)nw * kMeanStride * 4;   // one table per chunk group
     L.kmax = off;
     off += (uint32_t)nw * 4;
     L.s8 = off;
@@ -68,10 +68,28 @@ __device__ __forceinline__ uint4 ld_x8_swz(const uint8_t* xs, int row, int q) {
 struct BoxPos {
     int bkt, bkh, bkw;
     int t0, h0, w0;
+    int dt0, dh0, dw0;   // big cubes: position of the box's first token inside its cube
 };
 
 __device__ __forceinline__ BoxPos box_pos(const QuantParams& p, int b) {
     BoxPos B;
+    if (p.big) {
+        // box b = (token row (tt, hh), cube column kw, segment of up to 128 tokens)
+        const int th = b / p.nbw, rem = b % p.nbw;
+        const int kw = rem / p.nseg, seg = rem % p.nseg;
+        const int tt = th / p.g.H, hh = th % p.g.H;
+        B.bkt = tt / p.g.t;
+        B.bkh = hh / p.g.h;
+        B.bkw = kw;
+        B.t0 = tt;
+        B.h0 = hh;
+        B.dt0 = tt - B.bkt * p.g.t;
+        B.dh0 = hh - B.bkh * p.g.h;
+        B.dw0 = 128 * seg;
+        B.w0 = kw * p.g.w + B.dw0;
+        return B;
+    }
+    B.dt0 = B.dh0 = B.dw0 = 0;
     B.bkw = b % p.nbw;
     int r = b / p.nbw;
     B.bkh = r % p.g.KH;
@@ -86,6 +104,15 @@ __device__ __forceinline__ BoxPos box_pos(const QuantParams& p, int b) {
 __device__ __forceinline__ bool box_row(const QuantParams& p, const BoxPos& B, int row, int* j, long long* rho,
                                         long long* k) {
     const Geom& g = p.g;
+    if (p.big) {
+        const int kw = B.bkw, dw = B.dw0 + row;
+        const int sh = imin(g.h, g.H - B.bkh * g.h), sw = imin(g.w, g.W - kw * g.w);
+        if (row >= p.bw || dw >= sw) return false;
+        *j = 0;
+        *rho = cube_first_row(g, B.bkt, B.bkh, kw) + ((long long)B.dt0 * sh + B.dh0) * sw + dw;
+        *k = ((long long)B.bkt * g.KH + B.bkh) * g.KW + kw;
+        return true;
+    }
     int nrow = p.bt * p.bh * p.bw;
     if (row >= nrow) return false;
     int dt = row / (p.bh * p.bw);
@@ -142,6 +169,14 @@ __device__ __forceinline__ bool cube_mean8(const QuantParams& p, const BoxPos& B
     return true;
 }
 
+// Named barrier of one chunk group (constant barrier ids keep the CTA's barrier count at 3).
+__device__ __forceinline__ void group_sync(int grp) {
+    if (grp == 0)
+        bar_sync(1, 128);
+    else
+        bar_sync(2, 128);
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -157,6 +192,7 @@ __device__ __forceinline__ float warp_max(float v) {
 // X L1 MMAs.  One named barrier per chunk: the means table is double-buffered.
 
 constexpr int kQCompute = 256;
+constexpr int kQGroup = 128;   // compute threads per chunk group
 
 __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_constant__ CUtensorMap tm_x,
                                                                   const __grid_constant__ CUtensorMap tm_l1,
@@ -186,7 +222,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
     if (tid == 0) {
         for (int s = 0; s < kQStages; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kQCompute + 1);
+            mbar_init(&empty[s], kQGroup + 1);   // the chunk's group + the MMA commit
         }
         mbar_init(done, 1);
         *abort_flag = 0;
@@ -242,40 +278,44 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
         }
         __syncwarp();
     } else {
-        // ---------------- compute warps 0-7
-        const int row = tid & 127, half = tid >> 7;
+        // ---------------- compute warps 0-7: two groups of four warps take alternate chunks
+        // (group g: chunks i = g, g+2, ...), each with its own means table and named barrier,
+        // so that one group's waits overlap the other's work.  Thread = one token row.
+        const int grp = tid >> 7, row = tid & 127, half = grp;
         float damax = 0.f;
         int myj = -1;
         long long myrho = 0, myk = 0;
         const bool row_ok = box_row(p, B, row, &myj, &myrho, &myk);
         const int st = imin(p.g.t, p.g.T - B.t0), sh = imin(p.g.h, p.g.H - B.h0);
-        for (int i = 0; i < nchunks; i++) {
+        float* means = (float*)(sm + L.means) + grp * p.nw * kMeanStride;
+        for (int i = grp; i < nchunks; i += 2) {
             const int s = i % kQStages;
-            float* means = (float*)(sm + L.means) + (i & 1) * p.nw * kMeanStride;
             // a failed wait skips the work but keeps the barrier protocol
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (i / kQStages) & 1, abort_flag, p.status,
                                                               p.budget_ns));
             const uint8_t* xs = sm + L.x + s * 16384;
-            // kernel tokens of the box's cubes for these 64 channels
-            for (int q = tid; ok && q < p.nw * 8; q += kQCompute) {
-                const int j = q >> 3, g8 = q & 7;
-                float m[8];
-                if (!cube_mean8(p, B, xs, j, g8, st, sh, m)) continue;
-                float* dst = means + j * kMeanStride + 8 * g8;
-                *reinterpret_cast<float4*>(dst) = make_float4(m[0], m[1], m[2], m[3]);
-                *reinterpret_cast<float4*>(dst + 4) = make_float4(m[4], m[5], m[6], m[7]);
-                float am = 0.f;
+            if (!p.big) {
+                // kernel tokens of the box's cubes for these 64 channels
+                for (int q = row; ok && q < p.nw * 8; q += kQGroup) {
+                    const int j = q >> 3, g8 = q & 7;
+                    float m[8];
+                    if (!cube_mean8(p, B, xs, j, g8, st, sh, m)) continue;
+                    float* dst = means + j * kMeanStride + 8 * g8;
+                    *reinterpret_cast<float4*>(dst) = make_float4(m[0], m[1], m[2], m[3]);
+                    *reinterpret_cast<float4*>(dst + 4) = make_float4(m[4], m[5], m[6], m[7]);
+                    float am = 0.f;
 #pragma unroll
-                for (int e = 0; e < 8; e++) am = fmaxf(am, fabsf(m[e]));
-                atomicMax(&kmax[j], __float_as_uint(am));
+                    for (int e = 0; e < 8; e++) am = fmaxf(am, fabsf(m[e]));
+                    atomicMax(&kmax[j], __float_as_uint(am));
+                }
+                group_sync(grp);
             }
-            bar_sync(1, kQCompute);
-            // delta amax of this thread's half token row
+            // delta amax of this thread's token row (64 channels)
             if (ok && row_ok) {
-                const float* mj = means + myj * kMeanStride + 32 * half;
+                const float* mj = p.big ? p.means + (size_t)myk * p.Ci + c_base + i * 64 : means + myj * kMeanStride;
 #pragma unroll
-                for (int q8 = 0; q8 < 4; q8++) {
-                    uint4 xv = ld_x8_swz(xs, row, 4 * half + q8);
+                for (int q8 = 0; q8 < 8; q8++) {
+                    uint4 xv = ld_x8_swz(xs, row, q8);
                     float4 m0 = *reinterpret_cast<const float4*>(mj + q8 * 8);
                     float4 m1 = *reinterpret_cast<const float4*>(mj + q8 * 8 + 4);
                     damax = fmaxf(damax, fabsf(__fsub_rn(bf16_lo(xv.x), m0.x)));
@@ -288,6 +328,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                     damax = fmaxf(damax, fabsf(__fsub_rn(bf16_hi(xv.w), m1.w)));
                 }
             }
+            if (!p.big) group_sync(grp);   // this group's means table is rewritten next chunk
             mbar_arrive(&empty[s]);
         }
         // epilogue: U partial rows out of tensor memory (sub-partition warp % 4; this warp's column half)
@@ -310,7 +351,9 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
         }
         float wm = warp_max(damax);
         if (lane == 0) red[warp] = wm;
-        bar_sync(1, kQCompute);
+        // barrier 3: ids 1 and 2 belong to the chunk groups, and one group may still be in
+        // its loop when the other gets here (a barrier must not see two thread counts at once)
+        bar_sync(3, kQCompute);
         if (tid == 0) {
             float bm = 0.f;
             for (int w = 0; w < 8; w++) bm = fmaxf(bm, red[w]);
@@ -360,7 +403,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
     if (tid == 0) {
         for (int s = 0; s < kQStages; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kQCompute);
+            mbar_init(&empty[s], kQGroup);   // the chunk's group
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -402,26 +445,36 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                 mbar_wait(&full[i % kQStages], (i / kQStages) & 1, abort_flag, nullptr, p.budget_ns, false);
         }
     } else {
-        const int row = tid & 127, half = tid >> 7;
+        // two groups of four warps take alternate chunks (see k_cube_stats); thread = token row
+        const int grp = tid >> 7, row = tid & 127, half = grp;
         int myj = -1;
         long long myrho = 0, myk = 0;
         const bool row_ok = box_row(p, B, row, &myj, &myrho, &myk);
         const int st = imin(p.g.t, p.g.T - B.t0), sh = imin(p.g.h, p.g.H - B.h0);
-        for (int i = 0; i < nchunks; i++) {
+        float* means = (float*)(sm + L.means) + grp * p.nw * kMeanStride;
+        for (int i = grp; i < nchunks; i += 2) {
             const int s = i % kQStages;
-            float* means = (float*)(sm + L.means) + (i & 1) * p.nw * kMeanStride;
             const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (i / kQStages) & 1, abort_flag, p.status,
                                                               p.budget_ns));
             const uint8_t* xs = sm + L.x + s * 16384;
             const int c0 = c_base + i * 64;
             // kernel tokens: means, FP8 E4M3 codes with the per-token scale s8 = max|mean| / 448
-            for (int q = tid; ok && q < p.nw * 8; q += kQCompute) {
+            // (big cubes: means from the means kernel, encoded once per cube by its first box)
+            const bool enc_q8 = !p.big || (B.dt0 == 0 && B.dh0 == 0 && B.dw0 == 0);
+            for (int q = row; ok && enc_q8 && q < p.nw * 8; q += kQGroup) {
                 const int j = q >> 3, g8 = q & 7;
                 float m[8];
-                if (!cube_mean8(p, B, xs, j, g8, st, sh, m)) continue;
-                float* dst = means + j * kMeanStride + 8 * g8;
-                *reinterpret_cast<float4*>(dst) = make_float4(m[0], m[1], m[2], m[3]);
-                *reinterpret_cast<float4*>(dst + 4) = make_float4(m[4], m[5], m[6], m[7]);
+                if (p.big) {
+                    const float* src = p.means + (size_t)(((long long)B.bkt * p.g.KH + B.bkh) * p.g.KW + B.bkw) * Ci +
+                                       c0 + 8 * g8;
+                    const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
+                    m[0] = a.x; m[1] = a.y; m[2] = a.z; m[3] = a.w; m[4] = b.x; m[5] = b.y; m[6] = b.z; m[7] = b.w;
+                } else {
+                    if (!cube_mean8(p, B, xs, j, g8, st, sh, m)) continue;
+                    float* dst = means + j * kMeanStride + 8 * g8;
+                    *reinterpret_cast<float4*>(dst) = make_float4(m[0], m[1], m[2], m[3]);
+                    *reinterpret_cast<float4*>(dst + 4) = make_float4(m[4], m[5], m[6], m[7]);
+                }
                 const long long k = ((long long)B.bkt * p.g.KH + B.bkh) * p.g.KW + (B.bkw * p.nw + j);
                 const float s8 = s8s[j], rs8 = rs8s[j];
                 uint32_t c[4] = {0u, 0u, 0u, 0u};
@@ -440,18 +493,18 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                 *reinterpret_cast<uint4*>(p.q8_bf16 + (size_t)k * Ci + c0 + 8 * g8) =
                     make_uint4(bfw[0], bfw[1], bfw[2], bfw[3]);
             }
-            bar_sync(1, kQCompute);
-            // delta tokens: FP4 E2M1 with E4M3 group-16 scales under S (two groups per thread)
+            if (!p.big) group_sync(grp);
+            // delta tokens: FP4 E2M1 with E4M3 group-16 scales under S (four groups per thread)
             if (ok && row_ok) {
-                const float* mj = means + myj * kMeanStride + 32 * half;
-                uint32_t codes[4];
+                const float* mj = p.big ? p.means + (size_t)myk * Ci + c0 : means + myj * kMeanStride;
+                uint32_t codes[8];
                 uint32_t sc = 0;
 #pragma unroll
-                for (int b = 0; b < 2; b++) {
+                for (int b = 0; b < 4; b++) {
                     float z[16];
 #pragma unroll
                     for (int h = 0; h < 2; h++) {
-                        uint4 xv = ld_x8_swz(xs, row, 4 * half + 2 * b + h);
+                        uint4 xv = ld_x8_swz(xs, row, 2 * b + h);
                         float4 m0 = *reinterpret_cast<const float4*>(mj + 16 * b + 8 * h);
                         float4 m1 = *reinterpret_cast<const float4*>(mj + 16 * b + 8 * h + 4);
                         z[8 * h + 0] = __fsub_rn(bf16_lo(xv.x), m0.x);
@@ -482,10 +535,12 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                         codes[2 * b + e / 8] = wv;
                     }
                 }
-                uint8_t* dst = p.dcodes + (size_t)myrho * (Ci / 2) + c0 / 2 + 16 * half;
-                *reinterpret_cast<uint4*>(dst) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-                *reinterpret_cast<uint16_t*>(p.dscales + sf_offset(myrho, c0 / 16 + 2 * half, Ci)) = (uint16_t)sc;
+                uint8_t* dst = p.dcodes + (size_t)myrho * (Ci / 2) + c0 / 2;
+                reinterpret_cast<uint4*>(dst)[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                reinterpret_cast<uint4*>(dst)[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+                *reinterpret_cast<uint32_t*>(p.dscales + sf_offset(myrho, c0 / 16, Ci)) = sc;
             }
+            if (!p.big) group_sync(grp);   // this group's means table is rewritten next chunk
             mbar_arrive(&empty[s]);
         }
         // U' = (X L1) / (S_delta S_W) as BF16 hi + lo, slab zero-padded (split 0 only; half the columns each)
@@ -514,7 +569,89 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
     __syncthreads();
 }
 
+// ------------------------------------------------------------------ kernel tokens of big cubes
+//
+// Cubes of more than 128 tokens (up to one global cube over the whole lattice).
+// CTA = 64 channels of one cube: warp 2 streams the cube's rows through an
+// 8-stage TMA ring (the same row-segment boxes as the quantise kernels) and
+// threads 0-63 each keep one channel's fp32 running sum over the tokens in
+// (t,h,w) order (Eq. 1, the same arithmetic as cube_mean8), then divide by the
+// count; the per-cube max |mean| goes to kamax.
+
+constexpr int kMStages = 8;
+
+__global__ void __launch_bounds__(96) k_cube_means_big(const __grid_constant__ CUtensorMap tm_x, QuantParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t* full = (uint64_t*)(sm + kMStages * 16384);
+    uint64_t* empty = full + kMStages;
+    volatile int* abort_flag = (volatile int*)(empty + kMStages);
+    const Geom& g = p.g;
+    const long long k = blockIdx.x;
+    const int c0 = blockIdx.y * 64;
+    const int kw = (int)(k % g.KW), kh = (int)((k / g.KW) % g.KH), kt = (int)(k / ((long long)g.KW * g.KH));
+    const int st = imin(g.t, g.T - kt * g.t), sh = imin(g.h, g.H - kh * g.h), sw = imin(g.w, g.W - kw * g.w);
+    const int nbox = st * sh * p.nseg;
+    const uint32_t box_bytes = (uint32_t)p.bw * 128u;
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        for (int s = 0; s < kMStages; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 64);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (tid >= 64) {
+        if (tid == 64) {
+            int issued = 0;
+            prefetch_tmap(&tm_x);
+            for (int b = 0; b < nbox; b++) {
+                const int s = b % kMStages;
+                if (b >= kMStages && !mbar_wait(&empty[s], ((b / kMStages) - 1) & 1, abort_flag, p.status, p.budget_ns))
+                    break;
+                const int seg = b % p.nseg, dh = (b / p.nseg) % sh, dt = b / (p.nseg * sh);
+                mbar_arrive_expect_tx(&full[s], box_bytes);
+                tma_load_4d(sm + s * 16384, &tm_x, &full[s], c0, kw * g.w + 128 * seg, kh * g.h + dh, kt * g.t + dt);
+                issued = b + 1;
+            }
+            for (int b = (issued > kMStages ? issued - kMStages : 0); b < issued; b++)
+                mbar_wait(&full[b % kMStages], (b / kMStages) & 1, abort_flag, nullptr, p.budget_ns, false);
+        }
+    } else {
+        float acc = 0.f;
+        bool ok = true;
+        for (int b = 0; b < nbox; b++) {
+            const int s = b % kMStages;
+            ok = ok && mbar_wait(&full[s], (b / kMStages) & 1, abort_flag, p.status, p.budget_ns);
+            if (ok) {
+                const int seg = b % p.nseg;
+                const int rows = imin(p.bw, sw - 128 * seg);
+                const uint8_t* xs = sm + s * 16384;
+                for (int r = 0; r < rows; r++) acc = __fadd_rn(acc, ld_x_swz(xs, r, tid));
+            }
+            mbar_arrive(&empty[s]);
+        }
+        const int cnt = st * sh * sw;
+        const float m = ((cnt & (cnt - 1)) == 0) ? __fmul_rn(acc, __frcp_rn((float)cnt)) : __fdiv_rn(acc, (float)cnt);
+        p.means[k * p.Ci + c0 + tid] = m;
+        const float am = warp_max(fabsf(m));
+        if ((tid & 31) == 0) atomicMax(&p.kamax[k], __float_as_uint(am));
+    }
+    __syncthreads();
+}
+
 // ------------------------------------------------------------------ launchers
+
+cudaError_t launch_cube_means_big(const CUtensorMap& tm_x, const QuantParams& p, cudaStream_t st) {
+    const size_t smem = kMStages * 16384 + 2 * kMStages * 8 + 16 + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_cube_means_big, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)p.g.K, (unsigned)(p.Ci / 64));
+    k_cube_means_big<<<grid, 96, smem, st>>>(tm_x, p);
+    return cudaGetLastError();
+}
 
 size_t quant_smem_bytes(int nw, int rank, bool stats) {
     return q_smem_layout(nw, rank, stats).total + 1024;
