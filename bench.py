@@ -15,6 +15,7 @@ the same workload instead.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -64,6 +65,23 @@ def load_peaks():
         return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]), source="measured")
     except Exception:
         return dict(hbm=6650.0, bf16=1590.0, source="fallback")
+
+
+def committed_traffic(wl, stage):
+    """DRAM bytes per launch of `stage` from the committed ncu summary, or None
+    when the workload differs or the kernel's source has changed since the
+    counters were taken."""
+    try:
+        d = json.load(open(os.path.join(ROOT, "profiles", f"traffic_{wl.name}.json")))
+        s = d["stages"][stage]
+        if wl.N != s["full_tokens"]:
+            return None
+        src = open(os.path.join(ROOT, s["source"]), "rb").read()
+        if hashlib.sha256(src).hexdigest() != s["source_sha256"]:
+            return None
+        return float(s["bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 class ClockSampler:
@@ -329,7 +347,7 @@ def main():
         roof = dict(kernel="k_main_gemm" if dom == "main_gemm" else "k_kernel_gemm", bound="tensor", achieved=ach,
                     peak=pk, unit="TFLOP/s")
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = committed_traffic(wl, dom) if tuple(cube) == tuple(synth.WORKLOADS[args.workload].cube) else None
     roof["peak_source"] = ("measured" if peaks["source"] == "measured" else "fallback") + (
         " bf16 x 4 (nominal FP4:BF16)" if roof["unit"] == "TFLOP/s" and dom == "main_gemm" else "")
     stages = {}
@@ -353,7 +371,7 @@ def main():
                 roofline=roof, stages=stages,
                 e2e=dict(value=F * world / (e2e_ms * 1e-3) / 1e12, unit="TFLOP/s",
                          h2d_bytes_per_step=wl.N * wl.Ci * 2, d2h_bytes_per_step=wl.N * wl.Co * 2, ms_per_step=e2e_ms),
-                gpu_launches=4 * args.steps, pack_seconds=pack_s)
+                gpu_launches=(5 if t * h * w > 128 else 4) * args.steps, pack_seconds=pack_s)
     clk_sum = clk.summary()
     if clk_sum:
         line["clocks"] = clk_sum
