@@ -65,6 +65,22 @@ bool map_x(CUtensorMap* m, const void* X, const Geom& g, int Ci, int bw, int bh,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over a block-scale-factor array (layout in include/deltaquant.h) viewed
+// as 256-byte lines: dim 0 the bytes of a line, dim 1 the Ci/32 lines of one
+// 128-row group (4 k-blocks of 64 channels = 2048 bytes = 8 lines per K step of
+// 256 channels), dim 2 the row groups.  Boxes of 8 lines x `groups` row groups.
+bool map_sf(CUtensorMap* m, const void* base, int Ci, uint64_t row_groups, uint32_t groups) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {256, (cuuint64_t)Ci / 32, row_groups};
+    cuuint64_t strides[2] = {256, (cuuint64_t)Ci * 8};
+    cuuint32_t box[3] = {256, 8, groups};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p) { return ((uintptr_t)p & 255u) == 0; }
 
 // Text of the last CUDA runtime error an entry point of this thread returned DQ_ERR_CUDA for.
@@ -251,7 +267,7 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
         CUtensorMap tm_a, tm_b;
         if (!map_2d(&tm_a, ws + wl.off_q8_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, g.K, 64, 128))
             return map_fail("product A");
-        if (!map_2d(&tm_b, pw + pl.off_dqw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, Co, 64, 256)) return map_fail("product B");
+        if (!map_2d(&tm_b, pw + pl.off_dqw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, Co, 64, 128)) return map_fail("product B");
         dq::GemmParams p = gp;
         p.M = (int)g.K;
         p.k_stages = Ci / 64;
@@ -262,23 +278,23 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
     }
     rec(2);
     if (stage_mask & DQ_STAGE_MAIN_GEMM) {
-        CUtensorMap tm_a, tm_b, tm_sa, tm_sb;
+        CUtensorMap tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb;
         if (!map_2d(&tm_a, ws + wl.off_dcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Ci / 2, g.N, 128, 128))
             return map_fail("product A");
-        if (!map_2d(&tm_b, pw + pl.off_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Ci / 2, Co, 128, 256))
+        if (!map_2d(&tm_b, pw + pl.off_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Ci / 2, Co, 128, 128))
             return map_fail("product B");
         if (!map_2d(&tm_sa, ws + wl.off_u_hilo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wl.slab, g.N, 64, 128))
             return map_fail("slab A");
-        if (!map_2d(&tm_sb, L2_slab, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wl.slab, Co, 64, 256)) return map_fail("slab B");
+        if (!map_2d(&tm_sb, L2_slab, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wl.slab, Co, 64, 128)) return map_fail("slab B");
+        if (!map_sf(&tm_fa, ws + wl.off_dscales, Ci, (uint64_t)dq::cdiv(g.N, 128), 1)) return map_fail("delta scales");
+        if (!map_sf(&tm_fb, pw + pl.off_scales, Ci, (uint64_t)(Co / 128), 2)) return map_fail("weight scales");
         dq::GemmParams p = gp;
         p.M = (int)g.N;
         p.k_stages = Ci / 256;
         p.slab_stages = wl.slab / 64;
-        p.sfa = ws + wl.off_dscales;
-        p.sfb = pw + pl.off_scales;
         p.p = (const float*)(ws + wl.off_p);
         p.Y = (uint16_t*)Y;
-        cudaError_t e = dq::launch_main_gemm(tm_a, tm_b, tm_sa, tm_sb, p, st);
+        cudaError_t e = dq::launch_main_gemm(tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p, st);
         if (e != cudaSuccess) return cuda_fail(e, "main product");
     }
     rec(3);

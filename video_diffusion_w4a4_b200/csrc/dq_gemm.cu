@@ -14,19 +14,29 @@
 //       Y[n(rho)][o] = S_delta S_W acc + P'[k(rho)][o] and scatters each
 //       cube-major row back to its (t,h,w) position.
 //
-// One persistent kernel template serves both: one CTA per SM walks the
-// 128 x 256 output tiles tile = blockIdx.x + i * gridDim.x.  Warp 0 streams
-// operand tiles with TMA into a 4-stage shared-memory ring that runs on across
-// tiles; warp 1 owns tensor memory and issues the MMAs from one thread; warp 2
-// copies the block scale factors into tensor memory (main product); warps
-// 3-10 drain the fp32 accumulator, two warps per 32-lane sub-partition, each
-// half of the columns.  The kernel-token product double-buffers its
-// accumulator in tensor memory so the epilogue of one tile overlaps the MMAs
-// of the next; the main product needs tensor-memory columns for the block
-// scale factors (a 48-column slot per ring stage), so it keeps one
-// accumulator: its epilogue warps copy their slice of it into registers,
-// release tensor memory, and then fetch P' and write Y while the next tile's
-// MMAs run.
+// One persistent kernel template serves both.  A cluster of two CTAs (one per
+// SM) owns a 256 x 256 output tile at a time, walking tiles
+// tile = cluster + i * clusters.  Each CTA stages 128 rows of A and 128 rows of
+// B (half the tile's columns) per K step with TMA into its own shared-memory
+// ring, so every operand byte crosses from L2 once per 256 x 256 tile (a
+// third less traffic per FLOP than 128 x 256 tiles on one SM).  The even CTA
+// issues the paired (cta_group::2) MMAs, which read A and B from both CTAs
+// and leave 128 rows of fp32 accumulator in each CTA's tensor memory.  Roles:
+// warp 0 of each CTA streams its operand halves; warp 1 of the even CTA issues
+// the MMAs; warp 2 of the even CTA copies the block scale factors of both CTAs
+// into tensor memory (main product); warps 3-10 of each CTA drain that CTA's
+// accumulator rows, two warps per 32-lane sub-partition, each half of the
+// columns.  The operand copies of both CTAs count on the even CTA's
+// "stage full" barriers; the MMA thread's commits arrive on the "stage empty"
+// and "accumulator full" barriers of both CTAs; the epilogue warps of both
+// CTAs arrive on the even CTA's "accumulator empty" barrier.
+//
+// The kernel-token product double-buffers its accumulator in tensor memory so
+// the epilogue of one tile overlaps the MMAs of the next; the main product
+// needs tensor-memory columns for the block scale factors (a 48-column slot
+// per ring stage), so it keeps one accumulator: its epilogue warps copy their
+// slice into registers, release tensor memory, and then fetch P' and write Y
+// while the next tile's MMAs run.
 #include "dq_common.h"
 #include "dq_internal.h"
 #include "dq_ptx.cuh"
@@ -35,14 +45,17 @@ namespace dq {
 
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kTileM = 128, kTileN = 256;
+constexpr int kTileM = 128;                     // accumulator rows per CTA (256 per pair)
+constexpr int kTileN = 256;                     // output columns per pair tile
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 96 + 32 * kEpiWarps;   // producer, MMA, scale-factor copies, epilogue
-constexpr uint32_t kABytes = kTileM * 128;  // 128 rows x 128 bytes
-constexpr uint32_t kBBytes = kTileN * 128;  // 256 rows x 128 bytes
-constexpr uint32_t kSFABytes = 4 * 512;     // 128 rows x 4 k-steps of 64
-constexpr uint32_t kSFBBytes = 2 * 4 * 512; // 256 rows x 4 k-steps
+constexpr uint32_t kABytes = kTileM * 128;      // 128 rows x 128 bytes
+constexpr uint32_t kBBytes = (kTileN / 2) * 128;  // this CTA's 128 rows of B x 128 bytes
+constexpr uint32_t kSFABytes = 4 * 512;         // 128 rows x 4 k-blocks of 64
+constexpr uint32_t kSFBBytes = 2 * 4 * 512;     // all 256 columns x 4 k-blocks (each CTA holds a copy)
+constexpr uint16_t kPairMask = 0x3;
+
+__host__ __device__ constexpr int g_stages(bool scaled) { return scaled ? 5 : 6; }
 
 struct GSmem {
     uint32_t a, b, sfa, sfb, bars, misc, total;
@@ -50,17 +63,18 @@ struct GSmem {
 
 __host__ __device__ constexpr GSmem g_smem_layout(bool scaled) {
     GSmem L{};
+    const int S = g_stages(scaled);
     uint32_t off = 0;
     L.a = off;
-    off += kStages * kABytes;
+    off += S * kABytes;
     L.b = off;
-    off += kStages * kBBytes;
+    off += S * kBBytes;
     L.sfa = off;
-    if (scaled) off += kStages * kSFABytes;
+    if (scaled) off += S * kSFABytes;
     L.sfb = off;
-    if (scaled) off += kStages * kSFBBytes;
+    if (scaled) off += S * kSFBBytes;
     L.bars = off;
-    off += (3 * kStages + 6) * 8;
+    off += (3 * S + 6) * 8;
     L.misc = off;
     off += 64;
     L.total = off;
@@ -74,35 +88,40 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) { return smem_desc(s
 template <bool kMain>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-           const __grid_constant__ CUtensorMap tm_sa, const __grid_constant__ CUtensorMap tm_sb, GemmParams p) {
+           const __grid_constant__ CUtensorMap tm_sa, const __grid_constant__ CUtensorMap tm_sb,
+           const __grid_constant__ CUtensorMap tm_fa, const __grid_constant__ CUtensorMap tm_fb, GemmParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     constexpr GSmem L = g_smem_layout(kMain);
+    constexpr int S = g_stages(kMain);
     constexpr int kBufs = kMain ? 1 : 2;
-    uint64_t* full = (uint64_t*)(sm + L.bars);
-    uint64_t* empty = full + kStages;
-    uint64_t* accf = empty + kStages;   // [2]
-    uint64_t* acce = accf + 2;          // [2]
+    uint64_t* full = (uint64_t*)(sm + L.bars);   // [S], used in the even CTA
+    uint64_t* empty = full + S;                  // [S], both CTAs
+    uint64_t* sfready = empty + S;               // [S], even CTA: block scales of a stage are in tensor memory
+    uint64_t* accf = sfready + S;                // [2], both CTAs
+    uint64_t* acce = accf + 2;                   // [2], even CTA
     uint64_t* drain = acce + 2;
     uint64_t* drain_sf = drain + 1;
-    uint64_t* sfready = drain_sf + 1;   // [kStages]: block scales of a stage are in tensor memory
     uint32_t* tmem_slot = (uint32_t*)(sm + L.misc);
     volatile int* abort_flag = (volatile int*)(sm + L.misc + 8);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();     // 0: issues the MMAs; 1: its peer
+    const bool lead = rank == 0;
+    const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
     const int num_n = p.Nout / kTileN;
-    const int num_tiles = (int)cdiv(p.M, kTileM) * num_n;
+    const int num_tiles = (int)cdiv(p.M, 2 * kTileM) * num_n;
     const int nk = p.k_stages, ntot = p.k_stages + p.slab_stages;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; s++) {
+        for (int s = 0; s < S; s++) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kMain ? 2 : 1);   // main: MMA commit + scale-copy commit
             mbar_init(&sfready[s], 1);
         }
         for (int b = 0; b < 2; b++) {
             mbar_init(&accf[b], 1);
-            mbar_init(&acce[b], 32 * kEpiWarps);
+            mbar_init(&acce[b], 2 * kEpiWarps);     // one arrival per epilogue warp of each CTA
         }
         mbar_init(drain, 1);
         mbar_init(drain_sf, 1);
@@ -110,81 +129,89 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 512);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_slot, 512);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();   // barriers of both CTAs initialised, tensor memory allocated
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------ producer
+        // ------------------------------------------------ producer (both CTAs)
         if (lane == 0) {
             prefetch_tmap(&tm_a);
             prefetch_tmap(&tm_b);
             if (kMain) {
                 prefetch_tmap(&tm_sa);
                 prefetch_tmap(&tm_sb);
+                prefetch_tmap(&tm_fa);
+                prefetch_tmap(&tm_fb);
             }
-            const int kgroups = p.Ci / 64;
+            const uint32_t full0 = mapa_shared(smem_u32(full), 0);
             long long g = 0;
             bool alive = true;
-            for (int tile = blockIdx.x; alive && tile < num_tiles; tile += gridDim.x) {
-                const int m0 = (tile / num_n) * kTileM, n0 = (tile % num_n) * kTileN;
+            for (int tile = pair; alive && tile < num_tiles; tile += npairs) {
+                const int m0 = (tile / num_n) * (2 * kTileM) + (int)rank * kTileM;   // this CTA's A rows
+                const int n0 = (tile % num_n) * kTileN;                               // the pair's columns
+                const int nb = n0 + (int)rank * (kTileN / 2);                         // this CTA's B rows
                 for (int i = 0; i < ntot; i++, g++) {
-                    const int s = (int)(g % kStages);
-                    if (g >= kStages &&
-                        !mbar_wait(&empty[s], (uint32_t)((g / kStages) - 1) & 1, abort_flag, p.status, p.budget_ns)) {
+                    const int s = (int)(g % S);
+                    if (g >= S && !mbar_wait(&empty[s], (uint32_t)((g / S) - 1) & 1, abort_flag, p.status, p.budget_ns)) {
                         alive = false;
                         break;
                     }
+                    const uint32_t fb = full0 + (uint32_t)(s * 8);
+                    uint8_t* sa = sm + L.a + s * kABytes;
+                    uint8_t* sb = sm + L.b + s * kBBytes;
                     if (!kMain) {
-                        mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
-                        tma_load_2d(sm + L.a + s * kABytes, &tm_a, &full[s], i * 64, m0);
-                        tma_load_2d(sm + L.b + s * kBBytes, &tm_b, &full[s], i * 64, n0);
+                        if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes));
+                        tma_load_2d_pair(sa, &tm_a, fb, i * 64, m0);
+                        tma_load_2d_pair(sb, &tm_b, fb, i * 64, nb);
                     } else if (i < nk) {
-                        mbar_arrive_expect_tx(&full[s], kABytes + kBBytes + kSFABytes + kSFBBytes);
-                        tma_load_2d(sm + L.a + s * kABytes, &tm_a, &full[s], i * 128, m0);
-                        tma_load_2d(sm + L.b + s * kBBytes, &tm_b, &full[s], i * 128, n0);
-                        bulk_load(sm + L.sfa + s * kSFABytes, p.sfa + ((size_t)(m0 >> 7) * kgroups + 4 * i) * 512,
-                                  kSFABytes, &full[s]);
-#pragma unroll
-                        for (int h = 0; h < 2; h++)
-                            bulk_load(sm + L.sfb + s * kSFBBytes + h * (kSFBBytes / 2),
-                                      p.sfb + ((size_t)((n0 >> 7) + h) * kgroups + 4 * i) * 512, kSFBBytes / 2,
-                                      &full[s]);
+                        if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes + kSFABytes + kSFBBytes));
+                        tma_load_2d_pair(sa, &tm_a, fb, i * 128, m0);
+                        tma_load_2d_pair(sb, &tm_b, fb, i * 128, nb);
+                        // scale factors: 4 k-blocks x 512 B per 128-row group = 8 lines of 256 B
+                        tma_load_3d_pair(sm + L.sfa + s * kSFABytes, &tm_fa, fb, 0, 8 * i, m0 >> 7);
+                        tma_load_3d_pair(sm + L.sfb + s * kSFBBytes, &tm_fb, fb, 0, 8 * i, n0 >> 7);
                     } else {
-                        mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
-                        tma_load_2d(sm + L.a + s * kABytes, &tm_sa, &full[s], (i - nk) * 64, m0);
-                        tma_load_2d(sm + L.b + s * kBBytes, &tm_sb, &full[s], (i - nk) * 64, n0);
+                        if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes));
+                        tma_load_2d_pair(sa, &tm_sa, fb, (i - nk) * 64, m0);
+                        tma_load_2d_pair(sb, &tm_sb, fb, (i - nk) * 64, nb);
                     }
                 }
             }
-            // every issued load lands before shared memory is released
-            for (long long q = (g > kStages ? g - kStages : 0); q < g; q++)
-                mbar_wait(&full[q % kStages], (uint32_t)(q / kStages) & 1, abort_flag, nullptr, p.budget_ns, false);
+            // every issued copy lands before shared memory is released: the even CTA
+            // waits for its last stages to fill (they count both CTAs' bytes), the odd
+            // CTA for the MMAs that consumed its last stages
+            for (long long q = (g > S ? g - S : 0); q < g; q++) {
+                if (lead)
+                    mbar_wait(&full[q % S], (uint32_t)(q / S) & 1, abort_flag, nullptr, p.budget_ns, false);
+                else
+                    mbar_wait(&empty[q % S], (uint32_t)(q / S) & 1, abort_flag, nullptr, p.budget_ns);
+            }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t id_main = kMain ? idesc_nvfp4(kTileM, kTileN) : idesc_bf16(kTileM, kTileN);
-            const uint32_t id_slab = idesc_bf16(kTileM, kTileN);
+        // ------------------------------------------------ MMA issuer (even CTA)
+        if (lead && lane == 0) {
+            const uint32_t id_main = kMain ? idesc_nvfp4(2 * kTileM, kTileN) : idesc_bf16(2 * kTileM, kTileN);
+            const uint32_t id_slab = idesc_bf16(2 * kTileM, kTileN);
             // block scales: one 48-column slot per ring stage (16 SFA + 32 SFB columns),
             // so the copies for one stage never wait on the MMAs still reading another
             const uint32_t t_sf0 = tmem + 256;
             long long g = 0;
             int it = 0;
             bool alive = true;
-            for (int tile = blockIdx.x; alive && tile < num_tiles; tile += gridDim.x, it++) {
+            for (int tile = pair; alive && tile < num_tiles; tile += npairs, it++) {
                 const int buf = it % kBufs, use = it / kBufs;
                 const uint32_t acc = tmem + (uint32_t)(buf * 256);
                 if (use > 0 && !mbar_wait(&acce[buf], (uint32_t)(use - 1) & 1, abort_flag, p.status, p.budget_ns))
                     break;
                 tc_fence_after();
                 for (int i = 0; i < ntot; i++, g++) {
-                    const int s = (int)(g % kStages);
-                    if (!mbar_wait(&full[s], (uint32_t)(g / kStages) & 1, abort_flag, p.status, p.budget_ns)) {
+                    const int s = (int)(g % S);
+                    if (!mbar_wait(&full[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
                         alive = false;
                         break;
                     }
@@ -192,44 +219,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t aa = smem_u32(sm + L.a + s * kABytes), bb = smem_u32(sm + L.b + s * kBBytes);
                     if (kMain && i < nk) {
                         const uint32_t t_sfa = t_sf0 + (uint32_t)(s * 48), t_sfb = t_sfa + 16;
-                        if (!mbar_wait(&sfready[s], (uint32_t)(g / kStages) & 1, abort_flag, p.status, p.budget_ns)) {
+                        if (!mbar_wait(&sfready[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
                             alive = false;
                             break;
                         }
                         tc_fence_after();
 #pragma unroll
                         for (int k = 0; k < 4; k++)
-                            mma_nvfp4(acc, desc_k_sw128(aa + 32 * k), desc_k_sw128(bb + 32 * k), id_main,
-                                      t_sfa + 4 * k, t_sfb + 8 * k, (i | k) != 0);
+                            mma_nvfp4_pair(acc, desc_k_sw128(aa + 32 * k), desc_k_sw128(bb + 32 * k), id_main,
+                                           t_sfa + 4 * k, t_sfb + 8 * k, (i | k) != 0);
                     } else {
                         const uint32_t id = kMain ? id_slab : id_main;
 #pragma unroll
                         for (int k = 0; k < 4; k++)
-                            mma_bf16(acc, desc_k_sw128(aa + 32 * k), desc_k_sw128(bb + 32 * k), id,
-                                     (kMain || (i | k) != 0) ? 1u : 0u);
+                            mma_bf16_pair(acc, desc_k_sw128(aa + 32 * k), desc_k_sw128(bb + 32 * k), id,
+                                          (kMain || (i | k) != 0) ? 1u : 0u);
                     }
-                    tc_commit(&empty[s]);
+                    tc_commit_pair_both(&empty[s], kPairMask);
                 }
-                if (alive) tc_commit(&accf[buf]);
+                if (alive) tc_commit_pair_both(&accf[buf], kPairMask);
             }
             // no MMA may still run when tensor memory is released
-            tc_commit(drain);
+            tc_commit_pair(drain);
             mbar_wait(drain, 0, abort_flag, nullptr, p.budget_ns, false);
         }
         __syncwarp();
     } else if (warp == 2) {
-        // ------------------------------------------------ block-scale copies (main product)
-        // Copies each stage's scale factors from shared into tensor memory (its own
-        // 48-column slot) from a thread of its own, so the copies run ahead of the
-        // MMAs instead of sitting in the MMA thread's in-order stream.
-        if (kMain && lane == 0) {
+        // ------------------------------------------------ block-scale copies (main product, even CTA)
+        // One copy instruction moves each CTA's scale factors from its own shared
+        // memory into its own tensor memory; a thread of its own lets the copies
+        // run ahead of the MMAs instead of sitting in the MMA thread's stream.
+        if (kMain && lead && lane == 0) {
             const uint32_t t_sf0 = tmem + 256;
             long long g = 0;
             bool alive = true;
-            for (int tile = blockIdx.x; alive && tile < num_tiles; tile += gridDim.x) {
+            for (int tile = pair; alive && tile < num_tiles; tile += npairs) {
                 for (int i = 0; i < ntot; i++, g++) {
-                    const int s = (int)(g % kStages);
-                    if (!mbar_wait(&full[s], (uint32_t)(g / kStages) & 1, abort_flag, p.status, p.budget_ns)) {
+                    const int s = (int)(g % S);
+                    if (!mbar_wait(&full[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
                         alive = false;
                         break;
                     }
@@ -240,29 +267,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t fb = smem_u32(sm + L.sfb + s * kSFBBytes);
 #pragma unroll
                         for (int k = 0; k < 4; k++) {
-                            tmem_cp_32x128b_x4(t_sfa + 4 * k, desc_sf(fa + 512 * k));
-                            tmem_cp_32x128b_x4(t_sfb + 8 * k, desc_sf(fb + 512 * k));
-                            tmem_cp_32x128b_x4(t_sfb + 8 * k + 4, desc_sf(fb + kSFBBytes / 2 + 512 * k));
+                            tmem_cp_pair_32x128b_x4(t_sfa + 4 * k, desc_sf(fa + 512 * k));
+                            tmem_cp_pair_32x128b_x4(t_sfb + 8 * k, desc_sf(fb + 512 * k));
+                            tmem_cp_pair_32x128b_x4(t_sfb + 8 * k + 4, desc_sf(fb + kSFBBytes / 2 + 512 * k));
                         }
                     }
-                    tc_commit(&sfready[s]);
-                    tc_commit(&empty[s]);
+                    tc_commit_pair(&sfready[s]);
+                    tc_commit_pair_both(&empty[s], kPairMask);
                 }
             }
             // no copy may still run when tensor memory is released
-            tc_commit(drain_sf);
+            tc_commit_pair(drain_sf);
             mbar_wait(drain_sf, 0, abort_flag, nullptr, p.budget_ns, false);
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------ epilogue warps
+        // ------------------------------------------------ epilogue warps (both CTAs)
         const int quad = warp & 3, half = (warp - 3) >> 2;
         const float S_W = reinterpret_cast<const PackedHeader*>(p.packed_w)->S_W;
         const float SS = kMain ? __fmul_rn(__uint_as_float(p.scalars[1]), S_W) : 0.f;
+        const uint32_t acce0 = mapa_shared(smem_u32(acce), 0);
         int it = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, it++) {
+        for (int tile = pair; tile < num_tiles; tile += npairs, it++) {
             const int buf = it % kBufs, use = it / kBufs;
-            const int m0 = (tile / num_n) * kTileM, n0 = (tile % num_n) * kTileN;
+            const int m0 = (tile / num_n) * (2 * kTileM) + (int)rank * kTileM;
+            const int n0 = (tile % num_n) * kTileN;
             const long long rho = (long long)m0 + quad * 32 + lane;
             const bool row_ok = rho < p.M;
             const int c_base = n0 + half * 128;
@@ -283,7 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld_x16(tacc + (uint32_t)c, *reinterpret_cast<uint32_t(*)[16]>(&acc[c]));
                 tmem_ld_wait();
                 tc_fence_before();
-                mbar_arrive(&acce[buf]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acce0 + (uint32_t)(buf * 8));
                 if (row_ok) {
                     const float4* prow = reinterpret_cast<const float4*>(p.p + (size_t)k * p.Nout + c_base);
                     uint16_t* yrow = p.Y + (size_t)n * p.Nout + c_base;
@@ -315,7 +345,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int v = 0; v < 8; v++) pa[v] = pb[v];
                     }
                 }
-                continue;   // tensor memory already released
             } else {
                 const float scale = row_ok ? __fmul_rn(p.s8[rho], S_W) : 0.f;
                 const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], (uint32_t)use & 1, abort_flag,
@@ -341,53 +370,72 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
+                // tensor-memory buffer free for the next tile
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acce0 + (uint32_t)(buf * 8));
             }
-            // tensor-memory buffer free for the next tile
-            tc_fence_before();
-            mbar_arrive(&acce[buf]);
         }
     }
+    // Neither CTA leaves, nor frees tensor memory, while its peer may still
+    // touch its shared memory, barriers or tensor memory.
+    __syncwarp();
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc_pair(tmem, 512);
     }
 }
 
 // ------------------------------------------------------------------ launchers
 
 namespace {
-int sm_count() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
+
+template <bool kMain>
+cudaError_t launch_pairs(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_sa,
+                         const CUtensorMap& tm_sb, const CUtensorMap& tm_fa, const CUtensorMap& tm_fb,
+                         const GemmParams& p, cudaStream_t st) {
+    constexpr size_t smem = g_smem_layout(kMain).total + 1024;
+    cudaError_t e = cudaFuncSetAttribute(k_gemm<kMain>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int tiles = (int)cdiv(p.M, 2 * kTileM) * (p.Nout / kTileN);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // persistent: as many pairs as can be resident at once (one CTA per SM)
+    static int mp = 0;
+    if (mp == 0) {
+        cfg.gridDim = dim3(2 * tiles);
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, k_gemm<kMain>, &cfg);
+        if (e != cudaSuccess) return e;
+        if (n <= 0) return cudaErrorInvalidConfiguration;
+        mp = n;
     }
-    return n;
+    cfg.gridDim = dim3(2 * imin(tiles, mp));
+    return cudaLaunchKernelEx(&cfg, k_gemm<kMain>, tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p);
 }
+
 }  // namespace
 
 cudaError_t launch_kernel_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmParams& p,
                                cudaStream_t st) {
-    constexpr size_t smem = g_smem_layout(false).total + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int tiles = (int)cdiv(p.M, kTileM) * (p.Nout / kTileN);
-    k_gemm<false><<<imin(tiles, sm_count()), kThreads, smem, st>>>(tm_a, tm_b, tm_a, tm_b, p);
-    return cudaGetLastError();
+    return launch_pairs<false>(tm_a, tm_b, tm_a, tm_b, tm_a, tm_b, p, st);
 }
 
 cudaError_t launch_main_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_sa,
-                             const CUtensorMap& tm_sb, const GemmParams& p, cudaStream_t st) {
-    constexpr size_t smem = g_smem_layout(true).total + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int tiles = (int)cdiv(p.M, kTileM) * (p.Nout / kTileN);
-    k_gemm<true><<<imin(tiles, sm_count()), kThreads, smem, st>>>(tm_a, tm_b, tm_sa, tm_sb, p);
-    return cudaGetLastError();
+                             const CUtensorMap& tm_sb, const CUtensorMap& tm_fa, const CUtensorMap& tm_fb,
+                             const GemmParams& p, cudaStream_t st) {
+    return launch_pairs<true>(tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p, st);
 }
 
 }  // namespace dq

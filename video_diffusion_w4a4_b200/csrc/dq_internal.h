@@ -41,8 +41,6 @@ struct GemmParams {
     int Ci;
     int k_stages;        // main-operand K stages
     int slab_stages;     // extra BF16 K stages (low-rank slab), main product only
-    const uint8_t* sfa;  // delta scales (scale-factor layout, M rows)
-    const uint8_t* sfb;  // weight scales (scale-factor layout, Co rows)
     const float* p;      // per-cube kernel term, K x Co fp32 (main product)
     const uint32_t* scalars;
     const uint8_t* packed_w;
@@ -62,7 +60,8 @@ cudaError_t launch_cube_means_big(const CUtensorMap& tm_x, const QuantParams& p,
 cudaError_t launch_kernel_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmParams& p,
                                cudaStream_t st);
 cudaError_t launch_main_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_sa,
-                             const CUtensorMap& tm_sb, const GemmParams& p, cudaStream_t st);
+                             const CUtensorMap& tm_sb, const CUtensorMap& tm_fa, const CUtensorMap& tm_fb,
+                             const GemmParams& p, cudaStream_t st);
 
 cudaError_t launch_selftest_wait(int* status, uint64_t budget_ns, cudaStream_t st);
 cudaError_t launch_selftest_divide(long long n, uint64_t seed, unsigned long long* mismatches, float* first,
