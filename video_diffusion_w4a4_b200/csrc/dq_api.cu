@@ -206,12 +206,18 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
     qp.big = (long long)t * h * w > 128;
     if (!qp.big) {
         // boxes of t x h x (nw w) tokens: nw whole cubes side by side along w
-        qp.nw = dq::imin(128 / (t * h * w), g.KW);
+        // (as many as fit in 128 tokens, then evened out over the boxes of a cube row)
+        const int nw_max = dq::imin(128 / (t * h * w), g.KW);
+        qp.nbw = (int)dq::cdiv(g.KW, nw_max);
+        qp.nw = (int)dq::cdiv(g.KW, qp.nbw);
         qp.bt = t;
         qp.bh = h;
         qp.bw = qp.nw * w;
-        qp.nbw = (int)dq::cdiv(g.KW, qp.nw);
         qp.n_boxes = g.KT * g.KH * qp.nbw;
+        // 16 consecutive cube-major rows touch at most ceil(15 / n) + 1 cubes of n tokens;
+        // the boxes of the last slab in t or row in h hold the cubes cut shortest
+        const int n_min = (T - (g.KT - 1) * t) * (H - (g.KH - 1) * h) * w;
+        qp.tbl_rows = dq::imin(16, (int)dq::cdiv(15, n_min) + 1);
     } else {
         // boxes are segments of up to 128 tokens of one (t, h) row inside one cube
         qp.nw = 1;
@@ -222,6 +228,7 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
         qp.nbw = g.KW * qp.nseg;
         qp.n_boxes = g.T * g.H * qp.nbw;
         qp.means = (float*)(ws + wl.off_means);
+        qp.tbl_rows = 1;
     }
     qp.status = (int*)(ws + wl.off_status);
     qp.scalars = (uint32_t*)(ws + wl.off_scalars);

@@ -119,12 +119,13 @@ DQ_HD PackedLayout packed_layout(int Co, int Ci, int rank) {
     return L;
 }
 
-// Number of splits of the channel dimension in the cube-quantise kernels
-// (more work items than SMs for the small-Ci layers; deterministic partial
-// sums of X L1, reduced in a fixed order).
+// Number of splits of the channel dimension in the cube-quantise kernels:
+// work items are (box, split), so more splits even out the last wave of the
+// persistent grid; each split leaves its own partial sums of X L1, reduced in
+// a fixed order.
 DQ_HD int quant_splits(int Ci) {
     int chunks = Ci / 64;
-    int s = 4;
+    int s = 8;
     while (s > 1 && chunks % s) s--;
     return s;
 }

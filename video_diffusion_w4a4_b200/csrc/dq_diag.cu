@@ -38,10 +38,11 @@ __device__ __forceinline__ uint64_t mix64d(uint64_t x) {
     return x ^ (x >> 31);
 }
 
-// Compares the quantisers' quotient path (correctly rounded reciprocal, one
-// product, one FMA correction) with IEEE division, bit for bit, on operand
-// pairs drawn from a counter-based hash: a with exponent in [-40, 12] (and
-// exact zeros of either sign), b > 0 with exponent in [-30, 12].
+// Compares the quantisers' quotient paths (correctly rounded reciprocal, one
+// product, one FMA correction; div_pos, the negated div_neg and its packed
+// pair form f2_div_neg on (a, -a)) with IEEE division, bit for bit, on operand pairs drawn from a counter-based hash: a
+// with exponent in [-40, 12] (and exact zeros of either sign), b > 0 with
+// exponent in [-30, 12].  A pair counts once if either path differs.
 __global__ void k_selftest_divide(long long n, uint64_t seed, unsigned long long* mismatches, float* first) {
     long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long stride = (long long)gridDim.x * blockDim.x;
@@ -55,8 +56,15 @@ __global__ void k_selftest_divide(long long n, uint64_t seed, unsigned long long
         if (((h1 >> 41) & 1023u) == 0) a = __uint_as_float(sa);          // signed zeros
         float b = __uint_as_float(((uint32_t)(eb + 127) << 23) | mb);
         float q0 = __fdiv_rn(a, b);
-        float q1 = div_pos(a, b, __frcp_rn(b));
-        if (__float_as_uint(q0) != __float_as_uint(q1)) {
+        const float rb = __frcp_rn(b);
+        float q1 = div_pos(a, b, rb);
+        float q2 = -div_neg(a, b, rb);
+        float q3, q4;
+        f2_unpack(f2_div_neg(f2_pack(a, -a), f2_pack(b, b), f2_pack(-rb, -rb)), q3, q4);
+        q3 = -q3;
+        const float q5 = __fdiv_rn(-a, b);
+        if (__float_as_uint(q0) != __float_as_uint(q1) || __float_as_uint(q0) != __float_as_uint(q2) ||
+            __float_as_uint(q0) != __float_as_uint(q3) || __float_as_uint(q5) != __float_as_uint(-q4)) {
             if (atomicAdd(mismatches, 1ull) == 0ull) {
                 first[0] = a;
                 first[1] = b;

@@ -17,6 +17,7 @@ struct QuantParams {
     int bt, bh, bw;     // box extent in tokens: t x h x (nw w)
     int nbw;            // boxes along w
     int n_boxes;
+    int tbl_rows;       // rows of each compute warp's table of means
     int big;            // cubes of more than 128 tokens: boxes are row segments of one cube,
     int nseg;           //   nseg segments of up to 128 tokens per cube row; the kernel tokens
     float* means;       //   come from `means` (K x Ci fp32), written by k_cube_means_big
@@ -51,7 +52,7 @@ struct GemmParams {
     uint64_t budget_ns;
 };
 
-size_t quant_smem_bytes(int nw, int rank, bool stats);
+size_t quant_smem_bytes(int rank, bool stats, int tbl_rows);
 cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
                               cudaStream_t st);
 cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const QuantParams& p, cudaStream_t st);

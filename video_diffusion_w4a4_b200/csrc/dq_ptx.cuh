@@ -385,6 +385,95 @@ __device__ __forceinline__ float div_pos(float a, float b, float rb) {
     return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(a) & 0x80000000u));
 }
 
+// -fl32(a / b) for b > 0 from rb = fl32(1 / b): the same Markstein step as
+// div_pos with every operand of the correction negated, which returns the
+// correctly rounded quotient negated, zero quotients included (-(+0) for
+// a = +0, -(-0) for a = -0) without a sign fix-up.  Valid while the quotient
+// does not underflow.
+__device__ __forceinline__ float div_neg(float a, float b, float rb) {
+    const float q = __fmul_rn(a, rb);
+    const float r = __fmaf_rn(-q, b, a);
+    return __fmaf_rn(-r, rb, -q);
+}
+
+// ------------------------------------------------------------------ packed fp32 pairs
+//
+// sm_100 executes add / sub / mul / fma on two fp32 values held in one 64-bit
+// register pair, each correctly rounded as the scalar instruction would be.
+
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// a * b + c, one rounding per element
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// The two BF16 values of a 32-bit word (low half first) as an exact fp32 pair.
+__device__ __forceinline__ uint64_t f2_from_bf16x2(uint32_t w) {
+    return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// -fl32(a / b) for both elements of the pair a, b > 0 the same for both,
+// b2 = (b, b), nrb2 = (-rb, -rb) with rb = fl32(1 / b).  With p = a (-rb) =
+// -fl32(a rb), r = p b + a (exact) and p + r (-rb), every rounding is the one
+// of div_neg, so the result is div_neg's bit for bit (zero quotients keep
+// their sign the same way).
+__device__ __forceinline__ uint64_t f2_div_neg(uint64_t a, uint64_t b2, uint64_t nrb2) {
+    const uint64_t p = f2_mul(a, nrb2);
+    const uint64_t r = f2_fma(p, b2, a);
+    return f2_fma(r, nrb2, p);
+}
+
+// max(|a|, |b|, |c|)
+__device__ __forceinline__ float max3_abs(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(fabsf(a)), "f"(fabsf(b)), "f"(fabsf(c)));
+    return r;
+}
+
+// Eight fp32 -> eight E2M1 codes in one word (value 2i in the low nibble of
+// byte i), round to nearest even, saturating.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return r;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 

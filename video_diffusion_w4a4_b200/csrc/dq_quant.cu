@@ -12,6 +12,17 @@
 // channels straight from the flattened (t,h,w) layout, so that every box
 // holds nw whole cubes.  The two passes exist because the per-tensor delta
 // scale needs the amax of every delta before any delta can be encoded.
+//
+// Work item = (box, channel split): the box's tokens over Ci / splits
+// channels (chunks of 64).  The kernels are persistent: each CTA walks items
+// it = blockIdx.x + n * gridDim.x and one producer thread streams all their
+// chunks through one TMA ring.  The box's tokens are listed in cube-major
+// order and every compute warp owns 16 consecutive rows of that list: it
+// first forms the means of the cubes its rows touch (lane = cube x 8
+// channels) in a table of its own, then encodes its rows (two lanes per row,
+// 32 channels each).  A cube that spans two warps has its mean formed by
+// both (the same sequential sum), so the compute warps never wait on one
+// another.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -24,29 +35,29 @@ namespace dq {
 namespace {
 
 constexpr int kQStages = 4;
-constexpr int kMeanStride = 68;  // floats per cube row of the means table (bank spread)
+constexpr int kQWarps = 8;                 // compute warps
+constexpr int kQCompute = 32 * kQWarps;
+
+constexpr int kMeanStride = 68;            // floats per row of a warp's table of means (bank spread)
 
 struct QSmem {
     // offsets in bytes from the 1024-aligned dynamic smem base
-    uint32_t x, l1, means, kmax, s8, bars, misc, total;  // means: 2 slots of nw x kMeanStride floats
+    uint32_t x, l1, tbl, bars, misc, total;
 };
 
-__host__ __device__ inline QSmem q_smem_layout(int nw, int rank, bool with_l1) {
+// tbl_rows: rows of each compute warp's table of means (the cube slots that 16
+// consecutive cube-major rows can touch)
+__host__ __device__ inline QSmem q_smem_layout(int rank, bool with_l1, int tbl_rows) {
     QSmem L;
     uint32_t off = 0;
     L.x = off;
     off += kQStages * 16384;
     L.l1 = off;
     if (with_l1) off += kQStages * (uint32_t)align_up((size_t)rank * 128, 1024);
-    L.means = off;
-    off += 2u * (uint32_t)nw * kMeanStride * 4;   // one table per chunk group
-    L.kmax = off;
-    off += (uint32_t)nw * 4;
-    L.s8 = off;
-    off += (uint32_t)nw * 4;
-    off = (uint32_t)align_up(off, 16);
+    L.tbl = off;
+    off += (uint32_t)kQWarps * tbl_rows * kMeanStride * 4;
     L.bars = off;
-    off += (2 * kQStages + 2) * 8;
+    off += (2 * kQStages + 6) * 8;
     L.misc = off;
     off += 64;
     L.total = off;
@@ -100,17 +111,14 @@ __device__ __forceinline__ BoxPos box_pos(const QuantParams& p, int b) {
     return B;
 }
 
-// Row `row` of a box -> validity, cube slot j, cube-major row rho, cube index k.
-__device__ __forceinline__ bool box_row(const QuantParams& p, const BoxPos& B, int row, int* j, long long* rho,
-                                        long long* k) {
+// Row `row` of a box -> validity, cube-major row rho.
+__device__ __forceinline__ bool box_row(const QuantParams& p, const BoxPos& B, int row, long long* rho) {
     const Geom& g = p.g;
     if (p.big) {
         const int kw = B.bkw, dw = B.dw0 + row;
         const int sh = imin(g.h, g.H - B.bkh * g.h), sw = imin(g.w, g.W - kw * g.w);
         if (row >= p.bw || dw >= sw) return false;
-        *j = 0;
         *rho = cube_first_row(g, B.bkt, B.bkh, kw) + ((long long)B.dt0 * sh + B.dh0) * sw + dw;
-        *k = ((long long)B.bkt * g.KH + B.bkh) * g.KW + kw;
         return true;
     }
     int nrow = p.bt * p.bh * p.bw;
@@ -122,59 +130,258 @@ __device__ __forceinline__ bool box_row(const QuantParams& p, const BoxPos& B, i
     int kw = B.bkw * p.nw + jj;
     if (kw >= g.KW || B.t0 + dt >= g.T || B.h0 + dh >= g.H || B.w0 + x >= g.W) return false;
     int sh = imin(g.h, g.H - B.h0), sw = imin(g.w, g.W - kw * g.w);
-    *j = jj;
     *rho = cube_first_row(g, B.bkt, B.bkh, kw) + ((long long)dt * sh + dh) * sw + dw;
-    *k = ((long long)B.bkt * g.KH + B.bkh) * g.KW + kw;
     return true;
 }
 
-// Kernel tokens (Eq. 1) of cube slot j for channels [8g, 8g+8) of the chunk:
-// an fp32 running sum over the cube's tokens in (t,h,w) order, then the
+// The box's tokens as a cube-major row list.  Small cubes: the box's nv valid
+// cube slots share kt, kh (so st, sh); only the last one can be cut by the
+// lattice edge in w; cube j owns rows [j n, j n + n_j).  Big cubes: one cube,
+// the box's R valid rows.
+struct BoxRows {
+    int nv, n, R;
+    int st, sh, sw_last;
+    long long k0;        // cube index of slot 0
+    long long rho0;      // big cubes: cube-major row of box row 0
+};
+
+__device__ __forceinline__ BoxRows box_rows(const QuantParams& p, const BoxPos& B) {
+    const Geom& g = p.g;
+    BoxRows R;
+    R.k0 = ((long long)B.bkt * g.KH + B.bkh) * g.KW + (p.big ? B.bkw : B.bkw * p.nw);
+    if (p.big) {
+        const int sh = imin(g.h, g.H - B.bkh * g.h), sw = imin(g.w, g.W - B.bkw * g.w);
+        R.nv = 1;
+        R.R = imin(p.bw, sw - B.dw0);
+        R.n = R.R;
+        R.st = R.sh = 1;
+        R.sw_last = R.R;
+        R.rho0 = cube_first_row(g, B.bkt, B.bkh, B.bkw) + ((long long)B.dt0 * sh + B.dh0) * sw + B.dw0;
+        return R;
+    }
+    R.nv = imin(p.nw, g.KW - B.bkw * p.nw);
+    R.st = imin(g.t, g.T - B.t0);
+    R.sh = imin(g.h, g.H - B.h0);
+    R.sw_last = imin(g.w, g.W - (B.bkw * p.nw + R.nv - 1) * g.w);
+    R.n = R.st * R.sh * g.w;
+    R.R = (R.nv - 1) * R.n + R.st * R.sh * R.sw_last;
+    R.rho0 = 0;
+    return R;
+}
+
+__device__ __forceinline__ int cube_of_row(const BoxRows& R, int r) { return imin(r / R.n, R.nv - 1); }
+
+// Row r of the list -> box row (shared-memory row of the TMA box) and cube-major row.
+__device__ __forceinline__ void list_row(const QuantParams& p, const BoxPos& B, const BoxRows& R, int r, int* row,
+                                         long long* rho) {
+    if (p.big) {
+        *row = r;
+        *rho = R.rho0 + r;
+        return;
+    }
+    const int j = cube_of_row(R, r), i = r - j * R.n;
+    const int sw = (j == R.nv - 1) ? R.sw_last : p.g.w;
+    const int dw = i % sw, q = i / sw;
+    const int dh = q % R.sh, dt = q / R.sh;
+    *row = (dt * p.bh + dh) * p.bw + j * p.g.w + dw;
+    // cube-major rows of one cube are its tokens in (t,h,w) order
+    *rho = cube_first_row(p.g, B.bkt, B.bkh, B.bkw * p.nw + j) + i;
+}
+
+// Kernel token (Eq. 1) of cube slot j for channels [8 g8, 8 g8 + 8) of the
+// chunk: an fp32 running sum over the cube's tokens in (t,h,w) order, then the
 // division by the token count (a product with the exact reciprocal when the
-// count is a power of two, which gives the identical rounding).  Returns
-// false for cube slots past the end of the lattice.
-__device__ __forceinline__ bool cube_mean8(const QuantParams& p, const BoxPos& B, const uint8_t* xs, int j, int g,
-                                           int st, int sh, float (&m)[8]) {
-    const Geom& g_ = p.g;
-    const int kw = B.bkw * p.nw + j;
-    if (kw >= g_.KW) return false;
-    const int sw = imin(g_.w, g_.W - kw * g_.w);
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; e++) acc[e] = 0.f;
-    for (int dt = 0; dt < st; dt++)
-        for (int dh = 0; dh < sh; dh++) {
-            const int row0 = (dt * p.bh + dh) * p.bw + j * g_.w;
+// count is a power of two, which gives the identical rounding).
+__device__ __forceinline__ void cube_mean8(const QuantParams& p, const BoxRows& R, const uint8_t* xs, int j, int g8,
+                                           uint64_t (&m)[4]) {
+    const int sw = (j == R.nv - 1) ? R.sw_last : p.g.w;
+    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // (+0, +0) pairs
+    for (int dt = 0; dt < R.st; dt++)
+        for (int dh = 0; dh < R.sh; dh++) {
+            const int row0 = (dt * p.bh + dh) * p.bw + j * p.g.w;
+#pragma unroll 2
             for (int dw = 0; dw < sw; dw++) {
-                uint4 v = ld_x8_swz(xs, row0 + dw, g);
-                acc[0] = __fadd_rn(acc[0], bf16_lo(v.x));
-                acc[1] = __fadd_rn(acc[1], bf16_hi(v.x));
-                acc[2] = __fadd_rn(acc[2], bf16_lo(v.y));
-                acc[3] = __fadd_rn(acc[3], bf16_hi(v.y));
-                acc[4] = __fadd_rn(acc[4], bf16_lo(v.z));
-                acc[5] = __fadd_rn(acc[5], bf16_hi(v.z));
-                acc[6] = __fadd_rn(acc[6], bf16_lo(v.w));
-                acc[7] = __fadd_rn(acc[7], bf16_hi(v.w));
+                const uint4 v = ld_x8_swz(xs, row0 + dw, g8);
+                acc[0] = f2_add(acc[0], f2_from_bf16x2(v.x));
+                acc[1] = f2_add(acc[1], f2_from_bf16x2(v.y));
+                acc[2] = f2_add(acc[2], f2_from_bf16x2(v.z));
+                acc[3] = f2_add(acc[3], f2_from_bf16x2(v.w));
             }
         }
-    const int cnt = st * sh * sw;
+    const int cnt = R.st * R.sh * sw;
     if ((cnt & (cnt - 1)) == 0) {
         const float inv = __frcp_rn((float)cnt);
+        const uint64_t inv2 = f2_pack(inv, inv);
 #pragma unroll
-        for (int e = 0; e < 8; e++) m[e] = __fmul_rn(acc[e], inv);
+        for (int e = 0; e < 4; e++) m[e] = f2_mul(acc[e], inv2);
     } else {
 #pragma unroll
-        for (int e = 0; e < 8; e++) m[e] = __fdiv_rn(acc[e], (float)cnt);
+        for (int e = 0; e < 4; e++) {
+            float a, b;
+            f2_unpack(acc[e], a, b);
+            m[e] = f2_pack(__fdiv_rn(a, (float)cnt), __fdiv_rn(b, (float)cnt));
+        }
     }
-    return true;
 }
 
-// Named barrier of one chunk group (constant barrier ids keep the CTA's barrier count at 3).
-__device__ __forceinline__ void group_sync(int grp) {
-    if (grp == 0)
-        bar_sync(1, 128);
-    else
-        bar_sync(2, 128);
+// Eight fp32 values as four packed pairs (16-byte aligned).
+__device__ __forceinline__ void load8(const float* src, uint64_t (&m)[4]) {
+    const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(src);
+    const ulonglong2 b = *reinterpret_cast<const ulonglong2*>(src + 4);
+    m[0] = a.x; m[1] = a.y; m[2] = b.x; m[3] = b.y;
+}
+
+__device__ __forceinline__ void store8(float* dst, const uint64_t (&m)[4]) {
+    *reinterpret_cast<ulonglong2*>(dst) = make_ulonglong2(m[0], m[1]);
+    *reinterpret_cast<ulonglong2*>(dst + 4) = make_ulonglong2(m[2], m[3]);
+}
+
+// max |x - m| over 8 channels: x as four BF16 words, m as four fp32 pairs
+__device__ __forceinline__ float max_abs_diff8(const uint4 x, const uint64_t (&m)[4]) {
+    float d[8];
+    f2_unpack(f2_sub(f2_from_bf16x2(x.x), m[0]), d[0], d[1]);
+    f2_unpack(f2_sub(f2_from_bf16x2(x.y), m[1]), d[2], d[3]);
+    f2_unpack(f2_sub(f2_from_bf16x2(x.z), m[2]), d[4], d[5]);
+    f2_unpack(f2_sub(f2_from_bf16x2(x.w), m[3]), d[6], d[7]);
+    return fmaxf(max3_abs(d[0], d[1], d[2]), fmaxf(max3_abs(d[3], d[4], d[5]), max3_abs(d[6], d[7], 0.f)));
+}
+
+// This warp's rows [r_lo, r_hi) of the list and the cube slots they touch.
+struct WarpRows {
+    int r_lo, r_hi, j_lo, ncub;
+};
+
+__device__ __forceinline__ WarpRows warp_rows(const BoxRows& R, int warp) {
+    WarpRows W;
+    W.r_lo = 16 * warp;
+    W.r_hi = imin(W.r_lo + 16, R.R);
+    if (W.r_lo >= W.r_hi) {
+        W.j_lo = 0;
+        W.ncub = 0;
+        return W;
+    }
+    W.j_lo = cube_of_row(R, W.r_lo);
+    W.ncub = cube_of_row(R, W.r_hi - 1) - W.j_lo + 1;
+    return W;
+}
+
+// Phase 1 of a chunk: the kernel tokens of the warp's cubes into its table
+// (row jj = cube slot j_lo + jj, kMeanStride floats).  Big cubes: the means of
+// the box's one cube, computed by the means kernel.
+// Phase-1 task of a lane for one item (small cubes): cube slot jj of the warp's
+// table, channel group g8, and for cubes of up to 8 tokens the shared-memory
+// offsets of its tokens (fixed for all chunks of the item).
+struct MeanTask {
+    int jj, g8, j, ntok;   // ntok 0: no task
+    uint32_t off[8];
+};
+
+__device__ __forceinline__ MeanTask mean_task(const QuantParams& p, const BoxRows& R, const WarpRows& W, int q) {
+    MeanTask T;
+    T.jj = q >> 3;
+    T.g8 = q & 7;
+    T.j = W.j_lo + T.jj;
+    T.ntok = 0;
+    if (p.big || q >= W.ncub * 8) return T;
+    const int sw = (T.j == R.nv - 1) ? R.sw_last : p.g.w;
+    T.ntok = R.st * R.sh * sw;
+    // tokens in (t,h,w) order; entries past ntok repeat the last token (never read)
+    int dt = 0, dh = 0, dw = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const uint32_t row = (uint32_t)((dt * p.bh + dh) * p.bw + T.j * p.g.w + dw);
+        T.off[i] = row * 128u + ((((uint32_t)T.g8) ^ (row & 7u)) << 4);
+        if (i + 1 < T.ntok && ++dw == sw) {
+            dw = 0;
+            if (++dh == R.sh) {
+                dh = 0;
+                ++dt;
+            }
+        }
+    }
+    return T;
+}
+
+// fp32 running sum of N tokens of one 8-channel group in (t,h,w) order
+template <int N>
+__device__ __forceinline__ void sum_tokens(const uint8_t* xs, const uint32_t (&off)[8], uint64_t (&acc)[4]) {
+#pragma unroll
+    for (int i = 0; i < N; i++) {
+        const uint4 v = *reinterpret_cast<const uint4*>(xs + off[i]);
+        acc[0] = f2_add(acc[0], f2_from_bf16x2(v.x));
+        acc[1] = f2_add(acc[1], f2_from_bf16x2(v.y));
+        acc[2] = f2_add(acc[2], f2_from_bf16x2(v.z));
+        acc[3] = f2_add(acc[3], f2_from_bf16x2(v.w));
+    }
+}
+
+__device__ __forceinline__ void mean_from_sum(const uint64_t (&acc)[4], int cnt, uint64_t (&m)[4]) {
+    if ((cnt & (cnt - 1)) == 0) {
+        const float inv = __frcp_rn((float)cnt);
+        const uint64_t inv2 = f2_pack(inv, inv);
+#pragma unroll
+        for (int e = 0; e < 4; e++) m[e] = f2_mul(acc[e], inv2);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            float a, b;
+            f2_unpack(acc[e], a, b);
+            m[e] = f2_pack(__fdiv_rn(a, (float)cnt), __fdiv_rn(b, (float)cnt));
+        }
+    }
+}
+
+// Phase 1 of a chunk: the kernel tokens of the warp's cubes into its table
+// (row jj = cube slot j_lo + jj, kMeanStride floats).  T0 is this lane's first
+// task (q = lane) with its token offsets; further tasks (only when the warp's
+// rows touch more than four cubes) take the generic path.  Big cubes: the
+// means of the box's one cube, computed by the means kernel.
+__device__ __forceinline__ void fill_means(const QuantParams& p, const BoxRows& R, const WarpRows& W,
+                                           const MeanTask& T0, const uint8_t* xs, int c0, float* tbl, int lane) {
+    if (p.big) {
+        if (W.ncub > 0 && lane < 16) {
+            const float4 v = *reinterpret_cast<const float4*>(p.means + (size_t)R.k0 * p.Ci + c0 + 4 * lane);
+            *reinterpret_cast<float4*>(tbl + 4 * lane) = v;
+        }
+        return;
+    }
+    if (T0.ntok > 0) {
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // (+0, +0) pairs
+        switch (T0.ntok) {
+            case 1: sum_tokens<1>(xs, T0.off, acc); break;
+            case 2: sum_tokens<2>(xs, T0.off, acc); break;
+            case 4: sum_tokens<4>(xs, T0.off, acc); break;
+            case 8: sum_tokens<8>(xs, T0.off, acc); break;
+            default:
+                if (T0.ntok <= 8) {
+#pragma unroll
+                    for (int i = 0; i < 8; i++) {
+                        if (i >= T0.ntok) break;
+                        const uint4 v = *reinterpret_cast<const uint4*>(xs + T0.off[i]);
+                        acc[0] = f2_add(acc[0], f2_from_bf16x2(v.x));
+                        acc[1] = f2_add(acc[1], f2_from_bf16x2(v.y));
+                        acc[2] = f2_add(acc[2], f2_from_bf16x2(v.z));
+                        acc[3] = f2_add(acc[3], f2_from_bf16x2(v.w));
+                    }
+                } else {
+                    uint64_t m[4];
+                    cube_mean8(p, R, xs, T0.j, T0.g8, m);
+                    store8(tbl + T0.jj * kMeanStride + 8 * T0.g8, m);
+                    break;
+                }
+        }
+        if (T0.ntok <= 8) {
+            uint64_t m[4];
+            mean_from_sum(acc, T0.ntok, m);
+            store8(tbl + T0.jj * kMeanStride + 8 * T0.g8, m);
+        }
+    }
+    for (int q = lane + 32; q < W.ncub * 8; q += 32) {
+        const int jj = q >> 3, g8 = q & 7;
+        uint64_t m[4];
+        cube_mean8(p, R, xs, W.j_lo + jj, g8, m);
+        store8(tbl + jj * kMeanStride + 8 * g8, m);
+    }
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -187,50 +394,50 @@ __device__ __forceinline__ float warp_max(float v) {
 
 // ------------------------------------------------------------------ a1: statistics + X L1
 //
-// Warps 0-7 compute (thread t: token row t % 128, channel half t / 128 of each
-// 64-channel chunk), warp 8 loads, warp 9 owns tensor memory and issues the
-// X L1 MMAs.  One named barrier per chunk: the means table is double-buffered.
-
-constexpr int kQCompute = 256;
-constexpr int kQGroup = 128;   // compute threads per chunk group
+// Warps 0-7 compute, warp 8 loads, warp 9 owns tensor memory and issues the
+// X L1 MMAs (M = 128 box rows, N = rank, K = 64 per chunk) into one of two
+// tensor-memory accumulators per item, which the compute warps drain to the
+// item's partial sums after its last chunk.
 
 __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_constant__ CUtensorMap tm_x,
                                                                   const __grid_constant__ CUtensorMap tm_l1,
                                                                   QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const QSmem L = q_smem_layout(p.nw, p.rank, true);
+    const QSmem L = q_smem_layout(p.rank, true, p.tbl_rows);
     uint64_t* full = (uint64_t*)(sm + L.bars);
     uint64_t* empty = full + kQStages;
-    uint64_t* done = empty + kQStages;
+    uint64_t* accf = empty + kQStages;   // [2]
+    uint64_t* acce = accf + 2;           // [2]
+    uint64_t* done = acce + 2;
     uint32_t* tmem_slot = (uint32_t*)(sm + L.misc);
     volatile int* abort_flag = (volatile int*)(sm + L.misc + 8);
     float* red = (float*)(sm + L.misc + 16);  // 8 floats
-    uint32_t* kmax = (uint32_t*)(sm + L.kmax);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int box = blockIdx.x, split = blockIdx.y;
-    const BoxPos B = box_pos(p, box);
     const int nchunks = p.chunks_per_split;
-    const int c_base = split * nchunks * 64;
+    const int n_items = p.n_boxes * p.splits;
     const uint32_t l1_bytes = (uint32_t)p.rank * 128u;
     const uint32_t l1_stride = (uint32_t)align_up(l1_bytes, 1024);
     const uint32_t x_bytes = (uint32_t)p.bt * p.bh * p.bw * 128u;
-    uint32_t tmem_cols = 32;
-    while (tmem_cols < (uint32_t)p.rank) tmem_cols <<= 1;
+    uint32_t tcols = 32;
+    while (tcols < (uint32_t)p.rank) tcols <<= 1;
 
     if (tid == 0) {
         for (int s = 0; s < kQStages; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kQGroup + 1);   // the chunk's group + the MMA commit
+            mbar_init(&empty[s], kQWarps + 1);   // the compute warps + the MMA commit
+        }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(&accf[b], 1);
+            mbar_init(&acce[b], kQWarps);
         }
         mbar_init(done, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    for (int j = tid; j < p.nw; j += blockDim.x) kmax[j] = 0u;
     if (warp == 9) {
-        tmem_alloc(tmem_slot, tmem_cols);
+        tmem_alloc(tmem_slot, 2 * tcols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -239,38 +446,59 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 8) {
-        // ---------------- producer
+        // ---------------- producer: all chunks of all this CTA's items through one ring
         if (lane == 0) {
-            int issued = 0;
             prefetch_tmap(&tm_x);
             prefetch_tmap(&tm_l1);
-            for (int i = 0; i < nchunks; i++) {
-                int s = i % kQStages;
-                if (i >= kQStages && !mbar_wait(&empty[s], ((i / kQStages) - 1) & 1, abort_flag, p.status, p.budget_ns))
-                    break;
-                mbar_arrive_expect_tx(&full[s], x_bytes + l1_bytes);
-                int c0 = c_base + i * 64;
-                tma_load_4d(sm + L.x + s * 16384, &tm_x, &full[s], c0, B.w0, B.h0, B.t0);
-                tma_load_2d(sm + L.l1 + s * l1_stride, &tm_l1, &full[s], c0, 0);
-                issued = i + 1;
+            long long g = 0;
+            bool alive = true;
+            for (int it = blockIdx.x; alive && it < n_items; it += gridDim.x) {
+                const BoxPos B = box_pos(p, it / p.splits);
+                const int c_base = (it % p.splits) * nchunks * 64;
+                for (int i = 0; i < nchunks; i++, g++) {
+                    const int s = (int)(g % kQStages);
+                    if (g >= kQStages &&
+                        !mbar_wait(&empty[s], (uint32_t)((g / kQStages) - 1) & 1, abort_flag, p.status, p.budget_ns)) {
+                        alive = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[s], x_bytes + l1_bytes);
+                    const int c0 = c_base + i * 64;
+                    tma_load_4d(sm + L.x + s * 16384, &tm_x, &full[s], c0, B.w0, B.h0, B.t0);
+                    tma_load_2d(sm + L.l1 + s * l1_stride, &tm_l1, &full[s], c0, 0);
+                }
             }
             // drain: every issued load lands before shared memory is released
-            for (int i = (issued > kQStages ? issued - kQStages : 0); i < issued; i++)
-                mbar_wait(&full[i % kQStages], (i / kQStages) & 1, abort_flag, nullptr, p.budget_ns, false);
+            for (long long q = (g > kQStages ? g - kQStages : 0); q < g; q++)
+                mbar_wait(&full[q % kQStages], (uint32_t)(q / kQStages) & 1, abort_flag, nullptr, p.budget_ns, false);
         }
     } else if (warp == 9) {
-        // ---------------- MMA issuer: U += X_chunk L1_chunk^T (M = 128 rows, N = rank, K = 64)
+        // ---------------- MMA issuer: U_item = sum over its chunks of X_chunk L1_chunk^T
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(128, p.rank);
-            for (int i = 0; i < nchunks; i++) {
-                int s = i % kQStages;
-                if (!mbar_wait(&full[s], (i / kQStages) & 1, abort_flag, p.status, p.budget_ns)) break;
+            long long g = 0;
+            int n = 0;
+            bool alive = true;
+            for (int it = blockIdx.x; alive && it < n_items; it += gridDim.x, n++) {
+                const int buf = n & 1, use = n >> 1;
+                const uint32_t acc = tmem + (uint32_t)buf * tcols;
+                if (use > 0 && !mbar_wait(&acce[buf], (uint32_t)(use - 1) & 1, abort_flag, p.status, p.budget_ns))
+                    break;
                 tc_fence_after();
-                uint32_t xa = smem_u32(sm + L.x + s * 16384), la = smem_u32(sm + L.l1 + s * l1_stride);
+                for (int i = 0; i < nchunks; i++, g++) {
+                    const int s = (int)(g % kQStages);
+                    if (!mbar_wait(&full[s], (uint32_t)(g / kQStages) & 1, abort_flag, p.status, p.budget_ns)) {
+                        alive = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t xa = smem_u32(sm + L.x + s * 16384), la = smem_u32(sm + L.l1 + s * l1_stride);
 #pragma unroll
-                for (int k = 0; k < 4; k++)
-                    mma_bf16(tmem, desc_k_sw128(xa + 32 * k), desc_k_sw128(la + 32 * k), idesc, (i | k) != 0);
-                tc_commit(&empty[s]);
+                    for (int k = 0; k < 4; k++)
+                        mma_bf16(acc, desc_k_sw128(xa + 32 * k), desc_k_sw128(la + 32 * k), idesc, (i | k) != 0);
+                    tc_commit(&empty[s]);
+                }
+                if (alive) tc_commit(&accf[buf]);
             }
             tc_commit(done);
             // every MMA has retired before tensor memory is released
@@ -278,124 +506,142 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
         }
         __syncwarp();
     } else {
-        // ---------------- compute warps 0-7: two groups of four warps take alternate chunks
-        // (group g: chunks i = g, g+2, ...), each with its own means table and named barrier,
-        // so that one group's waits overlap the other's work.  Thread = one token row.
-        const int grp = tid >> 7, row = tid & 127, half = grp;
+        // ---------------- compute warps 0-7
+        float* tbl = (float*)(sm + L.tbl) + warp * p.tbl_rows * kMeanStride;
         float damax = 0.f;
-        int myj = -1;
-        long long myrho = 0, myk = 0;
-        const bool row_ok = box_row(p, B, row, &myj, &myrho, &myk);
-        const int st = imin(p.g.t, p.g.T - B.t0), sh = imin(p.g.h, p.g.H - B.h0);
-        float* means = (float*)(sm + L.means) + grp * p.nw * kMeanStride;
-        for (int i = grp; i < nchunks; i += 2) {
-            const int s = i % kQStages;
-            // a failed wait skips the work but keeps the barrier protocol
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (i / kQStages) & 1, abort_flag, p.status,
-                                                              p.budget_ns));
-            const uint8_t* xs = sm + L.x + s * 16384;
+        long long g = 0;
+        int n = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, n++) {
+            const BoxPos B = box_pos(p, it / p.splits);
+            const int split = it % p.splits;
+            const int c_base = split * nchunks * 64;
+            const BoxRows R = box_rows(p, B);
+            const WarpRows W = warp_rows(R, warp);
+            const MeanTask T0m = mean_task(p, R, W, lane);
+            // this lane's row (two lanes per row, 32 channels each)
+            const int r = W.r_lo + (lane >> 1), half = lane & 1;
+            const bool has_row = r < W.r_hi;
+            int row = 0;
+            long long rho = 0;
+            if (has_row) list_row(p, B, R, r, &row, &rho);
+            const int jj_row = has_row ? cube_of_row(R, r) - W.j_lo : 0;
+            // shared-memory offsets of this lane's four 8-channel pieces of its row (128-byte swizzle)
+            uint32_t xoff[4];
+#pragma unroll
+            for (int v = 0; v < 4; v++) xoff[v] = (uint32_t)row * 128u + ((((uint32_t)(4 * half + v)) ^ ((uint32_t)row & 7u)) << 4);
+            const float* mrow = tbl + jj_row * kMeanStride + 32 * half;
+            float kam[4] = {0.f, 0.f, 0.f, 0.f};   // max |mean| of this lane's cube tasks
+            for (int i = 0; i < nchunks; i++, g++) {
+                const int s = (int)(g % kQStages);
+                ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)(g / kQStages) & 1, abort_flag, p.status,
+                                                       p.budget_ns));
+                if (!ok) break;
+                const uint8_t* xs = sm + L.x + s * 16384;
+                const int c0 = c_base + i * 64;
+                fill_means(p, R, W, T0m, xs, c0, tbl, lane);
+                __syncwarp();
+                if (!p.big) {
+#pragma unroll
+                    for (int t = 0; t < 4; t++) {
+                        const int q = lane + 32 * t;
+                        if (q < W.ncub * 8) {
+                            const float* src = tbl + (q >> 3) * kMeanStride + 8 * (q & 7);
+                            const float4 a = *reinterpret_cast<const float4*>(src);
+                            const float4 b = *reinterpret_cast<const float4*>(src + 4);
+                            kam[t] = fmaxf(kam[t], fmaxf(max3_abs(a.x, a.y, a.z), fmaxf(max3_abs(a.w, b.x, b.y),
+                                                                                       max3_abs(b.z, b.w, 0.f))));
+                        }
+                    }
+                }
+                if (has_row) {
+                    float a[4];
+#pragma unroll
+                    for (int v = 0; v < 4; v++) {
+                        uint64_t m[4];
+                        load8(mrow + 8 * v, m);
+                        a[v] = max_abs_diff8(*reinterpret_cast<const uint4*>(xs + xoff[v]), m);
+                    }
+                    damax = max3_abs(damax, fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+            }
+            if (!ok) break;
+            // per-cube max |mean| over this item's channels -> kamax (small cubes; the means
+            // kernel has done it for big ones)
             if (!p.big) {
-                // kernel tokens of the box's cubes for these 64 channels
-                for (int q = row; ok && q < p.nw * 8; q += kQGroup) {
-                    const int j = q >> 3, g8 = q & 7;
-                    float m[8];
-                    if (!cube_mean8(p, B, xs, j, g8, st, sh, m)) continue;
-                    float* dst = means + j * kMeanStride + 8 * g8;
-                    *reinterpret_cast<float4*>(dst) = make_float4(m[0], m[1], m[2], m[3]);
-                    *reinterpret_cast<float4*>(dst + 4) = make_float4(m[4], m[5], m[6], m[7]);
-                    float am = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 8; e++) am = fmaxf(am, fabsf(m[e]));
-                    atomicMax(&kmax[j], __float_as_uint(am));
-                }
-                group_sync(grp);
-            }
-            // delta amax of this thread's token row (64 channels)
-            if (ok && row_ok) {
-                const float* mj = p.big ? p.means + (size_t)myk * p.Ci + c_base + i * 64 : means + myj * kMeanStride;
-#pragma unroll
-                for (int q8 = 0; q8 < 8; q8++) {
-                    uint4 xv = ld_x8_swz(xs, row, q8);
-                    float4 m0 = *reinterpret_cast<const float4*>(mj + q8 * 8);
-                    float4 m1 = *reinterpret_cast<const float4*>(mj + q8 * 8 + 4);
-                    damax = fmaxf(damax, fabsf(__fsub_rn(bf16_lo(xv.x), m0.x)));
-                    damax = fmaxf(damax, fabsf(__fsub_rn(bf16_hi(xv.x), m0.y)));
-                    damax = fmaxf(damax, fabsf(__fsub_rn(bf16_lo(xv.y), m0.z)));
-                    damax = fmaxf(damax, fabsf(__fsub_rn(bf16_hi(xv.y), m0.w)));
-                    damax = fmaxf(damax, fabsf(__fsub_rn(bf16_lo(xv.z), m1.x)));
-                    damax = fmaxf(damax, fabsf(__fsub_rn(bf16_hi(xv.z), m1.y)));
-                    damax = fmaxf(damax, fabsf(__fsub_rn(bf16_lo(xv.w), m1.z)));
-                    damax = fmaxf(damax, fabsf(__fsub_rn(bf16_hi(xv.w), m1.w)));
+                for (int t = 0; t < 4; t++) {
+                    const int q = lane + 32 * t;
+                    if (q < W.ncub * 8) {
+                        const uint32_t gm = 0xFFu << (lane & 24);
+                        float v = kam[t];
+                        v = fmaxf(v, __shfl_xor_sync(gm, v, 1));
+                        v = fmaxf(v, __shfl_xor_sync(gm, v, 2));
+                        v = fmaxf(v, __shfl_xor_sync(gm, v, 4));
+                        if ((q & 7) == 0) atomicMax(&p.kamax[R.k0 + W.j_lo + (q >> 3)], __float_as_uint(v));
+                    }
                 }
             }
-            if (!p.big) group_sync(grp);   // this group's means table is rewritten next chunk
-            mbar_arrive(&empty[s]);
-        }
-        // epilogue: U partial rows out of tensor memory (sub-partition warp % 4; this warp's column half)
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag, p.status, p.budget_ns));
-        tc_fence_after();
-        if (ok) {
-            float* urow = p.u_part + ((size_t)split * p.g.N + (size_t)myrho) * p.rank;
-            for (int c = 16 * half; c < p.rank; c += 32) {
-                uint32_t r[16];
-                tmem_ld_x16(tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)c, r);
+            // U partial rows of this item out of tensor memory (sub-partition warp % 4, column half warp / 4)
+            const int buf = n & 1, use = n >> 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], (uint32_t)use & 1, abort_flag, p.status, p.budget_ns));
+            if (!ok) break;
+            tc_fence_after();
+            const int urow_i = (warp & 3) * 32 + lane, uhalf = warp >> 2;
+            long long urho = 0;
+            const bool urow_ok = box_row(p, B, urow_i, &urho);
+            float* urow = p.u_part + ((size_t)split * p.g.N + (size_t)urho) * p.rank;
+            for (int c = 16 * uhalf; c < p.rank; c += 32) {
+                uint32_t rr[16];
+                tmem_ld_x16(tmem + (uint32_t)buf * tcols + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)c, rr);
                 tmem_ld_wait();
-                if (row_ok) {
+                if (urow_ok) {
 #pragma unroll
                     for (int v = 0; v < 16; v += 4)
                         *reinterpret_cast<float4*>(urow + c + v) =
-                            make_float4(__uint_as_float(r[v]), __uint_as_float(r[v + 1]), __uint_as_float(r[v + 2]),
-                                        __uint_as_float(r[v + 3]));
+                            make_float4(__uint_as_float(rr[v]), __uint_as_float(rr[v + 1]), __uint_as_float(rr[v + 2]),
+                                        __uint_as_float(rr[v + 3]));
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce[buf]);
         }
         float wm = warp_max(damax);
         if (lane == 0) red[warp] = wm;
-        // barrier 3: ids 1 and 2 belong to the chunk groups, and one group may still be in
-        // its loop when the other gets here (a barrier must not see two thread counts at once)
-        bar_sync(3, kQCompute);
+        bar_sync(1, kQCompute);
         if (tid == 0) {
             float bm = 0.f;
-            for (int w = 0; w < 8; w++) bm = fmaxf(bm, red[w]);
+            for (int w = 0; w < kQWarps; w++) bm = fmaxf(bm, red[w]);
             atomicMax(&p.scalars[0], __float_as_uint(bm));
-        }
-        for (int j = tid; j < p.nw; j += kQCompute) {
-            int kw = B.bkw * p.nw + j;
-            if (kw < p.g.KW) {
-                long long k = ((long long)B.bkt * p.g.KH + B.bkh) * p.g.KW + kw;
-                atomicMax(&p.kamax[k], kmax[j]);
-            }
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 9) {
         tc_fence_after();
-        tmem_dealloc(tmem, tmem_cols);
+        tmem_dealloc(tmem, 2 * tcols);
     }
 }
 
 // ------------------------------------------------------------------ a2: encode
 //
-// Warps 0-7 compute (thread t: token row t % 128, channel half t / 128 of each
-// 64-channel chunk, i.e. two FP4 groups of 16), warp 8 loads.
+// Warps 0-7 compute, warp 8 loads.
 
 __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_constant__ CUtensorMap tm_x,
                                                                   QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const QSmem L = q_smem_layout(p.nw, p.rank, false);
+    const QSmem L = q_smem_layout(p.rank, false, p.tbl_rows);
     uint64_t* full = (uint64_t*)(sm + L.bars);
     uint64_t* empty = full + kQStages;
     volatile int* abort_flag = (volatile int*)(sm + L.misc + 8);
-    float* s8s = (float*)(sm + L.s8);
-    float* rs8s = (float*)(sm + L.kmax);   // reciprocals of s8 (the kmax slot is unused in this kernel)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int box = blockIdx.x, split = blockIdx.y;
-    const BoxPos B = box_pos(p, box);
     const int nchunks = p.chunks_per_split;
-    const int c_base = split * nchunks * 64;
+    const int n_items = p.n_boxes * p.splits;
     const uint32_t x_bytes = (uint32_t)p.bt * p.bh * p.bw * 128u;
     const int Ci = p.Ci;
 
@@ -403,11 +649,11 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
     if (tid == 0) {
         for (int s = 0; s < kQStages; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kQGroup);   // the chunk's group
+            mbar_init(&empty[s], kQWarps);
         }
         *abort_flag = 0;
         fence_barrier_init();
-        if (box == 0 && split == 0 &&
+        if (blockIdx.x == 0 &&
             (hdr->magic != 0x31575144u || hdr->Ci != p.Ci || hdr->rank != p.rank || hdr->slab != p.slab))
             atomicCAS(p.status, 0, kStatusBadWeight);
     }
@@ -415,155 +661,189 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
     const float damax = __uint_as_float(p.scalars[0]);
     const float S = (damax == 0.f) ? 1.f : __fdiv_rn(damax, 2688.f);
     const float denom = __fmul_rn(6.f, S);
-    for (int j = tid; j < p.nw; j += blockDim.x) {
-        int kw = B.bkw * p.nw + j;
-        float s = 0.f;
-        if (kw < p.g.KW) {
-            long long k = ((long long)B.bkt * p.g.KH + B.bkh) * p.g.KW + kw;
-            s = __fdiv_rn(__uint_as_float(p.kamax[k]), 448.f);
-            if (split == 0) p.s8[k] = s;
-        }
-        s8s[j] = s;
-        rs8s[j] = (s != 0.f) ? __frcp_rn(s) : 0.f;
-    }
-    if (box == 0 && split == 0 && tid == 0) p.scalars[1] = __float_as_uint(S);
+    const float rdenom = __frcp_rn(denom);
+    if (blockIdx.x == 0 && tid == 0) p.scalars[1] = __float_as_uint(S);
     __syncthreads();
 
     if (warp == 8) {
         if (lane == 0) {
-            int issued = 0;
             prefetch_tmap(&tm_x);
-            for (int i = 0; i < nchunks; i++) {
-                int s = i % kQStages;
-                if (i >= kQStages && !mbar_wait(&empty[s], ((i / kQStages) - 1) & 1, abort_flag, p.status, p.budget_ns))
-                    break;
-                mbar_arrive_expect_tx(&full[s], x_bytes);
-                tma_load_4d(sm + L.x + s * 16384, &tm_x, &full[s], c_base + i * 64, B.w0, B.h0, B.t0);
-                issued = i + 1;
+            long long g = 0;
+            bool alive = true;
+            for (int it = blockIdx.x; alive && it < n_items; it += gridDim.x) {
+                const BoxPos B = box_pos(p, it / p.splits);
+                const int c_base = (it % p.splits) * nchunks * 64;
+                for (int i = 0; i < nchunks; i++, g++) {
+                    const int s = (int)(g % kQStages);
+                    if (g >= kQStages &&
+                        !mbar_wait(&empty[s], (uint32_t)((g / kQStages) - 1) & 1, abort_flag, p.status, p.budget_ns)) {
+                        alive = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[s], x_bytes);
+                    tma_load_4d(sm + L.x + s * 16384, &tm_x, &full[s], c_base + i * 64, B.w0, B.h0, B.t0);
+                }
             }
-            for (int i = (issued > kQStages ? issued - kQStages : 0); i < issued; i++)
-                mbar_wait(&full[i % kQStages], (i / kQStages) & 1, abort_flag, nullptr, p.budget_ns, false);
+            for (long long q = (g > kQStages ? g - kQStages : 0); q < g; q++)
+                mbar_wait(&full[q % kQStages], (uint32_t)(q / kQStages) & 1, abort_flag, nullptr, p.budget_ns, false);
         }
     } else {
-        // two groups of four warps take alternate chunks (see k_cube_stats); thread = token row
-        const int grp = tid >> 7, row = tid & 127, half = grp;
-        int myj = -1;
-        long long myrho = 0, myk = 0;
-        const bool row_ok = box_row(p, B, row, &myj, &myrho, &myk);
-        const int st = imin(p.g.t, p.g.T - B.t0), sh = imin(p.g.h, p.g.H - B.h0);
-        float* means = (float*)(sm + L.means) + grp * p.nw * kMeanStride;
-        for (int i = grp; i < nchunks; i += 2) {
-            const int s = i % kQStages;
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (i / kQStages) & 1, abort_flag, p.status,
-                                                              p.budget_ns));
-            const uint8_t* xs = sm + L.x + s * 16384;
-            const int c0 = c_base + i * 64;
-            // kernel tokens: means, FP8 E4M3 codes with the per-token scale s8 = max|mean| / 448
-            // (big cubes: means from the means kernel, encoded once per cube by its first box)
-            const bool enc_q8 = !p.big || (B.dt0 == 0 && B.dh0 == 0 && B.dw0 == 0);
-            for (int q = row; ok && enc_q8 && q < p.nw * 8; q += kQGroup) {
-                const int j = q >> 3, g8 = q & 7;
-                float m[8];
-                if (p.big) {
-                    const float* src = p.means + (size_t)(((long long)B.bkt * p.g.KH + B.bkh) * p.g.KW + B.bkw) * Ci +
-                                       c0 + 8 * g8;
-                    const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
-                    m[0] = a.x; m[1] = a.y; m[2] = a.z; m[3] = a.w; m[4] = b.x; m[5] = b.y; m[6] = b.z; m[7] = b.w;
-                } else {
-                    if (!cube_mean8(p, B, xs, j, g8, st, sh, m)) continue;
-                    float* dst = means + j * kMeanStride + 8 * g8;
-                    *reinterpret_cast<float4*>(dst) = make_float4(m[0], m[1], m[2], m[3]);
-                    *reinterpret_cast<float4*>(dst + 4) = make_float4(m[4], m[5], m[6], m[7]);
-                }
-                const long long k = ((long long)B.bkt * p.g.KH + B.bkh) * p.g.KW + (B.bkw * p.nw + j);
-                const float s8 = s8s[j], rs8 = rs8s[j];
-                uint32_t c[4] = {0u, 0u, 0u, 0u};
-                if (s8 != 0.f) {
+        float* tbl = (float*)(sm + L.tbl) + warp * p.tbl_rows * kMeanStride;
+        const float SS = __fmul_rn(S, hdr->S_W);
+        long long g = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+            const BoxPos B = box_pos(p, it / p.splits);
+            const int split = it % p.splits;
+            const int c_base = split * nchunks * 64;
+            const BoxRows R = box_rows(p, B);
+            const WarpRows W = warp_rows(R, warp);
+            const MeanTask T0m = mean_task(p, R, W, lane);
+            const int r = W.r_lo + (lane >> 1), half = lane & 1;
+            const bool has_row = r < W.r_hi;
+            int row = 0;
+            long long rho = 0;
+            if (has_row) list_row(p, B, R, r, &row, &rho);
+            const int jj_row = has_row ? cube_of_row(R, r) - W.j_lo : 0;
+            uint32_t xoff[4];
+#pragma unroll
+            for (int v = 0; v < 4; v++) xoff[v] = (uint32_t)row * 128u + ((((uint32_t)(4 * half + v)) ^ ((uint32_t)row & 7u)) << 4);
+            const float* mrow = tbl + jj_row * kMeanStride + 32 * half;
+            uint8_t* dcode_row = p.dcodes + (size_t)rho * (Ci / 2) + 16 * half;
+            // the kernel tokens of a cube are encoded by the warp that holds the cube's
+            // first row (big cubes: by warp 0 of the cube's first box)
+            const int j_own = p.big ? ((B.dt0 == 0 && B.dh0 == 0 && B.dw0 == 0 && warp == 0) ? 0 : 1)
+                                    : (W.ncub > 0 && W.j_lo * R.n < W.r_lo ? 1 : 0);
+            // s8 = max|mean| / 448 of the first kernel-token task of this lane (others, which only
+            // very small cubes have, are formed where they are used)
+            const int q_first = lane + 8 * j_own;
+            float s8_first = 0.f;
+            if (q_first < W.ncub * 8) {
+                const long long k = R.k0 + W.j_lo + (q_first >> 3);
+                s8_first = __fdiv_rn(__uint_as_float(p.kamax[k]), 448.f);
+                if (split == 0 && (q_first & 7) == 0) p.s8[k] = s8_first;
+            }
+            for (int i = 0; i < nchunks; i++, g++) {
+                const int s = (int)(g % kQStages);
+                ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)(g / kQStages) & 1, abort_flag, p.status,
+                                                       p.budget_ns));
+                if (!ok) break;
+                const uint8_t* xs = sm + L.x + s * 16384;
+                const int c0 = c_base + i * 64;
+                fill_means(p, R, W, T0m, xs, c0, tbl, lane);
+                __syncwarp();
+                // kernel tokens: FP8 E4M3 codes under s8 = max|mean| / 448, and their exact BF16 copy
+                for (int q = q_first; q < W.ncub * 8; q += 32) {
+                    const int jj = q >> 3, g8 = q & 7;
+                    const long long k = R.k0 + W.j_lo + jj;
+                    float s8 = s8_first;
+                    if (q != q_first) {
+                        s8 = __fdiv_rn(__uint_as_float(p.kamax[k]), 448.f);
+                        if (split == 0 && i == 0 && g8 == 0) p.s8[k] = s8;
+                    }
+                    uint64_t m[4];
+                    load8(tbl + jj * kMeanStride + 8 * g8, m);
+                    uint32_t c[4] = {0u, 0u, 0u, 0u};
+                    if (s8 != 0.f) {
+                        // codes of the negated quotients with the sign bit of each byte flipped
+                        // (E4M3 is sign-magnitude, saturation symmetric)
+                        const float rs8 = __frcp_rn(s8);
+                        const uint64_t b2 = f2_pack(s8, s8), nrb2 = f2_pack(-rs8, -rs8);
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            float lo, hi;
+                            f2_unpack(f2_div_neg(m[e], b2, nrb2), lo, hi);
+                            c[e] = cvt_e4m3x2(lo, hi) ^ 0x8080u;
+                        }
+                    }
+                    *reinterpret_cast<uint2*>(p.q8 + (size_t)k * Ci + c0 + 8 * g8) =
+                        make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+                    uint32_t bfw[4];
 #pragma unroll
                     for (int e = 0; e < 4; e++)
-                        c[e] = cvt_e4m3x2(div_pos(m[2 * e], s8, rs8), div_pos(m[2 * e + 1], s8, rs8));
+                        bfw[e] = (uint32_t)f32_to_bf16_rn(e4m3_to_f32(c[e] & 0xFF)) |
+                                 ((uint32_t)f32_to_bf16_rn(e4m3_to_f32(c[e] >> 8)) << 16);
+                    *reinterpret_cast<uint4*>(p.q8_bf16 + (size_t)k * Ci + c0 + 8 * g8) =
+                        make_uint4(bfw[0], bfw[1], bfw[2], bfw[3]);
                 }
-                *reinterpret_cast<uint2*>(p.q8 + (size_t)k * Ci + c0 + 8 * g8) =
-                    make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
-                uint32_t bfw[4];
+                // delta tokens: FP4 E2M1 with E4M3 group-16 scales under S (two groups per lane)
+                if (has_row) {
+                    uint32_t codes[4];
+                    uint32_t sc = 0;
 #pragma unroll
-                for (int e = 0; e < 4; e++)
-                    bfw[e] = (uint32_t)f32_to_bf16_rn(e4m3_to_f32(c[e] & 0xFF)) |
-                             ((uint32_t)f32_to_bf16_rn(e4m3_to_f32(c[e] >> 8)) << 16);
-                *reinterpret_cast<uint4*>(p.q8_bf16 + (size_t)k * Ci + c0 + 8 * g8) =
-                    make_uint4(bfw[0], bfw[1], bfw[2], bfw[3]);
-            }
-            if (!p.big) group_sync(grp);
-            // delta tokens: FP4 E2M1 with E4M3 group-16 scales under S (four groups per thread)
-            if (ok && row_ok) {
-                const float* mj = p.big ? p.means + (size_t)myk * Ci + c0 : means + myj * kMeanStride;
-                uint32_t codes[8];
-                uint32_t sc = 0;
+                    for (int b = 0; b < 2; b++) {
+                        uint64_t z[8];
 #pragma unroll
-                for (int b = 0; b < 4; b++) {
-                    float z[16];
-#pragma unroll
-                    for (int h = 0; h < 2; h++) {
-                        uint4 xv = ld_x8_swz(xs, row, 2 * b + h);
-                        float4 m0 = *reinterpret_cast<const float4*>(mj + 16 * b + 8 * h);
-                        float4 m1 = *reinterpret_cast<const float4*>(mj + 16 * b + 8 * h + 4);
-                        z[8 * h + 0] = __fsub_rn(bf16_lo(xv.x), m0.x);
-                        z[8 * h + 1] = __fsub_rn(bf16_hi(xv.x), m0.y);
-                        z[8 * h + 2] = __fsub_rn(bf16_lo(xv.y), m0.z);
-                        z[8 * h + 3] = __fsub_rn(bf16_hi(xv.y), m0.w);
-                        z[8 * h + 4] = __fsub_rn(bf16_lo(xv.z), m1.x);
-                        z[8 * h + 5] = __fsub_rn(bf16_hi(xv.z), m1.y);
-                        z[8 * h + 6] = __fsub_rn(bf16_lo(xv.w), m1.z);
-                        z[8 * h + 7] = __fsub_rn(bf16_hi(xv.w), m1.w);
-                    }
-                    float am = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 16; e++) am = fmaxf(am, fabsf(z[e]));
-                    uint32_t sb = cvt_e4m3x2(__fdiv_rn(am, denom), 0.f) & 0xFFu;
-                    float eff = __fmul_rn(e4m3_to_f32(sb), S);
-                    sc |= sb << (8 * b);
-                    const float reff = (eff != 0.f) ? __frcp_rn(eff) : 0.f;
-#pragma unroll
-                    for (int e = 0; e < 16; e += 8) {
-                        uint32_t wv = 0;
-                        if (eff != 0.f) {
-#pragma unroll
-                            for (int u = 0; u < 8; u += 2)
-                                wv |= cvt_e2m1x2(div_pos(z[e + u], eff, reff), div_pos(z[e + u + 1], eff, reff))
-                                      << (4 * u);
+                        for (int hh = 0; hh < 2; hh++) {
+                            const uint4 xv = *reinterpret_cast<const uint4*>(xs + xoff[2 * b + hh]);
+                            uint64_t m[4];
+                            load8(mrow + 16 * b + 8 * hh, m);
+                            z[4 * hh + 0] = f2_sub(f2_from_bf16x2(xv.x), m[0]);
+                            z[4 * hh + 1] = f2_sub(f2_from_bf16x2(xv.y), m[1]);
+                            z[4 * hh + 2] = f2_sub(f2_from_bf16x2(xv.z), m[2]);
+                            z[4 * hh + 3] = f2_sub(f2_from_bf16x2(xv.w), m[3]);
                         }
-                        codes[2 * b + e / 8] = wv;
+                        float zf[16];
+#pragma unroll
+                        for (int e = 0; e < 8; e++) f2_unpack(z[e], zf[2 * e], zf[2 * e + 1]);
+                        const float am = fmaxf(
+                            fmaxf(max3_abs(zf[0], zf[1], zf[2]), max3_abs(zf[3], zf[4], zf[5])),
+                            fmaxf(fmaxf(max3_abs(zf[6], zf[7], zf[8]), max3_abs(zf[9], zf[10], zf[11])),
+                                  fmaxf(max3_abs(zf[12], zf[13], zf[14]), fabsf(zf[15]))));
+                        const uint32_t sb = cvt_e4m3x2(div_pos(am, denom, rdenom), 0.f) & 0xFFu;
+                        const float eff = __fmul_rn(e4m3_to_f32(sb), S);
+                        sc |= sb << (8 * b);
+                        uint32_t w0 = 0, w1 = 0;
+                        if (eff != 0.f) {
+                            // codes of the negated quotients, then every nibble's sign bit flipped
+                            // (E2M1 is sign-magnitude: code(-v) = code(v) ^ 8, signed zeros included)
+                            const float reff = __frcp_rn(eff);
+                            const uint64_t b2 = f2_pack(eff, eff), nrb2 = f2_pack(-reff, -reff);
+                            float n[16];
+#pragma unroll
+                            for (int e = 0; e < 8; e++) f2_unpack(f2_div_neg(z[e], b2, nrb2), n[2 * e], n[2 * e + 1]);
+                            w0 = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(&n[0])) ^ 0x88888888u;
+                            w1 = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(&n[8])) ^ 0x88888888u;
+                        }
+                        codes[2 * b] = w0;
+                        codes[2 * b + 1] = w1;
                     }
+                    *reinterpret_cast<uint4*>(dcode_row + c0 / 2) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                    *reinterpret_cast<uint16_t*>(p.dscales + sf_offset(rho, c0 / 16 + 2 * half, Ci)) = (uint16_t)sc;
                 }
-                uint8_t* dst = p.dcodes + (size_t)myrho * (Ci / 2) + c0 / 2;
-                reinterpret_cast<uint4*>(dst)[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-                reinterpret_cast<uint4*>(dst)[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-                *reinterpret_cast<uint32_t*>(p.dscales + sf_offset(myrho, c0 / 16, Ci)) = sc;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
             }
-            if (!p.big) group_sync(grp);   // this group's means table is rewritten next chunk
-            mbar_arrive(&empty[s]);
-        }
-        // U' = (X L1) / (S_delta S_W) as BF16 hi + lo, slab zero-padded (split 0 only; half the columns each)
-        if (split == 0 && row_ok) {
-            const float SS = __fmul_rn(S, hdr->S_W);
-            uint16_t* dst = p.u_hilo + (size_t)myrho * p.slab;
-            const int cpb = p.rank / 2;
-            for (int c = half * cpb; c < (half + 1) * cpb; c += 2) {
-                float u0 = 0.f, u1 = 0.f;
-                for (int sp = 0; sp < p.splits; sp++) {
-                    const float* src = p.u_part + ((size_t)sp * p.g.N + (size_t)myrho) * p.rank + c;
-                    u0 = __fadd_rn(u0, src[0]);
-                    u1 = __fadd_rn(u1, src[1]);
+            if (!ok) break;
+            // U' = (X L1) / (S_delta S_W) as BF16 hi + lo for this item's slice of the rank columns
+            // (thread = box row x column half), the slab's zero padding by split 0
+            const int urow_i = tid & 127, uhalf = tid >> 7;
+            long long urho = 0;
+            if (box_row(p, B, urow_i, &urho)) {
+                uint16_t* dst = p.u_hilo + (size_t)urho * p.slab;
+                const int cps = 2 * (int)cdiv(p.rank, 2 * p.splits);
+                const int c_lo = imin(split * cps, p.rank), c_hi = imin(c_lo + cps, p.rank);
+                for (int c = c_lo + 2 * uhalf; c < c_hi; c += 4) {
+                    float u0 = 0.f, u1 = 0.f;
+                    for (int sp = 0; sp < p.splits; sp++) {
+                        const float2 v = *reinterpret_cast<const float2*>(
+                            p.u_part + ((size_t)sp * p.g.N + (size_t)urho) * p.rank + c);
+                        u0 = __fadd_rn(u0, v.x);
+                        u1 = __fadd_rn(u1, v.y);
+                    }
+                    float a0 = __fdiv_rn(u0, SS), a1 = __fdiv_rn(u1, SS);
+                    uint16_t h0 = f32_to_bf16_rn(a0), h1 = f32_to_bf16_rn(a1);
+                    uint16_t l0 = f32_to_bf16_rn(__fsub_rn(a0, __uint_as_float((uint32_t)h0 << 16)));
+                    uint16_t l1 = f32_to_bf16_rn(__fsub_rn(a1, __uint_as_float((uint32_t)h1 << 16)));
+                    *reinterpret_cast<uint32_t*>(dst + c) = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                    *reinterpret_cast<uint32_t*>(dst + p.rank + c) = (uint32_t)l0 | ((uint32_t)l1 << 16);
                 }
-                float a0 = __fdiv_rn(u0, SS), a1 = __fdiv_rn(u1, SS);
-                uint16_t h0 = f32_to_bf16_rn(a0), h1 = f32_to_bf16_rn(a1);
-                uint16_t l0 = f32_to_bf16_rn(__fsub_rn(a0, __uint_as_float((uint32_t)h0 << 16)));
-                uint16_t l1 = f32_to_bf16_rn(__fsub_rn(a1, __uint_as_float((uint32_t)h1 << 16)));
-                *reinterpret_cast<uint32_t*>(dst + c) = (uint32_t)h0 | ((uint32_t)h1 << 16);
-                *reinterpret_cast<uint32_t*>(dst + p.rank + c) = (uint32_t)l0 | ((uint32_t)l1 << 16);
+                if (split == 0) {
+                    const int zb = 2 * p.rank, zl = (p.slab - zb) / 2;
+                    for (int c = zb + uhalf * zl; c < zb + (uhalf + 1) * zl; c += 2)
+                        *reinterpret_cast<uint32_t*>(dst + c) = 0u;
+                }
             }
-            const int zb = 2 * p.rank, zl = (p.slab - zb) / 2;
-            for (int c = zb + half * zl; c < zb + (half + 1) * zl; c += 2) *reinterpret_cast<uint32_t*>(dst + c) = 0u;
         }
     }
     __syncthreads();
@@ -653,25 +933,56 @@ cudaError_t launch_cube_means_big(const CUtensorMap& tm_x, const QuantParams& p,
     return cudaGetLastError();
 }
 
-size_t quant_smem_bytes(int nw, int rank, bool stats) {
-    return q_smem_layout(nw, rank, stats).total + 1024;
+size_t quant_smem_bytes(int rank, bool stats, int tbl_rows) {
+    return q_smem_layout(rank, stats, tbl_rows).total + 1024;
 }
+
+namespace {
+// CTAs of a persistent quantise kernel: as many as can be resident at once,
+// from the kernel's registers and shared memory (the runtime's occupancy
+// query answers one CTA per SM for k_cube_stats where two fit and run).
+int resident_grid(const void* fn, int threads, size_t smem, int items) {
+    int dev = 0, sms = 148, smem_sm = 233472, reserved = 1024;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    cudaFuncAttributes fa;
+    int per_sm = 1;
+    if (cudaFuncGetAttributes(&fa, fn) == cudaSuccess && sms > 0) {
+        const int warps = (threads + 31) / 32;
+        const int regs_warp = (fa.numRegs * 32 + 255) / 256 * 256;
+        per_sm = 2048 / (warps * 32);
+        // the four sub-partitions of an SM each hold 16384 registers and a quarter of its warps
+        while (per_sm > 1 && ((per_sm * warps + 3) / 4) * regs_warp > 16384) per_sm--;
+        while (per_sm > 1 && (size_t)per_sm * (smem + fa.sharedSizeBytes + (size_t)reserved) > (size_t)smem_sm)
+            per_sm--;
+    }
+    return imin(items, (sms > 0 ? sms : 148) * per_sm);
+}
+}  // namespace
 
 cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
                               cudaStream_t st) {
-    size_t smem = quant_smem_bytes(p.nw, p.rank, true);
+    size_t smem = quant_smem_bytes(p.rank, true, p.tbl_rows);
     cudaError_t e = cudaFuncSetAttribute(k_cube_stats, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_cube_stats, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.n_boxes, p.splits);
+    const int grid = resident_grid((const void*)k_cube_stats, kQCompute + 64, smem, p.n_boxes * p.splits);
     k_cube_stats<<<grid, kQCompute + 64, smem, st>>>(tm_x, tm_l1, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const QuantParams& p, cudaStream_t st) {
-    size_t smem = quant_smem_bytes(p.nw, p.rank, false);
+    size_t smem = quant_smem_bytes(p.rank, false, p.tbl_rows);
     cudaError_t e = cudaFuncSetAttribute(k_cube_encode, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_cube_encode, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.n_boxes, p.splits);
+    const int grid = resident_grid((const void*)k_cube_encode, kQCompute + 32, smem, p.n_boxes * p.splits);
     k_cube_encode<<<grid, kQCompute + 32, smem, st>>>(tm_x, p);
     return cudaGetLastError();
 }
