@@ -384,6 +384,78 @@ __device__ __forceinline__ void fill_means(const QuantParams& p, const BoxRows& 
     }
 }
 
+// Element-wise max / min of two BF16 pairs (exact: no rounding involved).
+__device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_min(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("min.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Statistics task of a1: unit u (cube slot, or token row for big cubes) x
+// channel group g8 of the box, with the shared-memory offsets of the unit's
+// tokens when it has at most 8 (fixed for all chunks of the item).
+struct StatTask {
+    bool valid;
+    int u, g8, ntok;
+    uint32_t off[8];
+};
+
+__device__ __forceinline__ StatTask stat_task(const QuantParams& p, const BoxRows& R, int q) {
+    StatTask T;
+    T.u = q >> 3;
+    T.g8 = q & 7;
+    T.valid = T.u < (p.big ? R.R : R.nv);
+    T.ntok = 0;
+    if (!T.valid) return T;
+    if (p.big) {
+        T.ntok = 1;
+        const uint32_t row = (uint32_t)T.u;
+        T.off[0] = row * 128u + ((((uint32_t)T.g8) ^ (row & 7u)) << 4);
+        return T;
+    }
+    const int sw = (T.u == R.nv - 1) ? R.sw_last : p.g.w;
+    T.ntok = R.st * R.sh * sw;
+    int dt = 0, dh = 0, dw = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const uint32_t row = (uint32_t)((dt * p.bh + dh) * p.bw + T.u * p.g.w + dw);
+        T.off[i] = row * 128u + ((((uint32_t)T.g8) ^ (row & 7u)) << 4);
+        if (i + 1 < T.ntok && ++dw == sw) {
+            dw = 0;
+            if (++dh == R.sh) {
+                dh = 0;
+                ++dt;
+            }
+        }
+    }
+    return T;
+}
+
+// One token of a statistics task: running fp32 sum (pairs) and element-wise BF16 max / min.
+__device__ __forceinline__ void stat_token(const uint4 v, uint64_t (&acc)[4], uint32_t (&hi)[4], uint32_t (&lo)[4]) {
+    acc[0] = f2_add(acc[0], f2_from_bf16x2(v.x));
+    acc[1] = f2_add(acc[1], f2_from_bf16x2(v.y));
+    acc[2] = f2_add(acc[2], f2_from_bf16x2(v.z));
+    acc[3] = f2_add(acc[3], f2_from_bf16x2(v.w));
+    hi[0] = bf16x2_max(hi[0], v.x); lo[0] = bf16x2_min(lo[0], v.x);
+    hi[1] = bf16x2_max(hi[1], v.y); lo[1] = bf16x2_min(lo[1], v.y);
+    hi[2] = bf16x2_max(hi[2], v.z); lo[2] = bf16x2_min(lo[2], v.z);
+    hi[3] = bf16x2_max(hi[3], v.w); lo[3] = bf16x2_min(lo[3], v.w);
+}
+
+template <int N>
+__device__ __forceinline__ void stat_tokens(const uint8_t* xs, const uint32_t (&off)[8], uint64_t (&acc)[4],
+                                            uint32_t (&hi)[4], uint32_t (&lo)[4]) {
+#pragma unroll
+    for (int i = 1; i < N; i++) stat_token(*reinterpret_cast<const uint4*>(xs + off[i]), acc, hi, lo);
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -404,7 +476,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                                                                   QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const QSmem L = q_smem_layout(p.rank, true, p.tbl_rows);
+    const QSmem L = q_smem_layout(p.rank, true, 0);
     uint64_t* full = (uint64_t*)(sm + L.bars);
     uint64_t* empty = full + kQStages;
     uint64_t* accf = empty + kQStages;   // [2]
@@ -506,8 +578,11 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
         }
         __syncwarp();
     } else {
-        // ---------------- compute warps 0-7
-        float* tbl = (float*)(sm + L.tbl) + warp * p.tbl_rows * kMeanStride;
+        // ---------------- compute warps 0-7: thread = statistics task (unit x 8 channels).
+        // The largest |token - mean| of a cube and channel is |x_max - mean| or |x_min - mean|
+        // (fl(x - m) is monotone in x), so a cube's tokens are visited once: fp32 sum for the
+        // mean, BF16 max and min for the delta bound.
+        const int ntask = (int)cdiv((long long)(p.big ? p.bw : p.nw) * 8, kQCompute);
         float damax = 0.f;
         long long g = 0;
         int n = 0;
@@ -517,21 +592,8 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
             const int split = it % p.splits;
             const int c_base = split * nchunks * 64;
             const BoxRows R = box_rows(p, B);
-            const WarpRows W = warp_rows(R, warp);
-            const MeanTask T0m = mean_task(p, R, W, lane);
-            // this lane's row (two lanes per row, 32 channels each)
-            const int r = W.r_lo + (lane >> 1), half = lane & 1;
-            const bool has_row = r < W.r_hi;
-            int row = 0;
-            long long rho = 0;
-            if (has_row) list_row(p, B, R, r, &row, &rho);
-            const int jj_row = has_row ? cube_of_row(R, r) - W.j_lo : 0;
-            // shared-memory offsets of this lane's four 8-channel pieces of its row (128-byte swizzle)
-            uint32_t xoff[4];
-#pragma unroll
-            for (int v = 0; v < 4; v++) xoff[v] = (uint32_t)row * 128u + ((((uint32_t)(4 * half + v)) ^ ((uint32_t)row & 7u)) << 4);
-            const float* mrow = tbl + jj_row * kMeanStride + 32 * half;
-            float kam[4] = {0.f, 0.f, 0.f, 0.f};   // max |mean| of this lane's cube tasks
+            const StatTask T0 = stat_task(p, R, tid);
+            float kam[4] = {0.f, 0.f, 0.f, 0.f};   // max |mean| of this thread's cube tasks
             for (int i = 0; i < nchunks; i++, g++) {
                 const int s = (int)(g % kQStages);
                 ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)(g / kQStages) & 1, abort_flag, p.status,
@@ -539,48 +601,90 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                 if (!ok) break;
                 const uint8_t* xs = sm + L.x + s * 16384;
                 const int c0 = c_base + i * 64;
-                fill_means(p, R, W, T0m, xs, c0, tbl, lane);
-                __syncwarp();
-                if (!p.big) {
 #pragma unroll
-                    for (int t = 0; t < 4; t++) {
-                        const int q = lane + 32 * t;
-                        if (q < W.ncub * 8) {
-                            const float* src = tbl + (q >> 3) * kMeanStride + 8 * (q & 7);
-                            const float4 a = *reinterpret_cast<const float4*>(src);
-                            const float4 b = *reinterpret_cast<const float4*>(src + 4);
-                            kam[t] = fmaxf(kam[t], fmaxf(max3_abs(a.x, a.y, a.z), fmaxf(max3_abs(a.w, b.x, b.y),
-                                                                                       max3_abs(b.z, b.w, 0.f))));
+                for (int t = 0; t < 4; t++) {
+                    if (t >= ntask) break;
+                    const StatTask T = t == 0 ? T0 : stat_task(p, R, tid + kQCompute * t);
+                    if (!T.valid) continue;
+                    uint64_t m[4];
+                    if (p.big) {
+                        load8(p.means + (size_t)R.k0 * p.Ci + c0 + 8 * T.g8, m);
+                        damax = fmaxf(damax, max_abs_diff8(*reinterpret_cast<const uint4*>(xs + T.off[0]), m));
+                        continue;
+                    }
+                    // the sum starts at the first token (not at +0 + token: the two differ only in
+                    // the sign of an all-zero sum, and this kernel uses the mean only through |m|
+                    // and |x - m|)
+                    uint64_t acc[4];
+                    uint32_t hi[4], lo[4];
+                    if (T.ntok <= 8) {
+                        const uint4 v0 = *reinterpret_cast<const uint4*>(xs + T.off[0]);
+                        acc[0] = f2_from_bf16x2(v0.x);
+                        acc[1] = f2_from_bf16x2(v0.y);
+                        acc[2] = f2_from_bf16x2(v0.z);
+                        acc[3] = f2_from_bf16x2(v0.w);
+                        hi[0] = lo[0] = v0.x; hi[1] = lo[1] = v0.y; hi[2] = lo[2] = v0.z; hi[3] = lo[3] = v0.w;
+                        switch (T.ntok) {
+                            case 1: break;
+                            case 2: stat_tokens<2>(xs, T.off, acc, hi, lo); break;
+                            case 4: stat_tokens<4>(xs, T.off, acc, hi, lo); break;
+                            case 8: stat_tokens<8>(xs, T.off, acc, hi, lo); break;
+                            default:
+#pragma unroll
+                                for (int k = 1; k < 8; k++) {
+                                    if (k >= T.ntok) break;
+                                    stat_token(*reinterpret_cast<const uint4*>(xs + T.off[k]), acc, hi, lo);
+                                }
                         }
+                    } else {
+                        // larger cubes: walk the tokens in (t,h,w) order
+                        const int sw = (T.u == R.nv - 1) ? R.sw_last : p.g.w;
+                        bool first = true;
+                        for (int dt = 0; dt < R.st; dt++)
+                            for (int dh = 0; dh < R.sh; dh++) {
+                                const int row0 = (dt * p.bh + dh) * p.bw + T.u * p.g.w;
+                                for (int dw = 0; dw < sw; dw++) {
+                                    const uint4 v = ld_x8_swz(xs, row0 + dw, T.g8);
+                                    if (first) {
+                                        acc[0] = f2_from_bf16x2(v.x);
+                                        acc[1] = f2_from_bf16x2(v.y);
+                                        acc[2] = f2_from_bf16x2(v.z);
+                                        acc[3] = f2_from_bf16x2(v.w);
+                                        hi[0] = lo[0] = v.x; hi[1] = lo[1] = v.y; hi[2] = lo[2] = v.z; hi[3] = lo[3] = v.w;
+                                        first = false;
+                                    } else {
+                                        stat_token(v, acc, hi, lo);
+                                    }
+                                }
+                            }
                     }
-                }
-                if (has_row) {
-                    float a[4];
+                    mean_from_sum(acc, T.ntok, m);
+                    float mf[8];
 #pragma unroll
-                    for (int v = 0; v < 4; v++) {
-                        uint64_t m[4];
-                        load8(mrow + 8 * v, m);
-                        a[v] = max_abs_diff8(*reinterpret_cast<const uint4*>(xs + xoff[v]), m);
-                    }
-                    damax = max3_abs(damax, fmaxf(a[0], a[1]), fmaxf(a[2], a[3]));
+                    for (int e = 0; e < 4; e++) f2_unpack(m[e], mf[2 * e], mf[2 * e + 1]);
+                    kam[t] = fmaxf(kam[t], fmaxf(max3_abs(mf[0], mf[1], mf[2]),
+                                                 fmaxf(max3_abs(mf[3], mf[4], mf[5]), max3_abs(mf[6], mf[7], 0.f))));
+                    damax = fmaxf(damax, fmaxf(max_abs_diff8(make_uint4(hi[0], hi[1], hi[2], hi[3]), m),
+                                               max_abs_diff8(make_uint4(lo[0], lo[1], lo[2], lo[3]), m)));
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
             }
             if (!ok) break;
             // per-cube max |mean| over this item's channels -> kamax (small cubes; the means
-            // kernel has done it for big ones)
+            // kernel has done it for big ones); the eight threads of a cube are consecutive lanes
             if (!p.big) {
 #pragma unroll
                 for (int t = 0; t < 4; t++) {
-                    const int q = lane + 32 * t;
-                    if (q < W.ncub * 8) {
+                    if (t >= ntask) break;
+                    const int q = tid + kQCompute * t;
+                    if ((q >> 3) < R.nv) {
                         const uint32_t gm = 0xFFu << (lane & 24);
                         float v = kam[t];
                         v = fmaxf(v, __shfl_xor_sync(gm, v, 1));
                         v = fmaxf(v, __shfl_xor_sync(gm, v, 2));
                         v = fmaxf(v, __shfl_xor_sync(gm, v, 4));
-                        if ((q & 7) == 0) atomicMax(&p.kamax[R.k0 + W.j_lo + (q >> 3)], __float_as_uint(v));
+                        if ((q & 7) == 0) atomicMax(&p.kamax[R.k0 + (q >> 3)], __float_as_uint(v));
                     }
                 }
             }
@@ -964,7 +1068,7 @@ int resident_grid(const void* fn, int threads, size_t smem, int items) {
 
 cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
                               cudaStream_t st) {
-    size_t smem = quant_smem_bytes(p.rank, true, p.tbl_rows);
+    size_t smem = quant_smem_bytes(p.rank, true, 0);
     cudaError_t e = cudaFuncSetAttribute(k_cube_stats, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_cube_stats, cudaFuncAttributePreferredSharedMemoryCarveout,
