@@ -315,34 +315,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(acce0 + (uint32_t)(buf * 8));
                 if (row_ok) {
-                    const float4* prow = reinterpret_cast<const float4*>(p.p + (size_t)k * p.Nout + c_base);
+                    // 32-byte accesses: P' in 8-float pieces, Y in 16-value pieces
+                    const float* prow = p.p + (size_t)k * p.Nout + c_base;
                     uint16_t* yrow = p.Y + (size_t)n * p.Nout + c_base;
-                    float4 pa[8], pb[8];
+                    float pa[4][8], pb[4][8];
 #pragma unroll
-                    for (int v = 0; v < 8; v++) pa[v] = __ldg(prow + v);
+                    for (int v = 0; v < 4; v++) ld_global_nc_v8(prow + 8 * v, pa[v]);
 #pragma unroll
                     for (int c = 0; c < 128; c += 32) {
                         // software pipeline: the next 32 columns of P' are in flight while these are used
                         if (c + 32 < 128) {
 #pragma unroll
-                            for (int v = 0; v < 8; v++) pb[v] = __ldg(prow + (c + 32) / 4 + v);
+                            for (int v = 0; v < 4; v++) ld_global_nc_v8(prow + c + 32 + 8 * v, pb[v]);
                         }
-                        uint32_t pk[16];
+                        uint32_t pk[2][8];
 #pragma unroll
                         for (int v = 0; v < 32; v += 2) {
-                            const float4 q = pa[v / 4];
-                            const float a0 = (v & 2) ? q.z : q.x, a1 = (v & 2) ? q.w : q.y;
-                            pk[v / 2] = (uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(acc[c + v]), a0)) |
-                                        ((uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(acc[c + v + 1]), a1))
-                                         << 16);
+                            const float a0 = pa[v / 8][v % 8], a1 = pa[v / 8][v % 8 + 1];
+                            pk[v / 16][(v % 16) / 2] =
+                                (uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(acc[c + v]), a0)) |
+                                ((uint32_t)f32_to_bf16_rn(fmaf(SS, __uint_as_float(acc[c + v + 1]), a1)) << 16);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(yrow + c);
-                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                        dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
-                        dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+                        st_global_v8(yrow + c, pk[0]);
+                        st_global_v8(yrow + c + 16, pk[1]);
 #pragma unroll
-                        for (int v = 0; v < 8; v++) pa[v] = pb[v];
+                        for (int v = 0; v < 4; v++)
+#pragma unroll
+                            for (int e = 0; e < 8; e++) pa[v][e] = pb[v][e];
                     }
                 }
             } else {
@@ -359,14 +358,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld_x16(tacc + (uint32_t)c + 16, r1);
                     tmem_ld_wait();
                     if (row_ok) {
+                        // 32-byte stores
 #pragma unroll
-                        for (int v = 0; v < 16; v += 4) {
-                            *reinterpret_cast<float4*>(dst + c + v) =
-                                make_float4(__uint_as_float(r0[v]) * scale, __uint_as_float(r0[v + 1]) * scale,
-                                            __uint_as_float(r0[v + 2]) * scale, __uint_as_float(r0[v + 3]) * scale);
-                            *reinterpret_cast<float4*>(dst + c + 16 + v) =
-                                make_float4(__uint_as_float(r1[v]) * scale, __uint_as_float(r1[v + 1]) * scale,
-                                            __uint_as_float(r1[v + 2]) * scale, __uint_as_float(r1[v + 3]) * scale);
+                        for (int v = 0; v < 16; v += 8) {
+                            uint32_t o0[8], o1[8];
+#pragma unroll
+                            for (int e = 0; e < 8; e++) {
+                                o0[e] = __float_as_uint(__uint_as_float(r0[v + e]) * scale);
+                                o1[e] = __float_as_uint(__uint_as_float(r1[v + e]) * scale);
+                            }
+                            st_global_v8(dst + c + v, o0);
+                            st_global_v8(dst + c + 16 + v, o1);
                         }
                     }
                 }

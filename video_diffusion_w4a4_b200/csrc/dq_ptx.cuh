@@ -336,6 +336,21 @@ __device__ __forceinline__ void tmem_cp_pair_32x128b_x4(uint32_t taddr, uint64_t
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+// ------------------------------------------------------------------ 256-bit global access (sm_100)
+
+// Eight fp32 from 32-byte aligned global memory through the non-coherent path.
+__device__ __forceinline__ void ld_global_nc_v8(const float* src, float (&v)[8]) {
+    asm volatile("ld.global.nc.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+                 : "l"(src));
+}
+
+__device__ __forceinline__ void st_global_v8(void* dst, const uint32_t (&v)[8]) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(v[0]), "r"(v[1]),
+                 "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
 // ------------------------------------------------------------------ named barriers
 
 __device__ __forceinline__ void bar_sync(int id, int nthreads) {
