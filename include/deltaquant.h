@@ -99,6 +99,26 @@ int dq_cube_major_row(int T, int H, int W, int t, int h, int w, long long n, lon
 int dq_sf_offset(long long row, int block, int cols, size_t* offset);
 int dq_sf_bytes(long long rows, int cols, size_t* bytes);
 
+/*
+ * A-operand scale layout (the delta group scales in the workspace; cols a
+ * multiple of 256).  The block-scaled MMA reads the scales of row r of a
+ * 128-row tile from tensor-memory lane r, column (scale address + r / 32): the
+ * 32-lane quadrant q of the tensor memory uses the q-th 32-bit column of each
+ * 4-column group.  So one 128x256-bit copy per two 64-column blocks suffices
+ * (instead of one replicating 32x128-bit copy per block), from this layout:
+ * per 128-row group and 256-column K step, two 4096-byte blocks (one per pair
+ * of 64-column blocks), each 128 rows x 32 bytes stored as 8-row x 16-byte
+ * core matrices (row-group stride 256, column-half stride 128); row r holds
+ * the four scales of 64-column block kb at 32-bit word 4 (kb % 2) + r / 32:
+ *   offset = (((row/128) * (cols/256) + kb/4) * 2 + (kb/2) % 2) * 4096
+ *            + ((row%128)/8) * 256 + (kb % 2) * 128 + (row % 8) * 16
+ *            + ((row%128)/32) * 4 + block % 4,      kb = block / 4.
+ * A quarter of the bytes hold scales; the rest are never read.  Total size:
+ * ceil(rows/128) * (cols/256) * 8192.
+ */
+int dq_sfa_offset(long long row, int block, int cols, size_t* offset);
+int dq_sfa_bytes(long long rows, int cols, size_t* bytes);
+
 /* ------------------------------------------------------------------------ */
 /* Offline weight packing (host only, synchronous)                           */
 /* ------------------------------------------------------------------------ */
@@ -171,7 +191,7 @@ int dq_pack_weight(const uint16_t* W, int Co, int Ci, int rank, void* packed, si
  *   q8         K x Ci E4M3 kernel tokens
  *   q8_bf16    K_pad x Ci BF16 copy of q8 (the kernel-token product's A operand)
  *   dcodes     N x Ci/2 E2M1 delta codes, cube-major rows
- *   dscales    delta group scales, scale-factor layout over N rows
+ *   dscales    delta group scales, A-operand scale layout (dq_sfa_offset) over N rows
  *   u_part     splits x N x rank fp32 partial sums of X L1 (cube-major rows)
  *   u_hilo     N x slab BF16: U' = (X L1)/(S_delta S_W) split as hi + lo
  *   p          K x Co fp32: s8 S_W q8 dqw^T (the per-cube kernel term)

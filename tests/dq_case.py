@@ -22,6 +22,16 @@ def sf_unpermute(buf: np.ndarray, rows: int, cols: int) -> np.ndarray:
     return buf[off]
 
 
+def sfa_unpermute(buf: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """A-operand scale layout (include/deltaquant.h, dq_sfa_offset) -> plain rows x cols/16."""
+    r = np.arange(rows, dtype=np.int64)[:, None]
+    b = np.arange(cols // 16, dtype=np.int64)[None, :]
+    kb, rr = b // 4, r % 128
+    block = ((r // 128) * (cols // 256) + kb // 4) * 2 + (kb // 2) % 2
+    off = block * 4096 + (rr // 8) * 256 + (kb % 2) * 128 + (rr % 8) * 16 + (rr // 32) * 4 + b % 4
+    return buf[off]
+
+
 def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
@@ -81,7 +91,7 @@ class Case:
                    q8=wsh[lay.off_q8:lay.off_q8 + K * Ci].reshape(K, Ci),
                    q8_bf16=wsh[lay.off_q8_bf16:lay.off_q8_bf16 + 2 * K * Ci].view(np.uint16).reshape(K, Ci),
                    dcodes=wsh[lay.off_dcodes:lay.off_dcodes + N * Ci // 2].reshape(N, Ci // 2),
-                   dscales=sf_unpermute(wsh[lay.off_dscales:], N, Ci),
+                   dscales=sfa_unpermute(wsh[lay.off_dscales:], N, Ci),
                    p=wsh[lay.off_p:lay.off_p + 4 * K * wl.Co].view(np.float32).reshape(K, wl.Co))
         return out
 

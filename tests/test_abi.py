@@ -64,6 +64,31 @@ def test_sf_offset_is_a_bijection(dq):
     assert dq.dq_sf_bytes(129, 64) == 2 * 512
 
 
+def test_sfa_offset_places_each_scale_in_its_quadrant_column(dq):
+    """A-operand scale layout: injective; row r's scales of 64-column block kb land in the 16-byte
+    line (row r, column half kb % 2) of their 4 KB block, at 32-bit word r // 32 of that line, so that
+    after a 128x256-bit copy lane r holds them in tensor-memory column 4 (kb % 2) + r // 32."""
+    for rows, cols in ((128, 256), (256, 512), (300, 1024)):
+        total = dq.dq_sfa_bytes(rows, cols)
+        assert total == -(-rows // 128) * (cols // 256) * 8192
+        seen = np.zeros(total, bool)
+        for r in range(rows):
+            for b in range(cols // 16):
+                off = dq.dq_sfa_offset(r, b, cols)
+                assert not seen[off]
+                seen[off] = True
+                kb, rr = b // 4, r % 128
+                block, inner = divmod(off, 4096)
+                assert block == ((r // 128) * (cols // 256) + kb // 4) * 2 + (kb // 2) % 2
+                line, byte = divmod(inner, 16)
+                # core matrices of 8 rows x 16 bytes: row-group stride 256, column-half stride 128
+                assert line == (rr // 8) * 16 + (kb % 2) * 8 + rr % 8
+                assert byte == (rr // 32) * 4 + b % 4
+        assert seen.sum() == rows * cols // 16
+    with pytest.raises(dq.DQError):
+        dq.dq_sfa_offset(0, 0, 192)
+
+
 def test_layouts_are_aligned_and_ordered(dq):
     L = dq.dq_workspace_layout_get(21, 30, 52, 1, 2, 2, 5120, 5120, 32)
     offs = [L.off_status, L.off_scalars, L.off_kamax, L.off_s8, L.off_q8, L.off_q8_bf16, L.off_dcodes,

@@ -59,6 +59,8 @@ _SIGS = {
     "dq_cube_major_row": ([_I] * 6 + [_LL, ctypes.POINTER(_LL), ctypes.POINTER(_LL)], _I),
     "dq_sf_offset": ([_LL, _I, _I, ctypes.POINTER(_SZ)], _I),
     "dq_sf_bytes": ([_LL, _I, ctypes.POINTER(_SZ)], _I),
+    "dq_sfa_offset": ([_LL, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "dq_sfa_bytes": ([_LL, _I, ctypes.POINTER(_SZ)], _I),
     "dq_packed_weight_layout": ([_I, _I, _I, ctypes.POINTER(dq_packed_layout)], _I),
     "dq_packed_weight_bytes": ([_I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "dq_lowrank_slab_width": ([_I], _I),
@@ -139,6 +141,18 @@ def dq_sf_offset(row: int, block: int, cols: int) -> int:
     off = ctypes.c_size_t()
     _check("dq_sf_offset", _lib.dq_sf_offset(row, block, cols, ctypes.byref(off)))
     return off.value
+
+
+def dq_sfa_offset(row: int, block: int, cols: int) -> int:
+    off = _SZ()
+    _check("dq_sfa_offset", _lib.dq_sfa_offset(row, block, cols, ctypes.byref(off)))
+    return off.value
+
+
+def dq_sfa_bytes(rows: int, cols: int) -> int:
+    b = _SZ()
+    _check("dq_sfa_bytes", _lib.dq_sfa_bytes(rows, cols, ctypes.byref(b)))
+    return b.value
 
 
 def dq_sf_bytes(rows: int, cols: int) -> int:

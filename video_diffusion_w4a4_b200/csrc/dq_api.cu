@@ -81,6 +81,21 @@ bool map_sf(CUtensorMap* m, const void* base, int Ci, uint64_t row_groups, uint3
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over the A-operand scale layout (dq_sfa_offset): dim 0 the bytes of a
+// 256-byte line, dim 1 the 32 (Ci/256) lines of one 128-row group (8192 bytes
+// per K step of 256 channels), dim 2 the row groups.  Boxes of one K step.
+bool map_sfa(CUtensorMap* m, const void* base, int Ci, uint64_t row_groups) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {256, (cuuint64_t)Ci / 256 * 32, row_groups};
+    cuuint64_t strides[2] = {256, (cuuint64_t)Ci / 256 * 8192};
+    cuuint32_t box[3] = {256, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p) { return ((uintptr_t)p & 255u) == 0; }
 
 // Text of the last CUDA runtime error an entry point of this thread returned DQ_ERR_CUDA for.
@@ -293,7 +308,7 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
         if (!map_2d(&tm_sa, ws + wl.off_u_hilo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wl.slab, g.N, 64, 128))
             return map_fail("slab A");
         if (!map_2d(&tm_sb, L2_slab, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wl.slab, Co, 64, 128)) return map_fail("slab B");
-        if (!map_sf(&tm_fa, ws + wl.off_dscales, Ci, (uint64_t)dq::cdiv(g.N, 128), 1)) return map_fail("delta scales");
+        if (!map_sfa(&tm_fa, ws + wl.off_dscales, Ci, (uint64_t)dq::cdiv(g.N, 128))) return map_fail("delta scales");
         if (!map_sf(&tm_fb, pw + pl.off_scales, Ci, (uint64_t)(Co / 128), 2)) return map_fail("weight scales");
         dq::GemmParams p = gp;
         p.M = (int)g.N;

@@ -89,6 +89,19 @@ DQ_HD size_t sf_offset(long long row, int blk, int cols) {
 
 DQ_HD size_t sf_bytes(long long rows, int cols) { return (size_t)cdiv(rows, 128) * (size_t)(cols / 64) * 512; }
 
+// A-operand scale layout (the delta scales; see include/deltaquant.h): per
+// 128-row group and 256-column K step two 4 KB blocks, one per pair of
+// 64-column blocks, each 128 rows x 32 bytes in 8-row x 16-byte core matrices;
+// row r of the group holds the four scales of 64-column block kb at 32-bit
+// word 4 (kb % 2) + r / 32 of its 32 bytes (the other six words are unused).
+DQ_HD size_t sfa_offset(long long row, int blk, int cols) {
+    const int kb = blk >> 2, r = (int)(row & 127);
+    const long long block = ((row >> 7) * (long long)(cols >> 8) + (kb >> 2)) * 2 + ((kb >> 1) & 1);
+    return (size_t)block * 4096 + (size_t)((r >> 3) * 256 + (kb & 1) * 128 + (r & 7) * 16 + (r >> 5) * 4 + (blk & 3));
+}
+
+DQ_HD size_t sfa_bytes(long long rows, int cols) { return (size_t)cdiv(rows, 128) * (size_t)(cols / 256) * 8192; }
+
 DQ_HD int slab_width(int rank) { return (int)(cdiv(2 * rank, 64) * 64); }
 
 // Packed weight blob header (first 256 bytes of the blob).
@@ -152,7 +165,7 @@ DQ_HD WsLayout ws_layout(const Geom& g, int Ci, int Co, int rank) {
     L.off_q8 = off;       off = align_up(off + (size_t)g.K * Ci, kAlign);
     L.off_q8_bf16 = off;  off = align_up(off + (size_t)L.K_pad * Ci * 2, kAlign);
     L.off_dcodes = off;   off = align_up(off + (size_t)g.N * (Ci / 2), kAlign);
-    L.off_dscales = off;  off = align_up(off + sf_bytes(g.N, Ci), kAlign);
+    L.off_dscales = off;  off = align_up(off + sfa_bytes(g.N, Ci), kAlign);
     L.off_u_part = off;   off = align_up(off + (size_t)L.splits * g.N * rank * 4, kAlign);
     L.off_u_hilo = off;   off = align_up(off + (size_t)g.N * L.slab * 2, kAlign);
     L.off_p = off;        off = align_up(off + (size_t)g.K * Co * 4, kAlign);

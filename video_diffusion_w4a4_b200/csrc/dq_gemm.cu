@@ -51,7 +51,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = 96 + 32 * kEpiWarps;   // producer, MMA, scale-factor copies, epilogue
 constexpr uint32_t kABytes = kTileM * 128;      // 128 rows x 128 bytes
 constexpr uint32_t kBBytes = (kTileN / 2) * 128;  // this CTA's 128 rows of B x 128 bytes
-constexpr uint32_t kSFABytes = 4 * 512;         // 128 rows x 4 k-blocks of 64
+constexpr uint32_t kSFABytes = 2 * 4096;        // 128 rows x 4 k-blocks of 64, A-operand scale layout
 constexpr uint32_t kSFBBytes = 2 * 4 * 512;     // all 256 columns x 4 k-blocks (each CTA holds a copy)
 constexpr uint16_t kPairMask = 0x3;
 
@@ -172,8 +172,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes + kSFABytes + kSFBBytes));
                         tma_load_2d_pair(sa, &tm_a, fb, i * 128, m0);
                         tma_load_2d_pair(sb, &tm_b, fb, i * 128, nb);
-                        // scale factors: 4 k-blocks x 512 B per 128-row group = 8 lines of 256 B
-                        tma_load_3d_pair(sm + L.sfa + s * kSFABytes, &tm_fa, fb, 0, 8 * i, m0 >> 7);
+                        // scale factors: A 8192 B per 128-row group and K step (32 lines of 256 B),
+                        // B 4 k-blocks x 512 B per 128-row group (8 lines), for both row groups of the pair tile
+                        tma_load_3d_pair(sm + L.sfa + s * kSFABytes, &tm_fa, fb, 0, 32 * i, m0 >> 7);
                         tma_load_3d_pair(sm + L.sfb + s * kSFBBytes, &tm_fb, fb, 0, 8 * i, n0 >> 7);
                     } else {
                         if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes));
@@ -227,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int k = 0; k < 4; k++)
                             mma_nvfp4_pair(acc, desc_k_sw128(aa + 32 * k), desc_k_sw128(bb + 32 * k), id_main,
-                                           t_sfa + 4 * k, t_sfb + 8 * k, (i | k) != 0);
+                                           t_sfa + 8 * (k >> 1) + 4 * (k & 1), t_sfb + 8 * k, (i | k) != 0);
                     } else {
                         const uint32_t id = kMain ? id_slab : id_main;
 #pragma unroll
@@ -265,9 +266,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t t_sfa = t_sf0 + (uint32_t)(s * 48), t_sfb = t_sfa + 16;
                         const uint32_t fa = smem_u32(sm + L.sfa + s * kSFABytes);
                         const uint32_t fb = smem_u32(sm + L.sfb + s * kSFBBytes);
+                        // A: lane r receives 8 columns per copy, of which the MMA of k-block k reads
+                        // column 8 (k / 2) + 4 (k % 2) + r / 32; B: every quadrant needs every column's
+                        // scales, so they are replicated into the four 32-lane quadrants
+                        tmem_cp_pair_128x256b(t_sfa, smem_desc(fa, 128, 256, 0));
+                        tmem_cp_pair_128x256b(t_sfa + 8, smem_desc(fa + 4096, 128, 256, 0));
 #pragma unroll
                         for (int k = 0; k < 4; k++) {
-                            tmem_cp_pair_32x128b_x4(t_sfa + 4 * k, desc_sf(fa + 512 * k));
                             tmem_cp_pair_32x128b_x4(t_sfb + 8 * k, desc_sf(fb + 512 * k));
                             tmem_cp_pair_32x128b_x4(t_sfb + 8 * k + 4, desc_sf(fb + kSFBBytes / 2 + 512 * k));
                         }

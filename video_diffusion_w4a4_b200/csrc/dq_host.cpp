@@ -305,6 +305,18 @@ int dq_sf_bytes(long long rows, int cols, size_t* bytes) {
     return DQ_OK;
 }
 
+int dq_sfa_offset(long long row, int block, int cols, size_t* offset) {
+    if (!offset || row < 0 || cols <= 0 || cols % 256 || block < 0 || block >= cols / 16) return DQ_ERR_INVALID_ARG;
+    *offset = dq::sfa_offset(row, block, cols);
+    return DQ_OK;
+}
+
+int dq_sfa_bytes(long long rows, int cols, size_t* bytes) {
+    if (!bytes || rows < 0 || cols <= 0 || cols % 256) return DQ_ERR_INVALID_ARG;
+    *bytes = dq::sfa_bytes(rows, cols);
+    return DQ_OK;
+}
+
 int dq_lowrank_slab_width(int rank) { return (rank > 0) ? dq::slab_width(rank) : 0; }
 
 int dq_packed_weight_layout(int Co, int Ci, int rank, dq_packed_layout* out) {

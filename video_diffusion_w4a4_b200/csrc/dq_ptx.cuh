@@ -307,6 +307,12 @@ __device__ __forceinline__ void tc_commit_pair_both(uint64_t* bar, uint16_t cta_
         : "memory");
 }
 
+// 128 rows x 256 bits (8 columns per lane, no replication) from each CTA's
+// shared memory at `sdesc` to its own tensor memory at `taddr`.
+__device__ __forceinline__ void tmem_cp_pair_128x256b(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // Paired MMAs: M = 256 rows, 128 in each CTA's tensor memory; A and B are read
 // at the same shared-memory offsets in both CTAs (each holds half of B's rows).
 __device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,

@@ -913,7 +913,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                         codes[2 * b + 1] = w1;
                     }
                     *reinterpret_cast<uint4*>(dcode_row + c0 / 2) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-                    *reinterpret_cast<uint16_t*>(p.dscales + sf_offset(rho, c0 / 16 + 2 * half, Ci)) = (uint16_t)sc;
+                    *reinterpret_cast<uint16_t*>(p.dscales + sfa_offset(rho, c0 / 16 + 2 * half, Ci)) = (uint16_t)sc;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
