@@ -195,8 +195,7 @@ int dq_pack_weight(const uint16_t* W, int Co, int Ci, int rank, void* packed, si
  *   u_part     splits x N x rank fp32 partial sums of X L1 (cube-major rows)
  *   u_hilo     N x slab BF16: U' = (X L1)/(S_delta S_W) split as hi + lo
  *   p          K x Co fp32: s8 S_W q8 dqw^T (the per-cube kernel term)
- *   means      K x Ci fp32 kernel tokens before quantisation, only for cubes
- *              of more than 128 tokens (size 0 otherwise)
+ *   means      K x Ci fp32 kernel tokens before quantisation
  */
 typedef struct dq_workspace_layout {
     size_t total_bytes;

@@ -96,6 +96,19 @@ bool map_sfa(CUtensorMap* m, const void* base, int Ci, uint64_t row_groups) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over the K x Ci fp32 kernel tokens, boxes of 64 channels x `rows` consecutive cubes.
+bool map_means(CUtensorMap* m, const void* base, int Ci, long long K, int rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)Ci, (cuuint64_t)K};
+    cuuint64_t strides[1] = {(cuuint64_t)Ci * 4};
+    cuuint32_t box[2] = {64, (cuuint32_t)rows};
+    cuuint32_t estr[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned(const void* p) { return ((uintptr_t)p & 255u) == 0; }
 
 // Text of the last CUDA runtime error an entry point of this thread returned DQ_ERR_CUDA for.
@@ -229,10 +242,7 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
         qp.bh = h;
         qp.bw = qp.nw * w;
         qp.n_boxes = g.KT * g.KH * qp.nbw;
-        // 16 consecutive cube-major rows touch at most ceil(15 / n) + 1 cubes of n tokens;
-        // the boxes of the last slab in t or row in h hold the cubes cut shortest
-        const int n_min = (T - (g.KT - 1) * t) * (H - (g.KH - 1) * h) * w;
-        qp.tbl_rows = dq::imin(16, (int)dq::cdiv(15, n_min) + 1);
+        qp.m_rows = qp.nw;
     } else {
         // boxes are segments of up to 128 tokens of one (t, h) row inside one cube
         qp.nw = 1;
@@ -242,9 +252,9 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
         qp.nseg = (int)dq::cdiv(w, 128);
         qp.nbw = g.KW * qp.nseg;
         qp.n_boxes = g.T * g.H * qp.nbw;
-        qp.means = (float*)(ws + wl.off_means);
-        qp.tbl_rows = 1;
+        qp.m_rows = 1;
     }
+    qp.means = (float*)(ws + wl.off_means);
     qp.status = (int*)(ws + wl.off_status);
     qp.scalars = (uint32_t*)(ws + wl.off_scalars);
     qp.kamax = (uint32_t*)(ws + wl.off_kamax);
@@ -273,16 +283,17 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
     };
     rec(0);
     if (stage_mask & DQ_STAGE_QUANTIZE) {
-        CUtensorMap tm_x, tm_l1;
+        CUtensorMap tm_x, tm_l1, tm_m;
         cudaError_t e0;
         if (!map_x(&tm_x, X, g, Ci, qp.bw, qp.bh, qp.bt)) return map_fail("X");
+        if (!map_means(&tm_m, ws + wl.off_means, Ci, g.K, qp.m_rows)) return map_fail("kernel tokens");
         if (!map_2d(&tm_l1, L1_mma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, rank, 64, rank)) return map_fail("L1");
         if ((e0 = cudaMemsetAsync(ws + wl.off_scalars, 0, 16, st)) != cudaSuccess) return cuda_fail(e0, "memset");
         if ((e0 = cudaMemsetAsync(ws + wl.off_kamax, 0, (size_t)g.K * 4, st)) != cudaSuccess) return cuda_fail(e0, "memset");
         cudaError_t e;
         if (qp.big && (e = dq::launch_cube_means_big(tm_x, qp, st)) != cudaSuccess) return cuda_fail(e, "k_cube_means_big");
         if ((e = dq::launch_cube_stats(tm_x, tm_l1, qp, st)) != cudaSuccess) return cuda_fail(e, "k_cube_stats");
-        if ((e = dq::launch_cube_encode(tm_x, qp, st)) != cudaSuccess) return cuda_fail(e, "k_cube_encode");
+        if ((e = dq::launch_cube_encode(tm_x, tm_m, qp, st)) != cudaSuccess) return cuda_fail(e, "k_cube_encode");
     }
     rec(1);
     if (stage_mask & DQ_STAGE_KERNEL_GEMM) {

@@ -169,8 +169,8 @@ DQ_HD WsLayout ws_layout(const Geom& g, int Ci, int Co, int rank) {
     L.off_u_part = off;   off = align_up(off + (size_t)L.splits * g.N * rank * 4, kAlign);
     L.off_u_hilo = off;   off = align_up(off + (size_t)g.N * L.slab * 2, kAlign);
     L.off_p = off;        off = align_up(off + (size_t)g.K * Co * 4, kAlign);
-    // fp32 kernel tokens, only for cubes of more than 128 tokens (computed by a kernel of their own)
-    L.off_means = off;    off = align_up(off + ((long long)g.t * g.h * g.w > 128 ? (size_t)g.K * Ci * 4 : 0), kAlign);
+    // fp32 kernel tokens (written by the statistics pass, read by the encode pass)
+    L.off_means = off;    off = align_up(off + (size_t)g.K * Ci * 4, kAlign);
     L.total = off;
     return L;
 }

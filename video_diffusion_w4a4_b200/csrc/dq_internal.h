@@ -17,10 +17,10 @@ struct QuantParams {
     int bt, bh, bw;     // box extent in tokens: t x h x (nw w)
     int nbw;            // boxes along w
     int n_boxes;
-    int tbl_rows;       // rows of each compute warp's table of means
+    int m_rows;         // kernel tokens per box (rows of the encode kernel's per-stage tile)
     int big;            // cubes of more than 128 tokens: boxes are row segments of one cube,
     int nseg;           //   nseg segments of up to 128 tokens per cube row; the kernel tokens
-    float* means;       //   come from `means` (K x Ci fp32), written by k_cube_means_big
+    float* means;       //   K x Ci fp32 kernel tokens: written by k_cube_stats (by k_cube_means_big for big cubes)
     int* status;
     uint32_t* scalars;  // [0] bits of max|delta|, [1] S_delta
     uint32_t* kamax;
@@ -52,10 +52,11 @@ struct GemmParams {
     uint64_t budget_ns;
 };
 
-size_t quant_smem_bytes(int rank, bool stats, int tbl_rows);
+size_t quant_smem_bytes(int rank, bool stats, int m_rows);
 cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
                               cudaStream_t st);
-cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const QuantParams& p, cudaStream_t st);
+cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const CUtensorMap& tm_m, const QuantParams& p,
+                               cudaStream_t st);
 cudaError_t launch_cube_means_big(const CUtensorMap& tm_x, const QuantParams& p, cudaStream_t st);
 
 cudaError_t launch_kernel_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmParams& p,

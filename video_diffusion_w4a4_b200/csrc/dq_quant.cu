@@ -4,9 +4,10 @@
 //       max |mean| over channels (the FP8 kernel-token scale), the global
 //       max |token - mean| (the FP4 per-tensor scale), and X L1 (the SVD
 //       low-rank down-projection of Eq. 3) on the tensor cores.
-//   a2  k_cube_encode: recomputes the same means bit for bit, writes the FP8
-//       E4M3 kernel tokens, the FP4 E2M1 delta codes with their E4M3 group-16
-//       scales (Eq. 4 per group), and U' = (X L1) / (S_delta S_W) as BF16 hi+lo.
+//       It stores the means (K x Ci fp32) for the second pass.
+//   a2  k_cube_encode: reads X and the means again, writes the FP8 E4M3 kernel
+//       tokens, the FP4 E2M1 delta codes with their E4M3 group-16 scales (Eq. 4
+//       per group), and U' = (X L1) / (S_delta S_W) as BF16 hi+lo.
 //
 // Both stream X through 4-D TMA boxes of t x h x (nw w) tokens by 64
 // channels straight from the flattened (t,h,w) layout, so that every box
@@ -16,13 +17,11 @@
 // Work item = (box, channel split): the box's tokens over Ci / splits
 // channels (chunks of 64).  The kernels are persistent: each CTA walks items
 // it = blockIdx.x + n * gridDim.x and one producer thread streams all their
-// chunks through one TMA ring.  The box's tokens are listed in cube-major
-// order and every compute warp owns 16 consecutive rows of that list: it
-// first forms the means of the cubes its rows touch (lane = cube x 8
-// channels) in a table of its own, then encodes its rows (two lanes per row,
-// 32 channels each).  A cube that spans two warps has its mean formed by
-// both (the same sequential sum), so the compute warps never wait on one
-// another.
+// chunks through one TMA ring.  In a1 a thread owns one (cube, 8 channels)
+// task.  In a2 the box's tokens are listed in cube-major order and every
+// compute warp owns 16 consecutive rows of that list (two lanes per row, 32
+// channels each), with the box's kernel tokens streamed in next to X, so the
+// compute warps never wait on one another.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -38,24 +37,24 @@ constexpr int kQStages = 4;
 constexpr int kQWarps = 8;                 // compute warps
 constexpr int kQCompute = 32 * kQWarps;
 
-constexpr int kMeanStride = 68;            // floats per row of a warp's table of means (bank spread)
-
 struct QSmem {
     // offsets in bytes from the 1024-aligned dynamic smem base
-    uint32_t x, l1, tbl, bars, misc, total;
+    uint32_t x, l1, mt, mt_stride, eff, bars, misc, total;
 };
 
-// tbl_rows: rows of each compute warp's table of means (the cube slots that 16
-// consecutive cube-major rows can touch)
-__host__ __device__ inline QSmem q_smem_layout(int rank, bool with_l1, int tbl_rows) {
+// m_rows: rows of the per-stage tile of kernel tokens (encode kernel; 0 for the statistics kernel)
+__host__ __device__ inline QSmem q_smem_layout(int rank, bool with_l1, int m_rows) {
     QSmem L;
     uint32_t off = 0;
     L.x = off;
     off += kQStages * 16384;
     L.l1 = off;
     if (with_l1) off += kQStages * (uint32_t)align_up((size_t)rank * 128, 1024);
-    L.tbl = off;
-    off += (uint32_t)kQWarps * tbl_rows * kMeanStride * 4;
+    L.mt = off;
+    L.mt_stride = (uint32_t)align_up((size_t)m_rows * 256, 128);
+    off += kQStages * L.mt_stride;
+    L.eff = off;                 // 128 (eff, 1/eff) pairs, one per non-negative E4M3 scale code
+    off += 128 * 8;
     L.bars = off;
     off += (2 * kQStages + 6) * 8;
     L.misc = off;
@@ -188,52 +187,11 @@ __device__ __forceinline__ void list_row(const QuantParams& p, const BoxPos& B, 
     *rho = cube_first_row(p.g, B.bkt, B.bkh, B.bkw * p.nw + j) + i;
 }
 
-// Kernel token (Eq. 1) of cube slot j for channels [8 g8, 8 g8 + 8) of the
-// chunk: an fp32 running sum over the cube's tokens in (t,h,w) order, then the
-// division by the token count (a product with the exact reciprocal when the
-// count is a power of two, which gives the identical rounding).
-__device__ __forceinline__ void cube_mean8(const QuantParams& p, const BoxRows& R, const uint8_t* xs, int j, int g8,
-                                           uint64_t (&m)[4]) {
-    const int sw = (j == R.nv - 1) ? R.sw_last : p.g.w;
-    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // (+0, +0) pairs
-    for (int dt = 0; dt < R.st; dt++)
-        for (int dh = 0; dh < R.sh; dh++) {
-            const int row0 = (dt * p.bh + dh) * p.bw + j * p.g.w;
-#pragma unroll 2
-            for (int dw = 0; dw < sw; dw++) {
-                const uint4 v = ld_x8_swz(xs, row0 + dw, g8);
-                acc[0] = f2_add(acc[0], f2_from_bf16x2(v.x));
-                acc[1] = f2_add(acc[1], f2_from_bf16x2(v.y));
-                acc[2] = f2_add(acc[2], f2_from_bf16x2(v.z));
-                acc[3] = f2_add(acc[3], f2_from_bf16x2(v.w));
-            }
-        }
-    const int cnt = R.st * R.sh * sw;
-    if ((cnt & (cnt - 1)) == 0) {
-        const float inv = __frcp_rn((float)cnt);
-        const uint64_t inv2 = f2_pack(inv, inv);
-#pragma unroll
-        for (int e = 0; e < 4; e++) m[e] = f2_mul(acc[e], inv2);
-    } else {
-#pragma unroll
-        for (int e = 0; e < 4; e++) {
-            float a, b;
-            f2_unpack(acc[e], a, b);
-            m[e] = f2_pack(__fdiv_rn(a, (float)cnt), __fdiv_rn(b, (float)cnt));
-        }
-    }
-}
-
 // Eight fp32 values as four packed pairs (16-byte aligned).
 __device__ __forceinline__ void load8(const float* src, uint64_t (&m)[4]) {
     const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(src);
     const ulonglong2 b = *reinterpret_cast<const ulonglong2*>(src + 4);
     m[0] = a.x; m[1] = a.y; m[2] = b.x; m[3] = b.y;
-}
-
-__device__ __forceinline__ void store8(float* dst, const uint64_t (&m)[4]) {
-    *reinterpret_cast<ulonglong2*>(dst) = make_ulonglong2(m[0], m[1]);
-    *reinterpret_cast<ulonglong2*>(dst + 4) = make_ulonglong2(m[2], m[3]);
 }
 
 // max |x - m| over 8 channels: x as four BF16 words, m as four fp32 pairs
@@ -265,56 +223,6 @@ __device__ __forceinline__ WarpRows warp_rows(const BoxRows& R, int warp) {
     return W;
 }
 
-// Phase 1 of a chunk: the kernel tokens of the warp's cubes into its table
-// (row jj = cube slot j_lo + jj, kMeanStride floats).  Big cubes: the means of
-// the box's one cube, computed by the means kernel.
-// Phase-1 task of a lane for one item (small cubes): cube slot jj of the warp's
-// table, channel group g8, and for cubes of up to 8 tokens the shared-memory
-// offsets of its tokens (fixed for all chunks of the item).
-struct MeanTask {
-    int jj, g8, j, ntok;   // ntok 0: no task
-    uint32_t off[8];
-};
-
-__device__ __forceinline__ MeanTask mean_task(const QuantParams& p, const BoxRows& R, const WarpRows& W, int q) {
-    MeanTask T;
-    T.jj = q >> 3;
-    T.g8 = q & 7;
-    T.j = W.j_lo + T.jj;
-    T.ntok = 0;
-    if (p.big || q >= W.ncub * 8) return T;
-    const int sw = (T.j == R.nv - 1) ? R.sw_last : p.g.w;
-    T.ntok = R.st * R.sh * sw;
-    // tokens in (t,h,w) order; entries past ntok repeat the last token (never read)
-    int dt = 0, dh = 0, dw = 0;
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-        const uint32_t row = (uint32_t)((dt * p.bh + dh) * p.bw + T.j * p.g.w + dw);
-        T.off[i] = row * 128u + ((((uint32_t)T.g8) ^ (row & 7u)) << 4);
-        if (i + 1 < T.ntok && ++dw == sw) {
-            dw = 0;
-            if (++dh == R.sh) {
-                dh = 0;
-                ++dt;
-            }
-        }
-    }
-    return T;
-}
-
-// fp32 running sum of N tokens of one 8-channel group in (t,h,w) order
-template <int N>
-__device__ __forceinline__ void sum_tokens(const uint8_t* xs, const uint32_t (&off)[8], uint64_t (&acc)[4]) {
-#pragma unroll
-    for (int i = 0; i < N; i++) {
-        const uint4 v = *reinterpret_cast<const uint4*>(xs + off[i]);
-        acc[0] = f2_add(acc[0], f2_from_bf16x2(v.x));
-        acc[1] = f2_add(acc[1], f2_from_bf16x2(v.y));
-        acc[2] = f2_add(acc[2], f2_from_bf16x2(v.z));
-        acc[3] = f2_add(acc[3], f2_from_bf16x2(v.w));
-    }
-}
-
 __device__ __forceinline__ void mean_from_sum(const uint64_t (&acc)[4], int cnt, uint64_t (&m)[4]) {
     if ((cnt & (cnt - 1)) == 0) {
         const float inv = __frcp_rn((float)cnt);
@@ -328,59 +236,6 @@ __device__ __forceinline__ void mean_from_sum(const uint64_t (&acc)[4], int cnt,
             f2_unpack(acc[e], a, b);
             m[e] = f2_pack(__fdiv_rn(a, (float)cnt), __fdiv_rn(b, (float)cnt));
         }
-    }
-}
-
-// Phase 1 of a chunk: the kernel tokens of the warp's cubes into its table
-// (row jj = cube slot j_lo + jj, kMeanStride floats).  T0 is this lane's first
-// task (q = lane) with its token offsets; further tasks (only when the warp's
-// rows touch more than four cubes) take the generic path.  Big cubes: the
-// means of the box's one cube, computed by the means kernel.
-__device__ __forceinline__ void fill_means(const QuantParams& p, const BoxRows& R, const WarpRows& W,
-                                           const MeanTask& T0, const uint8_t* xs, int c0, float* tbl, int lane) {
-    if (p.big) {
-        if (W.ncub > 0 && lane < 16) {
-            const float4 v = *reinterpret_cast<const float4*>(p.means + (size_t)R.k0 * p.Ci + c0 + 4 * lane);
-            *reinterpret_cast<float4*>(tbl + 4 * lane) = v;
-        }
-        return;
-    }
-    if (T0.ntok > 0) {
-        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // (+0, +0) pairs
-        switch (T0.ntok) {
-            case 1: sum_tokens<1>(xs, T0.off, acc); break;
-            case 2: sum_tokens<2>(xs, T0.off, acc); break;
-            case 4: sum_tokens<4>(xs, T0.off, acc); break;
-            case 8: sum_tokens<8>(xs, T0.off, acc); break;
-            default:
-                if (T0.ntok <= 8) {
-#pragma unroll
-                    for (int i = 0; i < 8; i++) {
-                        if (i >= T0.ntok) break;
-                        const uint4 v = *reinterpret_cast<const uint4*>(xs + T0.off[i]);
-                        acc[0] = f2_add(acc[0], f2_from_bf16x2(v.x));
-                        acc[1] = f2_add(acc[1], f2_from_bf16x2(v.y));
-                        acc[2] = f2_add(acc[2], f2_from_bf16x2(v.z));
-                        acc[3] = f2_add(acc[3], f2_from_bf16x2(v.w));
-                    }
-                } else {
-                    uint64_t m[4];
-                    cube_mean8(p, R, xs, T0.j, T0.g8, m);
-                    store8(tbl + T0.jj * kMeanStride + 8 * T0.g8, m);
-                    break;
-                }
-        }
-        if (T0.ntok <= 8) {
-            uint64_t m[4];
-            mean_from_sum(acc, T0.ntok, m);
-            store8(tbl + T0.jj * kMeanStride + 8 * T0.g8, m);
-        }
-    }
-    for (int q = lane + 32; q < W.ncub * 8; q += 32) {
-        const int jj = q >> 3, g8 = q & 7;
-        uint64_t m[4];
-        cube_mean8(p, R, xs, W.j_lo + jj, g8, m);
-        store8(tbl + jj * kMeanStride + 8 * g8, m);
     }
 }
 
@@ -612,17 +467,16 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                         damax = fmaxf(damax, max_abs_diff8(*reinterpret_cast<const uint4*>(xs + T.off[0]), m));
                         continue;
                     }
-                    // the sum starts at the first token (not at +0 + token: the two differ only in
-                    // the sign of an all-zero sum, and this kernel uses the mean only through |m|
-                    // and |x - m|)
+                    // fp32 running sum from +0 in (t,h,w) order (Eq. 1; +0 + x keeps the sign of
+                    // an all-zero sum as the sequential definition has it)
                     uint64_t acc[4];
                     uint32_t hi[4], lo[4];
                     if (T.ntok <= 8) {
                         const uint4 v0 = *reinterpret_cast<const uint4*>(xs + T.off[0]);
-                        acc[0] = f2_from_bf16x2(v0.x);
-                        acc[1] = f2_from_bf16x2(v0.y);
-                        acc[2] = f2_from_bf16x2(v0.z);
-                        acc[3] = f2_from_bf16x2(v0.w);
+                        acc[0] = f2_add(0ull, f2_from_bf16x2(v0.x));
+                        acc[1] = f2_add(0ull, f2_from_bf16x2(v0.y));
+                        acc[2] = f2_add(0ull, f2_from_bf16x2(v0.z));
+                        acc[3] = f2_add(0ull, f2_from_bf16x2(v0.w));
                         hi[0] = lo[0] = v0.x; hi[1] = lo[1] = v0.y; hi[2] = lo[2] = v0.z; hi[3] = lo[3] = v0.w;
                         switch (T.ntok) {
                             case 1: break;
@@ -646,10 +500,10 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                                 for (int dw = 0; dw < sw; dw++) {
                                     const uint4 v = ld_x8_swz(xs, row0 + dw, T.g8);
                                     if (first) {
-                                        acc[0] = f2_from_bf16x2(v.x);
-                                        acc[1] = f2_from_bf16x2(v.y);
-                                        acc[2] = f2_from_bf16x2(v.z);
-                                        acc[3] = f2_from_bf16x2(v.w);
+                                        acc[0] = f2_add(0ull, f2_from_bf16x2(v.x));
+                                        acc[1] = f2_add(0ull, f2_from_bf16x2(v.y));
+                                        acc[2] = f2_add(0ull, f2_from_bf16x2(v.z));
+                                        acc[3] = f2_add(0ull, f2_from_bf16x2(v.w));
                                         hi[0] = lo[0] = v.x; hi[1] = lo[1] = v.y; hi[2] = lo[2] = v.z; hi[3] = lo[3] = v.w;
                                         first = false;
                                     } else {
@@ -659,6 +513,12 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                             }
                     }
                     mean_from_sum(acc, T.ntok, m);
+                    {
+                        const uint32_t mw[8] = {(uint32_t)m[0], (uint32_t)(m[0] >> 32), (uint32_t)m[1],
+                                                (uint32_t)(m[1] >> 32), (uint32_t)m[2], (uint32_t)(m[2] >> 32),
+                                                (uint32_t)m[3], (uint32_t)(m[3] >> 32)};
+                        st_global_v8(p.means + (size_t)(R.k0 + T.u) * p.Ci + c0 + 8 * T.g8, mw);
+                    }
                     float mf[8];
 #pragma unroll
                     for (int e = 0; e < 4; e++) f2_unpack(m[e], mf[2 * e], mf[2 * e + 1]);
@@ -735,10 +595,11 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
 // Warps 0-7 compute, warp 8 loads.
 
 __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_constant__ CUtensorMap tm_x,
+                                                                  const __grid_constant__ CUtensorMap tm_m,
                                                                   QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const QSmem L = q_smem_layout(p.rank, false, p.tbl_rows);
+    const QSmem L = q_smem_layout(p.rank, false, p.m_rows);
     uint64_t* full = (uint64_t*)(sm + L.bars);
     uint64_t* empty = full + kQStages;
     volatile int* abort_flag = (volatile int*)(sm + L.misc + 8);
@@ -747,6 +608,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
     const int nchunks = p.chunks_per_split;
     const int n_items = p.n_boxes * p.splits;
     const uint32_t x_bytes = (uint32_t)p.bt * p.bh * p.bw * 128u;
+    const uint32_t m_bytes = (uint32_t)p.m_rows * 256u;   // the box's kernel tokens for 64 channels
     const int Ci = p.Ci;
 
     const PackedHeader* hdr = reinterpret_cast<const PackedHeader*>(p.packed_w);
@@ -767,15 +629,24 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
     const float denom = __fmul_rn(6.f, S);
     const float rdenom = __frcp_rn(denom);
     if (blockIdx.x == 0 && tid == 0) p.scalars[1] = __float_as_uint(S);
+    // group scale s_b (E4M3 code c) -> effective scale eff = fl(s_b S) and fl(1 / eff), for every
+    // code a group's amax can produce (non-negative, finite)
+    float2* efft = (float2*)(sm + L.eff);
+    if (tid < 128) {
+        const float e = __fmul_rn(e4m3_to_f32((uint32_t)tid), S);
+        efft[tid] = make_float2(e, (e != 0.f) ? __frcp_rn(e) : 0.f);
+    }
     __syncthreads();
 
     if (warp == 8) {
         if (lane == 0) {
             prefetch_tmap(&tm_x);
+            prefetch_tmap(&tm_m);
             long long g = 0;
             bool alive = true;
             for (int it = blockIdx.x; alive && it < n_items; it += gridDim.x) {
                 const BoxPos B = box_pos(p, it / p.splits);
+                const int k0 = (int)box_rows(p, B).k0;
                 const int c_base = (it % p.splits) * nchunks * 64;
                 for (int i = 0; i < nchunks; i++, g++) {
                     const int s = (int)(g % kQStages);
@@ -784,15 +655,15 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                         alive = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[s], x_bytes);
+                    mbar_arrive_expect_tx(&full[s], x_bytes + m_bytes);
                     tma_load_4d(sm + L.x + s * 16384, &tm_x, &full[s], c_base + i * 64, B.w0, B.h0, B.t0);
+                    tma_load_2d(sm + L.mt + s * L.mt_stride, &tm_m, &full[s], c_base + i * 64, k0);
                 }
             }
             for (long long q = (g > kQStages ? g - kQStages : 0); q < g; q++)
                 mbar_wait(&full[q % kQStages], (uint32_t)(q / kQStages) & 1, abort_flag, nullptr, p.budget_ns, false);
         }
     } else {
-        float* tbl = (float*)(sm + L.tbl) + warp * p.tbl_rows * kMeanStride;
         const float SS = __fmul_rn(S, hdr->S_W);
         long long g = 0;
         bool ok = true;
@@ -802,17 +673,16 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
             const int c_base = split * nchunks * 64;
             const BoxRows R = box_rows(p, B);
             const WarpRows W = warp_rows(R, warp);
-            const MeanTask T0m = mean_task(p, R, W, lane);
             const int r = W.r_lo + (lane >> 1), half = lane & 1;
             const bool has_row = r < W.r_hi;
             int row = 0;
             long long rho = 0;
             if (has_row) list_row(p, B, R, r, &row, &rho);
-            const int jj_row = has_row ? cube_of_row(R, r) - W.j_lo : 0;
+            // the row's kernel tokens in the stage's tile (row = cube slot of the box, 64 fp32)
+            const uint32_t moff = (uint32_t)(has_row ? cube_of_row(R, r) : 0) * 256u + 128u * half;
             uint32_t xoff[4];
 #pragma unroll
             for (int v = 0; v < 4; v++) xoff[v] = (uint32_t)row * 128u + ((((uint32_t)(4 * half + v)) ^ ((uint32_t)row & 7u)) << 4);
-            const float* mrow = tbl + jj_row * kMeanStride + 32 * half;
             uint8_t* dcode_row = p.dcodes + (size_t)rho * (Ci / 2) + 16 * half;
             // the kernel tokens of a cube are encoded by the warp that holds the cube's
             // first row (big cubes: by warp 0 of the cube's first box)
@@ -833,9 +703,8 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                                                        p.budget_ns));
                 if (!ok) break;
                 const uint8_t* xs = sm + L.x + s * 16384;
+                const float* mt = (const float*)(sm + L.mt + s * L.mt_stride);
                 const int c0 = c_base + i * 64;
-                fill_means(p, R, W, T0m, xs, c0, tbl, lane);
-                __syncwarp();
                 // kernel tokens: FP8 E4M3 codes under s8 = max|mean| / 448, and their exact BF16 copy
                 for (int q = q_first; q < W.ncub * 8; q += 32) {
                     const int jj = q >> 3, g8 = q & 7;
@@ -846,7 +715,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                         if (split == 0 && i == 0 && g8 == 0) p.s8[k] = s8;
                     }
                     uint64_t m[4];
-                    load8(tbl + jj * kMeanStride + 8 * g8, m);
+                    load8(mt + (W.j_lo + jj) * 64 + 8 * g8, m);
                     uint32_t c[4] = {0u, 0u, 0u, 0u};
                     if (s8 != 0.f) {
                         // codes of the negated quotients with the sign bit of each byte flipped
@@ -872,6 +741,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                 }
                 // delta tokens: FP4 E2M1 with E4M3 group-16 scales under S (two groups per lane)
                 if (has_row) {
+                    const float* mrow = (const float*)((const uint8_t*)mt + moff);
                     uint32_t codes[4];
                     uint32_t sc = 0;
 #pragma unroll
@@ -894,14 +764,16 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                             fmaxf(max3_abs(zf[0], zf[1], zf[2]), max3_abs(zf[3], zf[4], zf[5])),
                             fmaxf(fmaxf(max3_abs(zf[6], zf[7], zf[8]), max3_abs(zf[9], zf[10], zf[11])),
                                   fmaxf(max3_abs(zf[12], zf[13], zf[14]), fabsf(zf[15]))));
-                        const uint32_t sb = cvt_e4m3x2(div_pos(am, denom, rdenom), 0.f) & 0xFFu;
-                        const float eff = __fmul_rn(e4m3_to_f32(sb), S);
+                        // am >= 0, so the code is one of 0x00..0x7E
+                        const uint32_t sb = cvt_e4m3x2(div_pos(am, denom, rdenom), 0.f) & 0x7Fu;
+                        const float2 er = efft[sb];
+                        const float eff = er.x;
                         sc |= sb << (8 * b);
                         uint32_t w0 = 0, w1 = 0;
                         if (eff != 0.f) {
                             // codes of the negated quotients, then every nibble's sign bit flipped
                             // (E2M1 is sign-magnitude: code(-v) = code(v) ^ 8, signed zeros included)
-                            const float reff = __frcp_rn(eff);
+                            const float reff = er.y;
                             const uint64_t b2 = f2_pack(eff, eff), nrb2 = f2_pack(-reff, -reff);
                             float n[16];
 #pragma unroll
@@ -1037,8 +909,8 @@ cudaError_t launch_cube_means_big(const CUtensorMap& tm_x, const QuantParams& p,
     return cudaGetLastError();
 }
 
-size_t quant_smem_bytes(int rank, bool stats, int tbl_rows) {
-    return q_smem_layout(rank, stats, tbl_rows).total + 1024;
+size_t quant_smem_bytes(int rank, bool stats, int m_rows) {
+    return q_smem_layout(rank, stats, m_rows).total + 1024;
 }
 
 namespace {
@@ -1079,15 +951,16 @@ cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1,
     return cudaGetLastError();
 }
 
-cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const QuantParams& p, cudaStream_t st) {
-    size_t smem = quant_smem_bytes(p.rank, false, p.tbl_rows);
+cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const CUtensorMap& tm_m, const QuantParams& p,
+                               cudaStream_t st) {
+    size_t smem = quant_smem_bytes(p.rank, false, p.m_rows);
     cudaError_t e = cudaFuncSetAttribute(k_cube_encode, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_cube_encode, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     const int grid = resident_grid((const void*)k_cube_encode, kQCompute + 32, smem, p.n_boxes * p.splits);
-    k_cube_encode<<<grid, kQCompute + 32, smem, st>>>(tm_x, p);
+    k_cube_encode<<<grid, kQCompute + 32, smem, st>>>(tm_x, tm_m, p);
     return cudaGetLastError();
 }
 
