@@ -218,7 +218,7 @@ def main():
     ap.add_argument("--cube", default=None, help="override the cube, e.g. 2,2,2")
     ap.add_argument("--frames", type=int, default=None, help="override T (smaller cases for profiling)")
     ap.add_argument("--sample-tokens", type=int, default=256, help="oracle sample size per reference step (tokens)")
-    ap.add_argument("--baseline-tokens", type=int, default=2048, help="oracle sample size of the cpu_baseline leg")
+    ap.add_argument("--baseline-tokens", type=int, default=4096, help="oracle sample size of the cpu_baseline leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     args = ap.parse_args()
