@@ -149,6 +149,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 prefetch_tmap(&tm_fb);
             }
             const uint32_t full0 = mapa_shared(smem_u32(full), 0);
+            // the weight-side operands are read by every row tile: keep them in L2
+            const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
             long long g = 0;
             bool alive = true;
             for (int tile = pair; alive && tile < num_tiles; tile += npairs) {
@@ -166,8 +168,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* sb = sm + L.b + s * kBBytes;
                     if (!kMain) {
                         if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes));
-                        tma_load_2d_pair(sa, &tm_a, fb, i * 64, m0);
-                        tma_load_2d_pair(sb, &tm_b, fb, i * 64, nb);
+                        tma_load_2d_pair_hint(sa, &tm_a, fb, i * 64, m0, stream);
+                        tma_load_2d_pair_hint(sb, &tm_b, fb, i * 64, nb, keep);
                     } else if (i < nk) {
                         if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes + kSFABytes + kSFBBytes));
                         tma_load_2d_pair(sa, &tm_a, fb, i * 128, m0);
@@ -372,8 +374,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 o0[e] = __float_as_uint(__uint_as_float(r0[v + e]) * scale);
                                 o1[e] = __float_as_uint(__uint_as_float(r1[v + e]) * scale);
                             }
-                            st_global_v8(dst + c + v, o0);
-                            st_global_v8(dst + c + 16 + v, o1);
+                            st_global_cs_v8(dst + c + v, o0);
+                            st_global_cs_v8(dst + c + 16 + v, o1);
                         }
                     }
                 }
