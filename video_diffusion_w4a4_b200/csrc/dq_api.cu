@@ -243,6 +243,7 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
         qp.bw = qp.nw * w;
         qp.n_boxes = g.KT * g.KH * qp.nbw;
         qp.m_rows = qp.nw;
+        qp.stat_pairs = t * h * w >= 16;   // then at most 8 cubes per box, one per compute warp
     } else {
         // boxes are segments of up to 128 tokens of one (t, h) row inside one cube
         qp.nw = 1;

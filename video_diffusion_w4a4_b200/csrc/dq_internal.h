@@ -18,6 +18,7 @@ struct QuantParams {
     int nbw;            // boxes along w
     int n_boxes;
     int m_rows;         // kernel tokens per box (rows of the encode kernel's per-stage tile)
+    int stat_pairs;     // statistics kernel: one warp per cube, a channel pair per lane (cubes of 16+ tokens)
     int big;            // cubes of more than 128 tokens: boxes are row segments of one cube,
     int nseg;           //   nseg segments of up to 128 tokens per cube row; the kernel tokens
     float* means;       //   K x Ci fp32 kernel tokens: written by k_cube_stats (by k_cube_means_big for big cubes)
@@ -52,7 +53,7 @@ struct GemmParams {
     uint64_t budget_ns;
 };
 
-size_t quant_smem_bytes(int rank, bool stats, int m_rows);
+size_t quant_smem_bytes(int rank, bool stats, int m_rows, int x_rows);
 cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
                               cudaStream_t st);
 cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const CUtensorMap& tm_m, const QuantParams& p,

@@ -72,6 +72,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep up to `suspend_ns` for the phase
+// to complete (it wakes as soon as it does), instead of returning at once and
+// spending issue slots on polling.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t suspend_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(suspend_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for phase `parity` of `bar`.  Returns false on timeout or, when
 // check_abort is set, as soon as another role of the CTA has given up (abort
 // flag raised).  Drain waits at teardown pass check_abort = false so that
@@ -82,7 +97,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(b, parity)) return true;
     uint64_t t0 = globaltimer();
     while (true) {
-        if (mbar_try_wait(b, parity)) return true;
+        if (mbar_try_wait_sleep(b, parity, 20000u)) return true;
         if (check_abort && *abort_flag) return false;
         if (globaltimer() - t0 > budget_ns) {
             *abort_flag = 1;

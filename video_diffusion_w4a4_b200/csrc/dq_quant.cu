@@ -39,15 +39,17 @@ constexpr int kQCompute = 32 * kQWarps;
 
 struct QSmem {
     // offsets in bytes from the 1024-aligned dynamic smem base
-    uint32_t x, l1, mt, mt_stride, eff, bars, misc, total;
+    uint32_t x, x_stride, l1, mt, mt_stride, eff, bars, misc, total;
 };
 
 // m_rows: rows of the per-stage tile of kernel tokens (encode kernel; 0 for the statistics kernel)
-__host__ __device__ inline QSmem q_smem_layout(int rank, bool with_l1, int m_rows) {
+// x_rows: tokens per TMA box (rows of the X stages; 128 at most)
+__host__ __device__ inline QSmem q_smem_layout(int rank, bool with_l1, int m_rows, int x_rows = 128) {
     QSmem L;
     uint32_t off = 0;
     L.x = off;
-    off += kQStages * 16384;
+    L.x_stride = (uint32_t)align_up((size_t)x_rows * 128, 1024);
+    off += kQStages * L.x_stride;
     L.l1 = off;
     if (with_l1) off += kQStages * (uint32_t)align_up((size_t)rank * 128, 1024);
     L.mt = off;
@@ -61,12 +63,6 @@ __host__ __device__ inline QSmem q_smem_layout(int rank, bool with_l1, int m_row
     off += 64;
     L.total = off;
     return L;
-}
-
-__device__ __forceinline__ float ld_x_swz(const uint8_t* xs, int row, int c) {
-    uint32_t off = (uint32_t)row * 128u + ((((uint32_t)c >> 3) ^ ((uint32_t)row & 7u)) << 4) + (((uint32_t)c & 7u) << 1);
-    uint16_t v = *reinterpret_cast<const uint16_t*>(xs + off);
-    return __uint_as_float((uint32_t)v << 16);
 }
 
 // 8 channels [8q, 8q+8) of a row as one 16-byte vector.
@@ -326,6 +322,7 @@ __device__ __forceinline__ float warp_max(float v) {
 // tensor-memory accumulators per item, which the compute warps drain to the
 // item's partial sums after its last chunk.
 
+template <bool kPairs>
 __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_constant__ CUtensorMap tm_x,
                                                                   const __grid_constant__ CUtensorMap tm_l1,
                                                                   QuantParams p) {
@@ -456,9 +453,46 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                 if (!ok) break;
                 const uint8_t* xs = sm + L.x + s * 16384;
                 const int c0 = c_base + i * 64;
+                if (kPairs) {
+                    // cubes of 16 or more tokens (at most 8 per box): warp = cube slot, lane = channel
+                    // pair (2 lane, 2 lane + 1), so that every cube of the box keeps a warp busy
+                    if (warp < R.nv) {
+                        const int u = warp;
+                        const int sw = (u == R.nv - 1) ? R.sw_last : p.g.w;
+                        uint64_t acc = 0ull;                          // (+0, +0)
+                        uint32_t hi = 0xFF80FF80u, lo = 0x7F807F80u;  // BF16 -inf / +inf pairs
+                        for (int dt = 0; dt < R.st; dt++)
+                            for (int dh = 0; dh < R.sh; dh++) {
+                                const int row0 = (dt * p.bh + dh) * p.bw + u * p.g.w;
+                                for (int dw = 0; dw < sw; dw++) {
+                                    const uint32_t row = (uint32_t)(row0 + dw);
+                                    const uint32_t v = *reinterpret_cast<const uint32_t*>(
+                                        xs + row * 128u + ((((uint32_t)lane >> 2) ^ (row & 7u)) << 4) + ((uint32_t)lane & 3u) * 4u);
+                                    acc = f2_add(acc, f2_from_bf16x2(v));
+                                    hi = bf16x2_max(hi, v);
+                                    lo = bf16x2_min(lo, v);
+                                }
+                            }
+                        const int cnt = R.st * R.sh * sw;
+                        float a0, a1, m0, m1;
+                        f2_unpack(acc, a0, a1);
+                        if ((cnt & (cnt - 1)) == 0) {
+                            const float inv = __frcp_rn((float)cnt);
+                            m0 = __fmul_rn(a0, inv);
+                            m1 = __fmul_rn(a1, inv);
+                        } else {
+                            m0 = __fdiv_rn(a0, (float)cnt);
+                            m1 = __fdiv_rn(a1, (float)cnt);
+                        }
+                        *reinterpret_cast<float2*>(p.means + (size_t)(R.k0 + u) * p.Ci + c0 + 2 * lane) = make_float2(m0, m1);
+                        kam[0] = fmaxf(kam[0], fmaxf(fabsf(m0), fabsf(m1)));
+                        damax = fmaxf(damax, fmaxf(fmaxf(fabsf(__fsub_rn(bf16_lo(hi), m0)), fabsf(__fsub_rn(bf16_hi(hi), m1))),
+                                                   fmaxf(fabsf(__fsub_rn(bf16_lo(lo), m0)), fabsf(__fsub_rn(bf16_hi(lo), m1)))));
+                    }
+                }
 #pragma unroll
                 for (int t = 0; t < 4; t++) {
-                    if (t >= ntask) break;
+                    if (kPairs || t >= ntask) break;
                     const StatTask T = t == 0 ? T0 : stat_task(p, R, tid + kQCompute * t);
                     if (!T.valid) continue;
                     uint64_t m[4];
@@ -532,8 +566,12 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
             }
             if (!ok) break;
             // per-cube max |mean| over this item's channels -> kamax (small cubes; the means
-            // kernel has done it for big ones); the eight threads of a cube are consecutive lanes
-            if (!p.big) {
+            // kernel has done it for big ones); the eight threads of a cube are consecutive lanes,
+            // or a whole warp in the channel-pair mode
+            if (kPairs) {
+                const float v = warp_max(kam[0]);
+                if (lane == 0 && warp < R.nv) atomicMax(&p.kamax[R.k0 + warp], __float_as_uint(v));
+            } else if (!p.big) {
 #pragma unroll
                 for (int t = 0; t < 4; t++) {
                     if (t >= ntask) break;
@@ -599,7 +637,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                                                                   QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const QSmem L = q_smem_layout(p.rank, false, p.m_rows);
+    const QSmem L = q_smem_layout(p.rank, false, p.m_rows, p.bt * p.bh * p.bw);
     uint64_t* full = (uint64_t*)(sm + L.bars);
     uint64_t* empty = full + kQStages;
     volatile int* abort_flag = (volatile int*)(sm + L.misc + 8);
@@ -656,7 +694,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                         break;
                     }
                     mbar_arrive_expect_tx(&full[s], x_bytes + m_bytes);
-                    tma_load_4d(sm + L.x + s * 16384, &tm_x, &full[s], c_base + i * 64, B.w0, B.h0, B.t0);
+                    tma_load_4d(sm + L.x + s * L.x_stride, &tm_x, &full[s], c_base + i * 64, B.w0, B.h0, B.t0);
                     tma_load_2d(sm + L.mt + s * L.mt_stride, &tm_m, &full[s], c_base + i * 64, k0);
                 }
             }
@@ -702,7 +740,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                 ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)(g / kQStages) & 1, abort_flag, p.status,
                                                        p.budget_ns));
                 if (!ok) break;
-                const uint8_t* xs = sm + L.x + s * 16384;
+                const uint8_t* xs = sm + L.x + s * L.x_stride;
                 const float* mt = (const float*)(sm + L.mt + s * L.mt_stride);
                 const int c0 = c_base + i * 64;
                 // kernel tokens: FP8 E4M3 codes under s8 = max|mean| / 448, and their exact BF16 copy
@@ -828,20 +866,31 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
 // ------------------------------------------------------------------ kernel tokens of big cubes
 //
 // Cubes of more than 128 tokens (up to one global cube over the whole lattice).
-// CTA = 64 channels of one cube: warp 2 streams the cube's rows through an
-// 8-stage TMA ring (the same row-segment boxes as the quantise kernels) and
-// threads 0-63 each keep one channel's fp32 running sum over the tokens in
-// (t,h,w) order (Eq. 1, the same arithmetic as cube_mean8), then divide by the
-// count; the per-cube max |mean| goes to kamax.
+// CTA = 64 channels of one cube: warp 1 streams the cube's rows through a TMA
+// ring of row-segment boxes (the same boxes as the quantise kernels; stages
+// sized to the box so that about 110 KB are in flight), and each lane of
+// warp 0 keeps the fp32 running sums of two channels (a packed pair) over the
+// tokens in (t,h,w) order (Eq. 1, the same arithmetic as the statistics
+// kernel), then divides by the count; the per-cube max |mean| goes to kamax.
+// The sums are dependent chains of one add per token, so the rows of a box
+// are visited in groups of eight whose swizzled offsets are fixed.
 
-constexpr int kMStages = 8;
+constexpr int kMStagesMax = 32;
 
-__global__ void __launch_bounds__(96) k_cube_means_big(const __grid_constant__ CUtensorMap tm_x, QuantParams p) {
+__host__ __device__ inline uint32_t means_stage_bytes(int bw) { return (uint32_t)align_up((size_t)bw * 128, 1024); }
+__host__ __device__ inline int means_stages(int bw) {
+    const int n = (int)(110u * 1024u / means_stage_bytes(bw));
+    return n < 2 ? 2 : (n > kMStagesMax ? kMStagesMax : n);
+}
+
+__global__ void __launch_bounds__(64) k_cube_means_big(const __grid_constant__ CUtensorMap tm_x, QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint64_t* full = (uint64_t*)(sm + kMStages * 16384);
-    uint64_t* empty = full + kMStages;
-    volatile int* abort_flag = (volatile int*)(empty + kMStages);
+    const uint32_t stage_bytes = means_stage_bytes(p.bw);
+    const int S = means_stages(p.bw);
+    uint64_t* full = (uint64_t*)(sm + (size_t)S * stage_bytes);
+    uint64_t* empty = full + kMStagesMax;
+    volatile int* abort_flag = (volatile int*)(empty + kMStagesMax);
     const Geom& g = p.g;
     const long long k = blockIdx.x;
     const int c0 = blockIdx.y * 64;
@@ -849,51 +898,76 @@ __global__ void __launch_bounds__(96) k_cube_means_big(const __grid_constant__ C
     const int st = imin(g.t, g.T - kt * g.t), sh = imin(g.h, g.H - kh * g.h), sw = imin(g.w, g.W - kw * g.w);
     const int nbox = st * sh * p.nseg;
     const uint32_t box_bytes = (uint32_t)p.bw * 128u;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     if (tid == 0) {
-        for (int s = 0; s < kMStages; s++) {
+        for (int s = 0; s < S; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 64);
+            mbar_init(&empty[s], 1);
         }
         *abort_flag = 0;
         fence_barrier_init();
     }
     __syncthreads();
-    if (tid >= 64) {
-        if (tid == 64) {
+    if (tid >= 32) {
+        if (tid == 32) {
             int issued = 0;
             prefetch_tmap(&tm_x);
             for (int b = 0; b < nbox; b++) {
-                const int s = b % kMStages;
-                if (b >= kMStages && !mbar_wait(&empty[s], ((b / kMStages) - 1) & 1, abort_flag, p.status, p.budget_ns))
-                    break;
+                const int s = b % S;
+                if (b >= S && !mbar_wait(&empty[s], ((b / S) - 1) & 1, abort_flag, p.status, p.budget_ns)) break;
                 const int seg = b % p.nseg, dh = (b / p.nseg) % sh, dt = b / (p.nseg * sh);
                 mbar_arrive_expect_tx(&full[s], box_bytes);
-                tma_load_4d(sm + s * 16384, &tm_x, &full[s], c0, kw * g.w + 128 * seg, kh * g.h + dh, kt * g.t + dt);
+                tma_load_4d(sm + (size_t)s * stage_bytes, &tm_x, &full[s], c0, kw * g.w + 128 * seg, kh * g.h + dh,
+                            kt * g.t + dt);
                 issued = b + 1;
             }
-            for (int b = (issued > kMStages ? issued - kMStages : 0); b < issued; b++)
-                mbar_wait(&full[b % kMStages], (b / kMStages) & 1, abort_flag, nullptr, p.budget_ns, false);
+            for (int b = (issued > S ? issued - S : 0); b < issued; b++)
+                mbar_wait(&full[b % S], (b / S) & 1, abort_flag, nullptr, p.budget_ns, false);
         }
     } else {
-        float acc = 0.f;
+        // lane l: channels 2l, 2l+1 = bytes 4 (l % 4) of 16-byte chunk l / 4 of each 128-byte row
+        uint32_t o[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) o[i] = (uint32_t)i * 128u + ((((uint32_t)lane >> 2) ^ (uint32_t)i) << 4) + ((uint32_t)lane & 3u) * 4u;
+        uint64_t acc = 0ull;   // (+0, +0)
         bool ok = true;
         for (int b = 0; b < nbox; b++) {
-            const int s = b % kMStages;
-            ok = ok && mbar_wait(&full[s], (b / kMStages) & 1, abort_flag, p.status, p.budget_ns);
+            const int s = b % S;
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(&full[s], (b / S) & 1, abort_flag, p.status, p.budget_ns));
             if (ok) {
                 const int seg = b % p.nseg;
                 const int rows = imin(p.bw, sw - 128 * seg);
-                const uint8_t* xs = sm + s * 16384;
-                for (int r = 0; r < rows; r++) acc = __fadd_rn(acc, ld_x_swz(xs, r, tid));
+                const uint8_t* xs = sm + (size_t)s * stage_bytes;
+                int r = 0;
+                for (; r + 8 <= rows; r += 8) {
+                    const uint8_t* x8 = xs + r * 128;
+#pragma unroll
+                    for (int i = 0; i < 8; i++) acc = f2_add(acc, f2_from_bf16x2(*reinterpret_cast<const uint32_t*>(x8 + o[i])));
+                }
+                for (; r < rows; r++) {
+                    const uint32_t off = (uint32_t)r * 128u + ((((uint32_t)lane >> 2) ^ ((uint32_t)r & 7u)) << 4) +
+                                         ((uint32_t)lane & 3u) * 4u;
+                    acc = f2_add(acc, f2_from_bf16x2(*reinterpret_cast<const uint32_t*>(xs + off)));
+                }
             }
-            mbar_arrive(&empty[s]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
         }
         const int cnt = st * sh * sw;
-        const float m = ((cnt & (cnt - 1)) == 0) ? __fmul_rn(acc, __frcp_rn((float)cnt)) : __fdiv_rn(acc, (float)cnt);
-        p.means[k * p.Ci + c0 + tid] = m;
-        const float am = warp_max(fabsf(m));
-        if ((tid & 31) == 0) atomicMax(&p.kamax[k], __float_as_uint(am));
+        float a0, a1;
+        f2_unpack(acc, a0, a1);
+        float m0, m1;
+        if ((cnt & (cnt - 1)) == 0) {
+            const float inv = __frcp_rn((float)cnt);
+            m0 = __fmul_rn(a0, inv);
+            m1 = __fmul_rn(a1, inv);
+        } else {
+            m0 = __fdiv_rn(a0, (float)cnt);
+            m1 = __fdiv_rn(a1, (float)cnt);
+        }
+        *reinterpret_cast<float2*>(p.means + k * p.Ci + c0 + 2 * lane) = make_float2(m0, m1);
+        const float am = warp_max(fmaxf(fabsf(m0), fabsf(m1)));
+        if (lane == 0) atomicMax(&p.kamax[k], __float_as_uint(am));
     }
     __syncthreads();
 }
@@ -901,16 +975,16 @@ __global__ void __launch_bounds__(96) k_cube_means_big(const __grid_constant__ C
 // ------------------------------------------------------------------ launchers
 
 cudaError_t launch_cube_means_big(const CUtensorMap& tm_x, const QuantParams& p, cudaStream_t st) {
-    const size_t smem = kMStages * 16384 + 2 * kMStages * 8 + 16 + 1024;
+    const size_t smem = (size_t)means_stages(p.bw) * means_stage_bytes(p.bw) + 2 * kMStagesMax * 8 + 16 + 1024;
     cudaError_t e = cudaFuncSetAttribute(k_cube_means_big, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)p.g.K, (unsigned)(p.Ci / 64));
-    k_cube_means_big<<<grid, 96, smem, st>>>(tm_x, p);
+    k_cube_means_big<<<grid, 64, smem, st>>>(tm_x, p);
     return cudaGetLastError();
 }
 
-size_t quant_smem_bytes(int rank, bool stats, int m_rows) {
-    return q_smem_layout(rank, stats, m_rows).total + 1024;
+size_t quant_smem_bytes(int rank, bool stats, int m_rows, int x_rows) {
+    return q_smem_layout(rank, stats, m_rows, x_rows).total + 1024;
 }
 
 namespace {
@@ -938,22 +1012,27 @@ int resident_grid(const void* fn, int threads, size_t smem, int items) {
 }
 }  // namespace
 
-cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
-                              cudaStream_t st) {
-    size_t smem = quant_smem_bytes(p.rank, true, 0);
-    cudaError_t e = cudaFuncSetAttribute(k_cube_stats, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <bool kPairs>
+cudaError_t launch_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p, cudaStream_t st) {
+    size_t smem = quant_smem_bytes(p.rank, true, 0, 128);
+    cudaError_t e = cudaFuncSetAttribute(k_cube_stats<kPairs>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_cube_stats, cudaFuncAttributePreferredSharedMemoryCarveout,
+        e = cudaFuncSetAttribute(k_cube_stats<kPairs>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    const int grid = resident_grid((const void*)k_cube_stats, kQCompute + 64, smem, p.n_boxes * p.splits);
-    k_cube_stats<<<grid, kQCompute + 64, smem, st>>>(tm_x, tm_l1, p);
+    const int grid = resident_grid((const void*)k_cube_stats<kPairs>, kQCompute + 64, smem, p.n_boxes * p.splits);
+    k_cube_stats<kPairs><<<grid, kQCompute + 64, smem, st>>>(tm_x, tm_l1, p);
     return cudaGetLastError();
+}
+
+cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
+                              cudaStream_t st) {
+    return p.stat_pairs ? launch_stats<true>(tm_x, tm_l1, p, st) : launch_stats<false>(tm_x, tm_l1, p, st);
 }
 
 cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const CUtensorMap& tm_m, const QuantParams& p,
                                cudaStream_t st) {
-    size_t smem = quant_smem_bytes(p.rank, false, p.m_rows);
+    size_t smem = quant_smem_bytes(p.rank, false, p.m_rows, p.bt * p.bh * p.bw);
     cudaError_t e = cudaFuncSetAttribute(k_cube_encode, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_cube_encode, cudaFuncAttributePreferredSharedMemoryCarveout,
