@@ -66,7 +66,7 @@ def test_full_size(env, name):
     _record(name, info)
 
 
-@pytest.mark.parametrize("cube", [(1, 1, 1), (1, 2, 2), (2, 2, 2), (2, 4, 4), (21, 30, 52)])
+@pytest.mark.parametrize("cube", [(1, 1, 1), (1, 2, 2), (2, 2, 2), (2, 4, 4), (4, 1, 4), (4, 2, 8), (21, 30, 52)])
 def test_cube_sweep(env, cube):
     dq, torch = env
     wl = synth.WORKLOADS["wan480p_cube_sweep"].with_cube(cube)

@@ -69,6 +69,9 @@ SMALL = [
     ("cube_244", _wl("cube_244", 4, 9, 18, 512, 256, 48, (2, 4, 4))),
     ("cube_418", _wl("cube_418", 6, 5, 20, 256, 256, 16, (4, 1, 8))),
     ("gelu_122", _wl("gelu_122", 2, 12, 40, 1024, 512, 64, (1, 2, 2), gelu=True)),
+    # the note's own operating point: 64-token cubes 4x1x4 and 4x2x8, low-rank branch of rank 128
+    ("cube_414_r128", _wl("cube_414_r128", 9, 6, 22, 512, 256, 128, (4, 1, 4))),
+    ("cube_428", _wl("cube_428", 8, 7, 27, 256, 512, 32, (4, 2, 8))),
     # cubes of more than 128 tokens: kernel tokens from the means kernel, boxes are row segments
     ("global", _wl("global", 3, 10, 37, 512, 256, 16, (3, 10, 37))),
     ("big_cube", _wl("big_cube", 5, 18, 21, 256, 256, 16, (2, 8, 16))),
