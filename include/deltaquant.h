@@ -42,7 +42,7 @@ extern "C" {
 #endif
 
 #define DQ_ABI_VERSION 1
-#define DQ_PACK_FORMAT_VERSION 1
+#define DQ_PACK_FORMAT_VERSION 2
 #define DQ_PACK_MAGIC 0x31575144u /* "DQW1" little-endian */
 
 typedef enum dq_status {
@@ -119,6 +119,26 @@ int dq_sf_bytes(long long rows, int cols, size_t* bytes);
 int dq_sfa_offset(long long row, int block, int cols, size_t* offset);
 int dq_sfa_bytes(long long rows, int cols, size_t* bytes);
 
+/*
+ * B-operand scale layout (the weight group scales of the packed weight; rows
+ * a multiple of 256).  Every 32-lane quadrant of the tensor memory needs the
+ * scales of all 256 columns of an output tile, in lane i the scales of rows
+ * 32 c + i and 128 + 32 c + i (c = 0..3) of the tile in its eight 32-bit
+ * columns.  Stored so that one 128x256-bit copy per 64-column block writes
+ * that (instead of two replicating 32x128-bit copies): per 256-row tile and
+ * 64-column block one 4096-byte block of 128 lanes x 32 bytes in 8-row x
+ * 16-byte core matrices (row-group stride 256, column-half stride 128), lanes
+ * i, i + 32, i + 64 and i + 96 holding the same bytes.  dq_sfb_offset gives
+ * the byte in lane row % 32; the copies in the other three lanes sit 1024,
+ * 2048 and 3072 bytes further:
+ *   n = row % 256, w = 4 (n / 128) + (n % 128) / 32, b = 4 w + block % 4,
+ *   offset = ((row/256) * (cols/64) + block/4) * 4096
+ *            + ((n%32)/8) * 256 + (b/16) * 128 + (n % 8) * 16 + b % 16.
+ * Total size: ceil(rows/256) * (cols/64) * 4096.
+ */
+int dq_sfb_offset(long long row, int block, int cols, size_t* offset);
+int dq_sfb_bytes(long long rows, int cols, size_t* bytes);
+
 /* ------------------------------------------------------------------------ */
 /* Offline weight packing (host only, synchronous)                           */
 /* ------------------------------------------------------------------------ */
@@ -130,7 +150,7 @@ int dq_sfa_bytes(long long rows, int cols, size_t* bytes);
  *           slab, float S_W, then uint64 byte offsets of the sections below.
  *   codes   Co x Ci/2 bytes, E2M1 codes of R, row o = output channel,
  *           channel 2i in the low nibble of byte i.
- *   scales  E4M3 group-16 scales of R in the scale-factor layout above.
+ *   scales  E4M3 group-16 scales of R in the B-operand scale layout above.
  *   dqw     Co x Ci BF16 values q * s_b of R (exact: at most 6 significant
  *           bits), the operand of the kernel-token product.
  * S_W is R's per-tensor scale.  dq_packed_weight_bytes gives the size.

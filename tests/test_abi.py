@@ -89,6 +89,31 @@ def test_sfa_offset_places_each_scale_in_its_quadrant_column(dq):
         dq.dq_sfa_offset(0, 0, 192)
 
 
+def test_sfb_offset_replicates_each_column_scale_into_every_quadrant(dq):
+    """B-operand scale layout: the four per-quadrant copies of all scales cover every byte exactly once;
+    the copy in lane r of the 4 KB block holds (row, block) with r % 32 == row % 32, in 32-bit word
+    4 (n / 128) + (n % 128) / 32 (n = row % 256), byte block % 4 of that word."""
+    for rows, cols in ((256, 64), (512, 256)):
+        total = dq.dq_sfb_bytes(rows, cols)
+        assert total == (rows // 256) * (cols // 64) * 4096
+        seen = np.zeros(total, bool)
+        for r in range(rows):
+            for b in range(cols // 16):
+                off0 = dq.dq_sfb_offset(r, b, cols)
+                for q in range(4):
+                    off = off0 + 1024 * q
+                    assert not seen[off]
+                    seen[off] = True
+                    block, inner = divmod(off, 4096)
+                    assert block == (r // 256) * (cols // 64) + b // 4
+                    lane = (inner // 256) * 8 + (inner % 128) // 16
+                    byte = ((inner % 256) // 128) * 16 + inner % 16
+                    n = r % 256
+                    assert lane == 32 * q + r % 32
+                    assert byte // 4 == 4 * (n // 128) + (n % 128) // 32 and byte % 4 == b % 4
+        assert seen.all()
+
+
 def test_layouts_are_aligned_and_ordered(dq):
     L = dq.dq_workspace_layout_get(21, 30, 52, 1, 2, 2, 5120, 5120, 32)
     offs = [L.off_status, L.off_scalars, L.off_kamax, L.off_s8, L.off_q8, L.off_q8_bf16, L.off_dcodes,

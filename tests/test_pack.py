@@ -21,8 +21,12 @@ def dq():
 
 
 def _unpack_scales(dq, blob, off, rows, cols):
-    idx = np.array([[dq.dq_sf_offset(r, b, cols) for b in range(cols // 16)] for r in range(rows)])
-    return blob[off + idx]
+    """Weight scales from the B-operand scale layout; the four per-quadrant copies must agree."""
+    idx = np.array([[dq.dq_sfb_offset(r, b, cols) for b in range(cols // 16)] for r in range(rows)])
+    copies = [blob[off + idx + 1024 * q] for q in range(4)]
+    for c in copies[1:]:
+        assert np.array_equal(c, copies[0])
+    return copies[0]
 
 
 @pytest.mark.parametrize("shape", [(256, 256, 16), (512, 1024, 32), (1024, 512, 48)])
@@ -35,7 +39,7 @@ def test_pack_bit_exact(dq, shape):
     packed, L1m, L2s, S_W = dq.dq_pack_weight_factors(Wb, L1, L2)
     lay = dq.dq_packed_weight_layout(Co, Ci, r)
     hdr = packed[:256].view(np.uint32)
-    assert hdr[0] == 0x31575144 and hdr[1] == 1
+    assert hdr[0] == 0x31575144 and hdr[1] == 2
     assert list(packed[8:24].view(np.int32)) == [Co, Ci, r, lay.slab]
     assert packed[24:28].view(np.float32)[0] == np.float32(wq["S_w"]) == np.float32(S_W)
     codes = packed[lay.off_codes:lay.off_codes + Co * Ci // 2].reshape(Co, Ci // 2)

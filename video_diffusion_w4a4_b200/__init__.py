@@ -60,6 +60,8 @@ _SIGS = {
     "dq_sf_offset": ([_LL, _I, _I, ctypes.POINTER(_SZ)], _I),
     "dq_sf_bytes": ([_LL, _I, ctypes.POINTER(_SZ)], _I),
     "dq_sfa_offset": ([_LL, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "dq_sfb_offset": ([_LL, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "dq_sfb_bytes": ([_LL, _I, ctypes.POINTER(_SZ)], _I),
     "dq_sfa_bytes": ([_LL, _I, ctypes.POINTER(_SZ)], _I),
     "dq_packed_weight_layout": ([_I, _I, _I, ctypes.POINTER(dq_packed_layout)], _I),
     "dq_packed_weight_bytes": ([_I, _I, _I, ctypes.POINTER(_SZ)], _I),
@@ -147,6 +149,18 @@ def dq_sfa_offset(row: int, block: int, cols: int) -> int:
     off = _SZ()
     _check("dq_sfa_offset", _lib.dq_sfa_offset(row, block, cols, ctypes.byref(off)))
     return off.value
+
+
+def dq_sfb_offset(row: int, block: int, cols: int) -> int:
+    off = _SZ()
+    _check("dq_sfb_offset", _lib.dq_sfb_offset(row, block, cols, ctypes.byref(off)))
+    return off.value
+
+
+def dq_sfb_bytes(rows: int, cols: int) -> int:
+    b = _SZ()
+    _check("dq_sfb_bytes", _lib.dq_sfb_bytes(rows, cols, ctypes.byref(b)))
+    return b.value
 
 
 def dq_sfa_bytes(rows: int, cols: int) -> int:

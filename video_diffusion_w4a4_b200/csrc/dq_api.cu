@@ -65,22 +65,6 @@ bool map_x(CUtensorMap* m, const void* X, const Geom& g, int Ci, int bw, int bh,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D map over a block-scale-factor array (layout in include/deltaquant.h) viewed
-// as 256-byte lines: dim 0 the bytes of a line, dim 1 the Ci/32 lines of one
-// 128-row group (4 k-blocks of 64 channels = 2048 bytes = 8 lines per K step of
-// 256 channels), dim 2 the row groups.  Boxes of 8 lines x `groups` row groups.
-bool map_sf(CUtensorMap* m, const void* base, int Ci, uint64_t row_groups, uint32_t groups) {
-    EncodeTiledFn f = encode_fn();
-    if (!f) return false;
-    cuuint64_t dims[3] = {256, (cuuint64_t)Ci / 32, row_groups};
-    cuuint64_t strides[2] = {256, (cuuint64_t)Ci * 8};
-    cuuint32_t box[3] = {256, 8, groups};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // 3-D map over the A-operand scale layout (dq_sfa_offset): dim 0 the bytes of a
 // 256-byte line, dim 1 the 32 (Ci/256) lines of one 128-row group (8192 bytes
 // per K step of 256 channels), dim 2 the row groups.  Boxes of one K step.
@@ -105,6 +89,21 @@ bool map_means(CUtensorMap* m, const void* base, int Ci, long long K, int rows) 
     cuuint32_t box[2] = {64, (cuuint32_t)rows};
     cuuint32_t estr[2] = {1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over the B-operand scale layout (dq_sfb_offset): dim 0 the bytes of a
+// 256-byte line, dim 1 the 16 (Ci/64) lines of one 256-row tile (16384 bytes
+// per K step of 256 channels), dim 2 the 256-row tiles.  Boxes of one K step.
+bool map_sfb(CUtensorMap* m, const void* base, int Ci, int Co) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {256, (cuuint64_t)Ci / 64 * 16, (cuuint64_t)Co / 256};
+    cuuint64_t strides[2] = {256, (cuuint64_t)Ci / 64 * 4096};
+    cuuint32_t box[3] = {256, 64, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -321,7 +320,7 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
             return map_fail("slab A");
         if (!map_2d(&tm_sb, L2_slab, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, wl.slab, Co, 64, 128)) return map_fail("slab B");
         if (!map_sfa(&tm_fa, ws + wl.off_dscales, Ci, (uint64_t)dq::cdiv(g.N, 128))) return map_fail("delta scales");
-        if (!map_sf(&tm_fb, pw + pl.off_scales, Ci, (uint64_t)(Co / 128), 2)) return map_fail("weight scales");
+        if (!map_sfb(&tm_fb, pw + pl.off_scales, Ci, Co)) return map_fail("weight scales");
         dq::GemmParams p = gp;
         p.M = (int)g.N;
         p.k_stages = Ci / 256;

@@ -102,6 +102,22 @@ DQ_HD size_t sfa_offset(long long row, int blk, int cols) {
 
 DQ_HD size_t sfa_bytes(long long rows, int cols) { return (size_t)cdiv(rows, 128) * (size_t)(cols / 256) * 8192; }
 
+// B-operand scale layout (the weight scales of the packed weight; see
+// include/deltaquant.h): per 256-row tile and 64-column block one 4 KB block
+// of 128 lanes x 32 bytes in 8-row x 16-byte core matrices, lane r holding the
+// scales of rows 32 c + r % 32 (c = 0..3) and 128 + 32 c + r % 32 in its eight
+// 32-bit words; lanes r, r + 32, r + 64, r + 96 hold the same bytes.  Returns
+// the offset of the copy in lane r % 32; the copy in lane r % 32 + 32 q sits
+// 1024 q bytes further.
+DQ_HD size_t sfb_offset(long long row, int blk, int cols) {
+    const int nl = (int)(row & 255), kb = blk >> 2;
+    const int i = nl & 31, word = 4 * (nl >> 7) + ((nl >> 5) & 3), b = 4 * word + (blk & 3);
+    const long long block = (row >> 8) * (long long)(cols >> 6) + kb;
+    return (size_t)block * 4096 + (size_t)((i >> 3) * 256 + (b >> 4) * 128 + (i & 7) * 16 + (b & 15));
+}
+
+DQ_HD size_t sfb_bytes(long long rows, int cols) { return (size_t)cdiv(rows, 256) * (size_t)(cols / 64) * 4096; }
+
 DQ_HD int slab_width(int rank) { return (int)(cdiv(2 * rank, 64) * 64); }
 
 // Packed weight blob header (first 256 bytes of the blob).
@@ -125,7 +141,7 @@ DQ_HD PackedLayout packed_layout(int Co, int Ci, int rank) {
     L.off_codes = off;
     off = align_up(off + (size_t)Co * (Ci / 2), kAlign);
     L.off_scales = off;
-    off = align_up(off + sf_bytes(Co, Ci), kAlign);
+    off = align_up(off + sfb_bytes(Co, Ci), kAlign);
     L.off_dqw = off;
     off = align_up(off + (size_t)Co * Ci * 2, kAlign);
     L.total = off;

@@ -52,10 +52,10 @@ constexpr int kThreads = 96 + 32 * kEpiWarps;   // producer, MMA, scale-factor c
 constexpr uint32_t kABytes = kTileM * 128;      // 128 rows x 128 bytes
 constexpr uint32_t kBBytes = (kTileN / 2) * 128;  // this CTA's 128 rows of B x 128 bytes
 constexpr uint32_t kSFABytes = 2 * 4096;        // 128 rows x 4 k-blocks of 64, A-operand scale layout
-constexpr uint32_t kSFBBytes = 2 * 4 * 512;     // all 256 columns x 4 k-blocks (each CTA holds a copy)
+constexpr uint32_t kSFBBytes = 4 * 4096;        // all 256 columns x 4 k-blocks, B-operand scale layout (each CTA)
 constexpr uint16_t kPairMask = 0x3;
 
-__host__ __device__ constexpr int g_stages(bool scaled) { return scaled ? 5 : 6; }
+__host__ __device__ constexpr int g_stages(bool scaled) { return scaled ? 4 : 6; }
 
 struct GSmem {
     uint32_t a, b, sfa, sfb, bars, misc, total;
@@ -81,7 +81,6 @@ __host__ __device__ constexpr GSmem g_smem_layout(bool scaled) {
     return L;
 }
 
-__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) { return smem_desc(saddr, 0, 128, 0); }
 
 }  // namespace
 
@@ -175,9 +174,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_2d_pair(sa, &tm_a, fb, i * 128, m0);
                         tma_load_2d_pair(sb, &tm_b, fb, i * 128, nb);
                         // scale factors: A 8192 B per 128-row group and K step (32 lines of 256 B),
-                        // B 4 k-blocks x 512 B per 128-row group (8 lines), for both row groups of the pair tile
+                        // B 16384 B per 256-column tile and K step (64 lines)
                         tma_load_3d_pair(sm + L.sfa + s * kSFABytes, &tm_fa, fb, 0, 32 * i, m0 >> 7);
-                        tma_load_3d_pair(sm + L.sfb + s * kSFBBytes, &tm_fb, fb, 0, 8 * i, n0 >> 7);
+                        tma_load_3d_pair(sm + L.sfb + s * kSFBBytes, &tm_fb, fb, 0, 64 * i, n0 >> 8);
                     } else {
                         if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes));
                         tma_load_2d_pair(sa, &tm_sa, fb, (i - nk) * 64, m0);
@@ -270,14 +269,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t fb = smem_u32(sm + L.sfb + s * kSFBBytes);
                         // A: lane r receives 8 columns per copy, of which the MMA of k-block k reads
                         // column 8 (k / 2) + 4 (k % 2) + r / 32; B: every quadrant needs every column's
-                        // scales, so they are replicated into the four 32-lane quadrants
+                        // scales, and the packed weight holds them once per quadrant, so one copy per
+                        // k-block fills all four
                         tmem_cp_pair_128x256b(t_sfa, smem_desc(fa, 128, 256, 0));
                         tmem_cp_pair_128x256b(t_sfa + 8, smem_desc(fa + 4096, 128, 256, 0));
 #pragma unroll
-                        for (int k = 0; k < 4; k++) {
-                            tmem_cp_pair_32x128b_x4(t_sfb + 8 * k, desc_sf(fb + 512 * k));
-                            tmem_cp_pair_32x128b_x4(t_sfb + 8 * k + 4, desc_sf(fb + kSFBBytes / 2 + 512 * k));
-                        }
+                        for (int k = 0; k < 4; k++) tmem_cp_pair_128x256b(t_sfb + 8 * k, smem_desc(fb + 4096 * k, 128, 256, 0));
                     }
                     tc_commit_pair(&sfready[s]);
                     tc_commit_pair_both(&empty[s], kPairMask);

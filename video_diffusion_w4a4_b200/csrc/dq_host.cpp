@@ -317,6 +317,18 @@ int dq_sfa_bytes(long long rows, int cols, size_t* bytes) {
     return DQ_OK;
 }
 
+int dq_sfb_offset(long long row, int block, int cols, size_t* offset) {
+    if (!offset || row < 0 || cols <= 0 || cols % 64 || block < 0 || block >= cols / 16) return DQ_ERR_INVALID_ARG;
+    *offset = dq::sfb_offset(row, block, cols);
+    return DQ_OK;
+}
+
+int dq_sfb_bytes(long long rows, int cols, size_t* bytes) {
+    if (!bytes || rows < 0 || cols <= 0 || cols % 64) return DQ_ERR_INVALID_ARG;
+    *bytes = dq::sfb_bytes(rows, cols);
+    return DQ_OK;
+}
+
 int dq_lowrank_slab_width(int rank) { return (rank > 0) ? dq::slab_width(rank) : 0; }
 
 int dq_packed_weight_layout(int Co, int Ci, int rank, dq_packed_layout* out) {
@@ -442,7 +454,8 @@ int dq_pack_weight_factors(const uint16_t* Wb, const uint16_t* L1, const uint16_
             uint8_t sb = float_to_e4m3(am / denom);
             float sbv = e4m3_to_float(sb);
             float eff = sbv * S;
-            scales[dq::sf_offset(o, b, Ci)] = sb;
+            const size_t so = dq::sfb_offset(o, b, Ci);
+            for (int q = 0; q < 4; q++) scales[so + 1024 * q] = sb;   // one copy per tensor-memory quadrant
             for (int i = 0; i < 16; i += 2) {
                 uint8_t q0 = (eff == 0.0f) ? 0 : float_to_e2m1(z[b * 16 + i] / eff);
                 uint8_t q1 = (eff == 0.0f) ? 0 : float_to_e2m1(z[b * 16 + i + 1] / eff);
