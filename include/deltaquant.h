@@ -41,8 +41,8 @@
 extern "C" {
 #endif
 
-#define DQ_ABI_VERSION 1
-#define DQ_PACK_FORMAT_VERSION 2
+#define DQ_ABI_VERSION 2
+#define DQ_PACK_FORMAT_VERSION 3
 #define DQ_PACK_MAGIC 0x31575144u /* "DQW1" little-endian */
 
 typedef enum dq_status {
@@ -147,17 +147,21 @@ int dq_sfb_bytes(long long rows, int cols, size_t* bytes);
  * Packed weight blob (device copy of what dq_pack_weight writes), all
  * sections 256-byte aligned:
  *   header  256 bytes: uint32 magic, uint32 version, int32 Co, Ci, rank,
- *           slab, float S_W, then uint64 byte offsets of the sections below.
+ *           slab, float S_W, uint32 flags (bit 0: the layer has a bias),
+ *           then uint64 byte offsets of codes, scales, dqw, the total size
+ *           and the offset of the bias section.
  *   codes   Co x Ci/2 bytes, E2M1 codes of R, row o = output channel,
  *           channel 2i in the low nibble of byte i.
  *   scales  E4M3 group-16 scales of R in the B-operand scale layout above.
  *   dqw     Co x Ci BF16 values q * s_b of R (exact: at most 6 significant
  *           bits), the operand of the kernel-token product.
+ *   bias    Co fp32, the layer's bias b (y = x W^T + b) widened exactly from
+ *           BF16 by dq_pack_bias; zeros and flag bit 0 clear when unset.
  * S_W is R's per-tensor scale.  dq_packed_weight_bytes gives the size.
  */
 typedef struct dq_packed_layout {
     size_t total_bytes;
-    size_t off_codes, off_scales, off_dqw;
+    size_t off_codes, off_scales, off_dqw, off_bias;
     int Co, Ci, rank, slab;
 } dq_packed_layout;
 
@@ -192,6 +196,18 @@ int dq_lowrank_factors(const uint16_t* W, int Co, int Ci, int rank, uint64_t see
 int dq_pack_weight_factors(const uint16_t* W, const uint16_t* L1, const uint16_t* L2, int Co, int Ci,
                            int rank, void* packed, size_t packed_bytes, uint16_t* L1_mma,
                            uint16_t* L2_slab, float* S_W);
+
+/*
+ * Set (bias != NULL) or clear (bias == NULL) the bias of a packed blob in
+ * host memory: bias is host, Co BF16 values; Co must equal the blob's Co and
+ * packed_bytes its total size.  The forward pass then returns x W^T + b: the
+ * bias is added once per cube to the kernel-token product P', which every
+ * token of the cube receives (no per-token cost).  Linear layers commonly
+ * carry such a bias; the method's equations leave it out.
+ * Returns DQ_ERR_BAD_PACKED_WEIGHT when the blob's header is not a packed
+ * weight of this format.
+ */
+int dq_pack_bias(const uint16_t* bias, int Co, void* packed, size_t packed_bytes);
 
 /* dq_lowrank_factors (seed 0) followed by dq_pack_weight_factors. */
 int dq_pack_weight(const uint16_t* W, int Co, int Ci, int rank, void* packed, size_t packed_bytes,

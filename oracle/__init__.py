@@ -256,8 +256,12 @@ def quantize_weight(Wbits, L1, L2) -> dict:
 # --------------------------------------------------------------------------- output
 
 def output_rows(act: dict, wq: dict, X, L1, L2, rows, kernel: bool = True, lowrank: bool = True,
-                cube_major: bool = True) -> np.ndarray:
-    """fp64 Y rows (Eq. 3) for natural token indices `rows`."""
+                cube_major: bool = True, bias=None) -> np.ndarray:
+    """fp64 Y rows (Eq. 3) for natural token indices `rows`.
+
+    bias (Co BF16 bits, optional): the linear layer's bias b, y = x W^T + b.  The
+    method's equations carry no bias; with one, the plain reading is that b is
+    added to every output row, after the three terms."""
     X = np.ascontiguousarray(X, dtype=np.uint16)
     rows = np.ascontiguousarray(rows, dtype=np.int64)
     Co, Ci = wq["wcodes"].shape[0], wq["wcodes"].shape[1] * 2
@@ -273,4 +277,6 @@ def output_rows(act: dict, wq: dict, X, L1, L2, rows, kernel: bool = True, lowra
                              _p(rows), rows.size, _p(Y))
     if rc:
         raise RuntimeError("or_output_rows failed")
+    if bias is not None:
+        Y += bf16_value(np.asarray(bias, np.uint16).reshape(1, Co))
     return Y

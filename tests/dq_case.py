@@ -64,9 +64,11 @@ class Case:
         self.L1, self.L2, _ = oracle.lowrank_factors(self.Wb, wl.rank)
 
     # ---------------------------------------------------------------- GPU
-    def run_gpu(self, dq, torch, stage_mask=7, packed_override=None):
+    def run_gpu(self, dq, torch, stage_mask=7, packed_override=None, bias=None):
         wl, (t, h, w) = self.wl, self.cube
         packed, L1m, L2s, S_W = dq.dq_pack_weight_factors(self.Wb, self.L1, self.L2)
+        if bias is not None:
+            dq.dq_pack_bias(packed, bias)
         if packed_override is not None:
             packed = packed_override(packed)
         dev = torch.device("cuda")
@@ -102,8 +104,8 @@ class Case:
         wq = oracle.quantize_weight(self.Wb, self.L1, self.L2)
         return act, wq
 
-    def oracle_rows(self, act, wq, rows):
-        return oracle.output_rows(act, wq, self.X, self.L1, self.L2, rows)
+    def oracle_rows(self, act, wq, rows, bias=None):
+        return oracle.output_rows(act, wq, self.X, self.L1, self.L2, rows, bias=bias)
 
 
 def compare_quantised(g: dict, act: dict, wq: dict) -> None:

@@ -28,7 +28,7 @@ def test_exports_every_declared_symbol(dq):
     lib = ctypes.CDLL(dq.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
-    assert dq.dq_abi_version() == 1
+    assert dq.dq_abi_version() == 2
 
 
 def test_status_strings(dq):
@@ -122,7 +122,8 @@ def test_layouts_are_aligned_and_ordered(dq):
     assert L.N == 32760 and L.K == 8190 and L.slab == 64
     P = dq.dq_packed_weight_layout(5120, 5120, 32)
     assert P.off_codes == 256 and P.off_codes % 256 == 0 and P.off_scales % 256 == 0 and P.off_dqw % 256 == 0
-    assert P.total_bytes >= P.off_dqw + 5120 * 5120 * 2
+    assert P.off_bias >= P.off_dqw + 5120 * 5120 * 2 and P.off_bias % 256 == 0
+    assert P.total_bytes >= P.off_bias + 5120 * 4
     assert dq.dq_lowrank_slab_width(16) == 64 and dq.dq_lowrank_slab_width(48) == 128
 
 

@@ -91,6 +91,25 @@ def test_parity_small(env, name, wl):
     assert_y_close(g["Y"], y_ref)
 
 
+@pytest.mark.parametrize("name", ["ragged_122", "unit_cube", "global"])
+def test_parity_bias(env, name):
+    """A bias in the packed weight: every quantised tensor unchanged and bit-exact,
+    Y = the oracle's x W^T + b within tolerance, for a ragged lattice, the
+    one-token cube (P' per token) and the whole-lattice cube (one P' row)."""
+    dq, torch = env
+    wl = dict(SMALL)[name]
+    case = Case(wl)
+    b = synth.normal_bf16((wl.Co,), sd=4.0, seed=21)
+    g = case.run_gpu(dq, torch, bias=b)
+    act, wq = case.run_oracle()
+    compare_quantised(g, act, wq)
+    assert_y_close(g["Y"], case.oracle_rows(act, wq, np.arange(wl.N), bias=b))
+    # clearing the bias again gives the no-bias layer bit for bit
+    g0 = case.run_gpu(dq, torch)
+    g1 = case.run_gpu(dq, torch, packed_override=lambda p: dq.dq_pack_bias(dq.dq_pack_bias(p.copy(), b), None))
+    assert np.array_equal(g0["Y"], g1["Y"])
+
+
 def test_worked_example_through_gpu(env):
     """The hand-derived example (tests/golden) padded to 256 channels with zeros."""
     dq, torch = env

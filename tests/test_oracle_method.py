@@ -254,6 +254,21 @@ def test_unit_cube_has_zero_deltas_and_reduces_to_w4a8(tiny_case):
     np.testing.assert_allclose(Y, Y_ref, rtol=1e-12, atol=1e-12 * np.abs(Y_ref).max())
 
 
+def test_bias_special_cases(tiny_case):
+    """y = x W^T + b: an all-zero X leaves exactly b in every row (every other
+    term vanishes: zero kernel tokens, zero deltas, zero low-rank input), and
+    the bias moves no row's three terms (an all-zero b changes nothing)."""
+    wl, X, Wb, L1, L2, sig, act, wq = tiny_case
+    b = synth.normal_bf16((wl.Co,), sd=3.0, seed=11)
+    X0 = np.zeros_like(X)
+    act0 = oracle.quantize_activations(X0, wl.T, wl.H, wl.W, wl.cube)
+    Y0 = oracle.output_rows(act0, wq, X0, L1, L2, np.arange(wl.N), bias=b)
+    assert np.array_equal(Y0, np.broadcast_to(oracle.bf16_value(b).astype(np.float64), Y0.shape))
+    rows = np.arange(0, wl.N, 7)
+    Yb = oracle.output_rows(act, wq, X, L1, L2, rows, bias=np.zeros(wl.Co, np.uint16))
+    assert np.array_equal(Yb, oracle.output_rows(act, wq, X, L1, L2, rows))
+
+
 def test_residual_against_library_matmul(tiny_case):
     wl, X, Wb, L1, L2, *_ = tiny_case
     R = oracle.residual(Wb, L1, L2)

@@ -39,7 +39,10 @@ def test_pack_bit_exact(dq, shape):
     packed, L1m, L2s, S_W = dq.dq_pack_weight_factors(Wb, L1, L2)
     lay = dq.dq_packed_weight_layout(Co, Ci, r)
     hdr = packed[:256].view(np.uint32)
-    assert hdr[0] == 0x31575144 and hdr[1] == 2
+    assert hdr[0] == 0x31575144 and hdr[1] == 3
+    assert hdr[7] == 0 and not packed[lay.off_bias:lay.total_bytes].any()     # no bias
+    assert list(packed[32:72].view(np.uint64)) == [lay.off_codes, lay.off_scales, lay.off_dqw, lay.total_bytes,
+                                                  lay.off_bias]
     assert list(packed[8:24].view(np.int32)) == [Co, Ci, r, lay.slab]
     assert packed[24:28].view(np.float32)[0] == np.float32(wq["S_w"]) == np.float32(S_W)
     codes = packed[lay.off_codes:lay.off_codes + Co * Ci // 2].reshape(Co, Ci // 2)
@@ -78,3 +81,30 @@ def test_pack_weight_end_to_end_matches_factor_path(dq):
     L1, L2 = dq.dq_lowrank_factors(Wb, wl.rank, seed=0)
     p2, L1m2, L2s2, _ = dq.dq_pack_weight_factors(Wb, L1, L2)
     assert np.array_equal(packed, p2) and np.array_equal(L1m, L1m2) and np.array_equal(L2s, L2s2)
+
+
+def test_pack_bias_section(dq):
+    """dq_pack_bias widens the BF16 bias exactly to fp32 in the bias section and
+    sets header flag bit 0; clearing restores the blob bit for bit; a bias of
+    the wrong length or a blob that is not a packed weight is refused."""
+    Co, Ci, r = 512, 256, 16
+    wl = synth.Workload("pack", 1, 1, 1, Ci, Co, r, (1, 1, 1), (1, 1, 1), (0.0, 1.0), (0.01, 20.0))
+    Wb = synth.weight(wl, seed=3)
+    L1, L2, _ = oracle.lowrank_factors(Wb, r)
+    packed, *_ = dq.dq_pack_weight_factors(Wb, L1, L2)
+    orig = packed.copy()
+    lay = dq.dq_packed_weight_layout(Co, Ci, r)
+    b = synth.normal_bf16((Co,), sd=2.0, seed=4)
+    dq.dq_pack_bias(packed, b)
+    assert packed[28:32].view(np.uint32)[0] == 1
+    got = packed[lay.off_bias:lay.off_bias + 4 * Co].view(np.float32)
+    assert np.array_equal(got, oracle.bf16_value(b))
+    assert np.array_equal(packed[:lay.off_bias][256:], orig[:lay.off_bias][256:])
+    dq.dq_pack_bias(packed, None)
+    assert np.array_equal(packed, orig)
+    with pytest.raises(ValueError):
+        dq.dq_pack_bias(packed, b[:-1])
+    bad = packed.copy()
+    bad[0] ^= 1
+    with pytest.raises(dq.DQError):
+        dq.dq_pack_bias(bad, b)

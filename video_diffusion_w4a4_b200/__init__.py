@@ -38,7 +38,7 @@ DQ_STAGE_QUANTIZE, DQ_STAGE_KERNEL_GEMM, DQ_STAGE_MAIN_GEMM, DQ_STAGE_ALL = 1, 2
 
 class dq_packed_layout(ctypes.Structure):
     _fields_ = [("total_bytes", ctypes.c_size_t), ("off_codes", ctypes.c_size_t), ("off_scales", ctypes.c_size_t),
-                ("off_dqw", ctypes.c_size_t), ("Co", ctypes.c_int), ("Ci", ctypes.c_int), ("rank", ctypes.c_int),
+                ("off_dqw", ctypes.c_size_t), ("off_bias", ctypes.c_size_t), ("Co", ctypes.c_int), ("Ci", ctypes.c_int), ("rank", ctypes.c_int),
                 ("slab", ctypes.c_int)]
 
 
@@ -69,6 +69,7 @@ _SIGS = {
     "dq_lowrank_factors": ([_P, _I, _I, _I, ctypes.c_uint64, _P, _P], _I),
     "dq_pack_weight_factors": ([_P, _P, _P, _I, _I, _I, _P, _SZ, _P, _P, ctypes.POINTER(ctypes.c_float)], _I),
     "dq_pack_weight": ([_P, _I, _I, _I, _P, _SZ, _P, _P], _I),
+    "dq_pack_bias": ([_P, _I, _P, _SZ], _I),
     "dq_workspace_layout_get": ([_I] * 9 + [ctypes.POINTER(dq_workspace_layout)], _I),
     "dq_workspace_bytes": ([_I] * 9 + [ctypes.POINTER(_SZ)], _I),
     "dq_linear_forward": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P], _I),
@@ -220,6 +221,18 @@ def dq_pack_weight_factors(W: np.ndarray, L1: np.ndarray, L2: np.ndarray):
            _lib.dq_pack_weight_factors(W.ctypes.data, L1.ctypes.data, L2.ctypes.data, Co, Ci, r, packed.ctypes.data,
                                        packed.size, L1m.ctypes.data, L2s.ctypes.data, ctypes.byref(S)))
     return packed, L1m, L2s, S.value
+
+
+def dq_pack_bias(packed: np.ndarray, bias: np.ndarray | None) -> np.ndarray:
+    """Set (bias: uint16 BF16 bits, (Co,)) or clear (None) the bias of a host packed blob, in place."""
+    assert packed.dtype == np.uint8 and packed.flags["C_CONTIGUOUS"]
+    Co = int(packed[8:12].view(np.int32)[0])
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16)
+    if b is not None and b.size != Co:
+        raise ValueError(f"bias has {b.size} values, the packed weight has Co = {Co}")
+    _check("dq_pack_bias", _lib.dq_pack_bias(None if b is None else b.ctypes.data, Co, packed.ctypes.data,
+                                             packed.size))
+    return packed
 
 
 def dq_pack_weight(W: np.ndarray, rank: int):

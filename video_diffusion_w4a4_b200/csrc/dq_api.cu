@@ -306,6 +306,7 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
         p.k_stages = Ci / 64;
         p.s8 = qp.s8;
         p.pout = (float*)(ws + wl.off_p);
+        p.bias = (const float*)(pw + pl.off_bias);
         cudaError_t e = dq::launch_kernel_gemm(tm_a, tm_b, p, st);
         if (e != cudaSuccess) return cuda_fail(e, "kernel-token product");
     }

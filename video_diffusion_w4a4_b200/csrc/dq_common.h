@@ -125,12 +125,14 @@ struct PackedHeader {
     uint32_t magic, version;
     int32_t Co, Ci, rank, slab;
     float S_W;
-    uint32_t pad0;
-    uint64_t off_codes, off_scales, off_dqw, total;
+    uint32_t flags;      // kPackedHasBias: the bias section holds the layer's bias
+    uint64_t off_codes, off_scales, off_dqw, total, off_bias;
 };
 
+constexpr uint32_t kPackedHasBias = 1u;
+
 struct PackedLayout {
-    size_t total, off_codes, off_scales, off_dqw;
+    size_t total, off_codes, off_scales, off_dqw, off_bias;
     int Co, Ci, rank, slab;
 };
 
@@ -144,6 +146,8 @@ DQ_HD PackedLayout packed_layout(int Co, int Ci, int rank) {
     off = align_up(off + sfb_bytes(Co, Ci), kAlign);
     L.off_dqw = off;
     off = align_up(off + (size_t)Co * Ci * 2, kAlign);
+    L.off_bias = off;
+    off = align_up(off + (size_t)Co * 4, kAlign);
     L.total = off;
     return L;
 }

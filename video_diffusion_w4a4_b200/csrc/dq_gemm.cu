@@ -3,7 +3,8 @@
 // DeltaQuant note (papernotes.org), key design 4, Eq. 2/3:
 //   Y = Q4(delta) Q4(R)  +  broadcast_cube(Q8(kernel) Q4(R))  +  X L1 L2
 //
-//   (c) kernel-token product: P'[k][o] = s8_k S_W sum_c q8[k][c] (q s_b)[o][c].
+//   (c) kernel-token product: P'[k][o] = s8_k S_W sum_c q8[k][c] (q s_b)[o][c] (+ b[o] when the
+//       packed weight holds a bias).
 //       Both operands (the E4M3 kernel tokens and the dequantised weight
 //       q*s_b) are exact in BF16, so it runs as kind::f16 (BF16 x BF16 -> fp32).
 //       No FP8 tensor-core kind takes E4M3 group-16 weight scales.
@@ -350,6 +351,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             } else {
                 const float scale = row_ok ? __fmul_rn(p.s8[rho], S_W) : 0.f;
+                // the layer's bias, when the packed weight holds one, joins P' once per cube
+                const float* bias =
+                    (reinterpret_cast<const PackedHeader*>(p.packed_w)->flags & kPackedHasBias) ? p.bias + c_base
+                                                                                                 : nullptr;
                 const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], (uint32_t)use & 1, abort_flag,
                                                                   p.status, p.budget_ns));
                 if (!ok) break;
@@ -365,11 +370,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // 32-byte stores
 #pragma unroll
                         for (int v = 0; v < 16; v += 8) {
+                            float b0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                            float b1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                            if (bias) {
+                                ld_global_nc_v8(bias + c + v, b0);
+                                ld_global_nc_v8(bias + c + 16 + v, b1);
+                            }
                             uint32_t o0[8], o1[8];
 #pragma unroll
                             for (int e = 0; e < 8; e++) {
-                                o0[e] = __float_as_uint(__uint_as_float(r0[v + e]) * scale);
-                                o1[e] = __float_as_uint(__uint_as_float(r1[v + e]) * scale);
+                                o0[e] = __float_as_uint(fmaf(__uint_as_float(r0[v + e]), scale, b0[e]));
+                                o1[e] = __float_as_uint(fmaf(__uint_as_float(r1[v + e]), scale, b1[e]));
                             }
                             st_global_cs_v8(dst + c + v, o0);
                             st_global_cs_v8(dst + c + 16 + v, o1);

@@ -339,6 +339,7 @@ int dq_packed_weight_layout(int Co, int Ci, int rank, dq_packed_layout* out) {
     out->off_codes = L.off_codes;
     out->off_scales = L.off_scales;
     out->off_dqw = L.off_dqw;
+    out->off_bias = L.off_bias;
     out->Co = Co; out->Ci = Ci; out->rank = rank; out->slab = L.slab;
     return DQ_OK;
 }
@@ -473,6 +474,8 @@ int dq_pack_weight_factors(const uint16_t* Wb, const uint16_t* L1, const uint16_
     hdr.Co = Co; hdr.Ci = Ci; hdr.rank = r; hdr.slab = L.slab;
     hdr.S_W = S;
     hdr.off_codes = L.off_codes; hdr.off_scales = L.off_scales; hdr.off_dqw = L.off_dqw; hdr.total = L.total;
+    hdr.off_bias = L.off_bias;
+    hdr.flags = 0;
     memcpy(base, &hdr, sizeof(hdr));
     if (L1_mma)
         for (int i = 0; i < Ci; i++)
@@ -482,6 +485,23 @@ int dq_pack_weight_factors(const uint16_t* Wb, const uint16_t* L1, const uint16_
             for (int c = 0; c < L.slab; c++)
                 L2_slab[(size_t)o * L.slab + c] = (c < 2 * r) ? L2[(size_t)(c % r) * Co + o] : (uint16_t)0;
     if (S_W_out) *S_W_out = S;
+    return DQ_OK;
+}
+
+int dq_pack_bias(const uint16_t* bias, int Co, void* packed, size_t packed_bytes) {
+    if (!packed || packed_bytes < sizeof(dq::PackedHeader)) return DQ_ERR_INVALID_ARG;
+    dq::PackedHeader hdr;
+    memcpy(&hdr, packed, sizeof(hdr));
+    if (hdr.magic != DQ_PACK_MAGIC || hdr.version != DQ_PACK_FORMAT_VERSION || hdr.Co != Co ||
+        !shape_ok(hdr.Co, hdr.Ci, hdr.rank))
+        return DQ_ERR_BAD_PACKED_WEIGHT;
+    const dq::PackedLayout L = dq::packed_layout(hdr.Co, hdr.Ci, hdr.rank);
+    if (hdr.total != L.total || hdr.off_bias != L.off_bias) return DQ_ERR_BAD_PACKED_WEIGHT;
+    if (packed_bytes < L.total) return DQ_ERR_INVALID_ARG;
+    float* b = (float*)((uint8_t*)packed + L.off_bias);
+    for (int o = 0; o < Co; o++) b[o] = bias ? bf16_to_float(bias[o]) : 0.0f;
+    hdr.flags = bias ? (hdr.flags | dq::kPackedHasBias) : (hdr.flags & ~dq::kPackedHasBias);
+    memcpy(packed, &hdr, sizeof(hdr));
     return DQ_OK;
 }
 

@@ -48,6 +48,7 @@ struct GemmParams {
     const uint8_t* packed_w;
     const float* s8;     // kernel-token scales (kernel-token product)
     float* pout;         // kernel-token product output, K x Co fp32
+    const float* bias;   // Co fp32 bias section of the packed weight (read when its flag is set)
     uint16_t* Y;         // main product output, N x Co BF16 (t,h,w) order
     int* status;
     uint64_t budget_ns;

@@ -25,6 +25,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "../../include/deltaquant.h"
 #include "dq_common.h"
 #include "dq_internal.h"
 #include "dq_ptx.cuh"
@@ -658,7 +659,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
         *abort_flag = 0;
         fence_barrier_init();
         if (blockIdx.x == 0 &&
-            (hdr->magic != 0x31575144u || hdr->Ci != p.Ci || hdr->rank != p.rank || hdr->slab != p.slab))
+            (hdr->magic != DQ_PACK_MAGIC || hdr->version != DQ_PACK_FORMAT_VERSION || hdr->Ci != p.Ci || hdr->rank != p.rank || hdr->slab != p.slab))
             atomicCAS(p.status, 0, kStatusBadWeight);
     }
     // per-tensor delta scale S = amax / (6*448) (1 if amax = 0); S_W from the packed weight
