@@ -195,6 +195,39 @@ def quantize_plain(X) -> dict:
     return dict(dcodes=codes, dscales=scales, S_delta=S)
 
 
+def fp4_dequantize(codes, scales, S: float) -> np.ndarray:
+    """fp64 values q * s_g * S of FP4 rows (codes: rows x cols/2, channel 2i in
+    the low nibble of byte i; scales: rows x cols/16 E4M3)."""
+    codes = np.asarray(codes, np.uint8)
+    rows, half = codes.shape
+    v = np.empty((rows, half * 2), np.float64)
+    v[:, 0::2] = e2m1_value(codes & 15)
+    v[:, 1::2] = e2m1_value(codes >> 4)
+    return v * np.repeat(e4m3_value(scales), 16, axis=1) * float(S)
+
+
+KERNEL_FORMATS = ("bf16", "fp8", "nvfp4")
+
+
+def kernel_tokens_dequantized(act: dict, fmt: str = "fp8") -> np.ndarray:
+    """The dequantised kernel tokens (K x Ci, fp64) at one of three precisions,
+    the kernel-token precision ablation of the DeltaQuant note (16 / 8 / 4 bit):
+      bf16   the fp32 cube means rounded to BF16 (nearest even);
+      fp8    E4M3 codes under the per-token fp32 scale, the layer's own format;
+      nvfp4  the means as two-level NVFP4: E2M1 codes, E4M3 group-16 scales and
+             a per-tensor fp32 scale amax / (6 * 448), the delta tokens' format.
+    The deltas stay those of the fp32 means in every variant; only the kernel
+    term's operand changes."""
+    m = np.asarray(act["means"], np.float32)
+    if fmt == "bf16":
+        return bf16_value(bf16_round(m)).astype(np.float64)
+    if fmt == "fp8":
+        return e4m3_value(act["q8"]) * np.asarray(act["s8"], np.float64)[:, None]
+    if fmt == "nvfp4":
+        return fp4_dequantize(*fp4_quantize(m))
+    raise ValueError(fmt)
+
+
 # --------------------------------------------------------------------------- weight side
 
 def lowrank_factors(Wbits, r: int, seed: int = 0):
@@ -256,12 +289,21 @@ def quantize_weight(Wbits, L1, L2) -> dict:
 # --------------------------------------------------------------------------- output
 
 def output_rows(act: dict, wq: dict, X, L1, L2, rows, kernel: bool = True, lowrank: bool = True,
-                cube_major: bool = True, bias=None) -> np.ndarray:
+                cube_major: bool = True, bias=None, kernel_values=None) -> np.ndarray:
     """fp64 Y rows (Eq. 3) for natural token indices `rows`.
 
     bias (Co BF16 bits, optional): the linear layer's bias b, y = x W^T + b.  The
     method's equations carry no bias; with one, the plain reading is that b is
-    added to every output row, after the three terms."""
+    added to every output row, after the three terms.
+
+    kernel_values (K x Ci fp64, optional): dequantised kernel tokens that replace
+    the FP8 ones in the kernel term (see kernel_tokens_dequantized); that term is
+    then the fp64 library product kernel_values[k(n)] dq(R)^T."""
+    if kernel_values is not None:
+        Y = output_rows(act, wq, X, L1, L2, rows, kernel=False, lowrank=lowrank, cube_major=cube_major, bias=bias)
+        dqR = fp4_dequantize(wq["wcodes"], wq["wscales"], wq["S_w"])
+        kv = np.asarray(kernel_values, np.float64)[np.asarray(act["cube_of_n"])[np.asarray(rows)]]
+        return Y + kv @ dqR.T
     X = np.ascontiguousarray(X, dtype=np.uint16)
     rows = np.ascontiguousarray(rows, dtype=np.int64)
     Co, Ci = wq["wcodes"].shape[0], wq["wcodes"].shape[1] * 2

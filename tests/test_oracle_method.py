@@ -352,3 +352,55 @@ def test_worked_example_fixture():
     assert act["S_delta"] == np.float32(g["S_delta"])
     assert np.array_equal(act["dscales"][:, 0], np.array(g["dscales"], np.uint8))
     assert np.array_equal(act["dcodes"], np.array(g["dcodes"], np.uint8))
+
+
+# ------------------------------------------------------------------ kernel-token precision variants
+
+def test_kernel_values_route_matches_fp8_kernel_term(tiny_case):
+    """The replaceable kernel term (library fp64 product of dequantised kernel
+    tokens) reproduces the oracle's own C kernel term for the FP8 tokens."""
+    wl, X, Wb, L1, L2, sig, act, wq = tiny_case
+    rows = np.arange(wl.N)
+    y_c = oracle.output_rows(act, wq, X, L1, L2, rows)
+    y_v = oracle.output_rows(act, wq, X, L1, L2, rows, kernel_values=oracle.kernel_tokens_dequantized(act, "fp8"))
+    np.testing.assert_allclose(y_v, y_c, rtol=1e-12, atol=1e-12 * np.abs(y_c).max())
+
+
+def test_kernel_variants_exact_on_representable_means():
+    """Means already on a format's grid come back unchanged: BF16 values under
+    the BF16 variant; E2M1 grid values times a power of two per group under the
+    NVFP4 variant (up to the fp32 rounding of the per-tensor scale)."""
+    rng = np.random.default_rng(5)
+    bf = synth.normal_bf16((6, 64), sd=3.0, seed=9)
+    m = oracle.bf16_value(bf)
+    assert np.array_equal(oracle.kernel_tokens_dequantized({"means": m}, "bf16"), m.astype(np.float64))
+    grid = oracle.e2m1_value(np.arange(8))
+    v = grid[rng.integers(0, 8, size=(6, 64))] * np.where(rng.random((6, 64)) < 0.5, -1.0, 1.0)
+    v[:, ::16] = 6.0                                   # every group reaches the top code
+    v *= np.repeat(2.0 ** rng.integers(-6, 3, size=(6, 4)), 16, axis=1)
+    got = oracle.kernel_tokens_dequantized({"means": v.astype(np.float32)}, "nvfp4")
+    np.testing.assert_allclose(got, v, rtol=2.0 ** -22, atol=0)
+
+
+@pytest.mark.parametrize("shape", [(4, 16, 16, 512, 384), (8, 16, 24, 512, 256)])
+def test_kernel_precision_ablation(shape):
+    """The note's kernel-token precision ablation (16 / 8 / 4 bit) on correlated
+    synthetic activations: an FP8 kernel token costs almost nothing over BF16,
+    an NVFP4 one loses accuracy (relative Frobenius error of Y against the
+    unquantised X W^T)."""
+    T, H, W, Ci, Co = shape
+    wl = synth.Workload("mid", T, H, W, Ci, Co, 16, (1, 2, 2), (T, math.ceil(H / 4), math.ceil(W / 4)),
+                        (0.01, 50.0), (0.01, 20.0))
+    X = synth.activations(wl, seed=77)
+    Wb = synth.weight(wl, seed=78)
+    L1, L2, _ = oracle.lowrank_factors(Wb, wl.rank)
+    wq = oracle.quantize_weight(Wb, L1, L2)
+    rows = np.arange(0, wl.N, max(1, wl.N // 256))
+    ref = _x_f64(X)[rows] @ oracle.bf16_value(Wb).astype(np.float64).T
+    act = oracle.quantize_activations(X, wl.T, wl.H, wl.W, wl.cube)
+    err = {}
+    for f in oracle.KERNEL_FORMATS:
+        y = oracle.output_rows(act, wq, X, L1, L2, rows, kernel_values=oracle.kernel_tokens_dequantized(act, f))
+        err[f] = np.linalg.norm(y - ref) / np.linalg.norm(ref)
+    assert err["bf16"] <= err["fp8"] < 1.01 * err["bf16"], err
+    assert err["nvfp4"] > 1.02 * err["fp8"], err
