@@ -61,7 +61,8 @@ def _L():
         lib.or_fp4_quantize.argtypes = [P, LL, I, F, P, P, P]
         lib.or_quantize_activations.argtypes = [P] + [I] * 7 + [P] * 7
         lib.or_residual.argtypes = [P, P, P, I, I, I, P]
-        lib.or_output_rows.argtypes = [P, P, F, P, P, P, P, P, P, F, I, I, P, P, P, I, P, LL, P]
+        lib.or_output_rows.argtypes = [P, P, F, P, P, P, I, P, P, P, F, I, I, P, P, P, I, P, LL, P]
+        lib.or_fp8_kernel_tokens.argtypes = [P, LL, I, I, P, P]
         _lib = lib
     return _lib
 
@@ -166,8 +167,24 @@ def fp4_quantize(Z, S: float | None = None):
     return codes, scales, float(S_out.value)
 
 
-def quantize_activations(X, T, H, W, cube) -> dict:
-    """Activation side of Eq. 2/3 over the whole X (natural (t,h,w) row order)."""
+def fp8_kernel_tokens(means, group: int):
+    """FP8 E4M3 kernel tokens with one fp32 scale per `group` channels:
+    returns (q8 K x Ci, s8 K x Ci/group)."""
+    m = np.ascontiguousarray(means, dtype=np.float32)
+    K, Ci = m.shape
+    q8 = np.empty((K, Ci), np.uint8)
+    s8 = np.empty((K, Ci // group), np.float32)
+    if _L().or_fp8_kernel_tokens(_p(m), K, Ci, group, _p(q8), _p(s8)):
+        raise RuntimeError("or_fp8_kernel_tokens failed")
+    return q8, s8
+
+
+def quantize_activations(X, T, H, W, cube, kernel_group: int = 0) -> dict:
+    """Activation side of Eq. 2/3 over the whole X (natural (t,h,w) row order).
+
+    kernel_group 0: one FP8 scale per kernel token (s8: K); 64: one per 64
+    channels of a kernel token, the note's per-group kernel quantisation
+    (s8: K x Ci/64)."""
     X = np.ascontiguousarray(X, dtype=np.uint16)
     N, Ci = X.shape
     assert N == T * H * W
@@ -184,6 +201,9 @@ def quantize_activations(X, T, H, W, cube) -> dict:
         raise RuntimeError("or_quantize_activations failed")
     out["S_delta"] = float(S.value)
     out["amax_delta"] = float(amax.value)
+    out["kernel_group"] = kernel_group
+    if kernel_group:
+        out["q8"], out["s8"] = fp8_kernel_tokens(out["means"], kernel_group)
     out.update(cube_order(T, H, W, *cube))
     return out
 
@@ -222,7 +242,8 @@ def kernel_tokens_dequantized(act: dict, fmt: str = "fp8") -> np.ndarray:
     if fmt == "bf16":
         return bf16_value(bf16_round(m)).astype(np.float64)
     if fmt == "fp8":
-        return e4m3_value(act["q8"]) * np.asarray(act["s8"], np.float64)[:, None]
+        s8 = np.asarray(act["s8"], np.float64).reshape(len(act["q8"]), -1)
+        return e4m3_value(act["q8"]) * np.repeat(s8, act["q8"].shape[1] // s8.shape[1], axis=1)
     if fmt == "nvfp4":
         return fp4_dequantize(*fp4_quantize(m))
     raise ValueError(fmt)
@@ -312,7 +333,8 @@ def output_rows(act: dict, wq: dict, X, L1, L2, rows, kernel: bool = True, lowra
     arow = np.ascontiguousarray(act["row_of_n"], np.int32) if cube_major else None
     cube = np.ascontiguousarray(act["cube_of_n"], np.int32) if kernel else None
     rc = _L().or_output_rows(_p(act["dcodes"]), _p(act["dscales"]), act["S_delta"], _p(arow),
-                             _p(act["q8"]) if kernel else None, _p(act["s8"]) if kernel else None, _p(cube),
+                             _p(act["q8"]) if kernel else None, _p(act["s8"]) if kernel else None,
+                             (act.get("kernel_group") or Ci) if kernel else Ci, _p(cube),
                              _p(wq["wcodes"]), _p(wq["wscales"]), wq["S_w"], Co, Ci, _p(X),
                              _p(np.ascontiguousarray(L1, np.uint16)) if r else None,
                              _p(np.ascontiguousarray(L2, np.uint16)) if r else None, r,

@@ -299,7 +299,8 @@ int or_fp4_quantize(const float* Z, long long rows, int cols, float S_in, uint8_
     return 0;
 }
 
-/* FP8 kernel tokens: s8 = max_c |m_c| / 448, q8 = E4M3(m / s8), 0 if s8 = 0. */
+/* FP8 kernel tokens: s8 = max_c |m_c| / 448, q8 = E4M3(m / s8), 0 if s8 = 0
+ * (over the Ci channels of a token, or over one group of channels). */
 static void fp8_token(const float* m, int Ci, uint8_t* q8, float* s8) {
     float amax = 0.0f;
     for (int c = 0; c < Ci; c++) {
@@ -309,6 +310,24 @@ static void fp8_token(const float* m, int Ci, uint8_t* q8, float* s8) {
     float s = amax / 448.0f;
     *s8 = s;
     for (int c = 0; c < Ci; c++) q8[c] = (uint8_t)((s == 0.0f) ? 0 : or_e4m3_encode(m[c] / s));
+}
+
+/*
+ * FP8 kernel tokens with one scale per `group` consecutive channels (the
+ * note's per-group-64 kernel quantisation; group = Ci is one scale per token):
+ * s8[k][j] = max |m[k][c]| over channels c of group j, / 448;
+ * q8[k][c] = E4M3(m[k][c] / s8[k][c / group]), 0 where that scale is 0.
+ * means: K x Ci fp32; q8: K x Ci; s8: K x Ci/group.
+ */
+int or_fp8_kernel_tokens(const float* means, long long K, int Ci, int group, uint8_t* q8, float* s8) {
+    if (group <= 0 || Ci % group) return 1;
+    const int ng = Ci / group;
+#pragma omp parallel for schedule(static)
+    for (long long k = 0; k < K; k++)
+        for (int j = 0; j < ng; j++)
+            fp8_token(means + (size_t)k * Ci + (size_t)j * group, group, q8 + (size_t)k * Ci + (size_t)j * group,
+                      s8 + (size_t)k * ng + j);
+    return 0;
 }
 
 /*
@@ -393,14 +412,14 @@ int or_residual(const uint16_t* Wt, const uint16_t* L1, const uint16_t* L2, int 
 /*
  * Y rows in fp64 from the dequantised operands:
  *   Y[n][o] =  sum_c dqA[a(n)][c] dqR[o][c]                    (low-bit term)
- *            + s8[k(n)] sum_c q8[k(n)][c] dqR[o][c]              (single-token term)
+ *            + sum_c s8[k(n)][c / s8_group] q8[k(n)][c] dqR[o][c] (single-token term)
  *            + sum_j (sum_c x[n][c] L1[c][j]) L2[j][o]           (low-rank term)
  * acodes/ascales: FP4 activation rows with per-tensor S_a; a(n) = arow_of_n[n]
  * (identity when NULL).  q8 == NULL drops the single-token term; L1 == NULL
  * drops the low-rank term.  rows[]: natural token indices to evaluate.
  */
 int or_output_rows(const uint8_t* acodes, const uint8_t* ascales, float S_a, const int* arow_of_n,
-                   const uint8_t* q8, const float* s8, const int* cube_of_n,
+                   const uint8_t* q8, const float* s8, int s8_group, const int* cube_of_n,
                    const uint8_t* wcodes, const uint8_t* wscales, float S_w, int Co, int Ci,
                    const uint16_t* X, const uint16_t* L1, const uint16_t* L2, int r,
                    const long long* rows, long long nrows, double* Y) {
@@ -426,7 +445,9 @@ int or_output_rows(const uint8_t* acodes, const uint8_t* ascales, float S_a, con
         }
         if (q8) {
             long long k = cube_of_n[n];
-            for (int c = 0; c < Ci; c++) dqK[c] = or_e4m3_value(q8[(size_t)k * Ci + c]) * (double)s8[k];
+            const int ng = Ci / s8_group;
+            for (int c = 0; c < Ci; c++)
+                dqK[c] = or_e4m3_value(q8[(size_t)k * Ci + c]) * (double)s8[(size_t)k * ng + c / s8_group];
         }
         if (L1) {
             for (int j = 0; j < r; j++) {

@@ -404,3 +404,55 @@ def test_kernel_precision_ablation(shape):
         err[f] = np.linalg.norm(y - ref) / np.linalg.norm(ref)
     assert err["bf16"] <= err["fp8"] < 1.01 * err["bf16"], err
     assert err["nvfp4"] > 1.02 * err["fp8"], err
+
+
+# ------------------------------------------------------------------ group-64 kernel scales
+
+def test_group_kernel_scales_closed_form():
+    """Per-group FP8 kernel tokens on a hand-built token whose group amaxes
+    are 448 times powers of two: every quotient m / s8 is exact, so the codes
+    are the E4M3 encodings of known values (E4M3: bias 7, three mantissa bits;
+    448 = 0x7E, 1 = 0x38, -2 = 0xC0, 0.5 = 0x30, -3.5 = 0xC6, 2^-9 = 0x01), an
+    all-zero group has scale 0 and zero codes, and one scale for the whole
+    token (group = Ci) shrinks the small group onto coarser codes."""
+    m = np.zeros((1, 192), np.float32)
+    m[0, :4] = [56.0, 0.125, -0.25, 0.0625]                 # amax 56 -> s8 = 1/8
+    m[0, 64:67] = [7.0, -7.0 / 128, 2.0 ** -15]             # amax 7  -> s8 = 1/64
+    q8, s8 = oracle.fp8_kernel_tokens(m, 64)
+    assert s8.tolist() == [[0.125, 1.0 / 64, 0.0]]
+    assert q8[0, :4].tolist() == [0x7E, 0x38, 0xC0, 0x30] and not q8[0, 4:64].any()
+    assert q8[0, 64:67].tolist() == [0x7E, 0xC6, 0x01] and not q8[0, 67:].any()
+    q1, s1 = oracle.fp8_kernel_tokens(m, 192)
+    assert s1.tolist() == [[0.125]]
+    assert q1[0, 64] == 0x66                                 # 7 / (1/8) = 56 = 1.75 * 2^5
+
+
+def test_group_equal_to_token_width_is_the_per_token_path(tiny_case):
+    wl, X, Wb, L1, L2, sig, act, wq = tiny_case
+    q8, s8 = oracle.fp8_kernel_tokens(act["means"], wl.Ci)
+    assert np.array_equal(q8, act["q8"]) and np.array_equal(s8[:, 0], act["s8"])
+
+
+@pytest.mark.parametrize("cube", [(1, 2, 2), (2, 4, 4)])
+def test_group64_kernel_tokens_are_finer(cube):
+    """With outlier channels, one scale per 64 channels quantises the kernel
+    tokens more finely than one per token (the note's per-group-64 choice):
+    lower error of the dequantised kernel tokens, no worse Y."""
+    T, H, W, Ci, Co = 4, 16, 16, 512, 384
+    wl = synth.Workload("mid", T, H, W, Ci, Co, 16, cube, (T, 4, 4), (0.01, 50.0), (0.01, 20.0))
+    X = synth.activations(wl, seed=77)
+    Wb = synth.weight(wl, seed=78)
+    L1, L2, _ = oracle.lowrank_factors(Wb, wl.rank)
+    wq = oracle.quantize_weight(Wb, L1, L2)
+    rows = np.arange(0, wl.N, 4)
+    ref = _x_f64(X)[rows] @ oracle.bf16_value(Wb).astype(np.float64).T
+    ek, ey = {}, {}
+    for kg in (0, 64):
+        act = oracle.quantize_activations(X, T, H, W, cube, kernel_group=kg)
+        assert act["s8"].shape == ((act["q8"].shape[0],) if kg == 0 else (act["q8"].shape[0], Ci // 64))
+        kd = oracle.kernel_tokens_dequantized(act, "fp8")
+        ek[kg] = np.linalg.norm(kd - act["means"]) / np.linalg.norm(act["means"])
+        y = oracle.output_rows(act, wq, X, L1, L2, rows)
+        ey[kg] = np.linalg.norm(y - ref) / np.linalg.norm(ref)
+    assert ek[64] < 0.8 * ek[0], ek
+    assert ey[64] <= ey[0], ey
