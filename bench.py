@@ -39,18 +39,18 @@ def layer_flops(wl, K):
     return 2.0 * wl.N * wl.Ci * wl.Co + 2.0 * K * wl.Ci * wl.Co + 2.0 * wl.N * wl.rank * (wl.Ci + wl.Co)
 
 
-def stage_model(wl, K, slab):
+def stage_model(wl, K, slab, kernel_group=0):
     """Algorithmic work per launch of each stage (bytes that must cross HBM,
     tensor FLOPs).  Stage 1 reads X twice (statistics, then encode: the
     per-tensor delta scale needs every delta first)."""
     N, Ci, Co, r = wl.N, wl.Ci, wl.Co, wl.rank
     quant_bytes = (4.0 * N * Ci                      # X read by a1 and a2
                    + N * Ci / 2 + N * Ci / 16        # delta codes + scales
-                   + K * Ci * 3                      # q8 (E4M3) + its BF16 copy
+                   + K * Ci * (5 if kernel_group else 3)  # q8 (E4M3) + its BF16 copy (hi + lo when grouped)
                    + N * r * 4 * 2                   # X L1 partials (write + read)
                    + N * slab * 2 + 2 * r * Ci)      # U hi/lo, L1
     kernel_flops = 2.0 * K * Ci * Co
-    kernel_bytes = K * Ci * 2 + Co * Ci * 2 + K * Co * 4
+    kernel_bytes = K * Ci * (4 if kernel_group else 2) + Co * Ci * 2 + K * Co * 4
     main_flops = 2.0 * N * Ci * Co + 2.0 * N * slab * Co
     main_bytes = N * Ci * 9 / 16 + Co * Ci * 9 / 16 + N * slab * 2 + Co * slab * 2 + K * Co * 4 + N * Co * 2
     return dict(quantize=dict(bytes=quant_bytes, flops=2.0 * N * Ci * r),
@@ -217,6 +217,8 @@ def main():
     ap.add_argument("--workload", default="wan480p_proj", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--cube", default=None, help="override the cube, e.g. 2,2,2")
     ap.add_argument("--frames", type=int, default=None, help="override T (smaller cases for profiling)")
+    ap.add_argument("--kernel-group", type=int, default=0, choices=[0, 64],
+                    help="FP8 kernel-token scales: 0 = one per token, 64 = one per 64 channels")
     ap.add_argument("--sample-tokens", type=int, default=256, help="oracle sample size per reference step (tokens)")
     ap.add_argument("--baseline-tokens", type=int, default=4096, help="oracle sample size of the cpu_baseline leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -262,13 +264,14 @@ def main():
     L1d = torch.from_numpy(L1m.view(np.int16)).to(dev)
     L2d = torch.from_numpy(L2s.view(np.int16)).to(dev)
     Yd = torch.empty((wl.N, wl.Co), dtype=torch.int16, device=dev)
-    lay = dq.dq_workspace_layout_get(wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank)
+    kg = args.kernel_group
+    lay = dq.dq_workspace_layout_grouped(wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, kg)
     ws = torch.zeros(lay.total_bytes, dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream(dev)
 
     def step(events=None):
-        dq.dq_linear_forward_ex(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd, ws,
-                                lay.total_bytes, dq.DQ_STAGE_ALL, events, st)
+        dq.dq_linear_forward_grouped(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, kg, Pd, L1d, L2d, Yd, ws,
+                                     lay.total_bytes, dq.DQ_STAGE_ALL, events, st)
 
     for _ in range(args.warmup):
         step()
@@ -314,18 +317,20 @@ def main():
         dq.dq_linear_forward_host(Xh, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yh, Xd2, Yd2,
                                   ws, lay.total_bytes, st)
 
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    if dist:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(st)
-    for _ in range(args.e2e_steps):
+    e2e_ms = None
+    if not kg:   # the host-buffer entry point takes per-token kernel scales
         e2e_step()
-    e1.record(st)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if dist:
+        torch.cuda.synchronize(dev)
+        if dist:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(st)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if dist and e2e_ms is not None:
         tm = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(tm, op=dist.ReduceOp.MAX)
         e2e_ms = float(tm.item())
@@ -335,7 +340,7 @@ def main():
     value = F * world / (ms * 1e-3) / 1e12
     peaks = load_peaks()
     fp4_peak = peaks["bf16"] * FP4_PER_BF16
-    model = stage_model(wl, K, lay.slab)
+    model = stage_model(wl, K, lay.slab, kg)
     # dominant kernel = the stage with the largest share of the step
     dom = max(stage_ms, key=stage_ms.get)
     if dom == "quantize":
@@ -363,14 +368,16 @@ def main():
                 ms_per_step=ms, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="e2m1/e4m3->f32",
                 data="synthetic",
                 config=dict(workload=wl.name, T=wl.T, H=wl.H, W=wl.W, N=wl.N, Ci=wl.Ci, Co=wl.Co, rank=wl.rank,
-                            cube=list(cube), K=K, parallelism=f"dp{world} (independent layer per GPU)",
+                            cube=list(cube), K=K,
+                            kernel_scale="per-token" if not kg else f"group{kg}", parallelism=f"dp{world} (independent layer per GPU)",
                             l2="inputs larger than L2 (X %.0f MB, Y %.0f MB)" % (wl.N * wl.Ci * 2 / 1e6,
                                                                                  wl.N * wl.Co * 2 / 1e6)),
                 tokens_per_s=wl.N * world / (ms * 1e-3),
                 layer_roofline_frac=layer_roof_ms / ms,
                 roofline=roof, stages=stages,
-                e2e=dict(value=F * world / (e2e_ms * 1e-3) / 1e12, unit="TFLOP/s",
-                         h2d_bytes_per_step=wl.N * wl.Ci * 2, d2h_bytes_per_step=wl.N * wl.Co * 2, ms_per_step=e2e_ms),
+                e2e=None if e2e_ms is None else dict(
+                    value=F * world / (e2e_ms * 1e-3) / 1e12, unit="TFLOP/s", h2d_bytes_per_step=wl.N * wl.Ci * 2,
+                    d2h_bytes_per_step=wl.N * wl.Co * 2, ms_per_step=e2e_ms),
                 gpu_launches=(5 if t * h * w > 128 else 4) * args.steps, pack_seconds=pack_s)
     clk_sum = clk.summary()
     if clk_sum:

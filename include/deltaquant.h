@@ -223,9 +223,11 @@ int dq_pack_weight(const uint16_t* W, int Co, int Ci, int rank, void* packed, si
  *   status     int32 device status word (0 = ok, else a dq_status)
  *   scalars    uint32[4]: [0] bits of max|delta| (fp32), [1] S_delta (fp32)
  *   kamax      K uint32: bits of max_c |mean_k[c]| per cube (fp32)
- *   s8         K fp32 kernel-token scales
+ *   s8         K fp32 kernel-token scales (per-token), or K x Ci/64 (group 64)
  *   q8         K x Ci E4M3 kernel tokens
- *   q8_bf16    K_pad x Ci BF16 copy of q8 (the kernel-token product's A operand)
+ *   q8_bf16    the kernel-token product's A operand: K_pad x Ci BF16 copy of q8
+ *              (per-token), or K_pad x 2Ci BF16 q8*s8 split as hi (columns
+ *              0..Ci-1) + lo (Ci..2Ci-1), |hi + lo - q8 s8| <= 2^-16 |q8 s8| (group 64)
  *   dcodes     N x Ci/2 E2M1 delta codes, cube-major rows
  *   dscales    delta group scales, A-operand scale layout (dq_sfa_offset) over N rows
  *   u_part     splits x N x rank fp32 partial sums of X L1 (cube-major rows)
@@ -239,12 +241,32 @@ typedef struct dq_workspace_layout {
         off_u_part, off_u_hilo, off_p, off_means;
     long long N, K, N_pad, K_pad;
     int splits, slab;
+    int kernel_group;
 } dq_workspace_layout;
 
+/*
+ * FP8 kernel-token scale granularity (argument kernel_group):
+ *   DQ_KERNEL_SCALE_PER_TOKEN  s8[k] = max_c |mean_k[c]| / 448, one per kernel token
+ *   DQ_KERNEL_SCALE_GROUP64    s8[k][j] = max |mean_k[c]| / 448 over channels
+ *                              c in [64 j, 64 j + 64): the DeltaQuant note's
+ *                              per-group-64 kernel quantisation (its section on
+ *                              the training strategy).  The kernel-token product then reads
+ *                              2 Ci BF16 columns per kernel token (hi + lo).
+ * q8[k][c] = E4M3(mean_k[c] / scale), 0 where the scale is 0, in both.
+ */
+#define DQ_KERNEL_SCALE_PER_TOKEN 0
+#define DQ_KERNEL_SCALE_GROUP64 64
+
+/* Workspace carve-up of a forward call with per-token kernel scales. */
 int dq_workspace_layout_get(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
                             dq_workspace_layout* out);
 int dq_workspace_bytes(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
                        size_t* bytes);
+/* The same for a kernel_group (DQ_KERNEL_SCALE_*; anything else: DQ_ERR_INVALID_ARG). */
+int dq_workspace_layout_grouped(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                                int kernel_group, dq_workspace_layout* out);
+int dq_workspace_bytes_grouped(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                               int kernel_group, size_t* bytes);
 
 /* Stage selection for dq_linear_forward_ex. */
 #define DQ_STAGE_QUANTIZE 1    /* cube statistics + cube encode (kernels a1, a2) */
@@ -277,6 +299,17 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
                          const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y,
                          void* workspace, size_t workspace_bytes, int stage_mask, void* const* stage_events,
                          void* stream);
+
+/*
+ * As dq_linear_forward_ex with the kernel-token scale granularity kernel_group
+ * (DQ_KERNEL_SCALE_*); the workspace is at least dq_workspace_bytes_grouped
+ * for the same kernel_group.  dq_linear_forward_ex is this call with
+ * DQ_KERNEL_SCALE_PER_TOKEN.
+ */
+int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                              int kernel_group, const void* packed_W, const void* L1_mma, const void* L2_slab,
+                              void* Y, void* workspace, size_t workspace_bytes, int stage_mask,
+                              void* const* stage_events, void* stream);
 
 /*
  * As dq_linear_forward_ex with HOST X and Y (pinned for asynchronous copies):

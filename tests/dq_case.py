@@ -56,8 +56,9 @@ def assert_y_close(y_bits: np.ndarray, y_ref: np.ndarray, what: str = "Y") -> di
 class Case:
     """One layer instance: workload, inputs, oracle factors."""
 
-    def __init__(self, wl: synth.Workload, cube=None, seed=None, tau: int = 0, X=None, Wb=None):
+    def __init__(self, wl: synth.Workload, cube=None, seed=None, tau: int = 0, X=None, Wb=None, kernel_group: int = 0):
         self.wl = wl
+        self.kernel_group = kernel_group
         self.cube = tuple(cube or wl.cube)
         self.X = synth.activations(wl, seed=seed, tau=tau) if X is None else X
         self.Wb = synth.weight(wl, seed=seed) if Wb is None else Wb
@@ -77,21 +78,28 @@ class Case:
         L1d = torch.from_numpy(L1m.view(np.int16)).to(dev)
         L2d = torch.from_numpy(L2s.view(np.int16)).to(dev)
         Yd = torch.empty((wl.N, wl.Co), dtype=torch.int16, device=dev)
-        lay = dq.dq_workspace_layout_get(wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank)
+        kg = self.kernel_group
+        lay = dq.dq_workspace_layout_grouped(wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, kg)
         ws = torch.zeros(lay.total_bytes, dtype=torch.uint8, device=dev)
-        dq.dq_linear_forward_ex(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd, ws,
-                                lay.total_bytes, stage_mask, None, torch.cuda.current_stream())
+        if kg:
+            dq.dq_linear_forward_grouped(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, kg, Pd, L1d, L2d, Yd,
+                                         ws, lay.total_bytes, stage_mask, None, torch.cuda.current_stream())
+        else:
+            dq.dq_linear_forward_ex(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd, ws,
+                                    lay.total_bytes, stage_mask, None, torch.cuda.current_stream())
         torch.cuda.synchronize()
         status = dq.dq_read_device_status(ws, torch.cuda.current_stream(), clear=True)
         wsh = ws.cpu().numpy()
         N, K, Ci = lay.N, lay.K, wl.Ci
+        ns8 = Ci // kg if kg else 1
+        acols = 2 * Ci if kg else Ci
         out = dict(status=status, layout=lay, S_W=S_W, packed=packed,
                    Y=Yd.cpu().numpy().view(np.uint16),
                    amax_delta=wsh[lay.off_scalars:lay.off_scalars + 4].view(np.float32)[0],
                    S_delta=wsh[lay.off_scalars + 4:lay.off_scalars + 8].view(np.float32)[0],
-                   s8=wsh[lay.off_s8:lay.off_s8 + 4 * K].view(np.float32),
+                   s8=wsh[lay.off_s8:lay.off_s8 + 4 * K * ns8].view(np.float32).reshape((K, ns8) if kg else (K,)),
                    q8=wsh[lay.off_q8:lay.off_q8 + K * Ci].reshape(K, Ci),
-                   q8_bf16=wsh[lay.off_q8_bf16:lay.off_q8_bf16 + 2 * K * Ci].view(np.uint16).reshape(K, Ci),
+                   q8_bf16=wsh[lay.off_q8_bf16:lay.off_q8_bf16 + 2 * K * acols].view(np.uint16).reshape(K, acols),
                    dcodes=wsh[lay.off_dcodes:lay.off_dcodes + N * Ci // 2].reshape(N, Ci // 2),
                    dscales=sfa_unpermute(wsh[lay.off_dscales:], N, Ci),
                    p=wsh[lay.off_p:lay.off_p + 4 * K * wl.Co].view(np.float32).reshape(K, wl.Co))
@@ -100,7 +108,7 @@ class Case:
     # ---------------------------------------------------------------- oracle
     def run_oracle(self):
         wl = self.wl
-        act = oracle.quantize_activations(self.X, wl.T, wl.H, wl.W, self.cube)
+        act = oracle.quantize_activations(self.X, wl.T, wl.H, wl.W, self.cube, kernel_group=self.kernel_group)
         wq = oracle.quantize_weight(self.Wb, self.L1, self.L2)
         return act, wq
 
@@ -117,7 +125,14 @@ def compare_quantised(g: dict, act: dict, wq: dict) -> None:
     assert np.array_equal(g["s8"], act["s8"]), "s8"
     bad = np.argwhere(g["q8"] != act["q8"])
     assert bad.size == 0, ("q8", bad[:5].tolist(), g["q8"][tuple(bad[0])], act["q8"][tuple(bad[0])])
-    assert np.array_equal(bf16_bits_to_f64(g["q8_bf16"]), oracle.e4m3_value(act["q8"])), "q8 as BF16"
+    if act.get("kernel_group"):
+        # the product's operand: q8 s8 as BF16 hi + lo, within 2^-16 of the exact product
+        Ci = act["q8"].shape[1]
+        want = oracle.kernel_tokens_dequantized(act, "fp8")
+        hl = bf16_bits_to_f64(g["q8_bf16"][:, :Ci]) + bf16_bits_to_f64(g["q8_bf16"][:, Ci:])
+        assert np.all(np.abs(hl - want) <= 2.0 ** -16 * np.abs(want)), "q8 s8 as BF16 hi + lo"
+    else:
+        assert np.array_equal(bf16_bits_to_f64(g["q8_bf16"]), oracle.e4m3_value(act["q8"])), "q8 as BF16"
     bad = np.argwhere(g["dscales"] != act["dscales"])
     assert bad.size == 0, ("delta scales", bad[:5].tolist())
     bad = np.argwhere(g["dcodes"] != act["dcodes"])

@@ -92,3 +92,20 @@ def test_cube_sweep(env, cube):
     if cube not in ((1, 1, 1), (21, 30, 52)):
         # local cubes beat plain FP4 (the note's cube-size ablation: the global kernel loses the local structure)
         assert info["rel_err_gpu"] < info["rel_err_plain_nvfp4"], info
+
+
+@pytest.mark.parametrize("cube", [(1, 2, 2), (4, 2, 8)])
+def test_full_size_group64_kernel_scales(env, cube):
+    """The 480p projection with one FP8 kernel scale per 64 channels (the note's
+    per-group kernel quantisation), at the bench's cube and at the note's
+    64-token cube."""
+    dq, torch = env
+    wl = synth.WORKLOADS["wan480p_cube_sweep"].with_cube(cube)
+    case = Case(wl, kernel_group=64)
+    g = case.run_gpu(dq, torch)
+    act, wq = case.run_oracle()
+    compare_quantised(g, act, wq)
+    rows = sample_rows(wl, cube, n_cubes=32)
+    info = assert_y_close(g["Y"][rows], case.oracle_rows(act, wq, rows))
+    info.update(cube=list(cube), kernel_group=64, rows=int(rows.size))
+    _record("group64_%d%d%d" % cube, info)

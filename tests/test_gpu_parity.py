@@ -110,6 +110,22 @@ def test_parity_bias(env, name):
     assert np.array_equal(g0["Y"], g1["Y"])
 
 
+@pytest.mark.parametrize("name", ["tiny", "ragged_122", "unit_cube", "cube_414_r128", "cube_428", "global",
+                                  "wide_cube"])
+def test_parity_group64_kernel_scales(env, name):
+    """One FP8 scale per 64 channels of each kernel token: codes and the
+    K x Ci/64 scales bit-exact, the hi + lo product operand within 2^-16, Y
+    within tolerance; across small and big cubes and ragged lattices."""
+    dq, torch = env
+    wl = dict(SMALL)[name] or synth.WORKLOADS["tiny"]
+    case = Case(wl, kernel_group=64)
+    g = case.run_gpu(dq, torch)
+    act, wq = case.run_oracle()
+    assert g["s8"].shape == act["s8"].shape
+    compare_quantised(g, act, wq)
+    assert_y_close(g["Y"], case.oracle_rows(act, wq, np.arange(wl.N)))
+
+
 def test_worked_example_through_gpu(env):
     """The hand-derived example (tests/golden) padded to 256 channels with zeros."""
     dq, torch = env

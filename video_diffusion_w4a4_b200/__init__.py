@@ -34,6 +34,7 @@ DQ_ERR_BAD_PACKED_WEIGHT = 7
 DQ_ERR_NO_DEVICE = 8
 DQ_ERR_ALLOC = 9
 DQ_STAGE_QUANTIZE, DQ_STAGE_KERNEL_GEMM, DQ_STAGE_MAIN_GEMM, DQ_STAGE_ALL = 1, 2, 4, 7
+DQ_KERNEL_SCALE_PER_TOKEN, DQ_KERNEL_SCALE_GROUP64 = 0, 64
 
 
 class dq_packed_layout(ctypes.Structure):
@@ -47,7 +48,7 @@ class dq_workspace_layout(ctypes.Structure):
         (n, ctypes.c_size_t) for n in ("off_status", "off_scalars", "off_kamax", "off_s8", "off_q8", "off_q8_bf16",
                                        "off_dcodes", "off_dscales", "off_u_part", "off_u_hilo", "off_p", "off_means")] + [
         ("N", ctypes.c_longlong), ("K", ctypes.c_longlong), ("N_pad", ctypes.c_longlong), ("K_pad", ctypes.c_longlong),
-        ("splits", ctypes.c_int), ("slab", ctypes.c_int)]
+        ("splits", ctypes.c_int), ("slab", ctypes.c_int), ("kernel_group", ctypes.c_int)]
 
 
 _P, _I, _SZ, _LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
@@ -74,6 +75,9 @@ _SIGS = {
     "dq_workspace_bytes": ([_I] * 9 + [ctypes.POINTER(_SZ)], _I),
     "dq_linear_forward": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P], _I),
     "dq_linear_forward_ex": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P, _SZ, _I, _P, _P], _I),
+    "dq_linear_forward_grouped": ([_P] + [_I] * 10 + [_P, _P, _P, _P, _P, _SZ, _I, _P, _P], _I),
+    "dq_workspace_layout_grouped": ([_I] * 10 + [ctypes.POINTER(dq_workspace_layout)], _I),
+    "dq_workspace_bytes_grouped": ([_I] * 10 + [ctypes.POINTER(_SZ)], _I),
     "dq_linear_forward_host": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
     "dq_linear_forward_noalloc": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P], _I),
     "dq_read_device_status": ([_P, _P, ctypes.POINTER(_I), _I], _I),
@@ -256,6 +260,20 @@ def dq_workspace_layout_get(T, H, W, t, h, w, Ci, Co, rank) -> dq_workspace_layo
     return L
 
 
+def dq_workspace_layout_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group) -> dq_workspace_layout:
+    L = dq_workspace_layout()
+    _check("dq_workspace_layout_grouped", _lib.dq_workspace_layout_grouped(T, H, W, t, h, w, Ci, Co, rank,
+                                                                           kernel_group, ctypes.byref(L)))
+    return L
+
+
+def dq_workspace_bytes_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group) -> int:
+    b = ctypes.c_size_t()
+    _check("dq_workspace_bytes_grouped", _lib.dq_workspace_bytes_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group,
+                                                                         ctypes.byref(b)))
+    return b.value
+
+
 def dq_workspace_bytes(T, H, W, t, h, w, Ci, Co, rank) -> int:
     b = ctypes.c_size_t()
     _check("dq_workspace_bytes", _lib.dq_workspace_bytes(T, H, W, t, h, w, Ci, Co, rank, ctypes.byref(b)))
@@ -267,15 +285,28 @@ def dq_linear_forward(X, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_sl
                                                        _ptr(L1_mma), _ptr(L2_slab), _ptr(Y), _stream(stream)))
 
 
+def _events(stage_events):
+    if stage_events is None:
+        return None
+    handles = [e.cuda_event if hasattr(e, "cuda_event") else e for e in stage_events]
+    if len(handles) != 4 or not all(handles):
+        raise ValueError("stage_events needs 4 created CUDA events (record a torch.cuda.Event once first)")
+    arr = (ctypes.c_void_p * 4)(*handles)
+    return ctypes.cast(arr, ctypes.c_void_p)
+
+
+def dq_linear_forward_grouped(X, T, H, W, t, h, w, Ci, Co, rank, kernel_group, packed_W, L1_mma, L2_slab, Y,
+                              workspace, workspace_bytes, stage_mask=DQ_STAGE_ALL, stage_events=None,
+                              stream=None) -> None:
+    _check("dq_linear_forward_grouped",
+           _lib.dq_linear_forward_grouped(_ptr(X), T, H, W, t, h, w, Ci, Co, rank, kernel_group, _ptr(packed_W),
+                                          _ptr(L1_mma), _ptr(L2_slab), _ptr(Y), _ptr(workspace), workspace_bytes,
+                                          stage_mask, _events(stage_events), _stream(stream)))
+
+
 def dq_linear_forward_ex(X, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y, workspace,
                          workspace_bytes, stage_mask=DQ_STAGE_ALL, stage_events=None, stream=None) -> None:
-    ev = None
-    if stage_events is not None:
-        handles = [e.cuda_event if hasattr(e, "cuda_event") else e for e in stage_events]
-        if len(handles) != 4 or not all(handles):
-            raise ValueError("stage_events needs 4 created CUDA events (record a torch.cuda.Event once first)")
-        arr = (ctypes.c_void_p * 4)(*handles)
-        ev = ctypes.cast(arr, ctypes.c_void_p)
+    ev = _events(stage_events)
     _check("dq_linear_forward_ex",
            _lib.dq_linear_forward_ex(_ptr(X), T, H, W, t, h, w, Ci, Co, rank, _ptr(packed_W), _ptr(L1_mma),
                                      _ptr(L2_slab), _ptr(Y), _ptr(workspace), workspace_bytes, stage_mask, ev,

@@ -166,12 +166,13 @@ int ensure_lib_workspace(size_t need, void** ws) {
 
 extern "C" {
 
-int dq_workspace_layout_get(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
-                            dq_workspace_layout* out) {
+int dq_workspace_layout_grouped(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank, int kernel_group,
+                                dq_workspace_layout* out) {
     if (!out) return DQ_ERR_INVALID_ARG;
     int rc = check_shape(T, H, W, t, h, w, Ci, Co, rank);
     if (rc) return rc;
-    dq::WsLayout L = dq::ws_layout(dq::make_geom(T, H, W, t, h, w), Ci, Co, rank);
+    if (kernel_group != DQ_KERNEL_SCALE_PER_TOKEN && kernel_group != DQ_KERNEL_SCALE_GROUP64) return DQ_ERR_INVALID_ARG;
+    dq::WsLayout L = dq::ws_layout(dq::make_geom(T, H, W, t, h, w), Ci, Co, rank, kernel_group);
     out->total_bytes = L.total;
     out->off_status = L.off_status;
     out->off_scalars = L.off_scalars;
@@ -191,6 +192,22 @@ int dq_workspace_layout_get(int T, int H, int W, int t, int h, int w, int Ci, in
     out->K_pad = L.K_pad;
     out->splits = L.splits;
     out->slab = L.slab;
+    out->kernel_group = kernel_group;
+    return DQ_OK;
+}
+
+int dq_workspace_layout_get(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                            dq_workspace_layout* out) {
+    return dq_workspace_layout_grouped(T, H, W, t, h, w, Ci, Co, rank, DQ_KERNEL_SCALE_PER_TOKEN, out);
+}
+
+int dq_workspace_bytes_grouped(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank, int kernel_group,
+                               size_t* bytes) {
+    if (!bytes) return DQ_ERR_INVALID_ARG;
+    dq_workspace_layout L;
+    int rc = dq_workspace_layout_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group, &L);
+    if (rc) return rc;
+    *bytes = L.total_bytes;
     return DQ_OK;
 }
 
@@ -203,18 +220,21 @@ int dq_workspace_bytes(int T, int H, int W, int t, int h, int w, int Ci, int Co,
     return DQ_OK;
 }
 
-int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
-                         const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y, void* workspace,
-                         size_t workspace_bytes, int stage_mask, void* const* stage_events, void* stream) {
+int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                              int kernel_group, const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y,
+                              void* workspace, size_t workspace_bytes, int stage_mask, void* const* stage_events,
+                              void* stream) {
     int rc = check_shape(T, H, W, t, h, w, Ci, Co, rank);
     if (rc) return rc;
+    if (kernel_group != DQ_KERNEL_SCALE_PER_TOKEN && kernel_group != DQ_KERNEL_SCALE_GROUP64) return DQ_ERR_INVALID_ARG;
+    const int kg = kernel_group;
     if (!X || !packed_W || !L1_mma || !L2_slab || !Y || !workspace) return DQ_ERR_INVALID_ARG;
     if (stage_mask <= 0 || stage_mask > DQ_STAGE_ALL) return DQ_ERR_INVALID_ARG;
     if (!aligned(X) || !aligned(packed_W) || !aligned(L1_mma) || !aligned(L2_slab) || !aligned(Y) ||
         !aligned(workspace))
         return DQ_ERR_ALIGNMENT;
     const Geom g = dq::make_geom(T, H, W, t, h, w);
-    const dq::WsLayout wl = dq::ws_layout(g, Ci, Co, rank);
+    const dq::WsLayout wl = dq::ws_layout(g, Ci, Co, rank, kg);
     if (workspace_bytes < wl.total) return DQ_ERR_WORKSPACE_TOO_SMALL;
     if (!encode_fn()) return DQ_ERR_NO_DEVICE;
     cudaStream_t st = (cudaStream_t)stream;
@@ -229,6 +249,7 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
     qp.rank = rank;
     qp.slab = wl.slab;
     qp.splits = wl.splits;
+    qp.kgroup = kg;
     qp.chunks_per_split = Ci / 64 / wl.splits;
     qp.big = (long long)t * h * w > 128;
     if (!qp.big) {
@@ -298,13 +319,15 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
     rec(1);
     if (stage_mask & DQ_STAGE_KERNEL_GEMM) {
         CUtensorMap tm_a, tm_b;
-        if (!map_2d(&tm_a, ws + wl.off_q8_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, g.K, 64, 128))
+        const int a_cols = kg ? 2 * Ci : Ci;   // grouped scales: [hi | lo]
+        if (!map_2d(&tm_a, ws + wl.off_q8_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a_cols, g.K, 64, 128))
             return map_fail("product A");
         if (!map_2d(&tm_b, pw + pl.off_dqw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, Co, 64, 128)) return map_fail("product B");
         dq::GemmParams p = gp;
         p.M = (int)g.K;
-        p.k_stages = Ci / 64;
-        p.s8 = qp.s8;
+        p.k_stages = a_cols / 64;
+        p.b_kblocks = Ci / 64;
+        p.s8 = kg ? nullptr : qp.s8;
         p.pout = (float*)(ws + wl.off_p);
         p.bias = (const float*)(pw + pl.off_bias);
         cudaError_t e = dq::launch_kernel_gemm(tm_a, tm_b, p, st);
@@ -333,6 +356,13 @@ int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w
     }
     rec(3);
     return DQ_OK;
+}
+
+int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                         const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y, void* workspace,
+                         size_t workspace_bytes, int stage_mask, void* const* stage_events, void* stream) {
+    return dq_linear_forward_grouped(X, T, H, W, t, h, w, Ci, Co, rank, DQ_KERNEL_SCALE_PER_TOKEN, packed_W, L1_mma,
+                                     L2_slab, Y, workspace, workspace_bytes, stage_mask, stage_events, stream);
 }
 
 int dq_linear_forward(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,

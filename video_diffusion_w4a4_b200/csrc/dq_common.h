@@ -170,7 +170,9 @@ struct WsLayout {
     int splits, slab;
 };
 
-DQ_HD WsLayout ws_layout(const Geom& g, int Ci, int Co, int rank) {
+// kgroup: 0 = one FP8 scale per kernel token; 64 = one per 64 channels, whose
+// kernel tokens enter the product as BF16 hi + lo (twice the columns)
+DQ_HD WsLayout ws_layout(const Geom& g, int Ci, int Co, int rank, int kgroup = 0) {
     WsLayout L;
     L.N = g.N; L.K = g.K;
     L.N_pad = cdiv(g.N, 128) * 128;
@@ -181,9 +183,9 @@ DQ_HD WsLayout ws_layout(const Geom& g, int Ci, int Co, int rank) {
     L.off_status = off;   off = align_up(off + 16, kAlign);
     L.off_scalars = off;  off = align_up(off + 16, kAlign);
     L.off_kamax = off;    off = align_up(off + (size_t)g.K * 4, kAlign);
-    L.off_s8 = off;       off = align_up(off + (size_t)g.K * 4, kAlign);
+    L.off_s8 = off;       off = align_up(off + (size_t)g.K * (kgroup ? Ci / kgroup : 1) * 4, kAlign);
     L.off_q8 = off;       off = align_up(off + (size_t)g.K * Ci, kAlign);
-    L.off_q8_bf16 = off;  off = align_up(off + (size_t)L.K_pad * Ci * 2, kAlign);
+    L.off_q8_bf16 = off;  off = align_up(off + (size_t)L.K_pad * Ci * 2 * (kgroup ? 2 : 1), kAlign);
     L.off_dcodes = off;   off = align_up(off + (size_t)g.N * (Ci / 2), kAlign);
     L.off_dscales = off;  off = align_up(off + sfa_bytes(g.N, Ci), kAlign);
     L.off_u_part = off;   off = align_up(off + (size_t)L.splits * g.N * rank * 4, kAlign);

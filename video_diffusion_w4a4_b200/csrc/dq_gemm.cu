@@ -8,6 +8,9 @@
 //       Both operands (the E4M3 kernel tokens and the dequantised weight
 //       q*s_b) are exact in BF16, so it runs as kind::f16 (BF16 x BF16 -> fp32).
 //       No FP8 tensor-core kind takes E4M3 group-16 weight scales.
+//       With one kernel scale per 64 channels the scale varies along K, so the
+//       A operand is q8 s8 itself as BF16 hi + lo (2 Ci columns: every weight
+//       k-block is read twice) and P' = S_W acc.
 //   (b) main product: acc[rho][o] = sum_c (q s)_delta (q s)_R with
 //       kind::mxf4nvf4 block-16 scaled FP4 MMAs, then the low-rank
 //       up-projection as extra BF16 K-steps [U_hi | U_lo] x [L2^T | L2^T] into
@@ -169,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!kMain) {
                         if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes));
                         tma_load_2d_pair_hint(sa, &tm_a, fb, i * 64, m0, stream);
-                        tma_load_2d_pair_hint(sb, &tm_b, fb, i * 64, nb, keep);
+                        tma_load_2d_pair_hint(sb, &tm_b, fb, (i < p.b_kblocks ? i : i - p.b_kblocks) * 64, nb, keep);
                     } else if (i < nk) {
                         if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes + kSFABytes + kSFBBytes));
                         tma_load_2d_pair(sa, &tm_a, fb, i * 128, m0);
@@ -350,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             } else {
-                const float scale = row_ok ? __fmul_rn(p.s8[rho], S_W) : 0.f;
+                const float scale = row_ok ? (p.s8 ? __fmul_rn(p.s8[rho], S_W) : S_W) : 0.f;
                 // the layer's bias, when the packed weight holds one, joins P' once per cube
                 const float* bias =
                     (reinterpret_cast<const PackedHeader*>(p.packed_w)->flags & kPackedHasBias) ? p.bias + c_base

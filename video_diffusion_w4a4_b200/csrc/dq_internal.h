@@ -19,6 +19,7 @@ struct QuantParams {
     int n_boxes;
     int m_rows;         // kernel tokens per box (rows of the encode kernel's per-stage tile)
     int stat_pairs;     // statistics kernel: one warp per cube, a channel pair per lane (cubes of 16+ tokens)
+    int kgroup;         // 0: s8 per kernel token (K); 64: per 64 channels (K x Ci/64), q8_bf16 = [hi | lo]
     int big;            // cubes of more than 128 tokens: boxes are row segments of one cube,
     int nseg;           //   nseg segments of up to 128 tokens per cube row; the kernel tokens
     float* means;       //   K x Ci fp32 kernel tokens: written by k_cube_stats (by k_cube_means_big for big cubes)
@@ -43,10 +44,11 @@ struct GemmParams {
     int Ci;
     int k_stages;        // main-operand K stages
     int slab_stages;     // extra BF16 K stages (low-rank slab), main product only
+    int b_kblocks;       // kernel-token product: B k-blocks (Ci/64); A k-block i reads B k-block i mod this
     const float* p;      // per-cube kernel term, K x Co fp32 (main product)
     const uint32_t* scalars;
     const uint8_t* packed_w;
-    const float* s8;     // kernel-token scales (kernel-token product)
+    const float* s8;     // per-row kernel-token scales (kernel-token product); null when A carries them
     float* pout;         // kernel-token product output, K x Co fp32
     const float* bias;   // Co fp32 bias section of the packed weight (read when its flag is set)
     uint16_t* Y;         // main product output, N x Co BF16 (t,h,w) order

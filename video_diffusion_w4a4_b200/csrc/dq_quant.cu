@@ -731,7 +731,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
             // very small cubes have, are formed where they are used)
             const int q_first = lane + 8 * j_own;
             float s8_first = 0.f;
-            if (q_first < W.ncub * 8) {
+            if (!p.kgroup && q_first < W.ncub * 8) {
                 const long long k = R.k0 + W.j_lo + (q_first >> 3);
                 s8_first = __fdiv_rn(__uint_as_float(p.kamax[k]), 448.f);
                 if (split == 0 && (q_first & 7) == 0) p.s8[k] = s8_first;
@@ -744,17 +744,33 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                 const uint8_t* xs = sm + L.x + s * L.x_stride;
                 const float* mt = (const float*)(sm + L.mt + s * L.mt_stride);
                 const int c0 = c_base + i * 64;
-                // kernel tokens: FP8 E4M3 codes under s8 = max|mean| / 448, and their exact BF16 copy
+                // kernel tokens: FP8 E4M3 codes under s8 = max|mean| / 448 (over the token, or over
+                // this stage's 64 channels), and their BF16 form for the kernel-token product
                 for (int q = q_first; q < W.ncub * 8; q += 32) {
                     const int jj = q >> 3, g8 = q & 7;
                     const long long k = R.k0 + W.j_lo + jj;
+                    uint64_t m[4];
+                    load8(mt + (W.j_lo + jj) * 64 + 8 * g8, m);
                     float s8 = s8_first;
-                    if (q != q_first) {
+                    if (p.kgroup) {
+                        // the cube's 64 channels of this stage are held by eight consecutive lanes
+                        float a = 0.f;
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            float lo, hi;
+                            f2_unpack(m[e], lo, hi);
+                            a = fmaxf(a, fmaxf(fabsf(lo), fabsf(hi)));
+                        }
+                        const uint32_t gm = 0xFFu << (lane & 24);
+                        a = fmaxf(a, __shfl_xor_sync(gm, a, 1));
+                        a = fmaxf(a, __shfl_xor_sync(gm, a, 2));
+                        a = fmaxf(a, __shfl_xor_sync(gm, a, 4));
+                        s8 = __fdiv_rn(a, 448.f);
+                        if (g8 == 0) p.s8[k * (Ci / 64) + (c0 >> 6)] = s8;
+                    } else if (q != q_first) {
                         s8 = __fdiv_rn(__uint_as_float(p.kamax[k]), 448.f);
                         if (split == 0 && i == 0 && g8 == 0) p.s8[k] = s8;
                     }
-                    uint64_t m[4];
-                    load8(mt + (W.j_lo + jj) * 64 + 8 * g8, m);
                     uint32_t c[4] = {0u, 0u, 0u, 0u};
                     if (s8 != 0.f) {
                         // codes of the negated quotients with the sign bit of each byte flipped
@@ -770,13 +786,32 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                     }
                     *reinterpret_cast<uint2*>(p.q8 + (size_t)k * Ci + c0 + 8 * g8) =
                         make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
-                    uint32_t bfw[4];
+                    if (p.kgroup) {
+                        // q8 s8 as BF16 hi + lo: hi in columns [0, Ci), lo in [Ci, 2 Ci) of row k
+                        uint32_t hw[4], lw[4];
 #pragma unroll
-                    for (int e = 0; e < 4; e++)
-                        bfw[e] = (uint32_t)f32_to_bf16_rn(e4m3_to_f32(c[e] & 0xFF)) |
-                                 ((uint32_t)f32_to_bf16_rn(e4m3_to_f32(c[e] >> 8)) << 16);
-                    *reinterpret_cast<uint4*>(p.q8_bf16 + (size_t)k * Ci + c0 + 8 * g8) =
-                        make_uint4(bfw[0], bfw[1], bfw[2], bfw[3]);
+                        for (int e = 0; e < 4; e++) {
+                            const float v0 = __fmul_rn(e4m3_to_f32(c[e] & 0xFF), s8);
+                            const float v1 = __fmul_rn(e4m3_to_f32(c[e] >> 8), s8);
+                            const uint16_t h0 = f32_to_bf16_rn(v0), h1 = f32_to_bf16_rn(v1);
+                            const uint16_t l0 = f32_to_bf16_rn(__fsub_rn(v0, __uint_as_float((uint32_t)h0 << 16)));
+                            const uint16_t l1 = f32_to_bf16_rn(__fsub_rn(v1, __uint_as_float((uint32_t)h1 << 16)));
+                            hw[e] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                            lw[e] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+                        }
+                        uint16_t* arow = p.q8_bf16 + (size_t)k * (2 * Ci) + c0 + 8 * g8;
+                        *reinterpret_cast<uint4*>(arow) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                        *reinterpret_cast<uint4*>(arow + Ci) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                    } else {
+                        // exact: E4M3 values have four significant bits
+                        uint32_t bfw[4];
+#pragma unroll
+                        for (int e = 0; e < 4; e++)
+                            bfw[e] = (uint32_t)f32_to_bf16_rn(e4m3_to_f32(c[e] & 0xFF)) |
+                                     ((uint32_t)f32_to_bf16_rn(e4m3_to_f32(c[e] >> 8)) << 16);
+                        *reinterpret_cast<uint4*>(p.q8_bf16 + (size_t)k * Ci + c0 + 8 * g8) =
+                            make_uint4(bfw[0], bfw[1], bfw[2], bfw[3]);
+                    }
                 }
                 // delta tokens: FP4 E2M1 with E4M3 group-16 scales under S (two groups per lane)
                 if (has_row) {
