@@ -449,6 +449,20 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
     return __half2float(__half(hr));
 }
 
+// Two E4M3 codes (the low byte of `codes` first) -> their values as a BF16 pair
+// (low code in the low half).  Exact: E4M3 values have at most four significant
+// bits and lie in BF16's range; f16 holds them exactly on the way.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t codes) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)(codes & 0xFFFFu)));
+    __half_raw lo, hi;
+    lo.x = (uint16_t)(h2 & 0xFFFFu);
+    hi.x = (uint16_t)(h2 >> 16);
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__half2float(__half(hi))), "f"(__half2float(__half(lo))));
+    return r;
+}
+
 // fl32(a / b) for b > 0 from rb = fl32(1 / b): one product and one FMA
 // correction step (Markstein), which returns the correctly rounded quotient
 // when rb is the correctly rounded reciprocal; the result takes a's sign, as

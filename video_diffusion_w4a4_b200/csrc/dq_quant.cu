@@ -220,9 +220,12 @@ __device__ __forceinline__ WarpRows warp_rows(const BoxRows& R, int warp) {
     return W;
 }
 
+// 1 / cnt for a power of two cnt, exactly (the exponent field of 2^-log2(cnt))
+__device__ __forceinline__ float inv_pow2(int cnt) { return __int_as_float((127 - (31 - __clz(cnt))) << 23); }
+
 __device__ __forceinline__ void mean_from_sum(const uint64_t (&acc)[4], int cnt, uint64_t (&m)[4]) {
     if ((cnt & (cnt - 1)) == 0) {
-        const float inv = __frcp_rn((float)cnt);
+        const float inv = inv_pow2(cnt);
         const uint64_t inv2 = f2_pack(inv, inv);
 #pragma unroll
         for (int e = 0; e < 4; e++) m[e] = f2_mul(acc[e], inv2);
@@ -478,7 +481,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                         float a0, a1, m0, m1;
                         f2_unpack(acc, a0, a1);
                         if ((cnt & (cnt - 1)) == 0) {
-                            const float inv = __frcp_rn((float)cnt);
+                            const float inv = inv_pow2(cnt);
                             m0 = __fmul_rn(a0, inv);
                             m1 = __fmul_rn(a1, inv);
                         } else {
@@ -730,10 +733,11 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
             // s8 = max|mean| / 448 of the first kernel-token task of this lane (others, which only
             // very small cubes have, are formed where they are used)
             const int q_first = lane + 8 * j_own;
-            float s8_first = 0.f;
+            float s8_first = 0.f, rs8_first = 0.f;
             if (!p.kgroup && q_first < W.ncub * 8) {
                 const long long k = R.k0 + W.j_lo + (q_first >> 3);
                 s8_first = __fdiv_rn(__uint_as_float(p.kamax[k]), 448.f);
+                rs8_first = (s8_first != 0.f) ? __frcp_rn(s8_first) : 0.f;
                 if (split == 0 && (q_first & 7) == 0) p.s8[k] = s8_first;
             }
             for (int i = 0; i < nchunks; i++, g++) {
@@ -751,7 +755,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                     const long long k = R.k0 + W.j_lo + jj;
                     uint64_t m[4];
                     load8(mt + (W.j_lo + jj) * 64 + 8 * g8, m);
-                    float s8 = s8_first;
+                    float s8 = s8_first, rs8 = rs8_first;
                     if (p.kgroup) {
                         // the cube's 64 channels of this stage are held by eight consecutive lanes
                         float a = 0.f;
@@ -766,16 +770,17 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                         a = fmaxf(a, __shfl_xor_sync(gm, a, 2));
                         a = fmaxf(a, __shfl_xor_sync(gm, a, 4));
                         s8 = __fdiv_rn(a, 448.f);
+                        rs8 = (s8 != 0.f) ? __frcp_rn(s8) : 0.f;
                         if (g8 == 0) p.s8[k * (Ci / 64) + (c0 >> 6)] = s8;
                     } else if (q != q_first) {
                         s8 = __fdiv_rn(__uint_as_float(p.kamax[k]), 448.f);
+                        rs8 = (s8 != 0.f) ? __frcp_rn(s8) : 0.f;
                         if (split == 0 && i == 0 && g8 == 0) p.s8[k] = s8;
                     }
                     uint32_t c[4] = {0u, 0u, 0u, 0u};
                     if (s8 != 0.f) {
                         // codes of the negated quotients with the sign bit of each byte flipped
                         // (E4M3 is sign-magnitude, saturation symmetric)
-                        const float rs8 = __frcp_rn(s8);
                         const uint64_t b2 = f2_pack(s8, s8), nrb2 = f2_pack(-rs8, -rs8);
 #pragma unroll
                         for (int e = 0; e < 4; e++) {
@@ -806,9 +811,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                         // exact: E4M3 values have four significant bits
                         uint32_t bfw[4];
 #pragma unroll
-                        for (int e = 0; e < 4; e++)
-                            bfw[e] = (uint32_t)f32_to_bf16_rn(e4m3_to_f32(c[e] & 0xFF)) |
-                                     ((uint32_t)f32_to_bf16_rn(e4m3_to_f32(c[e] >> 8)) << 16);
+                        for (int e = 0; e < 4; e++) bfw[e] = e4m3x2_to_bf16x2(c[e]);
                         *reinterpret_cast<uint4*>(p.q8_bf16 + (size_t)k * Ci + c0 + 8 * g8) =
                             make_uint4(bfw[0], bfw[1], bfw[2], bfw[3]);
                     }
