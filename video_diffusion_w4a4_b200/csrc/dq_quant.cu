@@ -450,6 +450,11 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
             const BoxRows R = box_rows(p, B);
             const StatTask T0 = stat_task(p, R, tid);
             float kam[4] = {0.f, 0.f, 0.f, 0.f};   // max |mean| of this thread's cube tasks
+            // channel-pair mode: with fewer cubes than warps, the warps form kQWarps / nv groups
+            // that take turns over the chunks, so that several stages of the ring are worked on at once
+            const int ngrp = kPairs ? kQWarps / R.nv : 1;
+            const int grp = kPairs ? warp / R.nv : 0, u_pair = kPairs ? warp - grp * R.nv : 0;
+            int phase = 0;
             for (int i = 0; i < nchunks; i++, g++) {
                 const int s = (int)(g % kQStages);
                 ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)(g / kQStages) & 1, abort_flag, p.status,
@@ -459,9 +464,11 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                 const int c0 = c_base + i * 64;
                 if (kPairs) {
                     // cubes of 16 or more tokens (at most 8 per box): warp = cube slot, lane = channel
-                    // pair (2 lane, 2 lane + 1), so that every cube of the box keeps a warp busy
-                    if (warp < R.nv) {
-                        const int u = warp;
+                    // pair (2 lane, 2 lane + 1)
+                    const bool mine = grp < ngrp && phase == grp;
+                    if (++phase == ngrp) phase = 0;
+                    if (mine) {
+                        const int u = u_pair;
                         const int sw = (u == R.nv - 1) ? R.sw_last : p.g.w;
                         uint64_t acc = 0ull;                          // (+0, +0)
                         uint32_t hi = 0xFF80FF80u, lo = 0x7F807F80u;  // BF16 -inf / +inf pairs
@@ -574,7 +581,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
             // or a whole warp in the channel-pair mode
             if (kPairs) {
                 const float v = warp_max(kam[0]);
-                if (lane == 0 && warp < R.nv) atomicMax(&p.kamax[R.k0 + warp], __float_as_uint(v));
+                if (lane == 0 && grp < ngrp) atomicMax(&p.kamax[R.k0 + u_pair], __float_as_uint(v));
             } else if (!p.big) {
 #pragma unroll
                 for (int t = 0; t < 4; t++) {
