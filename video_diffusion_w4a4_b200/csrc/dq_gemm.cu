@@ -59,7 +59,7 @@ constexpr uint32_t kSFABytes = 2 * 4096;        // 128 rows x 4 k-blocks of 64, 
 constexpr uint32_t kSFBBytes = 4 * 4096;        // all 256 columns x 4 k-blocks, B-operand scale layout (each CTA)
 constexpr uint16_t kPairMask = 0x3;
 
-__host__ __device__ constexpr int g_stages(bool scaled) { return scaled ? 4 : 6; }
+__host__ __device__ constexpr int g_stages(bool scaled) { return scaled ? 4 : 7; }
 
 struct GSmem {
     uint32_t a, b, sfa, sfb, bars, misc, total;
