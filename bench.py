@@ -58,6 +58,22 @@ def stage_model(wl, K, slab, kernel_group=0):
                 main_gemm=dict(bytes=main_bytes, flops=main_flops))
 
 
+def max_over_ranks(x, dist=None, device="cpu"):
+    """The largest of every rank's `x` (one all-reduce that every rank takes part in);
+    `x` itself with no process group."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank_step, world, ms_max):
+    """Whole-job throughput under weak scaling: every rank's FLOPs over the slowest rank's step time."""
+    return flops_per_rank_step * world / (ms_max * 1e-3) / 1e12
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -303,10 +319,7 @@ def main():
     status = dq.dq_read_device_status(ws, st, clear=True)
     if status != 0:
         raise RuntimeError(f"device status after timing: {dq.dq_status_string(status)}")
-    if dist:
-        tm = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        ms = float(tm.item())
+    ms = max_over_ranks(ms, dist, dev)
 
     # end to end through the host-buffer entry point: pinned X in, Y out, copies inside the timed region
     Xh = torch.from_numpy(X.view(np.int16)).pin_memory()
@@ -331,13 +344,11 @@ def main():
         torch.cuda.synchronize(dev)
         e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
     if dist and e2e_ms is not None:
-        tm = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tm.item())
+        e2e_ms = max_over_ranks(e2e_ms, dist, dev)
         dist.barrier()
 
     F = layer_flops(wl, K)
-    value = F * world / (ms * 1e-3) / 1e12
+    value = job_tflops(F, world, ms)
     peaks = load_peaks()
     fp4_peak = peaks["bf16"] * FP4_PER_BF16
     model = stage_model(wl, K, lay.slab, kg)
@@ -376,7 +387,7 @@ def main():
                 layer_roofline_frac=layer_roof_ms / ms,
                 roofline=roof, stages=stages,
                 e2e=None if e2e_ms is None else dict(
-                    value=F * world / (e2e_ms * 1e-3) / 1e12, unit="TFLOP/s", h2d_bytes_per_step=wl.N * wl.Ci * 2,
+                    value=job_tflops(F, world, e2e_ms), unit="TFLOP/s", h2d_bytes_per_step=wl.N * wl.Ci * 2,
                     d2h_bytes_per_step=wl.N * wl.Co * 2, ms_per_step=e2e_ms),
                 gpu_launches=(5 if t * h * w > 128 else 4) * args.steps, pack_seconds=pack_s)
     clk_sum = clk.summary()

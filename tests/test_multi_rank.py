@@ -1,0 +1,77 @@
+"""The multi-process (one rank per GPU) plumbing of bench.py, on CPU: two gloo
+ranks agree on the slowest rank's step time and the whole-job throughput, and
+under a two-rank launch the reference arm runs and prints on rank 0 only."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        local_ms = [1.5, 2.5][rank]
+        dist.barrier()
+        ms = bench.max_over_ranks(local_ms, dist)
+        value = bench.job_tflops(1.0e12, world, ms)
+        out.put((rank, ms, value))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_slowest_step():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.SimpleQueue()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get() for _ in range(world))
+    assert [r[1] for r in res] == [2.5, 2.5]
+    # 2 ranks x 1 TFLOP each over the slowest rank's 2.5 ms
+    assert all(abs(r[2] - 2 * 1.0 / 2.5e-3) < 1e-9 for r in res)
+
+
+def test_single_process_reduction_is_the_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.25) == 3.25
+    assert bench.job_tflops(2.0e12, 1, 4.0) == pytest.approx(500.0)
+
+
+@pytest.mark.parametrize("rank", [0, 1])
+def test_reference_arm_prints_on_rank_zero_only(rank):
+    env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank))
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "3", "--sample-tokens", "16"],
+                       env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    if rank:
+        assert lines == []
+    else:
+        d = json.loads(lines[-1])
+        assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+        assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
