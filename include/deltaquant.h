@@ -273,6 +273,16 @@ int dq_workspace_bytes_grouped(int T, int H, int W, int t, int h, int w, int Ci,
 #define DQ_STAGE_KERNEL_GEMM 2 /* kernel-token product P (kernel c) */
 #define DQ_STAGE_MAIN_GEMM 4   /* block-scaled FP4 product + low-rank slab + epilogue (kernel b) */
 #define DQ_STAGE_ALL 7
+/*
+ * The two halves of DQ_STAGE_QUANTIZE, for a layer sharded by cubes across
+ * devices: after DQ_STAGE_STATS the workspace's scalars[0] holds this shard's
+ * max |delta| (fp32 bits, non-negative); the caller replaces it with the
+ * maximum over all shards (one all-reduce) before DQ_STAGE_ENCODE, which
+ * derives S_delta from it.  Shards are slabs of whole cubes along T; every
+ * other quantity of the layer is local to a cube.
+ */
+#define DQ_STAGE_STATS 8       /* a1: cube means, max |mean| per cube, max |delta|, X L1 partial sums */
+#define DQ_STAGE_ENCODE 16     /* a2: FP8 kernel tokens, FP4 delta codes and scales, U' hi + lo */
 
 /*
  * Y = DeltaQuant linear layer of X (see top of file), on `stream`.

@@ -148,4 +148,4 @@ def test_argument_checks_before_any_launch(dq):
     assert call(Y=0x50008) == dq.DQ_ERR_ALIGNMENT
     assert call(ws_bytes=ws) == dq.DQ_ERR_WORKSPACE_TOO_SMALL
     assert dq._lib.dq_linear_forward_ex(0x10000, 4, 8, 8, 1, 2, 2, 256, 256, 16, 0x20000, 0x30000, 0x40000, 0x50000,
-                                        0x60000, 1 << 40, 9, None, None) == dq.DQ_ERR_INVALID_ARG
+                                        0x60000, 1 << 40, 32, None, None) == dq.DQ_ERR_INVALID_ARG   # unknown stage bit

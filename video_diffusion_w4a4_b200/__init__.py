@@ -34,6 +34,7 @@ DQ_ERR_BAD_PACKED_WEIGHT = 7
 DQ_ERR_NO_DEVICE = 8
 DQ_ERR_ALLOC = 9
 DQ_STAGE_QUANTIZE, DQ_STAGE_KERNEL_GEMM, DQ_STAGE_MAIN_GEMM, DQ_STAGE_ALL = 1, 2, 4, 7
+DQ_STAGE_STATS, DQ_STAGE_ENCODE = 8, 16
 DQ_KERNEL_SCALE_PER_TOKEN, DQ_KERNEL_SCALE_GROUP64 = 0, 64
 
 

@@ -229,7 +229,9 @@ int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, 
     if (kernel_group != DQ_KERNEL_SCALE_PER_TOKEN && kernel_group != DQ_KERNEL_SCALE_GROUP64) return DQ_ERR_INVALID_ARG;
     const int kg = kernel_group;
     if (!X || !packed_W || !L1_mma || !L2_slab || !Y || !workspace) return DQ_ERR_INVALID_ARG;
-    if (stage_mask <= 0 || stage_mask > DQ_STAGE_ALL) return DQ_ERR_INVALID_ARG;
+    if (stage_mask <= 0 || (stage_mask & ~(DQ_STAGE_ALL | DQ_STAGE_STATS | DQ_STAGE_ENCODE))) return DQ_ERR_INVALID_ARG;
+    const bool do_stats = stage_mask & (DQ_STAGE_QUANTIZE | DQ_STAGE_STATS);
+    const bool do_encode = stage_mask & (DQ_STAGE_QUANTIZE | DQ_STAGE_ENCODE);
     if (!aligned(X) || !aligned(packed_W) || !aligned(L1_mma) || !aligned(L2_slab) || !aligned(Y) ||
         !aligned(workspace))
         return DQ_ERR_ALIGNMENT;
@@ -303,18 +305,23 @@ int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, 
         if (stage_events && stage_events[i]) cudaEventRecord((cudaEvent_t)stage_events[i], st);
     };
     rec(0);
-    if (stage_mask & DQ_STAGE_QUANTIZE) {
+    if (do_stats || do_encode) {
         CUtensorMap tm_x, tm_l1, tm_m;
         cudaError_t e0;
         if (!map_x(&tm_x, X, g, Ci, qp.bw, qp.bh, qp.bt)) return map_fail("X");
         if (!map_means(&tm_m, ws + wl.off_means, Ci, g.K, qp.m_rows)) return map_fail("kernel tokens");
         if (!map_2d(&tm_l1, L1_mma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, rank, 64, rank)) return map_fail("L1");
-        if ((e0 = cudaMemsetAsync(ws + wl.off_scalars, 0, 16, st)) != cudaSuccess) return cuda_fail(e0, "memset");
-        if ((e0 = cudaMemsetAsync(ws + wl.off_kamax, 0, (size_t)g.K * 4, st)) != cudaSuccess) return cuda_fail(e0, "memset");
         cudaError_t e;
-        if (qp.big && (e = dq::launch_cube_means_big(tm_x, qp, st)) != cudaSuccess) return cuda_fail(e, "k_cube_means_big");
-        if ((e = dq::launch_cube_stats(tm_x, tm_l1, qp, st)) != cudaSuccess) return cuda_fail(e, "k_cube_stats");
-        if ((e = dq::launch_cube_encode(tm_x, tm_m, qp, st)) != cudaSuccess) return cuda_fail(e, "k_cube_encode");
+        if (do_stats) {
+            if ((e0 = cudaMemsetAsync(ws + wl.off_scalars, 0, 16, st)) != cudaSuccess) return cuda_fail(e0, "memset");
+            if ((e0 = cudaMemsetAsync(ws + wl.off_kamax, 0, (size_t)g.K * 4, st)) != cudaSuccess)
+                return cuda_fail(e0, "memset");
+            if (qp.big && (e = dq::launch_cube_means_big(tm_x, qp, st)) != cudaSuccess)
+                return cuda_fail(e, "k_cube_means_big");
+            if ((e = dq::launch_cube_stats(tm_x, tm_l1, qp, st)) != cudaSuccess) return cuda_fail(e, "k_cube_stats");
+        }
+        if (do_encode && (e = dq::launch_cube_encode(tm_x, tm_m, qp, st)) != cudaSuccess)
+            return cuda_fail(e, "k_cube_encode");
     }
     rec(1);
     if (stage_mask & DQ_STAGE_KERNEL_GEMM) {
