@@ -92,16 +92,19 @@ def test_two_ranks_exchange_only_the_largest_delta():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("name,slabs", [("ragged_122", 2), ("cube_414_r128", 3), ("ragged_222", 2)])
+@pytest.mark.parametrize("name,slabs", [("ragged_122", 2), ("cube_414_r128", 3), ("ragged_222", 2),
+                                        ("wan480p_proj", 3)])
 def test_sharded_equals_unsharded_on_one_gpu(name, slabs):
     """The slabs run one after the other on one GPU, the host taking the maximum that the
-    all-reduce would: Y of every row bit-identical to the unsharded layer."""
+    all-reduce would: Y of every row bit-identical to the unsharded layer (small ragged
+    lattices, and the 480p projection in three slabs of 7 frames)."""
     import torch
     sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import synth
     import video_diffusion_w4a4_b200 as dq
     from dq_case import Case
     from test_gpu_parity import SMALL
-    wl = dict(SMALL)[name]
+    wl = dict(SMALL).get(name) or synth.WORKLOADS[name]
     case = Case(wl)
     full = case.run_gpu(dq, torch)
     t, h, w = case.cube
