@@ -88,6 +88,17 @@ def test_cube_sweep(env, cube):
     rel = lambda y: float(np.linalg.norm(y - exact) / np.linalg.norm(exact))
     info.update(cube=list(cube), rel_err_gpu=rel(bf16_bits_to_f64(g["Y"][rows])), rel_err_oracle=rel(y_ref),
                 rel_err_plain_nvfp4=rel(y_plain))
+    # the same 512 seeded token rows for every cube, so that the errors compare across cube sizes
+    fixed = np.sort(np.random.default_rng(2026).choice(wl.N, size=512, replace=False))
+    xf = oracle.bf16_value(case.X[fixed]).astype(np.float64)
+    exact_f = xf @ w.T
+    relf = lambda y: float(np.linalg.norm(y - exact_f) / np.linalg.norm(exact_f))
+    plain_f = oracle.quantize_plain(case.X[fixed])
+    plain_f.update(row_of_n=None, cube_of_n=None, q8=None, s8=None)
+    y_plain_f = oracle.output_rows(plain_f, wq, case.X[fixed], case.L1, case.L2, np.arange(fixed.size), kernel=False,
+                                   cube_major=False)
+    info.update(fixed_rows=int(fixed.size), rel_err_gpu_fixed=relf(bf16_bits_to_f64(g["Y"][fixed])),
+                rel_err_plain_nvfp4_fixed=relf(y_plain_f))
     _record("sweep_%d%d%d" % cube, info)
     if cube not in ((1, 1, 1), (21, 30, 52)):
         # local cubes beat plain FP4 (the note's cube-size ablation: the global kernel loses the local structure)
