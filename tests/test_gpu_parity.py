@@ -12,7 +12,7 @@ import pytest
 
 import oracle
 import synth
-from dq_case import Case, assert_y_close, bf16_bits_to_f64, compare_quantised
+from dq_case import Case, assert_y_close, compare_quantised
 
 pytestmark = pytest.mark.gpu
 
