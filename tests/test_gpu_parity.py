@@ -91,14 +91,16 @@ def test_parity_small(env, name, wl):
     assert_y_close(g["Y"], y_ref)
 
 
-@pytest.mark.parametrize("name", ["ragged_122", "unit_cube", "global"])
-def test_parity_bias(env, name):
+@pytest.mark.parametrize("name,kernel_group", [("ragged_122", 0), ("unit_cube", 0), ("global", 0),
+                                                ("ragged_122", 64), ("cube_428", 64)])
+def test_parity_bias(env, name, kernel_group):
     """A bias in the packed weight: every quantised tensor unchanged and bit-exact,
     Y = the oracle's x W^T + b within tolerance, for a ragged lattice, the
-    one-token cube (P' per token) and the whole-lattice cube (one P' row)."""
+    one-token cube (P' per token), the whole-lattice cube (one P' row), and with
+    group-64 kernel scales (P' without a per-row scale)."""
     dq, torch = env
     wl = dict(SMALL)[name]
-    case = Case(wl)
+    case = Case(wl, kernel_group=kernel_group)
     b = synth.normal_bf16((wl.Co,), sd=4.0, seed=21)
     g = case.run_gpu(dq, torch, bias=b)
     act, wq = case.run_oracle()
