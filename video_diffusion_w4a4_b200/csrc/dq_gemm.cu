@@ -61,6 +61,24 @@ constexpr uint16_t kPairMask = 0x3;
 
 __host__ __device__ constexpr int g_stages(bool scaled) { return scaled ? 4 : 7; }
 
+// Output tile -> (row tile, column tile).  The main product walks row-major (its weight codes and
+// scales, 39 MB, stay in L2 while the row tiles stream).  The kernel-token product's BF16 weight
+// (Co x Ci x 2 bytes) does not stay in L2 next to the streaming rows, so it walks groups of 8 row
+// tiles column by column: a wave of CTA pairs then touches 8 row tiles and a few column tiles, and
+// each group reads the weight once.
+struct TileRC {
+    int m, n;
+};
+
+template <bool kMain>
+__device__ __forceinline__ TileRC tile_rc(int tile, int num_m, int num_n) {
+    if (kMain) return TileRC{tile / num_n, tile % num_n};
+    constexpr int kGroup = 8;
+    const int grp = tile / (kGroup * num_n), in = tile - grp * (kGroup * num_n);
+    const int gm = min(kGroup, num_m - grp * kGroup);
+    return TileRC{grp * kGroup + in % gm, in / gm};
+}
+
 struct GSmem {
     uint32_t a, b, sfa, sfb, bars, misc, total;
 };
@@ -113,7 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool lead = rank == 0;
     const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
     const int num_n = p.Nout / kTileN;
-    const int num_tiles = (int)cdiv(p.M, 2 * kTileM) * num_n;
+    const int num_m = (int)cdiv(p.M, 2 * kTileM);
+    const int num_tiles = num_m * num_n;
     const int nk = p.k_stages, ntot = p.k_stages + p.slab_stages;
 
     if (tid == 0) {
@@ -157,8 +176,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             long long g = 0;
             bool alive = true;
             for (int tile = pair; alive && tile < num_tiles; tile += npairs) {
-                const int m0 = (tile / num_n) * (2 * kTileM) + (int)rank * kTileM;   // this CTA's A rows
-                const int n0 = (tile % num_n) * kTileN;                               // the pair's columns
+                const TileRC rc = tile_rc<kMain>(tile, num_m, num_n);
+                const int m0 = rc.m * (2 * kTileM) + (int)rank * kTileM;   // this CTA's A rows
+                const int n0 = rc.n * kTileN;                               // the pair's columns
                 const int nb = n0 + (int)rank * (kTileN / 2);                         // this CTA's B rows
                 for (int i = 0; i < ntot; i++, g++) {
                     const int s = (int)(g % S);
@@ -298,8 +318,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int it = 0;
         for (int tile = pair; tile < num_tiles; tile += npairs, it++) {
             const int buf = it % kBufs, use = it / kBufs;
-            const int m0 = (tile / num_n) * (2 * kTileM) + (int)rank * kTileM;
-            const int n0 = (tile % num_n) * kTileN;
+            const TileRC rc = tile_rc<kMain>(tile, num_m, num_n);
+            const int m0 = rc.m * (2 * kTileM) + (int)rank * kTileM;
+            const int n0 = rc.n * kTileN;
             const long long rho = (long long)m0 + quad * 32 + lane;
             const bool row_ok = rho < p.M;
             const int c_base = n0 + half * 128;
