@@ -334,6 +334,7 @@ int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, 
         p.M = (int)g.K;
         p.k_stages = a_cols / 64;
         p.b_kblocks = Ci / 64;
+        p.tile_group = 8;   // the BF16 weight (Co x Ci x 2 bytes) does not stay in L2 beside the rows
         p.s8 = kg ? nullptr : qp.s8;
         p.pout = (float*)(ws + wl.off_p);
         p.bias = (const float*)(pw + pl.off_bias);
@@ -356,6 +357,9 @@ int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, 
         p.M = (int)g.N;
         p.k_stages = Ci / 256;
         p.slab_stages = wl.slab / 64;
+        // weight codes and scales above 32 MB (the 720p FFN layers) are re-read by every wave of a
+        // row-major walk; up to that size (the 480p projection, 20 MB) they stay in L2 and row-major wins
+        p.tile_group = ((size_t)Co * (Ci / 2) + pl.off_dqw - pl.off_scales > ((size_t)32 << 20)) ? 8 : 1;
         p.p = (const float*)(ws + wl.off_p);
         p.Y = (uint16_t*)Y;
         cudaError_t e = dq::launch_main_gemm(tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p, st);

@@ -61,22 +61,19 @@ constexpr uint16_t kPairMask = 0x3;
 
 __host__ __device__ constexpr int g_stages(bool scaled) { return scaled ? 4 : 7; }
 
-// Output tile -> (row tile, column tile).  The main product walks row-major (its weight codes and
-// scales, 39 MB, stay in L2 while the row tiles stream).  The kernel-token product's BF16 weight
-// (Co x Ci x 2 bytes) does not stay in L2 next to the streaming rows, so it walks groups of 8 row
-// tiles column by column: a wave of CTA pairs then touches 8 row tiles and a few column tiles, and
-// each group reads the weight once.
+// Output tile -> (row tile, column tile).  group <= 1: row-major, which suits a weight that stays
+// in L2 while the row tiles stream.  Otherwise groups of `group` row tiles walked column by column:
+// a wave of CTA pairs then touches `group` row tiles and a few column tiles, and each group reads
+// the weight once (the host picks this for weights too large to stay in L2 beside the rows).
 struct TileRC {
     int m, n;
 };
 
-template <bool kMain>
-__device__ __forceinline__ TileRC tile_rc(int tile, int num_m, int num_n) {
-    if (kMain) return TileRC{tile / num_n, tile % num_n};
-    constexpr int kGroup = 8;
-    const int grp = tile / (kGroup * num_n), in = tile - grp * (kGroup * num_n);
-    const int gm = min(kGroup, num_m - grp * kGroup);
-    return TileRC{grp * kGroup + in % gm, in / gm};
+__device__ __forceinline__ TileRC tile_rc(int tile, int num_m, int num_n, int group) {
+    if (group <= 1) return TileRC{tile / num_n, tile % num_n};
+    const int grp = tile / (group * num_n), in = tile - grp * (group * num_n);
+    const int gm = min(group, num_m - grp * group);
+    return TileRC{grp * group + in % gm, in / gm};
 }
 
 struct GSmem {
@@ -176,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             long long g = 0;
             bool alive = true;
             for (int tile = pair; alive && tile < num_tiles; tile += npairs) {
-                const TileRC rc = tile_rc<kMain>(tile, num_m, num_n);
+                const TileRC rc = tile_rc(tile, num_m, num_n, p.tile_group);
                 const int m0 = rc.m * (2 * kTileM) + (int)rank * kTileM;   // this CTA's A rows
                 const int n0 = rc.n * kTileN;                               // the pair's columns
                 const int nb = n0 + (int)rank * (kTileN / 2);                         // this CTA's B rows
@@ -318,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int it = 0;
         for (int tile = pair; tile < num_tiles; tile += npairs, it++) {
             const int buf = it % kBufs, use = it / kBufs;
-            const TileRC rc = tile_rc<kMain>(tile, num_m, num_n);
+            const TileRC rc = tile_rc(tile, num_m, num_n, p.tile_group);
             const int m0 = rc.m * (2 * kTileM) + (int)rank * kTileM;
             const int n0 = rc.n * kTileN;
             const long long rho = (long long)m0 + quad * 32 + lane;

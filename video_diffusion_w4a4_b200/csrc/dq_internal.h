@@ -45,6 +45,7 @@ struct GemmParams {
     int k_stages;        // main-operand K stages
     int slab_stages;     // extra BF16 K stages (low-rank slab), main product only
     int b_kblocks;       // kernel-token product: B k-blocks (Ci/64); A k-block i reads B k-block i mod this
+    int tile_group;      // tile order: 1 row-major, else groups of this many row tiles walked column by column
     const float* p;      // per-cube kernel term, K x Co fp32 (main product)
     const uint32_t* scalars;
     const uint8_t* packed_w;
