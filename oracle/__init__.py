@@ -60,6 +60,9 @@ def _L():
         lib.or_tensor_scale.restype = F
         lib.or_fp4_quantize.argtypes = [P, LL, I, F, P, P, P]
         lib.or_quantize_activations.argtypes = [P] + [I] * 7 + [P] * 7
+        lib.or_quantize_activations_opt.argtypes = [P] + [I] * 7 + [P] * 7 + [I]
+        lib.or_pow2_ceil.argtypes = [F]
+        lib.or_pow2_ceil.restype = F
         lib.or_residual.argtypes = [P, P, P, I, I, I, P]
         lib.or_output_rows.argtypes = [P, P, F, P, P, P, I, P, P, P, F, I, I, P, P, P, I, P, LL, P]
         lib.or_fp8_kernel_tokens.argtypes = [P, LL, I, I, P, P]
@@ -179,12 +182,16 @@ def fp8_kernel_tokens(means, group: int):
     return q8, s8
 
 
-def quantize_activations(X, T, H, W, cube, kernel_group: int = 0) -> dict:
+def quantize_activations(X, T, H, W, cube, kernel_group: int = 0, pow2_scales: bool = False) -> dict:
     """Activation side of Eq. 2/3 over the whole X (natural (t,h,w) row order).
 
     kernel_group 0: one FP8 scale per kernel token (s8: K); 64: one per 64
     channels of a kernel token, the note's per-group kernel quantisation
-    (s8: K x Ci/64)."""
+    (s8: K x Ci/64).
+
+    pow2_scales: a power-of-two per-tensor delta scale (the smallest power of two
+    >= amax / 2688), a deviation that lets an encoder fix a block's scale byte up
+    after the fact (see or_quantize_activations_opt)."""
     X = np.ascontiguousarray(X, dtype=np.uint16)
     N, Ci = X.shape
     assert N == T * H * W
@@ -194,14 +201,15 @@ def quantize_activations(X, T, H, W, cube, kernel_group: int = 0) -> dict:
                means=np.empty((K, Ci), np.float32))
     S = ctypes.c_float(0)
     amax = ctypes.c_float(0)
-    rc = _L().or_quantize_activations(_p(X), T, H, W, Ci, *cube, _p(out["dcodes"]), _p(out["dscales"]),
-                                      ctypes.byref(S), _p(out["q8"]), _p(out["s8"]), _p(out["means"]),
-                                      ctypes.byref(amax))
+    rc = _L().or_quantize_activations_opt(_p(X), T, H, W, Ci, *cube, _p(out["dcodes"]), _p(out["dscales"]),
+                                          ctypes.byref(S), _p(out["q8"]), _p(out["s8"]), _p(out["means"]),
+                                          ctypes.byref(amax), int(pow2_scales))
     if rc:
         raise RuntimeError("or_quantize_activations failed")
     out["S_delta"] = float(S.value)
     out["amax_delta"] = float(amax.value)
     out["kernel_group"] = kernel_group
+    out["pow2_scales"] = bool(pow2_scales)
     if kernel_group:
         out["q8"], out["s8"] = fp8_kernel_tokens(out["means"], kernel_group)
     out.update(cube_order(T, H, W, *cube))

@@ -252,6 +252,13 @@ float or_tensor_scale(float amax) {
     return amax / 2688.0f;
 }
 
+/* The smallest power of two >= v (v > 0), exactly: v = m 2^e with m in [0.5, 1). */
+float or_pow2_ceil(float v) {
+    int e;
+    const float m = frexpf(v, &e);
+    return (m == 0.5f) ? v : ldexpf(1.0f, e);
+}
+
 /*
  * One row of FP4 with E4M3 group-16 scales and the per-tensor scale S:
  *   s_b = E4M3(amax_b / (6 S)),  q = E2M1(z / (s_b S))   (Eq. 4 per group).
@@ -312,6 +319,7 @@ static void fp8_token(const float* m, int Ci, uint8_t* q8, float* s8) {
     for (int c = 0; c < Ci; c++) q8[c] = (uint8_t)((s == 0.0f) ? 0 : or_e4m3_encode(m[c] / s));
 }
 
+
 /*
  * FP8 kernel tokens with one scale per `group` consecutive channels (the
  * note's per-group-64 kernel quantisation; group = Ci is one scale per token):
@@ -339,9 +347,28 @@ int or_fp8_kernel_tokens(const float* means, long long K, int Ci, int group, uin
  *   means   K x Ci     fp32 kernel tokens before quantisation (optional)
  *   amax_delta        the global max |delta| (optional)
  */
+/*
+ * As or_quantize_activations, with pow2 != 0 taking a power-of-two per-tensor
+ * delta scale: S = the smallest power of two >= amax / 2688 (1 if amax = 0).
+ * A block encoded under another power-of-two scale then keeps its codes and
+ * only its E4M3 scale's exponent moves (unless that scale leaves E4M3's normal
+ * range): the property a single-read encoder with a scale fix-up pass relies
+ * on.  A deviation from the two-level form of Eq. 4.  The kernel-token scales
+ * keep max |m| / 448, which represents each token's largest element exactly.
+ */
+int or_quantize_activations_opt(const uint16_t* X, int T, int H, int W, int Ci, int t, int h, int w,
+                                uint8_t* dcodes, uint8_t* dscales, float* S_delta, uint8_t* q8, float* s8,
+                                float* means, float* amax_delta, int pow2);
+
 int or_quantize_activations(const uint16_t* X, int T, int H, int W, int Ci, int t, int h, int w,
                             uint8_t* dcodes, uint8_t* dscales, float* S_delta, uint8_t* q8, float* s8,
                             float* means, float* amax_delta) {
+    return or_quantize_activations_opt(X, T, H, W, Ci, t, h, w, dcodes, dscales, S_delta, q8, s8, means, amax_delta, 0);
+}
+
+int or_quantize_activations_opt(const uint16_t* X, int T, int H, int W, int Ci, int t, int h, int w,
+                                uint8_t* dcodes, uint8_t* dscales, float* S_delta, uint8_t* q8, float* s8,
+                                float* means, float* amax_delta, int pow2) {
     if (Ci % 16) return 1;
     geom_t g;
     if (geom_init(&g, T, H, W, t, h, w, Ci)) { geom_free(&g); return 2; }
@@ -363,6 +390,7 @@ int or_quantize_activations(const uint16_t* X, int T, int H, int W, int Ci, int 
         }
     }
     float S = or_tensor_scale(amax);
+    if (pow2 && amax != 0.0f) S = or_pow2_ceil(amax / 2688.0f);
     if (S_delta) *S_delta = S;
     if (amax_delta) *amax_delta = amax;
 

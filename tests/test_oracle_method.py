@@ -456,3 +456,62 @@ def test_group64_kernel_tokens_are_finer(cube):
         ey[kg] = np.linalg.norm(y - ref) / np.linalg.norm(ref)
     assert ek[64] < 0.8 * ek[0], ek
     assert ey[64] <= ey[0], ey
+
+
+# ------------------------------------------------------------------ power-of-two scales (single-read option)
+
+def _is_pow2(v):
+    m, _ = math.frexp(float(v))
+    return v > 0 and m == 0.5
+
+
+def test_pow2_delta_scale_closed_form(tiny_case):
+    """Power-of-two delta scale: S_delta is the smallest power of two >= amax / 2688; the
+    kernel tokens are untouched (their scale keeps max|m| / 448, which maps each token's
+    largest element exactly onto 448)."""
+    wl, X, *_ = tiny_case
+    act = oracle.quantize_activations(X, wl.T, wl.H, wl.W, wl.cube, pow2_scales=True)
+    ref = oracle.quantize_activations(X, wl.T, wl.H, wl.W, wl.cube)
+    S, amax = act["S_delta"], act["amax_delta"]
+    assert _is_pow2(S) and amax / 2688 <= S < amax / 1344
+    assert np.array_equal(act["q8"], ref["q8"]) and np.array_equal(act["s8"], ref["s8"])
+    assert np.array_equal(act["means"], ref["means"])
+
+
+def test_scale_byte_fixup_invariance():
+    """The property a single-read encoder's fix-up pass relies on: encoded under S and
+    under 2^j S (powers of two), a block keeps its E2M1 codes and its E4M3 scale code moves
+    down by j binades (8 j in the code) whenever the shifted scale stays in E4M3's normal
+    range, i.e. the scale's exponent field under S is at least j + 1.  Blocks below that
+    are rounded on the subnormal grid instead: the set that needs re-encoding."""
+    rng = np.random.default_rng(3)
+    Z = (rng.standard_normal((64, 256)) * np.exp(rng.uniform(-12, 6, size=(64, 1)))).astype(np.float32)
+    amax = float(np.abs(Z).max())
+    S = float(oracle._L().or_pow2_ceil(amax / 2688.0))
+    c1, s1, _ = oracle.fp4_quantize(Z, S)
+    normal_blocks = subnormal = 0
+    for j in (1, 2, 5):
+        cj, sj, _ = oracle.fp4_quantize(Z, S * 2.0 ** j)
+        ok = ((s1 >> 3) & 0xF) >= j + 1                           # the shifted scale stays normal
+        assert np.array_equal(sj[ok].astype(int), s1[ok].astype(int) - 8 * j)
+        blocks_ok = np.repeat(ok, 8, axis=1)                      # 8 code bytes per 16-channel block
+        assert np.array_equal(cj[blocks_ok], c1[blocks_ok])
+        normal_blocks += int(ok.sum())
+        subnormal += int((~ok).sum())
+    assert normal_blocks > 0 and subnormal > 0                    # both cases exercised
+
+
+def test_pow2_scales_cost_little_accuracy():
+    """The deviation's cost on correlated activations: the reconstruction error of the
+    deltas with a power-of-two per-tensor scale stays within 2 % of the two-level
+    reading's (the group-16 scales absorb the difference)."""
+    wl = synth.Workload("mid", 4, 16, 16, 512, 384, 16, (1, 2, 2), (4, 4, 4), (0.01, 50.0), (0.01, 20.0))
+    X = synth.activations(wl, seed=77)
+    x = _x_f64(X)
+    err = {}
+    for p2 in (False, True):
+        act = oracle.quantize_activations(X, wl.T, wl.H, wl.W, wl.cube, pow2_scales=p2)
+        dqd = _dequant_rows(act["dcodes"], act["dscales"], act["S_delta"])[act["row_of_n"]]
+        d = x - act["means"].astype(np.float64)[act["cube_of_n"]]
+        err[p2] = np.linalg.norm(dqd - d) / np.linalg.norm(d)
+    assert err[True] < 1.02 * err[False], err
