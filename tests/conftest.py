@@ -7,6 +7,12 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+# Test modules import the package at collection time, and the package refuses to load
+# without its library: build it first when it is missing (a fresh checkout).
+if not os.path.exists(os.path.join(ROOT, "video_diffusion_w4a4_b200", "libdeltaquant.so")):
+    import __graft_entry__
+    __graft_entry__.build()
+
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")

@@ -15,8 +15,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def dq():
-    from video_diffusion_w4a4_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import video_diffusion_w4a4_b200 as m
     return m
 

@@ -14,8 +14,8 @@ import synth
 
 @pytest.fixture(scope="module")
 def dq():
-    from video_diffusion_w4a4_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import video_diffusion_w4a4_b200 as m
     return m
 
