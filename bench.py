@@ -164,16 +164,18 @@ def parse_cube(s):
 # --------------------------------------------------------------------------- reference arm (CPU oracle)
 
 def oracle_sample(wl, cube, X, Wb, L1, L2, wq, ntok):
-    """Oracle over a bounded sample: the first `ntok`-token prefix of whole
-    cube rows (a slab of frames cut at cube boundaries), quantised as its own
-    tensor, then its Y rows.  Returns (seconds, flops of the sample)."""
+    """Oracle over a bounded sample of whole cubes, quantised as its own tensor, then
+    its Y rows: whole cube layers of frames [0, k t) while they fit in `ntok` tokens,
+    else the first cube rows of frames [0, t).  Returns (seconds, flops of the sample,
+    tokens)."""
     import oracle
     t, h, w = cube
-    # rows of whole cube-rows: take frames [0, t) and cube rows until ntok tokens
-    per_cube_row = t * h * wl.W
-    n_rows = max(1, ntok // per_cube_row)
-    Hs = min(wl.H, n_rows * h)
-    Ts = min(wl.T, t)
+    per_layer = t * wl.H * wl.W
+    if ntok >= per_layer:
+        Ts, Hs = min(wl.T, t * (ntok // per_layer)), wl.H
+    else:
+        n_rows = max(1, ntok // (t * h * wl.W))
+        Ts, Hs = min(wl.T, t), min(wl.H, n_rows * h)
     idx = (np.arange(Ts)[:, None, None] * wl.H * wl.W + np.arange(Hs)[None, :, None] * wl.W
            + np.arange(wl.W)[None, None, :]).reshape(-1)
     Xs = np.ascontiguousarray(X[idx])
@@ -236,7 +238,7 @@ def main():
     ap.add_argument("--kernel-group", type=int, default=0, choices=[0, 64],
                     help="FP8 kernel-token scales: 0 = one per token, 64 = one per 64 channels")
     ap.add_argument("--sample-tokens", type=int, default=256, help="oracle sample size per reference step (tokens)")
-    ap.add_argument("--baseline-tokens", type=int, default=4096, help="oracle sample size of the cpu_baseline leg")
+    ap.add_argument("--baseline-tokens", type=int, default=6144, help="oracle sample size of the cpu_baseline leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     args = ap.parse_args()
@@ -400,7 +402,7 @@ def main():
         wq = oracle.quantize_weight(Wb, L1, L2)
         dt, f, n = oracle_sample(wl, cube, X, Wb, L1, L2, wq, args.baseline_tokens)
         line["cpu_baseline"] = dict(value=f / dt / 1e12, unit="TFLOP/s", cores=os.cpu_count(), kind="oracle",
-                                    sample=f"{n} tokens of {wl.name} (whole cube rows, frame slab 0), "
+                                    sample=f"{n} tokens of {wl.name} (whole cubes of the first frames), "
                                            f"Ci={wl.Ci}, Co={wl.Co}, r={wl.rank}, {dt:.1f} s")
     if rank == 0:
         print(json.dumps(line), flush=True)
