@@ -62,6 +62,12 @@ def _L():
         lib.or_quantize_activations.argtypes = [P] + [I] * 7 + [P] * 7
         lib.or_quantize_activations_opt.argtypes = [P] + [I] * 7 + [P] * 7 + [I]
         lib.or_pow2_ceil.argtypes = [F]
+        lib.or_c2_scale_up.argtypes = [F]
+        lib.or_c2_scale_up.restype = F
+        lib.or_fp4_quantize_c2.argtypes = [P, LL, I, P, P, P]
+        lib.or_fp4_quantize_c2.restype = LL
+        lib.or_c2_fp8_operand.argtypes = [P, P, LL, I, P, P]
+        lib.or_c2_fp8_operand.restype = LL
         lib.or_pow2_ceil.restype = F
         lib.or_residual.argtypes = [P, P, P, I, I, I, P]
         lib.or_output_rows.argtypes = [P, P, F, P, P, P, I, P, P, P, F, I, I, P, P, P, I, P, LL, P]
@@ -309,10 +315,41 @@ def residual(Wbits, L1, L2) -> np.ndarray:
     return R
 
 
-def quantize_weight(Wbits, L1, L2) -> dict:
+def quantize_weight(Wbits, L1, L2, c2: bool = False) -> dict:
+    """The residual R = W - L1 L2 in NVFP4 (Eq. 4 per group of 16).  c2: the restricted
+    scale rule of or_fp4_quantize_c2 (an option for an exact FP8-rate kernel-token product)."""
     R = residual(Wbits, L1, L2)
-    codes, scales, S = fp4_quantize(R)
-    return dict(R=R, wcodes=codes, wscales=scales, S_w=S)
+    if not c2:
+        codes, scales, S = fp4_quantize(R)
+        return dict(R=R, wcodes=codes, wscales=scales, S_w=S)
+    codes, scales, S, raised = fp4_quantize_c2(R)
+    return dict(R=R, wcodes=codes, wscales=scales, S_w=S, raised=raised)
+
+
+def fp4_quantize_c2(Z):
+    """C2 FP4: restricted group scales {1, 1.5} x 2^e; returns (codes, scales, S, raised)."""
+    Z = np.ascontiguousarray(Z, dtype=np.float32)
+    rows, cols = Z.shape
+    codes = np.empty((rows, cols // 2), np.uint8)
+    scales = np.empty((rows, cols // 16), np.uint8)
+    S = ctypes.c_float(0)
+    raised = _L().or_fp4_quantize_c2(_p(Z), rows, cols, _p(codes), _p(scales), ctypes.byref(S))
+    if raised < 0:
+        raise ValueError("or_fp4_quantize_c2 needs a multiple of 32 columns")
+    return codes, scales, float(S.value), int(raised)
+
+
+def c2_fp8_operand(codes, scales):
+    """E4M3 codes of q s_b / 2^u and the UE8M0 exponents u + 127 per 32 channels; with
+    the count of elements not reproduced exactly."""
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    rows, half = codes.shape
+    cols = half * 2
+    fp8 = np.empty((rows, cols), np.uint8)
+    ue = np.empty((rows, cols // 32), np.uint8)
+    inexact = _L().or_c2_fp8_operand(_p(codes), _p(scales), rows, cols, _p(fp8), _p(ue))
+    return fp8, ue, int(inexact)
 
 
 # --------------------------------------------------------------------------- output

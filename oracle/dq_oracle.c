@@ -284,6 +284,126 @@ static void fp4_row(const float* z, int cols, float S, uint8_t* codes, uint8_t* 
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* C2: restricted weight scales for an exact FP8-rate kernel-token product   */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The smallest value of the form {1, 1.5} x 2^e (e >= -9, 1.5 x 2^-9 excluded:
+ * E4M3 cannot hold it) that is >= v, for v > 0; 0 for v <= 0.  Every such
+ * value is an E4M3 value, and so is its product with any E2M1 value times a
+ * common power of two (mantissas 1, 1.125, 1.5 need at most 3 bits).
+ */
+float or_c2_scale_up(float v) {
+    if (!(v > 0.0f)) return 0.0f;
+    if (v <= 0x1p-9f) return 0x1p-9f;
+    int e;
+    const float m = frexpf(v, &e);        /* v = m 2^e, m in [0.5, 1) */
+    float r;
+    if (m == 0.5f) r = v;                  /* a power of two */
+    else if (m <= 0.75f) r = ldexpf(0.75f, e);
+    else r = ldexpf(1.0f, e);
+    if (r == 0x1.8p-9f) r = 0x1p-8f;
+    return r;
+}
+
+/*
+ * C2 weight quantiser (the restricted-scale reading, an option; the default is
+ * fp4_row's Eq. 4 form).  Per-tensor S = amax / (6 * 384) (384 = 1.5 x 2^8,
+ * the largest restricted scale), group-16 scales s_b = or_c2_scale_up(amax_b /
+ * (6 S)), then, per 32 channels, the smaller of the two scales raised to at
+ * least 2^-10 times the larger (a power-of-two ratio keeps the form), so that
+ * the block's q s_b span at most E4M3's exact range under one power-of-two
+ * exponent; q = E2M1(z / (s_b S)).  Returns the number of raised scales.
+ */
+long long or_fp4_quantize_c2(const float* Z, long long rows, int cols, uint8_t* codes, uint8_t* scales,
+                             float* S_out) {
+    if (cols % 32) return -1;
+    float amax = 0.0f;
+    for (long long i = 0; i < rows * (long long)cols; i++) {
+        float a = fabsf(Z[i]);
+        if (a > amax) amax = a;
+    }
+    const float S = (amax == 0.0f) ? 1.0f : amax / 2304.0f;
+    const float denom = 6.0f * S;
+    long long raised = 0;
+#pragma omp parallel for schedule(static) reduction(+ : raised)
+    for (long long r = 0; r < rows; r++) {
+        const float* z = Z + (size_t)r * cols;
+        for (int b2 = 0; b2 < cols / 32; b2++) {
+            float sb[2];
+            for (int h = 0; h < 2; h++) {
+                const int b = 2 * b2 + h;
+                float am = 0.0f;
+                for (int i = 0; i < 16; i++) {
+                    float a = fabsf(z[b * 16 + i]);
+                    if (a > am) am = a;
+                }
+                sb[h] = or_c2_scale_up(am / denom);
+                if (sb[h] > 384.0f) sb[h] = 384.0f;   /* fp32 rounding of amax / denom just above 384 */
+            }
+            const float big = sb[0] > sb[1] ? sb[0] : sb[1];
+            for (int h = 0; h < 2; h++) {
+                const float floor_s = ldexpf(big, -10);
+                if (sb[h] < floor_s) {
+                    sb[h] = floor_s;
+                    raised++;
+                }
+            }
+            for (int h = 0; h < 2; h++) {
+                const int b = 2 * b2 + h;
+                scales[(size_t)r * (cols / 16) + b] = (uint8_t)or_e4m3_encode(sb[h]);
+                const float eff = sb[h] * S;
+                for (int i = 0; i < 16; i += 2) {
+                    int q0 = (eff == 0.0f) ? 0 : or_e2m1_encode(z[b * 16 + i] / eff);
+                    int q1 = (eff == 0.0f) ? 0 : or_e2m1_encode(z[b * 16 + i + 1] / eff);
+                    codes[(size_t)r * (cols / 2) + (b * 16 + i) / 2] = (uint8_t)(q0 | (q1 << 4));
+                }
+            }
+        }
+    }
+    if (S_out) *S_out = S;
+    return raised;
+}
+
+/*
+ * The FP8 form of C2 weights for a kind::mxf8f6f4 product: per 32 channels one
+ * UE8M0 exponent u (biased by 127) and E4M3 codes of q s_b / 2^u, with u chosen
+ * so that the block's largest |q s_b| lands in [256, 512).  Returns the number
+ * of elements whose E4M3 code does not reproduce q s_b exactly (0 for weights
+ * from or_fp4_quantize_c2).
+ */
+long long or_c2_fp8_operand(const uint8_t* codes, const uint8_t* scales, long long rows, int cols, uint8_t* fp8,
+                            uint8_t* ue8m0) {
+    long long inexact = 0;
+#pragma omp parallel for schedule(static) reduction(+ : inexact)
+    for (long long r = 0; r < rows; r++) {
+        for (int b2 = 0; b2 < cols / 32; b2++) {
+            double w[32], wmax = 0.0;
+            for (int i = 0; i < 32; i++) {
+                const int c = b2 * 32 + i;
+                const int code = (codes[(size_t)r * (cols / 2) + c / 2] >> (4 * (c & 1))) & 15;
+                w[i] = or_e2m1_value(code) * or_e4m3_value(scales[(size_t)r * (cols / 16) + c / 16]);
+                if (fabs(w[i]) > wmax) wmax = fabs(w[i]);
+            }
+            int u = 0;
+            if (wmax > 0.0) {
+                int e;
+                frexp(wmax, &e);          /* wmax in [2^(e-1), 2^e) */
+                u = e - 1 - 8;
+            }
+            ue8m0[(size_t)r * (cols / 32) + b2] = (uint8_t)(u + 127);
+            for (int i = 0; i < 32; i++) {
+                const double v = ldexp(w[i], -u);
+                const int q = or_e4m3_encode((float)v);
+                fp8[(size_t)r * cols + b2 * 32 + i] = (uint8_t)q;
+                if (or_e4m3_value(q) != v) inexact++;
+            }
+        }
+    }
+    return inexact;
+}
+
 /* FP4-quantise a rows x cols fp32 matrix with its own per-tensor scale
  * (computed from its amax) or with the given S when S_in > 0. */
 int or_fp4_quantize(const float* Z, long long rows, int cols, float S_in, uint8_t* codes,

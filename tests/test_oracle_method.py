@@ -515,3 +515,54 @@ def test_pow2_scales_cost_little_accuracy():
         d = x - act["means"].astype(np.float64)[act["cube_of_n"]]
         err[p2] = np.linalg.norm(dqd - d) / np.linalg.norm(d)
     assert err[True] < 1.02 * err[False], err
+
+
+# ------------------------------------------------------------------ C2: restricted weight scales (option)
+
+def test_c2_scale_up_closed_form():
+    """The restricted scale is the smallest value {1, 1.5} x 2^e (e >= -9, 1.5 x 2^-9
+    excluded) at or above its argument."""
+    L = oracle._L()
+    rng = np.random.default_rng(7)
+    vals = np.concatenate([np.exp(rng.uniform(np.log(2.0 ** -12), np.log(380.0), 4000)),
+                           [1.0, 1.5, 2.0, 0.75, 2.0 ** -9, 2.0 ** -10, 1.5 * 2.0 ** -9]]).astype(np.float32)
+    members = sorted({m * 2.0 ** e for e in range(-9, 9) for m in (1.0, 1.5)} - {1.5 * 2.0 ** -9})
+    for v in vals:
+        r = L.or_c2_scale_up(float(v))
+        assert r in members and r >= v
+        i = members.index(r)
+        assert i == 0 or members[i - 1] < v
+
+
+@pytest.mark.parametrize("shape", [(256, 256, 16), (512, 1024, 32)])
+def test_c2_weights_have_an_exact_fp8_form(shape):
+    """Under the restricted scales every q s_b of a 32-channel block is an E4M3 value times
+    one power of two: the FP8 operand with its UE8M0 exponents reproduces it exactly."""
+    Co, Ci, r = shape
+    wl = synth.Workload("c2", 1, 1, 1, Ci, Co, r, (1, 1, 1), (1, 1, 1), (0.0, 1.0), (0.01, 20.0))
+    Wb = synth.weight(wl, seed=Co + Ci)
+    L1, L2, _ = oracle.lowrank_factors(Wb, r)
+    q = oracle.quantize_weight(Wb, L1, L2, c2=True)
+    fp8, ue, inexact = oracle.c2_fp8_operand(q["wcodes"], q["wscales"])
+    assert inexact == 0
+    w = _dequant_rows(q["wcodes"], q["wscales"], 1.0)
+    back = oracle.e4m3_value(fp8) * np.repeat(np.exp2(ue.astype(np.float64) - 127), 32, axis=1)
+    assert np.array_equal(back, w)
+    # every scale is {1, 1.5} x 2^e: E4M3 mantissa field 0 or 4 (or a subnormal power of two)
+    s = q["wscales"].astype(int)
+    normal = (s >> 3) > 0
+    assert np.all(np.isin(s[normal] & 7, (0, 4))) and np.all(np.isin(s[~normal], (0, 1, 2, 3, 4, 6)))
+
+
+def test_c2_accuracy_cost():
+    """The price of the FP8-rate form: restricted scales leave the top E2M1 codes unused in
+    many blocks, so the weight error grows (the default keeps Eq. 4's scales)."""
+    wl = synth.Workload("c2", 1, 1, 1, 1024, 512, 32, (1, 1, 1), (1, 1, 1), (0.0, 1.0), (0.01, 20.0))
+    Wb = synth.weight(wl, seed=5)
+    L1, L2, _ = oracle.lowrank_factors(Wb, 32)
+    R = oracle.residual(Wb, L1, L2).astype(np.float64)
+    err = {}
+    for c2 in (False, True):
+        q = oracle.quantize_weight(Wb, L1, L2, c2=c2)
+        err[c2] = np.linalg.norm(_dequant_rows(q["wcodes"], q["wscales"], q["S_w"]) - R) / np.linalg.norm(R)
+    assert err[False] < err[True] < 2 * err[False], err
