@@ -7,12 +7,13 @@
  *   is viewed as T x H x W x Ci and cut into t x h x w cubes (design 2).  Each
  *   cube's fp32 mean is its kernel token, each token minus its cube's mean a
  *   delta token (Eq. 1).  Kernel tokens are quantised to FP8 E4M3 with one fp32
- *   scale per token; delta tokens to FP4 E2M1 with one E4M3 scale per 16
- *   channels and one fp32 per-tensor scale (Eq. 4 with the NVFP4 reading).
+ *   scale per token (or per 64 channels, dq_linear_forward_grouped); delta
+ *   tokens to FP4 E2M1 with one E4M3 scale per 16 channels and one fp32
+ *   per-tensor scale (Eq. 4 with the NVFP4 reading).
  *   W (Co x Ci) is split offline into rank-r BF16 factors L1, L2 from its SVD
  *   and a residual R = W - L1 L2 quantised to the same FP4 format (Eq. 3):
- *     Y = dq(delta) dq(R)^T + broadcast_cube(dq(kernel) dq(R)^T) + (X L1) L2
- *   Y is N x Co BF16 in (t,h,w) order.
+ *     Y = dq(delta) dq(R)^T + broadcast_cube(dq(kernel) dq(R)^T) + (X L1) L2  [+ b]
+ *   Y is N x Co BF16 in (t,h,w) order; b is an optional bias (dq_pack_bias).
  *
  * Conventions for every entry point:
  *   - The return value is a dq_status code; nothing aborts or exits.
@@ -27,8 +28,8 @@
  *   - Inputs are never modified; outputs are fully overwritten.
  *   - Shapes: Ci and Co multiples of 256; rank a multiple of 16 in [16, 128];
  *     1 <= t <= T, 1 <= h <= H, 1 <= w <= W (cubes of any size up to the whole
- *     lattice, which gives one global kernel token).  Anything else returns
- *     DQ_ERR_UNSUPPORTED_SHAPE.  Device pointers must be 256-byte aligned
+ *     lattice, which gives one global kernel token); N = T*H*W < 2^31.
+ *     Anything else returns DQ_ERR_UNSUPPORTED_SHAPE.  Device pointers must be 256-byte aligned
  *     (DQ_ERR_ALIGNMENT otherwise).
  */
 #ifndef DELTAQUANT_H
