@@ -25,7 +25,13 @@
  *     short average the tokens they hold.
  *   - every fp32 step is a single IEEE operation; this file is compiled with
  *     -ffp-contract=off so no multiply-add is fused.
- * Parity pins: see tests/test_oracle_*.py.
+ * Options beside the default (each pinned on its own): one kernel scale per 64
+ * channels (or_fp8_kernel_tokens), a power-of-two per-tensor delta scale
+ * (or_quantize_activations_opt), restricted weight scales with an exact FP8
+ * form (or_fp4_quantize_c2, or_c2_fp8_operand), an additive bias (Python side).
+ * Parity pins: see tests/test_oracle_*.py.  Parity unpinned: nothing in this
+ * file; the GPU's tensor-core accumulation order is covered only by the Y
+ * tolerance.
  */
 #include <math.h>
 #include <stdint.h>
