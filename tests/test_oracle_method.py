@@ -566,3 +566,31 @@ def test_c2_accuracy_cost():
         q = oracle.quantize_weight(Wb, L1, L2, c2=c2)
         err[c2] = np.linalg.norm(_dequant_rows(q["wcodes"], q["wscales"], q["S_w"]) - R) / np.linalg.norm(R)
     assert err[False] < err[True] < 2 * err[False], err
+
+
+def test_single_read_encode_with_fixup_equals_direct_encode():
+    """The single-read algorithm the power-of-two delta scale allows: each work item (rows x a
+    range of channels) encodes under its own power-of-two scale S0 from its local max, then,
+    once the global S is known, every block's scale code drops by 8 log2(S / S0) and its
+    codes stay, except blocks without the exponent headroom, which are encoded again under S.
+    The result equals encoding every item directly under S."""
+    L = oracle._L()
+    rng = np.random.default_rng(11)
+    # rows of very different magnitude, so that items' local scales differ by several binades
+    Z = (rng.standard_normal((96, 512)) * np.exp(rng.uniform(-9, 3, size=(96, 1)))).astype(np.float32)
+    S = float(L.or_pow2_ceil(float(np.abs(Z).max()) / 2688.0))
+    reencoded = 0
+    for r0 in range(0, 96, 32):
+        for c0 in range(0, 512, 128):
+            item = np.ascontiguousarray(Z[r0:r0 + 32, c0:c0 + 128])
+            S0 = float(L.or_pow2_ceil(float(np.abs(item).max()) / 2688.0))
+            j = int(round(math.log2(S / S0)))
+            codes0, scales0, _ = oracle.fp4_quantize(item, S0)
+            codesS, scalesS, _ = oracle.fp4_quantize(item, S)
+            ok = ((scales0.astype(int) >> 3) & 15) >= j + 1
+            fixed_scales = np.where(ok, scales0.astype(int) - 8 * j, scalesS.astype(int))
+            fixed_codes = np.where(np.repeat(ok, 8, axis=1), codes0, codesS)
+            reencoded += int((~ok).sum())
+            assert np.array_equal(fixed_scales, scalesS.astype(int))
+            assert np.array_equal(fixed_codes, codesS)
+    assert reencoded > 0      # the re-encode branch is exercised too
