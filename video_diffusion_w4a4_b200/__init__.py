@@ -262,6 +262,7 @@ def dq_workspace_layout_get(T, H, W, t, h, w, Ci, Co, rank) -> dq_workspace_layo
 
 
 def dq_workspace_layout_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group) -> dq_workspace_layout:
+    """Workspace carve-up for a kernel-token scale granularity (DQ_KERNEL_SCALE_*)."""
     L = dq_workspace_layout()
     _check("dq_workspace_layout_grouped", _lib.dq_workspace_layout_grouped(T, H, W, t, h, w, Ci, Co, rank,
                                                                            kernel_group, ctypes.byref(L)))
@@ -269,6 +270,7 @@ def dq_workspace_layout_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group) ->
 
 
 def dq_workspace_bytes_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group) -> int:
+    """Workspace bytes for a kernel-token scale granularity (DQ_KERNEL_SCALE_*)."""
     b = ctypes.c_size_t()
     _check("dq_workspace_bytes_grouped", _lib.dq_workspace_bytes_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group,
                                                                          ctypes.byref(b)))
@@ -299,6 +301,7 @@ def _events(stage_events):
 def dq_linear_forward_grouped(X, T, H, W, t, h, w, Ci, Co, rank, kernel_group, packed_W, L1_mma, L2_slab, Y,
                               workspace, workspace_bytes, stage_mask=DQ_STAGE_ALL, stage_events=None,
                               stream=None) -> None:
+    """dq_linear_forward_ex with kernel_group: DQ_KERNEL_SCALE_PER_TOKEN or DQ_KERNEL_SCALE_GROUP64."""
     _check("dq_linear_forward_grouped",
            _lib.dq_linear_forward_grouped(_ptr(X), T, H, W, t, h, w, Ci, Co, rank, kernel_group, _ptr(packed_W),
                                           _ptr(L1_mma), _ptr(L2_slab), _ptr(Y), _ptr(workspace), workspace_bytes,
