@@ -32,6 +32,33 @@ def sfa_unpermute(buf: np.ndarray, rows: int, cols: int) -> np.ndarray:
     return buf[off]
 
 
+def sfb_unpermute(buf: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """B-operand scale layout (include/deltaquant.h, dq_sfb_offset) -> plain rows x cols/16.
+    Each scale is stored four times, once per 32-lane quadrant (1024 bytes apart);
+    the four copies must agree."""
+    r = np.arange(rows, dtype=np.int64)[:, None]
+    b = np.arange(cols // 16, dtype=np.int64)[None, :]
+    n = r % 256
+    word = 4 * (n // 128) + (n % 128) // 32
+    bb = 4 * word + b % 4
+    off = ((r // 256) * (cols // 64) + b // 4) * 4096 + ((n % 32) // 8) * 256 + (bb // 16) * 128 + (n % 8) * 16 \
+        + bb % 16
+    copies = [buf[off + 1024 * q] for q in range(4)]
+    for q in range(1, 4):
+        assert np.array_equal(copies[q], copies[0]), f"weight scale copy of quadrant {q} differs"
+    return copies[0]
+
+
+def packed_weight_parts(packed: np.ndarray) -> dict:
+    """Codes, group scales (plain Co x Ci/16) and S_W of a packed weight blob, read
+    through the offsets in its header (include/deltaquant.h)."""
+    Co, Ci = (int(v) for v in packed[8:16].view(np.int32))
+    off_codes, off_scales = (int(v) for v in packed[32:48].view(np.uint64))
+    codes = packed[off_codes:off_codes + Co * Ci // 2].reshape(Co, Ci // 2)
+    scales = sfb_unpermute(packed[off_scales:], Co, Ci)
+    return dict(wcodes=codes, wscales=scales, S_w=packed[24:28].view(np.float32)[0], Co=Co, Ci=Ci)
+
+
 def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
@@ -117,8 +144,16 @@ class Case:
 
 
 def compare_quantised(g: dict, act: dict, wq: dict) -> None:
-    """Every quantised tensor bit-exact against the oracle."""
+    """Every quantised tensor bit-exact against the oracle: the delta codes and
+    scales, S_delta, the kernel tokens and their scales, and the packed weight's
+    residual codes, group scales (all four per-quadrant copies) and S_W."""
     assert g["status"] == 0, g["status"]
+    pw = packed_weight_parts(g["packed"])
+    bad = np.argwhere(pw["wcodes"] != wq["wcodes"])
+    assert bad.size == 0, ("weight codes", bad[:5].tolist())
+    bad = np.argwhere(pw["wscales"] != wq["wscales"])
+    assert bad.size == 0, ("weight scales", bad[:5].tolist())
+    assert np.float32(pw["S_w"]) == np.float32(wq["S_w"])
     assert np.float32(g["amax_delta"]) == np.float32(act["amax_delta"])
     assert np.float32(g["S_delta"]) == np.float32(act["S_delta"])
     assert np.float32(g["S_W"]) == np.float32(wq["S_w"])
@@ -137,3 +172,44 @@ def compare_quantised(g: dict, act: dict, wq: dict) -> None:
     assert bad.size == 0, ("delta scales", bad[:5].tolist())
     bad = np.argwhere(g["dcodes"] != act["dcodes"])
     assert bad.size == 0, ("delta codes", bad[:5].tolist(), g["dcodes"][tuple(bad[0])], act["dcodes"][tuple(bad[0])])
+
+
+def kernel_term_reference(act: dict, wq: dict, cubes: np.ndarray, bias=None):
+    """The per-cube kernel term P'[k][o] = S_W sum_c (q8 s8)[k][c] (q s_b)[o][c] (+ b[o])
+    of the sampled cubes, in fp64 from the oracle's kernel tokens and weight codes
+    (Eq. 2/3, the single-token term; the bias joins once per cube).  Also returns
+    S_W sum_c |(q8 s8)[k][c] (q s_b)[o][c]|, the magnitude that bounds the rounding
+    error of an fp32 accumulation of the same sum."""
+    cubes = np.asarray(cubes, np.int64)
+    Ci = act["q8"].shape[1]
+    s8 = np.asarray(act["s8"], np.float64).reshape(len(act["q8"]), -1)
+    kv = oracle.e4m3_value(act["q8"][cubes]) * np.repeat(s8[cubes], Ci // s8.shape[1], axis=1)
+    dqw = oracle.fp4_dequantize(wq["wcodes"], wq["wscales"], 1.0)
+    S_W = float(np.float32(wq["S_w"]))
+    ref = S_W * (kv @ dqw.T)
+    mag = S_W * (np.abs(kv) @ np.abs(dqw).T)
+    if bias is not None:
+        b = oracle.bf16_value(np.asarray(bias, np.uint16)).astype(np.float64)
+        ref = ref + b[None, :]
+        mag = mag + np.abs(b)[None, :]
+    return ref, mag
+
+
+def assert_kernel_term_close(p_gpu: np.ndarray, act: dict, wq: dict, cubes, bias=None, extra_rel: float = 0.0):
+    """P' (K x Co fp32, read from the workspace) on the sampled cubes against the fp64
+    kernel term.  Bound: the worst-case error of accumulating Ci products in fp32
+    (Ci * 2^-23 of the sum of |products|, twice the unit roundoff to allow for an
+    accumulator that truncates), one fp32 rounding of the scaled result, and, for
+    group-64 kernel scales, the BF16 hi + lo split of q8 s8 (extra_rel of the sum of
+    |products|)."""
+    cubes = np.asarray(cubes, np.int64)
+    ref, mag = kernel_term_reference(act, wq, cubes, bias)
+    Ci = act["q8"].shape[1]
+    tol = (Ci * 2.0 ** -23 + extra_rel) * mag + 2.0 ** -23 * np.abs(ref)
+    got = p_gpu[cubes].astype(np.float64)
+    err = np.abs(got - ref)
+    bad = err > tol
+    info = dict(max_err_over_tol=float((err / np.where(tol > 0, tol, 1.0)).max()), n_bad=int(bad.sum()),
+                n=int(err.size), max_rel_err=float((err / np.maximum(np.abs(ref), 1e-30)).max()))
+    assert not bad.any(), f"P': {info}, first bad at {np.argwhere(bad)[:5].tolist()}"
+    return info

@@ -12,7 +12,7 @@ import pytest
 
 import oracle
 import synth
-from dq_case import Case, assert_y_close, compare_quantised
+from dq_case import Case, assert_kernel_term_close, assert_y_close, compare_quantised
 
 pytestmark = pytest.mark.gpu
 
@@ -87,6 +87,7 @@ def test_parity_small(env, name, wl):
     g = case.run_gpu(dq, torch)
     act, wq = case.run_oracle()
     compare_quantised(g, act, wq)
+    assert_kernel_term_close(g["p"], act, wq, np.arange(g["layout"].K))
     y_ref = case.oracle_rows(act, wq, np.arange(wl.N))
     assert_y_close(g["Y"], y_ref)
 
@@ -105,6 +106,8 @@ def test_parity_bias(env, name, kernel_group):
     g = case.run_gpu(dq, torch, bias=b)
     act, wq = case.run_oracle()
     compare_quantised(g, act, wq)
+    assert_kernel_term_close(g["p"], act, wq, np.arange(g["layout"].K), bias=b,
+                             extra_rel=2.0 ** -16 if kernel_group else 0.0)
     assert_y_close(g["Y"], case.oracle_rows(act, wq, np.arange(wl.N), bias=b))
     # clearing the bias again gives the no-bias layer bit for bit
     g0 = case.run_gpu(dq, torch)
@@ -125,6 +128,7 @@ def test_parity_group64_kernel_scales(env, name):
     act, wq = case.run_oracle()
     assert g["s8"].shape == act["s8"].shape
     compare_quantised(g, act, wq)
+    assert_kernel_term_close(g["p"], act, wq, np.arange(g["layout"].K), extra_rel=2.0 ** -16)
     assert_y_close(g["Y"], case.oracle_rows(act, wq, np.arange(wl.N)))
 
 

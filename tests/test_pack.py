@@ -108,3 +108,22 @@ def test_pack_bias_section(dq):
     bad[0] ^= 1
     with pytest.raises(dq.DQError):
         dq.dq_pack_bias(bad, b)
+
+
+@pytest.mark.parametrize("shape", [(256, 256), (512, 1024)])
+def test_vectorised_weight_scale_map_matches_library(dq, shape):
+    """The parity tests read the packed weight's scales at full size through a
+    vectorised form of the B-operand scale layout; it must address the same bytes
+    as the library's dq_sfb_offset (a scrambled blob makes every scale distinct
+    enough to catch a wrong index)."""
+    from dq_case import sfb_unpermute
+    Co, Ci = shape
+    nbytes = dq.dq_sfb_bytes(Co, Ci)
+    blob = np.zeros(nbytes, np.uint8)
+    plain = np.random.default_rng(Co + Ci).integers(0, 256, size=(Co, Ci // 16), dtype=np.uint8)
+    for r in range(Co):
+        for b in range(Ci // 16):
+            off = dq.dq_sfb_offset(r, b, Ci)
+            for q in range(4):
+                blob[off + 1024 * q] = plain[r, b]
+    assert np.array_equal(sfb_unpermute(blob, Co, Ci), plain)
