@@ -3,14 +3,24 @@
 One step = one forward of the whole layer (cube statistics, cube encode,
 kernel-token product, main FP4 product with the low-rank slab and the
 scatter epilogue) over one synthetic activation tensor X resident in HBM.
-Default workload: the Wan-like 480p attention projection (T=21, H=30, W=52,
-N=32760 tokens, Ci=Co=5120, rank 32, cube 1x2x2).
+Default workload: the Wan-like 720p FFN down-projection (T=21, H=45, W=80,
+N=75600 tokens, Ci=13824 -> Co=5120, rank 32, cube 1x2x2), the largest
+layer that fits one GPU; --workload picks another.
 
 Prints one JSON line (rank 0).  `value` is whole-job TFLOP/s with
 F = 2 N Ci Co + 2 K Ci Co + 2 N r (Ci + Co) (main + kernel-token + low-rank
 products, real rows only) per step; tokens/s and the per-stage breakdown are
-extra keys.  --impl reference times the CPU oracle on a bounded sample of
-the same workload instead.
+extra keys.
+
+Several GPUs (one process each, under torchrun): by default ONE layer is
+sharded by cubes (slabs of whole cube layers along T, the weight replicated,
+one 4-byte NCCL all-reduce(max) of the delta amax between the statistics and
+encode stages), so the total work is fixed ("strong" scaling);
+--parallelism replicas runs an independent layer per GPU instead ("weak").
+
+--impl reference times the CPU oracle instead: each step a bounded slice of
+the same seeded cube sample as the GPU arm's cpu_baseline, under the delta
+scale of a whole-tensor statistics pass.
 """
 from __future__ import annotations
 
@@ -161,32 +171,59 @@ def parse_cube(s):
     return tuple(int(v) for v in s.split(",")) if s else None
 
 
-# --------------------------------------------------------------------------- reference arm (CPU oracle)
+# --------------------------------------------------------------------------- CPU oracle (baseline and reference arm)
 
-def oracle_sample(wl, cube, X, Wb, L1, L2, wq, ntok):
-    """Oracle over a bounded sample of whole cubes, quantised as its own tensor, then
-    its Y rows: whole cube layers of frames [0, k t) while they fit in `ntok` tokens,
-    else the first cube rows of frames [0, t).  Returns (seconds, flops of the sample,
-    tokens)."""
+SAMPLE_CUBES = 512        # seeded cube sample of the CPU baseline (layers too large for a full oracle run)
+SAMPLE_SEED = 0x5A3D
+REFERENCE_SLICE = 64      # cubes per reference-arm step (a slice of the same sample)
+
+
+def oracle_sample_cubes(wl, cube):
+    """All cubes for layers the oracle finishes in reasonable time on the whole tensor
+    (the tiny case and the 480p projection), else a seeded sample of SAMPLE_CUBES cubes."""
     import oracle
-    t, h, w = cube
-    per_layer = t * wl.H * wl.W
-    if ntok >= per_layer:
-        Ts, Hs = min(wl.T, t * (ntok // per_layer)), wl.H
-    else:
-        n_rows = max(1, ntok // (t * h * wl.W))
-        Ts, Hs = min(wl.T, t), min(wl.H, n_rows * h)
-    idx = (np.arange(Ts)[:, None, None] * wl.H * wl.W + np.arange(Hs)[None, :, None] * wl.W
-           + np.arange(wl.W)[None, None, :]).reshape(-1)
-    Xs = np.ascontiguousarray(X[idx])
-    t0 = time.perf_counter()
-    act = oracle.quantize_activations(Xs, Ts, Hs, wl.W, cube)
-    rows = np.arange(Xs.shape[0])
-    oracle.output_rows(act, wq, Xs, L1, L2, rows)
-    dt = time.perf_counter() - t0
-    K = oracle.num_cubes(Ts, Hs, wl.W, *cube)
-    sub = synth.Workload("sample", Ts, Hs, wl.W, wl.Ci, wl.Co, wl.rank, cube, wl.grid, wl.x_outliers, wl.w_outliers)
-    return dt, layer_flops(sub, K), Xs.shape[0]
+    K = oracle.num_cubes(wl.T, wl.H, wl.W, *cube)
+    if wl.name in ("tiny", "wan480p_proj") or K <= SAMPLE_CUBES:
+        return np.arange(K, dtype=np.int64), True
+    return np.sort(np.random.default_rng(SAMPLE_SEED).choice(K, size=SAMPLE_CUBES, replace=False)), False
+
+
+class OracleLayer:
+    """The oracle's weight side and whole-tensor statistics pass of one workload, and
+    timed runs over sets of its cubes."""
+
+    def __init__(self, wl, cube, X, L1, L2, wq):
+        import oracle
+        self.oracle, self.wl, self.cube, self.X, self.L1, self.L2, self.wq = oracle, wl, cube, X, L1, L2, wq
+        t0 = time.perf_counter()
+        # S_delta needs the max |delta| of the whole tensor: the oracle's statistics pass over all cubes
+        self.S = oracle.tensor_scale(oracle.delta_amax(X, wl.T, wl.H, wl.W, cube))
+        self.stats_s = time.perf_counter() - t0
+        self.K = oracle.num_cubes(wl.T, wl.H, wl.W, *cube)
+        self.threads = oracle.num_threads()
+
+    def run(self, cubes):
+        """Quantise the cubes (means, FP8 kernel tokens, FP4 deltas under S) and compute
+        their Y rows in fp64; returns (seconds, tokens)."""
+        o, wl = self.oracle, self.wl
+        t0 = time.perf_counter()
+        sub = o.quantize_cubes(self.X, wl.T, wl.H, wl.W, self.cube, cubes, self.S)
+        o.output_rows(sub, self.wq, self.X, self.L1, self.L2, sub["rows"])
+        return time.perf_counter() - t0, int(sub["rows"].size)
+
+    def full_seconds(self, sample_s, sample_tokens):
+        """Whole-layer oracle time: the statistics pass plus the sample's time scaled by tokens."""
+        return self.stats_s + sample_s * self.wl.N / sample_tokens
+
+
+def bench_config(wl, cube, K, kernel_group, world, parallelism):
+    """The `config` object of the JSON line, identical for the GPU arm and the reference arm."""
+    return dict(workload=wl.name, T=wl.T, H=wl.H, W=wl.W, N=wl.N, Ci=wl.Ci, Co=wl.Co, rank=wl.rank, cube=list(cube),
+                K=K, kernel_scale="per-token" if not kernel_group else f"group{kernel_group}",
+                parallelism=(f"cube-sharded x{world} (T-slabs of whole cube layers, NCCL all-reduce(max) of the "
+                             f"delta amax)" if parallelism == "sharded" and world > 1
+                             else f"dp{world} (independent layer per GPU)"),
+                l2="inputs larger than L2 (X %.0f MB, Y %.0f MB)" % (wl.N * wl.Ci * 2 / 1e6, wl.N * wl.Co * 2 / 1e6))
 
 
 def run_reference(args, wl, cube):
@@ -199,29 +236,45 @@ def run_reference(args, wl, cube):
     Wb = synth.weight(wl)
     L1, L2, _ = oracle.lowrank_factors(Wb, wl.rank)
     wq = oracle.quantize_weight(Wb, L1, L2)
-    ntok = args.sample_tokens
-    for _ in range(args.warmup):
-        oracle_sample(wl, cube, X, Wb, L1, L2, wq, ntok)
-    times, flops, toks = [], 0.0, 0
-    for _ in range(args.steps):
-        dt, f, n = oracle_sample(wl, cube, X, Wb, L1, L2, wq, ntok)
-        times.append(dt)
-        flops, toks = f, n
-    t = sum(times) / len(times)
-    value = flops / t / 1e12
-    cores = os.cpu_count()
-    sample = (f"{toks} tokens ({cube[0]}x{cube[1]}x{cube[2]} cubes, whole cube rows of frame slab 0) of "
-              f"{wl.name}, full Ci={wl.Ci}, Co={wl.Co}, r={wl.rank}; fp64 Y rows; per step")
+    layer = OracleLayer(wl, cube, X, L1, L2, wq)
+    cubes, full = oracle_sample_cubes(wl, cube)
+    if wl.name == "tiny":
+        slices = [cubes]
+    else:
+        slices = [cubes[i:i + REFERENCE_SLICE] for i in range(0, cubes.size, REFERENCE_SLICE)]
+    for i in range(args.warmup):
+        layer.run(slices[i % len(slices)])
+    secs, toks = [], []
+    for i in range(args.steps):
+        dt, n = layer.run(slices[i % len(slices)])
+        secs.append(dt)
+        toks.append(n)
+    sample_s, sample_tok = sum(secs), sum(toks)
+    t_full = layer.full_seconds(sample_s, sample_tok)
+    K = layer.K
+    F = layer_flops(wl, K)
+    value = F / t_full / 1e12
+    sample = (f"{args.steps} steps over slices of {REFERENCE_SLICE} cubes of a seeded {cubes.size}-cube sample "
+              f"({sample_tok} tokens, {sample_s:.1f} s) under the whole tensor's delta scale (statistics pass "
+              f"{layer.stats_s:.1f} s); value = whole-layer FLOPs / (statistics pass + sample time x N / sample "
+              f"tokens) = {t_full:.0f} s extrapolated")
     line = dict(metric=METRIC, value=value, unit="TFLOP/s", impl="reference", n_gpus=args.gpus, steps=args.steps,
-                warmup=args.warmup, ms_per_step=t * 1e3, higher_is_better=True, scaling="weak", vs_baseline=None,
-                dtype="f64", data="synthetic",
-                config=dict(workload=wl.name, T=wl.T, H=wl.H, W=wl.W, Ci=wl.Ci, Co=wl.Co, rank=wl.rank,
-                            cube=list(cube), sample_tokens=toks),
-                tokens_per_s=toks / t,
-                cpu_baseline=dict(value=value, unit="TFLOP/s", cores=cores, kind="oracle", sample=sample),
+                warmup=args.warmup, ms_per_step=sample_s / args.steps * 1e3, higher_is_better=True,
+                scaling="weak" if args.gpus == 1 or args.parallelism == "replicas" else "strong",
+                vs_baseline=None, dtype="f64", data="synthetic",
+                config=bench_config(wl, cube, K, args.kernel_group, args.gpus, args.parallelism),
+                tokens_per_s=wl.N / t_full, sample_tflops=sum(layer_flops_rows(wl, K, n) for n in toks) / sample_s / 1e12,
+                cpu_baseline=dict(value=value, unit="TFLOP/s", cores=layer.threads, kind="oracle", sample=sample,
+                                  sample_seconds=sample_s, extrapolated_full_seconds=t_full),
                 e2e=dict(value=value, unit="TFLOP/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
     print(json.dumps(line), flush=True)
     return 0
+
+
+def layer_flops_rows(wl, K, rows):
+    """FLOPs of `rows` output rows of the layer, with the kernel-token product counted
+    once per cube (K / N of it per row)."""
+    return rows * (2.0 * wl.Ci * wl.Co * (1.0 + K / wl.N) + 2.0 * wl.rank * (wl.Ci + wl.Co))
 
 
 # --------------------------------------------------------------------------- GPU arm
@@ -232,13 +285,13 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="dq", choices=["dq", "reference"])
-    ap.add_argument("--workload", default="wan480p_proj", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="wan720p_ffn_down", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--cube", default=None, help="override the cube, e.g. 2,2,2")
     ap.add_argument("--frames", type=int, default=None, help="override T (smaller cases for profiling)")
     ap.add_argument("--kernel-group", type=int, default=0, choices=[0, 64],
                     help="FP8 kernel-token scales: 0 = one per token, 64 = one per 64 channels")
-    ap.add_argument("--sample-tokens", type=int, default=256, help="oracle sample size per reference step (tokens)")
-    ap.add_argument("--baseline-tokens", type=int, default=6144, help="oracle sample size of the cpu_baseline leg")
+    ap.add_argument("--parallelism", default="sharded", choices=["sharded", "replicas"],
+                    help="with several GPUs: one layer sharded by cubes (default) or one layer per GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     args = ap.parse_args()
@@ -256,6 +309,7 @@ def main():
 
     import torch
     import video_diffusion_w4a4_b200 as dq
+    from video_diffusion_w4a4_b200 import shard
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -268,28 +322,49 @@ def main():
 
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    sharded = world > 1 and args.parallelism == "sharded"
+    kg = args.kernel_group
+    if sharded and kg:
+        ap.error("the cube-sharded layer takes per-token kernel scales")
 
     t, h, w = cube
     K = dq.dq_cube_count(wl.T, wl.H, wl.W, t, h, w)
-    # inputs: each rank its own activation tensor (a different denoising step), one shared weight
-    X = synth.activations(wl, tau=rank)
+    # inputs: replicas give each rank its own activation tensor (a different denoising step);
+    # the sharded layer gives every rank the same tensor, of which it keeps its slab of frames
+    X = synth.activations(wl, tau=0 if sharded else rank)
     Wb = synth.weight(wl)
     t0 = time.perf_counter()
     packed, L1m, L2s = dq.dq_pack_weight(Wb, wl.rank)
     pack_s = time.perf_counter() - t0
-    Xd = torch.from_numpy(X.view(np.int16)).to(dev)
+    if sharded:
+        f0, f1 = shard.slab_frames(wl.T, t, world, rank)
+        Ts = f1 - f0
+        ts, hs, ws_ = shard.slab_cube(cube, Ts)
+        X_mine = X[f0 * wl.H * wl.W:f1 * wl.H * wl.W]
+    else:
+        Ts, (ts, hs, ws_), X_mine = wl.T, cube, X
+    Nm = Ts * wl.H * wl.W
+    Xd = torch.from_numpy(X_mine.view(np.int16)).to(dev)
     Pd = torch.from_numpy(packed).to(dev)
     L1d = torch.from_numpy(L1m.view(np.int16)).to(dev)
     L2d = torch.from_numpy(L2s.view(np.int16)).to(dev)
-    Yd = torch.empty((wl.N, wl.Co), dtype=torch.int16, device=dev)
-    kg = args.kernel_group
-    lay = dq.dq_workspace_layout_grouped(wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, kg)
+    Yd = torch.empty((Nm, wl.Co), dtype=torch.int16, device=dev)
+    lay = dq.dq_workspace_layout_grouped(Ts, wl.H, wl.W, ts, hs, ws_, wl.Ci, wl.Co, wl.rank, kg)
     ws = torch.zeros(lay.total_bytes, dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream(dev)
 
-    def step(events=None):
-        dq.dq_linear_forward_grouped(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, kg, Pd, L1d, L2d, Yd, ws,
-                                     lay.total_bytes, dq.DQ_STAGE_ALL, events, st)
+    def allreduce_max(a):
+        dist.all_reduce(a, op=dist.ReduceOp.MAX)
+
+    def step(events=None, pre=None):
+        if not sharded:
+            dq.dq_linear_forward_grouped(Xd, Ts, wl.H, wl.W, ts, hs, ws_, wl.Ci, wl.Co, wl.rank, kg, Pd, L1d, L2d, Yd,
+                                         ws, lay.total_bytes, dq.DQ_STAGE_ALL, events, st)
+            return
+        # the cube-sharded layer: statistics of this slab, the one exchanged scalar (NCCL), then
+        # encode and both products
+        shard.forward_sharded(Xd, Ts, wl.H, wl.W, cube, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd, ws, allreduce_max,
+                              st, events, pre)
 
     for _ in range(args.warmup):
         step()
@@ -298,7 +373,7 @@ def main():
     if status != 0:
         raise RuntimeError(f"device status after warm-up: {dq.dq_status_string(status)}")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     for row in evs:          # torch creates CUDA events lazily; create them before handing them to the library
         for e in row:
             e.record(st)
@@ -310,27 +385,38 @@ def main():
         end = torch.cuda.Event(enable_timing=True)
         start.record(st)
         for i in range(args.steps):
-            step(evs[i])
+            step(evs[i][1:], evs[i][0])
         end.record(st)
         torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
     ms = start.elapsed_time(end) / args.steps
-    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+    stage_ms = {n: statistics.mean(evs[i][j + 1].elapsed_time(evs[i][j + 2]) for i in range(args.steps))
                 for j, n in enumerate(("quantize", "kernel_gemm", "main_gemm"))}
+    if sharded:
+        # statistics pass + all-reduce, before the encode stage's first event; the quantise stage
+        # below counts both halves (statistics, all-reduce and encode)
+        stage_ms["stats_allreduce"] = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps))
+        stage_ms["quantize"] += stage_ms["stats_allreduce"]
     status = dq.dq_read_device_status(ws, st, clear=True)
     if status != 0:
         raise RuntimeError(f"device status after timing: {dq.dq_status_string(status)}")
     ms = max_over_ranks(ms, dist, dev)
 
-    # end to end through the host-buffer entry point: pinned X in, Y out, copies inside the timed region
-    Xh = torch.from_numpy(X.view(np.int16)).pin_memory()
-    Yh = torch.empty((wl.N, wl.Co), dtype=torch.int16).pin_memory()
+    # end to end through the public API with host buffers: pinned X in, Y out, copies inside the timed region
+    Xh = torch.from_numpy(X_mine.view(np.int16)).pin_memory()
+    Yh = torch.empty((Nm, wl.Co), dtype=torch.int16).pin_memory()
     Xd2, Yd2 = torch.empty_like(Xd), torch.empty_like(Yd)
 
     def e2e_step():
-        dq.dq_linear_forward_host(Xh, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yh, Xd2, Yd2,
-                                  ws, lay.total_bytes, st)
+        if not sharded:
+            dq.dq_linear_forward_host(Xh, Ts, wl.H, wl.W, ts, hs, ws_, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yh, Xd2,
+                                      Yd2, ws, lay.total_bytes, st)
+            return
+        Xd2.copy_(Xh, non_blocking=True)
+        shard.forward_sharded(Xd2, Ts, wl.H, wl.W, cube, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd2, ws, allreduce_max,
+                              st)
+        Yh.copy_(Yd2, non_blocking=True)
 
     e2e_ms = None
     if not kg:   # the host-buffer entry point takes per-token kernel scales
@@ -350,60 +436,78 @@ def main():
         dist.barrier()
 
     F = layer_flops(wl, K)
-    value = job_tflops(F, world, ms)
+    # whole-job FLOPs per step: the one layer (sharded) or one layer per GPU (replicas)
+    value = (F / (ms * 1e-3) / 1e12) if sharded else job_tflops(F, world, ms)
     peaks = load_peaks()
     fp4_peak = peaks["bf16"] * FP4_PER_BF16
-    model = stage_model(wl, K, lay.slab, kg)
+    # per-stage work model of this rank's share (its slab when sharded)
+    wl_mine = wl if not sharded else synth.Workload(wl.name, Ts, wl.H, wl.W, wl.Ci, wl.Co, wl.rank, (ts, hs, ws_),
+                                                    wl.grid, wl.x_outliers, wl.w_outliers, wl.gelu)
+    model = stage_model(wl_mine, int(lay.K), lay.slab, kg)
     # dominant kernel = the stage with the largest share of the step
-    dom = max(stage_ms, key=stage_ms.get)
+    dom = max(("quantize", "kernel_gemm", "main_gemm"), key=stage_ms.get)
     if dom == "quantize":
         ach = model[dom]["bytes"] / (stage_ms[dom] * 1e-3) / 1e9
         roof = dict(kernel="k_cube_stats+k_cube_encode", bound="hbm", achieved=ach, peak=peaks["hbm"], unit="GB/s")
     else:
         pk = fp4_peak if dom == "main_gemm" else peaks["bf16"]
         ach = model[dom]["flops"] / (stage_ms[dom] * 1e-3) / 1e12
-        roof = dict(kernel="k_main_gemm" if dom == "main_gemm" else "k_kernel_gemm", bound="tensor", achieved=ach,
-                    peak=pk, unit="TFLOP/s")
+        roof = dict(kernel="k_gemm<true> (main FP4 product)" if dom == "main_gemm" else "k_gemm<false> (kernel-token product)",
+                    bound="tensor", achieved=ach, peak=pk, unit="TFLOP/s")
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = committed_traffic(wl, dom) if tuple(cube) == tuple(synth.WORKLOADS[args.workload].cube) else None
+    same_cube = tuple(cube) == tuple(synth.WORKLOADS[args.workload].cube)
+    roof["traffic"] = committed_traffic(wl_mine, dom) if same_cube and not kg else None
     roof["peak_source"] = ("measured" if peaks["source"] == "measured" else "fallback") + (
         " bf16 x 4 (nominal FP4:BF16)" if roof["unit"] == "TFLOP/s" and dom == "main_gemm" else "")
     stages = {}
     for n, tms in stage_ms.items():
+        if n not in model:
+            stages[n] = dict(ms=tms)
+            continue
         m = model[n]
         stages[n] = dict(ms=tms, tflops=m["flops"] / (tms * 1e-3) / 1e12, gbs=m["bytes"] / (tms * 1e-3) / 1e9)
     stages["quantize"]["frac_hbm"] = stages["quantize"]["gbs"] / peaks["hbm"]
     stages["kernel_gemm"]["frac_bf16"] = stages["kernel_gemm"]["tflops"] / peaks["bf16"]
     stages["main_gemm"]["frac_fp4"] = stages["main_gemm"]["tflops"] / fp4_peak
     layer_bytes = sum(m["bytes"] for m in model.values())
-    layer_roof_ms = max(F / (fp4_peak * 1e12), layer_bytes / (peaks["hbm"] * 1e9)) * 1e3
+    F_mine = layer_flops(wl_mine, int(lay.K))
+    layer_roof_ms = max(F_mine / (fp4_peak * 1e12), layer_bytes / (peaks["hbm"] * 1e9)) * 1e3
+    launches = (5 if t * h * w > 128 else 4)
     line = dict(metric=METRIC, value=value, unit="TFLOP/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
-                ms_per_step=ms, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="e2m1/e4m3->f32",
-                data="synthetic",
-                config=dict(workload=wl.name, T=wl.T, H=wl.H, W=wl.W, N=wl.N, Ci=wl.Ci, Co=wl.Co, rank=wl.rank,
-                            cube=list(cube), K=K,
-                            kernel_scale="per-token" if not kg else f"group{kg}", parallelism=f"dp{world} (independent layer per GPU)",
-                            l2="inputs larger than L2 (X %.0f MB, Y %.0f MB)" % (wl.N * wl.Ci * 2 / 1e6,
-                                                                                 wl.N * wl.Co * 2 / 1e6)),
-                tokens_per_s=wl.N * world / (ms * 1e-3),
+                ms_per_step=ms, higher_is_better=True, scaling="strong" if sharded else "weak", vs_baseline=None,
+                dtype="e2m1/e4m3->f32", data="synthetic",
+                config=bench_config(wl, cube, K, kg, world, args.parallelism),
+                tokens_per_s=wl.N * (1 if sharded else world) / (ms * 1e-3),
                 layer_roofline_frac=layer_roof_ms / ms,
                 roofline=roof, stages=stages,
                 e2e=None if e2e_ms is None else dict(
-                    value=job_tflops(F, world, e2e_ms), unit="TFLOP/s", h2d_bytes_per_step=wl.N * wl.Ci * 2,
-                    d2h_bytes_per_step=wl.N * wl.Co * 2, ms_per_step=e2e_ms),
-                gpu_launches=(5 if t * h * w > 128 else 4) * args.steps, pack_seconds=pack_s)
+                    value=(F / (e2e_ms * 1e-3) / 1e12) if sharded else job_tflops(F, world, e2e_ms), unit="TFLOP/s",
+                    h2d_bytes_per_step=Nm * wl.Ci * 2, d2h_bytes_per_step=Nm * wl.Co * 2, ms_per_step=e2e_ms),
+                gpu_launches=launches * args.steps, pack_seconds=pack_s)
+    if sharded:
+        line["shard"] = dict(frames=[f0, f1], tokens=Nm, cubes=int(lay.K))
     clk_sum = clk.summary()
     if clk_sum:
         line["clocks"] = clk_sum
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # the oracle on the machine's host cores: the whole tensor for the small layers, else a seeded
+        # sample of whole cubes under the whole tensor's delta scale, extrapolated by tokens
         import oracle
         oracle.build()
         L1, L2 = dq.dq_lowrank_factors(Wb, wl.rank)
         wq = oracle.quantize_weight(Wb, L1, L2)
-        dt, f, n = oracle_sample(wl, cube, X, Wb, L1, L2, wq, args.baseline_tokens)
-        line["cpu_baseline"] = dict(value=f / dt / 1e12, unit="TFLOP/s", cores=os.cpu_count(), kind="oracle",
-                                    sample=f"{n} tokens of {wl.name} (whole cubes of the first frames), "
-                                           f"Ci={wl.Ci}, Co={wl.Co}, r={wl.rank}, {dt:.1f} s")
+        layer = OracleLayer(wl, cube, X, L1, L2, wq)
+        cubes, full = oracle_sample_cubes(wl, cube)
+        dt, n = layer.run(cubes)
+        t_full = dt if full else layer.full_seconds(dt, n)
+        if full:
+            t_full += layer.stats_s
+        what = (f"the whole tensor ({n} tokens, {dt + layer.stats_s:.1f} s)" if full else
+                f"a seeded {cubes.size}-cube sample ({n} tokens, {dt:.1f} s) under the whole tensor's delta scale "
+                f"(statistics pass {layer.stats_s:.1f} s), extrapolated by tokens to {t_full:.0f} s for the layer")
+        line["cpu_baseline"] = dict(value=F / t_full / 1e12, unit="TFLOP/s", cores=layer.threads, kind="oracle",
+                                    sample=f"oracle over {what}; {wl.name}, Ci={wl.Ci}, Co={wl.Co}, r={wl.rank}",
+                                    sample_seconds=dt, extrapolated_full_seconds=None if full else t_full)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

@@ -72,6 +72,9 @@ def _L():
         lib.or_residual.argtypes = [P, P, P, I, I, I, P]
         lib.or_output_rows.argtypes = [P, P, F, P, P, P, I, P, P, P, F, I, I, P, P, P, I, P, LL, P]
         lib.or_fp8_kernel_tokens.argtypes = [P, LL, I, I, P, P]
+        lib.or_num_threads.restype = I
+        lib.or_delta_amax.argtypes = [P] + [I] * 7 + [P]
+        lib.or_quantize_cubes.argtypes = [P] + [I] * 7 + [P, LL, F, P, P, P, P, P]
         _lib = lib
     return _lib
 
@@ -219,6 +222,49 @@ def quantize_activations(X, T, H, W, cube, kernel_group: int = 0, pow2_scales: b
     if kernel_group:
         out["q8"], out["s8"] = fp8_kernel_tokens(out["means"], kernel_group)
     out.update(cube_order(T, H, W, *cube))
+    return out
+
+
+def num_threads() -> int:
+    """Threads the oracle's parallel loops use."""
+    return int(_L().or_num_threads())
+
+
+def delta_amax(X, T, H, W, cube) -> float:
+    """The whole tensor's max |delta| (cube means and deltas of Eq. 1 in fp32)."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    a = ctypes.c_float(0)
+    if _L().or_delta_amax(_p(X), T, H, W, X.shape[1], *cube, ctypes.byref(a)):
+        raise RuntimeError("or_delta_amax failed")
+    return float(a.value)
+
+
+def quantize_cubes(X, T, H, W, cube, cubes, S: float) -> dict:
+    """The activation side for the listed cubes only, under the per-tensor delta
+    scale S of the whole tensor (per-token kernel scales).  Returns a dict that
+    output_rows takes for the natural token rows of those cubes: compact delta rows
+    (list order, (t,h,w) inside a cube), compact kernel tokens, and N-long maps
+    row_of_n / cube_of_n into them (-1 outside the sample); `rows` lists the
+    sample's natural token indices in compact row order."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    N, Ci = X.shape
+    cubes = np.ascontiguousarray(cubes, dtype=np.int64)
+    o = cube_order(T, H, W, *cube)
+    counts = o["count"][cubes].astype(np.int64)
+    R = int(counts.sum())
+    out = dict(dcodes=np.empty((R, Ci // 2), np.uint8), dscales=np.empty((R, Ci // 16), np.uint8),
+               q8=np.empty((cubes.size, Ci), np.uint8), s8=np.empty(cubes.size, np.float32))
+    first = np.empty(cubes.size, np.int64)
+    if _L().or_quantize_cubes(_p(X), T, H, W, Ci, *cube, _p(cubes), cubes.size, float(S), _p(out["dcodes"]),
+                              _p(out["dscales"]), _p(out["q8"]), _p(out["s8"]), _p(first)):
+        raise RuntimeError("or_quantize_cubes failed")
+    rows = np.concatenate([o["n_of_row"][o["first"][k]:o["first"][k] + o["count"][k]] for k in cubes])
+    row_of_n = np.full(N, -1, np.int32)
+    row_of_n[rows] = np.arange(R, dtype=np.int32)
+    cube_of_n = np.full(N, -1, np.int32)
+    cube_of_n[rows] = np.repeat(np.arange(cubes.size, dtype=np.int32), counts)
+    out.update(S_delta=float(np.float32(S)), kernel_group=0, row_of_n=row_of_n, cube_of_n=cube_of_n,
+               rows=rows.astype(np.int64), first_row=first, cubes=cubes)
     return out
 
 

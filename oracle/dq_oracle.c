@@ -34,6 +34,7 @@
  * tolerance.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -464,6 +465,25 @@ int or_fp8_kernel_tokens(const float* means, long long K, int Ci, int group, uin
     return 0;
 }
 
+/* The global max |x - m| over every delta of the tensor (Eq. 1 deltas in fp32):
+ * the amax behind the per-tensor delta scale. */
+static float delta_amax(const uint16_t* X, const geom_t* g, const float* m) {
+    const int Ci = g->Ci;
+    float amax = 0.0f;
+#pragma omp parallel for reduction(max : amax) schedule(dynamic, 16)
+    for (long long k = 0; k < g->K; k++) {
+        const float* mk = m + (size_t)k * Ci;
+        for (int j = 0; j < g->count[k]; j++) {
+            const uint16_t* x = X + (size_t)g->n_of_row[g->first[k] + j] * Ci;
+            for (int c = 0; c < Ci; c++) {
+                float d = fabsf(or_bf16_value(x[c]) - mk[c]);
+                if (d > amax) amax = d;
+            }
+        }
+    }
+    return amax;
+}
+
 /*
  * The activation side of Eq. 2/3 for a whole X (N x Ci, natural order):
  *   dcodes  N x Ci/2   FP4 delta codes, rows in cube-major order
@@ -501,20 +521,7 @@ int or_quantize_activations_opt(const uint16_t* X, int T, int H, int W, int Ci, 
     float* m = means ? means : (float*)malloc(sizeof(float) * (size_t)g.K * Ci);
     if (!m) { geom_free(&g); return 2; }
     cube_means(X, &g, m);
-
-    /* global delta amax */
-    float amax = 0.0f;
-#pragma omp parallel for reduction(max : amax) schedule(dynamic, 16)
-    for (long long k = 0; k < g.K; k++) {
-        const float* mk = m + (size_t)k * Ci;
-        for (int j = 0; j < g.count[k]; j++) {
-            const uint16_t* x = X + (size_t)g.n_of_row[g.first[k] + j] * Ci;
-            for (int c = 0; c < Ci; c++) {
-                float d = fabsf(or_bf16_value(x[c]) - mk[c]);
-                if (d > amax) amax = d;
-            }
-        }
-    }
+    float amax = delta_amax(X, &g, m);
     float S = or_tensor_scale(amax);
     if (pow2 && amax != 0.0f) S = or_pow2_ceil(amax / 2688.0f);
     if (S_delta) *S_delta = S;
@@ -534,6 +541,70 @@ int or_quantize_activations_opt(const uint16_t* X, int T, int H, int W, int Ci, 
         free(z);
     }
     if (!means) free(m);
+    geom_free(&g);
+    return 0;
+}
+
+/*
+ * The statistics half of the activation side over the whole tensor: the cube
+ * means (Eq. 1) and the global max |delta|, from which the per-tensor delta
+ * scale follows.  Used with or_quantize_cubes to quantise a sample of cubes
+ * exactly as the whole tensor would be.
+ */
+int or_delta_amax(const uint16_t* X, int T, int H, int W, int Ci, int t, int h, int w, float* amax_delta) {
+    geom_t g;
+    if (geom_init(&g, T, H, W, t, h, w, Ci)) { geom_free(&g); return 2; }
+    float* m = (float*)malloc(sizeof(float) * (size_t)g.K * Ci);
+    if (!m) { geom_free(&g); return 2; }
+    cube_means(X, &g, m);
+    *amax_delta = delta_amax(X, &g, m);
+    free(m);
+    geom_free(&g);
+    return 0;
+}
+
+/*
+ * The activation side for the listed cubes only, under a given per-tensor
+ * delta scale S (the whole tensor's): for list entry i = cube k = cubes[i],
+ * its mean, its FP8 kernel token q8[i] / s8[i] (per-token scale), and its
+ * tokens' FP4 delta rows, written in list order and, inside a cube, in
+ * (t,h,w) order; first_row[i] = the first of cube i's rows in that order.
+ * The same arithmetic as or_quantize_activations row for row.
+ */
+int or_quantize_cubes(const uint16_t* X, int T, int H, int W, int Ci, int t, int h, int w, const long long* cubes,
+                      long long ncubes, float S, uint8_t* dcodes, uint8_t* dscales, uint8_t* q8, float* s8,
+                      long long* first_row) {
+    if (Ci % 16) return 1;
+    geom_t g;
+    if (geom_init(&g, T, H, W, t, h, w, Ci)) { geom_free(&g); return 2; }
+    long long row = 0;
+    for (long long i = 0; i < ncubes; i++) {
+        if (cubes[i] < 0 || cubes[i] >= g.K) { geom_free(&g); return 1; }
+        first_row[i] = row;
+        row += g.count[cubes[i]];
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long long i = 0; i < ncubes; i++) {
+        const long long k = cubes[i];
+        float* mk = (float*)malloc(sizeof(float) * (size_t)Ci);
+        float* z = (float*)malloc(sizeof(float) * (size_t)Ci);
+        for (int c = 0; c < Ci; c++) mk[c] = 0.0f;
+        for (int j = 0; j < g.count[k]; j++) {
+            const uint16_t* x = X + (size_t)g.n_of_row[g.first[k] + j] * Ci;
+            for (int c = 0; c < Ci; c++) mk[c] = mk[c] + or_bf16_value(x[c]);
+        }
+        const float cnt = (float)g.count[k];
+        for (int c = 0; c < Ci; c++) mk[c] = mk[c] / cnt;
+        fp8_token(mk, Ci, q8 + (size_t)i * Ci, s8 + i);
+        for (int j = 0; j < g.count[k]; j++) {
+            const uint16_t* x = X + (size_t)g.n_of_row[g.first[k] + j] * Ci;
+            const long long r = first_row[i] + j;
+            for (int c = 0; c < Ci; c++) z[c] = or_bf16_value(x[c]) - mk[c];
+            fp4_row(z, Ci, S, dcodes + (size_t)r * (Ci / 2), dscales + (size_t)r * (Ci / 16));
+        }
+        free(mk);
+        free(z);
+    }
     geom_free(&g);
     return 0;
 }
@@ -640,3 +711,6 @@ void or_e4m3_encode_array(const float* v, long long n, uint8_t* out) {
 #pragma omp parallel for schedule(static)
     for (long long i = 0; i < n; i++) out[i] = (uint8_t)or_e4m3_encode(v[i]);
 }
+
+/* Threads an OpenMP loop of this file uses (for reporting the CPU baseline). */
+int or_num_threads(void) { return omp_get_max_threads(); }

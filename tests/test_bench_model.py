@@ -3,6 +3,7 @@
 import os
 import sys
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -33,3 +34,17 @@ def test_stage_model_counts_both_reads_of_x():
     assert m["kernel_gemm"]["flops"] == 2.0 * 8190 * wl.Ci * wl.Co
     g = bench.stage_model(wl, 8190, 64, kernel_group=64)
     assert g["kernel_gemm"]["bytes"] > m["kernel_gemm"]["bytes"]  # hi + lo operand
+
+
+def test_cpu_baseline_sample():
+    """The CPU baseline's cube sample: the whole tensor for the small layers, else
+    512 distinct seeded cubes, the same on every call; per-row FLOPs add up to the
+    layer's."""
+    wl = synth.WORKLOADS["wan720p_ffn_down"]
+    a, full = bench.oracle_sample_cubes(wl, wl.cube)
+    b, _ = bench.oracle_sample_cubes(wl, wl.cube)
+    assert not full and a.size == 512 == np.unique(a).size and np.array_equal(a, b)
+    assert a.min() >= 0 and a.max() < 19320
+    t, full_t = bench.oracle_sample_cubes(synth.WORKLOADS["tiny"], (1, 2, 2))
+    assert full_t and np.array_equal(t, np.arange(64))
+    assert bench.layer_flops_rows(wl, 19320, wl.N) == pytest.approx(bench.layer_flops(wl, 19320), rel=1e-12)

@@ -65,7 +65,7 @@ def test_single_process_reduction_is_the_identity():
 def test_reference_arm_prints_on_rank_zero_only(rank):
     env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank))
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
-                        "--workload", "tiny", "--steps", "1", "--warmup", "3", "--sample-tokens", "16"],
+                        "--workload", "tiny", "--steps", "1", "--warmup", "3"],
                        env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.strip()]
@@ -75,3 +75,9 @@ def test_reference_arm_prints_on_rank_zero_only(rank):
         d = json.loads(lines[-1])
         assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
         assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+        # the reference arm names the same workload configuration as the GPU arm
+        sys.path.insert(0, ROOT)
+        import bench
+        import synth
+        wl = synth.WORKLOADS["tiny"]
+        assert d["config"] == bench.bench_config(wl, wl.cube, 64, 0, 2, "sharded")

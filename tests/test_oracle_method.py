@@ -594,3 +594,35 @@ def test_single_read_encode_with_fixup_equals_direct_encode():
             assert np.array_equal(fixed_scales, scalesS.astype(int))
             assert np.array_equal(fixed_codes, codesS)
     assert reencoded > 0      # the re-encode branch is exercised too
+
+
+# ------------------------------------------------------------------ sampled cubes (the CPU baseline's sample)
+
+@pytest.mark.parametrize("shape,cube", [((5, 9, 21), (2, 2, 2)), ((3, 10, 37), (1, 2, 2)), ((4, 6, 10), (4, 6, 10))])
+def test_sampled_cubes_match_the_whole_tensor(shape, cube):
+    """The CPU baseline quantises a seeded sample of cubes under the whole tensor's
+    delta scale: the whole-tensor statistics pass must give the same amax as the
+    full quantiser, the sampled cubes' codes, scales and kernel tokens the full
+    quantiser's rows bit for bit (ragged edge cubes included), and their Y rows
+    the full path's exactly."""
+    T, H, W = shape
+    wl = synth.Workload("sample", T, H, W, 256, 256, 16, cube, (T, 2, 2), (0.02, 40.0), (0.01, 20.0))
+    X = synth.activations(wl, seed=31)
+    act = oracle.quantize_activations(X, T, H, W, cube)
+    amax = oracle.delta_amax(X, T, H, W, cube)
+    assert np.float32(amax) == np.float32(act["amax_delta"])
+    assert np.float32(oracle.tensor_scale(amax)) == np.float32(act["S_delta"])
+    K = act["count"].size
+    ks = np.unique(np.r_[np.random.default_rng(3).choice(K, size=min(5, K), replace=False), K - 1])[::-1].copy()
+    sub = oracle.quantize_cubes(X, T, H, W, cube, ks, oracle.tensor_scale(amax))
+    rows_cm = np.concatenate([np.arange(act["first"][k], act["first"][k] + act["count"][k]) for k in ks])
+    assert np.array_equal(sub["dcodes"], act["dcodes"][rows_cm])
+    assert np.array_equal(sub["dscales"], act["dscales"][rows_cm])
+    assert np.array_equal(sub["q8"], act["q8"][ks]) and np.array_equal(sub["s8"], act["s8"][ks])
+    assert np.array_equal(sub["rows"], act["n_of_row"][rows_cm])
+    Wb = synth.weight(wl, seed=32)
+    L1, L2, _ = oracle.lowrank_factors(Wb, 16)
+    wq = oracle.quantize_weight(Wb, L1, L2)
+    y_sub = oracle.output_rows(sub, wq, X, L1, L2, sub["rows"])
+    y_full = oracle.output_rows(act, wq, X, L1, L2, sub["rows"])
+    assert np.array_equal(y_sub, y_full)

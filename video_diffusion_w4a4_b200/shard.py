@@ -35,21 +35,28 @@ def slab_cube(cube, T_slab: int) -> tuple[int, int, int]:
     return (min(t, T_slab), h, w)
 
 
-def forward_sharded(X_slab, T_slab: int, H: int, W: int, cube, Ci: int, Co: int, rank: int, packed_W, L1_mma,
-                    L2_slab, Y_slab, workspace, allreduce_max, stream=None) -> None:
-    """This rank's slab of the layer.  X_slab / Y_slab: the slab's rows (device, BF16 bits),
+def forward_sharded(X_slab, T_slab: int, H: int, W: int, cube, Ci: int, Co: int, lowrank: int, packed_W, L1_mma,
+                    L2_slab, Y_slab, workspace, allreduce_max, stream=None, stage_events=None,
+                    start_event=None) -> None:
+    """This process's slab of the layer.  X_slab / Y_slab: the slab's rows (device, BF16 bits),
+    lowrank: the rank r of the low-rank factors L1, L2 (not the process's distributed rank),
     workspace: a uint8 device tensor of at least dq_workspace_bytes for the slab.  allreduce_max
     takes the slab's max |delta| as a one-element float32 tensor viewing the workspace and must
     leave the maximum over all ranks in it (e.g. torch.distributed.all_reduce(..., ReduceOp.MAX)
-    on the stream's device)."""
+    on the stream's device).  stage_events (optional, 4 created CUDA events) time the encode
+    stage and the two products as dq_linear_forward_ex does; start_event (optional) is recorded
+    on the stream before the statistics pass."""
     import torch
     t, h, w = slab_cube(cube, T_slab)
-    lay = dq.dq_workspace_layout_get(T_slab, H, W, t, h, w, Ci, Co, rank)
+    lay = dq.dq_workspace_layout_get(T_slab, H, W, t, h, w, Ci, Co, lowrank)
     nbytes = lay.total_bytes
     if workspace.numel() < nbytes:
         raise ValueError(f"workspace of {workspace.numel()} bytes, the slab needs {nbytes}")
-    args = (X_slab, T_slab, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y_slab, workspace, nbytes)
+    args = (X_slab, T_slab, H, W, t, h, w, Ci, Co, lowrank, packed_W, L1_mma, L2_slab, Y_slab, workspace, nbytes)
+    if start_event is not None:
+        start_event.record(stream)
     dq.dq_linear_forward_ex(*args, dq.DQ_STAGE_STATS, None, stream)
     amax = workspace[lay.off_scalars:lay.off_scalars + 4].view(torch.float32)
     allreduce_max(amax)
-    dq.dq_linear_forward_ex(*args, dq.DQ_STAGE_ENCODE | dq.DQ_STAGE_KERNEL_GEMM | dq.DQ_STAGE_MAIN_GEMM, None, stream)
+    dq.dq_linear_forward_ex(*args, dq.DQ_STAGE_ENCODE | dq.DQ_STAGE_KERNEL_GEMM | dq.DQ_STAGE_MAIN_GEMM,
+                            stage_events, stream)
