@@ -344,20 +344,29 @@ int dq_linear_forward_host(const void* X_host, int T, int H, int W, int t, int h
  * dq_workspace_bytes exceeds 32 MiB are refused with
  * DQ_ERR_WORKSPACE_TOO_SMALL before anything is launched.  No cudaMalloc,
  * cudaFree or other allocating call is made.
- * The first call on a device looks up the array's device address and clears
- * its status word (a short synchronous call): make that first call before any
- * stream capture.  All calls share the one array and it keeps the previous
- * call's contents; calls that may overlap on the GPU (different streams
- * without ordering) race on it.  Device-side errors (bounded waits that ran
- * out) are written to the array's status word, which this entry point cannot
- * read back.
+ * The first call on a device looks up the array's device address (no stream
+ * operation); make that first call before any stream capture all the same,
+ * since the lookup may load the library's device code.  All calls share the
+ * one array and it keeps the previous call's contents: each call clears the
+ * status word and the accumulators it needs on its own stream, so calls
+ * ordered on one stream are independent, but calls that may overlap on the GPU
+ * (different streams without ordering) race on it.  Device-side errors (a
+ * packed weight that does not match, a bounded wait that ran out) go to the
+ * array's status word: read it with
+ * dq_read_device_status(DQ_NOALLOC_WORKSPACE, stream, ...).
  */
 int dq_linear_forward_noalloc(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
                               const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y, void* stream);
 
+/* The workspace argument of dq_read_device_status that names the fixed array
+ * of dq_linear_forward_noalloc. */
+#define DQ_NOALLOC_WORKSPACE ((const void*)1)
+
 /*
  * Synchronises `stream`, reads the workspace status word into *status, and
- * clears it when `clear` is nonzero.  workspace NULL = the library workspace.
+ * clears it when `clear` is nonzero.  workspace: a caller workspace, NULL for
+ * the library workspace of dq_linear_forward (DQ_OK when none exists yet), or
+ * DQ_NOALLOC_WORKSPACE for the array of dq_linear_forward_noalloc.
  */
 int dq_read_device_status(const void* workspace, void* stream, int* status, int clear);
 

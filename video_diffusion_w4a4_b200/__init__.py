@@ -36,6 +36,7 @@ DQ_ERR_ALLOC = 9
 DQ_STAGE_QUANTIZE, DQ_STAGE_KERNEL_GEMM, DQ_STAGE_MAIN_GEMM, DQ_STAGE_ALL = 1, 2, 4, 7
 DQ_STAGE_STATS, DQ_STAGE_ENCODE = 8, 16
 DQ_KERNEL_SCALE_PER_TOKEN, DQ_KERNEL_SCALE_GROUP64 = 0, 64
+DQ_NOALLOC_WORKSPACE = 1   # dq_read_device_status: the fixed array of dq_linear_forward_noalloc
 
 
 class dq_packed_layout(ctypes.Structure):

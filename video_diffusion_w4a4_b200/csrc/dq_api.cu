@@ -408,7 +408,12 @@ int dq_read_device_status(const void* workspace, void* stream, int* status, int 
     if (!status) return DQ_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     const void* ws = workspace;
-    if (!ws) {
+    if (ws == DQ_NOALLOC_WORKSPACE) {
+        void* p = nullptr;
+        const int rc = dq::noalloc_workspace(&p);
+        if (rc) return rc;
+        ws = p;
+    } else if (!ws) {
         int dev = 0;
         if (cudaGetDevice(&dev) != cudaSuccess) return DQ_ERR_NO_DEVICE;
         std::lock_guard<std::mutex> lk(g_ws_mu);

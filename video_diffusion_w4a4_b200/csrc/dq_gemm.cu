@@ -41,6 +41,8 @@
 // per ring stage), so it keeps one accumulator: its epilogue warps copy their
 // slice into registers, release tensor memory, and then fetch P' and write Y
 // while the next tile's MMAs run.
+#include <atomic>
+
 #include "dq_common.h"
 #include "dq_internal.h"
 #include "dq_ptx.cuh"
@@ -430,6 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 namespace {
 
+constexpr int kMaxDevices = 64;
+
 template <bool kMain>
 cudaError_t launch_pairs(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_sa,
                          const CUtensorMap& tm_sb, const CUtensorMap& tm_fa, const CUtensorMap& tm_fb,
@@ -449,8 +453,14 @@ cudaError_t launch_pairs(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // persistent: as many pairs as can be resident at once (one CTA per SM)
-    static int mp = 0;
+    // persistent: as many pairs as can be resident at once (one CTA per SM), queried once per
+    // device (concurrent first calls may both query; they store the same answer)
+    static std::atomic<int> resident[kMaxDevices];
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    int mp = resident[dev].load(std::memory_order_relaxed);
     if (mp == 0) {
         cfg.gridDim = dim3(2 * tiles);
         int n = 0;
@@ -458,6 +468,7 @@ cudaError_t launch_pairs(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const
         if (e != cudaSuccess) return e;
         if (n <= 0) return cudaErrorInvalidConfiguration;
         mp = n;
+        resident[dev].store(mp, std::memory_order_relaxed);
     }
     cfg.gridDim = dim3(2 * imin(tiles, mp));
     return cudaLaunchKernelEx(&cfg, k_gemm<kMain>, tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p);

@@ -70,6 +70,10 @@ cudaError_t launch_main_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, c
                              const CUtensorMap& tm_sb, const CUtensorMap& tm_fa, const CUtensorMap& tm_fb,
                              const GemmParams& p, cudaStream_t st);
 
+// Device address of the no-allocation entry point's fixed workspace on the
+// current device (dq_noalloc.cu); a dq_status code.
+int noalloc_workspace(void** out);
+
 cudaError_t launch_selftest_wait(int* status, uint64_t budget_ns, cudaStream_t st);
 cudaError_t launch_selftest_divide(long long n, uint64_t seed, unsigned long long* mismatches, float* first,
                                    cudaStream_t st);

@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "../../include/deltaquant.h"
+#include "dq_internal.h"
 
 namespace {
 
@@ -26,27 +27,30 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_addr[kMaxDevices] = {};
 
+bool aligned256(const void* p) { return ((uintptr_t)p & 255u) == 0; }
+
+}  // namespace
+
+namespace dq {
+
 // Device address of the array on the current device.  Host code may not use
 // the symbol itself as a pointer (it names a host-side stand-in), so the
 // address is looked up once per device, with that device current, and cached.
-// The first lookup also zeroes the status word at the start of the array.
-int static_workspace(void** out) {
+// The lookup is not a stream operation and writes nothing to the device.
+int noalloc_workspace(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DQ_ERR_NO_DEVICE;
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_addr[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || !p) return DQ_ERR_CUDA;
-        if (cudaMemset(p, 0, 256) != cudaSuccess) return DQ_ERR_CUDA;
         g_addr[dev] = p;
     }
     *out = g_addr[dev];
     return DQ_OK;
 }
 
-bool aligned256(const void* p) { return ((uintptr_t)p & 255u) == 0; }
-
-}  // namespace
+}  // namespace dq
 
 extern "C" int dq_linear_forward_noalloc(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co,
                                          int rank, const void* packed_W, const void* L1_mma, const void* L2_slab,
@@ -59,12 +63,14 @@ extern "C" int dq_linear_forward_noalloc(const void* X, int T, int H, int W, int
     if (!aligned256(X) || !aligned256(packed_W) || !aligned256(L1_mma) || !aligned256(L2_slab) || !aligned256(Y))
         return DQ_ERR_ALIGNMENT;
     void* ws = nullptr;
-    rc = static_workspace(&ws);
+    rc = dq::noalloc_workspace(&ws);
     if (rc) return rc;
     // The array keeps the previous call's contents.  Every scratch tensor of the
     // forward is fully rewritten by it, and the accumulators that must start at
     // zero (the amax words) are cleared by the forward's first stage; the status
-    // word is cleared here so that an earlier call's error does not carry over.
+    // word is cleared here, on the caller's stream, so that an earlier call's
+    // error does not carry over (dq_read_device_status(DQ_NOALLOC_WORKSPACE, ...)
+    // reads it after the call).
     if (cudaMemsetAsync(ws, 0, sizeof(int), (cudaStream_t)stream) != cudaSuccess) return DQ_ERR_CUDA;
     return dq_linear_forward_ex(X, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y, ws,
                                 kStaticWorkspaceBytes, DQ_STAGE_ALL, nullptr, stream);
