@@ -43,24 +43,30 @@ import synth  # noqa: E402
 
 METRIC = "W4A4 DeltaQuant linear TFLOPS & tokens/s; % of dense FP4 / HBM roofline"
 FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+FP8_PER_BF16 = 2.0  # nominal dense FP8 : BF16 (4.5 : 2.25 PFLOP/s)
 
 
 def layer_flops(wl, K):
     return 2.0 * wl.N * wl.Ci * wl.Co + 2.0 * K * wl.Ci * wl.Co + 2.0 * wl.N * wl.rank * (wl.Ci + wl.Co)
 
 
-def stage_model(wl, K, slab, kernel_group=0):
+def stage_model(wl, K, slab, kernel_group=0, fp8=False):
     """Algorithmic work per launch of each stage (bytes that must cross HBM,
     tensor FLOPs).  Stage 1 reads X twice (statistics, then encode: the
-    per-tensor delta scale needs every delta first)."""
+    per-tensor delta scale needs every delta first).  fp8: the FP8 kernel-token
+    product reads q8 and the FP8 weight (1 byte each) plus one exponent per 32."""
     N, Ci, Co, r = wl.N, wl.Ci, wl.Co, wl.rank
+    q8_copy = 0 if fp8 else (4 if kernel_group else 2)   # BF16 operand of the exact product (hi + lo when grouped)
     quant_bytes = (4.0 * N * Ci                      # X read by a1 and a2
                    + N * Ci / 2 + N * Ci / 16        # delta codes + scales
-                   + K * Ci * (5 if kernel_group else 3)  # q8 (E4M3) + its BF16 copy (hi + lo when grouped)
+                   + K * Ci * (1 + q8_copy)          # q8 (E4M3) + the product's BF16 operand
                    + N * r * 4 * 2                   # X L1 partials (write + read)
                    + N * slab * 2 + 2 * r * Ci)      # U hi/lo, L1
     kernel_flops = 2.0 * K * Ci * Co
-    kernel_bytes = K * Ci * (4 if kernel_group else 2) + Co * Ci * 2 + K * Co * 4
+    if fp8:
+        kernel_bytes = K * Ci + Co * Ci + Co * Ci / 32 + K * Co * 4
+    else:
+        kernel_bytes = K * Ci * (4 if kernel_group else 2) + Co * Ci * 2 + K * Co * 4
     main_flops = 2.0 * N * Ci * Co + 2.0 * N * slab * Co
     main_bytes = N * Ci * 9 / 16 + Co * Ci * 9 / 16 + N * slab * 2 + Co * slab * 2 + K * Co * 4 + N * Co * 2
     return dict(quantize=dict(bytes=quant_bytes, flops=2.0 * N * Ci * r),
@@ -216,10 +222,11 @@ class OracleLayer:
         return self.stats_s + sample_s * self.wl.N / sample_tokens
 
 
-def bench_config(wl, cube, K, kernel_group, world, parallelism):
+def bench_config(wl, cube, K, kernel_group, world, parallelism, fp8=False):
     """The `config` object of the JSON line, identical for the GPU arm and the reference arm."""
     return dict(workload=wl.name, T=wl.T, H=wl.H, W=wl.W, N=wl.N, Ci=wl.Ci, Co=wl.Co, rank=wl.rank, cube=list(cube),
                 K=K, kernel_scale="per-token" if not kernel_group else f"group{kernel_group}",
+                kernel_product="fp8 (restricted-scale C2 weights)" if fp8 else "bf16 (exact)",
                 parallelism=(f"cube-sharded x{world} (T-slabs of whole cube layers, NCCL all-reduce(max) of the "
                              f"delta amax)" if parallelism == "sharded" and world > 1
                              else f"dp{world} (independent layer per GPU)"),
@@ -235,7 +242,8 @@ def run_reference(args, wl, cube):
     X = synth.activations(wl)
     Wb = synth.weight(wl)
     L1, L2, _ = oracle.lowrank_factors(Wb, wl.rank)
-    wq = oracle.quantize_weight(Wb, L1, L2)
+    fp8 = args.kernel_product == "fp8"
+    wq = oracle.quantize_weight(Wb, L1, L2, c2=fp8)
     layer = OracleLayer(wl, cube, X, L1, L2, wq)
     cubes, full = oracle_sample_cubes(wl, cube)
     if wl.name == "tiny":
@@ -262,7 +270,7 @@ def run_reference(args, wl, cube):
                 warmup=args.warmup, ms_per_step=sample_s / args.steps * 1e3, higher_is_better=True,
                 scaling="weak" if args.gpus == 1 or args.parallelism == "replicas" else "strong",
                 vs_baseline=None, dtype="f64", data="synthetic",
-                config=bench_config(wl, cube, K, args.kernel_group, args.gpus, args.parallelism),
+                config=bench_config(wl, cube, K, args.kernel_group, args.gpus, args.parallelism, fp8),
                 tokens_per_s=wl.N / t_full, sample_tflops=sum(layer_flops_rows(wl, K, n) for n in toks) / sample_s / 1e12,
                 cpu_baseline=dict(value=value, unit="TFLOP/s", cores=layer.threads, kind="oracle", sample=sample,
                                   sample_seconds=sample_s, extrapolated_full_seconds=t_full),
@@ -290,6 +298,8 @@ def main():
     ap.add_argument("--frames", type=int, default=None, help="override T (smaller cases for profiling)")
     ap.add_argument("--kernel-group", type=int, default=0, choices=[0, 64],
                     help="FP8 kernel-token scales: 0 = one per token, 64 = one per 64 channels")
+    ap.add_argument("--kernel-product", default="bf16", choices=["bf16", "fp8"],
+                    help="kernel-token product: exact BF16 operands (default) or FP8 on restricted-scale (C2) weights")
     ap.add_argument("--parallelism", default="sharded", choices=["sharded", "replicas"],
                     help="with several GPUs: one layer sharded by cubes (default) or one layer per GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -324,8 +334,12 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     sharded = world > 1 and args.parallelism == "sharded"
     kg = args.kernel_group
-    if sharded and kg:
-        ap.error("the cube-sharded layer takes per-token kernel scales")
+    fp8 = args.kernel_product == "fp8"
+    kp = dq.DQ_KERNEL_PRODUCT_FP8 if fp8 else dq.DQ_KERNEL_PRODUCT_BF16
+    if sharded and (kg or fp8):
+        ap.error("the cube-sharded layer takes per-token kernel scales and the BF16 kernel-token product")
+    if fp8 and kg:
+        ap.error("the FP8 kernel-token product takes per-token kernel scales")
 
     t, h, w = cube
     K = dq.dq_cube_count(wl.T, wl.H, wl.W, t, h, w)
@@ -334,7 +348,11 @@ def main():
     X = synth.activations(wl, tau=0 if sharded else rank)
     Wb = synth.weight(wl)
     t0 = time.perf_counter()
-    packed, L1m, L2s = dq.dq_pack_weight(Wb, wl.rank)
+    if fp8:
+        L1f, L2f = dq.dq_lowrank_factors(Wb, wl.rank)
+        packed, L1m, L2s, _ = dq.dq_pack_weight_factors(Wb, L1f, L2f, pack_flags=dq.DQ_PACK_C2)
+    else:
+        packed, L1m, L2s = dq.dq_pack_weight(Wb, wl.rank)
     pack_s = time.perf_counter() - t0
     if sharded:
         f0, f1 = shard.slab_frames(wl.T, t, world, rank)
@@ -349,7 +367,8 @@ def main():
     L1d = torch.from_numpy(L1m.view(np.int16)).to(dev)
     L2d = torch.from_numpy(L2s.view(np.int16)).to(dev)
     Yd = torch.empty((Nm, wl.Co), dtype=torch.int16, device=dev)
-    lay = dq.dq_workspace_layout_grouped(Ts, wl.H, wl.W, ts, hs, ws_, wl.Ci, wl.Co, wl.rank, kg)
+    lay = dq.dq_workspace_layout_opts(Ts, wl.H, wl.W, ts, hs, ws_, wl.Ci, wl.Co, wl.rank, kernel_group=kg,
+                                      kernel_product=kp)
     ws = torch.zeros(lay.total_bytes, dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream(dev)
 
@@ -358,8 +377,8 @@ def main():
 
     def step(events=None, pre=None):
         if not sharded:
-            dq.dq_linear_forward_grouped(Xd, Ts, wl.H, wl.W, ts, hs, ws_, wl.Ci, wl.Co, wl.rank, kg, Pd, L1d, L2d, Yd,
-                                         ws, lay.total_bytes, dq.DQ_STAGE_ALL, events, st)
+            dq.dq_linear_forward_opts(Xd, Ts, wl.H, wl.W, ts, hs, ws_, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd, ws,
+                                      lay.total_bytes, dq.DQ_STAGE_ALL, events, st, kernel_group=kg, kernel_product=kp)
             return
         # the cube-sharded layer: statistics of this slab, the one exchanged scalar (NCCL), then
         # encode and both products
@@ -419,7 +438,7 @@ def main():
         Yh.copy_(Yd2, non_blocking=True)
 
     e2e_ms = None
-    if not kg:   # the host-buffer entry point takes per-token kernel scales
+    if not kg and not fp8:   # the host-buffer entry point takes the default options
         e2e_step()
         torch.cuda.synchronize(dev)
         if dist:
@@ -443,22 +462,24 @@ def main():
     # per-stage work model of this rank's share (its slab when sharded)
     wl_mine = wl if not sharded else synth.Workload(wl.name, Ts, wl.H, wl.W, wl.Ci, wl.Co, wl.rank, (ts, hs, ws_),
                                                     wl.grid, wl.x_outliers, wl.w_outliers, wl.gelu)
-    model = stage_model(wl_mine, int(lay.K), lay.slab, kg)
+    model = stage_model(wl_mine, int(lay.K), lay.slab, kg, fp8)
     # dominant kernel = the stage with the largest share of the step
     dom = max(("quantize", "kernel_gemm", "main_gemm"), key=stage_ms.get)
     if dom == "quantize":
         ach = model[dom]["bytes"] / (stage_ms[dom] * 1e-3) / 1e9
         roof = dict(kernel="k_cube_stats+k_cube_encode", bound="hbm", achieved=ach, peak=peaks["hbm"], unit="GB/s")
     else:
-        pk = fp4_peak if dom == "main_gemm" else peaks["bf16"]
+        # the kernel-token product's own kind: BF16, or FP8 at 2 x the BF16 rate (nominal 4.5 : 2.25)
+        pk = fp4_peak if dom == "main_gemm" else peaks["bf16"] * (FP8_PER_BF16 if fp8 else 1.0)
         ach = model[dom]["flops"] / (stage_ms[dom] * 1e-3) / 1e12
         roof = dict(kernel="k_gemm<true> (main FP4 product)" if dom == "main_gemm" else "k_gemm<false> (kernel-token product)",
                     bound="tensor", achieved=ach, peak=pk, unit="TFLOP/s")
     roof["frac"] = roof["achieved"] / roof["peak"]
     same_cube = tuple(cube) == tuple(synth.WORKLOADS[args.workload].cube)
-    roof["traffic"] = committed_traffic(wl_mine, dom) if same_cube and not kg else None
+    roof["traffic"] = committed_traffic(wl_mine, dom) if same_cube and not kg and not fp8 else None
     roof["peak_source"] = ("measured" if peaks["source"] == "measured" else "fallback") + (
-        " bf16 x 4 (nominal FP4:BF16)" if roof["unit"] == "TFLOP/s" and dom == "main_gemm" else "")
+        " bf16 x 4 (nominal FP4:BF16)" if roof["unit"] == "TFLOP/s" and dom == "main_gemm" else
+        " bf16 x 2 (nominal FP8:BF16)" if roof["unit"] == "TFLOP/s" and fp8 else "")
     stages = {}
     for n, tms in stage_ms.items():
         if n not in model:
@@ -468,6 +489,8 @@ def main():
         stages[n] = dict(ms=tms, tflops=m["flops"] / (tms * 1e-3) / 1e12, gbs=m["bytes"] / (tms * 1e-3) / 1e9)
     stages["quantize"]["frac_hbm"] = stages["quantize"]["gbs"] / peaks["hbm"]
     stages["kernel_gemm"]["frac_bf16"] = stages["kernel_gemm"]["tflops"] / peaks["bf16"]
+    if fp8:
+        stages["kernel_gemm"]["frac_fp8"] = stages["kernel_gemm"]["tflops"] / (peaks["bf16"] * FP8_PER_BF16)
     stages["main_gemm"]["frac_fp4"] = stages["main_gemm"]["tflops"] / fp4_peak
     layer_bytes = sum(m["bytes"] for m in model.values())
     F_mine = layer_flops(wl_mine, int(lay.K))
@@ -476,7 +499,7 @@ def main():
     line = dict(metric=METRIC, value=value, unit="TFLOP/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
                 ms_per_step=ms, higher_is_better=True, scaling="strong" if sharded else "weak", vs_baseline=None,
                 dtype="e2m1/e4m3->f32", data="synthetic",
-                config=bench_config(wl, cube, K, kg, world, args.parallelism),
+                config=bench_config(wl, cube, K, kg, world, args.parallelism, fp8),
                 tokens_per_s=wl.N * (1 if sharded else world) / (ms * 1e-3),
                 layer_roofline_frac=layer_roof_ms / ms,
                 roofline=roof, stages=stages,
@@ -495,7 +518,7 @@ def main():
         import oracle
         oracle.build()
         L1, L2 = dq.dq_lowrank_factors(Wb, wl.rank)
-        wq = oracle.quantize_weight(Wb, L1, L2)
+        wq = oracle.quantize_weight(Wb, L1, L2, c2=fp8)
         layer = OracleLayer(wl, cube, X, L1, L2, wq)
         cubes, full = oracle_sample_cubes(wl, cube)
         dt, n = layer.run(cubes)

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define DQ_ABI_VERSION 2
+#define DQ_ABI_VERSION 3
 #define DQ_PACK_FORMAT_VERSION 3
 #define DQ_PACK_MAGIC 0x31575144u /* "DQW1" little-endian */
 
@@ -199,6 +199,36 @@ int dq_pack_weight_factors(const uint16_t* W, const uint16_t* L1, const uint16_t
                            uint16_t* L2_slab, float* S_W);
 
 /*
+ * Packing options (pack_flags of dq_pack_weight_factors_ex):
+ *   DQ_PACK_C2  restricted group scales for an FP8-rate kernel-token product
+ *               (DQ_KERNEL_PRODUCT_FP8).  The note runs the kernel-token product
+ *               on FP8 tensor cores; with Eq. 4's E4M3 group-16 scales the
+ *               product q s_b needs up to 6 significant bits, which no FP8
+ *               operand holds.  C2 rounds each group scale up to the nearest
+ *               {1, 1.5} x 2^e (e >= -9, 1.5 x 2^-9 excluded), caps it at 384,
+ *               takes S_W = amax(R) / (6 * 384), and per 32 channels raises the
+ *               smaller of the two scales to at least 2^-10 times the larger;
+ *               then every q s_b of a 32-channel block is an E4M3 value times
+ *               one power of two 2^u.  The blob's dqw section then holds, in
+ *               place of BF16 q s_b: Co x Ci E4M3 codes of q s_b / 2^u (u such
+ *               that the block's largest |q s_b| / 2^u lies in [256, 512)),
+ *               followed by the exponents u + 127 (UE8M0) in the layout
+ *               dq_sfb_offset gives for a Co x (Ci / 2) matrix, block j of that
+ *               matrix standing for 32-channel block j (four copies, one per
+ *               tensor-memory quadrant, as for the weight scales).  Header flag
+ *               bit 1 marks such a blob.  The price is accuracy: rounding scales
+ *               up leaves the top E2M1 codes unused in many groups (weight
+ *               error about 1.2 to 1.5 times Eq. 4's on the synthetic weights).
+ */
+#define DQ_PACK_C2 1
+
+/* dq_pack_weight_factors with pack_flags (0 or DQ_PACK_C2; anything else:
+ * DQ_ERR_INVALID_ARG). */
+int dq_pack_weight_factors_ex(const uint16_t* W, const uint16_t* L1, const uint16_t* L2, int Co, int Ci, int rank,
+                              int pack_flags, void* packed, size_t packed_bytes, uint16_t* L1_mma, uint16_t* L2_slab,
+                              float* S_W);
+
+/*
  * Set (bias != NULL) or clear (bias == NULL) the bias of a packed blob in
  * host memory: bias is host, Co BF16 values; Co must equal the blob's Co and
  * packed_bytes its total size.  The forward pass then returns x W^T + b: the
@@ -228,7 +258,8 @@ int dq_pack_weight(const uint16_t* W, int Co, int Ci, int rank, void* packed, si
  *   q8         K x Ci E4M3 kernel tokens
  *   q8_bf16    the kernel-token product's A operand: K_pad x Ci BF16 copy of q8
  *              (per-token), or K_pad x 2Ci BF16 q8*s8 split as hi (columns
- *              0..Ci-1) + lo (Ci..2Ci-1), |hi + lo - q8 s8| <= 2^-16 |q8 s8| (group 64)
+ *              0..Ci-1) + lo (Ci..2Ci-1), |hi + lo - q8 s8| <= 2^-16 |q8 s8| (group 64);
+ *              empty with DQ_KERNEL_PRODUCT_FP8, whose A operand is q8 itself
  *   dcodes     N x Ci/2 E2M1 delta codes, cube-major rows
  *   dscales    delta group scales, A-operand scale layout (dq_sfa_offset) over N rows
  *   u_part     splits x N x rank fp32 partial sums of X L1 (cube-major rows)
@@ -321,6 +352,39 @@ int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, 
                               int kernel_group, const void* packed_W, const void* L1_mma, const void* L2_slab,
                               void* Y, void* workspace, size_t workspace_bytes, int stage_mask,
                               void* const* stage_events, void* stream);
+
+/*
+ * Forward options (dq_linear_forward_opts, dq_workspace_layout_opts):
+ *   kernel_group    DQ_KERNEL_SCALE_PER_TOKEN or DQ_KERNEL_SCALE_GROUP64
+ *   kernel_product  DQ_KERNEL_PRODUCT_BF16: the kernel-token product on exact
+ *                   BF16 operands (q8 widened, q s_b), kind::f16; any packed weight
+ *                   without DQ_PACK_C2.
+ *                   DQ_KERNEL_PRODUCT_FP8: q8 (E4M3) times the FP8 form of
+ *                   DQ_PACK_C2 weights with UE8M0 scales per 32 channels,
+ *                   kind::mxf8f6f4, at twice the BF16 rate; per-token kernel
+ *                   scales only.  The product is the same exact sum as with
+ *                   BF16 operands of the same (C2) weights.
+ *   reserved        must be 0
+ * A packed weight whose C2 flag does not match kernel_product is reported as
+ * DQ_ERR_BAD_PACKED_WEIGHT in the device status word.
+ */
+#define DQ_KERNEL_PRODUCT_BF16 0
+#define DQ_KERNEL_PRODUCT_FP8 1
+
+typedef struct dq_forward_options {
+    int kernel_group;
+    int kernel_product;
+    int reserved[2];
+} dq_forward_options;
+
+int dq_workspace_layout_opts(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                             const dq_forward_options* opts, dq_workspace_layout* out);
+
+/* dq_linear_forward_grouped with forward options (opts NULL: the defaults, all 0). */
+int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                           const dq_forward_options* opts, const void* packed_W, const void* L1_mma,
+                           const void* L2_slab, void* Y, void* workspace, size_t workspace_bytes, int stage_mask,
+                           void* const* stage_events, void* stream);
 
 /*
  * As dq_linear_forward_ex with HOST X and Y (pinned for asynchronous copies):

@@ -83,9 +83,12 @@ def assert_y_close(y_bits: np.ndarray, y_ref: np.ndarray, what: str = "Y") -> di
 class Case:
     """One layer instance: workload, inputs, oracle factors."""
 
-    def __init__(self, wl: synth.Workload, cube=None, seed=None, tau: int = 0, X=None, Wb=None, kernel_group: int = 0):
+    def __init__(self, wl: synth.Workload, cube=None, seed=None, tau: int = 0, X=None, Wb=None, kernel_group: int = 0,
+                 fp8_product: bool = False):
         self.wl = wl
         self.kernel_group = kernel_group
+        # the FP8 kernel-token product: weights packed with restricted (C2) scales
+        self.fp8_product = fp8_product
         self.cube = tuple(cube or wl.cube)
         self.X = synth.activations(wl, seed=seed, tau=tau) if X is None else X
         self.Wb = synth.weight(wl, seed=seed) if Wb is None else Wb
@@ -94,7 +97,8 @@ class Case:
     # ---------------------------------------------------------------- GPU
     def run_gpu(self, dq, torch, stage_mask=7, packed_override=None, bias=None):
         wl, (t, h, w) = self.wl, self.cube
-        packed, L1m, L2s, S_W = dq.dq_pack_weight_factors(self.Wb, self.L1, self.L2)
+        packed, L1m, L2s, S_W = dq.dq_pack_weight_factors(self.Wb, self.L1, self.L2,
+                                                          pack_flags=dq.DQ_PACK_C2 if self.fp8_product else 0)
         if bias is not None:
             dq.dq_pack_bias(packed, bias)
         if packed_override is not None:
@@ -106,9 +110,15 @@ class Case:
         L2d = torch.from_numpy(L2s.view(np.int16)).to(dev)
         Yd = torch.empty((wl.N, wl.Co), dtype=torch.int16, device=dev)
         kg = self.kernel_group
-        lay = dq.dq_workspace_layout_grouped(wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, kg)
+        kp = dq.DQ_KERNEL_PRODUCT_FP8 if self.fp8_product else dq.DQ_KERNEL_PRODUCT_BF16
+        lay = dq.dq_workspace_layout_opts(wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, kernel_group=kg,
+                                          kernel_product=kp)
         ws = torch.zeros(lay.total_bytes, dtype=torch.uint8, device=dev)
-        if kg:
+        if self.fp8_product:
+            dq.dq_linear_forward_opts(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd, ws,
+                                      lay.total_bytes, stage_mask, None, torch.cuda.current_stream(),
+                                      kernel_group=kg, kernel_product=kp)
+        elif kg:
             dq.dq_linear_forward_grouped(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, kg, Pd, L1d, L2d, Yd,
                                          ws, lay.total_bytes, stage_mask, None, torch.cuda.current_stream())
         else:
@@ -126,7 +136,8 @@ class Case:
                    S_delta=wsh[lay.off_scalars + 4:lay.off_scalars + 8].view(np.float32)[0],
                    s8=wsh[lay.off_s8:lay.off_s8 + 4 * K * ns8].view(np.float32).reshape((K, ns8) if kg else (K,)),
                    q8=wsh[lay.off_q8:lay.off_q8 + K * Ci].reshape(K, Ci),
-                   q8_bf16=wsh[lay.off_q8_bf16:lay.off_q8_bf16 + 2 * K * acols].view(np.uint16).reshape(K, acols),
+                   q8_bf16=None if self.fp8_product else
+                   wsh[lay.off_q8_bf16:lay.off_q8_bf16 + 2 * K * acols].view(np.uint16).reshape(K, acols),
                    dcodes=wsh[lay.off_dcodes:lay.off_dcodes + N * Ci // 2].reshape(N, Ci // 2),
                    dscales=sfa_unpermute(wsh[lay.off_dscales:], N, Ci),
                    p=wsh[lay.off_p:lay.off_p + 4 * K * wl.Co].view(np.float32).reshape(K, wl.Co))
@@ -136,7 +147,7 @@ class Case:
     def run_oracle(self):
         wl = self.wl
         act = oracle.quantize_activations(self.X, wl.T, wl.H, wl.W, self.cube, kernel_group=self.kernel_group)
-        wq = oracle.quantize_weight(self.Wb, self.L1, self.L2)
+        wq = oracle.quantize_weight(self.Wb, self.L1, self.L2, c2=self.fp8_product)
         return act, wq
 
     def oracle_rows(self, act, wq, rows, bias=None):
@@ -160,7 +171,9 @@ def compare_quantised(g: dict, act: dict, wq: dict) -> None:
     assert np.array_equal(g["s8"], act["s8"]), "s8"
     bad = np.argwhere(g["q8"] != act["q8"])
     assert bad.size == 0, ("q8", bad[:5].tolist(), g["q8"][tuple(bad[0])], act["q8"][tuple(bad[0])])
-    if act.get("kernel_group"):
+    if g["q8_bf16"] is None:
+        pass   # the FP8 kernel-token product reads q8 itself: no BF16 operand
+    elif act.get("kernel_group"):
         # the product's operand: q8 s8 as BF16 hi + lo, within 2^-16 of the exact product
         Ci = act["q8"].shape[1]
         want = oracle.kernel_tokens_dequantized(act, "fp8")

@@ -132,6 +132,50 @@ def test_parity_group64_kernel_scales(env, name):
     assert_y_close(g["Y"], case.oracle_rows(act, wq, np.arange(wl.N)))
 
 
+@pytest.mark.parametrize("name", ["tiny", "ragged_122", "ragged_222", "unit_cube", "cube_414_r128", "cube_428",
+                                  "global", "wide_cube"])
+def test_parity_fp8_kernel_product(env, name):
+    """The FP8-rate kernel-token product on restricted-scale (C2) weights: the packed
+    weight, every quantised tensor and S_delta bit-exact, P' within the fp32
+    accumulation bound of the oracle's kernel term, Y within tolerance of the
+    oracle's fp64 product with the same C2 weights; small and big cubes, ragged
+    lattices, partial last tiles."""
+    dq, torch = env
+    wl = dict(SMALL)[name] or synth.WORKLOADS["tiny"]
+    case = Case(wl, fp8_product=True)
+    g = case.run_gpu(dq, torch)
+    act, wq = case.run_oracle()
+    compare_quantised(g, act, wq)
+    assert_kernel_term_close(g["p"], act, wq, np.arange(g["layout"].K))
+    assert_y_close(g["Y"], case.oracle_rows(act, wq, np.arange(wl.N)))
+
+
+def test_fp8_kernel_product_with_bias(env):
+    dq, torch = env
+    wl = dict(SMALL)["ragged_122"]
+    case = Case(wl, fp8_product=True)
+    b = synth.normal_bf16((wl.Co,), sd=4.0, seed=22)
+    g = case.run_gpu(dq, torch, bias=b)
+    act, wq = case.run_oracle()
+    compare_quantised(g, act, wq)
+    assert_kernel_term_close(g["p"], act, wq, np.arange(g["layout"].K), bias=b)
+    assert_y_close(g["Y"], case.oracle_rows(act, wq, np.arange(wl.N), bias=b))
+
+
+def test_packed_weight_must_match_the_kernel_product(env):
+    """A C2 weight run with the BF16 product (or a default weight with the FP8
+    product) is reported in the device status word."""
+    dq, torch = env
+    def clear_flags(p):
+        q = p.copy()
+        q[28:32] = 0          # header flags word: the C2 bit cleared
+        return q
+
+    case = Case(synth.WORKLOADS["tiny"], fp8_product=True)
+    out = case.run_gpu(dq, torch, packed_override=clear_flags)
+    assert out["status"] == dq.DQ_ERR_BAD_PACKED_WEIGHT
+
+
 def test_worked_example_through_gpu(env):
     """The hand-derived example (tests/golden) padded to 256 channels with zeros."""
     dq, torch = env

@@ -127,3 +127,55 @@ def test_vectorised_weight_scale_map_matches_library(dq, shape):
             for q in range(4):
                 blob[off + 1024 * q] = plain[r, b]
     assert np.array_equal(sfb_unpermute(blob, Co, Ci), plain)
+
+
+@pytest.mark.parametrize("shape", [(256, 256, 16), (512, 1024, 32), (768, 512, 48)])
+def test_pack_c2_bit_exact(dq, shape):
+    """Restricted-scale (C2) packing against the oracle's C2 quantiser and FP8 form:
+    residual codes, group scales (all quadrant copies), S_W, the E4M3 codes of
+    q s_b / 2^u and the UE8M0 exponents (through the 1X scale layout, all four
+    copies), bit for bit; header flag bit 1 set; the FP8 form times 2^u equals
+    q s_b exactly."""
+    from dq_case import packed_weight_parts, sfb_unpermute
+    Co, Ci, r = shape
+    wl = synth.Workload("pack", 1, 1, 1, Ci, Co, r, (1, 1, 1), (1, 1, 1), (0.0, 1.0), (0.01, 20.0))
+    Wb = synth.weight(wl, seed=Co * 3 + Ci)
+    L1, L2, _ = oracle.lowrank_factors(Wb, r)
+    wq = oracle.quantize_weight(Wb, L1, L2, c2=True)
+    fp8_o, ue_o, inexact = oracle.c2_fp8_operand(wq["wcodes"], wq["wscales"])
+    assert inexact == 0
+    packed, L1m, L2s, S_W = dq.dq_pack_weight_factors(Wb, L1, L2, pack_flags=dq.DQ_PACK_C2)
+    lay = dq.dq_packed_weight_layout(Co, Ci, r)
+    assert packed[28:32].view(np.uint32)[0] == 2          # the C2 flag, no bias
+    pw = packed_weight_parts(packed)
+    assert np.array_equal(pw["wcodes"], wq["wcodes"]) and np.array_equal(pw["wscales"], wq["wscales"])
+    assert np.float32(S_W) == np.float32(wq["S_w"]) == np.float32(pw["S_w"])
+    fp8 = packed[lay.off_dqw:lay.off_dqw + Co * Ci].reshape(Co, Ci)
+    assert np.array_equal(fp8, fp8_o)
+    # exponents: the B-operand layout of a Co x Ci/2 matrix, one "16-column block" per 32 channels
+    ue = sfb_unpermute(packed[lay.off_dqw + Co * Ci:], Co, Ci // 2)
+    assert np.array_equal(ue, ue_o)
+    back = oracle.e4m3_value(fp8) * np.repeat(np.exp2(ue.astype(np.float64) - 127), 32, axis=1)
+    q = np.empty((Co, Ci))
+    q[:, 0::2] = oracle.e2m1_value(wq["wcodes"] & 15)
+    q[:, 1::2] = oracle.e2m1_value(wq["wcodes"] >> 4)
+    assert np.array_equal(back, q * np.repeat(oracle.e4m3_value(wq["wscales"]), 16, axis=1))
+    # the default packing is unchanged by the option's existence
+    p0, *_ = dq.dq_pack_weight_factors(Wb, L1, L2)
+    assert p0[28:32].view(np.uint32)[0] == 0
+
+
+def test_forward_options_are_checked(dq):
+    """The FP8 kernel-token product takes per-token kernel scales only; unknown
+    options are refused before anything runs."""
+    args = (4, 8, 8, 1, 2, 2, 256, 256, 16)
+    lay = dq.dq_workspace_layout_opts(*args, kernel_product=dq.DQ_KERNEL_PRODUCT_FP8)
+    full = dq.dq_workspace_layout_opts(*args)
+    assert lay.total_bytes < full.total_bytes and lay.off_dcodes == lay.off_q8_bf16   # no BF16 operand
+    for kw in (dict(kernel_product=2), dict(kernel_group=64, kernel_product=dq.DQ_KERNEL_PRODUCT_FP8),
+               dict(kernel_group=32)):
+        with pytest.raises(dq.DQError):
+            dq.dq_workspace_layout_opts(*args, **kw)
+    with pytest.raises(dq.DQError):
+        dq.dq_pack_weight_factors(np.zeros((256, 256), np.uint16), np.zeros((256, 16), np.uint16),
+                                  np.zeros((16, 256), np.uint16), pack_flags=4)

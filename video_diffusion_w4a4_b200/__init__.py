@@ -37,6 +37,8 @@ DQ_STAGE_QUANTIZE, DQ_STAGE_KERNEL_GEMM, DQ_STAGE_MAIN_GEMM, DQ_STAGE_ALL = 1, 2
 DQ_STAGE_STATS, DQ_STAGE_ENCODE = 8, 16
 DQ_KERNEL_SCALE_PER_TOKEN, DQ_KERNEL_SCALE_GROUP64 = 0, 64
 DQ_NOALLOC_WORKSPACE = 1   # dq_read_device_status: the fixed array of dq_linear_forward_noalloc
+DQ_PACK_C2 = 1
+DQ_KERNEL_PRODUCT_BF16, DQ_KERNEL_PRODUCT_FP8 = 0, 1
 
 
 class dq_packed_layout(ctypes.Structure):
@@ -51,6 +53,10 @@ class dq_workspace_layout(ctypes.Structure):
                                        "off_dcodes", "off_dscales", "off_u_part", "off_u_hilo", "off_p", "off_means")] + [
         ("N", ctypes.c_longlong), ("K", ctypes.c_longlong), ("N_pad", ctypes.c_longlong), ("K_pad", ctypes.c_longlong),
         ("splits", ctypes.c_int), ("slab", ctypes.c_int), ("kernel_group", ctypes.c_int)]
+
+
+class dq_forward_options(ctypes.Structure):
+    _fields_ = [("kernel_group", ctypes.c_int), ("kernel_product", ctypes.c_int), ("reserved", ctypes.c_int * 2)]
 
 
 _P, _I, _SZ, _LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
@@ -72,6 +78,11 @@ _SIGS = {
     "dq_lowrank_factors": ([_P, _I, _I, _I, ctypes.c_uint64, _P, _P], _I),
     "dq_pack_weight_factors": ([_P, _P, _P, _I, _I, _I, _P, _SZ, _P, _P, ctypes.POINTER(ctypes.c_float)], _I),
     "dq_pack_weight": ([_P, _I, _I, _I, _P, _SZ, _P, _P], _I),
+    "dq_pack_weight_factors_ex": ([_P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P, _P, ctypes.POINTER(ctypes.c_float)], _I),
+    "dq_workspace_layout_opts": ([_I] * 9 + [ctypes.POINTER(dq_forward_options), ctypes.POINTER(dq_workspace_layout)],
+                                 _I),
+    "dq_linear_forward_opts": ([_P] + [_I] * 9 + [ctypes.POINTER(dq_forward_options), _P, _P, _P, _P, _P, _SZ, _I, _P,
+                                                   _P], _I),
     "dq_pack_bias": ([_P, _I, _P, _SZ], _I),
     "dq_workspace_layout_get": ([_I] * 9 + [ctypes.POINTER(dq_workspace_layout)], _I),
     "dq_workspace_bytes": ([_I] * 9 + [ctypes.POINTER(_SZ)], _I),
@@ -211,8 +222,9 @@ def dq_lowrank_factors(W: np.ndarray, rank: int, seed: int = 0):
     return L1, L2
 
 
-def dq_pack_weight_factors(W: np.ndarray, L1: np.ndarray, L2: np.ndarray):
-    """Returns (packed blob uint8, L1_mma (r, Ci) BF16 bits, L2_slab (Co, slab) BF16 bits, S_W)."""
+def dq_pack_weight_factors(W: np.ndarray, L1: np.ndarray, L2: np.ndarray, pack_flags: int = 0):
+    """Returns (packed blob uint8, L1_mma (r, Ci) BF16 bits, L2_slab (Co, slab) BF16 bits, S_W).
+    pack_flags: 0 or DQ_PACK_C2 (dq_pack_weight_factors_ex)."""
     W = np.ascontiguousarray(W, dtype=np.uint16)
     L1 = np.ascontiguousarray(L1, dtype=np.uint16)
     L2 = np.ascontiguousarray(L2, dtype=np.uint16)
@@ -223,9 +235,10 @@ def dq_pack_weight_factors(W: np.ndarray, L1: np.ndarray, L2: np.ndarray):
     L1m = np.empty((r, Ci), np.uint16)
     L2s = np.empty((Co, lay.slab), np.uint16)
     S = ctypes.c_float()
-    _check("dq_pack_weight_factors",
-           _lib.dq_pack_weight_factors(W.ctypes.data, L1.ctypes.data, L2.ctypes.data, Co, Ci, r, packed.ctypes.data,
-                                       packed.size, L1m.ctypes.data, L2s.ctypes.data, ctypes.byref(S)))
+    _check("dq_pack_weight_factors_ex",
+           _lib.dq_pack_weight_factors_ex(W.ctypes.data, L1.ctypes.data, L2.ctypes.data, Co, Ci, r, pack_flags,
+                                          packed.ctypes.data, packed.size, L1m.ctypes.data, L2s.ctypes.data,
+                                          ctypes.byref(S)))
     return packed, L1m, L2s, S.value
 
 
@@ -268,6 +281,33 @@ def dq_workspace_layout_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group) ->
     _check("dq_workspace_layout_grouped", _lib.dq_workspace_layout_grouped(T, H, W, t, h, w, Ci, Co, rank,
                                                                            kernel_group, ctypes.byref(L)))
     return L
+
+
+def _options(kernel_group=DQ_KERNEL_SCALE_PER_TOKEN, kernel_product=DQ_KERNEL_PRODUCT_BF16):
+    o = dq_forward_options()
+    o.kernel_group, o.kernel_product = kernel_group, kernel_product
+    return o
+
+
+def dq_workspace_layout_opts(T, H, W, t, h, w, Ci, Co, rank, kernel_group=DQ_KERNEL_SCALE_PER_TOKEN,
+                             kernel_product=DQ_KERNEL_PRODUCT_BF16) -> dq_workspace_layout:
+    """Workspace carve-up for the forward options (dq_forward_options fields as keywords)."""
+    L = dq_workspace_layout()
+    o = _options(kernel_group, kernel_product)
+    _check("dq_workspace_layout_opts", _lib.dq_workspace_layout_opts(T, H, W, t, h, w, Ci, Co, rank, ctypes.byref(o),
+                                                                     ctypes.byref(L)))
+    return L
+
+
+def dq_linear_forward_opts(X, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y, workspace,
+                           workspace_bytes, stage_mask=DQ_STAGE_ALL, stage_events=None, stream=None,
+                           kernel_group=DQ_KERNEL_SCALE_PER_TOKEN, kernel_product=DQ_KERNEL_PRODUCT_BF16) -> None:
+    """dq_linear_forward_ex with forward options (dq_forward_options fields as keywords)."""
+    o = _options(kernel_group, kernel_product)
+    _check("dq_linear_forward_opts",
+           _lib.dq_linear_forward_opts(_ptr(X), T, H, W, t, h, w, Ci, Co, rank, ctypes.byref(o), _ptr(packed_W),
+                                       _ptr(L1_mma), _ptr(L2_slab), _ptr(Y), _ptr(workspace), workspace_bytes,
+                                       stage_mask, _events(stage_events), _stream(stream)))
 
 
 def dq_workspace_bytes_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group) -> int:

@@ -93,15 +93,18 @@ bool map_means(CUtensorMap* m, const void* base, int Ci, long long K, int rows) 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D map over the B-operand scale layout (dq_sfb_offset): dim 0 the bytes of a
-// 256-byte line, dim 1 the 16 (Ci/64) lines of one 256-row tile (16384 bytes
-// per K step of 256 channels), dim 2 the 256-row tiles.  Boxes of one K step.
-bool map_sfb(CUtensorMap* m, const void* base, int Ci, int Co) {
+// 3-D map over the B-operand scale layout (dq_sfb_offset) of a matrix with `cols`
+// 16-column blocks' worth of columns: dim 0 the bytes of a 256-byte line, dim 1 the
+// 16 lines of each 4096-byte block (cols / 64 blocks per 256-row tile), dim 2 the
+// 256-row tiles.  Boxes of `blocks` consecutive 4096-byte blocks: four (one K step
+// of 256 channels) for the FP4 weight scales, one (a 128-channel stage) for the
+// UE8M0 exponents of C2 weights (cols = Ci / 2).
+bool map_sfb(CUtensorMap* m, const void* base, int cols, int Co, int blocks = 4) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
-    cuuint64_t dims[3] = {256, (cuuint64_t)Ci / 64 * 16, (cuuint64_t)Co / 256};
-    cuuint64_t strides[2] = {256, (cuuint64_t)Ci / 64 * 4096};
-    cuuint32_t box[3] = {256, 64, 1};
+    cuuint64_t dims[3] = {256, (cuuint64_t)cols / 64 * 16, (cuuint64_t)Co / 256};
+    cuuint64_t strides[2] = {256, (cuuint64_t)cols / 64 * 4096};
+    cuuint32_t box[3] = {256, (cuuint32_t)(16 * blocks), 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -129,6 +132,17 @@ int check_shape(int T, int H, int W, int t, int h, int w, int Ci, int Co, int ra
     if (Ci < 256 || Co < 256 || Ci % 256 || Co % 256) return DQ_ERR_UNSUPPORTED_SHAPE;
     if (rank < 16 || rank > 128 || rank % 16 || rank > Ci || rank > Co) return DQ_ERR_UNSUPPORTED_SHAPE;
     if ((long long)T * H * W >= (1ll << 31)) return DQ_ERR_UNSUPPORTED_SHAPE;
+    return DQ_OK;
+}
+
+int check_options(const dq_forward_options& o) {
+    if (o.kernel_group != DQ_KERNEL_SCALE_PER_TOKEN && o.kernel_group != DQ_KERNEL_SCALE_GROUP64)
+        return DQ_ERR_INVALID_ARG;
+    if (o.kernel_product != DQ_KERNEL_PRODUCT_BF16 && o.kernel_product != DQ_KERNEL_PRODUCT_FP8) return DQ_ERR_INVALID_ARG;
+    // the FP8 product carries the kernel-token scale in its epilogue: one per token
+    if (o.kernel_product == DQ_KERNEL_PRODUCT_FP8 && o.kernel_group != DQ_KERNEL_SCALE_PER_TOKEN)
+        return DQ_ERR_INVALID_ARG;
+    if (o.reserved[0] || o.reserved[1]) return DQ_ERR_INVALID_ARG;
     return DQ_OK;
 }
 
@@ -166,13 +180,16 @@ int ensure_lib_workspace(size_t need, void** ws) {
 
 extern "C" {
 
-int dq_workspace_layout_grouped(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank, int kernel_group,
-                                dq_workspace_layout* out) {
+int dq_workspace_layout_opts(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                             const dq_forward_options* opts, dq_workspace_layout* out) {
     if (!out) return DQ_ERR_INVALID_ARG;
     int rc = check_shape(T, H, W, t, h, w, Ci, Co, rank);
     if (rc) return rc;
-    if (kernel_group != DQ_KERNEL_SCALE_PER_TOKEN && kernel_group != DQ_KERNEL_SCALE_GROUP64) return DQ_ERR_INVALID_ARG;
-    dq::WsLayout L = dq::ws_layout(dq::make_geom(T, H, W, t, h, w), Ci, Co, rank, kernel_group);
+    const dq_forward_options o = opts ? *opts : dq_forward_options{};
+    if ((rc = check_options(o))) return rc;
+    const int kernel_group = o.kernel_group;
+    dq::WsLayout L = dq::ws_layout(dq::make_geom(T, H, W, t, h, w), Ci, Co, rank, kernel_group,
+                                   o.kernel_product == DQ_KERNEL_PRODUCT_FP8);
     out->total_bytes = L.total;
     out->off_status = L.off_status;
     out->off_scalars = L.off_scalars;
@@ -194,6 +211,13 @@ int dq_workspace_layout_grouped(int T, int H, int W, int t, int h, int w, int Ci
     out->slab = L.slab;
     out->kernel_group = kernel_group;
     return DQ_OK;
+}
+
+int dq_workspace_layout_grouped(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank, int kernel_group,
+                                dq_workspace_layout* out) {
+    dq_forward_options o{};
+    o.kernel_group = kernel_group;
+    return dq_workspace_layout_opts(T, H, W, t, h, w, Ci, Co, rank, &o, out);
 }
 
 int dq_workspace_layout_get(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
@@ -220,14 +244,16 @@ int dq_workspace_bytes(int T, int H, int W, int t, int h, int w, int Ci, int Co,
     return DQ_OK;
 }
 
-int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
-                              int kernel_group, const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y,
-                              void* workspace, size_t workspace_bytes, int stage_mask, void* const* stage_events,
-                              void* stream) {
+int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                           const dq_forward_options* opts, const void* packed_W, const void* L1_mma,
+                           const void* L2_slab, void* Y, void* workspace, size_t workspace_bytes, int stage_mask,
+                           void* const* stage_events, void* stream) {
     int rc = check_shape(T, H, W, t, h, w, Ci, Co, rank);
     if (rc) return rc;
-    if (kernel_group != DQ_KERNEL_SCALE_PER_TOKEN && kernel_group != DQ_KERNEL_SCALE_GROUP64) return DQ_ERR_INVALID_ARG;
-    const int kg = kernel_group;
+    const dq_forward_options o = opts ? *opts : dq_forward_options{};
+    if ((rc = check_options(o))) return rc;
+    const int kg = o.kernel_group;
+    const bool fp8prod = o.kernel_product == DQ_KERNEL_PRODUCT_FP8;
     if (!X || !packed_W || !L1_mma || !L2_slab || !Y || !workspace) return DQ_ERR_INVALID_ARG;
     if (stage_mask <= 0 || (stage_mask & ~(DQ_STAGE_ALL | DQ_STAGE_STATS | DQ_STAGE_ENCODE))) return DQ_ERR_INVALID_ARG;
     const bool do_stats = stage_mask & (DQ_STAGE_QUANTIZE | DQ_STAGE_STATS);
@@ -236,7 +262,7 @@ int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, 
         !aligned(workspace))
         return DQ_ERR_ALIGNMENT;
     const Geom g = dq::make_geom(T, H, W, t, h, w);
-    const dq::WsLayout wl = dq::ws_layout(g, Ci, Co, rank, kg);
+    const dq::WsLayout wl = dq::ws_layout(g, Ci, Co, rank, kg, fp8prod);
     if (workspace_bytes < wl.total) return DQ_ERR_WORKSPACE_TOO_SMALL;
     if (!encode_fn()) return DQ_ERR_NO_DEVICE;
     cudaStream_t st = (cudaStream_t)stream;
@@ -252,6 +278,7 @@ int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, 
     qp.slab = wl.slab;
     qp.splits = wl.splits;
     qp.kgroup = kg;
+    qp.fp8_product = fp8prod;
     qp.chunks_per_split = Ci / 64 / wl.splits;
     qp.big = (long long)t * h * w > 128;
     if (!qp.big) {
@@ -324,7 +351,24 @@ int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, 
             return cuda_fail(e, "k_cube_encode");
     }
     rec(1);
-    if (stage_mask & DQ_STAGE_KERNEL_GEMM) {
+    if ((stage_mask & DQ_STAGE_KERNEL_GEMM) && fp8prod) {
+        // q8 (E4M3, K x Ci) times the FP8 form of C2 weights with their UE8M0 exponents per 32 channels
+        CUtensorMap tm_a, tm_b, tm_fb;
+        if (!map_2d(&tm_a, ws + wl.off_q8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Ci, g.K, 128, 128))
+            return map_fail("FP8 product A");
+        if (!map_2d(&tm_b, pw + pl.off_dqw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Ci, Co, 128, 128))
+            return map_fail("FP8 product B");
+        if (!map_sfb(&tm_fb, pw + pl.off_dqw + (size_t)Co * Ci, Ci / 2, Co, 1)) return map_fail("FP8 product scales");
+        dq::GemmParams p = gp;
+        p.M = (int)g.K;
+        p.k_stages = Ci / 128;
+        p.tile_group = 8;
+        p.s8 = qp.s8;
+        p.pout = (float*)(ws + wl.off_p);
+        p.bias = (const float*)(pw + pl.off_bias);
+        cudaError_t e = dq::launch_kernel_gemm_fp8(tm_a, tm_b, tm_fb, p, st);
+        if (e != cudaSuccess) return cuda_fail(e, "FP8 kernel-token product");
+    } else if (stage_mask & DQ_STAGE_KERNEL_GEMM) {
         CUtensorMap tm_a, tm_b;
         const int a_cols = kg ? 2 * Ci : Ci;   // grouped scales: [hi | lo]
         if (!map_2d(&tm_a, ws + wl.off_q8_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a_cols, g.K, 64, 128))
@@ -367,6 +411,16 @@ int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, 
     }
     rec(3);
     return DQ_OK;
+}
+
+int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                              int kernel_group, const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y,
+                              void* workspace, size_t workspace_bytes, int stage_mask, void* const* stage_events,
+                              void* stream) {
+    dq_forward_options o{};
+    o.kernel_group = kernel_group;
+    return dq_linear_forward_opts(X, T, H, W, t, h, w, Ci, Co, rank, &o, packed_W, L1_mma, L2_slab, Y, workspace,
+                                  workspace_bytes, stage_mask, stage_events, stream);
 }
 
 int dq_linear_forward_ex(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,

@@ -118,6 +118,15 @@ DQ_HD size_t sfb_offset(long long row, int blk, int cols) {
 
 DQ_HD size_t sfb_bytes(long long rows, int cols) { return (size_t)cdiv(rows, 256) * (size_t)(cols / 64) * 4096; }
 
+// Scale layout of the FP8 operand of C2 weights (one UE8M0 exponent per 32 channels, B operand of
+// a kind::mxf8f6f4 product with one scale per 32 K): the four MMAs (K = 32 each) of a 128-channel
+// stage read byte 0..3 of the same 32-bit tensor-memory word, so a stage's exponents of a 256-row
+// tile fill one 4 KB block laid out as the B-operand layout above with four 32-channel blocks in
+// place of four 16-channel blocks: block j of row o sits where sfb_offset puts 16-channel block j
+// of a matrix with cols / 2 columns.
+DQ_HD size_t c2_sf_offset(long long row, int blk32, int cols) { return sfb_offset(row, blk32, cols / 2); }
+DQ_HD size_t c2_sf_bytes(long long rows, int cols) { return sfb_bytes(rows, cols / 2); }
+
 DQ_HD int slab_width(int rank) { return (int)(cdiv(2 * rank, 64) * 64); }
 
 // Packed weight blob header (first 256 bytes of the blob).
@@ -130,6 +139,10 @@ struct PackedHeader {
 };
 
 constexpr uint32_t kPackedHasBias = 1u;
+// Restricted-scale (C2) weights: group scales {1, 1.5} x 2^e, S_W = amax / (6 * 384), and the
+// dqw section holding the FP8 form of q s_b (E4M3 codes, Co x Ci, then their UE8M0 exponents per
+// 32 channels in the 1X scale layout c2_sf_offset) instead of BF16 q s_b.
+constexpr uint32_t kPackedC2 = 2u;
 
 struct PackedLayout {
     size_t total, off_codes, off_scales, off_dqw, off_bias;
@@ -172,7 +185,7 @@ struct WsLayout {
 
 // kgroup: 0 = one FP8 scale per kernel token; 64 = one per 64 channels, whose
 // kernel tokens enter the product as BF16 hi + lo (twice the columns)
-DQ_HD WsLayout ws_layout(const Geom& g, int Ci, int Co, int rank, int kgroup = 0) {
+DQ_HD WsLayout ws_layout(const Geom& g, int Ci, int Co, int rank, int kgroup = 0, bool fp8_product = false) {
     WsLayout L;
     L.N = g.N; L.K = g.K;
     L.N_pad = cdiv(g.N, 128) * 128;
@@ -185,7 +198,8 @@ DQ_HD WsLayout ws_layout(const Geom& g, int Ci, int Co, int rank, int kgroup = 0
     L.off_kamax = off;    off = align_up(off + (size_t)g.K * 4, kAlign);
     L.off_s8 = off;       off = align_up(off + (size_t)g.K * (kgroup ? Ci / kgroup : 1) * 4, kAlign);
     L.off_q8 = off;       off = align_up(off + (size_t)g.K * Ci, kAlign);
-    L.off_q8_bf16 = off;  off = align_up(off + (size_t)L.K_pad * Ci * 2 * (kgroup ? 2 : 1), kAlign);
+    // BF16 operand of the exact kernel-token product (the FP8 product reads q8 itself)
+    L.off_q8_bf16 = off;  off = align_up(off + (fp8_product ? 0 : (size_t)L.K_pad * Ci * 2 * (kgroup ? 2 : 1)), kAlign);
     L.off_dcodes = off;   off = align_up(off + (size_t)g.N * (Ci / 2), kAlign);
     L.off_dscales = off;  off = align_up(off + sfa_bytes(g.N, Ci), kAlign);
     L.off_u_part = off;   off = align_up(off + (size_t)L.splits * g.N * rank * 4, kAlign);

@@ -35,12 +35,20 @@
 // and "accumulator full" barriers of both CTAs; the epilogue warps of both
 // CTAs arrive on the even CTA's "accumulator empty" barrier.
 //
-// The kernel-token product double-buffers its accumulator in tensor memory so
+//   (c') FP8 kernel-token product (weights packed with DQ_PACK_C2): the same P'
+//       from q8 (E4M3) and the FP8 form of q s_b (E4M3 codes times one UE8M0
+//       exponent per 32 channels) with kind::mxf8f6f4 MMAs at twice the BF16
+//       rate.  Every product q8 * (q s_b) is exact in fp32 either way; the A
+//       operand's scales are a constant 1 (UE8M0 127) written to tensor memory
+//       once, the B operand's exponents are copied in per 128-channel stage.
+//
+// The BF16 kernel-token product double-buffers its accumulator in tensor memory so
 // the epilogue of one tile overlaps the MMAs of the next; the main product
 // needs tensor-memory columns for the block scale factors (a 48-column slot
 // per ring stage), so it keeps one accumulator: its epilogue warps copy their
 // slice into registers, release tensor memory, and then fetch P' and write Y
-// while the next tile's MMAs run.
+// while the next tile's MMAs run.  The FP8 kernel-token product does the same
+// (an 8-column exponent slot per stage next to one accumulator).
 #include <atomic>
 
 #include "dq_common.h"
@@ -59,9 +67,14 @@ constexpr uint32_t kABytes = kTileM * 128;      // 128 rows x 128 bytes
 constexpr uint32_t kBBytes = (kTileN / 2) * 128;  // this CTA's 128 rows of B x 128 bytes
 constexpr uint32_t kSFABytes = 2 * 4096;        // 128 rows x 4 k-blocks of 64, A-operand scale layout
 constexpr uint32_t kSFBBytes = 4 * 4096;        // all 256 columns x 4 k-blocks, B-operand scale layout (each CTA)
+constexpr uint32_t kSFB8Bytes = 4096;           // FP8 product: UE8M0 exponents of 256 columns x 4 blocks of 32
 constexpr uint16_t kPairMask = 0x3;
+constexpr uint32_t kFp8SfaCol = 256;            // FP8 product: tensor-memory columns of the constant A scales
+constexpr uint32_t kFp8SfbCol = 264;            //   and of the first B-exponent slot (8 columns per stage)
 
-__host__ __device__ constexpr int g_stages(bool scaled) { return scaled ? 4 : 7; }
+__host__ __device__ constexpr int g_stages(int kind) {
+    return kind == kGemmMain ? 4 : (kind == kGemmKernelFp8 ? 6 : 7);
+}
 
 // Output tile -> (row tile, column tile).  group <= 1: row-major, which suits a weight that stays
 // in L2 while the row tiles stream.  Otherwise groups of `group` row tiles walked column by column:
@@ -82,18 +95,19 @@ struct GSmem {
     uint32_t a, b, sfa, sfb, bars, misc, total;
 };
 
-__host__ __device__ constexpr GSmem g_smem_layout(bool scaled) {
+__host__ __device__ constexpr GSmem g_smem_layout(int kind) {
     GSmem L{};
-    const int S = g_stages(scaled);
+    const int S = g_stages(kind);
     uint32_t off = 0;
     L.a = off;
     off += S * kABytes;
     L.b = off;
     off += S * kBBytes;
     L.sfa = off;
-    if (scaled) off += S * kSFABytes;
+    if (kind == kGemmMain) off += S * kSFABytes;
     L.sfb = off;
-    if (scaled) off += S * kSFBBytes;
+    if (kind == kGemmMain) off += S * kSFBBytes;
+    if (kind == kGemmKernelFp8) off += S * kSFB8Bytes;
     L.bars = off;
     off += (3 * S + 6) * 8;
     L.misc = off;
@@ -105,16 +119,19 @@ __host__ __device__ constexpr GSmem g_smem_layout(bool scaled) {
 
 }  // namespace
 
-template <bool kMain>
+template <int kKind>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
            const __grid_constant__ CUtensorMap tm_sa, const __grid_constant__ CUtensorMap tm_sb,
            const __grid_constant__ CUtensorMap tm_fa, const __grid_constant__ CUtensorMap tm_fb, GemmParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    constexpr GSmem L = g_smem_layout(kMain);
-    constexpr int S = g_stages(kMain);
-    constexpr int kBufs = kMain ? 1 : 2;
+    constexpr bool kMain = kKind == kGemmMain;
+    constexpr bool kFp8 = kKind == kGemmKernelFp8;
+    constexpr bool kScaled = kMain || kFp8;      // block scales copied into tensor memory, one accumulator
+    constexpr GSmem L = g_smem_layout(kKind);
+    constexpr int S = g_stages(kKind);
+    constexpr int kBufs = kScaled ? 1 : 2;
     uint64_t* full = (uint64_t*)(sm + L.bars);   // [S], used in the even CTA
     uint64_t* empty = full + S;                  // [S], both CTAs
     uint64_t* sfready = empty + S;               // [S], even CTA: block scales of a stage are in tensor memory
@@ -137,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < S; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kMain ? 2 : 1);   // main: MMA commit + scale-copy commit
+            mbar_init(&empty[s], kScaled ? 2 : 1);   // scaled kinds: MMA commit + scale-copy commit
             mbar_init(&sfready[s], 1);
         }
         for (int b = 0; b < 2; b++) {
@@ -157,12 +174,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     cluster_sync();   // barriers of both CTAs initialised, tensor memory allocated
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (kFp8) {
+        // the A operand (q8) carries its scale in the epilogue: its MMA scales are 1 (UE8M0 127),
+        // written once into four columns of every lane of both CTAs' tensor memory
+        if (warp >= 3 && warp < 7) {
+            const uint32_t v = 0x7F7F7F7Fu;
+            tmem_st_x4(tmem + ((uint32_t)((warp & 3) * 32) << 16) + kFp8SfaCol, v, v, v, v);
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        cluster_sync();
+        tc_fence_after();
+    }
 
     if (warp == 0) {
         // ------------------------------------------------ producer (both CTAs)
         if (lane == 0) {
             prefetch_tmap(&tm_a);
             prefetch_tmap(&tm_b);
+            if (kFp8) prefetch_tmap(&tm_fb);
             if (kMain) {
                 prefetch_tmap(&tm_sa);
                 prefetch_tmap(&tm_sb);
@@ -188,7 +218,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t fb = full0 + (uint32_t)(s * 8);
                     uint8_t* sa = sm + L.a + s * kABytes;
                     uint8_t* sb = sm + L.b + s * kBBytes;
-                    if (!kMain) {
+                    if (kFp8) {
+                        // 128 channels of q8 and of the FP8 weight, and the stage's 4 KB of exponents
+                        if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes + kSFB8Bytes));
+                        tma_load_2d_pair_hint(sa, &tm_a, fb, i * 128, m0, stream);
+                        tma_load_2d_pair_hint(sb, &tm_b, fb, i * 128, nb, keep);
+                        tma_load_3d_pair(sm + L.sfb + s * kSFB8Bytes, &tm_fb, fb, 0, 16 * i, n0 >> 8);
+                    } else if (!kMain) {
                         if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes));
                         tma_load_2d_pair_hint(sa, &tm_a, fb, i * 64, m0, stream);
                         tma_load_2d_pair_hint(sb, &tm_b, fb, (i < p.b_kblocks ? i : i - p.b_kblocks) * 64, nb, keep);
@@ -242,7 +278,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint32_t aa = smem_u32(sm + L.a + s * kABytes), bb = smem_u32(sm + L.b + s * kBBytes);
-                    if (kMain && i < nk) {
+                    if (kFp8) {
+                        if (!mbar_wait(&sfready[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
+                            alive = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        // four MMAs of 32 channels; MMA k reads byte k of the stage's scale words
+#pragma unroll
+                        for (int k = 0; k < 4; k++)
+                            mma_mxf8_pair(acc, desc_k_sw128(aa + 32 * k), desc_k_sw128(bb + 32 * k),
+                                          idesc_mxf8(2 * kTileM, kTileN, (uint32_t)k, (uint32_t)k), tmem + kFp8SfaCol,
+                                          tmem + kFp8SfbCol + (uint32_t)(8 * s), (i | k) != 0);
+                    } else if (kMain && i < nk) {
                         const uint32_t t_sfa = t_sf0 + (uint32_t)(s * 48), t_sfb = t_sfa + 16;
                         if (!mbar_wait(&sfready[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
                             alive = false;
@@ -274,6 +322,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         // One copy instruction moves each CTA's scale factors from its own shared
         // memory into its own tensor memory; a thread of its own lets the copies
         // run ahead of the MMAs instead of sitting in the MMA thread's stream.
+        if (kFp8 && lead && lane == 0) {
+            long long g = 0;
+            bool alive = true;
+            for (int tile = pair; alive && tile < num_tiles; tile += npairs) {
+                for (int i = 0; i < ntot; i++, g++) {
+                    const int s = (int)(g % S);
+                    if (!mbar_wait(&full[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
+                        alive = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    // one copy: lane i of every quadrant gets rows 32 c + i (c = 0..7) of the tile, four
+                    // exponent bytes (the stage's four 32-channel blocks) per row
+                    tmem_cp_pair_128x256b(tmem + kFp8SfbCol + (uint32_t)(8 * s),
+                                          smem_desc(smem_u32(sm + L.sfb + s * kSFB8Bytes), 128, 256, 0));
+                    tc_commit_pair(&sfready[s]);
+                    tc_commit_pair_both(&empty[s], kPairMask);
+                }
+            }
+            tc_commit_pair(drain_sf);
+            mbar_wait(drain_sf, 0, abort_flag, nullptr, p.budget_ns, false);
+        }
         if (kMain && lead && lane == 0) {
             const uint32_t t_sf0 = tmem + 256;
             long long g = 0;
@@ -372,6 +442,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int e = 0; e < 8; e++) pa[v][e] = pb[v][e];
                     }
                 }
+            } else if (kFp8) {
+                // the whole 128-column slice into registers, tensor memory released, then P'
+                const float scale = row_ok ? __fmul_rn(p.s8[rho], S_W) : 0.f;
+                const float* bias =
+                    (reinterpret_cast<const PackedHeader*>(p.packed_w)->flags & kPackedHasBias) ? p.bias + c_base
+                                                                                                 : nullptr;
+                const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], (uint32_t)use & 1, abort_flag,
+                                                                  p.status, p.budget_ns));
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t acc[128];
+#pragma unroll
+                for (int c = 0; c < 128; c += 16)
+                    tmem_ld_x16(tacc + (uint32_t)c, *reinterpret_cast<uint32_t(*)[16]>(&acc[c]));
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acce0 + (uint32_t)(buf * 8));
+                if (row_ok) {
+                    float* dst = p.pout + (size_t)rho * p.Nout + c_base;
+#pragma unroll
+                    for (int c = 0; c < 128; c += 8) {
+                        float b0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        if (bias) ld_global_nc_v8(bias + c, b0);
+                        uint32_t o0[8];
+#pragma unroll
+                        for (int e = 0; e < 8; e++) o0[e] = __float_as_uint(fmaf(__uint_as_float(acc[c + e]), scale, b0[e]));
+                        st_global_cs_v8(dst + c, o0);
+                    }
+                }
             } else {
                 const float scale = row_ok ? (p.s8 ? __fmul_rn(p.s8[rho], S_W) : S_W) : 0.f;
                 // the layer's bias, when the packed weight holds one, joins P' once per cube
@@ -434,12 +534,13 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-template <bool kMain>
+template <int kKind>
 cudaError_t launch_pairs(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_sa,
                          const CUtensorMap& tm_sb, const CUtensorMap& tm_fa, const CUtensorMap& tm_fb,
                          const GemmParams& p, cudaStream_t st) {
-    constexpr size_t smem = g_smem_layout(kMain).total + 1024;
-    cudaError_t e = cudaFuncSetAttribute(k_gemm<kMain>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    constexpr size_t smem = g_smem_layout(kKind).total + 1024;
+    static_assert(smem <= 232448, "shared memory of a paired product");
+    cudaError_t e = cudaFuncSetAttribute(k_gemm<kKind>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int tiles = (int)cdiv(p.M, 2 * kTileM) * (p.Nout / kTileN);
     cudaLaunchConfig_t cfg = {};
@@ -464,27 +565,32 @@ cudaError_t launch_pairs(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const
     if (mp == 0) {
         cfg.gridDim = dim3(2 * tiles);
         int n = 0;
-        e = cudaOccupancyMaxActiveClusters(&n, k_gemm<kMain>, &cfg);
+        e = cudaOccupancyMaxActiveClusters(&n, k_gemm<kKind>, &cfg);
         if (e != cudaSuccess) return e;
         if (n <= 0) return cudaErrorInvalidConfiguration;
         mp = n;
         resident[dev].store(mp, std::memory_order_relaxed);
     }
     cfg.gridDim = dim3(2 * imin(tiles, mp));
-    return cudaLaunchKernelEx(&cfg, k_gemm<kMain>, tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p);
+    return cudaLaunchKernelEx(&cfg, k_gemm<kKind>, tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p);
 }
 
 }  // namespace
 
 cudaError_t launch_kernel_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmParams& p,
                                cudaStream_t st) {
-    return launch_pairs<false>(tm_a, tm_b, tm_a, tm_b, tm_a, tm_b, p, st);
+    return launch_pairs<kGemmKernelBf16>(tm_a, tm_b, tm_a, tm_b, tm_a, tm_b, p, st);
+}
+
+cudaError_t launch_kernel_gemm_fp8(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_fb,
+                                   const GemmParams& p, cudaStream_t st) {
+    return launch_pairs<kGemmKernelFp8>(tm_a, tm_b, tm_a, tm_b, tm_a, tm_fb, p, st);
 }
 
 cudaError_t launch_main_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_sa,
                              const CUtensorMap& tm_sb, const CUtensorMap& tm_fa, const CUtensorMap& tm_fb,
                              const GemmParams& p, cudaStream_t st) {
-    return launch_pairs<true>(tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p, st);
+    return launch_pairs<kGemmMain>(tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p, st);
 }
 
 }  // namespace dq

@@ -104,6 +104,19 @@ inline float e2m1_to_float(uint8_t c) {
     return (c & 8) ? -v : v;
 }
 
+// The restricted group scale of C2 weights: the least value {1, 1.5} x 2^e with e >= -9 that is
+// >= v (v > 0), skipping 1.5 x 2^-9, which E4M3 cannot hold; every such value is an E4M3 value
+// whose product with an E2M1 value has at most three fraction bits.
+inline float c2_round_scale_up(float v) {
+    if (!(v > 0.0f)) return 0.0f;
+    const float lo = ldexpf(1.0f, -9);
+    if (v <= lo) return lo;
+    int e;
+    const float m = frexpf(v, &e);   // v = m 2^e, 0.5 <= m < 1
+    const float up = (m == 0.5f) ? v : ldexpf(m <= 0.75f ? 0.75f : 1.0f, e);
+    return (up == ldexpf(1.5f, -9)) ? ldexpf(1.0f, -8) : up;
+}
+
 // ------------------------------------------------------------------ small dense linear algebra (fp64)
 
 // Y (m x l) = A (m x n, row-major) * B (n x l, row-major)
@@ -413,9 +426,12 @@ int dq_lowrank_factors(const uint16_t* Wb, int Co, int Ci, int rank, uint64_t se
     return DQ_OK;
 }
 
-int dq_pack_weight_factors(const uint16_t* Wb, const uint16_t* L1, const uint16_t* L2, int Co, int Ci, int rank,
-                           void* packed, size_t packed_bytes, uint16_t* L1_mma, uint16_t* L2_slab, float* S_W_out) {
+int dq_pack_weight_factors_ex(const uint16_t* Wb, const uint16_t* L1, const uint16_t* L2, int Co, int Ci, int rank,
+                              int pack_flags, void* packed, size_t packed_bytes, uint16_t* L1_mma, uint16_t* L2_slab,
+                              float* S_W_out) {
     if (!Wb || !L1 || !L2 || !packed) return DQ_ERR_INVALID_ARG;
+    if (pack_flags & ~DQ_PACK_C2) return DQ_ERR_INVALID_ARG;
+    const bool c2 = (pack_flags & DQ_PACK_C2) != 0;
     if (!shape_ok(Co, Ci, rank)) return DQ_ERR_UNSUPPORTED_SHAPE;
     dq::PackedLayout L = dq::packed_layout(Co, Ci, rank);
     if (packed_bytes < L.total) return DQ_ERR_INVALID_ARG;
@@ -439,15 +455,62 @@ int dq_pack_weight_factors(const uint16_t* Wb, const uint16_t* L1, const uint16_
             amax = std::max(amax, fabsf(v));
         }
     }
-    const float S = (amax == 0.0f) ? 1.0f : amax / 2688.0f;
+    // per-tensor scale: amax / (6 q_max) with q_max the largest group scale (448; 384 = 1.5 x 2^8 for C2)
+    const float S = (amax == 0.0f) ? 1.0f : amax / (c2 ? 2304.0f : 2688.0f);
     const float denom = 6.0f * S;
     uint8_t* base = (uint8_t*)packed;
     memset(base, 0, L.total);
     uint8_t* codes = base + L.off_codes;
     uint8_t* scales = base + L.off_scales;
     uint16_t* dqw = (uint16_t*)(base + L.off_dqw);
+    if (c2) {
+        // C2: per 32 channels, two restricted group scales (the smaller raised to at least 2^-10 of the
+        // larger, so the 32 values q s_b fit one UE8M0 exponent exactly), E2M1 codes, and the FP8 form:
+        // E4M3 codes of q s_b / 2^u with the block's largest |q s_b| / 2^u in [256, 512)
+        uint8_t* fp8 = base + L.off_dqw;
+        uint8_t* ue = fp8 + (size_t)Co * Ci;
 #pragma omp parallel for schedule(static)
-    for (long o = 0; o < Co; o++) {
+        for (long o = 0; o < Co; o++) {
+            const float* z = &R[(size_t)o * Ci];
+            for (int j = 0; j < Ci / 32; j++) {
+                float sb[2];
+                for (int hh = 0; hh < 2; hh++) {
+                    float am = 0.0f;
+                    for (int i = 0; i < 16; i++) am = std::max(am, fabsf(z[32 * j + 16 * hh + i]));
+                    sb[hh] = std::min(c2_round_scale_up(am / denom), 384.0f);
+                }
+                const float floor_s = ldexpf(std::max(sb[0], sb[1]), -10);
+                float w[32], wmax = 0.0f;
+                for (int hh = 0; hh < 2; hh++) {
+                    const float sbv = std::max(sb[hh], floor_s);
+                    const uint8_t code = float_to_e4m3(sbv);   // exact: a restricted scale is an E4M3 value
+                    const int b = 2 * j + hh;
+                    const size_t so = dq::sfb_offset(o, b, Ci);
+                    for (int q = 0; q < 4; q++) scales[so + 1024 * q] = code;
+                    const float eff = sbv * S;
+                    for (int i = 0; i < 16; i += 2) {
+                        const uint8_t q0 = (eff == 0.0f) ? 0 : float_to_e2m1(z[b * 16 + i] / eff);
+                        const uint8_t q1 = (eff == 0.0f) ? 0 : float_to_e2m1(z[b * 16 + i + 1] / eff);
+                        codes[(size_t)o * (Ci / 2) + (b * 16 + i) / 2] = (uint8_t)(q0 | (q1 << 4));
+                        w[16 * hh + i] = e2m1_to_float(q0) * sbv;       // exact products
+                        w[16 * hh + i + 1] = e2m1_to_float(q1) * sbv;
+                    }
+                }
+                for (int i = 0; i < 32; i++) wmax = std::max(wmax, fabsf(w[i]));
+                int u = 0;
+                if (wmax > 0.0f) {
+                    int e;
+                    frexpf(wmax, &e);    // wmax in [2^(e-1), 2^e)
+                    u = e - 9;
+                }
+                for (int i = 0; i < 32; i++) fp8[(size_t)o * Ci + 32 * j + i] = float_to_e4m3(ldexpf(w[i], -u));
+                const size_t uo = dq::c2_sf_offset(o, j, Ci);
+                for (int q = 0; q < 4; q++) ue[uo + 1024 * q] = (uint8_t)(u + 127);
+            }
+        }
+    }
+#pragma omp parallel for schedule(static)
+    for (long o = 0; o < (c2 ? 0 : Co); o++) {
         const float* z = &R[(size_t)o * Ci];
         for (int b = 0; b < Ci / 16; b++) {
             float am = 0.0f;
@@ -475,7 +538,7 @@ int dq_pack_weight_factors(const uint16_t* Wb, const uint16_t* L1, const uint16_
     hdr.S_W = S;
     hdr.off_codes = L.off_codes; hdr.off_scales = L.off_scales; hdr.off_dqw = L.off_dqw; hdr.total = L.total;
     hdr.off_bias = L.off_bias;
-    hdr.flags = 0;
+    hdr.flags = c2 ? dq::kPackedC2 : 0u;
     memcpy(base, &hdr, sizeof(hdr));
     if (L1_mma)
         for (int i = 0; i < Ci; i++)
@@ -486,6 +549,11 @@ int dq_pack_weight_factors(const uint16_t* Wb, const uint16_t* L1, const uint16_
                 L2_slab[(size_t)o * L.slab + c] = (c < 2 * r) ? L2[(size_t)(c % r) * Co + o] : (uint16_t)0;
     if (S_W_out) *S_W_out = S;
     return DQ_OK;
+}
+
+int dq_pack_weight_factors(const uint16_t* Wb, const uint16_t* L1, const uint16_t* L2, int Co, int Ci, int rank,
+                           void* packed, size_t packed_bytes, uint16_t* L1_mma, uint16_t* L2_slab, float* S_W_out) {
+    return dq_pack_weight_factors_ex(Wb, L1, L2, Co, Ci, rank, 0, packed, packed_bytes, L1_mma, L2_slab, S_W_out);
 }
 
 int dq_pack_bias(const uint16_t* bias, int Co, void* packed, size_t packed_bytes) {

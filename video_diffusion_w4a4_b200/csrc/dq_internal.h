@@ -20,6 +20,7 @@ struct QuantParams {
     int m_rows;         // kernel tokens per box (rows of the encode kernel's per-stage tile)
     int stat_pairs;     // statistics kernel: one warp per cube, a channel pair per lane (cubes of 16+ tokens)
     int kgroup;         // 0: s8 per kernel token (K); 64: per 64 channels (K x Ci/64), q8_bf16 = [hi | lo]
+    int fp8_product;    // the kernel-token product reads q8 (C2 weights): no q8_bf16, packed weight must be C2
     int big;            // cubes of more than 128 tokens: boxes are row segments of one cube,
     int nseg;           //   nseg segments of up to 128 tokens per cube row; the kernel tokens
     float* means;       //   K x Ci fp32 kernel tokens: written by k_cube_stats (by k_cube_means_big for big cubes)
@@ -57,6 +58,10 @@ struct GemmParams {
     uint64_t budget_ns;
 };
 
+// Paired-GEMM kinds: the exact kernel-token product (BF16, kind::f16), the main block-scaled FP4
+// product, the FP8 kernel-token product on C2 weights (kind::mxf8f6f4, UE8M0 scales per 32).
+enum GemmKind { kGemmKernelBf16 = 0, kGemmMain = 1, kGemmKernelFp8 = 2 };
+
 size_t quant_smem_bytes(int rank, bool stats, int m_rows, int x_rows);
 cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
                               cudaStream_t st);
@@ -66,6 +71,8 @@ cudaError_t launch_cube_means_big(const CUtensorMap& tm_x, const QuantParams& p,
 
 cudaError_t launch_kernel_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmParams& p,
                                cudaStream_t st);
+cudaError_t launch_kernel_gemm_fp8(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_fb,
+                                   const GemmParams& p, cudaStream_t st);
 cudaError_t launch_main_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_sa,
                              const CUtensorMap& tm_sb, const CUtensorMap& tm_fa, const CUtensorMap& tm_fb,
                              const GemmParams& p, cudaStream_t st);

@@ -335,6 +335,39 @@ __device__ __forceinline__ void mma_nvfp4_pair(uint32_t d_tmem, uint64_t adesc, 
         : "memory");
 }
 
+// Paired block-scaled FP8 MMA (kind::mxf8f6f4, E4M3 x E4M3, one UE8M0 scale per 32 K of each row;
+// the instruction descriptor's scale-factor ids pick the byte of the 32-bit tensor-memory word).
+__device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Instruction descriptor, kind::mxf8f6f4: E4M3 x E4M3 -> fp32, K-major, K = 32, UE8M0 scales; the
+// MMA reads byte sf_a / sf_b of each scale word.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, uint32_t sf_a, uint32_t sf_b) {
+    return ((sf_b & 3u) << 4)           // B scale-factor byte
+           | (0u << 7)                  // A = E4M3
+           | (0u << 10)                 // B = E4M3
+           | ((uint32_t)(N >> 3) << 17) //
+           | (1u << 23)                 // scale format UE8M0
+           | ((uint32_t)(M >> 4) << 24) //
+           | ((sf_a & 3u) << 29);       // A scale-factor byte
+}
+
+// Each thread of the warp writes four consecutive 32-bit columns of its lane.
+__device__ __forceinline__ void tmem_st_x4(uint32_t taddr, uint32_t v0, uint32_t v1, uint32_t v2, uint32_t v3) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(v0), "r"(v1),
+                 "r"(v2), "r"(v3)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // ------------------------------------------------------------------ 256-bit global access (sm_100)
 
 // Eight fp32 from 32-byte aligned global memory through the non-coherent path.

@@ -669,7 +669,8 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
         *abort_flag = 0;
         fence_barrier_init();
         if (blockIdx.x == 0 &&
-            (hdr->magic != DQ_PACK_MAGIC || hdr->version != DQ_PACK_FORMAT_VERSION || hdr->Ci != p.Ci || hdr->rank != p.rank || hdr->slab != p.slab))
+            (hdr->magic != DQ_PACK_MAGIC || hdr->version != DQ_PACK_FORMAT_VERSION || hdr->Ci != p.Ci ||
+             hdr->rank != p.rank || hdr->slab != p.slab || ((hdr->flags & kPackedC2) != 0) != (p.fp8_product != 0)))
             atomicCAS(p.status, 0, kStatusBadWeight);
     }
     // per-tensor delta scale S = amax / (6*448) (1 if amax = 0); S_W from the packed weight
@@ -814,7 +815,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                         uint16_t* arow = p.q8_bf16 + (size_t)k * (2 * Ci) + c0 + 8 * g8;
                         *reinterpret_cast<uint4*>(arow) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
                         *reinterpret_cast<uint4*>(arow + Ci) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-                    } else {
+                    } else if (!p.fp8_product) {
                         // exact: E4M3 values have four significant bits
                         uint32_t bfw[4];
 #pragma unroll
