@@ -50,14 +50,15 @@ def layer_flops(wl, K):
     return 2.0 * wl.N * wl.Ci * wl.Co + 2.0 * K * wl.Ci * wl.Co + 2.0 * wl.N * wl.rank * (wl.Ci + wl.Co)
 
 
-def stage_model(wl, K, slab, kernel_group=0, fp8=False):
+def stage_model(wl, K, slab, kernel_group=0, fp8=False, pow2=False):
     """Algorithmic work per launch of each stage (bytes that must cross HBM,
     tensor FLOPs).  Stage 1 reads X twice (statistics, then encode: the
     per-tensor delta scale needs every delta first).  fp8: the FP8 kernel-token
     product reads q8 and the FP8 weight (1 byte each) plus one exponent per 32."""
     N, Ci, Co, r = wl.N, wl.Ci, wl.Co, wl.rank
     q8_copy = 0 if fp8 else (4 if kernel_group else 2)   # BF16 operand of the exact product (hi + lo when grouped)
-    quant_bytes = (4.0 * N * Ci                      # X read by a1 and a2
+    quant_bytes = ((2.0 if pow2 else 4.0) * N * Ci  # X read by a1 and a2 (once by the single-read quantiser)
+                   + (N * Ci / 64 * 2 + N * Ci / 16 * 2 if pow2 else 0.0)  # provisional exponents, scale fix-up
                    + N * Ci / 2 + N * Ci / 16        # delta codes + scales
                    + K * Ci * (1 + q8_copy)          # q8 (E4M3) + the product's BF16 operand
                    + N * r * 4 * 2                   # X L1 partials (write + read)
@@ -198,12 +199,13 @@ class OracleLayer:
     """The oracle's weight side and whole-tensor statistics pass of one workload, and
     timed runs over sets of its cubes."""
 
-    def __init__(self, wl, cube, X, L1, L2, wq):
+    def __init__(self, wl, cube, X, L1, L2, wq, pow2=False):
         import oracle
         self.oracle, self.wl, self.cube, self.X, self.L1, self.L2, self.wq = oracle, wl, cube, X, L1, L2, wq
         t0 = time.perf_counter()
         # S_delta needs the max |delta| of the whole tensor: the oracle's statistics pass over all cubes
-        self.S = oracle.tensor_scale(oracle.delta_amax(X, wl.T, wl.H, wl.W, cube))
+        amax = oracle.delta_amax(X, wl.T, wl.H, wl.W, cube)
+        self.S = oracle.pow2_scale(amax) if pow2 else oracle.tensor_scale(amax)
         self.stats_s = time.perf_counter() - t0
         self.K = oracle.num_cubes(wl.T, wl.H, wl.W, *cube)
         self.threads = oracle.num_threads()
@@ -222,11 +224,12 @@ class OracleLayer:
         return self.stats_s + sample_s * self.wl.N / sample_tokens
 
 
-def bench_config(wl, cube, K, kernel_group, world, parallelism, fp8=False):
+def bench_config(wl, cube, K, kernel_group, world, parallelism, fp8=False, pow2=False):
     """The `config` object of the JSON line, identical for the GPU arm and the reference arm."""
     return dict(workload=wl.name, T=wl.T, H=wl.H, W=wl.W, N=wl.N, Ci=wl.Ci, Co=wl.Co, rank=wl.rank, cube=list(cube),
                 K=K, kernel_scale="per-token" if not kernel_group else f"group{kernel_group}",
                 kernel_product="fp8 (restricted-scale C2 weights)" if fp8 else "bf16 (exact)",
+                delta_scale="power of two (single read of X)" if pow2 else "amax / 2688 (two reads of X)",
                 parallelism=(f"cube-sharded x{world} (T-slabs of whole cube layers, NCCL all-reduce(max) of the "
                              f"delta amax)" if parallelism == "sharded" and world > 1
                              else f"dp{world} (independent layer per GPU)"),
@@ -243,8 +246,9 @@ def run_reference(args, wl, cube):
     Wb = synth.weight(wl)
     L1, L2, _ = oracle.lowrank_factors(Wb, wl.rank)
     fp8 = args.kernel_product == "fp8"
+    pow2 = args.delta_scale == "pow2"
     wq = oracle.quantize_weight(Wb, L1, L2, c2=fp8)
-    layer = OracleLayer(wl, cube, X, L1, L2, wq)
+    layer = OracleLayer(wl, cube, X, L1, L2, wq, pow2)
     cubes, full = oracle_sample_cubes(wl, cube)
     if wl.name == "tiny":
         slices = [cubes]
@@ -270,7 +274,7 @@ def run_reference(args, wl, cube):
                 warmup=args.warmup, ms_per_step=sample_s / args.steps * 1e3, higher_is_better=True,
                 scaling="weak" if args.gpus == 1 or args.parallelism == "replicas" else "strong",
                 vs_baseline=None, dtype="f64", data="synthetic",
-                config=bench_config(wl, cube, K, args.kernel_group, args.gpus, args.parallelism, fp8),
+                config=bench_config(wl, cube, K, args.kernel_group, args.gpus, args.parallelism, fp8, pow2),
                 tokens_per_s=wl.N / t_full, sample_tflops=sum(layer_flops_rows(wl, K, n) for n in toks) / sample_s / 1e12,
                 cpu_baseline=dict(value=value, unit="TFLOP/s", cores=layer.threads, kind="oracle", sample=sample,
                                   sample_seconds=sample_s, extrapolated_full_seconds=t_full),
@@ -300,6 +304,9 @@ def main():
                     help="FP8 kernel-token scales: 0 = one per token, 64 = one per 64 channels")
     ap.add_argument("--kernel-product", default="bf16", choices=["bf16", "fp8"],
                     help="kernel-token product: exact BF16 operands (default) or FP8 on restricted-scale (C2) weights")
+    ap.add_argument("--delta-scale", default="amax", choices=["amax", "pow2"],
+                    help="per-tensor delta scale: amax / 2688 (default, two reads of X) or its power of two "
+                         "(single-read quantiser)")
     ap.add_argument("--parallelism", default="sharded", choices=["sharded", "replicas"],
                     help="with several GPUs: one layer sharded by cubes (default) or one layer per GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -336,8 +343,12 @@ def main():
     kg = args.kernel_group
     fp8 = args.kernel_product == "fp8"
     kp = dq.DQ_KERNEL_PRODUCT_FP8 if fp8 else dq.DQ_KERNEL_PRODUCT_BF16
-    if sharded and (kg or fp8):
-        ap.error("the cube-sharded layer takes per-token kernel scales and the BF16 kernel-token product")
+    pow2 = args.delta_scale == "pow2"
+    ds = dq.DQ_DELTA_SCALE_POW2 if pow2 else dq.DQ_DELTA_SCALE_AMAX
+    if pow2 and kg:
+        ap.error("the single-read quantiser takes per-token kernel scales")
+    if sharded and (kg or fp8 or pow2):
+        ap.error("the cube-sharded layer takes the default options")
     if fp8 and kg:
         ap.error("the FP8 kernel-token product takes per-token kernel scales")
 
@@ -368,7 +379,7 @@ def main():
     L2d = torch.from_numpy(L2s.view(np.int16)).to(dev)
     Yd = torch.empty((Nm, wl.Co), dtype=torch.int16, device=dev)
     lay = dq.dq_workspace_layout_opts(Ts, wl.H, wl.W, ts, hs, ws_, wl.Ci, wl.Co, wl.rank, kernel_group=kg,
-                                      kernel_product=kp)
+                                      kernel_product=kp, delta_scale=ds)
     ws = torch.zeros(lay.total_bytes, dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream(dev)
 
@@ -378,7 +389,8 @@ def main():
     def step(events=None, pre=None):
         if not sharded:
             dq.dq_linear_forward_opts(Xd, Ts, wl.H, wl.W, ts, hs, ws_, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd, ws,
-                                      lay.total_bytes, dq.DQ_STAGE_ALL, events, st, kernel_group=kg, kernel_product=kp)
+                                      lay.total_bytes, dq.DQ_STAGE_ALL, events, st, kernel_group=kg, kernel_product=kp,
+                                      delta_scale=ds)
             return
         # the cube-sharded layer: statistics of this slab, the one exchanged scalar (NCCL), then
         # encode and both products
@@ -438,7 +450,7 @@ def main():
         Yh.copy_(Yd2, non_blocking=True)
 
     e2e_ms = None
-    if not kg and not fp8:   # the host-buffer entry point takes the default options
+    if not kg and not fp8 and not pow2:   # the host-buffer entry point takes the default options
         e2e_step()
         torch.cuda.synchronize(dev)
         if dist:
@@ -462,7 +474,7 @@ def main():
     # per-stage work model of this rank's share (its slab when sharded)
     wl_mine = wl if not sharded else synth.Workload(wl.name, Ts, wl.H, wl.W, wl.Ci, wl.Co, wl.rank, (ts, hs, ws_),
                                                     wl.grid, wl.x_outliers, wl.w_outliers, wl.gelu)
-    model = stage_model(wl_mine, int(lay.K), lay.slab, kg, fp8)
+    model = stage_model(wl_mine, int(lay.K), lay.slab, kg, fp8, pow2)
     # dominant kernel = the stage with the largest share of the step
     dom = max(("quantize", "kernel_gemm", "main_gemm"), key=stage_ms.get)
     if dom == "quantize":
@@ -476,7 +488,7 @@ def main():
                     bound="tensor", achieved=ach, peak=pk, unit="TFLOP/s")
     roof["frac"] = roof["achieved"] / roof["peak"]
     same_cube = tuple(cube) == tuple(synth.WORKLOADS[args.workload].cube)
-    roof["traffic"] = committed_traffic(wl_mine, dom) if same_cube and not kg and not fp8 else None
+    roof["traffic"] = committed_traffic(wl_mine, dom) if same_cube and not kg and not fp8 and not pow2 else None
     roof["peak_source"] = ("measured" if peaks["source"] == "measured" else "fallback") + (
         " bf16 x 4 (nominal FP4:BF16)" if roof["unit"] == "TFLOP/s" and dom == "main_gemm" else
         " bf16 x 2 (nominal FP8:BF16)" if roof["unit"] == "TFLOP/s" and fp8 else "")
@@ -499,7 +511,7 @@ def main():
     line = dict(metric=METRIC, value=value, unit="TFLOP/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
                 ms_per_step=ms, higher_is_better=True, scaling="strong" if sharded else "weak", vs_baseline=None,
                 dtype="e2m1/e4m3->f32", data="synthetic",
-                config=bench_config(wl, cube, K, kg, world, args.parallelism, fp8),
+                config=bench_config(wl, cube, K, kg, world, args.parallelism, fp8, pow2),
                 tokens_per_s=wl.N * (1 if sharded else world) / (ms * 1e-3),
                 layer_roofline_frac=layer_roof_ms / ms,
                 roofline=roof, stages=stages,
@@ -519,7 +531,7 @@ def main():
         oracle.build()
         L1, L2 = dq.dq_lowrank_factors(Wb, wl.rank)
         wq = oracle.quantize_weight(Wb, L1, L2, c2=fp8)
-        layer = OracleLayer(wl, cube, X, L1, L2, wq)
+        layer = OracleLayer(wl, cube, X, L1, L2, wq, pow2)
         cubes, full = oracle_sample_cubes(wl, cube)
         dt, n = layer.run(cubes)
         t_full = dt if full else layer.full_seconds(dt, n)

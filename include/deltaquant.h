@@ -266,6 +266,9 @@ int dq_pack_weight(const uint16_t* W, int Co, int Ci, int rank, void* packed, si
  *   u_hilo     N x slab BF16: U' = (X L1)/(S_delta S_W) split as hi + lo
  *   p          K x Co fp32: s8 S_W q8 dqw^T (the per-cube kernel term)
  *   means      K x Ci fp32 kernel tokens before quantisation
+ *   prov       DQ_DELTA_SCALE_POW2 only: N x Ci/64 int8 exponents of the
+ *              provisional per-chunk delta scales (-128: all deltas of the
+ *              chunk are zero); empty otherwise
  */
 typedef struct dq_workspace_layout {
     size_t total_bytes;
@@ -274,6 +277,7 @@ typedef struct dq_workspace_layout {
     long long N, K, N_pad, K_pad;
     int splits, slab;
     int kernel_group;
+    size_t off_prov;
 } dq_workspace_layout;
 
 /*
@@ -364,17 +368,35 @@ int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, 
  *                   kind::mxf8f6f4, at twice the BF16 rate; per-token kernel
  *                   scales only.  The product is the same exact sum as with
  *                   BF16 operands of the same (C2) weights.
+ *   delta_scale     DQ_DELTA_SCALE_AMAX: the per-tensor delta scale S = amax / 2688
+ *                   (Eq. 4 with two levels); the quantise stage reads X twice, since
+ *                   no delta can be encoded before every delta's amax is known.
+ *                   DQ_DELTA_SCALE_POW2: S = the smallest power of two >= amax / 2688
+ *                   (1 if amax = 0), a deviation from Eq. 4 that lets X be read once:
+ *                   the statistics pass also encodes each 64-channel chunk under
+ *                   the chunk's own power-of-two scale S_c <= S (its exponent kept in
+ *                   the workspace section prov), and the encode stage then lowers
+ *                   each group's E4M3 scale code by 8 log2(S / S_c), keeping its E2M1
+ *                   codes, or encodes the group again under S when the code's
+ *                   exponent field is below log2(S / S_c) + 1 (E4M3's subnormal
+ *                   grid); the result equals encoding every group under S.  The
+ *                   encode stage also forms the kernel tokens and U' from the stored
+ *                   means and partial sums (no read of X apart from re-encoded
+ *                   groups).  Per-token kernel scales only.
  *   reserved        must be 0
  * A packed weight whose C2 flag does not match kernel_product is reported as
  * DQ_ERR_BAD_PACKED_WEIGHT in the device status word.
  */
 #define DQ_KERNEL_PRODUCT_BF16 0
 #define DQ_KERNEL_PRODUCT_FP8 1
+#define DQ_DELTA_SCALE_AMAX 0
+#define DQ_DELTA_SCALE_POW2 1
 
 typedef struct dq_forward_options {
     int kernel_group;
     int kernel_product;
-    int reserved[2];
+    int delta_scale;
+    int reserved;
 } dq_forward_options;
 
 int dq_workspace_layout_opts(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,

@@ -126,6 +126,14 @@ def tensor_scale(amax: float) -> float:
     return float(_L().or_tensor_scale(amax))
 
 
+def pow2_scale(amax: float) -> float:
+    """The power-of-two per-tensor delta scale: the smallest power of two >= amax / 2688
+    (1 if amax = 0), as quantize_activations(pow2_scales=True) takes it."""
+    if amax == 0.0:
+        return 1.0
+    return float(_L().or_pow2_ceil(float(np.float32(np.float32(amax) / np.float32(2688.0)))))
+
+
 # --------------------------------------------------------------------------- cubes
 
 def num_cubes(T, H, W, t, h, w) -> int:

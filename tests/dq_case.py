@@ -84,9 +84,11 @@ class Case:
     """One layer instance: workload, inputs, oracle factors."""
 
     def __init__(self, wl: synth.Workload, cube=None, seed=None, tau: int = 0, X=None, Wb=None, kernel_group: int = 0,
-                 fp8_product: bool = False):
+                 fp8_product: bool = False, pow2: bool = False):
         self.wl = wl
         self.kernel_group = kernel_group
+        # the single-read quantiser: power-of-two per-tensor delta scale
+        self.pow2 = pow2
         # the FP8 kernel-token product: weights packed with restricted (C2) scales
         self.fp8_product = fp8_product
         self.cube = tuple(cube or wl.cube)
@@ -111,13 +113,15 @@ class Case:
         Yd = torch.empty((wl.N, wl.Co), dtype=torch.int16, device=dev)
         kg = self.kernel_group
         kp = dq.DQ_KERNEL_PRODUCT_FP8 if self.fp8_product else dq.DQ_KERNEL_PRODUCT_BF16
+        ds = dq.DQ_DELTA_SCALE_POW2 if self.pow2 else dq.DQ_DELTA_SCALE_AMAX
         lay = dq.dq_workspace_layout_opts(wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, kernel_group=kg,
-                                          kernel_product=kp)
+                                          kernel_product=kp, delta_scale=ds)
         ws = torch.zeros(lay.total_bytes, dtype=torch.uint8, device=dev)
-        if self.fp8_product:
+        self.last_ws, self.last_layout, self.last_inputs = ws, lay, (Xd, Pd, L1d, L2d, Yd)
+        if self.fp8_product or self.pow2:
             dq.dq_linear_forward_opts(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd, ws,
                                       lay.total_bytes, stage_mask, None, torch.cuda.current_stream(),
-                                      kernel_group=kg, kernel_product=kp)
+                                      kernel_group=kg, kernel_product=kp, delta_scale=ds)
         elif kg:
             dq.dq_linear_forward_grouped(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, kg, Pd, L1d, L2d, Yd,
                                          ws, lay.total_bytes, stage_mask, None, torch.cuda.current_stream())
@@ -141,12 +145,15 @@ class Case:
                    dcodes=wsh[lay.off_dcodes:lay.off_dcodes + N * Ci // 2].reshape(N, Ci // 2),
                    dscales=sfa_unpermute(wsh[lay.off_dscales:], N, Ci),
                    p=wsh[lay.off_p:lay.off_p + 4 * K * wl.Co].view(np.float32).reshape(K, wl.Co))
+        if self.pow2:
+            out["prov"] = wsh[lay.off_prov:lay.off_prov + N * (Ci // 64)].view(np.int8).reshape(N, Ci // 64)
         return out
 
     # ---------------------------------------------------------------- oracle
     def run_oracle(self):
         wl = self.wl
-        act = oracle.quantize_activations(self.X, wl.T, wl.H, wl.W, self.cube, kernel_group=self.kernel_group)
+        act = oracle.quantize_activations(self.X, wl.T, wl.H, wl.W, self.cube, kernel_group=self.kernel_group,
+                                          pow2_scales=self.pow2)
         wq = oracle.quantize_weight(self.Wb, self.L1, self.L2, c2=self.fp8_product)
         return act, wq
 

@@ -176,6 +176,67 @@ def test_packed_weight_must_match_the_kernel_product(env):
     assert out["status"] == dq.DQ_ERR_BAD_PACKED_WEIGHT
 
 
+@pytest.mark.parametrize("name", ["tiny", "ragged_122", "ragged_222", "unit_cube", "cube_244", "cube_418", "gelu_122",
+                                  "cube_414_r128", "cube_428", "global", "big_cube", "wide_cube"])
+def test_parity_single_read(env, name):
+    """The single-read quantiser (power-of-two S_delta, one read of X): every
+    quantised tensor bit-exact against the oracle's direct encode under the final
+    power-of-two scale, S_delta too; P' and Y within tolerance; every cube shape,
+    ragged lattices, big cubes whose means come from the means kernel."""
+    dq, torch = env
+    wl = dict(SMALL)[name] or synth.WORKLOADS["tiny"]
+    case = Case(wl, pow2=True)
+    g = case.run_gpu(dq, torch)
+    act, wq = case.run_oracle()
+    assert act["pow2_scales"] and float(act["S_delta"]) == 2.0 ** round(np.log2(act["S_delta"]))
+    compare_quantised(g, act, wq)
+    assert_kernel_term_close(g["p"], act, wq, np.arange(g["layout"].K))
+    assert_y_close(g["Y"], case.oracle_rows(act, wq, np.arange(wl.N)))
+
+
+def test_single_read_with_fp8_product(env):
+    """Both options together: single-read quantiser and the FP8 kernel-token product."""
+    dq, torch = env
+    wl = dict(SMALL)["ragged_122"]
+    case = Case(wl, pow2=True, fp8_product=True)
+    g = case.run_gpu(dq, torch)
+    act, wq = case.run_oracle()
+    compare_quantised(g, act, wq)
+    assert_kernel_term_close(g["p"], act, wq, np.arange(g["layout"].K))
+    assert_y_close(g["Y"], case.oracle_rows(act, wq, np.arange(wl.N)))
+
+
+def _spiky(wl, seed=5):
+    """Low-amplitude activations with large outliers in the last frame's last 64 channels: every
+    other 64-channel chunk's own power-of-two scale lies about 20 binades below the final one, so
+    the fix-up pass must encode their groups again (E4M3's exponent field has no such headroom)."""
+    x = oracle.bf16_value(synth.activations(wl, seed=seed)).astype(np.float64) * 1e-4
+    last = np.arange((wl.T - 1) * wl.H * wl.W, wl.N)
+    sign = np.where(np.arange(64) % 2 == 0, 1.0, -1.0)
+    x[np.ix_(last, np.arange(wl.Ci - 64, wl.Ci))] = sign[None, :] * (500.0 + 7.0 * (last[:, None] % 13))
+    return oracle.bf16_round_fast(x)
+
+
+def test_single_read_reencodes_groups_without_headroom(env):
+    """The fix-up pass's re-encode branch, forced: after the statistics pass alone,
+    many groups have provisional scale codes whose exponent field is below the shift
+    j + 1; after the encode stage every tensor equals the oracle's direct encode."""
+    dq, torch = env
+    wl = dict(SMALL)["ragged_122"]
+    case = Case(wl, X=_spiky(wl), pow2=True)
+    act, wq = case.run_oracle()
+    g1 = case.run_gpu(dq, torch, stage_mask=dq.DQ_STAGE_STATS)
+    es = int(round(np.log2(act["S_delta"])))
+    prov = g1["prov"].astype(int)                              # N x Ci/64, cube-major rows
+    codes = g1["dscales"].astype(int)                          # provisional, N x Ci/16
+    j = es - np.repeat(prov, 4, axis=1)
+    need = (np.repeat(prov, 4, axis=1) != -128) & (codes != 0) & (((codes >> 3) & 15) < j + 1)
+    assert need.sum() > 100, int(need.sum())
+    g = case.run_gpu(dq, torch)
+    compare_quantised(g, act, wq)
+    assert_y_close(g["Y"], case.oracle_rows(act, wq, np.arange(wl.N)))
+
+
 def test_worked_example_through_gpu(env):
     """The hand-derived example (tests/golden) padded to 256 channels with zeros."""
     dq, torch = env

@@ -474,6 +474,7 @@ def test_pow2_delta_scale_closed_form(tiny_case):
     ref = oracle.quantize_activations(X, wl.T, wl.H, wl.W, wl.cube)
     S, amax = act["S_delta"], act["amax_delta"]
     assert _is_pow2(S) and amax / 2688 <= S < amax / 1344
+    assert oracle.pow2_scale(amax) == S and oracle.pow2_scale(0.0) == 1.0
     assert np.array_equal(act["q8"], ref["q8"]) and np.array_equal(act["s8"], ref["s8"])
     assert np.array_equal(act["means"], ref["means"])
 

@@ -39,6 +39,7 @@ DQ_KERNEL_SCALE_PER_TOKEN, DQ_KERNEL_SCALE_GROUP64 = 0, 64
 DQ_NOALLOC_WORKSPACE = 1   # dq_read_device_status: the fixed array of dq_linear_forward_noalloc
 DQ_PACK_C2 = 1
 DQ_KERNEL_PRODUCT_BF16, DQ_KERNEL_PRODUCT_FP8 = 0, 1
+DQ_DELTA_SCALE_AMAX, DQ_DELTA_SCALE_POW2 = 0, 1
 
 
 class dq_packed_layout(ctypes.Structure):
@@ -52,11 +53,12 @@ class dq_workspace_layout(ctypes.Structure):
         (n, ctypes.c_size_t) for n in ("off_status", "off_scalars", "off_kamax", "off_s8", "off_q8", "off_q8_bf16",
                                        "off_dcodes", "off_dscales", "off_u_part", "off_u_hilo", "off_p", "off_means")] + [
         ("N", ctypes.c_longlong), ("K", ctypes.c_longlong), ("N_pad", ctypes.c_longlong), ("K_pad", ctypes.c_longlong),
-        ("splits", ctypes.c_int), ("slab", ctypes.c_int), ("kernel_group", ctypes.c_int)]
+        ("splits", ctypes.c_int), ("slab", ctypes.c_int), ("kernel_group", ctypes.c_int), ("off_prov", ctypes.c_size_t)]
 
 
 class dq_forward_options(ctypes.Structure):
-    _fields_ = [("kernel_group", ctypes.c_int), ("kernel_product", ctypes.c_int), ("reserved", ctypes.c_int * 2)]
+    _fields_ = [("kernel_group", ctypes.c_int), ("kernel_product", ctypes.c_int), ("delta_scale", ctypes.c_int),
+                ("reserved", ctypes.c_int)]
 
 
 _P, _I, _SZ, _LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
@@ -283,17 +285,19 @@ def dq_workspace_layout_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group) ->
     return L
 
 
-def _options(kernel_group=DQ_KERNEL_SCALE_PER_TOKEN, kernel_product=DQ_KERNEL_PRODUCT_BF16):
+def _options(kernel_group=DQ_KERNEL_SCALE_PER_TOKEN, kernel_product=DQ_KERNEL_PRODUCT_BF16,
+             delta_scale=DQ_DELTA_SCALE_AMAX):
     o = dq_forward_options()
-    o.kernel_group, o.kernel_product = kernel_group, kernel_product
+    o.kernel_group, o.kernel_product, o.delta_scale = kernel_group, kernel_product, delta_scale
     return o
 
 
 def dq_workspace_layout_opts(T, H, W, t, h, w, Ci, Co, rank, kernel_group=DQ_KERNEL_SCALE_PER_TOKEN,
-                             kernel_product=DQ_KERNEL_PRODUCT_BF16) -> dq_workspace_layout:
+                             kernel_product=DQ_KERNEL_PRODUCT_BF16,
+                             delta_scale=DQ_DELTA_SCALE_AMAX) -> dq_workspace_layout:
     """Workspace carve-up for the forward options (dq_forward_options fields as keywords)."""
     L = dq_workspace_layout()
-    o = _options(kernel_group, kernel_product)
+    o = _options(kernel_group, kernel_product, delta_scale)
     _check("dq_workspace_layout_opts", _lib.dq_workspace_layout_opts(T, H, W, t, h, w, Ci, Co, rank, ctypes.byref(o),
                                                                      ctypes.byref(L)))
     return L
@@ -301,9 +305,10 @@ def dq_workspace_layout_opts(T, H, W, t, h, w, Ci, Co, rank, kernel_group=DQ_KER
 
 def dq_linear_forward_opts(X, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y, workspace,
                            workspace_bytes, stage_mask=DQ_STAGE_ALL, stage_events=None, stream=None,
-                           kernel_group=DQ_KERNEL_SCALE_PER_TOKEN, kernel_product=DQ_KERNEL_PRODUCT_BF16) -> None:
+                           kernel_group=DQ_KERNEL_SCALE_PER_TOKEN, kernel_product=DQ_KERNEL_PRODUCT_BF16,
+                           delta_scale=DQ_DELTA_SCALE_AMAX) -> None:
     """dq_linear_forward_ex with forward options (dq_forward_options fields as keywords)."""
-    o = _options(kernel_group, kernel_product)
+    o = _options(kernel_group, kernel_product, delta_scale)
     _check("dq_linear_forward_opts",
            _lib.dq_linear_forward_opts(_ptr(X), T, H, W, t, h, w, Ci, Co, rank, ctypes.byref(o), _ptr(packed_W),
                                        _ptr(L1_mma), _ptr(L2_slab), _ptr(Y), _ptr(workspace), workspace_bytes,

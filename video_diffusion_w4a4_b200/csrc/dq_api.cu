@@ -142,7 +142,10 @@ int check_options(const dq_forward_options& o) {
     // the FP8 product carries the kernel-token scale in its epilogue: one per token
     if (o.kernel_product == DQ_KERNEL_PRODUCT_FP8 && o.kernel_group != DQ_KERNEL_SCALE_PER_TOKEN)
         return DQ_ERR_INVALID_ARG;
-    if (o.reserved[0] || o.reserved[1]) return DQ_ERR_INVALID_ARG;
+    if (o.delta_scale != DQ_DELTA_SCALE_AMAX && o.delta_scale != DQ_DELTA_SCALE_POW2) return DQ_ERR_INVALID_ARG;
+    // the single-read quantiser forms per-token kernel scales in its fix-up pass
+    if (o.delta_scale == DQ_DELTA_SCALE_POW2 && o.kernel_group != DQ_KERNEL_SCALE_PER_TOKEN) return DQ_ERR_INVALID_ARG;
+    if (o.reserved) return DQ_ERR_INVALID_ARG;
     return DQ_OK;
 }
 
@@ -189,7 +192,7 @@ int dq_workspace_layout_opts(int T, int H, int W, int t, int h, int w, int Ci, i
     if ((rc = check_options(o))) return rc;
     const int kernel_group = o.kernel_group;
     dq::WsLayout L = dq::ws_layout(dq::make_geom(T, H, W, t, h, w), Ci, Co, rank, kernel_group,
-                                   o.kernel_product == DQ_KERNEL_PRODUCT_FP8);
+                                   o.kernel_product == DQ_KERNEL_PRODUCT_FP8, o.delta_scale == DQ_DELTA_SCALE_POW2);
     out->total_bytes = L.total;
     out->off_status = L.off_status;
     out->off_scalars = L.off_scalars;
@@ -210,6 +213,7 @@ int dq_workspace_layout_opts(int T, int H, int W, int t, int h, int w, int Ci, i
     out->splits = L.splits;
     out->slab = L.slab;
     out->kernel_group = kernel_group;
+    out->off_prov = L.off_prov;
     return DQ_OK;
 }
 
@@ -254,6 +258,7 @@ int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int
     if ((rc = check_options(o))) return rc;
     const int kg = o.kernel_group;
     const bool fp8prod = o.kernel_product == DQ_KERNEL_PRODUCT_FP8;
+    const bool pow2 = o.delta_scale == DQ_DELTA_SCALE_POW2;
     if (!X || !packed_W || !L1_mma || !L2_slab || !Y || !workspace) return DQ_ERR_INVALID_ARG;
     if (stage_mask <= 0 || (stage_mask & ~(DQ_STAGE_ALL | DQ_STAGE_STATS | DQ_STAGE_ENCODE))) return DQ_ERR_INVALID_ARG;
     const bool do_stats = stage_mask & (DQ_STAGE_QUANTIZE | DQ_STAGE_STATS);
@@ -262,7 +267,7 @@ int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int
         !aligned(workspace))
         return DQ_ERR_ALIGNMENT;
     const Geom g = dq::make_geom(T, H, W, t, h, w);
-    const dq::WsLayout wl = dq::ws_layout(g, Ci, Co, rank, kg, fp8prod);
+    const dq::WsLayout wl = dq::ws_layout(g, Ci, Co, rank, kg, fp8prod, pow2);
     if (workspace_bytes < wl.total) return DQ_ERR_WORKSPACE_TOO_SMALL;
     if (!encode_fn()) return DQ_ERR_NO_DEVICE;
     cudaStream_t st = (cudaStream_t)stream;
@@ -279,6 +284,7 @@ int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int
     qp.splits = wl.splits;
     qp.kgroup = kg;
     qp.fp8_product = fp8prod;
+    qp.pow2 = pow2;
     qp.chunks_per_split = Ci / 64 / wl.splits;
     qp.big = (long long)t * h * w > 128;
     if (!qp.big) {
@@ -315,6 +321,7 @@ int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int
     qp.dscales = ws + wl.off_dscales;
     qp.u_part = (float*)(ws + wl.off_u_part);
     qp.u_hilo = (uint16_t*)(ws + wl.off_u_hilo);
+    qp.prov = (int8_t*)(ws + wl.off_prov);
     qp.packed_w = pw;
     qp.budget_ns = kWaitBudgetNs;
 
@@ -345,10 +352,18 @@ int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int
                 return cuda_fail(e0, "memset");
             if (qp.big && (e = dq::launch_cube_means_big(tm_x, qp, st)) != cudaSuccess)
                 return cuda_fail(e, "k_cube_means_big");
-            if ((e = dq::launch_cube_stats(tm_x, tm_l1, qp, st)) != cudaSuccess) return cuda_fail(e, "k_cube_stats");
+            if (pow2) {
+                if ((e = dq::launch_cube_single(tm_x, tm_l1, qp, st)) != cudaSuccess)
+                    return cuda_fail(e, "k_cube_stats (single read)");
+            } else if ((e = dq::launch_cube_stats(tm_x, tm_l1, qp, st)) != cudaSuccess) {
+                return cuda_fail(e, "k_cube_stats");
+            }
         }
-        if (do_encode && (e = dq::launch_cube_encode(tm_x, tm_m, qp, st)) != cudaSuccess)
+        if (do_encode && pow2) {
+            if ((e = dq::launch_single_finish(X, qp, st)) != cudaSuccess) return cuda_fail(e, "k_single_finish");
+        } else if (do_encode && (e = dq::launch_cube_encode(tm_x, tm_m, qp, st)) != cudaSuccess) {
             return cuda_fail(e, "k_cube_encode");
+        }
     }
     rec(1);
     if ((stage_mask & DQ_STAGE_KERNEL_GEMM) && fp8prod) {

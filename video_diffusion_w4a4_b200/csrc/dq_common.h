@@ -178,14 +178,17 @@ DQ_HD int quant_splits(int Ci) {
 
 struct WsLayout {
     size_t total, off_status, off_scalars, off_kamax, off_s8, off_q8, off_q8_bf16, off_dcodes, off_dscales,
-        off_u_part, off_u_hilo, off_p, off_means;
+        off_u_part, off_u_hilo, off_p, off_means, off_prov;
     long long N, K, N_pad, K_pad;
     int splits, slab;
 };
 
 // kgroup: 0 = one FP8 scale per kernel token; 64 = one per 64 channels, whose
 // kernel tokens enter the product as BF16 hi + lo (twice the columns)
-DQ_HD WsLayout ws_layout(const Geom& g, int Ci, int Co, int rank, int kgroup = 0, bool fp8_product = false) {
+// pow2_single: the single-read quantiser (power-of-two delta scale), which also keeps one provisional
+// scale exponent per (row, 64-channel chunk)
+DQ_HD WsLayout ws_layout(const Geom& g, int Ci, int Co, int rank, int kgroup = 0, bool fp8_product = false,
+                         bool pow2_single = false) {
     WsLayout L;
     L.N = g.N; L.K = g.K;
     L.N_pad = cdiv(g.N, 128) * 128;
@@ -207,6 +210,7 @@ DQ_HD WsLayout ws_layout(const Geom& g, int Ci, int Co, int rank, int kgroup = 0
     L.off_p = off;        off = align_up(off + (size_t)g.K * Co * 4, kAlign);
     // fp32 kernel tokens (written by the statistics pass, read by the encode pass)
     L.off_means = off;    off = align_up(off + (size_t)g.K * Ci * 4, kAlign);
+    L.off_prov = off;     off = align_up(off + (pow2_single ? (size_t)g.N * (Ci / 64) : 0), kAlign);
     L.total = off;
     return L;
 }

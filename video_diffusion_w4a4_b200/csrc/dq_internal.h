@@ -21,6 +21,8 @@ struct QuantParams {
     int stat_pairs;     // statistics kernel: one warp per cube, a channel pair per lane (cubes of 16+ tokens)
     int kgroup;         // 0: s8 per kernel token (K); 64: per 64 channels (K x Ci/64), q8_bf16 = [hi | lo]
     int fp8_product;    // the kernel-token product reads q8 (C2 weights): no q8_bf16, packed weight must be C2
+    int pow2;           // single-read quantiser: power-of-two S_delta, provisional per-chunk scales, fix-up pass
+    int8_t* prov;       //   N x Ci/64 provisional scale exponents (-128: a chunk whose deltas are all zero)
     int big;            // cubes of more than 128 tokens: boxes are row segments of one cube,
     int nseg;           //   nseg segments of up to 128 tokens per cube row; the kernel tokens
     float* means;       //   K x Ci fp32 kernel tokens: written by k_cube_stats (by k_cube_means_big for big cubes)
@@ -68,6 +70,11 @@ cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1,
 cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const CUtensorMap& tm_m, const QuantParams& p,
                                cudaStream_t st);
 cudaError_t launch_cube_means_big(const CUtensorMap& tm_x, const QuantParams& p, cudaStream_t st);
+// single-read quantiser: statistics + provisional encode (one read of X), then the fix-up pass with
+// the kernel tokens and U' (no read of X except for re-encoded groups)
+cudaError_t launch_cube_single(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
+                               cudaStream_t st);
+cudaError_t launch_single_finish(const void* X, const QuantParams& p, cudaStream_t st);
 
 cudaError_t launch_kernel_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const GemmParams& p,
                                cudaStream_t st);

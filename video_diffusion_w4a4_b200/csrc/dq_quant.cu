@@ -40,12 +40,15 @@ constexpr int kQCompute = 32 * kQWarps;
 
 struct QSmem {
     // offsets in bytes from the 1024-aligned dynamic smem base
-    uint32_t x, x_stride, l1, mt, mt_stride, eff, bars, misc, total;
+    uint32_t x, x_stride, l1, mt, mt_stride, ms, ms_stride, red2, eff, bars, misc, total;
 };
 
 // m_rows: rows of the per-stage tile of kernel tokens (encode kernel; 0 for the statistics kernel)
 // x_rows: tokens per TMA box (rows of the X stages; 128 at most)
-__host__ __device__ inline QSmem q_smem_layout(int rank, bool with_l1, int m_rows, int x_rows = 128) {
+// single: the single-read statistics kernel, which also keeps the means of two chunks (m_rows cube
+// slots x 64 fp32 each) and their per-warp delta maxima
+__host__ __device__ inline QSmem q_smem_layout(int rank, bool with_l1, int m_rows, int x_rows = 128,
+                                               bool single = false) {
     QSmem L;
     uint32_t off = 0;
     L.x = off;
@@ -54,12 +57,17 @@ __host__ __device__ inline QSmem q_smem_layout(int rank, bool with_l1, int m_row
     L.l1 = off;
     if (with_l1) off += kQStages * (uint32_t)align_up((size_t)rank * 128, 1024);
     L.mt = off;
-    L.mt_stride = (uint32_t)align_up((size_t)m_rows * 256, 128);
+    L.mt_stride = single ? 0u : (uint32_t)align_up((size_t)m_rows * 256, 128);
     off += kQStages * L.mt_stride;
+    L.ms = off;
+    L.ms_stride = single ? (uint32_t)align_up((size_t)m_rows * 256, 128) : 0u;
+    off += 2 * L.ms_stride;
+    L.red2 = off;
+    if (single) off += 2 * kQWarps * 4;
     L.eff = off;                 // 128 (eff, 1/eff) pairs, one per non-negative E4M3 scale code
     off += 128 * 8;
     L.bars = off;
-    off += (2 * kQStages + 6) * 8;
+    off += (2 * kQStages + 8) * 8;
     L.misc = off;
     off += 64;
     L.total = off;
@@ -220,6 +228,14 @@ __device__ __forceinline__ WarpRows warp_rows(const BoxRows& R, int warp) {
     return W;
 }
 
+// The smallest power of two >= v (v > 0) and its exponent: v = m 2^e with m in [0.5, 1).
+__device__ __forceinline__ float pow2_ceil(float v, int* exp2) {
+    int e;
+    const float m = frexpf(v, &e);
+    *exp2 = (m == 0.5f) ? e - 1 : e;
+    return (m == 0.5f) ? v : ldexpf(1.0f, e);
+}
+
 // 1 / cnt for a power of two cnt, exactly (the exponent field of 2^-log2(cnt))
 __device__ __forceinline__ float inv_pow2(int cnt) { return __int_as_float((127 - (31 - __clz(cnt))) << 23); }
 
@@ -317,6 +333,59 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+// 32 channels of one delta row (Eq. 1 delta, Eq. 4 per 16-channel group): z = x - m in fp32 from
+// four 16-byte X pieces of the box in shared memory (swizzled offsets xoff) and the 32 fp32 means at
+// mrow; per group the E4M3 scale code s_b = E4M3(max|z| / (6 S)) (denom = 6 S, rdenom = fl(1/denom)),
+// eff = s_b S from the table efft of (eff, 1/eff) per code, and the E2M1 codes of z / eff (+0 where
+// eff = 0).  kPow2: efft holds the codes' values at S = 1 and S = sc, a power of two with
+// reciprocal rsc, scales them exactly.  codes: 16 bytes, channel 2i in the low nibble of byte i;
+// scw: the two scale codes, the first group's in the low byte.
+template <bool kPow2>
+__device__ __forceinline__ void encode_delta32(const uint8_t* xs, const uint32_t (&xoff)[4], const float* mrow,
+                                               float denom, float rdenom, const float2* efft, float sc, float rsc,
+                                               uint32_t (&codes)[4], uint32_t& scw) {
+    scw = 0;
+#pragma unroll
+    for (int b = 0; b < 2; b++) {
+        uint64_t z[8];
+#pragma unroll
+        for (int hh = 0; hh < 2; hh++) {
+            const uint4 xv = *reinterpret_cast<const uint4*>(xs + xoff[2 * b + hh]);
+            uint64_t m[4];
+            load8(mrow + 16 * b + 8 * hh, m);
+            z[4 * hh + 0] = f2_sub(f2_from_bf16x2(xv.x), m[0]);
+            z[4 * hh + 1] = f2_sub(f2_from_bf16x2(xv.y), m[1]);
+            z[4 * hh + 2] = f2_sub(f2_from_bf16x2(xv.z), m[2]);
+            z[4 * hh + 3] = f2_sub(f2_from_bf16x2(xv.w), m[3]);
+        }
+        float zf[16];
+#pragma unroll
+        for (int e = 0; e < 8; e++) f2_unpack(z[e], zf[2 * e], zf[2 * e + 1]);
+        const float am = fmaxf(fmaxf(max3_abs(zf[0], zf[1], zf[2]), max3_abs(zf[3], zf[4], zf[5])),
+                               fmaxf(fmaxf(max3_abs(zf[6], zf[7], zf[8]), max3_abs(zf[9], zf[10], zf[11])),
+                                     fmaxf(max3_abs(zf[12], zf[13], zf[14]), fabsf(zf[15]))));
+        // am >= 0, so the code is one of 0x00..0x7E
+        const uint32_t sb = cvt_e4m3x2(div_pos(am, denom, rdenom), 0.f) & 0x7Fu;
+        const float2 er = efft[sb];
+        const float eff = kPow2 ? __fmul_rn(er.x, sc) : er.x;
+        scw |= sb << (8 * b);
+        uint32_t w0 = 0, w1 = 0;
+        if (eff != 0.f) {
+            // codes of the negated quotients, then every nibble's sign bit flipped
+            // (E2M1 is sign-magnitude: code(-v) = code(v) ^ 8, signed zeros included)
+            const float reff = kPow2 ? __fmul_rn(er.y, rsc) : er.y;
+            const uint64_t b2 = f2_pack(eff, eff), nrb2 = f2_pack(-reff, -reff);
+            float n[16];
+#pragma unroll
+            for (int e = 0; e < 8; e++) f2_unpack(f2_div_neg(z[e], b2, nrb2), n[2 * e], n[2 * e + 1]);
+            w0 = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(&n[0])) ^ 0x88888888u;
+            w1 = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(&n[8])) ^ 0x88888888u;
+        }
+        codes[2 * b] = w0;
+        codes[2 * b + 1] = w1;
+    }
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ a1: statistics + X L1
@@ -326,18 +395,26 @@ __device__ __forceinline__ float warp_max(float v) {
 // tensor-memory accumulators per item, which the compute warps drain to the
 // item's partial sums after its last chunk.
 
-template <bool kPairs>
+//
+// kSingle (the single-read quantiser, power-of-two S_delta): each chunk's means also go to shared
+// memory, the compute warps exchange the chunk's max |delta| (a bounded mbarrier per chunk), and
+// then encode the chunk's delta rows as the encode kernel would, under the chunk's own power-of-two
+// scale S_c = pow2(max|delta of the chunk| / 2688) <= S_delta; the exponent of S_c goes to p.prov
+// for the fix-up pass (k_single_finish), which also encodes the kernel tokens.
+
+template <bool kPairs, bool kSingle>
 __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_constant__ CUtensorMap tm_x,
                                                                   const __grid_constant__ CUtensorMap tm_l1,
                                                                   QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const QSmem L = q_smem_layout(p.rank, true, 0);
+    const QSmem L = q_smem_layout(p.rank, true, kSingle ? p.m_rows : 0, 128, kSingle);
     uint64_t* full = (uint64_t*)(sm + L.bars);
     uint64_t* empty = full + kQStages;
     uint64_t* accf = empty + kQStages;   // [2]
     uint64_t* acce = accf + 2;           // [2]
     uint64_t* done = acce + 2;
+    uint64_t* sdone = done + 1;          // [2], kSingle: a chunk's statistics are in shared memory
     uint32_t* tmem_slot = (uint32_t*)(sm + L.misc);
     volatile int* abort_flag = (volatile int*)(sm + L.misc + 8);
     float* red = (float*)(sm + L.misc + 16);  // 8 floats
@@ -361,8 +438,16 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
             mbar_init(&acce[b], kQWarps);
         }
         mbar_init(done, 1);
+        mbar_init(&sdone[0], kQWarps);
+        mbar_init(&sdone[1], kQWarps);
         *abort_flag = 0;
         fence_barrier_init();
+    }
+    float2* efft = (float2*)(sm + L.eff);
+    if (kSingle && tid < 128) {
+        // E4M3 code -> (value, 1 / value) at S = 1; a chunk's power-of-two scale multiplies both exactly
+        const float e = e4m3_to_f32((uint32_t)tid);
+        efft[tid] = make_float2(e, (e != 0.f) ? __frcp_rn(e) : 0.f);
     }
     if (warp == 9) {
         tmem_alloc(tmem_slot, 2 * tcols);
@@ -450,6 +535,19 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
             const BoxRows R = box_rows(p, B);
             const StatTask T0 = stat_task(p, R, tid);
             float kam[4] = {0.f, 0.f, 0.f, 0.f};   // max |mean| of this thread's cube tasks
+            // kSingle: the delta rows this warp encodes, as in the encode kernel (16 consecutive rows
+            // of the box's cube-major list, two lanes per row, 32 channels each)
+            const WarpRows W = warp_rows(R, warp);
+            const int er = W.r_lo + (lane >> 1), ehalf = lane & 1;
+            const bool has_row = kSingle && er < W.r_hi;
+            int erow = 0;
+            long long erho = 0;
+            if (has_row) list_row(p, B, R, er, &erow, &erho);
+            uint32_t xoff[4];
+#pragma unroll
+            for (int v = 0; v < 4; v++)
+                xoff[v] = (uint32_t)erow * 128u + ((((uint32_t)(4 * ehalf + v)) ^ ((uint32_t)erow & 7u)) << 4);
+            const uint32_t moff = (uint32_t)(has_row ? cube_of_row(R, er) : 0) * 256u + 128u * ehalf;
             // channel-pair mode: with fewer cubes than warps, the warps form kQWarps / nv groups
             // that take turns over the chunks, so that several stages of the ring are worked on at once
             const int ngrp = kPairs ? kQWarps / R.nv : 1;
@@ -462,6 +560,9 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                 if (!ok) break;
                 const uint8_t* xs = sm + L.x + s * 16384;
                 const int c0 = c_base + i * 64;
+                const int par = (int)(g & 1);
+                float* mts = (float*)(sm + L.ms + (uint32_t)par * L.ms_stride);   // kSingle: this chunk's means
+                float dch = 0.f;                                                 // this chunk's max |delta|
                 if (kPairs) {
                     // cubes of 16 or more tokens (at most 8 per box): warp = cube slot, lane = channel
                     // pair (2 lane, 2 lane + 1)
@@ -496,9 +597,10 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                             m1 = __fdiv_rn(a1, (float)cnt);
                         }
                         *reinterpret_cast<float2*>(p.means + (size_t)(R.k0 + u) * p.Ci + c0 + 2 * lane) = make_float2(m0, m1);
+                        if (kSingle) *reinterpret_cast<float2*>(mts + u * 64 + 2 * lane) = make_float2(m0, m1);
                         kam[0] = fmaxf(kam[0], fmaxf(fabsf(m0), fabsf(m1)));
-                        damax = fmaxf(damax, fmaxf(fmaxf(fabsf(__fsub_rn(bf16_lo(hi), m0)), fabsf(__fsub_rn(bf16_hi(hi), m1))),
-                                                   fmaxf(fabsf(__fsub_rn(bf16_lo(lo), m0)), fabsf(__fsub_rn(bf16_hi(lo), m1)))));
+                        dch = fmaxf(dch, fmaxf(fmaxf(fabsf(__fsub_rn(bf16_lo(hi), m0)), fabsf(__fsub_rn(bf16_hi(hi), m1))),
+                                               fmaxf(fabsf(__fsub_rn(bf16_lo(lo), m0)), fabsf(__fsub_rn(bf16_hi(lo), m1)))));
                     }
                 }
 #pragma unroll
@@ -509,7 +611,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                     uint64_t m[4];
                     if (p.big) {
                         load8(p.means + (size_t)R.k0 * p.Ci + c0 + 8 * T.g8, m);
-                        damax = fmaxf(damax, max_abs_diff8(*reinterpret_cast<const uint4*>(xs + T.off[0]), m));
+                        dch = fmaxf(dch, max_abs_diff8(*reinterpret_cast<const uint4*>(xs + T.off[0]), m));
                         continue;
                     }
                     // fp32 running sum from +0 in (t,h,w) order (Eq. 1; +0 + x keeps the sign of
@@ -563,14 +665,56 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                                                 (uint32_t)(m[1] >> 32), (uint32_t)m[2], (uint32_t)(m[2] >> 32),
                                                 (uint32_t)m[3], (uint32_t)(m[3] >> 32)};
                         st_global_v8(p.means + (size_t)(R.k0 + T.u) * p.Ci + c0 + 8 * T.g8, mw);
+                        if (kSingle) {
+                            float4* md = reinterpret_cast<float4*>(mts + T.u * 64 + 8 * T.g8);
+                            md[0] = make_float4(__uint_as_float(mw[0]), __uint_as_float(mw[1]), __uint_as_float(mw[2]),
+                                                __uint_as_float(mw[3]));
+                            md[1] = make_float4(__uint_as_float(mw[4]), __uint_as_float(mw[5]), __uint_as_float(mw[6]),
+                                                __uint_as_float(mw[7]));
+                        }
                     }
                     float mf[8];
 #pragma unroll
                     for (int e = 0; e < 4; e++) f2_unpack(m[e], mf[2 * e], mf[2 * e + 1]);
                     kam[t] = fmaxf(kam[t], fmaxf(max3_abs(mf[0], mf[1], mf[2]),
                                                  fmaxf(max3_abs(mf[3], mf[4], mf[5]), max3_abs(mf[6], mf[7], 0.f))));
-                    damax = fmaxf(damax, fmaxf(max_abs_diff8(make_uint4(hi[0], hi[1], hi[2], hi[3]), m),
-                                               max_abs_diff8(make_uint4(lo[0], lo[1], lo[2], lo[3]), m)));
+                    dch = fmaxf(dch, fmaxf(max_abs_diff8(make_uint4(hi[0], hi[1], hi[2], hi[3]), m),
+                                           max_abs_diff8(make_uint4(lo[0], lo[1], lo[2], lo[3]), m)));
+                }
+                damax = fmaxf(damax, dch);
+                if (kSingle) {
+                    // big cubes: the chunk's means, formed by the means kernel, into shared memory
+                    if (p.big && tid < 16)
+                        reinterpret_cast<float4*>(mts)[tid] =
+                            *reinterpret_cast<const float4*>(p.means + (size_t)R.k0 * p.Ci + c0 + 4 * tid);
+                    // the chunk's max |delta| over all compute warps, then its power-of-two scale
+                    const float wmx = warp_max(dch);
+                    float* red = (float*)(sm + L.red2) + par * kQWarps;
+                    __syncwarp();
+                    if (lane == 0) {
+                        red[warp] = wmx;
+                        mbar_arrive(&sdone[par]);
+                    }
+                    ok = __all_sync(0xffffffffu, mbar_wait(&sdone[par], (uint32_t)(g >> 1) & 1, abort_flag, p.status,
+                                                           p.budget_ns));
+                    if (!ok) break;
+                    float amc = 0.f;
+#pragma unroll
+                    for (int w = 0; w < kQWarps; w++) amc = fmaxf(amc, red[w]);
+                    int ec = -128;   // an all-zero chunk: its codes and scales are 0 under any scale
+                    float Sc = 1.f;
+                    if (amc > 0.f) Sc = pow2_ceil(__fdiv_rn(amc, 2688.f), &ec);
+                    const float den = __fmul_rn(6.f, Sc), rden = __frcp_rn(den), rSc = __frcp_rn(Sc);
+                    if (has_row) {
+                        uint32_t codes[4], scw;
+                        encode_delta32<true>(xs, xoff, (const float*)((const uint8_t*)mts + moff), den, rden, efft,
+                                             Sc, rSc, codes, scw);
+                        *reinterpret_cast<uint4*>(p.dcodes + (size_t)erho * (p.Ci / 2) + 16 * ehalf + c0 / 2) =
+                            make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                        *reinterpret_cast<uint16_t*>(p.dscales + sfa_offset(erho, c0 / 16 + 2 * ehalf, p.Ci)) =
+                            (uint16_t)scw;
+                        if (ehalf == 0) p.prov[(size_t)erho * (p.Ci / 64) + c0 / 64] = (int8_t)ec;
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
@@ -829,46 +973,7 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                     const float* mrow = (const float*)((const uint8_t*)mt + moff);
                     uint32_t codes[4];
                     uint32_t sc = 0;
-#pragma unroll
-                    for (int b = 0; b < 2; b++) {
-                        uint64_t z[8];
-#pragma unroll
-                        for (int hh = 0; hh < 2; hh++) {
-                            const uint4 xv = *reinterpret_cast<const uint4*>(xs + xoff[2 * b + hh]);
-                            uint64_t m[4];
-                            load8(mrow + 16 * b + 8 * hh, m);
-                            z[4 * hh + 0] = f2_sub(f2_from_bf16x2(xv.x), m[0]);
-                            z[4 * hh + 1] = f2_sub(f2_from_bf16x2(xv.y), m[1]);
-                            z[4 * hh + 2] = f2_sub(f2_from_bf16x2(xv.z), m[2]);
-                            z[4 * hh + 3] = f2_sub(f2_from_bf16x2(xv.w), m[3]);
-                        }
-                        float zf[16];
-#pragma unroll
-                        for (int e = 0; e < 8; e++) f2_unpack(z[e], zf[2 * e], zf[2 * e + 1]);
-                        const float am = fmaxf(
-                            fmaxf(max3_abs(zf[0], zf[1], zf[2]), max3_abs(zf[3], zf[4], zf[5])),
-                            fmaxf(fmaxf(max3_abs(zf[6], zf[7], zf[8]), max3_abs(zf[9], zf[10], zf[11])),
-                                  fmaxf(max3_abs(zf[12], zf[13], zf[14]), fabsf(zf[15]))));
-                        // am >= 0, so the code is one of 0x00..0x7E
-                        const uint32_t sb = cvt_e4m3x2(div_pos(am, denom, rdenom), 0.f) & 0x7Fu;
-                        const float2 er = efft[sb];
-                        const float eff = er.x;
-                        sc |= sb << (8 * b);
-                        uint32_t w0 = 0, w1 = 0;
-                        if (eff != 0.f) {
-                            // codes of the negated quotients, then every nibble's sign bit flipped
-                            // (E2M1 is sign-magnitude: code(-v) = code(v) ^ 8, signed zeros included)
-                            const float reff = er.y;
-                            const uint64_t b2 = f2_pack(eff, eff), nrb2 = f2_pack(-reff, -reff);
-                            float n[16];
-#pragma unroll
-                            for (int e = 0; e < 8; e++) f2_unpack(f2_div_neg(z[e], b2, nrb2), n[2 * e], n[2 * e + 1]);
-                            w0 = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(&n[0])) ^ 0x88888888u;
-                            w1 = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(&n[8])) ^ 0x88888888u;
-                        }
-                        codes[2 * b] = w0;
-                        codes[2 * b + 1] = w1;
-                    }
+                    encode_delta32<false>(xs, xoff, mrow, denom, rdenom, efft, 1.f, 1.f, codes, sc);
                     *reinterpret_cast<uint4*>(dcode_row + c0 / 2) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
                     *reinterpret_cast<uint16_t*>(p.dscales + sfa_offset(rho, c0 / 16 + 2 * half, Ci)) = (uint16_t)sc;
                 }
@@ -1019,6 +1124,146 @@ __global__ void __launch_bounds__(64) k_cube_means_big(const __grid_constant__ C
     __syncthreads();
 }
 
+// ------------------------------------------------------------------ single-read quantiser: fix-up pass
+//
+// After k_cube_stats<., true> every delta group is encoded under its chunk's power-of-two scale
+// S_c = 2^e_c, and the global max |delta| gives S_delta = 2^e = pow2(amax / 2688) >= S_c.  Under
+// S_delta a group keeps its E2M1 codes and its E4M3 scale code drops by 8 j (j = e - e_c) exactly
+// when the code's exponent field is at least j + 1; the other groups are encoded again under
+// S_delta from X and their cube's mean.  Part 1 (blockIdx.y == 0) does that per (row, 64-channel
+// chunk); part 2 encodes the FP8 kernel tokens from the stored means and the per-cube max |mean|;
+// part 3 forms U' = (X L1) / (S_delta S_W) as BF16 hi + lo and the slab's zero padding.
+
+// One 16-channel delta group of cube-major row rho under the power-of-two scale S (exponent e_s),
+// from X and the cube's means in global memory: the encode kernels' arithmetic.  Returns the scale
+// code; writes the 8 code bytes.
+__device__ uint32_t reencode_group(const QuantParams& p, const uint16_t* X, long long rho, int blk, float S,
+                                   uint8_t* code_out) {
+    long long n = 0, k = 0;
+    row_to_token(p.g, rho, &n, &k);
+    const uint16_t* x = X + (size_t)n * p.Ci + 16 * blk;
+    const float* m = p.means + (size_t)k * p.Ci + 16 * blk;
+    float z[16], am = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+        z[i] = __fsub_rn(__uint_as_float((uint32_t)x[i] << 16), m[i]);
+        am = fmaxf(am, fabsf(z[i]));
+    }
+    const float den = __fmul_rn(6.f, S);
+    const uint32_t sb = cvt_e4m3x2(div_pos(am, den, __frcp_rn(den)), 0.f) & 0x7Fu;
+    const float eff = __fmul_rn(e4m3_to_f32(sb), S);
+    uint32_t w[2] = {0u, 0u};
+    if (eff != 0.f) {
+        const float reff = __frcp_rn(eff);
+        float q[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++) q[i] = div_neg(z[i], eff, reff);
+        w[0] = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(&q[0])) ^ 0x88888888u;
+        w[1] = cvt_e2m1x8(*reinterpret_cast<const float(*)[8]>(&q[8])) ^ 0x88888888u;
+    }
+    *reinterpret_cast<uint2*>(code_out) = make_uint2(w[0], w[1]);
+    return sb;
+}
+
+__global__ void __launch_bounds__(256) k_single_finish(const uint16_t* X, QuantParams p) {
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+        const PackedHeader* hdr = reinterpret_cast<const PackedHeader*>(p.packed_w);
+        if (hdr->magic != DQ_PACK_MAGIC || hdr->version != DQ_PACK_FORMAT_VERSION || hdr->Ci != p.Ci ||
+            hdr->rank != p.rank || hdr->slab != p.slab || ((hdr->flags & kPackedC2) != 0) != (p.fp8_product != 0))
+            atomicCAS(p.status, 0, kStatusBadWeight);
+    }
+    const float amax = __uint_as_float(p.scalars[0]);
+    int es = 0;
+    const float S = (amax == 0.f) ? 1.f : pow2_ceil(__fdiv_rn(amax, 2688.f), &es);
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) p.scalars[1] = __float_as_uint(S);
+    const int Ci = p.Ci, chunks = Ci / 64;
+    const int lane = threadIdx.x & 31;
+    const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+    if (blockIdx.y == 0) {
+        // scale codes: a warp per cube-major row, a lane per 64-channel chunk, whose four group scale
+        // codes sit in one 32-bit word of the A-operand scale layout; shift each by the chunk's exponent
+        // difference, or encode the group again
+        for (long long rho = warp0; rho < p.g.N; rho += nwarps) {
+            const int8_t* prow = p.prov + (size_t)rho * chunks;
+            for (int ch = lane; ch < chunks; ch += 32) {
+                const int ec = prow[ch];
+                if (ec == -128 || ec == es) continue;   // an all-zero chunk, or no shift
+                const int j = es - ec;
+                uint32_t* sp = reinterpret_cast<uint32_t*>(p.dscales + sfa_offset(rho, 4 * ch, Ci));
+                const uint32_t scw = *sp;
+                uint32_t out = 0;
+#pragma unroll
+                for (int h = 0; h < 4; h++) {
+                    const uint32_t c = (scw >> (8 * h)) & 0xFFu;
+                    uint32_t nc;
+                    if (c == 0u)
+                        nc = 0u;                              // a zero scale stays zero, its codes +0
+                    else if ((int)((c >> 3) & 15u) >= j + 1)
+                        nc = c - 8u * (uint32_t)j;            // same codes, scale j binades lower
+                    else
+                        nc = reencode_group(p, X, rho, 4 * ch + h, S, p.dcodes + (size_t)rho * (Ci / 2) + 32 * ch + 8 * h);
+                    out |= nc << (8 * h);
+                }
+                if (out != scw) *sp = out;
+            }
+        }
+    } else if (blockIdx.y == 1) {
+        // FP8 kernel tokens under s8 = max |mean| / 448 (and their BF16 copy for the exact product):
+        // a warp per cube, a lane per 8 channels
+        for (long long k = warp0; k < p.g.K; k += nwarps) {
+            const float s8 = __fdiv_rn(__uint_as_float(p.kamax[k]), 448.f);
+            if (lane == 0) p.s8[k] = s8;
+            const float rs8 = (s8 != 0.f) ? __frcp_rn(s8) : 0.f;
+            const uint64_t b2 = f2_pack(s8, s8), nrb2 = f2_pack(-rs8, -rs8);
+            for (int c0 = 8 * lane; c0 < Ci; c0 += 256) {
+                uint32_t c[4] = {0u, 0u, 0u, 0u};
+                if (s8 != 0.f) {
+                    uint64_t m[4];
+                    load8(p.means + (size_t)k * Ci + c0, m);
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        float lo, hi;
+                        f2_unpack(f2_div_neg(m[e], b2, nrb2), lo, hi);
+                        c[e] = cvt_e4m3x2(lo, hi) ^ 0x8080u;
+                    }
+                }
+                *reinterpret_cast<uint2*>(p.q8 + (size_t)k * Ci + c0) = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+                if (!p.fp8_product) {
+                    uint32_t bfw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; e++) bfw[e] = e4m3x2_to_bf16x2(c[e]);
+                    *reinterpret_cast<uint4*>(p.q8_bf16 + (size_t)k * Ci + c0) = make_uint4(bfw[0], bfw[1], bfw[2], bfw[3]);
+                }
+            }
+        }
+    } else {
+        // U' = (X L1) / (S_delta S_W) as BF16 hi + lo, the partial sums added in split order
+        const float SS = __fmul_rn(S, reinterpret_cast<const PackedHeader*>(p.packed_w)->S_W);
+        // a warp per row, a lane per two columns of the slab row
+        for (long long rho = warp0; rho < p.g.N; rho += nwarps)
+        for (int c = 2 * lane; c < p.slab; c += 64) {
+            uint16_t* dst = p.u_hilo + (size_t)rho * p.slab;
+            if (c >= p.rank) {
+                if (c >= 2 * p.rank) *reinterpret_cast<uint32_t*>(dst + c) = 0u;   // padding
+                continue;
+            }
+            float u0 = 0.f, u1 = 0.f;
+            for (int sp = 0; sp < p.splits; sp++) {
+                const float2 v = *reinterpret_cast<const float2*>(p.u_part + ((size_t)sp * p.g.N + (size_t)rho) * p.rank + c);
+                u0 = __fadd_rn(u0, v.x);
+                u1 = __fadd_rn(u1, v.y);
+            }
+            const float a0 = __fdiv_rn(u0, SS), a1 = __fdiv_rn(u1, SS);
+            const uint16_t h0 = f32_to_bf16_rn(a0), h1 = f32_to_bf16_rn(a1);
+            const uint16_t l0 = f32_to_bf16_rn(__fsub_rn(a0, __uint_as_float((uint32_t)h0 << 16)));
+            const uint16_t l1 = f32_to_bf16_rn(__fsub_rn(a1, __uint_as_float((uint32_t)h1 << 16)));
+            *reinterpret_cast<uint32_t*>(dst + c) = (uint32_t)h0 | ((uint32_t)h1 << 16);
+            *reinterpret_cast<uint32_t*>(dst + p.rank + c) = (uint32_t)l0 | ((uint32_t)l1 << 16);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ launchers
 
 cudaError_t launch_cube_means_big(const CUtensorMap& tm_x, const QuantParams& p, cudaStream_t st) {
@@ -1027,6 +1272,14 @@ cudaError_t launch_cube_means_big(const CUtensorMap& tm_x, const QuantParams& p,
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)p.g.K, (unsigned)(p.Ci / 64));
     k_cube_means_big<<<grid, 64, smem, st>>>(tm_x, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_single_finish(const void* X, const QuantParams& p, cudaStream_t st) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    k_single_finish<<<dim3((unsigned)(4 * (sms > 0 ? sms : 148)), 3), 256, 0, st>>>((const uint16_t*)X, p);
     return cudaGetLastError();
 }
 
@@ -1059,22 +1312,27 @@ int resident_grid(const void* fn, int threads, size_t smem, int items) {
 }
 }  // namespace
 
-template <bool kPairs>
+template <bool kPairs, bool kSingle>
 cudaError_t launch_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p, cudaStream_t st) {
-    size_t smem = quant_smem_bytes(p.rank, true, 0, 128);
-    cudaError_t e = cudaFuncSetAttribute(k_cube_stats<kPairs>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    size_t smem = q_smem_layout(p.rank, true, kSingle ? p.m_rows : 0, 128, kSingle).total + 1024;
+    auto fn = k_cube_stats<kPairs, kSingle>;
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_cube_stats<kPairs>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 cudaSharedmemCarveoutMaxShared);
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    const int grid = resident_grid((const void*)k_cube_stats<kPairs>, kQCompute + 64, smem, p.n_boxes * p.splits);
-    k_cube_stats<kPairs><<<grid, kQCompute + 64, smem, st>>>(tm_x, tm_l1, p);
+    const int grid = resident_grid((const void*)fn, kQCompute + 64, smem, p.n_boxes * p.splits);
+    fn<<<grid, kQCompute + 64, smem, st>>>(tm_x, tm_l1, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
                               cudaStream_t st) {
-    return p.stat_pairs ? launch_stats<true>(tm_x, tm_l1, p, st) : launch_stats<false>(tm_x, tm_l1, p, st);
+    return p.stat_pairs ? launch_stats<true, false>(tm_x, tm_l1, p, st) : launch_stats<false, false>(tm_x, tm_l1, p, st);
+}
+
+cudaError_t launch_cube_single(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
+                               cudaStream_t st) {
+    return p.stat_pairs ? launch_stats<true, true>(tm_x, tm_l1, p, st) : launch_stats<false, true>(tm_x, tm_l1, p, st);
 }
 
 cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const CUtensorMap& tm_m, const QuantParams& p,
