@@ -267,19 +267,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int tile = pair; alive && tile < num_tiles; tile += npairs, it++) {
                 const int buf = it % kBufs, use = it / kBufs;
                 const uint32_t acc = tmem + (uint32_t)(buf * 256);
-                if (use > 0 && !mbar_wait(&acce[buf], (uint32_t)(use - 1) & 1, abort_flag, p.status, p.budget_ns))
+                if (use > 0 && !mbar_wait_spin(&acce[buf], (uint32_t)(use - 1) & 1, abort_flag, p.status, p.budget_ns))
                     break;
                 tc_fence_after();
                 for (int i = 0; i < ntot; i++, g++) {
                     const int s = (int)(g % S);
-                    if (!mbar_wait(&full[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
+                    if (!mbar_wait_spin(&full[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
                         alive = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t aa = smem_u32(sm + L.a + s * kABytes), bb = smem_u32(sm + L.b + s * kBBytes);
                     if (kFp8) {
-                        if (!mbar_wait(&sfready[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
+                        if (!mbar_wait_spin(&sfready[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
                             alive = false;
                             break;
                         }
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                           tmem + kFp8SfbCol + (uint32_t)(8 * s), (i | k) != 0);
                     } else if (kMain && i < nk) {
                         const uint32_t t_sfa = t_sf0 + (uint32_t)(s * 48), t_sfb = t_sfa + 16;
-                        if (!mbar_wait(&sfready[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
+                        if (!mbar_wait_spin(&sfready[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
                             alive = false;
                             break;
                         }
@@ -328,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int tile = pair; alive && tile < num_tiles; tile += npairs) {
                 for (int i = 0; i < ntot; i++, g++) {
                     const int s = (int)(g % S);
-                    if (!mbar_wait(&full[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
+                    if (!mbar_wait_spin(&full[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
                         alive = false;
                         break;
                     }
@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int tile = pair; alive && tile < num_tiles; tile += npairs) {
                 for (int i = 0; i < ntot; i++, g++) {
                     const int s = (int)(g % S);
-                    if (!mbar_wait(&full[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
+                    if (!mbar_wait_spin(&full[s], (uint32_t)(g / S) & 1, abort_flag, p.status, p.budget_ns)) {
                         alive = false;
                         break;
                     }
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // tile's P' rows are fetched and its Y rows are written.
                 long long n = 0, k = 0;
                 if (row_ok) row_to_token(p.g, rho, &n, &k);
-                const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], (uint32_t)use & 1, abort_flag,
+                const bool ok = __all_sync(0xffffffffu, mbar_wait_spin(&accf[buf], (uint32_t)use & 1, abort_flag,
                                                                   p.status, p.budget_ns));
                 if (!ok) break;
                 tc_fence_after();
@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float* bias =
                     (reinterpret_cast<const PackedHeader*>(p.packed_w)->flags & kPackedHasBias) ? p.bias + c_base
                                                                                                  : nullptr;
-                const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], (uint32_t)use & 1, abort_flag,
+                const bool ok = __all_sync(0xffffffffu, mbar_wait_spin(&accf[buf], (uint32_t)use & 1, abort_flag,
                                                                   p.status, p.budget_ns));
                 if (!ok) break;
                 tc_fence_after();
@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float* bias =
                     (reinterpret_cast<const PackedHeader*>(p.packed_w)->flags & kPackedHasBias) ? p.bias + c_base
                                                                                                  : nullptr;
-                const bool ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], (uint32_t)use & 1, abort_flag,
+                const bool ok = __all_sync(0xffffffffu, mbar_wait_spin(&accf[buf], (uint32_t)use & 1, abort_flag,
                                                                   p.status, p.budget_ns));
                 if (!ok) break;
                 tc_fence_after();

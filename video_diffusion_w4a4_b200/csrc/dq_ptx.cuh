@@ -93,6 +93,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// Bounded wait that polls without a suspend hint, for the products' stage and accumulator
+// hand-offs, where the wake-up of a suspended wait showed in the step time (about 1 %).
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                               uint64_t budget_ns) {
+    uint32_t b = smem_u32(bar);
+    if (mbar_try_wait(b, parity)) return true;
+    uint64_t t0 = globaltimer();
+    for (uint32_t n = 1;; n++) {
+        if (mbar_try_wait(b, parity)) return true;
+        if ((n & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > budget_ns) {
+                *abort_flag = 1;
+                if (status) atomicCAS(status, 0, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
