@@ -289,6 +289,32 @@ def test_entry_points_agree(env):
     assert np.array_equal(Yh.numpy().view(np.uint16), g["Y"])
 
 
+@pytest.mark.parametrize("name", ["ragged_122", "ragged_222", "cube_414_r128", "cube_428", "tiny"])
+def test_host_entry_point_pipeline(env, name):
+    """The host-buffer entry point copies X in T-slabs overlapped with the statistics pass
+    and copies finished frames of Y back while later row tiles compute: Y bit-identical to
+    the device-buffer entry point's, for slabs of 1-, 2- and 4-frame cube layers, a ragged
+    last layer, and a layer of one cube layer (no pipelining)."""
+    dq, torch = env
+    wl = dict(SMALL)[name] or synth.WORKLOADS["tiny"]
+    case = Case(wl)
+    g = case.run_gpu(dq, torch)
+    t, h, w = case.cube
+    Xd, Pd, L1d, L2d, _ = case.last_inputs
+    Xh = torch.from_numpy(case.X.view(np.int16)).pin_memory()
+    Yh = torch.full((wl.N, wl.Co), 0x7FC0, dtype=torch.int16).pin_memory()
+    nbytes = dq.dq_workspace_bytes(wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=Xd.device)
+    Xd2, Yd2 = torch.empty_like(Xd), torch.empty((wl.N, wl.Co), dtype=torch.int16, device=Xd.device)
+    st = torch.cuda.current_stream()
+    for _ in range(2):   # the second call reuses the copy streams and events
+        dq.dq_linear_forward_host(Xh, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yh, Xd2, Yd2,
+                                  ws, nbytes, st)
+        st.synchronize()
+        assert np.array_equal(Yh.numpy().view(np.uint16), g["Y"])
+        assert dq.dq_read_device_status(ws, st, clear=True) == 0
+
+
 def test_stage_mask_reuses_workspace(env):
     """Running the three stages as three calls on one workspace equals one call."""
     dq, torch = env

@@ -8,8 +8,10 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <functional>
 #include <map>
 #include <mutex>
+#include <vector>
 
 #include "../../include/deltaquant.h"
 #include "dq_common.h"
@@ -149,6 +151,37 @@ int check_options(const dq_forward_options& o) {
     return DQ_OK;
 }
 
+// Copy streams and events of the pipelined host-buffer entry point, one set per device, created on
+// first use and kept until the process exits; one call at a time uses them.
+constexpr int kHostSlabs = 8;    // T-slabs of X copied in (at most; whole cube layers)
+constexpr int kHostChunks = 4;   // row-tile ranges of the main product whose frames are copied out
+struct Aux {
+    std::mutex mu;
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t ev[2 + kHostSlabs + kHostChunks] = {};
+};
+std::mutex g_aux_mu;
+std::map<int, Aux> g_aux;
+
+int cuda_fail(cudaError_t e, const char* where);
+
+int host_aux(Aux** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DQ_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lk(g_aux_mu);
+    Aux& A = g_aux[dev];
+    if (!A.in) {
+        cudaError_t e;
+        if ((e = cudaStreamCreateWithFlags(&A.in, cudaStreamNonBlocking)) != cudaSuccess ||
+            (e = cudaStreamCreateWithFlags(&A.out, cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(e, "copy streams");
+        for (cudaEvent_t& ev : A.ev)
+            if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e, "events");
+    }
+    *out = &A;
+    return DQ_OK;
+}
+
 struct LibWorkspace {
     void* ptr = nullptr;
     size_t bytes = 0;
@@ -248,10 +281,24 @@ int dq_workspace_bytes(int T, int H, int W, int t, int h, int w, int Ci, int Co,
     return DQ_OK;
 }
 
-int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
-                           const dq_forward_options* opts, const void* packed_W, const void* L1_mma,
-                           const void* L2_slab, void* Y, void* workspace, size_t workspace_bytes, int stage_mask,
-                           void* const* stage_events, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// A split of one forward into pieces for the host-buffer entry point: the statistics pass in T-slabs
+// of whole cube layers (before_slab(i) runs before slab i's launch, e.g. to wait for its copy of X),
+// the main product in ranges of 256-row tiles (after_chunk(k, last cube-major row done) after each).
+struct Pipeline {
+    std::vector<int> kt_cuts;    // cube-layer boundaries of the slabs: 0 = kt_cuts[0] < ... = KT
+    std::vector<int> tile_cuts;  // row-tile boundaries of the main-product launches: 0 = ... = ceil(N / 256)
+    std::function<int(int)> before_slab;
+    std::function<int(int, long long)> after_chunk;
+};
+
+int forward_impl(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                 const dq_forward_options* opts, const void* packed_W, const void* L1_mma, const void* L2_slab,
+                 void* Y, void* workspace, size_t workspace_bytes, int stage_mask, void* const* stage_events,
+                 void* stream, const Pipeline* pipe) {
     int rc = check_shape(T, H, W, t, h, w, Ci, Co, rank);
     if (rc) return rc;
     const dq_forward_options o = opts ? *opts : dq_forward_options{};
@@ -310,6 +357,8 @@ int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int
         qp.n_boxes = g.T * g.H * qp.nbw;
         qp.m_rows = 1;
     }
+    qp.item0 = 0;
+    qp.item1 = qp.n_boxes * qp.splits;
     qp.means = (float*)(ws + wl.off_means);
     qp.status = (int*)(ws + wl.off_status);
     qp.scalars = (uint32_t*)(ws + wl.off_scalars);
@@ -352,11 +401,22 @@ int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int
                 return cuda_fail(e0, "memset");
             if (qp.big && (e = dq::launch_cube_means_big(tm_x, qp, st)) != cudaSuccess)
                 return cuda_fail(e, "k_cube_means_big");
-            if (pow2) {
-                if ((e = dq::launch_cube_single(tm_x, tm_l1, qp, st)) != cudaSuccess)
-                    return cuda_fail(e, "k_cube_stats (single read)");
-            } else if ((e = dq::launch_cube_stats(tm_x, tm_l1, qp, st)) != cudaSuccess) {
-                return cuda_fail(e, "k_cube_stats");
+            // one launch over all work items, or one per T-slab (items of boxes in cube layers [kt0, kt1))
+            const int items_per_layer = (qp.big ? g.t * g.H * qp.nbw : g.KH * qp.nbw) * qp.splits;
+            const int nslab = pipe ? (int)pipe->kt_cuts.size() - 1 : 1;
+            for (int sl = 0; sl < nslab; sl++) {
+                dq::QuantParams qs = qp;
+                if (pipe) {
+                    if ((rc = pipe->before_slab(sl))) return rc;
+                    qs.item0 = pipe->kt_cuts[sl] * items_per_layer;
+                    qs.item1 = dq::imin(pipe->kt_cuts[sl + 1] * items_per_layer, qp.item1);
+                }
+                if (pow2) {
+                    if ((e = dq::launch_cube_single(tm_x, tm_l1, qs, st)) != cudaSuccess)
+                        return cuda_fail(e, "k_cube_stats (single read)");
+                } else if ((e = dq::launch_cube_stats(tm_x, tm_l1, qs, st)) != cudaSuccess) {
+                    return cuda_fail(e, "k_cube_stats");
+                }
             }
         }
         if (do_encode && pow2) {
@@ -376,6 +436,8 @@ int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int
         if (!map_sfb(&tm_fb, pw + pl.off_dqw + (size_t)Co * Ci, Ci / 2, Co, 1)) return map_fail("FP8 product scales");
         dq::GemmParams p = gp;
         p.M = (int)g.K;
+        p.tile_m0 = 0;
+        p.tile_m1 = (int)dq::cdiv(g.K, 256);
         p.k_stages = Ci / 128;
         p.tile_group = 8;
         p.s8 = qp.s8;
@@ -391,6 +453,8 @@ int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int
         if (!map_2d(&tm_b, pw + pl.off_dqw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, Co, 64, 128)) return map_fail("product B");
         dq::GemmParams p = gp;
         p.M = (int)g.K;
+        p.tile_m0 = 0;
+        p.tile_m1 = (int)dq::cdiv(g.K, 256);
         p.k_stages = a_cols / 64;
         p.b_kblocks = Ci / 64;
         p.tile_group = 8;   // the BF16 weight (Co x Ci x 2 bytes) does not stay in L2 beside the rows
@@ -414,6 +478,8 @@ int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int
         if (!map_sfb(&tm_fb, pw + pl.off_scales, Ci, Co)) return map_fail("weight scales");
         dq::GemmParams p = gp;
         p.M = (int)g.N;
+        p.tile_m0 = 0;
+        p.tile_m1 = (int)dq::cdiv(g.N, 256);
         p.k_stages = Ci / 256;
         p.slab_stages = wl.slab / 64;
         // weight codes and scales above 32 MB (the 720p FFN layers) are re-read by every wave of a
@@ -421,11 +487,32 @@ int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int
         p.tile_group = ((size_t)Co * (Ci / 2) + pl.off_dqw - pl.off_scales > ((size_t)32 << 20)) ? 8 : 1;
         p.p = (const float*)(ws + wl.off_p);
         p.Y = (uint16_t*)Y;
-        cudaError_t e = dq::launch_main_gemm(tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p, st);
-        if (e != cudaSuccess) return cuda_fail(e, "main product");
+        const int nchunk = pipe ? (int)pipe->tile_cuts.size() - 1 : 1;
+        for (int c = 0; c < nchunk; c++) {
+            if (pipe) {
+                p.tile_m0 = pipe->tile_cuts[c];
+                p.tile_m1 = pipe->tile_cuts[c + 1];
+            }
+            cudaError_t e = dq::launch_main_gemm(tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p, st);
+            if (e != cudaSuccess) return cuda_fail(e, "main product");
+            if (pipe && (rc = pipe->after_chunk(c, dq::imin(p.tile_m1 * 256, (int)g.N))))
+                return rc;
+        }
     }
     rec(3);
     return DQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                           const dq_forward_options* opts, const void* packed_W, const void* L1_mma,
+                           const void* L2_slab, void* Y, void* workspace, size_t workspace_bytes, int stage_mask,
+                           void* const* stage_events, void* stream) {
+    return forward_impl(X, T, H, W, t, h, w, Ci, Co, rank, opts, packed_W, L1_mma, L2_slab, Y, workspace,
+                        workspace_bytes, stage_mask, stage_events, stream, nullptr);
 }
 
 int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
@@ -464,12 +551,75 @@ int dq_linear_forward_host(const void* X_host, int T, int H, int W, int t, int h
     if (rc) return rc;
     if (!X_host || !Y_host || !X_dev || !Y_dev) return DQ_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
-    size_t N = (size_t)T * H * W;
-    if (cudaMemcpyAsync(X_dev, X_host, N * Ci * 2, cudaMemcpyHostToDevice, st) != cudaSuccess) return DQ_ERR_CUDA;
-    rc = dq_linear_forward_ex(X_dev, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y_dev, workspace,
-                              workspace_bytes, DQ_STAGE_ALL, nullptr, stream);
+    const Geom g = dq::make_geom(T, H, W, t, h, w);
+    const size_t HW = (size_t)H * W;
+    if ((long long)t * h * w > 128 || g.KT < 2) {
+        // one copy in, the layer, one copy out
+        size_t N = (size_t)T * HW;
+        cudaError_t e;
+        if ((e = cudaMemcpyAsync(X_dev, X_host, N * Ci * 2, cudaMemcpyHostToDevice, st)) != cudaSuccess)
+            return cuda_fail(e, "copy of X");
+        rc = dq_linear_forward_ex(X_dev, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y_dev, workspace,
+                                  workspace_bytes, DQ_STAGE_ALL, nullptr, stream);
+        if (rc) return rc;
+        if ((e = cudaMemcpyAsync(Y_host, Y_dev, N * Co * 2, cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+            return cuda_fail(e, "copy of Y");
+        return DQ_OK;
+    }
+    // Pipelined: X crosses in T-slabs of whole cube layers on a copy stream, and the statistics pass of
+    // each slab starts as soon as its rows are on the device; the encode stage and the kernel-token
+    // product need every slab's statistics (the per-tensor delta scale); the main product then runs in
+    // ranges of row tiles, and the frames each range completes cross back on a second copy stream while
+    // the next range computes.  `stream` waits for the last copy, so the call's work ends on `stream`.
+    Aux* aux = nullptr;
+    if ((rc = host_aux(&aux))) return rc;
+    std::lock_guard<std::mutex> lk(aux->mu);
+    const int nslab = dq::imin(g.KT, kHostSlabs);
+    const int tiles = (int)dq::cdiv(g.N, 256);
+    const int nchunk = dq::imin(tiles, kHostChunks);
+    Pipeline pipe;
+    for (int i = 0; i <= nslab; i++) pipe.kt_cuts.push_back((int)((long long)g.KT * i / nslab));
+    for (int i = 0; i <= nchunk; i++) pipe.tile_cuts.push_back((int)((long long)tiles * i / nchunk));
+    cudaError_t e;
+    // the copies in wait for earlier work on `stream` (which may still read X_dev)
+    if ((e = cudaEventRecord(aux->ev[0], st)) != cudaSuccess || (e = cudaStreamWaitEvent(aux->in, aux->ev[0], 0)))
+        return cuda_fail(e, "stream order");
+    for (int i = 0; i < nslab; i++) {
+        const size_t f0 = (size_t)pipe.kt_cuts[i] * t, f1 = dq::imin(pipe.kt_cuts[i + 1] * t, T);
+        const size_t off = f0 * HW * Ci * 2, bytes = (f1 - f0) * HW * Ci * 2;
+        if ((e = cudaMemcpyAsync((uint8_t*)X_dev + off, (const uint8_t*)X_host + off, bytes, cudaMemcpyHostToDevice,
+                                 aux->in)) != cudaSuccess ||
+            (e = cudaEventRecord(aux->ev[1 + i], aux->in)) != cudaSuccess)
+            return cuda_fail(e, "copy of X");
+    }
+    pipe.before_slab = [&](int i) {
+        cudaError_t e1 = cudaStreamWaitEvent(st, aux->ev[1 + i], 0);
+        return e1 == cudaSuccess ? DQ_OK : cuda_fail(e1, "stream order");
+    };
+    // frames whose rows are complete after a range of row tiles: whole cube layers below the last row done
+    size_t frames_out = 0;
+    const long long layer_rows = (long long)t * H * W;
+    pipe.after_chunk = [&](int c, long long rows_done) {
+        const int last = c == nchunk - 1;
+        const size_t f1 = last ? (size_t)T : dq::imin((int)(rows_done / layer_rows) * t, T);
+        if (f1 <= frames_out) return (int)DQ_OK;
+        cudaEvent_t ev = aux->ev[1 + kHostSlabs + c];
+        cudaError_t e1;
+        if ((e1 = cudaEventRecord(ev, st)) != cudaSuccess || (e1 = cudaStreamWaitEvent(aux->out, ev, 0)) != cudaSuccess)
+            return cuda_fail(e1, "stream order");
+        const size_t off = frames_out * HW * Co * 2, bytes = (f1 - frames_out) * HW * Co * 2;
+        if ((e1 = cudaMemcpyAsync((uint8_t*)Y_host + off, (const uint8_t*)Y_dev + off, bytes, cudaMemcpyDeviceToHost,
+                                  aux->out)) != cudaSuccess)
+            return cuda_fail(e1, "copy of Y");
+        frames_out = f1;
+        return (int)DQ_OK;
+    };
+    rc = forward_impl(X_dev, T, H, W, t, h, w, Ci, Co, rank, nullptr, packed_W, L1_mma, L2_slab, Y_dev, workspace,
+                      workspace_bytes, DQ_STAGE_ALL, nullptr, stream, &pipe);
     if (rc) return rc;
-    if (cudaMemcpyAsync(Y_host, Y_dev, N * Co * 2, cudaMemcpyDeviceToHost, st) != cudaSuccess) return DQ_ERR_CUDA;
+    cudaEvent_t done = aux->ev[1 + kHostSlabs + kHostChunks];
+    if ((e = cudaEventRecord(done, aux->out)) != cudaSuccess || (e = cudaStreamWaitEvent(st, done, 0)) != cudaSuccess)
+        return cuda_fail(e, "stream order");
     return DQ_OK;
 }
 

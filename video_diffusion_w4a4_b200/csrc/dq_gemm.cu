@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool lead = rank == 0;
     const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
     const int num_n = p.Nout / kTileN;
-    const int num_m = (int)cdiv(p.M, 2 * kTileM);
+    const int m_lo = p.tile_m0, num_m = p.tile_m1 - p.tile_m0;   // this launch's row tiles
     const int num_tiles = num_m * num_n;
     const int nk = p.k_stages, ntot = p.k_stages + p.slab_stages;
 
@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool alive = true;
             for (int tile = pair; alive && tile < num_tiles; tile += npairs) {
                 const TileRC rc = tile_rc(tile, num_m, num_n, p.tile_group);
-                const int m0 = rc.m * (2 * kTileM) + (int)rank * kTileM;   // this CTA's A rows
+                const int m0 = (m_lo + rc.m) * (2 * kTileM) + (int)rank * kTileM;   // this CTA's A rows
                 const int n0 = rc.n * kTileN;                               // the pair's columns
                 const int nb = n0 + (int)rank * (kTileN / 2);                         // this CTA's B rows
                 for (int i = 0; i < ntot; i++, g++) {
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int tile = pair; tile < num_tiles; tile += npairs, it++) {
             const int buf = it % kBufs, use = it / kBufs;
             const TileRC rc = tile_rc(tile, num_m, num_n, p.tile_group);
-            const int m0 = rc.m * (2 * kTileM) + (int)rank * kTileM;
+            const int m0 = (m_lo + rc.m) * (2 * kTileM) + (int)rank * kTileM;
             const int n0 = rc.n * kTileN;
             const long long rho = (long long)m0 + quad * 32 + lane;
             const bool row_ok = rho < p.M;
@@ -542,7 +542,8 @@ cudaError_t launch_pairs(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const
     static_assert(smem <= 232448, "shared memory of a paired product");
     cudaError_t e = cudaFuncSetAttribute(k_gemm<kKind>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int tiles = (int)cdiv(p.M, 2 * kTileM) * (p.Nout / kTileN);
+    const int tiles = (p.tile_m1 - p.tile_m0) * (p.Nout / kTileN);
+    if (tiles <= 0) return cudaSuccess;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;

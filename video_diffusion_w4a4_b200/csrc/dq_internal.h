@@ -17,6 +17,7 @@ struct QuantParams {
     int bt, bh, bw;     // box extent in tokens: t x h x (nw w)
     int nbw;            // boxes along w
     int n_boxes;
+    int item0, item1;   // the statistics kernel's work items [item0, item1) of n_boxes * splits (a T-slab)
     int m_rows;         // kernel tokens per box (rows of the encode kernel's per-stage tile)
     int stat_pairs;     // statistics kernel: one warp per cube, a channel pair per lane (cubes of 16+ tokens)
     int kgroup;         // 0: s8 per kernel token (K); 64: per 64 channels (K x Ci/64), q8_bf16 = [hi | lo]
@@ -49,6 +50,7 @@ struct GemmParams {
     int slab_stages;     // extra BF16 K stages (low-rank slab), main product only
     int b_kblocks;       // kernel-token product: B k-blocks (Ci/64); A k-block i reads B k-block i mod this
     int tile_group;      // tile order: 1 row-major, else groups of this many row tiles walked column by column
+    int tile_m0, tile_m1;  // the launch's row tiles [tile_m0, tile_m1) of 256 rows
     const float* p;      // per-cube kernel term, K x Co fp32 (main product)
     const uint32_t* scalars;
     const uint8_t* packed_w;

@@ -421,7 +421,6 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nchunks = p.chunks_per_split;
-    const int n_items = p.n_boxes * p.splits;
     const uint32_t l1_bytes = (uint32_t)p.rank * 128u;
     const uint32_t l1_stride = (uint32_t)align_up(l1_bytes, 1024);
     const uint32_t x_bytes = (uint32_t)p.bt * p.bh * p.bw * 128u;
@@ -465,7 +464,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
             prefetch_tmap(&tm_l1);
             long long g = 0;
             bool alive = true;
-            for (int it = blockIdx.x; alive && it < n_items; it += gridDim.x) {
+            for (int it = p.item0 + blockIdx.x; alive && it < p.item1; it += gridDim.x) {
                 const BoxPos B = box_pos(p, it / p.splits);
                 const int c_base = (it % p.splits) * nchunks * 64;
                 for (int i = 0; i < nchunks; i++, g++) {
@@ -492,7 +491,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
             long long g = 0;
             int n = 0;
             bool alive = true;
-            for (int it = blockIdx.x; alive && it < n_items; it += gridDim.x, n++) {
+            for (int it = p.item0 + blockIdx.x; alive && it < p.item1; it += gridDim.x, n++) {
                 const int buf = n & 1, use = n >> 1;
                 const uint32_t acc = tmem + (uint32_t)buf * tcols;
                 if (use > 0 && !mbar_wait(&acce[buf], (uint32_t)(use - 1) & 1, abort_flag, p.status, p.budget_ns))
@@ -528,7 +527,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
         long long g = 0;
         int n = 0;
         bool ok = true;
-        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, n++) {
+        for (int it = p.item0 + blockIdx.x; ok && it < p.item1; it += gridDim.x, n++) {
             const BoxPos B = box_pos(p, it / p.splits);
             const int split = it % p.splits;
             const int c_base = split * nchunks * 64;
@@ -1320,7 +1319,7 @@ cudaError_t launch_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, cons
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    const int grid = resident_grid((const void*)fn, kQCompute + 64, smem, p.n_boxes * p.splits);
+    const int grid = resident_grid((const void*)fn, kQCompute + 64, smem, p.item1 - p.item0);
     fn<<<grid, kQCompute + 64, smem, st>>>(tm_x, tm_l1, p);
     return cudaGetLastError();
 }
