@@ -479,12 +479,13 @@ def main():
     dom = max(("quantize", "kernel_gemm", "main_gemm"), key=stage_ms.get)
     if dom == "quantize":
         ach = model[dom]["bytes"] / (stage_ms[dom] * 1e-3) / 1e9
-        roof = dict(kernel="k_cube_stats+k_cube_encode", bound="hbm", achieved=ach, peak=peaks["hbm"], unit="GB/s")
+        roof = dict(kernel="k_cube_stats<.,.>+k_cube_encode", bound="hbm", achieved=ach, peak=peaks["hbm"], unit="GB/s")
     else:
         # the kernel-token product's own kind: BF16, or FP8 at 2 x the BF16 rate (nominal 4.5 : 2.25)
         pk = fp4_peak if dom == "main_gemm" else peaks["bf16"] * (FP8_PER_BF16 if fp8 else 1.0)
         ach = model[dom]["flops"] / (stage_ms[dom] * 1e-3) / 1e12
-        roof = dict(kernel="k_gemm<true> (main FP4 product)" if dom == "main_gemm" else "k_gemm<false> (kernel-token product)",
+        roof = dict(kernel="k_gemm<1> (main FP4 product)" if dom == "main_gemm" else
+                    ("k_gemm<2> (FP8 kernel-token product)" if fp8 else "k_gemm<0> (kernel-token product)"),
                     bound="tensor", achieved=ach, peak=pk, unit="TFLOP/s")
     roof["frac"] = roof["achieved"] / roof["peak"]
     same_cube = tuple(cube) == tuple(synth.WORKLOADS[args.workload].cube)

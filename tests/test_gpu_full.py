@@ -133,3 +133,24 @@ def test_full_size_group64_kernel_scales(env, cube):
     info = assert_y_close(g["Y"][rows], case.oracle_rows(act, wq, rows))
     info.update(cube=list(cube), kernel_group=64, rows=int(rows.size))
     _record("group64_%d%d%d" % cube, info)
+
+
+@pytest.mark.parametrize("name,fp8,pow2", [("wan720p_ffn_down", True, False), ("wan480p_proj", True, False),
+                                           ("wan480p_proj", False, True), ("wan720p_ffn_up", True, True)],
+                         ids=["ffn_down_fp8", "proj_fp8", "proj_single_read", "ffn_up_fp8_single_read"])
+def test_full_size_options(env, name, fp8, pow2):
+    """The layer's options at full size: the FP8-rate kernel-token product on
+    restricted-scale (C2) weights and the single-read quantiser (power-of-two
+    S_delta).  Every quantised tensor and the packed C2 weight bit-exact against
+    the oracle's option, P' and Y on sampled cubes within tolerance."""
+    dq, torch = env
+    wl = synth.WORKLOADS[name]
+    case = Case(wl, fp8_product=fp8, pow2=pow2)
+    g = case.run_gpu(dq, torch)
+    act, wq = case.run_oracle()
+    compare_quantised(g, act, wq)
+    ks, rows = sample_cubes(wl, case.cube, n_cubes=32)
+    pinfo = assert_kernel_term_close(g["p"], act, wq, ks)
+    info = assert_y_close(g["Y"][rows], case.oracle_rows(act, wq, rows))
+    info.update(rows=int(rows.size), fp8_product=fp8, pow2=pow2, p_max_err_over_tol=pinfo["max_err_over_tol"])
+    _record(f"options_{name}_{int(fp8)}{int(pow2)}", info)
