@@ -419,6 +419,28 @@ int dq_linear_forward_host(const void* X_host, int T, int H, int W, int t, int h
                            void* stream);
 
 /*
+ * As dq_linear_forward_host with host_flags:
+ *   DQ_HOST_OVERLAP_PREVIOUS  the copy of X into X_dev may start as soon as the
+ *       previous call of this entry point on the device has read X_dev for the
+ *       last time (its encode stage), instead of after all work enqueued on
+ *       `stream` so far: the copy of one step's input then overlaps the previous
+ *       step's products and copy out.  Work the caller enqueues on `stream`
+ *       between two such calls must not touch X_dev.
+ * dq_linear_forward_host is this call with host_flags = 0.  Both copy X in
+ * T-slabs of whole cube layers, start each slab's statistics pass when its
+ * rows have arrived, and copy the frames finished by each range of the main
+ * product's row tiles back while the next range computes; the call's work
+ * (copies included) ends on `stream`.  Copy streams and events are created on
+ * the first call on a device and kept until exit.
+ */
+#define DQ_HOST_OVERLAP_PREVIOUS 1
+
+int dq_linear_forward_host_ex(const void* X_host, int T, int H, int W, int t, int h, int w, int Ci, int Co,
+                              int rank, const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y_host,
+                              void* X_dev, void* Y_dev, void* workspace, size_t workspace_bytes, int host_flags,
+                              void* stream);
+
+/*
  * Forward pass for callers that cannot allocate device memory (code running
  * under a fixed memory plan such as CUDA-graph capture, processes whose
  * allocator owns all device memory, embedded callers that may not grow their

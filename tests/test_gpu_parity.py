@@ -315,6 +315,42 @@ def test_host_entry_point_pipeline(env, name):
         assert dq.dq_read_device_status(ws, st, clear=True) == 0
 
 
+def test_host_entry_point_overlapping_calls(env):
+    """Back-to-back host-buffer calls with DQ_HOST_OVERLAP_PREVIOUS on one X_dev / Y_dev
+    and different inputs: the second call's copy of X overlaps the first call's
+    products and copy out, and each call's Y equals the device-buffer entry point's
+    for its own input."""
+    dq, torch = env
+    wl = dict(SMALL)["ragged_122"]
+    cases = [Case(wl), Case(wl, seed=99)]
+    refs = [c.run_gpu(dq, torch)["Y"] for c in cases]
+    t, h, w = cases[0].cube
+    _, Pd, L1d, L2d, _ = cases[0].last_inputs
+    Xhs = [torch.from_numpy(c.X.view(np.int16)).pin_memory() for c in cases]
+    Yhs = [torch.full((wl.N, wl.Co), 0x7FC0, dtype=torch.int16).pin_memory() for _ in cases]
+    nbytes = dq.dq_workspace_bytes(wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank)
+    dev = torch.device("cuda")
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    Xd = torch.empty((wl.N, wl.Ci), dtype=torch.int16, device=dev)
+    Yd = torch.empty((wl.N, wl.Co), dtype=torch.int16, device=dev)
+    st = torch.cuda.current_stream()
+    for _ in range(2):
+        for i in range(2):
+            dq.dq_linear_forward_host_ex(Xhs[i], wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d,
+                                         Yhs[i], Xd, Yd, ws, nbytes, dq.DQ_HOST_OVERLAP_PREVIOUS, st)
+        st.synchronize()
+        # the packed weight is the first case's; the second case's reference used its own weight, so
+        # compare the second call against a device-buffer run of its X with the first case's weight
+        assert np.array_equal(Yhs[0].numpy().view(np.uint16), refs[0])
+        Xd2 = torch.from_numpy(cases[1].X.view(np.int16)).to(dev)
+        Y2 = torch.empty_like(Yd)
+        dq.dq_linear_forward_ex(Xd2, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Y2, ws, nbytes,
+                                dq.DQ_STAGE_ALL, None, st)
+        st.synchronize()
+        assert np.array_equal(Yhs[1].numpy().view(np.uint16), Y2.cpu().numpy().view(np.uint16))
+        assert dq.dq_read_device_status(ws, st, clear=True) == 0
+
+
 def test_stage_mask_reuses_workspace(env):
     """Running the three stages as three calls on one workspace equals one call."""
     dq, torch = env

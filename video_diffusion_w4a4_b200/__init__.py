@@ -40,6 +40,7 @@ DQ_NOALLOC_WORKSPACE = 1   # dq_read_device_status: the fixed array of dq_linear
 DQ_PACK_C2 = 1
 DQ_KERNEL_PRODUCT_BF16, DQ_KERNEL_PRODUCT_FP8 = 0, 1
 DQ_DELTA_SCALE_AMAX, DQ_DELTA_SCALE_POW2 = 0, 1
+DQ_HOST_OVERLAP_PREVIOUS = 1
 
 
 class dq_packed_layout(ctypes.Structure):
@@ -94,6 +95,7 @@ _SIGS = {
     "dq_workspace_layout_grouped": ([_I] * 10 + [ctypes.POINTER(dq_workspace_layout)], _I),
     "dq_workspace_bytes_grouped": ([_I] * 10 + [ctypes.POINTER(_SZ)], _I),
     "dq_linear_forward_host": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I),
+    "dq_linear_forward_host_ex": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P, _P, _P, _SZ, _I, _P], _I),
     "dq_linear_forward_noalloc": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P], _I),
     "dq_read_device_status": ([_P, _P, ctypes.POINTER(_I), _I], _I),
     "dq_selftest_bounded_wait": ([_I, _P, ctypes.POINTER(_I)], _I),
@@ -369,6 +371,15 @@ def dq_linear_forward_host(X_host, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_
            _lib.dq_linear_forward_host(_ptr(X_host), T, H, W, t, h, w, Ci, Co, rank, _ptr(packed_W), _ptr(L1_mma),
                                        _ptr(L2_slab), _ptr(Y_host), _ptr(X_dev), _ptr(Y_dev), _ptr(workspace),
                                        workspace_bytes, _stream(stream)))
+
+
+def dq_linear_forward_host_ex(X_host, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y_host, X_dev,
+                              Y_dev, workspace, workspace_bytes, host_flags=0, stream=None) -> None:
+    """dq_linear_forward_host with host_flags (DQ_HOST_OVERLAP_PREVIOUS)."""
+    _check("dq_linear_forward_host_ex",
+           _lib.dq_linear_forward_host_ex(_ptr(X_host), T, H, W, t, h, w, Ci, Co, rank, _ptr(packed_W),
+                                          _ptr(L1_mma), _ptr(L2_slab), _ptr(Y_host), _ptr(X_dev), _ptr(Y_dev),
+                                          _ptr(workspace), workspace_bytes, host_flags, _stream(stream)))
 
 
 def dq_linear_forward_noalloc(X, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y, stream=None) -> None:

@@ -159,6 +159,8 @@ struct Aux {
     std::mutex mu;
     cudaStream_t in = nullptr, out = nullptr;
     cudaEvent_t ev[2 + kHostSlabs + kHostChunks] = {};
+    cudaEvent_t x_free = nullptr;   // recorded after a call's last read of X_dev (its encode pass)
+    bool x_free_recorded = false;
 };
 std::mutex g_aux_mu;
 std::map<int, Aux> g_aux;
@@ -177,6 +179,7 @@ int host_aux(Aux** out) {
             return cuda_fail(e, "copy streams");
         for (cudaEvent_t& ev : A.ev)
             if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e, "events");
+        if ((e = cudaEventCreateWithFlags(&A.x_free, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e, "events");
     }
     *out = &A;
     return DQ_OK;
@@ -292,6 +295,7 @@ struct Pipeline {
     std::vector<int> kt_cuts;    // cube-layer boundaries of the slabs: 0 = kt_cuts[0] < ... = KT
     std::vector<int> tile_cuts;  // row-tile boundaries of the main-product launches: 0 = ... = ceil(N / 256)
     std::function<int(int)> before_slab;
+    std::function<int()> after_encode;
     std::function<int(int, long long)> after_chunk;
 };
 
@@ -424,6 +428,7 @@ int forward_impl(const void* X, int T, int H, int W, int t, int h, int w, int Ci
         } else if (do_encode && (e = dq::launch_cube_encode(tm_x, tm_m, qp, st)) != cudaSuccess) {
             return cuda_fail(e, "k_cube_encode");
         }
+        if (pipe && pipe->after_encode && (rc = pipe->after_encode())) return rc;
     }
     rec(1);
     if ((stage_mask & DQ_STAGE_KERNEL_GEMM) && fp8prod) {
@@ -547,14 +552,29 @@ int dq_linear_forward(const void* X, int T, int H, int W, int t, int h, int w, i
 int dq_linear_forward_host(const void* X_host, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
                            const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y_host, void* X_dev,
                            void* Y_dev, void* workspace, size_t workspace_bytes, void* stream) {
+    return dq_linear_forward_host_ex(X_host, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y_host, X_dev,
+                                     Y_dev, workspace, workspace_bytes, 0, stream);
+}
+
+int dq_linear_forward_host_ex(const void* X_host, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
+                              const void* packed_W, const void* L1_mma, const void* L2_slab, void* Y_host, void* X_dev,
+                              void* Y_dev, void* workspace, size_t workspace_bytes, int host_flags, void* stream) {
     int rc = check_shape(T, H, W, t, h, w, Ci, Co, rank);
     if (rc) return rc;
     if (!X_host || !Y_host || !X_dev || !Y_dev) return DQ_ERR_INVALID_ARG;
+    if (host_flags & ~DQ_HOST_OVERLAP_PREVIOUS) return DQ_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     const Geom g = dq::make_geom(T, H, W, t, h, w);
     const size_t HW = (size_t)H * W;
     if ((long long)t * h * w > 128 || g.KT < 2) {
-        // one copy in, the layer, one copy out
+        // one copy in, the layer, one copy out, all on `stream` (a later overlapping call then waits
+        // for all of it)
+        Aux* aux = nullptr;
+        if ((rc = host_aux(&aux))) return rc;
+        {
+            std::lock_guard<std::mutex> lk(aux->mu);
+            aux->x_free_recorded = false;
+        }
         size_t N = (size_t)T * HW;
         cudaError_t e;
         if ((e = cudaMemcpyAsync(X_dev, X_host, N * Ci * 2, cudaMemcpyHostToDevice, st)) != cudaSuccess)
@@ -581,9 +601,15 @@ int dq_linear_forward_host(const void* X_host, int T, int H, int W, int t, int h
     for (int i = 0; i <= nslab; i++) pipe.kt_cuts.push_back((int)((long long)g.KT * i / nslab));
     for (int i = 0; i <= nchunk; i++) pipe.tile_cuts.push_back((int)((long long)tiles * i / nchunk));
     cudaError_t e;
-    // the copies in wait for earlier work on `stream` (which may still read X_dev)
-    if ((e = cudaEventRecord(aux->ev[0], st)) != cudaSuccess || (e = cudaStreamWaitEvent(aux->in, aux->ev[0], 0)))
-        return cuda_fail(e, "stream order");
+    if ((host_flags & DQ_HOST_OVERLAP_PREVIOUS) && aux->x_free_recorded) {
+        // the copies in wait only for the previous call's last read of X_dev, so that they overlap its
+        // products and its copies out
+        if ((e = cudaStreamWaitEvent(aux->in, aux->x_free, 0)) != cudaSuccess) return cuda_fail(e, "stream order");
+    } else {
+        // the copies in wait for earlier work on `stream` (which may still read X_dev)
+        if ((e = cudaEventRecord(aux->ev[0], st)) != cudaSuccess || (e = cudaStreamWaitEvent(aux->in, aux->ev[0], 0)))
+            return cuda_fail(e, "stream order");
+    }
     for (int i = 0; i < nslab; i++) {
         const size_t f0 = (size_t)pipe.kt_cuts[i] * t, f1 = dq::imin(pipe.kt_cuts[i + 1] * t, T);
         const size_t off = f0 * HW * Ci * 2, bytes = (f1 - f0) * HW * Ci * 2;
@@ -592,6 +618,12 @@ int dq_linear_forward_host(const void* X_host, int T, int H, int W, int t, int h
             (e = cudaEventRecord(aux->ev[1 + i], aux->in)) != cudaSuccess)
             return cuda_fail(e, "copy of X");
     }
+    pipe.after_encode = [&]() {
+        cudaError_t e1 = cudaEventRecord(aux->x_free, st);
+        if (e1 != cudaSuccess) return cuda_fail(e1, "stream order");
+        aux->x_free_recorded = true;
+        return (int)DQ_OK;
+    };
     pipe.before_slab = [&](int i) {
         cudaError_t e1 = cudaStreamWaitEvent(st, aux->ev[1 + i], 0);
         return e1 == cudaSuccess ? DQ_OK : cuda_fail(e1, "stream order");
