@@ -204,21 +204,22 @@ int dq_pack_weight_factors(const uint16_t* W, const uint16_t* L1, const uint16_t
  *               (DQ_KERNEL_PRODUCT_FP8).  The note runs the kernel-token product
  *               on FP8 tensor cores; with Eq. 4's E4M3 group-16 scales the
  *               product q s_b needs up to 6 significant bits, which no FP8
- *               operand holds.  C2 rounds each group scale up to the nearest
- *               {1, 1.5} x 2^e (e >= -9, 1.5 x 2^-9 excluded), caps it at 384,
- *               takes S_W = amax(R) / (6 * 384), and per 32 channels raises the
- *               smaller of the two scales to at least 2^-10 times the larger;
- *               then every q s_b of a 32-channel block is an E4M3 value times
- *               one power of two 2^u.  The blob's dqw section then holds, in
- *               place of BF16 q s_b: Co x Ci E4M3 codes of q s_b / 2^u (u such
- *               that the block's largest |q s_b| / 2^u lies in [256, 512)),
+ *               operand holds.  C2 takes S_W = amax(R) / (6 * 384) and rounds
+ *               each group scale to the nearest member (ties to the larger) of
+ *               {0} and the E4M3 values m 2^e with m in {1, 1.25, 1.5}, up to
+ *               384; per 32 channels a nonzero smaller scale is raised to the
+ *               smallest member >= 2^-9 times the larger.  Then every q s_b of a
+ *               32-channel block is an E4M3 value times one power of two 2^u.
+ *               The blob's dqw section then holds, in place of BF16 q s_b:
+ *               Co x Ci E4M3 codes of q s_b / 2^u (u such that the block's
+ *               largest |q s_b| / 2^u lies in [128, 256)),
  *               followed by the exponents u + 127 (UE8M0) in the layout
  *               dq_sfb_offset gives for a Co x (Ci / 2) matrix, block j of that
  *               matrix standing for 32-channel block j (four copies, one per
  *               tensor-memory quadrant, as for the weight scales).  Header flag
- *               bit 1 marks such a blob.  The price is accuracy: rounding scales
- *               up leaves the top E2M1 codes unused in many groups (weight
- *               error about 1.2 to 1.5 times Eq. 4's on the synthetic weights).
+ *               bit 1 marks such a blob.  The price is accuracy: three scale
+ *               mantissas instead of E4M3's eight (weight error 1.06 to 1.14
+ *               times Eq. 4's on the synthetic weights).
  */
 #define DQ_PACK_C2 1
 

@@ -62,8 +62,8 @@ def _L():
         lib.or_quantize_activations.argtypes = [P] + [I] * 7 + [P] * 7
         lib.or_quantize_activations_opt.argtypes = [P] + [I] * 7 + [P] * 7 + [I]
         lib.or_pow2_ceil.argtypes = [F]
-        lib.or_c2_scale_up.argtypes = [F]
-        lib.or_c2_scale_up.restype = F
+        lib.or_c2_scale_nearest.argtypes = [F]
+        lib.or_c2_scale_nearest.restype = F
         lib.or_fp4_quantize_c2.argtypes = [P, LL, I, P, P, P]
         lib.or_fp4_quantize_c2.restype = LL
         lib.or_c2_fp8_operand.argtypes = [P, P, LL, I, P, P]
@@ -381,7 +381,7 @@ def quantize_weight(Wbits, L1, L2, c2: bool = False) -> dict:
 
 
 def fp4_quantize_c2(Z):
-    """C2 FP4: restricted group scales {1, 1.5} x 2^e; returns (codes, scales, S, raised)."""
+    """C2 FP4: restricted group scales {1, 1.25, 1.5} x 2^e (nearest); returns (codes, scales, S, raised)."""
     Z = np.ascontiguousarray(Z, dtype=np.float32)
     rows, cols = Z.shape
     codes = np.empty((rows, cols // 2), np.uint8)

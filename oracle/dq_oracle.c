@@ -296,32 +296,60 @@ static void fp4_row(const float* z, int cols, float S, uint8_t* codes, uint8_t* 
 /* ------------------------------------------------------------------------ */
 
 /*
- * The smallest value of the form {1, 1.5} x 2^e (e >= -9, 1.5 x 2^-9 excluded:
- * E4M3 cannot hold it) that is >= v, for v > 0; 0 for v <= 0.  Every such
- * value is an E4M3 value, and so is its product with any E2M1 value times a
- * common power of two (mantissas 1, 1.125, 1.5 need at most 3 bits).
+ * The restricted group scale of C2 weights: the member of
+ *   A = {0} U { m 2^e : m in {1, 1.25, 1.5}, m 2^e an E4M3 value, m 2^e <= 384 }
+ * nearest to v >= 0 (ties to the larger member).  The product of a member with
+ * an E2M1 value has at most three fraction bits (1.5 x 1.25 = 1.875,
+ * 1.5 x 1.5 = 1.125 x 2), so it is an E4M3 value times a power of two; m = 1.75
+ * is left out because 1.5 x 1.75 needs four.  Below 2^-6 the E4M3 members are
+ * k 2^-9 with k in {1, 2, 3, 4, 5, 6} (5 2^-9 = 1.25 x 2^-7; 7 2^-9 is not of
+ * the form).  Found by search over A.
  */
-float or_c2_scale_up(float v) {
-    if (!(v > 0.0f)) return 0.0f;
-    if (v <= 0x1p-9f) return 0x1p-9f;
+static int c2_member(double c) {
+    if (c == 0.0) return 1;
+    if (c > 384.0) return 0;
     int e;
-    const float m = frexpf(v, &e);        /* v = m 2^e, m in [0.5, 1) */
-    float r;
-    if (m == 0.5f) r = v;                  /* a power of two */
-    else if (m <= 0.75f) r = ldexpf(0.75f, e);
-    else r = ldexpf(1.0f, e);
-    if (r == 0x1.8p-9f) r = 0x1p-8f;
-    return r;
+    const double m = 2.0 * frexp(c, &e);          /* c = m 2^(e-1), m in [1, 2) */
+    if (m != 1.0 && m != 1.25 && m != 1.5) return 0;
+    return or_e4m3_value(or_e4m3_encode((float)c)) == c;
+}
+
+/* The smallest member of A that is >= v > 0. */
+static double c2_member_at_least(double v) {
+    double best = 1e300;
+    for (int e = -9; e <= 9; e++)
+        for (int i = 0; i < 3; i++) {
+            const double c = ldexp(i == 0 ? 1.0 : (i == 1 ? 1.25 : 1.5), e);
+            if (c2_member(c) && c >= v && c < best) best = c;
+        }
+    return best;
+}
+
+float or_c2_scale_nearest(float v) {
+    if (!(v > 0.0f)) return 0.0f;
+    double best = 0.0, bd = (double)v;
+    for (int e = -9; e <= 9; e++)
+        for (int i = 0; i < 3; i++) {
+            const double c = ldexp(i == 0 ? 1.0 : (i == 1 ? 1.25 : 1.5), e);
+            if (!c2_member(c)) continue;
+            const double d = fabs(c - (double)v);
+            if (d < bd || (d == bd && c > best)) {
+                best = c;
+                bd = d;
+            }
+        }
+    return (float)best;
 }
 
 /*
  * C2 weight quantiser (the restricted-scale reading, an option; the default is
  * fp4_row's Eq. 4 form).  Per-tensor S = amax / (6 * 384) (384 = 1.5 x 2^8,
- * the largest restricted scale), group-16 scales s_b = or_c2_scale_up(amax_b /
- * (6 S)), then, per 32 channels, the smaller of the two scales raised to at
- * least 2^-10 times the larger (a power-of-two ratio keeps the form), so that
- * the block's q s_b span at most E4M3's exact range under one power-of-two
- * exponent; q = E2M1(z / (s_b S)).  Returns the number of raised scales.
+ * the largest member), group-16 scales s_b = or_c2_scale_nearest(amax_b /
+ * (6 S)), then, per 32 channels, a nonzero smaller scale raised to the
+ * smallest member >= 2^-9 times the larger, so that the block's values q s_b
+ * span at most 2^14 and fit E4M3's normal range under one power-of-two
+ * exponent; q = E2M1(z / (s_b S)) (nearest even, saturating at 6).  Returns
+ * the number of raised scales.
  */
 long long or_fp4_quantize_c2(const float* Z, long long rows, int cols, uint8_t* codes, uint8_t* scales,
                              float* S_out) {
@@ -346,14 +374,12 @@ long long or_fp4_quantize_c2(const float* Z, long long rows, int cols, uint8_t* 
                     float a = fabsf(z[b * 16 + i]);
                     if (a > am) am = a;
                 }
-                sb[h] = or_c2_scale_up(am / denom);
-                if (sb[h] > 384.0f) sb[h] = 384.0f;   /* fp32 rounding of amax / denom just above 384 */
+                sb[h] = or_c2_scale_nearest(am / denom);
             }
             const float big = sb[0] > sb[1] ? sb[0] : sb[1];
             for (int h = 0; h < 2; h++) {
-                const float floor_s = ldexpf(big, -10);
-                if (sb[h] < floor_s) {
-                    sb[h] = floor_s;
+                if (sb[h] > 0.0f && sb[h] < ldexpf(big, -9)) {
+                    sb[h] = (float)c2_member_at_least(ldexp((double)big, -9));
                     raised++;
                 }
             }
@@ -376,9 +402,10 @@ long long or_fp4_quantize_c2(const float* Z, long long rows, int cols, uint8_t* 
 /*
  * The FP8 form of C2 weights for a kind::mxf8f6f4 product: per 32 channels one
  * UE8M0 exponent u (biased by 127) and E4M3 codes of q s_b / 2^u, with u chosen
- * so that the block's largest |q s_b| lands in [256, 512).  Returns the number
- * of elements whose E4M3 code does not reproduce q s_b exactly (0 for weights
- * from or_fp4_quantize_c2).
+ * so that the block's largest |q s_b| lands in [128, 256) (a significand of
+ * 1.875 in [256, 512) would exceed E4M3's 448).  Returns the number of elements
+ * whose E4M3 code does not reproduce q s_b exactly (0 for weights from
+ * or_fp4_quantize_c2).
  */
 long long or_c2_fp8_operand(const uint8_t* codes, const uint8_t* scales, long long rows, int cols, uint8_t* fp8,
                             uint8_t* ue8m0) {
@@ -397,7 +424,7 @@ long long or_c2_fp8_operand(const uint8_t* codes, const uint8_t* scales, long lo
             if (wmax > 0.0) {
                 int e;
                 frexp(wmax, &e);          /* wmax in [2^(e-1), 2^e) */
-                u = e - 1 - 8;
+                u = e - 1 - 7;
             }
             ue8m0[(size_t)r * (cols / 32) + b2] = (uint8_t)(u + 127);
             for (int i = 0; i < 32; i++) {

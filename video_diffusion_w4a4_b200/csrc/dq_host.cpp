@@ -104,17 +104,42 @@ inline float e2m1_to_float(uint8_t c) {
     return (c & 8) ? -v : v;
 }
 
-// The restricted group scale of C2 weights: the least value {1, 1.5} x 2^e with e >= -9 that is
-// >= v (v > 0), skipping 1.5 x 2^-9, which E4M3 cannot hold; every such value is an E4M3 value
-// whose product with an E2M1 value has at most three fraction bits.
-inline float c2_round_scale_up(float v) {
-    if (!(v > 0.0f)) return 0.0f;
-    const float lo = ldexpf(1.0f, -9);
-    if (v <= lo) return lo;
-    int e;
-    const float m = frexpf(v, &e);   // v = m 2^e, 0.5 <= m < 1
-    const float up = (m == 0.5f) ? v : ldexpf(m <= 0.75f ? 0.75f : 1.0f, e);
-    return (up == ldexpf(1.5f, -9)) ? ldexpf(1.0f, -8) : up;
+// Restricted group scales of C2 weights: 0 and the values m 2^e (m in {1, 1.25, 1.5}) that E4M3
+// holds, up to 384, in increasing order.  Their products with E2M1 values have at most three
+// fraction bits, so each product is an E4M3 value times a power of two.  Built from the E4M3
+// code table: normal codes whose 3-bit mantissa is 0, 2 or 4, and subnormal codes 1..6 (k 2^-9,
+// each of the form m 2^e; 7 2^-9 = 1.75 x 2^-7 is not).
+const std::vector<float>& c2_scale_set() {
+    static const std::vector<float> set = [] {
+        std::vector<float> v{0.0f};
+        for (int code = 1; code < 0x7F; code++) {
+            const int e = code >> 3, m = code & 7;
+            const bool ok = e == 0 ? m <= 6 : (m == 0 || m == 2 || m == 4);
+            const float val = e4m3_to_float((uint8_t)code);
+            if (ok && val <= 384.0f) v.push_back(val);
+        }
+        std::sort(v.begin(), v.end());
+        return v;
+    }();
+    return set;
+}
+
+// The member nearest to v >= 0, ties to the larger.
+inline float c2_scale_nearest(float v) {
+    const std::vector<float>& S = c2_scale_set();
+    const auto it = std::lower_bound(S.begin(), S.end(), v);   // first member >= v
+    if (it == S.end()) return S.back();
+    if (it == S.begin()) return *it;
+    const float hi = *it, lo = *(it - 1);
+    return ((double)hi - v <= (double)v - lo) ? hi : lo;
+}
+
+// The smallest member >= v (v > 0, at most the largest member).
+inline float c2_scale_at_least(double v) {
+    const std::vector<float>& S = c2_scale_set();
+    for (float c : S)
+        if ((double)c >= v) return c;
+    return S.back();
 }
 
 // ------------------------------------------------------------------ small dense linear algebra (fp64)
@@ -464,9 +489,10 @@ int dq_pack_weight_factors_ex(const uint16_t* Wb, const uint16_t* L1, const uint
     uint8_t* scales = base + L.off_scales;
     uint16_t* dqw = (uint16_t*)(base + L.off_dqw);
     if (c2) {
-        // C2: per 32 channels, two restricted group scales (the smaller raised to at least 2^-10 of the
-        // larger, so the 32 values q s_b fit one UE8M0 exponent exactly), E2M1 codes, and the FP8 form:
-        // E4M3 codes of q s_b / 2^u with the block's largest |q s_b| / 2^u in [256, 512)
+        // C2: per 32 channels, two restricted group scales (a nonzero smaller one raised to the smallest
+        // member >= 2^-9 of the larger, so the 32 values q s_b fit E4M3 exactly under one UE8M0 exponent),
+        // E2M1 codes, and the FP8 form: E4M3 codes of q s_b / 2^u with the block's largest |q s_b| / 2^u in
+        // [128, 256) (E4M3 stops at 448, below 1.875 x 256)
         uint8_t* fp8 = base + L.off_dqw;
         uint8_t* ue = fp8 + (size_t)Co * Ci;
 #pragma omp parallel for schedule(static)
@@ -477,12 +503,12 @@ int dq_pack_weight_factors_ex(const uint16_t* Wb, const uint16_t* L1, const uint
                 for (int hh = 0; hh < 2; hh++) {
                     float am = 0.0f;
                     for (int i = 0; i < 16; i++) am = std::max(am, fabsf(z[32 * j + 16 * hh + i]));
-                    sb[hh] = std::min(c2_round_scale_up(am / denom), 384.0f);
+                    sb[hh] = c2_scale_nearest(am / denom);
                 }
-                const float floor_s = ldexpf(std::max(sb[0], sb[1]), -10);
+                const double floor_s = ldexp((double)std::max(sb[0], sb[1]), -9);
                 float w[32], wmax = 0.0f;
                 for (int hh = 0; hh < 2; hh++) {
-                    const float sbv = std::max(sb[hh], floor_s);
+                    const float sbv = (sb[hh] > 0.0f && sb[hh] < floor_s) ? c2_scale_at_least(floor_s) : sb[hh];
                     const uint8_t code = float_to_e4m3(sbv);   // exact: a restricted scale is an E4M3 value
                     const int b = 2 * j + hh;
                     const size_t so = dq::sfb_offset(o, b, Ci);
@@ -501,7 +527,7 @@ int dq_pack_weight_factors_ex(const uint16_t* Wb, const uint16_t* L1, const uint
                 if (wmax > 0.0f) {
                     int e;
                     frexpf(wmax, &e);    // wmax in [2^(e-1), 2^e)
-                    u = e - 9;
+                    u = e - 8;
                 }
                 for (int i = 0; i < 32; i++) fp8[(size_t)o * Ci + 32 * j + i] = float_to_e4m3(ldexpf(w[i], -u));
                 const size_t uo = dq::c2_sf_offset(o, j, Ci);
