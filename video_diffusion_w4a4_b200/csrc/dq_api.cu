@@ -438,12 +438,12 @@ int forward_impl(const void* X, int T, int H, int W, int t, int h, int w, int Ci
             return map_fail("FP8 product A");
         if (!map_2d(&tm_b, pw + pl.off_dqw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Ci, Co, 128, 128))
             return map_fail("FP8 product B");
-        if (!map_sfb(&tm_fb, pw + pl.off_dqw + (size_t)Co * Ci, Ci / 2, Co, 1)) return map_fail("FP8 product scales");
+        if (!map_sfb(&tm_fb, pw + pl.off_dqw + (size_t)Co * Ci, Ci / 2, Co, 2)) return map_fail("FP8 product scales");
         dq::GemmParams p = gp;
         p.M = (int)g.K;
         p.tile_m0 = 0;
         p.tile_m1 = (int)dq::cdiv(g.K, 256);
-        p.k_stages = Ci / 128;
+        p.k_stages = Ci / 256;
         p.tile_group = 8;
         p.s8 = qp.s8;
         p.pout = (float*)(ws + wl.off_p);
