@@ -460,7 +460,7 @@ int forward_impl(const void* X, int T, int H, int W, int t, int h, int w, int Ci
         p.M = (int)g.K;
         p.tile_m0 = 0;
         p.tile_m1 = (int)dq::cdiv(g.K, 256);
-        p.k_stages = a_cols / 64;
+        p.k_stages = a_cols / 128;
         p.b_kblocks = Ci / 64;
         p.tile_group = 8;   // the BF16 weight (Co x Ci x 2 bytes) does not stay in L2 beside the rows
         p.s8 = kg ? nullptr : qp.s8;

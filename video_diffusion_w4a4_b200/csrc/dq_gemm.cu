@@ -74,11 +74,13 @@ constexpr uint32_t kFp8SfaCol = 256;            // FP8 product: tensor-memory co
 constexpr uint32_t kFp8SfbCol = 264;            //   and of the first B-exponent slot (16 columns per stage)
 
 __host__ __device__ constexpr int g_stages(int kind) {
-    return kind == kGemmMain ? 4 : (kind == kGemmKernelFp8 ? 3 : 7);
+    return kind == kGemmMain ? 4 : 3;
 }
-// Operand tiles per stage: the FP8 product stages 256 channels (two 128-byte-row boxes of each
-// operand, eight MMAs) between barrier hand-offs; measured 7 % faster than 128-channel stages.
-__host__ __device__ constexpr uint32_t stage_mul(int kind) { return kind == kGemmKernelFp8 ? 2u : 1u; }
+// Operand tiles per stage: the kernel-token products stage two 128-byte-row boxes of each operand
+// (128 channels of BF16, 256 of FP8; eight MMAs) between barrier hand-offs, measured 6-8 % faster
+// than one box per stage with twice the stages; the main product keeps one (its scale copies and
+// TMEM slots are per box).
+__host__ __device__ constexpr uint32_t stage_mul(int kind) { return kind == kGemmMain ? 1u : 2u; }
 
 // Output tile -> (row tile, column tile).  group <= 1: row-major, which suits a weight that stays
 // in L2 while the row tiles stream.  Otherwise groups of `group` row tiles walked column by column:
@@ -231,9 +233,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_2d_pair_hint(sb + kBBytes, &tm_b, fb, i * 256 + 128, nb, keep);
                         tma_load_3d_pair(sm + L.sfb + s * 2 * kSFB8Bytes, &tm_fb, fb, 0, 32 * i, n0 >> 8);
                     } else if (!kMain) {
-                        if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes));
-                        tma_load_2d_pair_hint(sa, &tm_a, fb, i * 64, m0, stream);
-                        tma_load_2d_pair_hint(sb, &tm_b, fb, (i < p.b_kblocks ? i : i - p.b_kblocks) * 64, nb, keep);
+                        // 128 channels of A (two 64-channel boxes); B's channels are A's modulo Ci
+                        // (the grouped-scale operand repeats the weight for its hi and lo halves)
+                        if (lead) mbar_arrive_expect_tx(&full[s], 2 * (2 * kABytes + 2 * kBBytes));
+                        tma_load_2d_pair_hint(sa, &tm_a, fb, i * 128, m0, stream);
+                        tma_load_2d_pair_hint(sa + kABytes, &tm_a, fb, i * 128 + 64, m0, stream);
+                        tma_load_2d_pair_hint(sb, &tm_b, fb, (i * 128) % p.Ci, nb, keep);
+                        tma_load_2d_pair_hint(sb + kBBytes, &tm_b, fb, (i * 128 + 64) % p.Ci, nb, keep);
                     } else if (i < nk) {
                         if (lead) mbar_arrive_expect_tx(&full[s], 2 * (kABytes + kBBytes + kSFABytes + kSFBBytes));
                         tma_load_2d_pair(sa, &tm_a, fb, i * 128, m0);
@@ -312,8 +318,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         const uint32_t id = kMain ? id_slab : id_main;
 #pragma unroll
-                        for (int k = 0; k < 4; k++)
-                            mma_bf16_pair(acc, desc_k_sw128(aa + 32 * k), desc_k_sw128(bb + 32 * k), id,
+                        for (int k = 0; k < 4 * (int)stage_mul(kKind); k++)
+                            mma_bf16_pair(acc, desc_k_sw128(aa + (k / 4) * kABytes + 32 * (k % 4)),
+                                          desc_k_sw128(bb + (k / 4) * kBBytes + 32 * (k % 4)), id,
                                           (kMain || (i | k) != 0) ? 1u : 0u);
                     }
                     tc_commit_pair_both(&empty[s], kPairMask);
