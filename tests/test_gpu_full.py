@@ -154,3 +154,31 @@ def test_full_size_options(env, name, fp8, pow2):
     info = assert_y_close(g["Y"][rows], case.oracle_rows(act, wq, rows))
     info.update(rows=int(rows.size), fp8_product=fp8, pow2=pow2, p_max_err_over_tol=pinfo["max_err_over_tol"])
     _record(f"options_{name}_{int(fp8)}{int(pow2)}", info)
+
+
+def test_full_size_host_entry_point(env):
+    """The end-to-end path the bench times, at the 720p FFN down-projection: pinned X in
+    T-slabs, the statistics pass per slab, Y's finished frames back per range of row
+    tiles, and a second call overlapping the first (DQ_HOST_OVERLAP_PREVIOUS); both
+    calls' Y bit-identical to the device-buffer entry point's."""
+    dq, torch = env
+    wl = synth.WORKLOADS["wan720p_ffn_down"]
+    case = Case(wl)
+    g = case.run_gpu(dq, torch)
+    t, h, w = case.cube
+    _, Pd, L1d, L2d, _ = case.last_inputs
+    dev = torch.device("cuda")
+    Xh = torch.from_numpy(case.X.view(np.int16)).pin_memory()
+    Yhs = [torch.empty((wl.N, wl.Co), dtype=torch.int16).pin_memory() for _ in range(2)]
+    nbytes = dq.dq_workspace_bytes(wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    Xd = torch.empty((wl.N, wl.Ci), dtype=torch.int16, device=dev)
+    Yd = torch.empty((wl.N, wl.Co), dtype=torch.int16, device=dev)
+    st = torch.cuda.current_stream()
+    for i in range(2):
+        dq.dq_linear_forward_host_ex(Xh, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yhs[i], Xd,
+                                     Yd, ws, nbytes, dq.DQ_HOST_OVERLAP_PREVIOUS if i else 0, st)
+    st.synchronize()
+    assert dq.dq_read_device_status(ws, st, clear=True) == 0
+    for i in range(2):
+        assert np.array_equal(Yhs[i].numpy().view(np.uint16), g["Y"]), i
