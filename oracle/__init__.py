@@ -73,6 +73,7 @@ def _L():
         lib.or_output_rows.argtypes = [P, P, F, P, P, P, I, P, P, P, F, I, I, P, P, P, I, P, LL, P]
         lib.or_fp8_kernel_tokens.argtypes = [P, LL, I, I, P, P]
         lib.or_num_threads.restype = I
+        lib.or_gelu_erf.argtypes = [P, LL, P]
         lib.or_delta_amax.argtypes = [P] + [I] * 7 + [P]
         lib.or_quantize_cubes.argtypes = [P] + [I] * 7 + [P, LL, F, P, P, P, P, P]
         _lib = lib
@@ -443,3 +444,21 @@ def output_rows(act: dict, wq: dict, X, L1, L2, rows, kernel: bool = True, lowra
     if bias is not None:
         Y += bf16_value(np.asarray(bias, np.uint16).reshape(1, Co))
     return Y
+
+
+# --------------------------------------------------------------------------- feed-forward block
+
+def gelu_erf(y) -> np.ndarray:
+    """GELU(y) = y Phi(y) = y erfc(-y / sqrt 2) / 2, element by element in fp64 (or_gelu_erf)."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    out = np.empty_like(y)
+    _L().or_gelu_erf(_p(y), y.size, _p(out))
+    return out
+
+
+def ffn_hidden_rows(act: dict, wq: dict, X, L1, L2, rows, bias=None) -> np.ndarray:
+    """fp64 hidden rows of a feed-forward block: GELU of the up-projection's Y rows
+    (output_rows, natural token indices `rows`), before the hidden tensor's one
+    rounding to BF16.  The down-projection then quantises that BF16 tensor as any
+    layer input (quantize_activations)."""
+    return gelu_erf(output_rows(act, wq, X, L1, L2, rows, bias=bias))

@@ -28,7 +28,10 @@
  * Options beside the default (each pinned on its own): one kernel scale per 64
  * channels (or_fp8_kernel_tokens), a power-of-two per-tensor delta scale
  * (or_quantize_activations_opt), restricted weight scales with an exact FP8
- * form (or_fp4_quantize_c2, or_c2_fp8_operand), an additive bias (Python side).
+ * form (or_fp4_quantize_c2, or_c2_fp8_operand), an additive bias (Python side),
+ * and the step between the two layers of a feed-forward block (or_gelu_erf).
+ *   - the feed-forward activation, which the note does not name, is GELU in its
+ *     exact form y * Phi(y), evaluated in fp64 on the producer layer's output.
  * Parity pins: see tests/test_oracle_*.py.  Parity unpinned: nothing in this
  * file; the GPU's tensor-core accumulation order is covered only by the Y
  * tolerance.
@@ -737,6 +740,17 @@ void or_e2m1_encode_array(const float* v, long long n, uint8_t* out) {
 void or_e4m3_encode_array(const float* v, long long n, uint8_t* out) {
 #pragma omp parallel for schedule(static)
     for (long long i = 0; i < n; i++) out[i] = (uint8_t)or_e4m3_encode(v[i]);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Feed-forward block: the activation between the up- and down-projection     */
+/* ------------------------------------------------------------------------ */
+
+/* GELU in its exact form: GELU(y) = y * Phi(y), Phi the standard normal CDF,
+ * Phi(y) = erfc(-y / sqrt 2) / 2 (erfc keeps Phi accurate for large negative
+ * y, where 1 + erf would cancel).  fp64, element by element. */
+void or_gelu_erf(const double* y, long long n, double* out) {
+    for (long long i = 0; i < n; i++) out[i] = 0.5 * y[i] * erfc(-y[i] / sqrt(2.0));
 }
 
 /* Threads an OpenMP loop of this file uses (for reporting the CPU baseline). */
