@@ -18,6 +18,11 @@ one 4-byte NCCL all-reduce(max) of the delta amax between the statistics and
 encode stages), so the total work is fixed ("strong" scaling);
 --parallelism replicas runs an independent layer per GPU instead ("weak").
 
+--ffn fused|separate times the 720p feed-forward block instead (one GPU): the
+up-projection (5120 -> 13824, cube 2x2x2) with GELU in its main product's
+epilogue, then the down-projection (13824 -> 5120, cube 1x2x2); `fused` forms the
+down-projection's statistics pass in that epilogue, `separate` runs it on its own.
+
 --impl reference times the CPU oracle instead: each step a bounded slice of
 the same seeded cube sample as the GPU arm's cpu_baseline, under the delta
 scale of a whole-tensor statistics pass.
@@ -291,6 +296,94 @@ def layer_flops_rows(wl, K, rows):
 
 # --------------------------------------------------------------------------- GPU arm
 
+def run_ffn(args):
+    """The feed-forward block through dq_ffn_forward: one JSON line with the block's TFLOP/s and the six
+    stage times (each layer's quantise, kernel-token product and main product)."""
+    import torch
+    import video_diffusion_w4a4_b200 as dq
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--ffn runs on one GPU")
+    up, down = synth.WORKLOADS["wan720p_ffn_up"], synth.WORKLOADS["wan720p_ffn_down"]
+    if args.frames:
+        shrink = lambda wl: synth.Workload(f"{wl.name}_T{args.frames}", args.frames, wl.H, wl.W, wl.Ci, wl.Co, wl.rank,
+                                           wl.cube, (args.frames,) + tuple(wl.grid[1:]), wl.x_outliers, wl.w_outliers,
+                                           wl.gelu)
+        up, down = shrink(up), shrink(down)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    X = synth.activations(up)
+    pu, L1u, L2u = dq.dq_pack_weight(synth.weight(up), up.rank)
+    pd, L1d, L2d = dq.dq_pack_weight(synth.weight(down), down.rank)
+    t16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev)
+    Xd, L1u, L2u, L1d, L2d = t16(X), t16(L1u), t16(L2u), t16(L1d), t16(L2d)
+    Pu, Pd = torch.from_numpy(pu).to(dev), torch.from_numpy(pd).to(dev)
+    Hd = torch.empty((up.N, up.Co), dtype=torch.int16, device=dev)
+    Yd = torch.empty((up.N, down.Co), dtype=torch.int16, device=dev)
+    lu = dq.dq_workspace_layout_opts(up.T, up.H, up.W, *up.cube, up.Ci, up.Co, up.rank)
+    ld = dq.dq_workspace_layout_opts(down.T, down.H, down.W, *down.cube, down.Ci, down.Co, down.rank)
+    wsu = torch.zeros(lu.total_bytes, dtype=torch.uint8, device=dev)
+    wsd = torch.zeros(ld.total_bytes, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream(dev)
+    flags = 0 if args.ffn == "fused" else dq.DQ_FFN_SEPARATE_STATISTICS
+    fused = args.ffn == "fused" and dq.dq_ffn_fused_statistics(up.T, up.H, up.W, up.cube, down.cube)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(args.steps)]
+    for row in evs:
+        for e in row:
+            e.record(st)
+    def step(ev=None):
+        dq.dq_ffn_forward(Xd, up.T, up.H, up.W, up.cube, down.cube, up.Ci, up.Co, down.Co, up.rank, down.rank, Pu,
+                          L1u, L2u, Pd, L1d, L2d, Hd, Yd, wsu, lu.total_bytes, wsd, ld.total_bytes, flags, ev, st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    for ws in (wsu, wsd):
+        status = dq.dq_read_device_status(ws, st, clear=True)
+        if status != 0:
+            raise RuntimeError(f"device status after warm-up: {dq.dq_status_string(status)}")
+    with ClockSampler(0) as clk:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(st)
+        for i in range(args.steps):
+            step(evs[i])
+        end.record(st)
+        torch.cuda.synchronize(dev)
+    ms = start.elapsed_time(end) / args.steps
+    names = ("up_quantize", "up_kernel_gemm", "up_main_gemm_gelu", None, "down_quantize", "down_kernel_gemm",
+             "down_main_gemm")
+    stage_ms = {n: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps))
+                for j, n in enumerate(names) if n}
+    Ku, Kd = int(lu.K), int(ld.K)
+    F = layer_flops(up, Ku) + layer_flops(down, Kd)
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16"] * FP4_PER_BF16
+    mu, md = stage_model(up, Ku, lu.slab), stage_model(down, Kd, ld.slab)
+    dom = max(("up_main_gemm_gelu", "down_main_gemm"), key=stage_ms.get)
+    m = mu if dom.startswith("up") else md
+    ach = m["main_gemm"]["flops"] / (stage_ms[dom] * 1e-3) / 1e12
+    line = dict(metric=METRIC, value=F / (ms * 1e-3) / 1e12, unit="TFLOP/s", n_gpus=1, steps=args.steps,
+                warmup=args.warmup, ms_per_step=ms, higher_is_better=True, scaling="weak", vs_baseline=None,
+                dtype="e2m1/e4m3->f32", data="synthetic",
+                config=dict(workload="wan720p_ffn_block" + (f"_T{args.frames}" if args.frames else ""), T=up.T, H=up.H,
+                            W=up.W, N=up.N, Ci=up.Ci, Cf=up.Co, Co=down.Co, rank=[up.rank, down.rank],
+                            cube_up=list(up.cube), cube_down=list(down.cube), activation="GELU (erf form) in the "
+                            "up-projection's main-product epilogue",
+                            down_statistics=("formed in the up-projection's epilogue (the down-projection's "
+                                             "statistics kernel forms X L1 only)" if fused else "separate pass"),
+                            l2="inputs larger than L2"),
+                tokens_per_s=up.N / (ms * 1e-3), stages={n: dict(ms=v) for n, v in stage_ms.items()},
+                roofline=dict(kernel="k_gemm<3> (main FP4 product, feed-forward epilogue)" if dom.startswith("up")
+                              else "k_gemm<1> (main FP4 product)", bound="tensor", achieved=ach, peak=fp4_peak,
+                              unit="TFLOP/s", frac=ach / fp4_peak, traffic=None,
+                              peak_source=peaks["source"] + " bf16 x 4 (nominal FP4:BF16)"),
+                e2e=None, gpu_launches=8 * args.steps)
+    clk_sum = clk.summary()
+    if clk_sum:
+        line["clocks"] = clk_sum
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -309,6 +402,9 @@ def main():
                          "(single-read quantiser)")
     ap.add_argument("--parallelism", default="sharded", choices=["sharded", "replicas"],
                     help="with several GPUs: one layer sharded by cubes (default) or one layer per GPU")
+    ap.add_argument("--ffn", default=None, choices=["fused", "separate"],
+                    help="time the 720p feed-forward block (up-projection + GELU + down-projection) instead, with the "
+                         "down-projection's statistics fused into the up-projection's epilogue or as their own pass")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     args = ap.parse_args()
@@ -323,6 +419,8 @@ def main():
                             wl.w_outliers, wl.gelu)
     if args.impl == "reference":
         return run_reference(args, wl, cube)
+    if args.ffn:
+        return run_ffn(args)
 
     import torch
     import video_diffusion_w4a4_b200 as dq

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define DQ_ABI_VERSION 3
+#define DQ_ABI_VERSION 4
 #define DQ_PACK_FORMAT_VERSION 3
 #define DQ_PACK_MAGIC 0x31575144u /* "DQW1" little-endian */
 
@@ -384,7 +384,13 @@ int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, 
  *                   encode stage also forms the kernel tokens and U' from the stored
  *                   means and partial sums (no read of X apart from re-encoded
  *                   groups).  Per-token kernel scales only.
- *   reserved        must be 0
+ *   epilogue        DQ_EPILOGUE_NONE: Y = BF16(y), y = S_delta S_W acc + P'[k(n)] in fp32.
+ *                   DQ_EPILOGUE_GELU: Y = BF16(GELU(y)), GELU(y) = y Phi(y) =
+ *                   y erfc(-y / sqrt 2) / 2 in fp32 (erfcf), one rounding to BF16:
+ *                   the up-projection of a transformer feed-forward block with its
+ *                   activation in the main product's epilogue (the note's
+ *                   overall pipeline ends in a fused kernel; the activation itself
+ *                   is not on the pages and is taken in its exact erf form).
  * A packed weight whose C2 flag does not match kernel_product is reported as
  * DQ_ERR_BAD_PACKED_WEIGHT in the device status word.
  */
@@ -392,12 +398,14 @@ int dq_linear_forward_grouped(const void* X, int T, int H, int W, int t, int h, 
 #define DQ_KERNEL_PRODUCT_FP8 1
 #define DQ_DELTA_SCALE_AMAX 0
 #define DQ_DELTA_SCALE_POW2 1
+#define DQ_EPILOGUE_NONE 0
+#define DQ_EPILOGUE_GELU 1
 
 typedef struct dq_forward_options {
     int kernel_group;
     int kernel_product;
     int delta_scale;
-    int reserved;
+    int epilogue;
 } dq_forward_options;
 
 int dq_workspace_layout_opts(int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
@@ -408,6 +416,59 @@ int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int
                            const dq_forward_options* opts, const void* packed_W, const void* L1_mma,
                            const void* L2_slab, void* Y, void* workspace, size_t workspace_bytes, int stage_mask,
                            void* const* stage_events, void* stream);
+
+/*
+ * A transformer feed-forward block as two DeltaQuant layers with the producer
+ * step fused (the note's overall pipeline, "fused kernel output"; its
+ * training-strategy section fuses kernel-token generation into the activation
+ * quantisation kernel):
+ *   Hid = BF16(GELU(up(X)))        up:   T x H x W lattice, cube cube_up,   Ci -> Cf
+ *   Y   = down(Hid)                down: the same lattice, cube cube_down, Cf -> Co
+ * Each layer computes exactly what dq_linear_forward_opts computes for it (the
+ * up-projection with DQ_EPILOGUE_GELU, both with the default options); Hid and Y
+ * are bit-identical to those two calls.  The fusion: when every cube_down cube
+ * of the lattice occupies consecutive cube-major rows of the cube_up partition,
+ * in its own (t,h,w) order, inside one aligned group of 32 rows
+ * (dq_ffn_fused_statistics; e.g. cube_down = (1, h, w) inside cube_up =
+ * (t', h, w), or cube_down = cube_up, with at most 32 tokens), the
+ * up-projection's main-product epilogue also forms the down-projection's
+ * statistics pass over the BF16 Hid it writes: the fp32 cube means (K_down x Cf,
+ * the running sum from +0 in (t,h,w) order divided by the count), max |mean| per
+ * cube and max |Hid - mean|.  The down-projection's statistics kernel then only
+ * forms Hid L1_down, one read of Hid fewer per cube statistic.  Otherwise, or with
+ * DQ_FFN_SEPARATE_STATISTICS, the down-projection runs its own statistics pass.
+ *
+ *   X        device, N x Ci BF16, (t,h,w) order; read only
+ *   cube_up, cube_down  host, 3 ints each (t, h, w)
+ *   packed_up, L1_up, L2_up       the up-projection's (Co = Cf, rank_up) weight as
+ *                                  dq_pack_weight makes it (no DQ_PACK_C2)
+ *   packed_down, L1_down, L2_down the down-projection's (Ci = Cf, Co, rank_down)
+ *   Hid      device, N x Cf BF16, (t,h,w) order; written (the hidden activation)
+ *   Y        device, N x Co BF16, (t,h,w) order; written
+ *   ws_up    device workspace of dq_workspace_bytes(T,H,W, cube_up, Ci, Cf, rank_up)
+ *   ws_down  device workspace of dq_workspace_bytes(T,H,W, cube_down, Cf, Co, rank_down)
+ *   ffn_flags      0 or DQ_FFN_SEPARATE_STATISTICS
+ *   stage_events   NULL or 8 cudaEvent_t (as void*): the up-projection's 4 (before its
+ *                  first stage and after each of its three stages) then the
+ *                  down-projection's 4
+ *   stream         the CUDA stream of every launch
+ * All buffers are caller-owned; nothing is allocated.  Errors as
+ * dq_linear_forward_ex (each layer's shape is checked as for that call); device
+ * errors land in each layer's workspace status word (dq_read_device_status).
+ */
+#define DQ_FFN_SEPARATE_STATISTICS 1
+int dq_ffn_forward(const void* X, int T, int H, int W, const int* cube_up, const int* cube_down, int Ci, int Cf,
+                   int Co, int rank_up, int rank_down, const void* packed_up, const void* L1_up, const void* L2_up,
+                   const void* packed_down, const void* L1_down, const void* L2_down, void* Hid, void* Y,
+                   void* ws_up, size_t ws_up_bytes, void* ws_down, size_t ws_down_bytes, int ffn_flags,
+                   void* const* stage_events, void* stream);
+
+/*
+ * *fused = 1 when dq_ffn_forward forms the down-projection's statistics in the
+ * up-projection's epilogue for this lattice and pair of cubes, else 0.  Host
+ * only (no device call); O(T H W) the first time a pair of partitions is asked.
+ */
+int dq_ffn_fused_statistics(int T, int H, int W, const int* cube_up, const int* cube_down, int* fused);
 
 /*
  * As dq_linear_forward_ex with HOST X and Y (pinned for asynchronous copies):

@@ -28,7 +28,7 @@ def test_exports_every_declared_symbol(dq):
     lib = ctypes.CDLL(dq.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
-    assert dq.dq_abi_version() == 3
+    assert dq.dq_abi_version() == 4
 
 
 def test_status_strings(dq):

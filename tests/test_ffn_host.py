@@ -1,0 +1,45 @@
+"""Host logic of the feed-forward block (no GPU): which pairs of cube partitions
+let the up-projection's epilogue form the down-projection's statistics.
+
+dq_ffn_fused_statistics (the library's O(N) check on its own cube-major row map)
+against a statement built on the oracle's cube enumeration: every down cube's
+tokens, in its (t,h,w) order, sit on consecutive rows of the up-projection's
+cube-major order inside one aligned group of 32 rows, and hold at most 32 tokens."""
+import numpy as np
+import pytest
+
+import oracle
+
+
+def _fusable(T, H, W, cu, cd):
+    if int(np.prod(cd)) > 32:
+        return False
+    ou, od = oracle.cube_order(T, H, W, *cu), oracle.cube_order(T, H, W, *cd)
+    for k in range(od["count"].size):
+        f, c = od["first"][k], od["count"][k]
+        ru = ou["row_of_n"][od["n_of_row"][f:f + c]]
+        if not np.array_equal(ru, ru[0] + np.arange(c)) or ru[0] // 32 != ru[-1] // 32:
+            return False
+    return True
+
+
+CASES = [(21, 45, 80, (2, 2, 2), (1, 2, 2)), (3, 5, 12, (2, 2, 2), (1, 2, 2)), (4, 8, 8, (1, 2, 2), (1, 2, 2)),
+         (5, 6, 16, (2, 2, 4), (1, 1, 4)), (3, 7, 9, (1, 1, 1), (1, 1, 1)), (4, 8, 8, (1, 2, 2), (2, 1, 1)),
+         (5, 7, 9, (2, 2, 2), (2, 2, 2)), (5, 7, 9, (1, 2, 2), (1, 1, 2)), (8, 6, 16, (4, 2, 8), (4, 2, 8)),
+         (4, 4, 16, (2, 2, 8), (2, 2, 8)), (6, 16, 24, (2, 2, 2), (1, 2, 2)), (21, 30, 52, (1, 2, 2), (1, 2, 2)),
+         (7, 9, 11, (1, 1, 1), (1, 1, 1)), (6, 8, 8, (2, 4, 4), (1, 4, 4)), (6, 8, 8, (2, 4, 4), (2, 2, 2)),
+         (2, 3, 5, (2, 3, 5), (1, 1, 1))]
+
+
+@pytest.mark.parametrize("T,H,W,cu,cd", CASES)
+def test_fused_statistics_predicate(T, H, W, cu, cd):
+    import video_diffusion_w4a4_b200 as dq
+    assert dq.dq_ffn_fused_statistics(T, H, W, cu, cd) == _fusable(T, H, W, cu, cd)
+
+
+def test_fused_statistics_rejects_bad_arguments():
+    import video_diffusion_w4a4_b200 as dq
+    with pytest.raises(dq.DQError):
+        dq.dq_ffn_fused_statistics(4, 8, 8, (0, 2, 2), (1, 2, 2))
+    with pytest.raises(dq.DQError):
+        dq.dq_ffn_fused_statistics(4, 8, 8, (1, 2, 2), (5, 2, 2))

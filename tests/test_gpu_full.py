@@ -182,3 +182,25 @@ def test_full_size_host_entry_point(env):
     assert dq.dq_read_device_status(ws, st, clear=True) == 0
     for i in range(2):
         assert np.array_equal(Yhs[i].numpy().view(np.uint16), g["Y"]), i
+
+
+def test_full_size_ffn_block(env):
+    """The 720p feed-forward block (up-projection 5120 -> 13824 at cube 2x2x2, GELU,
+    down-projection 13824 -> 5120 at cube 1x2x2) through dq_ffn_forward with the
+    down-projection's statistics formed in the up-projection's epilogue: the hidden
+    activation and Y on sampled rows against the oracle, every quantised tensor of the
+    down-projection (and its cube means) in full and bit-exact, and Hid, Y and the
+    down-projection's tensors bit-identical to the unfused path."""
+    from ffn_case import FfnCase
+    dq, torch = env
+    up, down = synth.WORKLOADS["wan720p_ffn_up"], synth.WORKLOADS["wan720p_ffn_down"]
+    case = FfnCase("wan720p_ffn", up.T, up.H, up.W, up.cube, down.cube, up.Ci, up.Co, down.Co, up.rank, down.rank)
+    assert case.fused_expected(dq)
+    g = case.run_gpu(dq, torch)
+    _, rows = sample_cubes(case.up, case.up.cube, n_cubes=24)
+    info = case.check(g, rows)
+    s = case.run_gpu(dq, torch, ffn_flags=dq.DQ_FFN_SEPARATE_STATISTICS)
+    for key in ("H", "Y", "means", "q8", "s8", "dcodes"):
+        assert np.array_equal(g[key], s[key]), key
+    info.update(rows=int(rows.size), N=case.up.N)
+    _record("ffn_block_720p", info)

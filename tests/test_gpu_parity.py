@@ -400,3 +400,40 @@ def test_quotient_path_matches_ieee_division(env):
     dq, torch = env
     bad, first = dq.dq_selftest_divide(1 << 28, seed=12345, stream=torch.cuda.current_stream())
     assert bad == 0, (bad, first)
+
+
+# ------------------------------------------------------------------ feed-forward block (producer-epilogue fusion)
+
+FFN = [
+    # name, T, H, W, cube_up, cube_down, Ci, Cf, Co, rank_up, rank_down, statistics fused
+    ("ragged_222_122", 3, 5, 12, (2, 2, 2), (1, 2, 2), 256, 512, 256, 32, 32, True),
+    ("same_cube_122", 4, 8, 8, (1, 2, 2), (1, 2, 2), 512, 256, 512, 16, 32, True),
+    ("nested_224_114", 5, 6, 16, (2, 2, 4), (1, 1, 4), 256, 256, 512, 32, 16, True),
+    ("unit_cubes", 3, 7, 9, (1, 1, 1), (1, 1, 1), 256, 512, 256, 32, 32, True),
+    ("cube_32_tokens", 4, 4, 16, (2, 2, 8), (2, 2, 8), 256, 256, 256, 16, 16, True),
+    ("multi_tile", 6, 16, 24, (2, 2, 2), (1, 2, 2), 512, 1024, 512, 32, 32, True),
+    # partitions the epilogue cannot serve: the down-projection runs its own statistics pass
+    ("not_nested", 4, 8, 8, (1, 2, 2), (2, 1, 1), 256, 256, 256, 32, 32, False),
+    ("straddling", 5, 7, 9, (2, 2, 2), (2, 2, 2), 256, 256, 256, 16, 16, False),
+    ("cube_64_tokens", 8, 6, 16, (4, 2, 8), (4, 2, 8), 256, 256, 256, 16, 16, False),
+]
+
+
+@pytest.mark.parametrize("name,T,H,W,cu,cd,Ci,Cf,Co,ru,rd,fused", FFN, ids=[c[0] for c in FFN])
+def test_parity_ffn_block(env, name, T, H, W, cu, cd, Ci, Cf, Co, ru, rd, fused):
+    """dq_ffn_forward against the oracle: the hidden activation within the GELU-carried
+    tolerance; the down-projection's cube means (formed in the up-projection's epilogue
+    when `fused`), its quantised tensors bit for bit and its Y within tolerance; and
+    the same Hid and Y bits as the unfused path and as the up-projection alone with
+    the GELU epilogue."""
+    from ffn_case import FfnCase
+    dq, torch = env
+    case = FfnCase(name, T, H, W, cu, cd, Ci, Cf, Co, ru, rd)
+    assert case.fused_expected(dq) == fused
+    g = case.run_gpu(dq, torch, gelu_layer=True)
+    case.check(g)
+    assert np.array_equal(g["H"], g["H_layer"]), "the GELU epilogue of the layer alone"
+    s = case.run_gpu(dq, torch, ffn_flags=dq.DQ_FFN_SEPARATE_STATISTICS)
+    assert s["status"] == 0 and s["status_up"] == 0
+    for key in ("H", "Y", "means", "q8", "s8", "dcodes"):
+        assert np.array_equal(g[key], s[key]), key

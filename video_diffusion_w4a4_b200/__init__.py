@@ -41,6 +41,8 @@ DQ_PACK_C2 = 1
 DQ_KERNEL_PRODUCT_BF16, DQ_KERNEL_PRODUCT_FP8 = 0, 1
 DQ_DELTA_SCALE_AMAX, DQ_DELTA_SCALE_POW2 = 0, 1
 DQ_HOST_OVERLAP_PREVIOUS = 1
+DQ_EPILOGUE_NONE, DQ_EPILOGUE_GELU = 0, 1
+DQ_FFN_SEPARATE_STATISTICS = 1
 
 
 class dq_packed_layout(ctypes.Structure):
@@ -59,7 +61,7 @@ class dq_workspace_layout(ctypes.Structure):
 
 class dq_forward_options(ctypes.Structure):
     _fields_ = [("kernel_group", ctypes.c_int), ("kernel_product", ctypes.c_int), ("delta_scale", ctypes.c_int),
-                ("reserved", ctypes.c_int)]
+                ("epilogue", ctypes.c_int)]
 
 
 _P, _I, _SZ, _LL = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong
@@ -98,6 +100,8 @@ _SIGS = {
     "dq_linear_forward_host_ex": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P, _P, _P, _SZ, _I, _P], _I),
     "dq_linear_forward_noalloc": ([_P] + [_I] * 9 + [_P, _P, _P, _P, _P], _I),
     "dq_read_device_status": ([_P, _P, ctypes.POINTER(_I), _I], _I),
+    "dq_ffn_forward": ([_P, _I, _I, _I, _P, _P] + [_I] * 5 + [_P] * 8 + [_P, _SZ, _P, _SZ, _I, _P, _P], _I),
+    "dq_ffn_fused_statistics": ([_I, _I, _I, _P, _P, ctypes.POINTER(_I)], _I),
     "dq_selftest_bounded_wait": ([_I, _P, ctypes.POINTER(_I)], _I),
     "dq_selftest_convert": ([_P, _LL, _P, _P, _P, _P], _I),
     "dq_selftest_divide": ([_LL, ctypes.c_uint64, ctypes.POINTER(ctypes.c_ulonglong), _P, _P], _I),
@@ -288,9 +292,9 @@ def dq_workspace_layout_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group) ->
 
 
 def _options(kernel_group=DQ_KERNEL_SCALE_PER_TOKEN, kernel_product=DQ_KERNEL_PRODUCT_BF16,
-             delta_scale=DQ_DELTA_SCALE_AMAX):
+             delta_scale=DQ_DELTA_SCALE_AMAX, epilogue=DQ_EPILOGUE_NONE):
     o = dq_forward_options()
-    o.kernel_group, o.kernel_product, o.delta_scale = kernel_group, kernel_product, delta_scale
+    o.kernel_group, o.kernel_product, o.delta_scale, o.epilogue = kernel_group, kernel_product, delta_scale, epilogue
     return o
 
 
@@ -308,13 +312,33 @@ def dq_workspace_layout_opts(T, H, W, t, h, w, Ci, Co, rank, kernel_group=DQ_KER
 def dq_linear_forward_opts(X, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_slab, Y, workspace,
                            workspace_bytes, stage_mask=DQ_STAGE_ALL, stage_events=None, stream=None,
                            kernel_group=DQ_KERNEL_SCALE_PER_TOKEN, kernel_product=DQ_KERNEL_PRODUCT_BF16,
-                           delta_scale=DQ_DELTA_SCALE_AMAX) -> None:
+                           delta_scale=DQ_DELTA_SCALE_AMAX, epilogue=DQ_EPILOGUE_NONE) -> None:
     """dq_linear_forward_ex with forward options (dq_forward_options fields as keywords)."""
-    o = _options(kernel_group, kernel_product, delta_scale)
+    o = _options(kernel_group, kernel_product, delta_scale, epilogue)
     _check("dq_linear_forward_opts",
            _lib.dq_linear_forward_opts(_ptr(X), T, H, W, t, h, w, Ci, Co, rank, ctypes.byref(o), _ptr(packed_W),
                                        _ptr(L1_mma), _ptr(L2_slab), _ptr(Y), _ptr(workspace), workspace_bytes,
                                        stage_mask, _events(stage_events), _stream(stream)))
+
+
+def dq_ffn_fused_statistics(T, H, W, cube_up, cube_down) -> bool:
+    """Whether dq_ffn_forward forms the down-projection's statistics in the up-projection's epilogue."""
+    cu, cd = (ctypes.c_int * 3)(*cube_up), (ctypes.c_int * 3)(*cube_down)
+    f = ctypes.c_int()
+    _check("dq_ffn_fused_statistics", _lib.dq_ffn_fused_statistics(T, H, W, cu, cd, ctypes.byref(f)))
+    return bool(f.value)
+
+
+def dq_ffn_forward(X, T, H, W, cube_up, cube_down, Ci, Cf, Co, rank_up, rank_down, packed_up, L1_up, L2_up,
+                   packed_down, L1_down, L2_down, Hid, Y, ws_up, ws_up_bytes, ws_down, ws_down_bytes, ffn_flags=0,
+                   stage_events=None, stream=None) -> None:
+    """A feed-forward block: Hid = BF16(GELU(up(X))), Y = down(Hid) (include/deltaquant.h)."""
+    cu, cd = (ctypes.c_int * 3)(*cube_up), (ctypes.c_int * 3)(*cube_down)
+    _check("dq_ffn_forward",
+           _lib.dq_ffn_forward(_ptr(X), T, H, W, cu, cd, Ci, Cf, Co, rank_up, rank_down, _ptr(packed_up), _ptr(L1_up),
+                               _ptr(L2_up), _ptr(packed_down), _ptr(L1_down), _ptr(L2_down), _ptr(Hid), _ptr(Y),
+                               _ptr(ws_up), ws_up_bytes, _ptr(ws_down), ws_down_bytes, ffn_flags,
+                               _events(stage_events, 8), _stream(stream)))
 
 
 def dq_workspace_bytes_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group) -> int:
@@ -336,13 +360,13 @@ def dq_linear_forward(X, T, H, W, t, h, w, Ci, Co, rank, packed_W, L1_mma, L2_sl
                                                        _ptr(L1_mma), _ptr(L2_slab), _ptr(Y), _stream(stream)))
 
 
-def _events(stage_events):
+def _events(stage_events, n: int = 4):
     if stage_events is None:
         return None
     handles = [e.cuda_event if hasattr(e, "cuda_event") else e for e in stage_events]
-    if len(handles) != 4 or not all(handles):
-        raise ValueError("stage_events needs 4 created CUDA events (record a torch.cuda.Event once first)")
-    arr = (ctypes.c_void_p * 4)(*handles)
+    if len(handles) != n or not all(handles):
+        raise ValueError(f"stage_events needs {n} created CUDA events (record a torch.cuda.Event once first)")
+    arr = (ctypes.c_void_p * n)(*handles)
     return ctypes.cast(arr, ctypes.c_void_p)
 
 

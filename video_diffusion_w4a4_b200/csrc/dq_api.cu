@@ -147,7 +147,7 @@ int check_options(const dq_forward_options& o) {
     if (o.delta_scale != DQ_DELTA_SCALE_AMAX && o.delta_scale != DQ_DELTA_SCALE_POW2) return DQ_ERR_INVALID_ARG;
     // the single-read quantiser forms per-token kernel scales in its fix-up pass
     if (o.delta_scale == DQ_DELTA_SCALE_POW2 && o.kernel_group != DQ_KERNEL_SCALE_PER_TOKEN) return DQ_ERR_INVALID_ARG;
-    if (o.reserved) return DQ_ERR_INVALID_ARG;
+    if (o.epilogue != DQ_EPILOGUE_NONE && o.epilogue != DQ_EPILOGUE_GELU) return DQ_ERR_INVALID_ARG;
     return DQ_OK;
 }
 
@@ -299,10 +299,54 @@ struct Pipeline {
     std::function<int(int, long long)> after_chunk;
 };
 
+// The two halves of the producer-epilogue fusion of a feed-forward block: the up-projection's main
+// product forms the down-projection's statistics pass (c_means set), and the down-projection's
+// statistics kernel then only forms X L1 (stats_given).
+struct FfnHooks {
+    Geom cg{};
+    float* c_means = nullptr;
+    uint32_t* c_kamax = nullptr;
+    uint32_t* c_scalars = nullptr;
+    bool stats_given = false;
+};
+
+// Whether the down-projection's statistics pass can run in the up-projection's epilogue: every
+// cube of the consumer partition gd must hold at most 32 tokens and occupy consecutive cube-major
+// rows of the producer partition gu, in its own (t,h,w) order, inside one aligned group of 32 rows
+// (the rows one epilogue warp holds).  O(N) on the host; the answer is kept per pair of partitions.
+bool ffn_stats_fusable(const Geom& gu, const Geom& gd) {
+    if ((long long)gd.t * gd.h * gd.w > 32) return false;
+    static std::mutex mu;
+    static std::map<std::vector<int>, bool> memo;
+    const std::vector<int> key = {gu.T, gu.H, gu.W, gu.t, gu.h, gu.w, gd.t, gd.h, gd.w};
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        auto it = memo.find(key);
+        if (it != memo.end()) return it->second;
+    }
+    std::vector<long long> base((size_t)gd.K, -1);
+    bool ok = true;
+    for (long long n = 0; ok && n < gu.N; n++) {
+        long long ru = 0, ku = 0, kd = 0;
+        int pos = 0, cnt = 0;
+        dq::token_to_row(gu, n, &ru, &ku);
+        dq::cube_pos(gd, n, &kd, &pos, &cnt);
+        const long long b = ru - pos;
+        if (base[(size_t)kd] < 0)
+            base[(size_t)kd] = b;
+        else if (base[(size_t)kd] != b)
+            ok = false;
+        if ((b >> 5) != ((b + cnt - 1) >> 5)) ok = false;
+    }
+    std::lock_guard<std::mutex> lk(mu);
+    memo[key] = ok;
+    return ok;
+}
+
 int forward_impl(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
                  const dq_forward_options* opts, const void* packed_W, const void* L1_mma, const void* L2_slab,
                  void* Y, void* workspace, size_t workspace_bytes, int stage_mask, void* const* stage_events,
-                 void* stream, const Pipeline* pipe) {
+                 void* stream, const Pipeline* pipe, const FfnHooks* hk = nullptr) {
     int rc = check_shape(T, H, W, t, h, w, Ci, Co, rank);
     if (rc) return rc;
     const dq_forward_options o = opts ? *opts : dq_forward_options{};
@@ -310,6 +354,8 @@ int forward_impl(const void* X, int T, int H, int W, int t, int h, int w, int Ci
     const int kg = o.kernel_group;
     const bool fp8prod = o.kernel_product == DQ_KERNEL_PRODUCT_FP8;
     const bool pow2 = o.delta_scale == DQ_DELTA_SCALE_POW2;
+    const bool stats_given = hk && hk->stats_given;
+    if (stats_given && (pow2 || (long long)t * h * w > 32)) return DQ_ERR_INVALID_ARG;
     if (!X || !packed_W || !L1_mma || !L2_slab || !Y || !workspace) return DQ_ERR_INVALID_ARG;
     if (stage_mask <= 0 || (stage_mask & ~(DQ_STAGE_ALL | DQ_STAGE_STATS | DQ_STAGE_ENCODE))) return DQ_ERR_INVALID_ARG;
     const bool do_stats = stage_mask & (DQ_STAGE_QUANTIZE | DQ_STAGE_STATS);
@@ -336,6 +382,7 @@ int forward_impl(const void* X, int T, int H, int W, int t, int h, int w, int Ci
     qp.kgroup = kg;
     qp.fp8_product = fp8prod;
     qp.pow2 = pow2;
+    qp.u_only = stats_given;
     qp.chunks_per_split = Ci / 64 / wl.splits;
     qp.big = (long long)t * h * w > 128;
     if (!qp.big) {
@@ -399,10 +446,12 @@ int forward_impl(const void* X, int T, int H, int W, int t, int h, int w, int Ci
         if (!map_means(&tm_m, ws + wl.off_means, Ci, g.K, qp.m_rows)) return map_fail("kernel tokens");
         if (!map_2d(&tm_l1, L1_mma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Ci, rank, 64, rank)) return map_fail("L1");
         cudaError_t e;
-        if (do_stats) {
+        if (do_stats && !stats_given) {
             if ((e0 = cudaMemsetAsync(ws + wl.off_scalars, 0, 16, st)) != cudaSuccess) return cuda_fail(e0, "memset");
             if ((e0 = cudaMemsetAsync(ws + wl.off_kamax, 0, (size_t)g.K * 4, st)) != cudaSuccess)
                 return cuda_fail(e0, "memset");
+        }
+        if (do_stats) {
             if (qp.big && (e = dq::launch_cube_means_big(tm_x, qp, st)) != cudaSuccess)
                 return cuda_fail(e, "k_cube_means_big");
             // one launch over all work items, or one per T-slab (items of boxes in cube layers [kt0, kt1))
@@ -492,13 +541,22 @@ int forward_impl(const void* X, int T, int H, int W, int t, int h, int w, int Ci
         p.tile_group = ((size_t)Co * (Ci / 2) + pl.off_dqw - pl.off_scales > ((size_t)32 << 20)) ? 8 : 1;
         p.p = (const float*)(ws + wl.off_p);
         p.Y = (uint16_t*)Y;
+        // the feed-forward epilogue: GELU, and the consumer's statistics when a fused block asks for them
+        const bool ffn = o.epilogue == DQ_EPILOGUE_GELU;
+        if (ffn && hk && hk->c_means) {
+            p.cg = hk->cg;
+            p.c_means = hk->c_means;
+            p.c_kamax = hk->c_kamax;
+            p.c_scalars = hk->c_scalars;
+        }
         const int nchunk = pipe ? (int)pipe->tile_cuts.size() - 1 : 1;
         for (int c = 0; c < nchunk; c++) {
             if (pipe) {
                 p.tile_m0 = pipe->tile_cuts[c];
                 p.tile_m1 = pipe->tile_cuts[c + 1];
             }
-            cudaError_t e = dq::launch_main_gemm(tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p, st);
+            cudaError_t e = ffn ? dq::launch_main_gemm_ffn(tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p, st)
+                                : dq::launch_main_gemm(tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p, st);
             if (e != cudaSuccess) return cuda_fail(e, "main product");
             if (pipe && (rc = pipe->after_chunk(c, dq::imin(p.tile_m1 * 256, (int)g.N))))
                 return rc;
@@ -511,6 +569,62 @@ int forward_impl(const void* X, int T, int H, int W, int t, int h, int w, int Ci
 }  // namespace
 
 extern "C" {
+
+int dq_ffn_fused_statistics(int T, int H, int W, const int* cube_up, const int* cube_down, int* fused) {
+    if (!cube_up || !cube_down || !fused) return DQ_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; i++)
+        if (cube_up[i] <= 0 || cube_down[i] <= 0) return DQ_ERR_INVALID_ARG;
+    if (T <= 0 || H <= 0 || W <= 0) return DQ_ERR_INVALID_ARG;
+    if (cube_up[0] > T || cube_up[1] > H || cube_up[2] > W || cube_down[0] > T || cube_down[1] > H ||
+        cube_down[2] > W || (long long)T * H * W >= (1ll << 31))
+        return DQ_ERR_UNSUPPORTED_SHAPE;
+    *fused = ffn_stats_fusable(dq::make_geom(T, H, W, cube_up[0], cube_up[1], cube_up[2]),
+                               dq::make_geom(T, H, W, cube_down[0], cube_down[1], cube_down[2]))
+                 ? 1
+                 : 0;
+    return DQ_OK;
+}
+
+int dq_ffn_forward(const void* X, int T, int H, int W, const int* cube_up, const int* cube_down, int Ci, int Cf,
+                   int Co, int rank_up, int rank_down, const void* packed_up, const void* L1_up, const void* L2_up,
+                   const void* packed_down, const void* L1_down, const void* L2_down, void* Hid, void* Y,
+                   void* ws_up, size_t ws_up_bytes, void* ws_down, size_t ws_down_bytes, int ffn_flags,
+                   void* const* stage_events, void* stream) {
+    if (!cube_up || !cube_down || (ffn_flags & ~DQ_FFN_SEPARATE_STATISTICS)) return DQ_ERR_INVALID_ARG;
+    int rc = check_shape(T, H, W, cube_up[0], cube_up[1], cube_up[2], Ci, Cf, rank_up);
+    if (rc) return rc;
+    if ((rc = check_shape(T, H, W, cube_down[0], cube_down[1], cube_down[2], Cf, Co, rank_down))) return rc;
+    if (!X || !Hid || !Y || !ws_up || !ws_down) return DQ_ERR_INVALID_ARG;
+    if (!aligned(ws_down)) return DQ_ERR_ALIGNMENT;
+    const Geom gu = dq::make_geom(T, H, W, cube_up[0], cube_up[1], cube_up[2]);
+    const Geom gd = dq::make_geom(T, H, W, cube_down[0], cube_down[1], cube_down[2]);
+    const dq::WsLayout wd = dq::ws_layout(gd, Cf, Co, rank_down, 0, false, false);
+    if (ws_down_bytes < wd.total) return DQ_ERR_WORKSPACE_TOO_SMALL;
+    const bool fuse = !(ffn_flags & DQ_FFN_SEPARATE_STATISTICS) && ffn_stats_fusable(gu, gd);
+    FfnHooks up, down;
+    if (fuse) {
+        // the up-projection's epilogue takes the maxima of the down-projection's statistics pass
+        cudaStream_t st = (cudaStream_t)stream;
+        uint8_t* wsd = (uint8_t*)ws_down;
+        cudaError_t e;
+        if ((e = cudaMemsetAsync(wsd + wd.off_scalars, 0, 16, st)) != cudaSuccess) return cuda_fail(e, "memset");
+        if ((e = cudaMemsetAsync(wsd + wd.off_kamax, 0, (size_t)gd.K * 4, st)) != cudaSuccess)
+            return cuda_fail(e, "memset");
+        up.cg = gd;
+        up.c_means = (float*)(wsd + wd.off_means);
+        up.c_kamax = (uint32_t*)(wsd + wd.off_kamax);
+        up.c_scalars = (uint32_t*)(wsd + wd.off_scalars);
+        down.stats_given = true;
+    }
+    dq_forward_options ou{};
+    ou.epilogue = DQ_EPILOGUE_GELU;
+    rc = forward_impl(X, T, H, W, cube_up[0], cube_up[1], cube_up[2], Ci, Cf, rank_up, &ou, packed_up, L1_up, L2_up,
+                      Hid, ws_up, ws_up_bytes, DQ_STAGE_ALL, stage_events, stream, nullptr, &up);
+    if (rc) return rc;
+    return forward_impl(Hid, T, H, W, cube_down[0], cube_down[1], cube_down[2], Cf, Co, rank_down, nullptr,
+                        packed_down, L1_down, L2_down, Y, ws_down, ws_down_bytes, DQ_STAGE_ALL,
+                        stage_events ? stage_events + 4 : nullptr, stream, nullptr, &down);
+}
 
 int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
                            const dq_forward_options* opts, const void* packed_W, const void* L1_mma,

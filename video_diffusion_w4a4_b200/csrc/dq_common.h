@@ -80,6 +80,19 @@ DQ_HD void row_to_token(const Geom& g, long long row, long long* n, long long* c
     *cube = ((long long)kt * g.KH + kh) * g.KW + kw;
 }
 
+// Natural token n -> its cube in the partition g, its place in the cube's (t,h,w) order and the
+// cube's token count (edge cubes hold the tokens the lattice leaves them).
+DQ_HD void cube_pos(const Geom& g, long long n, long long* cube, int* pos, int* count) {
+    int ww = (int)(n % g.W);
+    int hh = (int)((n / g.W) % g.H);
+    int tt = (int)(n / ((long long)g.W * g.H));
+    int kt = tt / g.t, kh = hh / g.h, kw = ww / g.w;
+    int st = imin(g.t, g.T - kt * g.t), sh = imin(g.h, g.H - kh * g.h), sw = imin(g.w, g.W - kw * g.w);
+    *pos = ((tt - kt * g.t) * sh + (hh - kh * g.h)) * sw + (ww - kw * g.w);
+    *count = st * sh * sw;
+    *cube = ((long long)kt * g.KH + kh) * g.KW + kw;
+}
+
 // Scale-factor layout (see include/deltaquant.h): byte offset of the scale of
 // 16-column block `blk` in row `row` of a matrix with `cols` columns.
 DQ_HD size_t sf_offset(long long row, int blk, int cols) {

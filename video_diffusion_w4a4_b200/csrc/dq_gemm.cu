@@ -30,7 +30,8 @@
 // the MMAs; warp 2 of the even CTA copies the block scale factors of both CTAs
 // into tensor memory (main product); warps 3-10 of each CTA drain that CTA's
 // accumulator rows, two warps per 32-lane sub-partition, each half of the
-// columns.  The operand copies of both CTAs count on the even CTA's
+// columns (warps 3-18, four per sub-partition and a quarter of the columns
+// each, for the feed-forward epilogue).  The operand copies of both CTAs count on the even CTA's
 // "stage full" barriers; the MMA thread's commits arrive on the "stage empty"
 // and "accumulator full" barriers of both CTAs; the epilogue warps of both
 // CTAs arrive on the even CTA's "accumulator empty" barrier.
@@ -42,6 +43,11 @@
 //       operand's scales are a constant 1 (UE8M0 127) written to tensor memory
 //       once, the B operand's exponents are copied in per 256-channel stage
 //       (two 4 KB copies).
+//
+//   (b') main product with the feed-forward epilogue (kGemmMainFfn, the up-projection of a
+//       transformer feed-forward block): Y = BF16(GELU(y)), and optionally the statistics pass of
+//       the down-projection over that Y (cube means, max |mean| per cube, max |Y - mean|), so that
+//       the down-projection's statistics kernel only forms Y L1.
 //
 // The BF16 kernel-token product double-buffers its accumulator in tensor memory so
 // the epilogue of one tile overlaps the MMAs of the next; the main product
@@ -62,8 +68,10 @@ namespace {
 
 constexpr int kTileM = 128;                     // accumulator rows per CTA (256 per pair)
 constexpr int kTileN = 256;                     // output columns per pair tile
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 96 + 32 * kEpiWarps;   // producer, MMA, scale-factor copies, epilogue
+// Epilogue warps: two per 32-lane sub-partition of tensor memory (128 columns each), four (64 columns
+// each) for the feed-forward epilogue, whose GELU and statistics want more warps to hide their latency.
+__host__ __device__ constexpr int epi_warps(int kind) { return kind == kGemmMainFfn ? 16 : 8; }
+__host__ __device__ constexpr int g_threads(int kind) { return 96 + 32 * epi_warps(kind); }   // + producer, MMA, copies
 constexpr uint32_t kABytes = kTileM * 128;      // 128 rows x 128 bytes
 constexpr uint32_t kBBytes = (kTileN / 2) * 128;  // this CTA's 128 rows of B x 128 bytes
 constexpr uint32_t kSFABytes = 2 * 4096;        // 128 rows x 4 k-blocks of 64, A-operand scale layout
@@ -73,14 +81,16 @@ constexpr uint16_t kPairMask = 0x3;
 constexpr uint32_t kFp8SfaCol = 256;            // FP8 product: tensor-memory columns of the constant A scales
 constexpr uint32_t kFp8SfbCol = 264;            //   and of the first B-exponent slot (16 columns per stage)
 
+__host__ __device__ constexpr bool is_main(int kind) { return kind == kGemmMain || kind == kGemmMainFfn; }
+
 __host__ __device__ constexpr int g_stages(int kind) {
-    return kind == kGemmMain ? 4 : 3;
+    return is_main(kind) ? 4 : 3;
 }
 // Operand tiles per stage: the kernel-token products stage two 128-byte-row boxes of each operand
 // (128 channels of BF16, 256 of FP8; eight MMAs) between barrier hand-offs, measured 6-8 % faster
 // than one box per stage with twice the stages; the main product keeps one (its scale copies and
 // TMEM slots are per box).
-__host__ __device__ constexpr uint32_t stage_mul(int kind) { return kind == kGemmMain ? 1u : 2u; }
+__host__ __device__ constexpr uint32_t stage_mul(int kind) { return is_main(kind) ? 1u : 2u; }
 
 // Output tile -> (row tile, column tile).  group <= 1: row-major, which suits a weight that stays
 // in L2 while the row tiles stream.  Otherwise groups of `group` row tiles walked column by column:
@@ -110,9 +120,9 @@ __host__ __device__ constexpr GSmem g_smem_layout(int kind) {
     L.b = off;
     off += S * kBBytes * stage_mul(kind);
     L.sfa = off;
-    if (kind == kGemmMain) off += S * kSFABytes;
+    if (is_main(kind)) off += S * kSFABytes;
     L.sfb = off;
-    if (kind == kGemmMain) off += S * kSFBBytes;
+    if (is_main(kind)) off += S * kSFBBytes;
     if (kind == kGemmKernelFp8) off += S * 2 * kSFB8Bytes;
     L.bars = off;
     off += (3 * S + 6) * 8;
@@ -123,16 +133,68 @@ __host__ __device__ constexpr GSmem g_smem_layout(int kind) {
 }
 
 
+// Consumer statistics of the feed-forward epilogue (see k_gemm<kGemmMainFfn>) over one warp's 64-column
+// slice, held as 32 BF16 pairs pk per lane (lane = row).  Cubes of S tokens on S aligned consecutive lanes,
+// rows in cube order: lane li of a cube gathers the 32/S pairs li*32/S.. of every row of its cube (S - 1
+// exchange rounds with lane li ^ r, each lane sending the chunk its partner gathers), sums the rows in cube
+// order from +0 (the statistics kernel's order), and keeps max |mean| and max |x - mean| of its columns;
+// `valid` lanes store their 64/S means at mrow (the slice's first column of the cube's row of means).
+template <int S>
+__device__ __forceinline__ void ffn_stats_aligned(const uint32_t (&pk)[32], int li, bool valid, float* mrow,
+                                                  float& kam, float& dmx) {
+    constexpr int W = 32 / S;
+    const float inv = inv_pow2(S);
+    uint32_t mw[8];
+#pragma unroll
+    for (int q = 0; q < W; q++) {
+        uint32_t v[S];   // v[r]: pair li * W + q of the row li ^ r
+#pragma unroll
+        for (int r = 0; r < S; r++) {
+            const int c = li ^ r;
+            uint32_t send = pk[q];
+#pragma unroll
+            for (int cc = 1; cc < S; cc++) send = (c == cc) ? pk[cc * W + q] : send;
+            v[r] = r ? __shfl_xor_sync(0xffffffffu, send, r) : send;
+        }
+        uint64_t s2 = 0ull;   // (+0, +0)
+#pragma unroll
+        for (int j = 0; j < S; j++) {
+            // row j arrived in round li ^ j
+            const int r = li ^ j;
+            uint32_t x = v[0];
+#pragma unroll
+            for (int rr = 1; rr < S; rr++) x = (r == rr) ? v[rr] : x;
+            s2 = f2_add(s2, f2_from_bf16x2(x));
+        }
+        const uint64_t m2 = f2_mul(s2, f2_pack(inv, inv));
+        float m0, m1;
+        f2_unpack(m2, m0, m1);
+        if (valid) {
+            kam = max3_abs(m0, m1, kam);
+#pragma unroll
+            for (int r = 0; r < S; r++) {
+                float d0, d1;
+                f2_unpack(f2_sub(f2_from_bf16x2(v[r]), m2), d0, d1);
+                dmx = max3_abs(d0, d1, dmx);
+            }
+        }
+        mw[(2 * q) & 7] = __float_as_uint(m0);
+        mw[(2 * q + 1) & 7] = __float_as_uint(m1);
+        if ((q & 3) == 3 && valid) st_global_v8(mrow + 2 * li * W + 2 * (q - 3), mw);
+    }
+}
+
 }  // namespace
 
 template <int kKind>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(g_threads(kKind), 1)
     k_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
            const __grid_constant__ CUtensorMap tm_sa, const __grid_constant__ CUtensorMap tm_sb,
            const __grid_constant__ CUtensorMap tm_fa, const __grid_constant__ CUtensorMap tm_fb, GemmParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    constexpr bool kMain = kKind == kGemmMain;
+    constexpr bool kMain = is_main(kKind);          // the main product, with either epilogue
+    constexpr bool kFfn = kKind == kGemmMainFfn;    // its feed-forward epilogue
     constexpr bool kFp8 = kKind == kGemmKernelFp8;
     constexpr bool kScaled = kMain || kFp8;      // block scales copied into tensor memory, one accumulator
     constexpr GSmem L = g_smem_layout(kKind);
@@ -165,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; b++) {
             mbar_init(&accf[b], 1);
-            mbar_init(&acce[b], 2 * kEpiWarps);     // one arrival per epilogue warp of each CTA
+            mbar_init(&acce[b], 2 * epi_warps(kKind));   // one arrival per epilogue warp of each CTA
         }
         mbar_init(drain, 1);
         mbar_init(drain_sf, 1);
@@ -397,6 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue warps (both CTAs)
+        constexpr int kSlice = 256 / (epi_warps(kKind) / 4);   // accumulator columns per epilogue warp
         const int quad = warp & 3, half = (warp - 3) >> 2;
         const float S_W = reinterpret_cast<const PackedHeader*>(p.packed_w)->S_W;
         const float SS = kMain ? __fmul_rn(__uint_as_float(p.scalars[1]), S_W) : 0.f;
@@ -409,9 +472,123 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n0 = rc.n * kTileN;
             const long long rho = (long long)m0 + quad * 32 + lane;
             const bool row_ok = rho < p.M;
-            const int c_base = n0 + half * 128;
-            const uint32_t tacc = tmem + (uint32_t)(buf * 256) + ((uint32_t)(quad * 32) << 16) + (uint32_t)(half * 128);
-            if (kMain) {
+            const int c_base = n0 + half * kSlice;
+            const uint32_t tacc = tmem + (uint32_t)(buf * 256) + ((uint32_t)(quad * 32) << 16) + (uint32_t)(half * kSlice);
+            if (kFfn) {
+                // Feed-forward epilogue: Y = BF16(GELU(S_delta S_W acc + P')).  With c_means set, the
+                // statistics pass of the consumer layer runs here over these BF16 values: per cube of
+                // its partition the fp32 running sum from +0 in (t,h,w) order and the mean (as the
+                // statistics kernel forms them), max |mean| over the channels, and max |Y - mean|.
+                // Every consumer cube's rows are consecutive rows of one 32-row group (the host checks
+                // this before it asks for the statistics), so the lanes of a cube form its sums from
+                // one another's values by shuffles, each of them the same sums in the same order.
+                const bool cst = p.c_means != nullptr;
+                long long n = 0, k = 0, kc = 0;
+                int c_first = lane, c_size = 0;
+                if (row_ok) {
+                    row_to_token(p.g, rho, &n, &k);
+                    if (cst) {
+                        int pos = 0;
+                        cube_pos(p.cg, n, &kc, &pos, &c_size);
+                        c_first = lane - pos;
+                    }
+                }
+                const int c_span = (int)__reduce_max_sync(0xffffffffu, (uint32_t)c_size);
+                const bool ok = __all_sync(0xffffffffu, mbar_wait_spin(&accf[buf], (uint32_t)use & 1, abort_flag,
+                                                                  p.status, p.budget_ns));
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t acc[kSlice];
+#pragma unroll
+                for (int c = 0; c < kSlice; c += 16)
+                    tmem_ld_x16(tacc + (uint32_t)c, *reinterpret_cast<uint32_t(*)[16]>(&acc[c]));
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(acce0 + (uint32_t)(buf * 8));
+                const float* prow = p.p + (size_t)k * p.Nout + c_base;
+                uint16_t* yrow = p.Y + (size_t)n * p.Nout + c_base;
+                float* mrow = cst ? p.c_means + (size_t)kc * p.Nout + c_base : nullptr;
+                const bool writer = cst && row_ok && lane == c_first;   // stores the cube's means
+                float kam = 0.f, dmx = 0.f;
+                // y = S_delta S_W acc + P' in place over the whole slice first (the P' loads of all pieces
+                // in flight together), then GELU, the BF16 rounding and the statistics piece by piece
+                if (row_ok) {
+#pragma unroll
+                    for (int c = 0; c < kSlice; c += 8) {
+                        float pv[8];
+                        ld_global_nc_v8(prow + c, pv);
+#pragma unroll
+                        for (int e = 0; e < 8; e++)
+                            acc[c + e] = __float_as_uint(fmaf(SS, __uint_as_float(acc[c + e]), pv[e]));
+                    }
+                }
+                static_assert(!kFfn || kSlice == 64, "the feed-forward epilogue takes 64-column slices");
+                uint32_t pk[32];   // the slice as BF16 pairs
+#pragma unroll
+                for (int v = 0; v < 32; v++) {
+                    float h0, h1;
+                    f2_unpack(gelu_erf2(f2_pack(__uint_as_float(acc[2 * v]), __uint_as_float(acc[2 * v + 1]))), h0,
+                              h1);
+                    pk[v] = bf16x2_rn(h0, h1);
+                }
+                if (row_ok) {
+#pragma unroll
+                    for (int c = 0; c < 4; c++) st_global_v8(yrow + 16 * c, *reinterpret_cast<const uint32_t(*)[8]>(&pk[8 * c]));
+                }
+                // statistics: the transposed form when every cube of the warp holds 2 or 4 tokens on aligned
+                // lanes (the 720p feed-forward block's down-projection cubes), else one shuffle per row and pair
+                const int aligned = cst ? (int)__reduce_min_sync(
+                                              0xffffffffu, (uint32_t)(!row_ok ? 7 : (c_first == (lane & ~(c_size - 1)) &&
+                                                                                      (c_size == 2 || c_size == 4))
+                                                                                         ? c_size
+                                                                                         : 0))
+                                        : 0;
+                const int span_all = cst ? (int)__reduce_max_sync(0xffffffffu, (uint32_t)(row_ok ? c_size : 0)) : 0;
+                if (cst && aligned != 0 && aligned != 7 && aligned == span_all) {
+                    float* mchunk = mrow;   // this cube's row of means at the slice's first column
+                    if (aligned == 4)
+                        ffn_stats_aligned<4>(pk, lane & 3, row_ok, mchunk, kam, dmx);
+                    else
+                        ffn_stats_aligned<2>(pk, lane & 1, row_ok, mchunk, kam, dmx);
+                    // the cube's max |mean| over the lanes that hold its columns, to its first lane
+                    kam = fmaxf(kam, __shfl_xor_sync(0xffffffffu, kam, 1));
+                    if (aligned == 4) kam = fmaxf(kam, __shfl_xor_sync(0xffffffffu, kam, 2));
+                } else if (cst) {
+#pragma unroll
+                    for (int c = 0; c < kSlice; c += 16) {
+                        uint32_t mw[8];
+#pragma unroll
+                        for (int j = 0; j < 8; j++) {
+                            const uint32_t w = pk[c / 2 + j];
+                            uint64_t s2 = 0ull;   // (+0, +0)
+                            for (int i = 0; i < c_span; i++) {
+                                const uint32_t o = __shfl_sync(0xffffffffu, w, (c_first + i) & 31);
+                                if (i < c_size) s2 = f2_add(s2, f2_from_bf16x2(o));
+                            }
+                            float s0, s1, m0 = 0.f, m1 = 0.f;
+                            f2_unpack(s2, s0, s1);
+                            if (c_size > 0) {
+                                m0 = mean_of_sum(s0, c_size);
+                                m1 = mean_of_sum(s1, c_size);
+                                float d0, d1;
+                                f2_unpack(f2_sub(f2_from_bf16x2(w), f2_pack(m0, m1)), d0, d1);
+                                kam = max3_abs(m0, m1, kam);
+                                dmx = max3_abs(d0, d1, dmx);
+                            }
+                            mw[(2 * j) & 7] = __float_as_uint(m0);
+                            mw[(2 * j + 1) & 7] = __float_as_uint(m1);
+                            if ((j & 3) == 3 && writer) st_global_v8(mrow + c + 8 * (j >> 2), mw);
+                        }
+                    }
+                }
+                if (cst) {
+                    if (writer) atomicMax(&p.c_kamax[kc], __float_as_uint(kam));
+                    // non-negative floats order as their bit patterns
+                    const uint32_t wd = __reduce_max_sync(0xffffffffu, __float_as_uint(dmx));
+                    if (lane == 0) atomicMax(&p.c_scalars[0], wd);
+                }
+            } else if (kMain) {
                 // Pull this warp's 128-column slice of the accumulator into registers and
                 // release tensor memory at once, so the next tile's MMAs start while this
                 // tile's P' rows are fetched and its Y rows are written.
@@ -567,7 +744,7 @@ cudaError_t launch_pairs(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(g_threads(kKind));
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = attr;
@@ -609,6 +786,12 @@ cudaError_t launch_main_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, c
                              const CUtensorMap& tm_sb, const CUtensorMap& tm_fa, const CUtensorMap& tm_fb,
                              const GemmParams& p, cudaStream_t st) {
     return launch_pairs<kGemmMain>(tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p, st);
+}
+
+cudaError_t launch_main_gemm_ffn(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_sa,
+                                 const CUtensorMap& tm_sb, const CUtensorMap& tm_fa, const CUtensorMap& tm_fb,
+                                 const GemmParams& p, cudaStream_t st) {
+    return launch_pairs<kGemmMainFfn>(tm_a, tm_b, tm_sa, tm_sb, tm_fa, tm_fb, p, st);
 }
 
 }  // namespace dq

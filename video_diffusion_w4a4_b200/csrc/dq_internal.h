@@ -23,6 +23,8 @@ struct QuantParams {
     int kgroup;         // 0: s8 per kernel token (K); 64: per 64 channels (K x Ci/64), q8_bf16 = [hi | lo]
     int fp8_product;    // the kernel-token product reads q8 (C2 weights): no q8_bf16, packed weight must be C2
     int pow2;           // single-read quantiser: power-of-two S_delta, provisional per-chunk scales, fix-up pass
+    int u_only;         // statistics kernel: X L1 partial sums only; the cube means, kamax and scalars[0]
+                        //   are already in the workspace (a producer's epilogue formed them)
     int8_t* prov;       //   N x Ci/64 provisional scale exponents (-128: a chunk whose deltas are all zero)
     int big;            // cubes of more than 128 tokens: boxes are row segments of one cube,
     int nseg;           //   nseg segments of up to 128 tokens per cube row; the kernel tokens
@@ -58,13 +60,23 @@ struct GemmParams {
     float* pout;         // kernel-token product output, K x Co fp32
     const float* bias;   // Co fp32 bias section of the packed weight (read when its flag is set)
     uint16_t* Y;         // main product output, N x Co BF16 (t,h,w) order
+    // feed-forward epilogue (kGemmMainFfn): Y = BF16(GELU(y)); with c_means set, also the statistics
+    // pass of the consumer layer over that Y, for its cube partition cg of the same lattice: the fp32
+    // cube means (K_c x Co), max |mean| per cube (atomic max into c_kamax) and max |Y - mean| (atomic
+    // max into c_scalars[0]); every consumer cube's rows are consecutive rows of one 32-row group here
+    Geom cg;
+    float* c_means;
+    uint32_t* c_kamax;
+    uint32_t* c_scalars;
     int* status;
     uint64_t budget_ns;
 };
 
 // Paired-GEMM kinds: the exact kernel-token product (BF16, kind::f16), the main block-scaled FP4
 // product, the FP8 kernel-token product on C2 weights (kind::mxf8f6f4, UE8M0 scales per 32).
-enum GemmKind { kGemmKernelBf16 = 0, kGemmMain = 1, kGemmKernelFp8 = 2 };
+// The main product with the feed-forward epilogue (GELU, consumer statistics) is a kind of its own
+// so that the plain main product keeps its registers.
+enum GemmKind { kGemmKernelBf16 = 0, kGemmMain = 1, kGemmKernelFp8 = 2, kGemmMainFfn = 3 };
 
 size_t quant_smem_bytes(int rank, bool stats, int m_rows, int x_rows);
 cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,
@@ -85,6 +97,10 @@ cudaError_t launch_kernel_gemm_fp8(const CUtensorMap& tm_a, const CUtensorMap& t
 cudaError_t launch_main_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_sa,
                              const CUtensorMap& tm_sb, const CUtensorMap& tm_fa, const CUtensorMap& tm_fb,
                              const GemmParams& p, cudaStream_t st);
+// the main product with the feed-forward epilogue (kGemmMainFfn)
+cudaError_t launch_main_gemm_ffn(const CUtensorMap& tm_a, const CUtensorMap& tm_b, const CUtensorMap& tm_sa,
+                                 const CUtensorMap& tm_sb, const CUtensorMap& tm_fa, const CUtensorMap& tm_fb,
+                                 const GemmParams& p, cudaStream_t st);
 
 // Device address of the no-allocation entry point's fixed workspace on the
 // current device (dq_noalloc.cu); a dq_status code.

@@ -562,6 +562,58 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
     return r;
 }
 
+// 1 / cnt for a power of two cnt (exact)
+__device__ __forceinline__ float inv_pow2(int cnt) { return __int_as_float((127 - (31 - __clz(cnt))) << 23); }
+
+// The cube mean from its fp32 running sum (Eq. 1): the sum divided by the token count, the
+// division being an exact multiplication when the count is a power of two.
+__device__ __forceinline__ float mean_of_sum(float s, int cnt) {
+    return (cnt & (cnt - 1)) == 0 ? __fmul_rn(s, inv_pow2(cnt)) : __fdiv_rn(s, (float)cnt);
+}
+
+// GELU(y) = y Phi(y), Phi(y) = 1 - erfc(y / sqrt 2) / 2 for y >= 0 and erfc(-y / sqrt 2) / 2 for y < 0, with
+// erfc(x) = t (a1 + a2 t + a3 t^2 + a4 t^3 + a5 t^4) exp(-x^2), t = 1 / (1 + p x), x >= 0: the rational
+// approximation of Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26 (absolute error
+// at most 1.5e-7), in fp32 with the hardware's approximate reciprocal and base-2 exponential:
+// |GELU error| <= 3e-7 max(1, |y|), far below the BF16 rounding of the result.  Two values at once in
+// packed f32x2 arithmetic.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t gelu_erf2(uint64_t y2) {
+    float y0, y1, d0, d1, q0, q1, a0, a1, b0, b1;
+    f2_unpack(y2, y0, y1);
+    const uint64_t x2 = f2_mul(f2_pack(fabsf(y0), fabsf(y1)), f2_pack(0.70710678118654752f, 0.70710678118654752f));
+    f2_unpack(f2_fma(f2_pack(0.3275911f, 0.3275911f), x2, f2_pack(1.0f, 1.0f)), d0, d1);
+    const uint64_t t2 = f2_pack(rcp_approx(d0), rcp_approx(d1));
+    uint64_t P = f2_fma(f2_pack(1.061405429f, 1.061405429f), t2, f2_pack(-1.453152027f, -1.453152027f));
+    P = f2_fma(P, t2, f2_pack(1.421413741f, 1.421413741f));
+    P = f2_fma(P, t2, f2_pack(-0.284496736f, -0.284496736f));
+    P = f2_fma(P, t2, f2_pack(0.254829592f, 0.254829592f));
+    // exp(-x^2) = 2^(-x^2 log2 e)
+    f2_unpack(f2_mul(f2_mul(x2, x2), f2_pack(-1.4426950408889634f, -1.4426950408889634f)), q0, q1);
+    const uint64_t e2 = f2_mul(f2_mul(t2, P), f2_pack(ex2_approx(q0), ex2_approx(q1)));   // erfc(x)
+    f2_unpack(f2_fma(f2_pack(-0.5f, -0.5f), e2, f2_pack(1.0f, 1.0f)), a0, a1);             // 1 - erfc / 2
+    f2_unpack(f2_mul(f2_pack(0.5f, 0.5f), e2), b0, b1);                                      // erfc / 2
+    return f2_mul(y2, f2_pack(y0 >= 0.f ? a0 : b0, y1 >= 0.f ? a1 : b1));
+}
+
+// Two fp32 -> BF16 (round to nearest even) in one word, the first in the low half.
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 

@@ -236,9 +236,6 @@ __device__ __forceinline__ float pow2_ceil(float v, int* exp2) {
     return (m == 0.5f) ? v : ldexpf(1.0f, e);
 }
 
-// 1 / cnt for a power of two cnt, exactly (the exponent field of 2^-log2(cnt))
-__device__ __forceinline__ float inv_pow2(int cnt) { return __int_as_float((127 - (31 - __clz(cnt))) << 23); }
-
 __device__ __forceinline__ void mean_from_sum(const uint64_t (&acc)[4], int cnt, uint64_t (&m)[4]) {
     if ((cnt & (cnt - 1)) == 0) {
         const float inv = inv_pow2(cnt);
@@ -562,7 +559,9 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                 const int par = (int)(g & 1);
                 float* mts = (float*)(sm + L.ms + (uint32_t)par * L.ms_stride);   // kSingle: this chunk's means
                 float dch = 0.f;                                                 // this chunk's max |delta|
-                if (kPairs) {
+                if (!kSingle && p.u_only) {
+                    // the statistics are in the workspace already: only X L1 (issued by the MMA warp)
+                } else if (kPairs) {
                     // cubes of 16 or more tokens (at most 8 per box): warp = cube slot, lane = channel
                     // pair (2 lane, 2 lane + 1)
                     const bool mine = grp < ngrp && phase == grp;
@@ -604,7 +603,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                 }
 #pragma unroll
                 for (int t = 0; t < 4; t++) {
-                    if (kPairs || t >= ntask) break;
+                    if (kPairs || t >= ntask || (!kSingle && p.u_only)) break;
                     const StatTask T = t == 0 ? T0 : stat_task(p, R, tid + kQCompute * t);
                     if (!T.valid) continue;
                     uint64_t m[4];
@@ -722,7 +721,9 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
             // per-cube max |mean| over this item's channels -> kamax (small cubes; the means
             // kernel has done it for big ones); the eight threads of a cube are consecutive lanes,
             // or a whole warp in the channel-pair mode
-            if (kPairs) {
+            if (!kSingle && p.u_only) {
+                // kamax is in the workspace already
+            } else if (kPairs) {
                 const float v = warp_max(kam[0]);
                 if (lane == 0 && grp < ngrp) atomicMax(&p.kamax[R.k0 + u_pair], __float_as_uint(v));
             } else if (!p.big) {
@@ -768,7 +769,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
         float wm = warp_max(damax);
         if (lane == 0) red[warp] = wm;
         bar_sync(1, kQCompute);
-        if (tid == 0) {
+        if (tid == 0 && (kSingle || !p.u_only)) {
             float bm = 0.f;
             for (int w = 0; w < kQWarps; w++) bm = fmaxf(bm, red[w]);
             atomicMax(&p.scalars[0], __float_as_uint(bm));
