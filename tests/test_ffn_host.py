@@ -43,3 +43,34 @@ def test_fused_statistics_rejects_bad_arguments():
         dq.dq_ffn_fused_statistics(4, 8, 8, (0, 2, 2), (1, 2, 2))
     with pytest.raises(dq.DQError):
         dq.dq_ffn_fused_statistics(4, 8, 8, (1, 2, 2), (5, 2, 2))
+
+
+def test_ffn_forward_argument_errors():
+    """dq_ffn_forward's argument checks, which run before any device call: flags, cubes,
+    each layer's shape, and the down-projection's workspace size."""
+    import ctypes
+
+    import video_diffusion_w4a4_b200 as dq
+    T, H, W, cu, cd = 4, 8, 8, (2, 2, 2), (1, 2, 2)
+    Ci, Cf, Co, r = 256, 512, 256, 32
+    fake = 1 << 20   # a 256-byte-aligned stand-in address; nothing is dereferenced on these paths
+    ld = dq.dq_workspace_layout_opts(T, H, W, *cd, Cf, Co, r)
+
+    def call(flags=0, cube_up=cu, Ci_=Ci, rank_down=r, ws_down_bytes=ld.total_bytes):
+        a3 = lambda c: (ctypes.c_int * 3)(*c)
+        return dq._lib.dq_ffn_forward(fake, T, H, W, a3(cube_up), a3(cd), Ci_, Cf, Co, r, rank_down, fake, fake,
+                                      fake, fake, fake, fake, fake, fake, fake, 1 << 30, fake, ws_down_bytes, flags,
+                                      None, None)
+
+    assert call(flags=2) == dq.DQ_ERR_INVALID_ARG
+    assert call(cube_up=(0, 2, 2)) == dq.DQ_ERR_INVALID_ARG
+    assert call(Ci_=300) == dq.DQ_ERR_UNSUPPORTED_SHAPE
+    assert call(rank_down=8) == dq.DQ_ERR_UNSUPPORTED_SHAPE
+    assert call(ws_down_bytes=ld.total_bytes - 1) == dq.DQ_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_epilogue_option_is_checked():
+    import video_diffusion_w4a4_b200 as dq
+    dq.dq_workspace_layout_opts(4, 8, 8, 1, 2, 2, 256, 256, 16, epilogue=dq.DQ_EPILOGUE_GELU)
+    with pytest.raises(dq.DQError):
+        dq.dq_workspace_layout_opts(4, 8, 8, 1, 2, 2, 256, 256, 16, epilogue=2)

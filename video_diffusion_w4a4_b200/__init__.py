@@ -299,11 +299,11 @@ def _options(kernel_group=DQ_KERNEL_SCALE_PER_TOKEN, kernel_product=DQ_KERNEL_PR
 
 
 def dq_workspace_layout_opts(T, H, W, t, h, w, Ci, Co, rank, kernel_group=DQ_KERNEL_SCALE_PER_TOKEN,
-                             kernel_product=DQ_KERNEL_PRODUCT_BF16,
-                             delta_scale=DQ_DELTA_SCALE_AMAX) -> dq_workspace_layout:
+                             kernel_product=DQ_KERNEL_PRODUCT_BF16, delta_scale=DQ_DELTA_SCALE_AMAX,
+                             epilogue=DQ_EPILOGUE_NONE) -> dq_workspace_layout:
     """Workspace carve-up for the forward options (dq_forward_options fields as keywords)."""
     L = dq_workspace_layout()
-    o = _options(kernel_group, kernel_product, delta_scale)
+    o = _options(kernel_group, kernel_product, delta_scale, epilogue)
     _check("dq_workspace_layout_opts", _lib.dq_workspace_layout_opts(T, H, W, t, h, w, Ci, Co, rank, ctypes.byref(o),
                                                                      ctypes.byref(L)))
     return L
