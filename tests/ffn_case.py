@@ -24,7 +24,7 @@ def h_tolerance(y_ref: np.ndarray, h_ref: np.ndarray) -> np.ndarray:
 
 
 class FfnCase:
-    def __init__(self, name, T, H, W, cube_up, cube_down, Ci, Cf, Co, r_up, r_down, seed=0x0FF0):
+    def __init__(self, name, T, H, W, cube_up, cube_down, Ci, Cf, Co, r_up, r_down, seed=0x0FF0, bias=False):
         grid = (T, max(1, -(-H // 4)), max(1, -(-W // 4)))
         self.up = synth.Workload(name + "_up", T, H, W, Ci, Cf, r_up, tuple(cube_up), grid, (0.01, 50.0),
                                  (0.01, 20.0))
@@ -35,6 +35,9 @@ class FfnCase:
         self.Wd = synth.weight(self.down, seed=seed + 1)
         self.L1u, self.L2u, _ = oracle.lowrank_factors(self.Wu, r_up)
         self.L1d, self.L2d, _ = oracle.lowrank_factors(self.Wd, r_down)
+        # optional linear biases of both layers (BF16 bits)
+        self.bu = synth.normal_bf16((Cf,), 0.5, seed, 7) if bias else None
+        self.bd = synth.normal_bf16((Co,), 0.5, seed, 8) if bias else None
         self.packed = None
 
     def fused_expected(self, dq) -> bool:
@@ -48,6 +51,9 @@ class FfnCase:
         if self.packed is None:
             pu, L1mu, L2su, _ = dq.dq_pack_weight_factors(self.Wu, self.L1u, self.L2u)
             pd, L1md, L2sd, S_Wd = dq.dq_pack_weight_factors(self.Wd, self.L1d, self.L2d)
+            if self.bu is not None:
+                dq.dq_pack_bias(pu, self.bu)
+                dq.dq_pack_bias(pd, self.bd)
             self.packed = (pu, L1mu, L2su, pd, L1md, L2sd, S_Wd)
         pu, L1mu, L2su, pd, L1md, L2sd, S_Wd = self.packed
         dev = torch.device("cuda")
@@ -95,8 +101,8 @@ class FfnCase:
         rows = np.arange(u.N) if rows is None else rows
         act_u = oracle.quantize_activations(self.X, u.T, u.H, u.W, u.cube)
         wq_u = oracle.quantize_weight(self.Wu, self.L1u, self.L2u)
-        y_ref = oracle.output_rows(act_u, wq_u, self.X, self.L1u, self.L2u, rows)
-        h_ref = oracle.ffn_hidden_rows(act_u, wq_u, self.X, self.L1u, self.L2u, rows)
+        y_ref = oracle.output_rows(act_u, wq_u, self.X, self.L1u, self.L2u, rows, bias=self.bu)
+        h_ref = oracle.ffn_hidden_rows(act_u, wq_u, self.X, self.L1u, self.L2u, rows, bias=self.bu)
         h = bf16_bits_to_f64(g["H"][rows])
         tol = h_tolerance(y_ref, h_ref)
         err = np.abs(h - h_ref)
@@ -108,6 +114,7 @@ class FfnCase:
         bad = np.argwhere(g["means"] != means.view(np.uint32))
         assert bad.size == 0, ("cube means", bad[:5].tolist())
         compare_quantised(g, act_d, wq_d)
-        info = assert_y_close(g["Y"][rows], oracle.output_rows(act_d, wq_d, g["H"], self.L1d, self.L2d, rows))
+        info = assert_y_close(g["Y"][rows], oracle.output_rows(act_d, wq_d, g["H"], self.L1d, self.L2d, rows,
+                                                               bias=self.bd))
         info.update(hidden_max_err_over_tol=float((err / tol).max()))
         return info

@@ -437,3 +437,14 @@ def test_parity_ffn_block(env, name, T, H, W, cu, cd, Ci, Cf, Co, ru, rd, fused)
     assert s["status"] == 0 and s["status_up"] == 0
     for key in ("H", "Y", "means", "q8", "s8", "dcodes"):
         assert np.array_equal(g[key], s[key]), key
+
+
+def test_parity_ffn_block_with_biases(env):
+    """The feed-forward block with a linear bias in both layers (added once per cube in
+    each layer's kernel term, so GELU sees y + b)."""
+    from ffn_case import FfnCase
+    dq, torch = env
+    case = FfnCase("bias_222_122", 3, 6, 16, (2, 2, 2), (1, 2, 2), 256, 512, 256, 32, 16, bias=True)
+    assert case.fused_expected(dq)
+    g = case.run_gpu(dq, torch)
+    case.check(g)
