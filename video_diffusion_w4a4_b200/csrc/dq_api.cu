@@ -382,7 +382,6 @@ int forward_impl(const void* X, int T, int H, int W, int t, int h, int w, int Ci
     qp.kgroup = kg;
     qp.fp8_product = fp8prod;
     qp.pow2 = pow2;
-    qp.u_only = stats_given;
     qp.chunks_per_split = Ci / 64 / wl.splits;
     qp.big = (long long)t * h * w > 128;
     if (!qp.big) {
@@ -451,7 +450,9 @@ int forward_impl(const void* X, int T, int H, int W, int t, int h, int w, int Ci
             if ((e0 = cudaMemsetAsync(ws + wl.off_kamax, 0, (size_t)g.K * 4, st)) != cudaSuccess)
                 return cuda_fail(e0, "memset");
         }
-        if (do_stats) {
+        // with the statistics given (a producer's epilogue formed them) no statistics pass runs: the
+        // encode pass also forms X L1
+        if (do_stats && !stats_given) {
             if (qp.big && (e = dq::launch_cube_means_big(tm_x, qp, st)) != cudaSuccess)
                 return cuda_fail(e, "k_cube_means_big");
             // one launch over all work items, or one per T-slab (items of boxes in cube layers [kt0, kt1))
@@ -474,6 +475,9 @@ int forward_impl(const void* X, int T, int H, int W, int t, int h, int w, int Ci
         }
         if (do_encode && pow2) {
             if ((e = dq::launch_single_finish(X, qp, st)) != cudaSuccess) return cuda_fail(e, "k_single_finish");
+        } else if (do_encode && stats_given) {
+            if ((e = dq::launch_cube_encode_lowrank(tm_x, tm_m, tm_l1, qp, st)) != cudaSuccess)
+                return cuda_fail(e, "k_cube_encode (with X L1)");
         } else if (do_encode && (e = dq::launch_cube_encode(tm_x, tm_m, qp, st)) != cudaSuccess) {
             return cuda_fail(e, "k_cube_encode");
         }

@@ -23,8 +23,6 @@ struct QuantParams {
     int kgroup;         // 0: s8 per kernel token (K); 64: per 64 channels (K x Ci/64), q8_bf16 = [hi | lo]
     int fp8_product;    // the kernel-token product reads q8 (C2 weights): no q8_bf16, packed weight must be C2
     int pow2;           // single-read quantiser: power-of-two S_delta, provisional per-chunk scales, fix-up pass
-    int u_only;         // statistics kernel: X L1 partial sums only; the cube means, kamax and scalars[0]
-                        //   are already in the workspace (a producer's epilogue formed them)
     int8_t* prov;       //   N x Ci/64 provisional scale exponents (-128: a chunk whose deltas are all zero)
     int big;            // cubes of more than 128 tokens: boxes are row segments of one cube,
     int nseg;           //   nseg segments of up to 128 tokens per cube row; the kernel tokens
@@ -84,6 +82,10 @@ cudaError_t launch_cube_stats(const CUtensorMap& tm_x, const CUtensorMap& tm_l1,
 cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const CUtensorMap& tm_m, const QuantParams& p,
                                cudaStream_t st);
 cudaError_t launch_cube_means_big(const CUtensorMap& tm_x, const QuantParams& p, cudaStream_t st);
+// the encode pass with X L1 on the tensor cores (for a layer whose statistics a producer's epilogue
+// formed, so that no statistics pass runs), then U' from the partial sums (k_u_hilo)
+cudaError_t launch_cube_encode_lowrank(const CUtensorMap& tm_x, const CUtensorMap& tm_m, const CUtensorMap& tm_l1,
+                                       const QuantParams& p, cudaStream_t st);
 // single-read quantiser: statistics + provisional encode (one read of X), then the fix-up pass with
 // the kernel tokens and U' (no read of X except for re-encoded groups)
 cudaError_t launch_cube_single(const CUtensorMap& tm_x, const CUtensorMap& tm_l1, const QuantParams& p,

@@ -559,9 +559,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                 const int par = (int)(g & 1);
                 float* mts = (float*)(sm + L.ms + (uint32_t)par * L.ms_stride);   // kSingle: this chunk's means
                 float dch = 0.f;                                                 // this chunk's max |delta|
-                if (!kSingle && p.u_only) {
-                    // the statistics are in the workspace already: only X L1 (issued by the MMA warp)
-                } else if (kPairs) {
+                if (kPairs) {
                     // cubes of 16 or more tokens (at most 8 per box): warp = cube slot, lane = channel
                     // pair (2 lane, 2 lane + 1)
                     const bool mine = grp < ngrp && phase == grp;
@@ -603,7 +601,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
                 }
 #pragma unroll
                 for (int t = 0; t < 4; t++) {
-                    if (kPairs || t >= ntask || (!kSingle && p.u_only)) break;
+                    if (kPairs || t >= ntask) break;
                     const StatTask T = t == 0 ? T0 : stat_task(p, R, tid + kQCompute * t);
                     if (!T.valid) continue;
                     uint64_t m[4];
@@ -721,9 +719,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
             // per-cube max |mean| over this item's channels -> kamax (small cubes; the means
             // kernel has done it for big ones); the eight threads of a cube are consecutive lanes,
             // or a whole warp in the channel-pair mode
-            if (!kSingle && p.u_only) {
-                // kamax is in the workspace already
-            } else if (kPairs) {
+            if (kPairs) {
                 const float v = warp_max(kam[0]);
                 if (lane == 0 && grp < ngrp) atomicMax(&p.kamax[R.k0 + u_pair], __float_as_uint(v));
             } else if (!p.big) {
@@ -769,7 +765,7 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
         float wm = warp_max(damax);
         if (lane == 0) red[warp] = wm;
         bar_sync(1, kQCompute);
-        if (tid == 0 && (kSingle || !p.u_only)) {
+        if (tid == 0) {
             float bm = 0.f;
             for (int w = 0; w < kQWarps; w++) bm = fmaxf(bm, red[w]);
             atomicMax(&p.scalars[0], __float_as_uint(bm));
@@ -787,14 +783,19 @@ __global__ void __launch_bounds__(kQCompute + 64, 2) k_cube_stats(const __grid_c
 //
 // Warps 0-7 compute, warp 8 loads.
 
-__global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_constant__ CUtensorMap tm_x,
-                                                                  const __grid_constant__ CUtensorMap tm_m,
-                                                                  QuantParams p) {
+template <bool kLR>
+__global__ void __launch_bounds__(kQCompute + (kLR ? 64 : 32), 2)
+    k_cube_encode(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_m,
+                  const __grid_constant__ CUtensorMap tm_l1, QuantParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const QSmem L = q_smem_layout(p.rank, false, p.m_rows, p.bt * p.bh * p.bw);
+    const QSmem L = q_smem_layout(p.rank, kLR, p.m_rows, p.bt * p.bh * p.bw);
     uint64_t* full = (uint64_t*)(sm + L.bars);
     uint64_t* empty = full + kQStages;
+    uint64_t* accf = empty + kQStages;   // [2], kLR
+    uint64_t* acce = accf + 2;           // [2], kLR
+    uint64_t* done = acce + 2;           // kLR
+    uint32_t* tmem_slot = (uint32_t*)(sm + L.misc);
     volatile int* abort_flag = (volatile int*)(sm + L.misc + 8);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -802,13 +803,24 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
     const int n_items = p.n_boxes * p.splits;
     const uint32_t x_bytes = (uint32_t)p.bt * p.bh * p.bw * 128u;
     const uint32_t m_bytes = (uint32_t)p.m_rows * 256u;   // the box's kernel tokens for 64 channels
+    const uint32_t l1_bytes = kLR ? (uint32_t)p.rank * 128u : 0u;
+    const uint32_t l1_stride = (uint32_t)align_up(l1_bytes, 1024);
+    uint32_t tcols = 32;
+    while (tcols < (uint32_t)p.rank) tcols <<= 1;
     const int Ci = p.Ci;
 
     const PackedHeader* hdr = reinterpret_cast<const PackedHeader*>(p.packed_w);
     if (tid == 0) {
         for (int s = 0; s < kQStages; s++) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kQWarps);
+            mbar_init(&empty[s], kQWarps + (kLR ? 1 : 0));   // the compute warps (+ the MMA commit)
+        }
+        if (kLR) {
+            for (int b = 0; b < 2; b++) {
+                mbar_init(&accf[b], 1);
+                mbar_init(&acce[b], kQWarps);
+            }
+            mbar_init(done, 1);
         }
         *abort_flag = 0;
         fence_barrier_init();
@@ -830,12 +842,20 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
         const float e = __fmul_rn(e4m3_to_f32((uint32_t)tid), S);
         efft[tid] = make_float2(e, (e != 0.f) ? __frcp_rn(e) : 0.f);
     }
+    if (kLR && warp == 9) {
+        tmem_alloc(tmem_slot, 2 * tcols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = kLR ? *tmem_slot : 0u;
 
     if (warp == 8) {
         if (lane == 0) {
             prefetch_tmap(&tm_x);
             prefetch_tmap(&tm_m);
+            if (kLR) prefetch_tmap(&tm_l1);
             long long g = 0;
             bool alive = true;
             for (int it = blockIdx.x; alive && it < n_items; it += gridDim.x) {
@@ -849,19 +869,54 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                         alive = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[s], x_bytes + m_bytes);
+                    mbar_arrive_expect_tx(&full[s], x_bytes + m_bytes + l1_bytes);
                     tma_load_4d(sm + L.x + s * L.x_stride, &tm_x, &full[s], c_base + i * 64, B.w0, B.h0, B.t0);
                     tma_load_2d(sm + L.mt + s * L.mt_stride, &tm_m, &full[s], c_base + i * 64, k0);
+                    if (kLR) tma_load_2d(sm + L.l1 + s * l1_stride, &tm_l1, &full[s], c_base + i * 64, 0);
                 }
             }
             for (long long q = (g > kQStages ? g - kQStages : 0); q < g; q++)
                 mbar_wait(&full[q % kQStages], (uint32_t)(q / kQStages) & 1, abort_flag, nullptr, p.budget_ns, false);
         }
+    } else if (warp == 9) {
+        // ---------------- kLR: X L1 on the tensor cores, the statistics kernel's MMAs in its order
+        if (kLR && lane == 0) {
+            const uint32_t idesc = idesc_bf16(128, p.rank);
+            long long g = 0;
+            int n = 0;
+            bool alive = true;
+            for (int it = blockIdx.x; alive && it < n_items; it += gridDim.x, n++) {
+                const int buf = n & 1, use = n >> 1;
+                const uint32_t acc = tmem + (uint32_t)buf * tcols;
+                if (use > 0 && !mbar_wait(&acce[buf], (uint32_t)(use - 1) & 1, abort_flag, p.status, p.budget_ns))
+                    break;
+                tc_fence_after();
+                for (int i = 0; i < nchunks; i++, g++) {
+                    const int s = (int)(g % kQStages);
+                    if (!mbar_wait(&full[s], (uint32_t)(g / kQStages) & 1, abort_flag, p.status, p.budget_ns)) {
+                        alive = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t xa = smem_u32(sm + L.x + s * L.x_stride), la = smem_u32(sm + L.l1 + s * l1_stride);
+#pragma unroll
+                    for (int k = 0; k < 4; k++)
+                        mma_bf16(acc, desc_k_sw128(xa + 32 * k), desc_k_sw128(la + 32 * k), idesc, (i | k) != 0);
+                    tc_commit(&empty[s]);
+                }
+                if (alive) tc_commit(&accf[buf]);
+            }
+            tc_commit(done);
+            // every MMA has retired before tensor memory is released
+            mbar_wait(done, 0, abort_flag, nullptr, p.budget_ns, false);
+        }
+        __syncwarp();
     } else {
         const float SS = __fmul_rn(S, hdr->S_W);
         long long g = 0;
+        int n_it = 0;
         bool ok = true;
-        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+        for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, n_it++) {
             const BoxPos B = box_pos(p, it / p.splits);
             const int split = it % p.splits;
             const int c_base = split * nchunks * 64;
@@ -981,6 +1036,34 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
                 if (lane == 0) mbar_arrive(&empty[s]);
             }
             if (!ok) break;
+            if (kLR) {
+                // this item's X L1 partial sums out of tensor memory (sub-partition warp % 4, column half
+                // warp / 4), as the statistics kernel stores them; U' follows in k_u_hilo
+                const int buf = n_it & 1, use = n_it >> 1;
+                ok = __all_sync(0xffffffffu, mbar_wait(&accf[buf], (uint32_t)use & 1, abort_flag, p.status, p.budget_ns));
+                if (!ok) break;
+                tc_fence_after();
+                const int urow_i = (warp & 3) * 32 + lane, uhalf = warp >> 2;
+                long long urho = 0;
+                const bool urow_ok = box_row(p, B, urow_i, &urho);
+                float* urow = p.u_part + ((size_t)split * p.g.N + (size_t)urho) * p.rank;
+                for (int c = 16 * uhalf; c < p.rank; c += 32) {
+                    uint32_t rr[16];
+                    tmem_ld_x16(tmem + (uint32_t)buf * tcols + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)c, rr);
+                    tmem_ld_wait();
+                    if (urow_ok) {
+#pragma unroll
+                        for (int v = 0; v < 16; v += 4)
+                            *reinterpret_cast<float4*>(urow + c + v) =
+                                make_float4(__uint_as_float(rr[v]), __uint_as_float(rr[v + 1]), __uint_as_float(rr[v + 2]),
+                                            __uint_as_float(rr[v + 3]));
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acce[buf]);
+                continue;
+            }
             // U' = (X L1) / (S_delta S_W) as BF16 hi + lo for this item's slice of the rank columns
             // (thread = box row x column half), the slab's zero padding by split 0
             const int urow_i = tid & 127, uhalf = tid >> 7;
@@ -1012,7 +1095,43 @@ __global__ void __launch_bounds__(kQCompute + 32, 2) k_cube_encode(const __grid_
             }
         }
     }
+    tc_fence_before();
     __syncthreads();
+    if (kLR && warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 2 * tcols);
+    }
+}
+
+// U' = (X L1) / (S_delta S_W) as BF16 hi + lo from the X L1 partial sums, summed in split order (the
+// arithmetic of k_cube_encode's own U' step), and the slab's zero padding: thread = (row, column pair).
+__global__ void __launch_bounds__(256) k_u_hilo(QuantParams p) {
+    const PackedHeader* hdr = reinterpret_cast<const PackedHeader*>(p.packed_w);
+    const float SS = __fmul_rn(__uint_as_float(p.scalars[1]), hdr->S_W);
+    const int pairs = p.slab / 2;
+    const long long total = p.g.N * pairs;
+    for (long long q = blockIdx.x * (long long)blockDim.x + threadIdx.x; q < total; q += (long long)gridDim.x * blockDim.x) {
+        const long long rho = q / pairs;
+        const int c2 = (int)(q - rho * pairs) * 2;
+        uint16_t* dst = p.u_hilo + (size_t)rho * p.slab;
+        if (c2 >= 2 * p.rank) {
+            *reinterpret_cast<uint32_t*>(dst + c2) = 0u;
+            continue;
+        }
+        if (c2 >= p.rank) continue;   // the lo half of the slab, written with its hi pair below
+        float u0 = 0.f, u1 = 0.f;
+        for (int sp = 0; sp < p.splits; sp++) {
+            const float2 v = *reinterpret_cast<const float2*>(p.u_part + ((size_t)sp * p.g.N + (size_t)rho) * p.rank + c2);
+            u0 = __fadd_rn(u0, v.x);
+            u1 = __fadd_rn(u1, v.y);
+        }
+        const float a0 = __fdiv_rn(u0, SS), a1 = __fdiv_rn(u1, SS);
+        const uint16_t h0 = f32_to_bf16_rn(a0), h1 = f32_to_bf16_rn(a1);
+        const uint16_t l0 = f32_to_bf16_rn(__fsub_rn(a0, __uint_as_float((uint32_t)h0 << 16)));
+        const uint16_t l1 = f32_to_bf16_rn(__fsub_rn(a1, __uint_as_float((uint32_t)h1 << 16)));
+        *reinterpret_cast<uint32_t*>(dst + c2) = (uint32_t)h0 | ((uint32_t)h1 << 16);
+        *reinterpret_cast<uint32_t*>(dst + p.rank + c2) = (uint32_t)l0 | ((uint32_t)l1 << 16);
+    }
 }
 
 // ------------------------------------------------------------------ kernel tokens of big cubes
@@ -1338,13 +1457,32 @@ cudaError_t launch_cube_single(const CUtensorMap& tm_x, const CUtensorMap& tm_l1
 cudaError_t launch_cube_encode(const CUtensorMap& tm_x, const CUtensorMap& tm_m, const QuantParams& p,
                                cudaStream_t st) {
     size_t smem = quant_smem_bytes(p.rank, false, p.m_rows, p.bt * p.bh * p.bw);
-    cudaError_t e = cudaFuncSetAttribute(k_cube_encode, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_cube_encode<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_cube_encode, cudaFuncAttributePreferredSharedMemoryCarveout,
+        e = cudaFuncSetAttribute(k_cube_encode<false>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
-    const int grid = resident_grid((const void*)k_cube_encode, kQCompute + 32, smem, p.n_boxes * p.splits);
-    k_cube_encode<<<grid, kQCompute + 32, smem, st>>>(tm_x, tm_m, p);
+    const int grid = resident_grid((const void*)k_cube_encode<false>, kQCompute + 32, smem, p.n_boxes * p.splits);
+    k_cube_encode<false><<<grid, kQCompute + 32, smem, st>>>(tm_x, tm_m, tm_m, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cube_encode_lowrank(const CUtensorMap& tm_x, const CUtensorMap& tm_m, const CUtensorMap& tm_l1,
+                                       const QuantParams& p, cudaStream_t st) {
+    size_t smem = quant_smem_bytes(p.rank, true, p.m_rows, p.bt * p.bh * p.bw);
+    cudaError_t e = cudaFuncSetAttribute(k_cube_encode<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_cube_encode<true>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    const int grid = resident_grid((const void*)k_cube_encode<true>, kQCompute + 64, smem, p.n_boxes * p.splits);
+    k_cube_encode<true><<<grid, kQCompute + 64, smem, st>>>(tm_x, tm_m, tm_l1, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long work = p.g.N * (p.slab / 2);
+    k_u_hilo<<<(int)imin((int)cdiv(work, 256), 8 * sms), 256, 0, st>>>(p);
     return cudaGetLastError();
 }
 
