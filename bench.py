@@ -368,8 +368,9 @@ def run_ffn(args):
                             W=up.W, N=up.N, Ci=up.Ci, Cf=up.Co, Co=down.Co, rank=[up.rank, down.rank],
                             cube_up=list(up.cube), cube_down=list(down.cube), activation="GELU (erf form) in the "
                             "up-projection's main-product epilogue",
-                            down_statistics=("formed in the up-projection's epilogue (the down-projection's "
-                                             "statistics kernel forms X L1 only)" if fused else "separate pass"),
+                            down_statistics=("formed in the up-projection's epilogue (the down-projection runs "
+                                             "no statistics pass; its encode pass forms X L1)" if fused
+                                             else "separate pass"),
                             l2="inputs larger than L2"),
                 tokens_per_s=up.N / (ms * 1e-3), stages={n: dict(ms=v) for n, v in stage_ms.items()},
                 roofline=dict(kernel="k_gemm<3> (main FP4 product, feed-forward epilogue)" if dom.startswith("up")
