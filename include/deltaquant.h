@@ -434,9 +434,10 @@ int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int
  * up-projection's main-product epilogue also forms the down-projection's
  * statistics pass over the BF16 Hid it writes: the fp32 cube means (K_down x Cf,
  * the running sum from +0 in (t,h,w) order divided by the count), max |mean| per
- * cube and max |Hid - mean|.  The down-projection's statistics kernel then only
- * forms Hid L1_down, one read of Hid fewer per cube statistic.  Otherwise, or with
- * DQ_FFN_SEPARATE_STATISTICS, the down-projection runs its own statistics pass.
+ * cube and max |Hid - mean|.  The down-projection then runs no statistics pass:
+ * its encode pass also forms Hid L1_down on the tensor cores, so Hid is read once
+ * instead of twice.  Otherwise, or with DQ_FFN_SEPARATE_STATISTICS, the
+ * down-projection runs its own statistics pass.
  *
  *   X        device, N x Ci BF16, (t,h,w) order; read only
  *   cube_up, cube_down  host, 3 ints each (t, h, w)
