@@ -47,7 +47,7 @@ def test_fused_statistics_rejects_bad_arguments():
 
 def test_ffn_forward_argument_errors():
     """dq_ffn_forward's argument checks, which run before any device call: flags, cubes,
-    each layer's shape, and the down-projection's workspace size."""
+    each layer's shape, the pointers, and both workspaces' sizes."""
     import ctypes
 
     import video_diffusion_w4a4_b200 as dq
@@ -56,17 +56,20 @@ def test_ffn_forward_argument_errors():
     fake = 1 << 20   # a 256-byte-aligned stand-in address; nothing is dereferenced on these paths
     ld = dq.dq_workspace_layout_opts(T, H, W, *cd, Cf, Co, r)
 
-    def call(flags=0, cube_up=cu, Ci_=Ci, rank_down=r, ws_down_bytes=ld.total_bytes):
+    def call(flags=0, cube_up=cu, Ci_=Ci, rank_down=r, ws_down_bytes=ld.total_bytes, ws_up_bytes=1 << 30, hid=fake):
         a3 = lambda c: (ctypes.c_int * 3)(*c)
         return dq._lib.dq_ffn_forward(fake, T, H, W, a3(cube_up), a3(cd), Ci_, Cf, Co, r, rank_down, fake, fake,
-                                      fake, fake, fake, fake, fake, fake, fake, 1 << 30, fake, ws_down_bytes, flags,
-                                      None, None)
+                                      fake, fake, fake, fake, hid or None, fake, fake, ws_up_bytes, fake,
+                                      ws_down_bytes, flags, None, None)
 
     assert call(flags=2) == dq.DQ_ERR_INVALID_ARG
     assert call(cube_up=(0, 2, 2)) == dq.DQ_ERR_INVALID_ARG
     assert call(Ci_=300) == dq.DQ_ERR_UNSUPPORTED_SHAPE
     assert call(rank_down=8) == dq.DQ_ERR_UNSUPPORTED_SHAPE
     assert call(ws_down_bytes=ld.total_bytes - 1) == dq.DQ_ERR_WORKSPACE_TOO_SMALL
+    assert call(ws_up_bytes=16) == dq.DQ_ERR_WORKSPACE_TOO_SMALL
+    assert call(hid=0) == dq.DQ_ERR_INVALID_ARG
+    assert call(hid=fake + 16) == dq.DQ_ERR_ALIGNMENT
 
 
 def test_epilogue_option_is_checked():

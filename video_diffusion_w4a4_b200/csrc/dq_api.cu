@@ -598,12 +598,17 @@ int dq_ffn_forward(const void* X, int T, int H, int W, const int* cube_up, const
     int rc = check_shape(T, H, W, cube_up[0], cube_up[1], cube_up[2], Ci, Cf, rank_up);
     if (rc) return rc;
     if ((rc = check_shape(T, H, W, cube_down[0], cube_down[1], cube_down[2], Cf, Co, rank_down))) return rc;
-    if (!X || !Hid || !Y || !ws_up || !ws_down) return DQ_ERR_INVALID_ARG;
-    if (!aligned(ws_down)) return DQ_ERR_ALIGNMENT;
+    // every argument is checked before the first device call, so a refused call changes nothing
+    const void* ptrs[] = {X, packed_up, L1_up, L2_up, packed_down, L1_down, L2_down, Hid, Y, ws_up, ws_down};
+    for (const void* q : ptrs) {
+        if (!q) return DQ_ERR_INVALID_ARG;
+        if (!aligned(q)) return DQ_ERR_ALIGNMENT;
+    }
     const Geom gu = dq::make_geom(T, H, W, cube_up[0], cube_up[1], cube_up[2]);
     const Geom gd = dq::make_geom(T, H, W, cube_down[0], cube_down[1], cube_down[2]);
+    const dq::WsLayout wu = dq::ws_layout(gu, Ci, Cf, rank_up, 0, false, false);
     const dq::WsLayout wd = dq::ws_layout(gd, Cf, Co, rank_down, 0, false, false);
-    if (ws_down_bytes < wd.total) return DQ_ERR_WORKSPACE_TOO_SMALL;
+    if (ws_up_bytes < wu.total || ws_down_bytes < wd.total) return DQ_ERR_WORKSPACE_TOO_SMALL;
     const bool fuse = !(ffn_flags & DQ_FFN_SEPARATE_STATISTICS) && ffn_stats_fusable(gu, gd);
     FfnHooks up, down;
     if (fuse) {
