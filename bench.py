@@ -312,15 +312,24 @@ def run_ffn(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     X = synth.activations(up)
-    pu, L1u, L2u = dq.dq_pack_weight(synth.weight(up), up.rank)
-    pd, L1d, L2d = dq.dq_pack_weight(synth.weight(down), down.rank)
+    fp8 = args.kernel_product == "fp8"
+    if fp8:
+        # the FP8 kernel-token product in both layers: restricted-scale (C2) weights
+        def pack(Wb, r):
+            L1f, L2f = dq.dq_lowrank_factors(Wb, r)
+            return dq.dq_pack_weight_factors(Wb, L1f, L2f, pack_flags=dq.DQ_PACK_C2)[:3]
+    else:
+        pack = dq.dq_pack_weight
+    pu, L1u, L2u = pack(synth.weight(up), up.rank)
+    pd, L1d, L2d = pack(synth.weight(down), down.rank)
+    opts = dict(kernel_product=dq.DQ_KERNEL_PRODUCT_FP8 if fp8 else dq.DQ_KERNEL_PRODUCT_BF16)
     t16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev)
     Xd, L1u, L2u, L1d, L2d = t16(X), t16(L1u), t16(L2u), t16(L1d), t16(L2d)
     Pu, Pd = torch.from_numpy(pu).to(dev), torch.from_numpy(pd).to(dev)
     Hd = torch.empty((up.N, up.Co), dtype=torch.int16, device=dev)
     Yd = torch.empty((up.N, down.Co), dtype=torch.int16, device=dev)
-    lu = dq.dq_workspace_layout_opts(up.T, up.H, up.W, *up.cube, up.Ci, up.Co, up.rank)
-    ld = dq.dq_workspace_layout_opts(down.T, down.H, down.W, *down.cube, down.Ci, down.Co, down.rank)
+    lu = dq.dq_workspace_layout_opts(up.T, up.H, up.W, *up.cube, up.Ci, up.Co, up.rank, **opts)
+    ld = dq.dq_workspace_layout_opts(down.T, down.H, down.W, *down.cube, down.Ci, down.Co, down.rank, **opts)
     wsu = torch.zeros(lu.total_bytes, dtype=torch.uint8, device=dev)
     wsd = torch.zeros(ld.total_bytes, dtype=torch.uint8, device=dev)
     st = torch.cuda.current_stream(dev)
@@ -331,8 +340,9 @@ def run_ffn(args):
         for e in row:
             e.record(st)
     def step(ev=None):
-        dq.dq_ffn_forward(Xd, up.T, up.H, up.W, up.cube, down.cube, up.Ci, up.Co, down.Co, up.rank, down.rank, Pu,
-                          L1u, L2u, Pd, L1d, L2d, Hd, Yd, wsu, lu.total_bytes, wsd, ld.total_bytes, flags, ev, st)
+        dq.dq_ffn_forward_opts(Xd, up.T, up.H, up.W, up.cube, down.cube, up.Ci, up.Co, down.Co, up.rank, down.rank,
+                               Pu, L1u, L2u, Pd, L1d, L2d, Hd, Yd, wsu, lu.total_bytes, wsd, ld.total_bytes, flags, ev,
+                               st, opts_up=opts, opts_down=opts)
 
     for _ in range(args.warmup):
         step()
@@ -357,7 +367,7 @@ def run_ffn(args):
     F = layer_flops(up, Ku) + layer_flops(down, Kd)
     peaks = load_peaks()
     fp4_peak = peaks["bf16"] * FP4_PER_BF16
-    mu, md = stage_model(up, Ku, lu.slab), stage_model(down, Kd, ld.slab)
+    mu, md = stage_model(up, Ku, lu.slab, fp8=fp8), stage_model(down, Kd, ld.slab, fp8=fp8)
     dom = max(("up_main_gemm_gelu", "down_main_gemm"), key=stage_ms.get)
     m = mu if dom.startswith("up") else md
     ach = m["main_gemm"]["flops"] / (stage_ms[dom] * 1e-3) / 1e12
@@ -368,6 +378,7 @@ def run_ffn(args):
                             W=up.W, N=up.N, Ci=up.Ci, Cf=up.Co, Co=down.Co, rank=[up.rank, down.rank],
                             cube_up=list(up.cube), cube_down=list(down.cube), activation="GELU (erf form) in the "
                             "up-projection's main-product epilogue",
+                            kernel_product="fp8 (restricted-scale C2 weights)" if fp8 else "bf16 (exact)",
                             down_statistics=("formed in the up-projection's epilogue (the down-projection runs "
                                              "no statistics pass; its encode pass forms X L1)" if fused
                                              else "separate pass"),

@@ -465,6 +465,22 @@ int dq_ffn_forward(const void* X, int T, int H, int W, const int* cube_up, const
                    void* const* stage_events, void* stream);
 
 /*
+ * dq_ffn_forward with forward options per layer (NULL: the defaults): kernel_group,
+ * kernel_product and delta_scale as dq_linear_forward_opts takes them (an FP8
+ * kernel-token product needs that layer's weight packed with DQ_PACK_C2, and
+ * each workspace is sized by dq_workspace_layout_opts for its layer's options).
+ * The up-projection's epilogue is GELU whatever opts_up->epilogue says; the
+ * down-projection's must be DQ_EPILOGUE_NONE.  The statistics fuse only under the
+ * two-pass delta scale (opts_down->delta_scale = DQ_DELTA_SCALE_AMAX).
+ */
+int dq_ffn_forward_opts(const void* X, int T, int H, int W, const int* cube_up, const int* cube_down, int Ci, int Cf,
+                        int Co, int rank_up, int rank_down, const dq_forward_options* opts_up,
+                        const dq_forward_options* opts_down, const void* packed_up, const void* L1_up,
+                        const void* L2_up, const void* packed_down, const void* L1_down, const void* L2_down, void* Hid,
+                        void* Y, void* ws_up, size_t ws_up_bytes, void* ws_down, size_t ws_down_bytes, int ffn_flags,
+                        void* const* stage_events, void* stream);
+
+/*
  * *fused = 1 when dq_ffn_forward forms the down-projection's statistics in the
  * up-projection's epilogue for this lattice and pair of cubes, else 0.  Host
  * only (no device call); O(T H W) the first time a pair of partitions is asked.

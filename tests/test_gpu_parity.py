@@ -439,6 +439,24 @@ def test_parity_ffn_block(env, name, T, H, W, cu, cd, Ci, Cf, Co, ru, rd, fused)
         assert np.array_equal(g[key], s[key]), key
 
 
+@pytest.mark.parametrize("fp8,kgroup_down", [(True, 0), (False, 64)], ids=["fp8_products", "group64_down"])
+def test_parity_ffn_block_options(env, fp8, kgroup_down):
+    """dq_ffn_forward_opts: the FP8 kernel-token product in both layers (restricted-scale
+    weights), or one kernel scale per 64 channels in the down-projection, with the statistics
+    fused; the same oracle checks, and the same bits as the unfused path."""
+    from ffn_case import FfnCase
+    dq, torch = env
+    case = FfnCase("opts_222_122", 3, 6, 16, (2, 2, 2), (1, 2, 2), 256, 512, 256, 32, 16, fp8=fp8,
+                   kgroup_down=kgroup_down)
+    assert case.fused_expected(dq)
+    g = case.run_gpu(dq, torch, gelu_layer=True)
+    case.check(g)
+    assert np.array_equal(g["H"], g["H_layer"])
+    s = case.run_gpu(dq, torch, ffn_flags=dq.DQ_FFN_SEPARATE_STATISTICS)
+    for key in ("H", "Y", "q8", "s8", "dcodes"):
+        assert np.array_equal(g[key], s[key]), key
+
+
 def test_parity_ffn_block_with_biases(env):
     """The feed-forward block with a linear bias in both layers (added once per cube in
     each layer's kernel term, so GELU sees y + b)."""

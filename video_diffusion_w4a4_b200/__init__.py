@@ -102,6 +102,9 @@ _SIGS = {
     "dq_read_device_status": ([_P, _P, ctypes.POINTER(_I), _I], _I),
     "dq_ffn_forward": ([_P, _I, _I, _I, _P, _P] + [_I] * 5 + [_P] * 8 + [_P, _SZ, _P, _SZ, _I, _P, _P], _I),
     "dq_ffn_fused_statistics": ([_I, _I, _I, _P, _P, ctypes.POINTER(_I)], _I),
+    "dq_ffn_forward_opts": ([_P, _I, _I, _I, _P, _P] + [_I] * 5 +
+                            [ctypes.POINTER(dq_forward_options), ctypes.POINTER(dq_forward_options)] + [_P] * 8 +
+                            [_P, _SZ, _P, _SZ, _I, _P, _P], _I),
     "dq_selftest_bounded_wait": ([_I, _P, ctypes.POINTER(_I)], _I),
     "dq_selftest_convert": ([_P, _LL, _P, _P, _P, _P], _I),
     "dq_selftest_divide": ([_LL, ctypes.c_uint64, ctypes.POINTER(ctypes.c_ulonglong), _P, _P], _I),
@@ -339,6 +342,22 @@ def dq_ffn_forward(X, T, H, W, cube_up, cube_down, Ci, Cf, Co, rank_up, rank_dow
                                _ptr(L2_up), _ptr(packed_down), _ptr(L1_down), _ptr(L2_down), _ptr(Hid), _ptr(Y),
                                _ptr(ws_up), ws_up_bytes, _ptr(ws_down), ws_down_bytes, ffn_flags,
                                _events(stage_events, 8), _stream(stream)))
+
+
+def dq_ffn_forward_opts(X, T, H, W, cube_up, cube_down, Ci, Cf, Co, rank_up, rank_down, packed_up, L1_up, L2_up,
+                        packed_down, L1_down, L2_down, Hid, Y, ws_up, ws_up_bytes, ws_down, ws_down_bytes, ffn_flags=0,
+                        stage_events=None, stream=None, opts_up=None, opts_down=None) -> None:
+    """dq_ffn_forward with per-layer forward options: opts_up / opts_down are dicts of
+    dq_forward_options fields (kernel_group, kernel_product, delta_scale), None for the defaults."""
+    cu, cd = (ctypes.c_int * 3)(*cube_up), (ctypes.c_int * 3)(*cube_down)
+    ou = _options(**(opts_up or {}))
+    od = _options(**(opts_down or {}))
+    _check("dq_ffn_forward_opts",
+           _lib.dq_ffn_forward_opts(_ptr(X), T, H, W, cu, cd, Ci, Cf, Co, rank_up, rank_down, ctypes.byref(ou),
+                                    ctypes.byref(od), _ptr(packed_up), _ptr(L1_up), _ptr(L2_up), _ptr(packed_down),
+                                    _ptr(L1_down), _ptr(L2_down), _ptr(Hid), _ptr(Y), _ptr(ws_up), ws_up_bytes,
+                                    _ptr(ws_down), ws_down_bytes, ffn_flags, _events(stage_events, 8),
+                                    _stream(stream)))
 
 
 def dq_workspace_bytes_grouped(T, H, W, t, h, w, Ci, Co, rank, kernel_group) -> int:

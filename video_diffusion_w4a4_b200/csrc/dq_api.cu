@@ -589,15 +589,23 @@ int dq_ffn_fused_statistics(int T, int H, int W, const int* cube_up, const int* 
     return DQ_OK;
 }
 
-int dq_ffn_forward(const void* X, int T, int H, int W, const int* cube_up, const int* cube_down, int Ci, int Cf,
-                   int Co, int rank_up, int rank_down, const void* packed_up, const void* L1_up, const void* L2_up,
-                   const void* packed_down, const void* L1_down, const void* L2_down, void* Hid, void* Y,
-                   void* ws_up, size_t ws_up_bytes, void* ws_down, size_t ws_down_bytes, int ffn_flags,
-                   void* const* stage_events, void* stream) {
+int dq_ffn_forward_opts(const void* X, int T, int H, int W, const int* cube_up, const int* cube_down, int Ci, int Cf,
+                        int Co, int rank_up, int rank_down, const dq_forward_options* opts_up,
+                        const dq_forward_options* opts_down, const void* packed_up, const void* L1_up,
+                        const void* L2_up, const void* packed_down, const void* L1_down, const void* L2_down, void* Hid,
+                        void* Y, void* ws_up, size_t ws_up_bytes, void* ws_down, size_t ws_down_bytes, int ffn_flags,
+                        void* const* stage_events, void* stream) {
     if (!cube_up || !cube_down || (ffn_flags & ~DQ_FFN_SEPARATE_STATISTICS)) return DQ_ERR_INVALID_ARG;
     int rc = check_shape(T, H, W, cube_up[0], cube_up[1], cube_up[2], Ci, Cf, rank_up);
     if (rc) return rc;
     if ((rc = check_shape(T, H, W, cube_down[0], cube_down[1], cube_down[2], Cf, Co, rank_down))) return rc;
+    // each layer's options; the up-projection's epilogue is GELU whatever opts_up says, the
+    // down-projection's none
+    dq_forward_options ou = opts_up ? *opts_up : dq_forward_options{};
+    dq_forward_options od = opts_down ? *opts_down : dq_forward_options{};
+    ou.epilogue = DQ_EPILOGUE_GELU;
+    if (od.epilogue != DQ_EPILOGUE_NONE) return DQ_ERR_INVALID_ARG;
+    if ((rc = check_options(ou)) || (rc = check_options(od))) return rc;
     // every argument is checked before the first device call, so a refused call changes nothing
     const void* ptrs[] = {X, packed_up, L1_up, L2_up, packed_down, L1_down, L2_down, Hid, Y, ws_up, ws_down};
     for (const void* q : ptrs) {
@@ -606,10 +614,16 @@ int dq_ffn_forward(const void* X, int T, int H, int W, const int* cube_up, const
     }
     const Geom gu = dq::make_geom(T, H, W, cube_up[0], cube_up[1], cube_up[2]);
     const Geom gd = dq::make_geom(T, H, W, cube_down[0], cube_down[1], cube_down[2]);
-    const dq::WsLayout wu = dq::ws_layout(gu, Ci, Cf, rank_up, 0, false, false);
-    const dq::WsLayout wd = dq::ws_layout(gd, Cf, Co, rank_down, 0, false, false);
+    const dq::WsLayout wu = dq::ws_layout(gu, Ci, Cf, rank_up, ou.kernel_group,
+                                          ou.kernel_product == DQ_KERNEL_PRODUCT_FP8,
+                                          ou.delta_scale == DQ_DELTA_SCALE_POW2);
+    const dq::WsLayout wd = dq::ws_layout(gd, Cf, Co, rank_down, od.kernel_group,
+                                          od.kernel_product == DQ_KERNEL_PRODUCT_FP8,
+                                          od.delta_scale == DQ_DELTA_SCALE_POW2);
     if (ws_up_bytes < wu.total || ws_down_bytes < wd.total) return DQ_ERR_WORKSPACE_TOO_SMALL;
-    const bool fuse = !(ffn_flags & DQ_FFN_SEPARATE_STATISTICS) && ffn_stats_fusable(gu, gd);
+    // the fused statistics are those of the two-pass quantiser (S_delta = amax / 2688)
+    const bool fuse = !(ffn_flags & DQ_FFN_SEPARATE_STATISTICS) && od.delta_scale == DQ_DELTA_SCALE_AMAX &&
+                      ffn_stats_fusable(gu, gd);
     FfnHooks up, down;
     if (fuse) {
         // the up-projection's epilogue takes the maxima of the down-projection's statistics pass
@@ -625,14 +639,22 @@ int dq_ffn_forward(const void* X, int T, int H, int W, const int* cube_up, const
         up.c_scalars = (uint32_t*)(wsd + wd.off_scalars);
         down.stats_given = true;
     }
-    dq_forward_options ou{};
-    ou.epilogue = DQ_EPILOGUE_GELU;
     rc = forward_impl(X, T, H, W, cube_up[0], cube_up[1], cube_up[2], Ci, Cf, rank_up, &ou, packed_up, L1_up, L2_up,
                       Hid, ws_up, ws_up_bytes, DQ_STAGE_ALL, stage_events, stream, nullptr, &up);
     if (rc) return rc;
-    return forward_impl(Hid, T, H, W, cube_down[0], cube_down[1], cube_down[2], Cf, Co, rank_down, nullptr,
+    return forward_impl(Hid, T, H, W, cube_down[0], cube_down[1], cube_down[2], Cf, Co, rank_down, &od,
                         packed_down, L1_down, L2_down, Y, ws_down, ws_down_bytes, DQ_STAGE_ALL,
                         stage_events ? stage_events + 4 : nullptr, stream, nullptr, &down);
+}
+
+int dq_ffn_forward(const void* X, int T, int H, int W, const int* cube_up, const int* cube_down, int Ci, int Cf,
+                   int Co, int rank_up, int rank_down, const void* packed_up, const void* L1_up, const void* L2_up,
+                   const void* packed_down, const void* L1_down, const void* L2_down, void* Hid, void* Y,
+                   void* ws_up, size_t ws_up_bytes, void* ws_down, size_t ws_down_bytes, int ffn_flags,
+                   void* const* stage_events, void* stream) {
+    return dq_ffn_forward_opts(X, T, H, W, cube_up, cube_down, Ci, Cf, Co, rank_up, rank_down, nullptr, nullptr,
+                               packed_up, L1_up, L2_up, packed_down, L1_down, L2_down, Hid, Y, ws_up, ws_up_bytes,
+                               ws_down, ws_down_bytes, ffn_flags, stage_events, stream);
 }
 
 int dq_linear_forward_opts(const void* X, int T, int H, int W, int t, int h, int w, int Ci, int Co, int rank,
