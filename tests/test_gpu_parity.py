@@ -466,3 +466,45 @@ def test_parity_ffn_block_with_biases(env):
     assert case.fused_expected(dq)
     g = case.run_gpu(dq, torch)
     case.check(g)
+
+
+def test_forward_replays_from_a_cuda_graph(env):
+    """The layer captured into a CUDA graph (every launch and memset of a call is a stream
+    operation on the caller's stream): replays give the eager bits, with new inputs copied
+    into the captured buffers between replays."""
+    dq, torch = env
+    wl = _wl("graph_122", 3, 10, 37, 512, 512, 32, (1, 2, 2))
+    case = Case(wl)
+    eager = case.run_gpu(dq, torch)
+    Xd, Pd, L1d, L2d, Yd = case.last_inputs
+    ws, lay = case.last_ws, case.last_layout
+    t, h, w = case.cube
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):   # warm-up on the capture stream (first-use attribute calls)
+        dq.dq_linear_forward_ex(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd, ws,
+                                lay.total_bytes, dq.DQ_STAGE_ALL, None, s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        dq.dq_linear_forward_ex(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd, ws,
+                                lay.total_bytes, dq.DQ_STAGE_ALL, None, s)
+    X2 = synth.activations(wl, tau=3)
+    for X_in in (X2, case.X):
+        Xd.copy_(torch.from_numpy(X_in.view(np.int16)))
+        Yd.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        if X_in is case.X:
+            assert np.array_equal(Yd.cpu().numpy().view(np.uint16), eager["Y"])
+    assert dq.dq_read_device_status(ws, torch.cuda.current_stream(), clear=True) == 0
+    # the second replay ran on other inputs first: compare it with an eager call on them
+    Xd.copy_(torch.from_numpy(X2.view(np.int16)))
+    graph.replay()
+    torch.cuda.synchronize()
+    y_graph = Yd.cpu().numpy().copy()
+    dq.dq_linear_forward_ex(Xd, wl.T, wl.H, wl.W, t, h, w, wl.Ci, wl.Co, wl.rank, Pd, L1d, L2d, Yd, ws,
+                            lay.total_bytes, dq.DQ_STAGE_ALL, None, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert np.array_equal(Yd.cpu().numpy(), y_graph)
+    del graph
