@@ -565,6 +565,13 @@ int dq_read_device_status(const void* workspace, void* stream, int* status, int 
 int dq_selftest_bounded_wait(int budget_us, void* stream, int* status);
 
 /*
+ * GELU self test: out[i] = the feed-forward epilogue's GELU of in[i] (DQ_EPILOGUE_GELU's
+ * fp32 evaluation, two values at a time as the epilogue takes them), for n device fp32
+ * values; asynchronous.
+ */
+int dq_selftest_gelu(const float* in, long long n, float* out, void* stream);
+
+/*
  * Format self test: for each of the n fp32 values in `in` (device), writes the
  * E2M1 code (low nibble, round to nearest even, saturating), the E4M3 code
  * (same rules) and that E4M3 code's value, using the very conversions the

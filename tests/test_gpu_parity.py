@@ -508,3 +508,23 @@ def test_forward_replays_from_a_cuda_graph(env):
     torch.cuda.synchronize()
     assert np.array_equal(Yd.cpu().numpy(), y_graph)
     del graph
+
+
+def test_device_gelu_error_bound(env):
+    """The feed-forward epilogue's GELU (Abramowitz & Stegun 7.1.26 erfc with the hardware's
+    approximate reciprocal and 2^x, in fp32) against the oracle's exact-form GELU in fp64:
+    |error| <= 3e-7 max(1, |y|) over a dense grid, a wide normal sample and the extremes."""
+    dq, torch = env
+    rng = np.random.default_rng(11)
+    y = np.concatenate([np.linspace(-12.0, 12.0, 480001), rng.normal(0.0, 8.0, 200000),
+                        [0.0, -0.0, 1e-30, -1e-30, 40.0, -40.0, 1e3, -1e3, 6.5, -6.5]]).astype(np.float32)
+    dev = torch.device("cuda")
+    yd = torch.from_numpy(y).to(dev)
+    out = torch.empty_like(yd)
+    dq.dq_selftest_gelu(yd, y.size, out, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    h = out.cpu().numpy().astype(np.float64)
+    ref = oracle.gelu_erf(y.astype(np.float64))
+    err = np.abs(h - ref) / np.maximum(1.0, np.abs(y.astype(np.float64)))
+    assert np.all(np.isfinite(h))
+    assert err.max() <= 3e-7, (float(err.max()), float(y[np.argmax(err)]))

@@ -107,6 +107,7 @@ _SIGS = {
                             [_P, _SZ, _P, _SZ, _I, _P, _P], _I),
     "dq_selftest_bounded_wait": ([_I, _P, ctypes.POINTER(_I)], _I),
     "dq_selftest_convert": ([_P, _LL, _P, _P, _P, _P], _I),
+    "dq_selftest_gelu": ([_P, _LL, _P, _P], _I),
     "dq_selftest_divide": ([_LL, ctypes.c_uint64, ctypes.POINTER(ctypes.c_ulonglong), _P, _P], _I),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -447,6 +448,10 @@ def dq_selftest_bounded_wait(budget_us: int, stream=None) -> int:
 def dq_selftest_convert(inp, n, e2m1, e4m3, e4m3_value, stream=None) -> None:
     _check("dq_selftest_convert", _lib.dq_selftest_convert(_ptr(inp), n, _ptr(e2m1), _ptr(e4m3), _ptr(e4m3_value),
                                                            _stream(stream)))
+
+
+def dq_selftest_gelu(inp, n, out, stream=None) -> None:
+    _check("dq_selftest_gelu", _lib.dq_selftest_gelu(_ptr(inp), n, _ptr(out), _stream(stream)))
 
 
 def dq_selftest_divide(n: int, seed: int = 1, stream=None):

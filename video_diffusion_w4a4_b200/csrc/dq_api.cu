@@ -848,6 +848,12 @@ int dq_selftest_bounded_wait(int budget_us, void* stream, int* status) {
     return rc;
 }
 
+int dq_selftest_gelu(const float* in, long long n, float* out, void* stream) {
+    if (n < 0 || (n > 0 && (!in || !out))) return DQ_ERR_INVALID_ARG;
+    if (dq::launch_selftest_gelu(in, n, out, (cudaStream_t)stream) != cudaSuccess) return DQ_ERR_CUDA;
+    return DQ_OK;
+}
+
 int dq_selftest_convert(const float* in, long long n, uint8_t* e2m1, uint8_t* e4m3, float* e4m3_value,
                         void* stream) {
     if (n < 0 || (n > 0 && (!in || !e2m1 || !e4m3 || !e4m3_value))) return DQ_ERR_INVALID_ARG;

@@ -31,6 +31,17 @@ __global__ void k_selftest_convert(const float* in, long long n, uint8_t* e2m1, 
     e4m3_back[i] = e4m3_to_f32(c);
 }
 
+// The feed-forward epilogue's GELU (gelu_erf2, two values per call) on n fp32 values.
+__global__ void k_selftest_gelu(const float* in, long long n, float* out) {
+    const long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float y0 = in[i], y1 = (i + 1 < n) ? in[i + 1] : 0.f;
+    float h0, h1;
+    f2_unpack(gelu_erf2(f2_pack(y0, y1)), h0, h1);
+    out[i] = h0;
+    if (i + 1 < n) out[i + 1] = h1;
+}
+
 __device__ __forceinline__ uint64_t mix64d(uint64_t x) {
     x += 0x9E3779B97F4A7C15ull;
     x = (x ^ (x >> 30)) * 0xBF58476D1CE4E5B9ull;
@@ -82,6 +93,12 @@ cudaError_t launch_selftest_divide(long long n, uint64_t seed, unsigned long lon
 
 cudaError_t launch_selftest_wait(int* status, uint64_t budget_ns, cudaStream_t st) {
     k_selftest_wait<<<1, 32, 0, st>>>(status, budget_ns);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_gelu(const float* in, long long n, float* out, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    k_selftest_gelu<<<(unsigned)((n + 511) / 512), 256, 0, st>>>(in, n, out);
     return cudaGetLastError();
 }
 

@@ -109,6 +109,7 @@ cudaError_t launch_main_gemm_ffn(const CUtensorMap& tm_a, const CUtensorMap& tm_
 int noalloc_workspace(void** out);
 
 cudaError_t launch_selftest_wait(int* status, uint64_t budget_ns, cudaStream_t st);
+cudaError_t launch_selftest_gelu(const float* in, long long n, float* out, cudaStream_t st);
 cudaError_t launch_selftest_divide(long long n, uint64_t seed, unsigned long long* mismatches, float* first,
                                    cudaStream_t st);
 cudaError_t launch_selftest_convert(const float* in, long long n, uint8_t* e2m1, uint8_t* e4m3, float* back,
